@@ -1,0 +1,181 @@
+"""fp64 CPU oracle of the gated delta rule -- TEST INFRASTRUCTURE ONLY.
+
+This package is the reference the CUDA library is checked against.  Only the
+tests, ``__graft_entry__.smoke()`` and the CPU-baseline leg of ``bench.py`` may
+import it.  It shares no code with the CUDA path and never calls it.
+
+``gdr_oracle.c`` holds the token-by-token definition (compiled here with gcc,
+no fast-math); ``forms.py`` holds independent formulations from the pages
+(the chunked WY form, the pseudo-value form, gated linear attention by brute
+force) used to pin it.  Every function here is pinned by
+``tests/test_oracle_pins.py`` (closed forms, worked examples printed on the
+pages, independent formulations, brute force, invariants); none is left
+unpinned.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "gdr_oracle.c")
+_BUILD = os.path.join(_HERE, "_build")
+_LIB_PATH = os.path.join(_BUILD, "libgdr_oracle.so")
+_lock = threading.Lock()
+_lib = None
+
+__all__ = ["build", "lib", "prologue", "chunk_fwd", "recurrent_step", "threads"]
+
+
+def build(force: bool = False) -> str:
+    """Compile gdr_oracle.c into oracle/_build/libgdr_oracle.so (gcc, -O2 -fopenmp)."""
+    os.makedirs(_BUILD, exist_ok=True)
+    if force or not os.path.exists(_LIB_PATH) or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC):
+        tmp = _LIB_PATH + f".tmp{os.getpid()}"
+        cmd = ["gcc", "-O2", "-std=c11", "-fopenmp", "-fPIC", "-shared", "-Wall", _SRC, "-o", tmp, "-lm"]
+        subprocess.run(cmd, check=True)
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def lib() -> ctypes.CDLL:
+    global _lib
+    with _lock:
+        if _lib is None:
+            path = build()
+            L = ctypes.CDLL(path)
+            dp = ctypes.POINTER(ctypes.c_double)
+            ip = ctypes.POINTER(ctypes.c_int32)
+            c_int, c_double = ctypes.c_int, ctypes.c_double
+            L.gdr_oracle_prologue.restype = None
+            L.gdr_oracle_prologue.argtypes = [dp, dp, dp, dp, dp, dp, c_double, c_int, c_int, c_int, c_int, c_int,
+                                              dp, dp, dp, dp]
+            L.gdr_oracle_chunk_fwd.restype = c_int
+            L.gdr_oracle_chunk_fwd.argtypes = [dp, dp, dp, dp, dp, dp, ip, c_double, c_int, c_int, c_int, c_int,
+                                               c_int, c_int, dp, dp]
+            L.gdr_oracle_recurrent_step.restype = c_int
+            L.gdr_oracle_recurrent_step.argtypes = [dp, dp, dp, dp, dp, dp, dp, c_int, ip, ip, ip, c_double, c_int,
+                                                    c_int, c_int, c_int, c_int, c_int, dp]
+            L.gdr_oracle_threads.restype = c_int
+            L.gdr_oracle_threads.argtypes = []
+            _lib = L
+    return _lib
+
+
+def _f64(x):
+    if x is None:
+        return None
+    return np.ascontiguousarray(np.asarray(x, dtype=np.float64))
+
+
+def _i32(x):
+    if x is None:
+        return None
+    return np.ascontiguousarray(np.asarray(x, dtype=np.int32))
+
+
+def _dp(a):
+    if a is None:
+        return None
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
+
+
+def _ip(a):
+    if a is None:
+        return None
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))
+
+
+def threads() -> int:
+    """OpenMP threads the C oracle runs with."""
+    return int(lib().gdr_oracle_threads())
+
+
+def prologue(q=None, k=None, b=None, a=None, A_log=None, dt_bias=None, eps: float = 1e-6):
+    """fp64 prologue: l2norm(q), l2norm(k) (eps inside the sqrt), sigmoid(b),
+    g = -exp(A_log) * softplus(a + dt_bias).
+
+    q, k: (B, Nk, S, Dk); b, a: (B, Nv, S); A_log, dt_bias: (Nv).
+    Returns a dict with whichever of q_hat, k_hat, beta, g could be formed.
+    Follows the transformers GatedDeltaNet forward (blog page, beta and g
+    lines, l2norm in torch_recurrent_gated_delta_rule) and deltanet.rs
+    (module docstring, l2norm, softplus).
+    """
+    L = lib()
+    res = {}
+    qa, ka = _f64(q), _f64(k)
+    if qa is not None or ka is not None:
+        B, Nk, S, Dk = (qa if qa is not None else ka).shape
+        qh = np.empty_like(qa) if qa is not None else None
+        kh = np.empty_like(ka) if ka is not None else None
+        L.gdr_oracle_prologue(_dp(qa), _dp(ka), None, None, None, None, float(eps), B, Nk, 1, S, Dk,
+                              _dp(qh), _dp(kh), None, None)
+        if qh is not None:
+            res["q_hat"] = qh
+        if kh is not None:
+            res["k_hat"] = kh
+    ba, aa = _f64(b), _f64(a)
+    if ba is not None or aa is not None:
+        B, Nv, S = (ba if ba is not None else aa).shape
+        be = np.empty_like(ba) if ba is not None else None
+        gg = None
+        Al, dtb = _f64(A_log), _f64(dt_bias)
+        if aa is not None:
+            if Al is None or dtb is None or Al.shape != (Nv,) or dtb.shape != (Nv,):
+                raise ValueError("a needs A_log and dt_bias of shape (Nv,)")
+            gg = np.empty_like(aa)
+        L.gdr_oracle_prologue(None, None, _dp(ba), _dp(aa), _dp(Al), _dp(dtb), float(eps), B, 1, Nv, S, 1,
+                              None, None, _dp(be), _dp(gg))
+        if be is not None:
+            res["beta"] = be
+        if gg is not None:
+            res["g"] = gg
+    return res
+
+
+def chunk_fwd(q, k, v, beta, g=None, initial_state=None, actual_seq_lengths=None, scale: float = 1.0):
+    """fp64 semantics of the chunked-prefill call, token by token.
+
+    Returns (out (B,Nv,S,Dv), final_state (B,Nv,Dk,Dv)).  Raises ValueError on
+    the shape errors the lite_boost chunk op defines (Nv % Nk, lengths
+    outside [0, S]).
+    """
+    qa, ka, va, ba = _f64(q), _f64(k), _f64(v), _f64(beta)
+    B, Nk, S, Dk = qa.shape
+    Nv, Dv = va.shape[1], va.shape[3]
+    ga, s0, L = _f64(g), _f64(initial_state), _i32(actual_seq_lengths)
+    out = np.empty((B, Nv, S, Dv), np.float64)
+    fin = np.empty((B, Nv, Dk, Dv), np.float64)
+    rc = lib().gdr_oracle_chunk_fwd(_dp(qa), _dp(ka), _dp(va), _dp(ba), _dp(ga), _dp(s0), _ip(L), float(scale),
+                                    B, Nk, Nv, S, Dk, Dv, _dp(out), _dp(fin))
+    if rc != 0:
+        raise ValueError(f"oracle chunk_fwd rejected the arguments (code {rc})")
+    return out, fin
+
+
+def recurrent_step(q, k, v, beta, g, gk, state_pool, ssm_state_indices, actual_seq_lengths,
+                   num_accepted_tokens=None, scale: float = 1.0):
+    """fp64 semantics of the decode call over a slot pool.
+
+    Returns (out (B,Nv,S,Dv), new_pool (slots,Nv,Dk,Dv)); the input pool is
+    not modified (a copy is updated).  See gdr_oracle.c for the reading of
+    num_accepted_tokens.
+    """
+    qa, ka, va, ba = _f64(q), _f64(k), _f64(v), _f64(beta)
+    B, Nk, S, Dk = qa.shape
+    Nv, Dv = va.shape[1], va.shape[3]
+    ga, gka = _f64(g), _f64(gk)
+    pool = np.array(state_pool, dtype=np.float64, copy=True, order="C")
+    slots = pool.shape[0]
+    idx, L = _i32(ssm_state_indices), _i32(actual_seq_lengths)
+    A = _i32(num_accepted_tokens)
+    out = np.empty((B, Nv, S, Dv), np.float64)
+    rc = lib().gdr_oracle_recurrent_step(_dp(qa), _dp(ka), _dp(va), _dp(ba), _dp(ga), _dp(gka), _dp(pool), slots,
+                                         _ip(idx), _ip(L), _ip(A), float(scale), B, Nk, Nv, S, Dk, Dv, _dp(out))
+    if rc != 0:
+        raise ValueError(f"oracle recurrent_step rejected the arguments (code {rc})")
+    return out, pool

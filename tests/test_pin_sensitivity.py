@@ -1,0 +1,80 @@
+"""The pins catch plausible mistakes.
+
+A plain numpy copy of the token-by-token rule is run through every pin in
+``_pins``: unmodified it must pass them all (so the harness itself is sound),
+and with each planted mistake (a dropped term, a wrong sign, an operation in
+the wrong order, a wrong head index, padding left dirty) at least one pin
+must fail.  Everything here runs on the CPU; nothing touches the CUDA path.
+"""
+import numpy as np
+import pytest
+
+from tests import _pins
+
+
+def make_impl(mutation=None):
+    def impl(q, k, v, beta, g, S0, lengths, scale):
+        q, k, v, beta = (np.asarray(x, np.float64) for x in (q, k, v, beta))
+        B, Nk, S, Dk = q.shape
+        Nv, Dv = v.shape[1], v.shape[3]
+        grp = Nv // Nk
+        out = np.zeros((B, Nv, S, Dv))
+        fin = np.zeros((B, Nv, Dk, Dv))
+        for b in range(B):
+            L = S if lengths is None else int(lengths[b])
+            for h in range(Nv):
+                kh = (h % Nk) if mutation == "gqa_modulo" else h // grp
+                St = np.zeros((Dk, Dv)) if S0 is None else np.array(S0[b, h], np.float64)
+                for t in range(S):
+                    if t >= L:
+                        if mutation == "dirty_padding":
+                            out[b, h, t] = 1.0
+                        continue
+                    x = q[b, kh, t] * (1.0 if mutation == "no_scale" else scale)
+                    y = k[b, kh, t]
+                    gt = 0.0 if g is None else float(g[b, h, t])
+                    a = np.exp(-gt) if mutation == "gate_sign" else np.exp(gt)
+                    if mutation != "decay_after_readout":
+                        St = St * a
+                    m = y @ St
+                    if mutation == "decay_after_readout":
+                        St = St * a
+                    if mutation == "beta_on_v_only":
+                        d = beta[b, h, t] * v[b, h, t] - m
+                    else:
+                        d = beta[b, h, t] * (v[b, h, t] - m)
+                    if mutation == "output_before_write":
+                        out[b, h, t] = x @ St
+                    if mutation == "write_sign":
+                        St = St - np.outer(y, d)
+                    elif mutation == "write_uses_query":
+                        St = St + np.outer(x / max(scale, 1e-300), d)
+                    else:
+                        St = St + np.outer(y, d)
+                    if mutation != "output_before_write":
+                        out[b, h, t] = x @ St
+                fin[b, h] = St
+        return out, fin
+    return impl
+
+
+MUTATIONS = ["decay_after_readout", "beta_on_v_only", "output_before_write", "write_sign", "write_uses_query",
+             "gqa_modulo", "no_scale", "gate_sign", "dirty_padding"]
+
+
+def test_unmodified_copy_passes_every_pin():
+    impl = make_impl(None)
+    for check in _pins.ALL_CHECKS:
+        check(impl)
+
+
+@pytest.mark.parametrize("mutation", MUTATIONS)
+def test_planted_mistake_is_caught(mutation):
+    impl = make_impl(mutation)
+    failed = []
+    for check in _pins.ALL_CHECKS:
+        try:
+            check(impl)
+        except (AssertionError, ValueError, IndexError):
+            failed.append(check.__name__)
+    assert failed, f"no pin caught the planted mistake {mutation!r}"
