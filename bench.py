@@ -1,0 +1,415 @@
+"""Benchmark of the gated delta rule hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step = one pass of the prefill hot path over the prefill workload
+(B=4, S=4096, Nk=16, Nv=32, Dk=Dv=128, bf16 q/k/v/beta/state, fp32 gate):
+raw q/k, beta logits and the raw gate a go through gdr_chunk_fwd with the fused
+prologue (l2norm, sigmoid, softplus gate), the cumulative gate, the WY solve,
+the intra-chunk products and the inter-chunk carry, writing out and the final
+state.  The decode row is measured in the same run on the decode workload
+(B=64, one token, 128-slot bf16 pool) and the multi-token per-key-gate decode
+workload (B=256, S=4, 512 slots), reported under "decode".
+
+Timing: W warm-up steps, then K timed steps bracketed by a barrier and
+torch.cuda.synchronize(); each step is timed with CUDA events on the launching
+stream, with a 256 MiB L2 flush between steps (the prefill inputs, 414 MB, are
+larger than the 126 MB L2 as well).  For N > 1 (torchrun), every rank runs its
+own batch (weak scaling, no data-path collective) and the max over ranks is used.
+
+`--impl reference` times the fp64 CPU oracle (the only reference this path has)
+on a bounded sample of the same workload on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+METRIC = "chunked GDR prefill tokens/s; decode state GB/s vs B200 HBM peak (1 GPU)"
+UNIT = "tokens/s"
+FLUSH_BYTES = 256 << 20
+
+
+def algorithmic_prefill_bytes(w) -> int:
+    """HBM bytes one prefill call must move at minimum: per valid token q, k (Nk heads),
+    v and out (Nv heads) in bf16, beta (bf16) and the fp32 gate input per value head;
+    per (b, h) the initial state read and the final state written (bf16)."""
+    e = 2  # bf16
+    per_token = 2 * w.Nk * w.Dk * e + w.Nv * w.Dv * e + w.Nv * w.Dv * e + w.Nv * e + w.Nv * 4
+    tokens = int(w.lengths.sum())
+    state = 2 * w.B * w.Nv * w.Dk * w.Dv * e
+    # padding rows of out are written as zeros too
+    pad_out = (w.B * w.S - tokens) * w.Nv * w.Dv * e
+    return tokens * per_token + state + pad_out
+
+
+def algorithmic_decode_bytes(w) -> dict:
+    """State bytes (read once and written once per referenced (slot, head)) and the
+    per-token I/O bytes of one decode call."""
+    e = 2
+    seqs = int((w.lengths > 0).sum())
+    state = 2 * seqs * w.Nv * w.Dk * w.Dv * e
+    tok = int(w.lengths.sum())
+    io = tok * (2 * w.Nk * w.Dk * e + w.Nv * w.Dv * e + w.Nv * e + w.Nv * 4)
+    if w.gk is not None:
+        io += tok * w.Nv * w.Dk * 4
+    io += w.B * w.S * w.Nv * w.Dv * e  # out, all positions
+    return {"state": state, "io": io}
+
+
+def measured_peaks() -> dict:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def profiled_traffic(kernel: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on the
+    current kernel source (matching hash), else None."""
+    import hashlib
+    p = os.path.join(ROOT, "profiles", "dram_traffic.txt")
+    if not os.path.exists(p):
+        return None
+    srcs = {"chunk": ["gated_deltanet_gdr_b200/csrc/chunk_tc.cu", "gated_deltanet_gdr_b200/csrc/chunk_simt.cu"],
+            "decode": ["gated_deltanet_gdr_b200/csrc/decode.cu"]}
+    for line in open(p):
+        parts = line.split()
+        if len(parts) >= 4 and parts[0] == kernel and not line.startswith("#"):
+            src = os.path.join(ROOT, parts[1])
+            if not os.path.exists(src):
+                return None
+            h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+            return float(parts[3]) if h == parts[2] else None
+    return None
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event (throttle) reasons through NVML every ~2 ms in a
+    background thread while `active` is set (read-only queries; no setting is changed)."""
+    REASONS = {"hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+               "hw_power_brake_slowdown": 0x80, "sw_power_cap": 0x4}
+
+    def __init__(self, index: int):
+        self.index = index
+        self.samples = []
+        self.active = False
+        self._stop = False
+        self.max_mhz = None
+        self.ok = False
+
+    def __enter__(self):
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            uuid = None
+            try:
+                uuid = torch.cuda.get_device_properties(self.index).uuid
+            except Exception:
+                pass
+            h = None
+            if uuid is not None:
+                try:
+                    h = pynvml.nvmlDeviceGetHandleByUUID(("GPU-" + str(uuid)).encode())
+                except Exception:
+                    h = None
+            if h is None:
+                h = pynvml.nvmlDeviceGetHandleByIndex(self.index)
+            self.nv, self.h = pynvml, h
+            self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM))
+            self.ok = True
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        except Exception:
+            self.ok = False
+        return self
+
+    def _run(self):
+        while not self._stop:
+            if self.active:
+                try:
+                    mhz = self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM)
+                    rs = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                    self.samples.append((float(mhz), int(rs)))
+                except Exception:
+                    pass
+            time.sleep(0.002)
+
+    def __exit__(self, *exc):
+        self._stop = True
+        if self.ok:
+            self.t.join(timeout=2)
+
+    def summary(self) -> dict:
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        sm = [m for m, _ in self.samples]
+        reasons = sorted(n for n, bit in self.REASONS.items() if any(r & bit for _, r in self.samples))
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": self.max_mhz, "reasons": reasons,
+                "samples": len(sm), "source": "NVML, 2 ms polling during the timed steps"}
+
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def all_max(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def timed_steps(fn, K, flush, stream):
+    """Per-step CUDA-event times (ms) on `stream`, with an L2 flush before each step."""
+    evs = []
+    with torch.cuda.stream(stream):
+        for _ in range(K):
+            flush.zero_()
+            s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            s.record(stream)
+            fn()
+            e.record(stream)
+            evs.append((s, e))
+    torch.cuda.synchronize()
+    return [s.elapsed_time(e) for s, e in evs]
+
+
+def cpu_oracle_sample(w):
+    """The fp64 oracle as it stands on one sequence of the prefill workload (all
+    value heads, all 4096 tokens), prologue included.  Returns (tokens/s, seconds, threads)."""
+    import oracle
+    sl = slice(0, 1)
+    to_bf16 = lambda x: torch.from_numpy(np.ascontiguousarray(x)).to(torch.bfloat16).double().numpy()
+    q, k, v, b = (to_bf16(x[sl]) for x in (w.q, w.k, w.v, w.b))
+    s0 = to_bf16(w.initial_state[sl])
+    t0 = time.perf_counter()
+    p = oracle.prologue(q=q, k=k, b=b, a=w.a[sl], A_log=w.A_log, dt_bias=w.dt_bias)
+    oracle.chunk_fwd(p["q_hat"], p["k_hat"], v, p["beta"], p["g"], s0, None, w.scale)
+    dt = time.perf_counter() - t0
+    return w.S / dt, dt, oracle.threads()
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return
+    w = workloads.generate("prefill", B=1)
+    vals = []
+    for i in range(args.warmup + args.steps):
+        tps, dt, thr = cpu_oracle_sample(w)
+        if i >= args.warmup:
+            vals.append(dt)
+    tot = sum(vals)
+    value = w.S * len(vals) / tot
+    sample = f"1 sequence x 4096 tokens x 32 value heads of the prefill workload per step, prologue included"
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot / len(vals),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": "prefill B=4 S=4096 Nk=16 Nv=32 Dk=Dv=128 (oracle sample: B=1)",
+                       "global_batch": 1, "seq_len": 4096, "parallelism": "host cores"},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": thr, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def bf16_dev(x):
+    return torch.from_numpy(np.ascontiguousarray(x)).to(torch.bfloat16).cuda()
+
+
+def f32_dev(x):
+    return torch.from_numpy(np.ascontiguousarray(np.asarray(x, np.float32))).cuda()
+
+
+def run_ours(args, world, rank, local):
+    import gated_deltanet_gdr_b200 as gdr
+    gdr.lib()  # fails loudly if the library is missing
+    peaks = measured_peaks()
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+
+    # ---------------- prefill (the headline) ----------------
+    w = workloads.generate("prefill", seed=2 + 1000 * rank)
+    q, k, v, b = bf16_dev(w.q), bf16_dev(w.k), bf16_dev(w.v), bf16_dev(w.b)
+    a = f32_dev(w.a)
+    s0 = bf16_dev(w.initial_state)
+    pro = gdr.Prologue(l2norm_qk=True, eps=1e-6, beta_logits=True, A_log=f32_dev(w.A_log), dt_bias=f32_dev(w.dt_bias))
+    out = torch.empty((w.B, w.Nv, w.S, w.Dv), dtype=torch.bfloat16, device="cuda")
+    fin = torch.empty_like(s0)
+
+    def step():
+        gdr.chunk_fwd(q, k, v, b, a, s0, None, w.scale, prologue=pro, out=out, final_state=fin)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if gdr.get_error() != 0:
+        raise RuntimeError("device error word set during warm-up")
+
+    clk = ClockSampler(local).__enter__()
+    barrier(world)
+    torch.cuda.synchronize()
+    clk.active = True
+    times = timed_steps(step, args.steps, flush, stream)
+    clk.active = False
+    barrier(world)
+    total_ms = all_max(sum(times), world)
+    ms_per_step = total_ms / args.steps
+    tokens = int(w.lengths.sum())
+    value = world * tokens * args.steps / (total_ms / 1e3)
+    alg_bytes = algorithmic_prefill_bytes(w)
+    achieved = alg_bytes / (ms_per_step / 1e3) / 1e9
+    traffic = profiled_traffic("chunk")
+    roofline = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / peaks["hbm_gbs"], "traffic": traffic,
+                "peak_source": peaks["source"], "algorithmic_bytes_per_launch": alg_bytes,
+                "kernel": "gdr_chunk_fwd (fused prologue)"}
+
+    # ---------------- e2e through the public call with host buffers ----------------
+    hq, hk, hv, hb = (t.cpu().pin_memory() for t in (q, k, v, b))
+    ha, hs0 = a.cpu().pin_memory(), s0.cpu().pin_memory()
+    hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    hfin = torch.empty(fin.shape, dtype=fin.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hb, ha, hs0))
+    d2h = hout.numel() * hout.element_size() + hfin.numel() * hfin.element_size()
+
+    def e2e_step():
+        for d, h in ((q, hq), (k, hk), (v, hv), (b, hb), (a, ha), (s0, hs0)):
+            d.copy_(h, non_blocking=True)
+        gdr.chunk_fwd(q, k, v, b, a, s0, None, w.scale, prologue=pro, out=out, final_state=fin)
+        hout.copy_(out, non_blocking=True)
+        hfin.copy_(fin, non_blocking=True)
+
+    e2e_steps = max(3, min(args.steps, 10))
+    for _ in range(2):
+        e2e_step()
+    barrier(world)
+    torch.cuda.synchronize()
+    e2e_times = timed_steps(e2e_step, e2e_steps, flush, stream)
+    barrier(world)
+    e2e_ms = all_max(sum(e2e_times), world) / e2e_steps
+    e2e = {"value": world * tokens / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+           "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
+    del hq, hk, hv, hb, ha, hs0, hout, hfin
+
+    # ---------------- decode row ----------------
+    decode = {}
+    launches = args.steps
+    for name in ("decode", "decode_gk"):
+        wd = workloads.generate(name, seed=(1 if name == "decode" else 4) + 1000 * rank)
+        dq, dk, dv, db = bf16_dev(wd.q), bf16_dev(wd.k), bf16_dev(wd.v), bf16_dev(wd.b)
+        dg = f32_dev(wd.g)
+        dgk = f32_dev(wd.gk) if wd.gk is not None else None
+        pool = bf16_dev(wd.pool)
+        idx = torch.from_numpy(wd.indices).cuda()
+        lens = torch.from_numpy(wd.lengths).cuda()
+        acc = torch.from_numpy(wd.accepted).cuda()
+        dout = torch.empty((wd.B, wd.Nv, wd.S, wd.Dv), dtype=torch.bfloat16, device="cuda")
+        dpro = gdr.Prologue(l2norm_qk=True, eps=1e-6, beta_logits=True)
+
+        def dstep():
+            gdr.recurrent_step(dq, dk, dv, db, dg, dgk, pool, idx, lens, acc, wd.scale, prologue=dpro, out=dout)
+
+        for _ in range(args.warmup):
+            dstep()
+        barrier(world)
+        torch.cuda.synchronize()
+        clk.active = True
+        dt_ms = timed_steps(dstep, args.steps, flush, stream)
+        clk.active = False
+        barrier(world)
+        d_ms = all_max(sum(dt_ms), world) / args.steps
+        nb = algorithmic_decode_bytes(wd)
+        launches += args.steps
+        gbs = nb["state"] / (d_ms / 1e3) / 1e9
+        tot = (nb["state"] + nb["io"]) / (d_ms / 1e3) / 1e9
+        decode[name] = {"workload": f"B={wd.B} S={wd.S} Nk={wd.Nk} Nv={wd.Nv} D={wd.Dk} bf16 pool of "
+                                    f"{wd.pool.shape[0]} slots" + (", per-key gate" if wd.gk is not None else ""),
+                        "us_per_call": d_ms * 1e3, "steps_per_s": world * 1e3 / d_ms,
+                        "state_GBps": gbs, "state_frac_of_hbm": gbs / peaks["hbm_gbs"],
+                        "roofline": {"bound": "hbm", "achieved": tot, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                                     "frac": tot / peaks["hbm_gbs"], "traffic": profiled_traffic("decode"),
+                                     "algorithmic_bytes_per_launch": nb["state"] + nb["io"]}}
+        del pool
+
+    clk.__exit__(None, None, None)
+    if gdr.get_error() != 0:
+        raise RuntimeError("device error word set during the benchmark")
+
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": f"prefill B={w.B} S={w.S} Nk={w.Nk} Nv={w.Nv} Dk=Dv={w.Dk} bf16, fused prologue, "
+                                   "equal lengths", "global_batch": w.B * world, "seq_len": w.S,
+                       "parallelism": f"dp{world} (independent batches per GPU)",
+                       "l2": "inputs larger than L2, plus a 256 MiB flush before every timed step"},
+            "roofline": roofline, "e2e": e2e, "decode": decode, "gpu_launches": launches,
+            "clocks": clk.summary()}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        tps, dt, thr = cpu_oracle_sample(workloads.generate("prefill", B=1))
+        line["cpu_baseline"] = {"value": tps, "unit": UNIT, "cores": thr, "kind": "oracle",
+                                "sample": f"1 sequence x 4096 tokens x 32 value heads, prologue included, {dt:.1f} s"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing (for profiling runs)")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    world, rank, local = dist_setup() if args.impl == "ours" or int(os.environ.get("WORLD_SIZE", "1")) > 1 \
+        else (1, 0, 0)
+    try:
+        if args.impl == "reference":
+            run_reference(args, world, rank)
+        else:
+            run_ours(args, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

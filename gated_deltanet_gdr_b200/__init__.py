@@ -1,0 +1,245 @@
+"""B200 (sm_100a) gated delta rule: Python binding of libgdr.so.
+
+The functions here only check and marshal arguments (torch tensors to device
+pointers and sizes) and call the C ABI declared in ``include/gdr.h``; every
+step of the computation runs in the library's CUDA kernels.  PyTorch supplies
+device memory and streams.  If the compiled library is missing, importing the
+binding's functions raises: there is no fallback.
+
+    out, final_state = chunk_fwd(q, k, v, beta, g, initial_state, actual_seq_lengths, scale)
+    out, state_pool  = recurrent_step(q, k, v, beta, g, gk, state_pool, ssm_state_indices,
+                                      actual_seq_lengths, num_accepted_tokens, scale)
+
+Layouts are BNSD: q, k (B, Nk, S, Dk); v (B, Nv, S, Dv); beta, g (B, Nv, S).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+from dataclasses import dataclass
+from typing import Optional
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libgdr.so")
+
+GDR_OK, GDR_ERR_SHAPE, GDR_ERR_DTYPE, GDR_ERR_NULL, GDR_ERR_ALIGN, GDR_ERR_UNSUPPORTED, GDR_ERR_DEVICE, \
+    GDR_ERR_LAUNCH = range(8)
+GDR_F32, GDR_BF16 = 0, 1
+DEVERR_SLOT_INDEX, DEVERR_LENGTH = 0x1, 0x2
+
+# Every symbol the C header declares (checked by the ABI test).
+EXPORTED = ("gdr_chunk_fwd", "gdr_recurrent_step", "gdr_prologue_apply", "gdr_get_error", "gdr_status_string",
+            "gdr_version")
+
+
+class GdrPrologueStruct(ctypes.Structure):
+    _fields_ = [("l2norm_qk", ctypes.c_int), ("eps", ctypes.c_float), ("beta_logits", ctypes.c_int),
+                ("A_log", ctypes.c_void_p), ("dt_bias", ctypes.c_void_p)]
+
+
+_lib = None
+_lock = threading.Lock()
+
+
+def lib() -> ctypes.CDLL:
+    """Load libgdr.so (built in-tree by ``python -m gated_deltanet_gdr_b200.build``)."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"libgdr.so is not built ({LIB_PATH} missing); run "
+                               "`python -m gated_deltanet_gdr_b200.build` -- there is no fallback path")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, i32, f32 = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+        L.gdr_chunk_fwd.restype = i32
+        L.gdr_chunk_fwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, f32, i32, i32, i32, i32, i32, i32, i32,
+                                    ctypes.POINTER(GdrPrologueStruct), vp, vp, vp]
+        L.gdr_recurrent_step.restype = i32
+        L.gdr_recurrent_step.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, vp, vp, vp, f32, i32, i32, i32, i32, i32,
+                                         i32, i32, i32, ctypes.POINTER(GdrPrologueStruct), vp, vp]
+        L.gdr_prologue_apply.restype = i32
+        L.gdr_prologue_apply.argtypes = [vp, vp, vp, vp, vp, vp, f32, i32, i32, i32, i32, i32, i32, vp, vp, vp, vp,
+                                         vp]
+        L.gdr_get_error.restype = i32
+        L.gdr_get_error.argtypes = [vp, ctypes.POINTER(ctypes.c_int)]
+        L.gdr_status_string.restype = ctypes.c_char_p
+        L.gdr_status_string.argtypes = [i32]
+        L.gdr_version.restype = i32
+        L.gdr_version.argtypes = []
+        _lib = L
+        return L
+
+
+@dataclass
+class Prologue:
+    """Fused pre-processing (see ``gdr_prologue`` in include/gdr.h): l2norm of raw
+    q/k with eps inside the sqrt, beta from logits, g from raw a via A_log/dt_bias."""
+    l2norm_qk: bool = True
+    eps: float = 1e-6
+    beta_logits: bool = True
+    A_log: Optional[torch.Tensor] = None
+    dt_bias: Optional[torch.Tensor] = None
+
+    def as_struct(self) -> GdrPrologueStruct:
+        return GdrPrologueStruct(int(self.l2norm_qk), float(self.eps), int(self.beta_logits), _ptr(self.A_log),
+                                 _ptr(self.dt_bias))
+
+
+def _check(status: int, what: str):
+    if status == GDR_OK:
+        return
+    msg = f"{what}: {lib().gdr_status_string(status).decode()} (status {status})"
+    if status == GDR_ERR_SHAPE:
+        raise ValueError(msg)
+    raise RuntimeError(msg)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _dtype_code(dt: torch.dtype) -> int:
+    if dt == torch.float32:
+        return GDR_F32
+    if dt == torch.bfloat16:
+        return GDR_BF16
+    raise RuntimeError(f"unsupported dtype {dt}; use torch.float32 or torch.bfloat16")
+
+
+def _dev(t: torch.Tensor, name: str, dtype=None, shape=None):
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor):
+        raise RuntimeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise RuntimeError(f"{name} must be a CUDA tensor")
+    if dtype is not None and t.dtype != dtype:
+        raise RuntimeError(f"{name} must have dtype {dtype}, got {t.dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise RuntimeError(f"{name} must be contiguous")
+    return t
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def chunk_fwd(q, k, v, beta, g=None, initial_state=None, actual_seq_lengths=None, scale: float = 1.0, *,
+              prologue: Optional[Prologue] = None, out=None, final_state=None, output_final_state: bool = True,
+              stream=None):
+    """Chunked prefill (``gdr_chunk_fwd``).  Returns (out, final_state or None)."""
+    if q.dim() != 4 or v.dim() != 4:
+        raise ValueError("q, k must be (B, Nk, S, Dk) and v (B, Nv, S, Dv)")
+    B, Nk, S, Dk = q.shape
+    Nv, Dv = v.shape[1], v.shape[3]
+    dt = q.dtype
+    code = _dtype_code(dt)
+    _dev(q, "q", dt)
+    _dev(k, "k", dt, (B, Nk, S, Dk))
+    _dev(v, "v", dt, (B, Nv, S, Dv))
+    _dev(beta, "beta", dt, (B, Nv, S))
+    _dev(g, "g", torch.float32, (B, Nv, S))
+    _dev(initial_state, "initial_state", dt, (B, Nv, Dk, Dv))
+    _dev(actual_seq_lengths, "actual_seq_lengths", torch.int32, (B,))
+    if out is None:
+        out = torch.empty((B, Nv, S, Dv), dtype=dt, device=q.device)
+    _dev(out, "out", dt, (B, Nv, S, Dv))
+    if output_final_state and final_state is None:
+        final_state = torch.empty((B, Nv, Dk, Dv), dtype=dt, device=q.device)
+    _dev(final_state, "final_state", dt, (B, Nv, Dk, Dv))
+    pro = prologue.as_struct() if prologue is not None else None
+    if prologue is not None:
+        _dev(prologue.A_log, "A_log", torch.float32, (Nv,))
+        _dev(prologue.dt_bias, "dt_bias", torch.float32, (Nv,))
+    st = lib().gdr_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(g), _ptr(initial_state),
+                             _ptr(actual_seq_lengths), float(scale), B, Nk, Nv, S, Dk, Dv, code,
+                             ctypes.byref(pro) if pro is not None else None, _ptr(out), _ptr(final_state),
+                             _stream(stream))
+    _check(st, "gdr_chunk_fwd")
+    return out, final_state
+
+
+def recurrent_step(q, k, v, beta, g, gk, state_pool, ssm_state_indices, actual_seq_lengths,
+                   num_accepted_tokens=None, scale: float = 1.0, *, prologue: Optional[Prologue] = None, out=None,
+                   stream=None):
+    """Recurrent decode over a slot pool (``gdr_recurrent_step``), updating
+    ``state_pool`` in place.  Returns (out, state_pool)."""
+    if q.dim() != 4 or v.dim() != 4 or state_pool.dim() != 4:
+        raise ValueError("q, k (B, Nk, S, Dk), v (B, Nv, S, Dv), state_pool (slots, Nv, Dk, Dv)")
+    B, Nk, S, Dk = q.shape
+    Nv, Dv = v.shape[1], v.shape[3]
+    dt = q.dtype
+    code = _dtype_code(dt)
+    scode = _dtype_code(state_pool.dtype)
+    _dev(q, "q", dt)
+    _dev(k, "k", dt, (B, Nk, S, Dk))
+    _dev(v, "v", dt, (B, Nv, S, Dv))
+    _dev(beta, "beta", dt, (B, Nv, S))
+    _dev(g, "g", torch.float32, (B, Nv, S))
+    _dev(gk, "gk", torch.float32, (B, Nv, S, Dk))
+    _dev(state_pool, "state_pool", state_pool.dtype, (state_pool.shape[0], Nv, Dk, Dv))
+    if ssm_state_indices is None or ssm_state_indices.numel() != B * S:
+        raise ValueError("ssm_state_indices must hold B * S int32 slot indices, one per flattened token")
+    _dev(ssm_state_indices.reshape(-1), "ssm_state_indices", torch.int32)
+    _dev(actual_seq_lengths, "actual_seq_lengths", torch.int32, (B,))
+    _dev(num_accepted_tokens, "num_accepted_tokens", torch.int32, (B,))
+    if out is None:
+        out = torch.empty((B, Nv, S, Dv), dtype=dt, device=q.device)
+    _dev(out, "out", dt, (B, Nv, S, Dv))
+    pro = prologue.as_struct() if prologue is not None else None
+    st = lib().gdr_recurrent_step(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(g), _ptr(gk), _ptr(state_pool),
+                                  int(state_pool.shape[0]), _ptr(ssm_state_indices), _ptr(actual_seq_lengths),
+                                  _ptr(num_accepted_tokens), float(scale), B, Nk, Nv, S, Dk, Dv, code, scode,
+                                  ctypes.byref(pro) if pro is not None else None, _ptr(out), _stream(stream))
+    _check(st, "gdr_recurrent_step")
+    return out, state_pool
+
+
+def prologue(q=None, k=None, b=None, a=None, A_log=None, dt_bias=None, eps: float = 1e-6, *, stream=None):
+    """Stand-alone prologue (``gdr_prologue_apply``): returns a dict with q_hat,
+    k_hat (l2norm, eps inside the sqrt), beta = sigmoid(b) and
+    g = -exp(A_log) * softplus(a + dt_bias) for whichever inputs are given."""
+    ref = next(t for t in (q, k, b) if t is not None) if any(t is not None for t in (q, k, b)) else None
+    dt = ref.dtype if ref is not None else torch.float32
+    code = _dtype_code(dt)
+    if q is not None or k is not None:
+        B, Nk, S, Dk = (q if q is not None else k).shape
+    else:
+        B, Nk, S, Dk = (b if b is not None else a).shape[0], 1, (b if b is not None else a).shape[2], 16
+    Nv = (b if b is not None else a).shape[1] if (b is not None or a is not None) else Nk
+    res = {}
+    for name, t in (("q", q), ("k", k)):
+        if t is not None:
+            _dev(t, name, dt, (B, Nk, S, Dk))
+            res[name + "_hat"] = torch.empty_like(t)
+    if b is not None:
+        _dev(b, "b", dt, (B, Nv, S))
+        res["beta"] = torch.empty_like(b)
+    if a is not None:
+        _dev(a, "a", torch.float32, (B, Nv, S))
+        _dev(A_log, "A_log", torch.float32, (Nv,))
+        _dev(dt_bias, "dt_bias", torch.float32, (Nv,))
+        res["g"] = torch.empty_like(a)
+    st = lib().gdr_prologue_apply(_ptr(q), _ptr(k), _ptr(b), _ptr(a), _ptr(A_log), _ptr(dt_bias), float(eps), B, Nk,
+                                  Nv, S, Dk, code, _ptr(res.get("q_hat")), _ptr(res.get("k_hat")),
+                                  _ptr(res.get("beta")), _ptr(res.get("g")), _stream(stream))
+    _check(st, "gdr_prologue_apply")
+    return res
+
+
+def get_error(stream=None) -> int:
+    """Synchronise the stream and return (and clear) the device error word."""
+    v = ctypes.c_int(0)
+    _check(lib().gdr_get_error(_stream(stream), ctypes.byref(v)), "gdr_get_error")
+    return v.value
+
+
+def version() -> int:
+    return int(lib().gdr_version())

@@ -1,0 +1,203 @@
+// api.cu -- the C ABI of libgdr.so: argument checks, dispatch, device error word.
+//
+// Every entry point validates its arguments on the host before touching the GPU; on a
+// non-zero status nothing has been launched.  The library allocates no device memory.
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstdlib>
+#include <mutex>
+
+#include "../../include/gdr.h"
+#include "kernels.h"
+
+namespace gdr {
+
+// The device error word (GDR_DEVERR_* bits) of this library, one per device.
+__device__ unsigned int g_device_error = 0;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::mutex g_mu;
+int g_dev_checked[kMaxDevices];        // 0 unknown, 1 sm_100, -1 unusable
+unsigned int *g_err_ptr[kMaxDevices];  // device address of g_device_error per device
+
+bool supported_head(int d) { return d == 16 || d == 32 || d == 64 || d == 128; }
+bool aligned16(const void *p) { return p == nullptr || (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Checks the current device once (sm_100 family) and fetches the address of the error
+// word on it.  Returns GDR_OK, GDR_ERR_DEVICE or GDR_ERR_LAUNCH.
+int device_setup(unsigned int **err) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+        cudaGetLastError();
+        return GDR_ERR_DEVICE;
+    }
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (g_dev_checked[dev] == 0) {
+        int major = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) {
+            cudaGetLastError();
+            return GDR_ERR_DEVICE;
+        }
+        if (major != 10) {
+            g_dev_checked[dev] = -1;
+            return GDR_ERR_DEVICE;
+        }
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) {
+            cudaGetLastError();
+            return GDR_ERR_LAUNCH;
+        }
+        g_err_ptr[dev] = static_cast<unsigned int *>(p);
+        g_dev_checked[dev] = 1;
+    }
+    if (g_dev_checked[dev] < 0) return GDR_ERR_DEVICE;
+    *err = g_err_ptr[dev];
+    return GDR_OK;
+}
+
+int check_common(int B, int Nk, int Nv, int S, int Dk, int Dv, int dtype) {
+    if (dtype != GDR_F32 && dtype != GDR_BF16) return GDR_ERR_DTYPE;
+    if (B < 0 || S < 0 || Nk < 1 || Nv < 1 || Dk < 1 || Dv < 1) return GDR_ERR_SHAPE;
+    if (Nv % Nk != 0) return GDR_ERR_SHAPE;
+    if (!supported_head(Dk) || !supported_head(Dv)) return GDR_ERR_UNSUPPORTED;
+    // grids are one-dimensional: B * Nv * (column slabs) blocks
+    if ((long long)B * Nv * 8 >= (1LL << 31)) return GDR_ERR_SHAPE;
+    return GDR_OK;
+}
+
+int check_prologue(const gdr_prologue *p, const float *g) {
+    if (!p) return GDR_OK;
+    if (p->A_log && (!p->dt_bias || !g)) return GDR_ERR_NULL;
+    if (p->l2norm_qk && !(p->eps >= 0.f)) return GDR_ERR_SHAPE;
+    return GDR_OK;
+}
+
+}  // namespace
+}  // namespace gdr
+
+using namespace gdr;
+
+extern "C" int gdr_chunk_fwd(const void *q, const void *k, const void *v, const void *beta, const float *g,
+                             const void *initial_state, const int32_t *actual_seq_lengths, float scale, int B,
+                             int Nk, int Nv, int S, int Dk, int Dv, gdr_dtype dtype, const gdr_prologue *prologue,
+                             void *out, void *final_state, gdr_stream_t stream) {
+    int st = check_common(B, Nk, Nv, S, Dk, Dv, dtype);
+    if (st) return st;
+    if ((st = check_prologue(prologue, g))) return st;
+    if ((long long)B * S > 0 && (!q || !k || !v || !beta || !out)) return GDR_ERR_NULL;
+    const void *ptrs[] = {q, k, v, beta, g, initial_state, actual_seq_lengths, out, final_state};
+    for (const void *p : ptrs)
+        if (!aligned16(p)) return GDR_ERR_ALIGN;
+    if (B == 0 || (S == 0 && !final_state)) return GDR_OK;
+    unsigned int *err = nullptr;
+    if ((st = device_setup(&err))) return st;
+
+    ChunkArgs a{};
+    a.q = q; a.k = k; a.v = v; a.beta = beta; a.g = g;
+    a.initial_state = initial_state;
+    a.lengths = actual_seq_lengths;
+    a.scale = scale;
+    a.B = B; a.Nk = Nk; a.Nv = Nv; a.S = S;
+    a.out = out; a.final_state = final_state;
+    a.l2norm = prologue ? prologue->l2norm_qk : 0;
+    a.eps = prologue ? prologue->eps : 0.f;
+    a.beta_logits = prologue ? prologue->beta_logits : 0;
+    a.A_log = prologue ? prologue->A_log : nullptr;
+    a.dt_bias = prologue ? prologue->dt_bias : nullptr;
+    a.err = err;
+    cudaError_t e = launch_chunk_simt(a, Dk, Dv, dtype, reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? GDR_OK : GDR_ERR_LAUNCH;
+}
+
+extern "C" int gdr_recurrent_step(const void *q, const void *k, const void *v, const void *beta, const float *g,
+                                  const float *gk, void *state_pool, int slots, const int32_t *ssm_state_indices,
+                                  const int32_t *actual_seq_lengths, const int32_t *num_accepted_tokens,
+                                  float scale, int B, int Nk, int Nv, int S, int Dk, int Dv, gdr_dtype dtype,
+                                  gdr_dtype state_dtype, const gdr_prologue *prologue, void *out,
+                                  gdr_stream_t stream) {
+    int st = check_common(B, Nk, Nv, S, Dk, Dv, dtype);
+    if (st) return st;
+    if (state_dtype != GDR_F32 && state_dtype != GDR_BF16) return GDR_ERR_DTYPE;
+    if (S < 1 || S > kDecodeMaxTokens || slots < 1) return GDR_ERR_SHAPE;
+    if ((st = check_prologue(prologue, g))) return st;
+    if (B > 0 && (!q || !k || !v || !beta || !out || !state_pool || !ssm_state_indices || !actual_seq_lengths))
+        return GDR_ERR_NULL;
+    const void *ptrs[] = {q, k, v, beta, g, gk, state_pool, ssm_state_indices, actual_seq_lengths,
+                          num_accepted_tokens, out};
+    for (const void *p : ptrs)
+        if (!aligned16(p)) return GDR_ERR_ALIGN;
+    if (B == 0) return GDR_OK;
+    unsigned int *err = nullptr;
+    if ((st = device_setup(&err))) return st;
+
+    DecodeArgs a{};
+    a.q = q; a.k = k; a.v = v; a.beta = beta; a.g = g; a.gk = gk;
+    a.pool = state_pool; a.slots = slots;
+    a.idx = ssm_state_indices; a.lengths = actual_seq_lengths; a.accepted = num_accepted_tokens;
+    a.scale = scale;
+    a.B = B; a.Nk = Nk; a.Nv = Nv; a.S = S;
+    a.out = out;
+    a.l2norm = prologue ? prologue->l2norm_qk : 0;
+    a.eps = prologue ? prologue->eps : 0.f;
+    a.beta_logits = prologue ? prologue->beta_logits : 0;
+    a.A_log = prologue ? prologue->A_log : nullptr;
+    a.dt_bias = prologue ? prologue->dt_bias : nullptr;
+    a.err = err;
+    cudaError_t e = launch_decode(a, Dk, Dv, dtype, state_dtype, reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? GDR_OK : GDR_ERR_LAUNCH;
+}
+
+extern "C" int gdr_prologue_apply(const void *q, const void *k, const void *b, const float *a, const float *A_log,
+                                  const float *dt_bias, float eps, int B, int Nk, int Nv, int S, int Dk,
+                                  gdr_dtype dtype, void *q_hat, void *k_hat, void *beta, float *g,
+                                  gdr_stream_t stream) {
+    if (dtype != GDR_F32 && dtype != GDR_BF16) return GDR_ERR_DTYPE;
+    if (B < 0 || S < 0 || Nk < 1 || Nv < 1 || Dk < 1) return GDR_ERR_SHAPE;
+    if (!(eps >= 0.f)) return GDR_ERR_SHAPE;
+    if ((q && !q_hat) || (k && !k_hat) || (b && !beta) || (a && (!g || !A_log || !dt_bias))) return GDR_ERR_NULL;
+    const void *ptrs[] = {q, k, b, a, A_log, dt_bias, q_hat, k_hat, beta, g};
+    for (const void *p : ptrs)
+        if (!aligned16(p)) return GDR_ERR_ALIGN;
+    if ((long long)B * S == 0 || (!q && !k && !b && !a)) return GDR_OK;
+    unsigned int *err = nullptr;
+    int st = device_setup(&err);
+    if (st) return st;
+    cudaError_t e = launch_prologue(q, k, b, a, A_log, dt_bias, eps, B, Nk, Nv, S, Dk, dtype, q_hat, k_hat, beta, g,
+                                    reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? GDR_OK : GDR_ERR_LAUNCH;
+}
+
+extern "C" int gdr_get_error(gdr_stream_t stream, int *device_error) {
+    if (!device_error) return GDR_ERR_NULL;
+    *device_error = 0;
+    unsigned int *err = nullptr;
+    int st = device_setup(&err);
+    if (st) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    unsigned int host = 0;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return GDR_ERR_LAUNCH;
+    if (cudaMemcpyAsync(&host, err, sizeof(host), cudaMemcpyDeviceToHost, s) != cudaSuccess) return GDR_ERR_LAUNCH;
+    if (cudaMemsetAsync(err, 0, sizeof(unsigned int), s) != cudaSuccess) return GDR_ERR_LAUNCH;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return GDR_ERR_LAUNCH;
+    *device_error = (int)host;
+    return GDR_OK;
+}
+
+extern "C" const char *gdr_status_string(int status) {
+    switch (status) {
+        case GDR_OK: return "ok";
+        case GDR_ERR_SHAPE: return "invalid shape or size argument";
+        case GDR_ERR_DTYPE: return "unsupported dtype";
+        case GDR_ERR_NULL: return "a required pointer is NULL";
+        case GDR_ERR_ALIGN: return "a pointer is not 16-byte aligned";
+        case GDR_ERR_UNSUPPORTED: return "head size not built (Dk and Dv must be 16, 32, 64 or 128)";
+        case GDR_ERR_DEVICE: return "no usable sm_100 CUDA device";
+        case GDR_ERR_LAUNCH: return "a CUDA call or kernel launch failed";
+        default: return "unknown status";
+    }
+}
+
+extern "C" int gdr_version(void) { return 100; }

@@ -1,0 +1,83 @@
+// common.cuh -- small device helpers shared by the kernels of libgdr.so.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/gdr.h"
+
+namespace gdr {
+
+// Kernels receive the device address of the library's error word (GDR_DEVERR_* bits)
+// as an argument and OR their bits into it; nothing ever traps.
+__device__ __forceinline__ void raise_device_error(unsigned int *err, unsigned int bits) {
+    if (err) atomicOr(err, bits);
+}
+
+// ---- scalar conversions -------------------------------------------------------------------
+
+template <typename T> __device__ __forceinline__ float to_f32(T x);
+template <> __device__ __forceinline__ float to_f32<float>(float x) { return x; }
+template <> __device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+template <typename T> __device__ __forceinline__ T from_f32(float x);
+template <> __device__ __forceinline__ float from_f32<float>(float x) { return x; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) { return __float2bfloat16_rn(x); }
+
+// ---- 8-element vectors: one 16-byte access for bf16, two for fp32 ---------------------------
+
+template <typename T> struct Vec8;
+
+template <> struct Vec8<__nv_bfloat16> {
+    static __device__ __forceinline__ void load(const __nv_bfloat16 *p, float (&x)[8]) {
+        uint4 u = *reinterpret_cast<const uint4 *>(p);
+        const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&u);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            float2 f = __bfloat1622float2(h[i]);
+            x[2 * i] = f.x;
+            x[2 * i + 1] = f.y;
+        }
+    }
+    static __device__ __forceinline__ void store(__nv_bfloat16 *p, const float (&x)[8]) {
+        uint4 u;
+        __nv_bfloat162 *h = reinterpret_cast<__nv_bfloat162 *>(&u);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) h[i] = __floats2bfloat162_rn(x[2 * i], x[2 * i + 1]);
+        *reinterpret_cast<uint4 *>(p) = u;
+    }
+};
+
+template <> struct Vec8<float> {
+    static __device__ __forceinline__ void load(const float *p, float (&x)[8]) {
+        float4 a = *reinterpret_cast<const float4 *>(p);
+        float4 b = *reinterpret_cast<const float4 *>(p + 4);
+        x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
+        x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+    }
+    static __device__ __forceinline__ void store(float *p, const float (&x)[8]) {
+        *reinterpret_cast<float4 *>(p) = make_float4(x[0], x[1], x[2], x[3]);
+        *reinterpret_cast<float4 *>(p + 4) = make_float4(x[4], x[5], x[6], x[7]);
+    }
+};
+
+// ---- prologue arithmetic (fp32) ----------------------------------------------------------------
+
+// softplus(z) = log(1 + e^z) in the overflow-free form max(z, 0) + log1p(e^{-|z|}).
+__device__ __forceinline__ float softplus_f32(float z) { return fmaxf(z, 0.f) + log1pf(__expf(-fabsf(z))); }
+
+__device__ __forceinline__ float sigmoid_f32(float b) { return 1.f / (1.f + __expf(-b)); }
+
+// g = -exp(A_log) * softplus(a + dt_bias)
+__device__ __forceinline__ float gate_from_raw(float a, float A_log, float dt_bias) {
+    return -expf(A_log) * softplus_f32(a + dt_bias);
+}
+
+__device__ __forceinline__ float warp_sum(float x) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+    return x;
+}
+
+}  // namespace gdr

@@ -1,0 +1,51 @@
+// kernels.h -- argument blocks and launchers of the device kernels (internal to libgdr.so).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/gdr.h"
+
+namespace gdr {
+
+constexpr int kChunk = 64;            // tokens per chunk of the prefill kernels
+constexpr int kDecodeMaxTokens = 8;   // decode tokens per call (the operator is decode-only)
+
+struct DecodeArgs {
+    const void *q, *k, *v, *beta;
+    const float *g, *gk;
+    void *pool;
+    int slots;
+    const int32_t *idx, *lengths, *accepted;
+    float scale;
+    int B, Nk, Nv, S;
+    void *out;
+    int l2norm;
+    float eps;
+    int beta_logits;
+    const float *A_log, *dt_bias;
+    unsigned int *err;
+};
+
+struct ChunkArgs {
+    const void *q, *k, *v, *beta;
+    const float *g;
+    const void *initial_state;
+    const int32_t *lengths;
+    float scale;
+    int B, Nk, Nv, S;
+    void *out, *final_state;
+    int l2norm;
+    float eps;
+    int beta_logits;
+    const float *A_log, *dt_bias;
+    unsigned int *err;
+};
+
+cudaError_t launch_decode(const DecodeArgs &a, int Dk, int Dv, gdr_dtype dt, gdr_dtype st, cudaStream_t s);
+cudaError_t launch_chunk_simt(const ChunkArgs &a, int Dk, int Dv, gdr_dtype dt, cudaStream_t s);
+cudaError_t launch_prologue(const void *q, const void *k, const void *b, const float *a, const float *A_log,
+                            const float *dt_bias, float eps, int B, int Nk, int Nv, int S, int Dk, gdr_dtype dt,
+                            void *q_hat, void *k_hat, void *beta, float *g, cudaStream_t stream);
+
+}  // namespace gdr

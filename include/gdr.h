@@ -1,0 +1,194 @@
+/*
+ * gdr.h -- C ABI of the B200 (sm_100a) gated delta rule library, libgdr.so.
+ *
+ * The gated delta rule keeps, per (batch row b, value head h), a state
+ * S in R^{Dk x Dv} (row i over the key dimension, column j over the value
+ * dimension, row-major) and for each token t applies, in this order:
+ *
+ *     S   <- S * exp(g_t)            (and, for decode, row i also * exp(gk_t[i]))
+ *     m    = k_t^T S                 (readout, length Dv)
+ *     d    = beta_t * (v_t - m)      (delta)
+ *     S   <- S + k_t d^T             (rank-1 write)
+ *     o_t  = (scale * q_t)^T S       (output)
+ *
+ * Sources: the torch_recurrent_gated_delta_rule token loop of the
+ * transformers GatedDeltaNet layer (blog "gated-delta-net" page), delta_step
+ * in inferencelayer deltanet.rs, and the algorithm statement of the
+ * lite_boost recurrent_gated_delta_rule and chunk_gated_delta_rule operators.
+ *
+ * Conventions for every entry point:
+ *   - Tensors are dense, row-major (C-contiguous), in DEVICE memory of the
+ *     current CUDA device, in the BNSD layout of the lite_boost operators:
+ *       q, k           (B, Nk, S, Dk)
+ *       v, out         (B, Nv, S, Dv)
+ *       beta, g        (B, Nv, S)
+ *       gk             (B, Nv, S, Dk)
+ *       initial/final  (B, Nv, Dk, Dv)
+ *       state_pool     (slots, Nv, Dk, Dv)
+ *   - Grouped heads: Nv must be a multiple of Nk; value head h reads key head
+ *     h / (Nv / Nk) (contiguous groups, the repeat_interleave grouping).
+ *   - dtype names the type of q, k, v, beta, the state and out: GDR_F32 or
+ *     GDR_BF16.  g, gk and the prologue's a, A_log, dt_bias are always fp32.
+ *     Index arrays are int32.  Stores to bf16 round to nearest even, once.
+ *   - The caller owns every buffer.  The library allocates no device memory
+ *     and keeps no pointer after a call returns.  Work is enqueued on
+ *     `stream` (a cudaStream_t; NULL = the legacy default stream) and runs
+ *     asynchronously: the call returns before the kernels finish.
+ *   - Host-side argument checks run before anything is launched; on a non-zero
+ *     status nothing is launched and no buffer is touched.
+ *   - Device-side checks (slot index outside [0, slots), length outside
+ *     [0, S]) never trap: the affected sequence is skipped, its output rows
+ *     are written as zero, and a bit is set in the device error word read by
+ *     gdr_get_error().
+ *   - g and gk are not range-checked (the lite_boost operators document that a
+ *     min/max reduction would cost visible time on the inference path);
+ *     positive values give meaningless but finite-or-inf results.
+ */
+#ifndef GDR_H
+#define GDR_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A cudaStream_t, declared without the CUDA headers. */
+typedef struct CUstream_st *gdr_stream_t;
+
+/* Status codes.  The Python binding maps GDR_ERR_SHAPE to ValueError (the
+ * shape errors the lite_boost operators raise as ValueError) and every other
+ * non-zero status to RuntimeError. */
+typedef enum gdr_status {
+    GDR_OK = 0,
+    GDR_ERR_SHAPE = 1,       /* Nv % Nk != 0, sizes < 0, decode S > 8, slots < 1, ... */
+    GDR_ERR_DTYPE = 2,       /* unknown dtype code or unsupported dtype combination */
+    GDR_ERR_NULL = 3,        /* a required pointer is NULL */
+    GDR_ERR_ALIGN = 4,       /* a pointer is not 16-byte aligned */
+    GDR_ERR_UNSUPPORTED = 5, /* valid per the API but not built: Dk or Dv not in {16,32,64,128} */
+    GDR_ERR_DEVICE = 6,      /* no usable device, or it is not sm_100 */
+    GDR_ERR_LAUNCH = 7       /* a kernel launch or a CUDA call failed */
+} gdr_status;
+
+typedef enum gdr_dtype { GDR_F32 = 0, GDR_BF16 = 1 } gdr_dtype;
+
+/* Bits of the device error word (gdr_get_error). */
+#define GDR_DEVERR_SLOT_INDEX 0x1u /* a referenced slot index was outside [0, slots) */
+#define GDR_DEVERR_LENGTH 0x2u     /* a length was outside [0, S] */
+
+/*
+ * Optional fused prologue (the layer's pre-processing, computed in fp32
+ * inside the kernels' load stage so it costs no extra pass over memory).
+ * Source: the transformers GatedDeltaNet forward (blog page: beta =
+ * b.sigmoid(), g = -A_log.exp() * softplus(a + dt_bias), l2norm of q and k
+ * with eps 1e-6) and deltanet.rs (l2norm with eps INSIDE the square root).
+ */
+typedef struct gdr_prologue {
+    int l2norm_qk;         /* non-zero: q and k are raw; each row x becomes x / sqrt(sum x^2 + eps) */
+    float eps;             /* the l2norm epsilon (1e-6 in the layer) */
+    int beta_logits;       /* non-zero: the beta buffer holds logits b and beta = 1 / (1 + exp(-b)) */
+    const float *A_log;    /* non-NULL: the g buffer holds the raw a (fp32) and
+                              g = -exp(A_log[h]) * softplus(a + dt_bias[h]); device, (Nv) */
+    const float *dt_bias;  /* device, (Nv); required when A_log is non-NULL */
+} gdr_prologue;
+
+/*
+ * Chunked prefill.  Source: lite_boost chunk_gated_delta_rule (arguments,
+ * BNSD layout, GQA, variable lengths with padding written as zero, optional
+ * gate, final state) and torch_chunk_gated_delta_rule (chunk size 64,
+ * cumulative gate, WY/UT transform, inter-chunk carry).
+ *
+ *   q, k, v, beta          device, see layouts above (raw q, k and logits when
+ *                          the prologue asks for them)
+ *   g                      device fp32 (B, Nv, S) log-decay, or NULL: no decay
+ *                          (with prologue->A_log set: the raw a, required)
+ *   initial_state          device (B, Nv, Dk, Dv) or NULL: zeros
+ *   actual_seq_lengths     device int32 (B) or NULL: every sequence has S
+ *                          tokens.  Tokens t >= L_b are padding: their input
+ *                          contents are ignored (they may hold any finite or
+ *                          non-finite values) and out rows t >= L_b are zero.
+ *                          L_b = 0 gives final_state = initial_state exactly.
+ *   scale                  multiplies q before the rule (1/sqrt(Dk) in the layer)
+ *   out                    device (B, Nv, S, Dv), written in full
+ *   final_state            device (B, Nv, Dk, Dv) or NULL: not written.  It
+ *                          may alias initial_state (in-place update).
+ * Constraints: B, S >= 0; Nk, Nv >= 1; Nv % Nk == 0; Dk, Dv in {16,32,64,128};
+ * every pointer 16-byte aligned.  bf16 with Dk = Dv = 128 runs on the
+ * tensor-core (tcgen05) path; other shapes and fp32 run the CUDA-core path.
+ */
+int gdr_chunk_fwd(const void *q, const void *k, const void *v, const void *beta, const float *g,
+                  const void *initial_state, const int32_t *actual_seq_lengths, float scale, int B, int Nk,
+                  int Nv, int S, int Dk, int Dv, gdr_dtype dtype, const gdr_prologue *prologue, void *out,
+                  void *final_state, gdr_stream_t stream);
+
+/*
+ * Recurrent decode over a pool of state slots.  Source: lite_boost
+ * recurrent_gated_delta_rule (state pool, ssm_state_indices with one slot per
+ * flattened token, gk, num_accepted_tokens, S <= 8, the decay
+ * S * exp(g) * exp(gk)).
+ *
+ *   q, k, v, beta, g       as for gdr_chunk_fwd (g may be NULL: no decay)
+ *   gk                     device fp32 (B, Nv, S, Dk) per-key-row log-decay,
+ *                          or NULL
+ *   state_pool             device (slots, Nv, Dk, Dv) in state_dtype, read and
+ *                          updated IN PLACE.  Slots no token commits to are
+ *                          left byte-identical.
+ *   ssm_state_indices      device int32 (B * S): slot of token (b, t) is
+ *                          ssm_state_indices[b * S + t]
+ *   actual_seq_lengths     device int32 (B): tokens processed for sequence b,
+ *                          in [0, S]; out rows t >= L_b are zero
+ *   num_accepted_tokens    device int32 (B), or NULL (= actual_seq_lengths)
+ *   out                    device (B, Nv, S, Dv), written in full
+ * Reading of num_accepted_tokens (the operator defines it only as the count of
+ * accepted tokens, equal to the lengths in plain inference): the chain starts
+ * from slot ssm_state_indices[b * S]; all L_b tokens are processed and
+ * output; the state after token t is committed to slot
+ * ssm_state_indices[b * S + t] only when t < min(A_b, L_b).  Two sequences
+ * must not reference the same slot (their updates would race).
+ * Constraints: 1 <= S <= 8 (the operator is decode-only), slots >= 1, other
+ * constraints as for gdr_chunk_fwd.  state_dtype may be GDR_F32 or GDR_BF16
+ * independently of dtype.
+ */
+int gdr_recurrent_step(const void *q, const void *k, const void *v, const void *beta, const float *g,
+                       const float *gk, void *state_pool, int slots, const int32_t *ssm_state_indices,
+                       const int32_t *actual_seq_lengths, const int32_t *num_accepted_tokens, float scale, int B,
+                       int Nk, int Nv, int S, int Dk, int Dv, gdr_dtype dtype, gdr_dtype state_dtype,
+                       const gdr_prologue *prologue, void *out, gdr_stream_t stream);
+
+/*
+ * Stand-alone prologue (the same arithmetic the fused prologue applies), for
+ * callers that want the normalised tensors materialised.  Source: as for
+ * gdr_prologue.
+ *   q, k      device (B, Nk, S, Dk) raw, or NULL to skip; written to q_hat,
+ *             k_hat (same dtype, may alias the inputs) as x / sqrt(sum x^2 + eps)
+ *   b         device (B, Nv, S) logits in dtype, or NULL; beta = sigmoid(b)
+ *             written to beta (dtype, may alias b)
+ *   a         device fp32 (B, Nv, S), or NULL; g = -exp(A_log[h]) *
+ *             softplus(a + dt_bias[h]) written to g (fp32, may alias a);
+ *             A_log and dt_bias are device fp32 (Nv), required with a
+ */
+int gdr_prologue_apply(const void *q, const void *k, const void *b, const float *a, const float *A_log,
+                       const float *dt_bias, float eps, int B, int Nk, int Nv, int S, int Dk, gdr_dtype dtype,
+                       void *q_hat, void *k_hat, void *beta, float *g, gdr_stream_t stream);
+
+/*
+ * Waits for `stream`, then returns in *device_error the device error word
+ * (GDR_DEVERR_* bits accumulated by every kernel of this library on the
+ * current device since the last call) and clears it.  Returns GDR_OK or
+ * GDR_ERR_LAUNCH if a CUDA call failed (including an earlier asynchronous
+ * kernel fault on the stream).
+ */
+int gdr_get_error(gdr_stream_t stream, int *device_error);
+
+/* Static description of a status code; never NULL. */
+const char *gdr_status_string(int status);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+int gdr_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GDR_H */

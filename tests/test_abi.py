@@ -1,0 +1,129 @@
+"""The C ABI library: it builds, loads without a GPU, exports what the header
+declares, and rejects bad arguments on the host before launching anything.
+
+Every call below that passes placeholder pointers is built so that host-side
+validation must reject it; none can reach a kernel launch.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+import gated_deltanet_gdr_b200 as gdr
+from gated_deltanet_gdr_b200 import build as gbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "gdr.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    gbuild.build()
+    return gdr.lib()
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(gdr_[a-z_0-9]+)\s*\(", src)))
+
+
+def test_exports_every_declared_symbol(L):
+    names = declared_functions()
+    assert set(names) == set(gdr.EXPORTED), names
+    for n in names:
+        assert hasattr(L, n), f"libgdr.so does not export {n}"
+
+
+def test_status_strings_and_version(L):
+    for s in range(8):
+        assert L.gdr_status_string(s)
+    assert b"unknown" in L.gdr_status_string(99)
+    assert gdr.version() == 100
+
+
+P = ctypes.c_void_p(4096)  # placeholder: aligned, non-NULL, never dereferenced (every call is rejected first)
+NUL = None
+
+
+def chunk(L, **kw):
+    a = dict(q=P, k=P, v=P, beta=P, g=NUL, s0=NUL, lens=NUL, scale=1.0, B=1, Nk=2, Nv=4, S=8, Dk=128, Dv=128,
+             dt=gdr.GDR_BF16, pro=None, out=P, fin=NUL)
+    a.update(kw)
+    return L.gdr_chunk_fwd(a["q"], a["k"], a["v"], a["beta"], a["g"], a["s0"], a["lens"], a["scale"], a["B"],
+                           a["Nk"], a["Nv"], a["S"], a["Dk"], a["Dv"], a["dt"], a["pro"], a["out"], a["fin"], None)
+
+
+def decode(L, **kw):
+    a = dict(q=P, k=P, v=P, beta=P, g=NUL, gk=NUL, pool=P, slots=4, idx=P, lens=P, acc=NUL, scale=1.0, B=1, Nk=2,
+             Nv=4, S=1, Dk=128, Dv=128, dt=gdr.GDR_BF16, sdt=gdr.GDR_BF16, pro=None, out=P)
+    a.update(kw)
+    return L.gdr_recurrent_step(a["q"], a["k"], a["v"], a["beta"], a["g"], a["gk"], a["pool"], a["slots"], a["idx"],
+                                a["lens"], a["acc"], a["scale"], a["B"], a["Nk"], a["Nv"], a["S"], a["Dk"], a["Dv"],
+                                a["dt"], a["sdt"], a["pro"], a["out"], None)
+
+
+def test_chunk_host_validation(L):
+    assert chunk(L, Nv=3) == gdr.GDR_ERR_SHAPE  # Nv % Nk != 0
+    assert chunk(L, Nk=0) == gdr.GDR_ERR_SHAPE
+    assert chunk(L, B=-1) == gdr.GDR_ERR_SHAPE
+    assert chunk(L, S=-5) == gdr.GDR_ERR_SHAPE
+    assert chunk(L, dt=7) == gdr.GDR_ERR_DTYPE
+    assert chunk(L, Dk=96) == gdr.GDR_ERR_UNSUPPORTED
+    assert chunk(L, Dv=256) == gdr.GDR_ERR_UNSUPPORTED
+    assert chunk(L, q=NUL) == gdr.GDR_ERR_NULL
+    assert chunk(L, out=NUL) == gdr.GDR_ERR_NULL
+    assert chunk(L, v=ctypes.c_void_p(4104)) == gdr.GDR_ERR_ALIGN
+    assert chunk(L, fin=ctypes.c_void_p(4097)) == gdr.GDR_ERR_ALIGN
+    pro = gdr.GdrPrologueStruct(1, 1e-6, 1, 4096, None)  # A_log without dt_bias
+    assert chunk(L, pro=ctypes.byref(pro), g=P) == gdr.GDR_ERR_NULL
+    pro = gdr.GdrPrologueStruct(1, 1e-6, 1, 4096, 8192)  # A_log without the raw a (g buffer)
+    assert chunk(L, pro=ctypes.byref(pro)) == gdr.GDR_ERR_NULL
+    pro = gdr.GdrPrologueStruct(1, -1.0, 0, None, None)  # negative eps
+    assert chunk(L, pro=ctypes.byref(pro)) == gdr.GDR_ERR_SHAPE
+    # nothing to do: B == 0 returns OK without touching a device
+    assert chunk(L, B=0, q=NUL, k=NUL, v=NUL, beta=NUL, out=NUL) == gdr.GDR_OK
+
+
+def test_decode_host_validation(L):
+    assert decode(L, S=9) == gdr.GDR_ERR_SHAPE  # decode-only operator: S <= 8
+    assert decode(L, S=0) == gdr.GDR_ERR_SHAPE
+    assert decode(L, slots=0) == gdr.GDR_ERR_SHAPE
+    assert decode(L, Nv=6, Nk=4) == gdr.GDR_ERR_SHAPE
+    assert decode(L, sdt=3) == gdr.GDR_ERR_DTYPE
+    assert decode(L, pool=NUL) == gdr.GDR_ERR_NULL
+    assert decode(L, idx=NUL) == gdr.GDR_ERR_NULL
+    assert decode(L, lens=NUL) == gdr.GDR_ERR_NULL
+    assert decode(L, gk=ctypes.c_void_p(4100)) == gdr.GDR_ERR_ALIGN
+    assert decode(L, Dk=48) == gdr.GDR_ERR_UNSUPPORTED
+    assert decode(L, B=0) == gdr.GDR_OK
+
+
+def test_prologue_host_validation(L):
+    f = L.gdr_prologue_apply
+    assert f(P, NUL, NUL, NUL, NUL, NUL, 1e-6, 1, 1, 1, 4, 16, 5, P, NUL, NUL, NUL, None) == gdr.GDR_ERR_DTYPE
+    assert f(P, NUL, NUL, NUL, NUL, NUL, 1e-6, 1, 1, 1, 4, 16, 0, NUL, NUL, NUL, NUL, None) == gdr.GDR_ERR_NULL
+    assert f(NUL, NUL, NUL, P, NUL, P, 1e-6, 1, 1, 1, 4, 16, 0, NUL, NUL, NUL, P, None) == gdr.GDR_ERR_NULL
+    assert f(P, NUL, NUL, NUL, NUL, NUL, -1.0, 1, 1, 1, 4, 16, 0, P, NUL, NUL, NUL, None) == gdr.GDR_ERR_SHAPE
+    assert f(NUL, NUL, NUL, NUL, NUL, NUL, 1e-6, 1, 1, 1, 4, 16, 0, NUL, NUL, NUL, NUL, None) == gdr.GDR_OK
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device status; on a GPU host the "
+                    "placeholder pointers would be launched on")
+def test_no_device_status(L):
+    assert chunk(L) == gdr.GDR_ERR_DEVICE
+    v = ctypes.c_int(5)
+    assert L.gdr_get_error(None, ctypes.byref(v)) == gdr.GDR_ERR_DEVICE
+    assert v.value == 0
+
+
+def test_binding_rejects_host_tensors_and_bad_dtypes():
+    q = torch.zeros(1, 1, 4, 16)
+    with pytest.raises(RuntimeError):
+        gdr.chunk_fwd(q, q, q, torch.zeros(1, 1, 4))
+    with pytest.raises(RuntimeError):
+        gdr._dtype_code(torch.float16)
+    with pytest.raises(ValueError):
+        gdr.chunk_fwd(torch.zeros(4, 16), q, q, q)
