@@ -108,7 +108,8 @@ extern "C" int gdr_chunk_fwd(const void *q, const void *k, const void *v, const 
     a.A_log = prologue ? prologue->A_log : nullptr;
     a.dt_bias = prologue ? prologue->dt_bias : nullptr;
     a.err = err;
-    cudaError_t e = launch_chunk_simt(a, Dk, Dv, dtype, reinterpret_cast<cudaStream_t>(stream));
+    cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = chunk_tc_supported(Dk, Dv, dtype, S) ? launch_chunk_tc(a, cs) : launch_chunk_simt(a, Dk, Dv, dtype, cs);
     return e == cudaSuccess ? GDR_OK : GDR_ERR_LAUNCH;
 }
 

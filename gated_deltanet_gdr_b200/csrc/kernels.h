@@ -43,6 +43,8 @@ struct ChunkArgs {
 };
 
 cudaError_t launch_decode(const DecodeArgs &a, int Dk, int Dv, gdr_dtype dt, gdr_dtype st, cudaStream_t s);
+bool chunk_tc_supported(int Dk, int Dv, gdr_dtype dt, int S);
+cudaError_t launch_chunk_tc(const ChunkArgs &a, cudaStream_t s);
 cudaError_t launch_chunk_simt(const ChunkArgs &a, int Dk, int Dv, gdr_dtype dt, cudaStream_t s);
 cudaError_t launch_prologue(const void *q, const void *k, const void *b, const float *a, const float *A_log,
                             const float *dt_bias, float eps, int B, int Nk, int Nv, int S, int Dk, gdr_dtype dt,
