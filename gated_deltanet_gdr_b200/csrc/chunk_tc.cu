@@ -3,27 +3,32 @@
 // The chunked (WY / UT transform) form of torch_chunk_gated_delta_rule (blog
 // "gated-delta-net" page, steps 1-8), chunk C = 64, head size Dk = Dv = 128, bf16 in
 // and out, fp32 accumulation and an fp32 state.  One CTA owns one (b, value head)
-// chain and walks its chunks in order; per chunk:
+// chain.  Per chunk:
 //
 //   a1  G_t = cumulative log-gate (tokens past the length count 0).
-//   a2  [G; P] = [K; Q] K^T                 tcgen05.mma  M=128 N=64  K=128
-//   a3  A = strictLower(beta_t k_t.k_s e^{G_t-G_s}),  T = (I + A)^{-1}  (fp32, CUDA cores:
-//       16x16 diagonal blocks by forward substitution, merged 16 -> 32 -> 64 with
-//       T21 = -T22 A21 T11)
-//   a4  W = T diag(beta e^G) K,  U = T diag(beta) V   tcgen05.mma  M=128 N=128 K=64 (x2)
-//   a5  R = [W; diag(e^G) X] S              tcgen05.mma  M=128 N=128 K=128
+//   a2  [G; P] = [K; Q] K^T                       tcgen05.mma  M=128 N=64  K=128
+//   a3  A = strictLower(beta_t k_t.k_s e^{G_t-G_s});  T = (I + A)^{-1} in fp32 on the CUDA
+//       cores: 16x16 diagonal blocks by forward substitution, merged 16 -> 32 -> 64 with
+//       T21 = -T22 A21 T11 (register-blocked, fully unrolled).
+//   a4  W = T diag(beta e^G) K,  U = T diag(beta) V        tcgen05.mma  M=128 N=128 K=64
+//   a5  R = [W; diag(e^G) X] S                    tcgen05.mma  M=128 N=128 K=128
 //       v_new = U - R[0:64]
-//       dS = (diag(e^{G_last-G}) K)^T v_new tcgen05.mma  M=128 N=128 K=64
-//       R[64:128] += Pm v_new, Pm = (X K^T) * e^{G_t-G_s} (causal)  -> o
-//       S = e^{G_last} S + dS               (fp32, in registers)
-//   a6  o -> bf16 -> TMA store; padding rows and chunks zero; final state once.
+//       S <- e^{G_last} S  (in TMEM, while R is computed)
+//       S += (diag(e^{G_last-G}) K)^T v_new       tcgen05.mma  accumulate into the TMEM state
+//       R[64:128] += Pm v_new,  Pm = (X K^T) e^{G_t-G_s} (causal)  -> o
+//   a6  o -> bf16 -> TMA store; padding rows and chunks are zero; the final state is
+//       written once from TMEM.
 //
-// X = scale * q / |q| (the fused l2norm and the 1/|k| factors are folded into the
-// row/column scalings above, so raw q/k tiles feed the tensor cores directly).
-// Operands are staged by TMA with 128-byte swizzle; accumulators live in TMEM
-// (448 of 512 columns); the MMA is issued by one thread and completion is signalled
-// through tcgen05.commit on an mbarrier.  Every wait is bounded: on a timeout the
-// CTA sets GDR_DEVERR_TIMEOUT, releases TMEM and returns.
+// X = scale * q / |q| (the fused l2norm and the 1/|k| factors are folded into row and
+// column scalings, so the raw q/k tiles feed the tensor cores directly).
+//
+// Warp roles: warps 0-7 ("carry") run the serial chain of chunk c -- the three MMAs that
+// touch the state and their epilogues; warps 8-15 ("prep") meanwhile prepare chunk c+1
+// (tile loads, norms, gate scan, [G; P], the solve, W and U, the X_g and K~ operands).
+// They hand over through mbarriers: a1_ready (prep -> carry: operands of chunk c are in
+// place) and mma2_done (carry -> prep: the MMAs of chunk c-1 that read the shared
+// operand buffers have completed).  Every wait is bounded: on a timeout the CTA sets
+// the timeout bit of the device error word, releases TMEM and returns.
 #include <cuda.h>
 
 #include "common.cuh"
@@ -33,35 +38,59 @@
 namespace gdr {
 using namespace sm100;
 
+#ifdef GDR_PHASE_TIMERS
+// Development aid, compiled only with -DGDR_PHASE_TIMERS: accumulated clock64() cycles per
+// phase of CTA 0 (slots 0..15 prep group, 16..31 carry group), read by gdr_phase_timers_read.
+__device__ unsigned long long g_phase[64];
+#define PHASE(slot)                                                            \
+    do {                                                                       \
+        if (blockIdx.x == 0 && (tid == 0 || tid == NGRP)) {                    \
+            const unsigned long long now_ = clock64();                         \
+            g_phase[(slot)] += now_ - t_prev_;                                 \
+            t_prev_ = now_;                                                    \
+        }                                                                      \
+    } while (0)
+#else
+#define PHASE(slot) \
+    do {            \
+    } while (0)
+#endif
+
 namespace {
 
-constexpr int C = 64, D = 128, NT = 256;
+constexpr int C = 64, D = 128, NT = 512, NGRP = 256;
+constexpr int BAR_CARRY = 1, BAR_PREP = 2;
 constexpr uint32_t kTimeoutBit = 0x4u;
 
 // ---- shared memory map (bytes from a 1024-aligned base) ----
 // input stage: [K_b0 | Q_b0 | K_b1 | Q_b1 | V_b0 | V_b1], each 64 rows x 128 B (64 bf16)
-constexpr uint32_t OFF_K0 = 0, OFF_Q0 = 8192, OFF_K1 = 16384, OFF_Q1 = 24576, OFF_V0 = 32768, OFF_V1 = 40960;
+constexpr uint32_t OFF_K0 = 0, OFF_Q0 = 8192, OFF_K1 = 16384, OFF_Q1 = 24576, OFF_V0 = 32768;
 constexpr uint32_t STAGE_BYTES = 49152;
 constexpr uint32_t OFF_A1 = 49152;   // [W; X_g] K-major 128 x 128: dk blocks at +0, +16K
 constexpr uint32_t OFF_S = 81920;    // S bf16, MN-major (K = dk rows, N = dv): dv blocks at +0, +16K
 constexpr uint32_t OFF_KT = 114688;  // K~ MN-major (M = dk, K = tok): dk blocks at +0, +8K
-constexpr uint32_t OFF_TT = 131072;  // [T diag(beta); T diag(c_W)] K-major 128 x 64
-constexpr uint32_t OFF_PM = 147456;  // [0; Pm] K-major 128 x 64
-constexpr uint32_t OFF_O = 163840;   // out tile [tok][dv]: dv blocks at +0, +8K (TMA store source)
-constexpr uint32_t OFF_R1 = 180224;  // solve workspace, aliased later in the chunk by VN
-constexpr uint32_t OFF_VN = OFF_R1;  // v_new MN-major (K = tok, N = dv): dv blocks at +0, +8K
-constexpr int FP = 65;               // padded fp32 row stride of the solve matrices
-constexpr uint32_t OFF_AF = OFF_R1;
-constexpr uint32_t OFF_TF = OFF_AF + 64 * FP * 4;
-constexpr uint32_t OFF_X = OFF_TF + 64 * FP * 4;  // 32 x 33 fp32 scratch
-constexpr uint32_t OFF_VEC = OFF_X + 32 * 33 * 4;
-constexpr uint32_t OFF_BAR = OFF_VEC + 8 * 64 * 4;
-constexpr uint32_t SMEM_USED = OFF_BAR + 64;
+constexpr uint32_t OFF_PM = 131072;  // [0; Pm] K-major 128 x 64
+constexpr uint32_t OFF_VO = 147456;  // v_new (MN-major, K = tok, N = dv) then the out tile: dv blocks +0, +8K
+constexpr int FP = 68;               // row stride (floats) of T and E: 16-byte aligned rows for float4 access
+constexpr int FA = 65;               // row stride of A: odd, so the row-per-thread stores are conflict-free
+constexpr int XP = 36;               // row stride of the merge scratch
+constexpr uint32_t OFF_AF = 163840;  // A (fp32); after the solve it holds TT = [T diag(beta); T diag(c_W)]
+constexpr uint32_t OFF_TT = OFF_AF;
+constexpr uint32_t OFF_TF = OFF_AF + 64 * FA * 4;  // T (fp32)
+constexpr uint32_t OFF_E = OFF_TF + 64 * FP * 4;   // E[t][s] = e^{G_t - G_s} (s <= t), fp32
+constexpr uint32_t OFF_X = OFF_E + 64 * FP * 4;
+constexpr uint32_t OFF_VEC = OFF_X + 32 * XP * 4;  // 2 sets x 8 vectors x 64 floats
+constexpr uint32_t OFF_BAR = OFF_VEC + 2 * 8 * 64 * 4;
+constexpr uint32_t SMEM_USED = OFF_BAR + 128;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;  // + alignment slack
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+static_assert(OFF_TF % 16 == 0 && OFF_E % 16 == 0 && OFF_X % 16 == 0, "float4 alignment");
+static_assert(OFF_TF >= OFF_TT + 16384, "TT must fit inside the A matrix area");
 
-// TMEM columns
-constexpr uint32_t TM_GP = 0, TM_WD = 64, TM_U = 192, TM_R = 320, TM_COLS = 512;
+// TMEM columns (all 128 lanes): [G;P] then W, U, R = [W S; o], the fp32 state S
+constexpr uint32_t TM_GPW = 0, TM_U = 128, TM_R = 256, TM_S = 384, TM_COLS = 512;
+
+enum { V_BETA = 0, V_GAM, V_EG, V_TAIL, V_RK, V_RQ, V_CW, V_N };
 
 struct TcArgs {
     const void *beta;
@@ -82,7 +111,6 @@ __device__ __forceinline__ uint32_t blk_off(uint32_t row, uint32_t col) {  // wi
     return (row >> 3) * 1024u + sw128_offset(row & 7u, col);
 }
 
-// 16 bytes of 8 bf16 <-> 8 floats
 __device__ __forceinline__ void unpack8(uint4 u, float (&f)[8]) {
     const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&u);
 #pragma unroll
@@ -97,17 +125,18 @@ __device__ __forceinline__ uint4 pack8(const float *f) {
                       pack_bf16x2(f[6], f[7]));
 }
 
-// T = (I + A)^{-1} for a strictly lower 64 x 64 A (fp32, row stride FP), 256 threads.
-__device__ void solve_unit_lower(const float *sA, float *sT, float *sX, int tid) {
-    // 16 x 16 diagonal blocks, one column per thread (64 threads)
-    if (tid < 64) {
-        const int base = (tid >> 4) * 16, j = tid & 15;
+// T = (I + A)^{-1} for a strictly lower 64 x 64 A (fp32, row stride FA; T row stride FP), by the 256 prep
+// threads (p = 0..255).  Writes the lower triangle of T and zeros in the upper 16 x 16
+// blocks that the merges read.
+__device__ __forceinline__ void solve_unit_lower(const float *sA, float *sT, float *sX, int p) {
+    if (p < 64) {  // 16 x 16 diagonal blocks, one column per thread
+        const int base = (p >> 4) * 16, j = p & 15;
         float x[16];
 #pragma unroll
         for (int t = 0; t < 16; ++t) x[t] = (t == j) ? 1.f : 0.f;
 #pragma unroll
         for (int t = 1; t < 16; ++t) {
-            const float *ar = sA + (base + t) * FP + base;
+            const float *ar = sA + (base + t) * FA + base;
             float a0 = 0.f, a1 = 0.f;
 #pragma unroll
             for (int s = 0; s < t; ++s) {
@@ -118,38 +147,65 @@ __device__ void solve_unit_lower(const float *sA, float *sT, float *sX, int tid)
         }
 #pragma unroll
         for (int t = 0; t < 16; ++t) sT[(base + t) * FP + base + j] = x[t];
+    } else {  // zero the upper 16 x 16 blocks inside the two 32 x 32 diagonal blocks
+        for (int e = p - 64; e < 512; e += NGRP - 64) {
+            const int blk = e >> 8, r = (e >> 4) & 15, c = e & 15;
+            sT[(32 * blk + r) * FP + 32 * blk + 16 + c] = 0.f;
+        }
     }
-    __syncthreads();
-    // 16 -> 32: for p in {0,1}: T[r0.., c0..] = -T22 (A21 T11), r0 = 32p + 16, c0 = 32p
-    for (int e = tid; e < 512; e += NT) {
-        const int p = e >> 8, r = (e >> 4) & 15, c = e & 15, r0 = 32 * p + 16, c0 = 32 * p;
-        float acc = 0.f;
-        for (int k = c; k < 16; ++k) acc = fmaf(sA[(r0 + r) * FP + c0 + k], sT[(c0 + k) * FP + c0 + c], acc);
-        sX[e] = acc;
+    named_sync(BAR_PREP, NGRP);
+    // 16 -> 32: X_b = A21 T11, then T21 = -T22 X_b, for the blocks at rows 32b+16, cols 32b
+    {
+        const int blk = p >> 7, r = (p >> 3) & 15, c2 = (p & 7) * 2, r0 = 32 * blk + 16, c0 = 32 * blk;
+        float x0 = 0.f, x1 = 0.f;
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+            const float a = sA[(r0 + r) * FA + c0 + k];
+            const float2 t = *reinterpret_cast<const float2 *>(sT + (c0 + k) * FP + c0 + c2);
+            x0 = fmaf(a, t.x, x0);
+            x1 = fmaf(a, t.y, x1);
+        }
+        *reinterpret_cast<float2 *>(sX + (blk * 16 + r) * XP + c2) = make_float2(x0, x1);
+        named_sync(BAR_PREP, NGRP);
+        float y0 = 0.f, y1 = 0.f;
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+            const float t = sT[(r0 + r) * FP + r0 + k];
+            const float2 xx = *reinterpret_cast<const float2 *>(sX + (blk * 16 + k) * XP + c2);
+            y0 = fmaf(t, xx.x, y0);
+            y1 = fmaf(t, xx.y, y1);
+        }
+        *reinterpret_cast<float2 *>(sT + (r0 + r) * FP + c0 + c2) = make_float2(-y0, -y1);
     }
-    __syncthreads();
-    for (int e = tid; e < 512; e += NT) {
-        const int p = e >> 8, r = (e >> 4) & 15, c = e & 15, r0 = 32 * p + 16, c0 = 32 * p;
-        float acc = 0.f;
-        for (int k = 0; k <= r; ++k) acc = fmaf(sT[(r0 + r) * FP + r0 + k], sX[(p << 8) + (k << 4) + c], acc);
-        sT[(r0 + r) * FP + c0 + c] = -acc;
+    named_sync(BAR_PREP, NGRP);
+    // 32 -> 64: X = A21 T11, T21 = -T22 X with 32 x 32 blocks; one row x 4 columns per thread
+    {
+        const int r = p >> 3, c4 = (p & 7) * 4;
+        float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int k = 0; k < 32; ++k) {
+            const float a = sA[(32 + r) * FA + k];
+            const float4 t = *reinterpret_cast<const float4 *>(sT + k * FP + c4);
+            x.x = fmaf(a, t.x, x.x);
+            x.y = fmaf(a, t.y, x.y);
+            x.z = fmaf(a, t.z, x.z);
+            x.w = fmaf(a, t.w, x.w);
+        }
+        *reinterpret_cast<float4 *>(sX + r * XP + c4) = x;
+        named_sync(BAR_PREP, NGRP);
+        float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int k = 0; k < 32; ++k) {
+            const float t = sT[(32 + r) * FP + 32 + k];
+            const float4 xx = *reinterpret_cast<const float4 *>(sX + k * XP + c4);
+            y.x = fmaf(t, xx.x, y.x);
+            y.y = fmaf(t, xx.y, y.y);
+            y.z = fmaf(t, xx.z, y.z);
+            y.w = fmaf(t, xx.w, y.w);
+        }
+        *reinterpret_cast<float4 *>(sT + (32 + r) * FP + c4) = make_float4(-y.x, -y.y, -y.z, -y.w);
     }
-    __syncthreads();
-    // 32 -> 64: T[32.., 0..32] = -T22 (A21 T11)
-    for (int e = tid; e < 1024; e += NT) {
-        const int r = e >> 5, c = e & 31;
-        float acc = 0.f;
-        for (int k = c; k < 32; ++k) acc = fmaf(sA[(32 + r) * FP + k], sT[k * FP + c], acc);
-        sX[r * 33 + c] = acc;
-    }
-    __syncthreads();
-    for (int e = tid; e < 1024; e += NT) {
-        const int r = e >> 5, c = e & 31;
-        float acc = 0.f;
-        for (int k = 0; k <= r; ++k) acc = fmaf(sT[(32 + r) * FP + 32 + k], sX[k * 33 + c], acc);
-        sT[(32 + r) * FP + c] = -acc;
-    }
-    __syncthreads();
+    named_sync(BAR_PREP, NGRP);
 }
 
 __global__ void __launch_bounds__(NT, 1)
@@ -158,16 +214,18 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     extern __shared__ uint8_t smraw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smraw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = smem_u32(sm);
-    float *sBeta = reinterpret_cast<float *>(sm + OFF_VEC);
-    float *sGam = sBeta + 64, *sEG = sGam + 64, *sTail = sEG + 64, *sRk = sTail + 64, *sRq = sRk + 64;
-    float *sCw = sRq + 64;
+    float *vecs = reinterpret_cast<float *>(sm + OFF_VEC);
     uint64_t *bar_ld = reinterpret_cast<uint64_t *>(sm + OFF_BAR);
-    uint64_t *bar_mma = bar_ld + 1;
-    uint32_t *s_tmem = reinterpret_cast<uint32_t *>(bar_ld + 2);
+    uint64_t *bar_gp = bar_ld + 1, *bar_wu = bar_ld + 2, *bar_m1 = bar_ld + 3, *bar_m2 = bar_ld + 4;
+    uint64_t *bar_a1 = bar_ld + 5;
+    uint32_t *s_tmem = reinterpret_cast<uint32_t *>(bar_ld + 8);
+    volatile int *s_abort = reinterpret_cast<volatile int *>(s_tmem + 1);
     float *sA = reinterpret_cast<float *>(sm + OFF_AF), *sT = reinterpret_cast<float *>(sm + OFF_TF);
     float *sX = reinterpret_cast<float *>(sm + OFF_X);
+    float *sE = reinterpret_cast<float *>(sm + OFF_E);
 
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, q4 = warp & 3, hf = warp >> 2;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, q4 = warp & 3, hf = (warp >> 2) & 1;
+    const bool carry = warp < 8;
     const int bh = blockIdx.x, h = bh % a.Nv, b = bh / a.Nv, kh = h / (a.Nv / a.Nk);
     const int S = a.S;
     int L = a.lengths ? a.lengths[b] : S;
@@ -176,11 +234,12 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const int nvalid = (L + C - 1) / C, ntotal = (S + C - 1) / C;
     const int zq = b * a.Nk + kh;  // TMA z coordinate of q/k rows
     const uint32_t lane_base = (uint32_t)(q4 * 32) << 16;
+    const int row = q4 * 32 + lane;  // TMEM lane of this thread
 
     if (tid == 0) {
         if (bad_len) raise_device_error(a.err, GDR_DEVERR_LENGTH);
-        mbar_init(bar_ld, 1);
-        mbar_init(bar_mma, 1);
+        for (int i = 0; i < 6; ++i) mbar_init(bar_ld + i, 1);
+        *s_abort = 0;
         fence_mbar_init();
         prefetch_tmap(&tm_q);
         prefetch_tmap(&tm_k);
@@ -188,301 +247,389 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         prefetch_tmap(&tm_o);
     }
     if (warp == 0) tmem_alloc(s_tmem, TM_COLS);
-    // rows 0..63 of the [0; Pm] operand stay zero
     for (int e = tid; e < 8192 / 16; e += NT) reinterpret_cast<uint4 *>(sm + OFF_PM)[e] = make_uint4(0, 0, 0, 0);
-
-    // ---- initial state: thread owns dk row i, dv columns [64 hf, 64 hf + 64) ----
-    const int srow = q4 * 32 + lane;
-    float st[64];
-    {
-        const __nv_bfloat16 *s0 = reinterpret_cast<const __nv_bfloat16 *>(a.initial_state);
-        const size_t off = ((size_t)bh * D + srow) * D + 64 * hf;
-#pragma unroll
-        for (int c8 = 0; c8 < 8; ++c8) {
-            float f[8];
-            if (s0) {
-                unpack8(*reinterpret_cast<const uint4 *>(s0 + off + 8 * c8), f);
-            } else {
-#pragma unroll
-                for (int i = 0; i < 8; ++i) f[i] = 0.f;
-            }
-#pragma unroll
-            for (int i = 0; i < 8; ++i) st[8 * c8 + i] = f[i];
-            *reinterpret_cast<uint4 *>(sm + OFF_S + hf * 16384 + blk_off(srow, 8 * c8)) = pack8(&st[8 * c8]);
-        }
-    }
-    fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *s_tmem;
 
-    uint32_t ph_ld = 0, ph_mma = 0;
-    bool ok = true;
-    auto issue_loads = [&](int chunk) {
-        const int y = chunk * C;
-        mbar_arrive_expect_tx(bar_ld, STAGE_BYTES);
-        tma_load_3d(sm + OFF_K0, &tm_k, bar_ld, 0, y, zq);
-        tma_load_3d(sm + OFF_K1, &tm_k, bar_ld, 64, y, zq);
-        tma_load_3d(sm + OFF_Q0, &tm_q, bar_ld, 0, y, zq);
-        tma_load_3d(sm + OFF_Q1, &tm_q, bar_ld, 64, y, zq);
-        tma_load_3d(sm + OFF_V0, &tm_v, bar_ld, 0, y, bh);
-        tma_load_3d(sm + OFF_V1, &tm_v, bar_ld, 64, y, bh);
-    };
-    auto mma_wait = [&]() {
-        bool w = mbar_wait(bar_mma, ph_mma);
-        ph_mma ^= 1u;
-        tc_fence_after();
-        return w;
-    };
-    if (tid == 0 && nvalid > 0) issue_loads(0);
+    if (carry) {
+        // ---- initial state into TMEM (fp32) and the bf16 operand tile ----
+        const __nv_bfloat16 *s0 = reinterpret_cast<const __nv_bfloat16 *>(a.initial_state);
+        const size_t off = ((size_t)bh * D + row) * D + 64 * hf;
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+            float v[32];
+#pragma unroll
+            for (int c8 = 0; c8 < 4; ++c8) {
+                float f[8];
+                if (s0) {
+                    unpack8(*reinterpret_cast<const uint4 *>(s0 + off + 32 * half + 8 * c8), f);
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) f[i] = 0.f;
+                }
+#pragma unroll
+                for (int i = 0; i < 8; ++i) v[8 * c8 + i] = f[i];
+                *reinterpret_cast<uint4 *>(sm + OFF_S + hf * 16384 + blk_off(row, 32 * half + 8 * c8)) =
+                    pack8(&v[8 * c8]);
+            }
+            tmem_st32(tmem + TM_S + lane_base + 64 * hf + 32 * half, v);
+        }
+        tmem_st_wait();
+        fence_proxy_async_smem();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
 
-    const float gA = (a.A_log && a.g) ? a.A_log[h] : 0.f, gB = (a.A_log && a.g) ? a.dt_bias[h] : 0.f;
-    const __nv_bfloat16 *bg = reinterpret_cast<const __nv_bfloat16 *>(a.beta) + (size_t)bh * S;
-    const float *gg = a.g ? a.g + (size_t)bh * S : nullptr;
-
-    for (int c = 0; c < nvalid; ++c) {
-        const int t0 = c * C, n = min(C, L - t0);
-        // ---- a1: per-token scalars ----
-        if (tid < C) {
-            float bt = 0.f, gt = 0.f;
-            if (tid < n) {
-                bt = __bfloat162float(bg[t0 + tid]);
-                if (a.beta_logits) bt = sigmoid_f32(bt);
-                if (gg) gt = a.A_log ? gate_from_raw(gg[t0 + tid], gA, gB) : gg[t0 + tid];
+#ifdef GDR_PHASE_TIMERS
+    unsigned long long t_prev_ = clock64();
+#endif
+    if (!carry) {
+        // =============================== prep group ===============================
+        const int p = tid - NGRP;
+        const float gA = (a.A_log && a.g) ? a.A_log[h] : 0.f, gB = (a.A_log && a.g) ? a.dt_bias[h] : 0.f;
+        const __nv_bfloat16 *bg = reinterpret_cast<const __nv_bfloat16 *>(a.beta) + (size_t)bh * S;
+        const float *gg = a.g ? a.g + (size_t)bh * S : nullptr;
+        float nb = 0.f, ng = 0.f;  // prefetched raw beta / gate of the next chunk (threads p < 64)
+        auto fetch = [&](int chunk) {
+            nb = 0.f;
+            ng = 0.f;
+            const int t = chunk * C + p;
+            if (p < C && chunk < nvalid && t < L) {
+                nb = __bfloat162float(bg[t]);
+                if (gg) ng = gg[t];
             }
-            sBeta[tid] = bt;
-            sGam[tid] = gt;
-        }
-        bool w = mbar_wait(bar_ld, ph_ld);
-        ph_ld ^= 1u;
-        if (!__syncthreads_and(w)) { ok = false; break; }
-        if (n < C) {  // padding rows of the last chunk: zero them so no padding value reaches a product
-            for (int e = tid; e < (C - n) * 48; e += NT) {
-                const int r = n + e / 48, k = e % 48, blk = k >> 3, ch = k & 7;
-                const uint32_t base = blk == 0 ? OFF_K0 : blk == 1 ? OFF_Q0 : blk == 2 ? OFF_K1 : blk == 3 ? OFF_Q1
-                                      : blk == 4 ? OFF_V0 : OFF_V1;
-                *reinterpret_cast<uint4 *>(sm + base + r * 128 + ch * 16) = make_uint4(0, 0, 0, 0);
+        };
+        auto issue_loads = [&](int chunk) {
+            const int y = chunk * C;
+            mbar_arrive_expect_tx(bar_ld, STAGE_BYTES);
+            tma_load_3d(sm + OFF_K0, &tm_k, bar_ld, 0, y, zq);
+            tma_load_3d(sm + OFF_K1, &tm_k, bar_ld, 64, y, zq);
+            tma_load_3d(sm + OFF_Q0, &tm_q, bar_ld, 0, y, zq);
+            tma_load_3d(sm + OFF_Q1, &tm_q, bar_ld, 64, y, zq);
+            tma_load_3d(sm + OFF_V0, &tm_v, bar_ld, 0, y, bh);
+            tma_load_3d(sm + OFF_V0 + 8192, &tm_v, bar_ld, 64, y, bh);
+        };
+        bool to = false;  // a wait of this thread timed out
+        auto wait_ok = [&](uint64_t *bar, uint32_t parity) {
+            if (!mbar_wait(bar, parity)) to = true;
+        };
+        if (p == 0 && nvalid > 0) issue_loads(0);
+        fetch(0);
+        for (int c = 0; c < nvalid; ++c) {
+            const uint32_t par = c & 1;
+            float *vec = vecs + (c & 1) * 8 * 64;
+            float *vBeta = vec + V_BETA * 64, *vGam = vec + V_GAM * 64, *vEG = vec + V_EG * 64;
+            float *vTail = vec + V_TAIL * 64, *vRk = vec + V_RK * 64, *vRq = vec + V_RQ * 64, *vCw = vec + V_CW * 64;
+            const int n = min(C, L - c * C);
+            if (p < C) {
+                const bool valid = p < n;
+                vBeta[p] = valid ? (a.beta_logits ? sigmoid_f32(nb) : nb) : 0.f;
+                vGam[p] = valid ? (a.A_log ? gate_from_raw(ng, gA, gB) : ng) : 0.f;
             }
-        }
-        if (warp == 0) {  // inclusive scan of the gate over the chunk
-            float x0 = sGam[2 * lane], x1 = sGam[2 * lane + 1];
-            x1 += x0;
-            float s = x1;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                float y = __shfl_up_sync(0xffffffffu, s, o);
-                if (lane >= o) s += y;
+            fetch(c + 1);
+            wait_ok(bar_ld, par);
+            if (named_sync_or(BAR_PREP, NGRP, to)) break;
+            PHASE(0);
+            if (n < C) {  // padding rows of the last chunk: zero them so no padding value reaches a product
+                for (int e = p; e < (C - n) * 48; e += NGRP) {
+                    const int r = n + e / 48, k = e % 48;
+                    *reinterpret_cast<uint4 *>(sm + (k >> 3) * 8192 + r * 128 + (k & 7) * 16) = make_uint4(0, 0, 0, 0);
+                }
+                fence_proxy_async_smem();
             }
-            const float excl = s - x1;
-            sGam[2 * lane] = excl + x0;
-            sGam[2 * lane + 1] = excl + x1;
-        }
-        if (tid >= 64 && tid < 192) {  // row norms of k (tid 64..127) and q (tid 128..191)
-            const int r = tid & 63;
-            const bool isq = tid >= 128;
-            float ss = 0.f;
-            if (r < n) {
+            named_sync(BAR_PREP, NGRP);
+            // ---- a2: [G; P] = [K; Q] K^T, issued first; the scalar work below overlaps it ----
+            if (p == 0) {
+                tc_fence_after();
+                const uint32_t id = idesc_bf16(128, 64, false, false);
 #pragma unroll
-                for (int blk = 0; blk < 2; ++blk) {
-                    const uint8_t *rowp = sm + (isq ? (blk ? OFF_Q1 : OFF_Q0) : (blk ? OFF_K1 : OFF_K0)) + r * 128;
+                for (int k = 0; k < 8; ++k) {
+                    const uint32_t addr = sbase + OFF_K0 + (k >> 2) * 16384 + (k & 3) * 32;
+                    mma_bf16(tmem + TM_GPW, sdesc_sw128(addr, 16, 1024), sdesc_sw128(addr, 16, 1024), id, k > 0);
+                }
+                mma_commit(bar_gp);
+            }
+            PHASE(10);
+            if (p < 32) {  // inclusive scan of the gate over the chunk (warp 8)
+                float x0 = vGam[2 * p], x1 = vGam[2 * p + 1];
+                x1 += x0;
+                float s = x1;
 #pragma unroll
-                    for (int ch = 0; ch < 8; ++ch) {
-                        float f[8];
-                        unpack8(*reinterpret_cast<const uint4 *>(rowp + ch * 16), f);
+                for (int o = 1; o < 32; o <<= 1) {
+                    const float y = __shfl_up_sync(0xffffffffu, s, o);
+                    if (p >= o) s += y;
+                }
+                const float excl = s - x1;
+                vGam[2 * p] = excl + x0;
+                vGam[2 * p + 1] = excl + x1;
+            }
+            {  // row norms of k and q: 4 threads per row, 32 elements each
+                const int r = p >> 2, part = p & 3;
+                const uint32_t off = (part >> 1) * 16384 + r * 128 + (part & 1) * 64;
+                float sk = 0.f, sq = 0.f;
 #pragma unroll
-                        for (int i = 0; i < 8; ++i) ss = fmaf(f[i], f[i], ss);
+                for (int ch = 0; ch < 4; ++ch) {
+                    float fk[8], fq[8];
+                    unpack8(*reinterpret_cast<const uint4 *>(sm + OFF_K0 + off + ch * 16), fk);
+                    unpack8(*reinterpret_cast<const uint4 *>(sm + OFF_Q0 + off + ch * 16), fq);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        sk = fmaf(fk[i], fk[i], sk);
+                        sq = fmaf(fq[i], fq[i], sq);
                     }
                 }
-            }
-            const float rn = r < n ? (a.l2norm ? rsqrtf(ss + a.eps) : 1.f) : 0.f;
-            if (isq) sRq[r] = a.scale * rn;
-            else sRk[r] = rn;
-        }
-        __syncthreads();
-        if (tid < C) {
-            const float gl = sGam[C - 1], gt = sGam[tid];
-            sEG[tid] = __expf(gt);
-            sTail[tid] = __expf(gl - gt) * sRk[tid];
-            sCw[tid] = sBeta[tid] * __expf(gt) * sRk[tid];
-        }
-        fence_proxy_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        tc_fence_after();
-
-        // ---- a2: [G; P] = [K; Q] K^T ----
-        if (tid == 0) {
-            const uint32_t id = idesc_bf16(128, 64, false, false);
-#pragma unroll
-            for (int k = 0; k < 8; ++k) {
-                const uint32_t addr = sbase + OFF_K0 + (k >> 2) * 16384 + (k & 3) * 32;
-                mma_bf16(tmem + TM_GP, sdesc_sw128(addr, 16, 1024), sdesc_sw128(addr, 16, 1024), id, k > 0);
-            }
-            mma_commit(bar_mma);
-        }
-        if (!__syncthreads_and(mma_wait())) { ok = false; break; }
-        {
-            float v[32];
-            tmem_ld32(tmem + TM_GP + lane_base + 32 * hf, v);
-            tmem_ld_wait();
-            const int t = (q4 & 1) * 32 + lane;  // token (row of G or P)
-            const float gt = sGam[t];
-            if (q4 < 2) {  // A row t
-                const float rb = sBeta[t] * sRk[t];
-#pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    const int s = 32 * hf + j;
-                    sA[t * FP + s] = (s < t && t < n) ? rb * sRk[s] * v[j] * __expf(gt - sGam[s]) : 0.f;
+                sk += __shfl_xor_sync(0xffffffffu, sk, 1);
+                sq += __shfl_xor_sync(0xffffffffu, sq, 1);
+                sk += __shfl_xor_sync(0xffffffffu, sk, 2);
+                sq += __shfl_xor_sync(0xffffffffu, sq, 2);
+                if (part == 0) {
+                    vRk[r] = r < n ? (a.l2norm ? rsqrtf(sk + a.eps) : 1.f) : 0.f;
+                    vRq[r] = r < n ? a.scale * (a.l2norm ? rsqrtf(sq + a.eps) : 1.f) : 0.f;
                 }
-            } else {  // Pm row t -> rows 64 + t of the [0; Pm] operand
-                const float rq = sRq[t];
-                float pm[32];
+            }
+            named_sync(BAR_PREP, NGRP);
+            PHASE(11);
+            {  // decay matrix E[t][s] = e^{G_t - G_s} for s <= t, 16 entries per thread
+                const int t = p >> 2, s0 = (p & 3) * 16;
+                const float gt = vGam[t];
+                float e[16];
 #pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    const int s = 32 * hf + j;
-                    pm[j] = (s <= t && t < n) ? rq * sRk[s] * v[j] * __expf(gt - sGam[s]) : 0.f;
+                for (int i = 0; i < 16; ++i) e[i] = (s0 + i <= t) ? __expf(gt - vGam[s0 + i]) : 0.f;
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    *reinterpret_cast<float4 *>(sE + t * FP + s0 + 4 * i) =
+                        make_float4(e[4 * i], e[4 * i + 1], e[4 * i + 2], e[4 * i + 3]);
+            }
+            if (p < C) {
+                const float gl = vGam[C - 1], gt = vGam[p];
+                vEG[p] = __expf(gt);
+                vTail[p] = __expf(gl - gt) * vRk[p];
+                vCw[p] = vBeta[p] * __expf(gt) * vRk[p];
+                if (p == 0) vec[V_N * 64] = (float)n;
+            }
+            named_sync(BAR_PREP, NGRP);
+            PHASE(1);
+            wait_ok(bar_gp, par);
+            tc_fence_after();
+            PHASE(2);
+            {  // A rows (from G, lanes 0..63) and Pm rows (from P, lanes 64..127; parked in TMEM as fp32)
+                float v[32];
+                const uint32_t ta = tmem + TM_GPW + lane_base + 32 * hf;
+                tmem_ld32(ta, v);
+                tmem_ld_wait();
+                PHASE(12);
+                const int t = row & 63;
+                const float *et = sE + t * FP + 32 * hf;
+                if (q4 < 2) {
+                    const float rb = t < n ? vBeta[t] * vRk[t] : 0.f;
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        const int s = 32 * hf + j;
+                        sA[t * FA + s] = s < t ? rb * vRk[s] * v[j] * et[j] : 0.f;
+                    }
+                } else {
+                    const float rq = t < n ? vRq[t] : 0.f;
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) v[j] = rq * vRk[32 * hf + j] * v[j] * et[j];
+                    tmem_st32(ta, v);
+                    tmem_st_wait();
                 }
+            }
+            tc_fence_before();
+            if (named_sync_or(BAR_PREP, NGRP, to)) break;
+            PHASE(3);
+            // ---- a3: T = (I + A)^{-1} and the bf16 operand [T diag(beta); T diag(c_W)] ----
+            solve_unit_lower(sA, sT, sX, p);
+            PHASE(4);
+            for (int e = p; e < 128 * 8; e += NGRP) {
+                const int R = e >> 3, j = e & 7, t = R & 63;
+                const float *scl = (R < 64 ? vBeta : vCw) + 8 * j;
+                const float4 t0 = *reinterpret_cast<const float4 *>(sT + t * FP + 8 * j);
+                const float4 t1 = *reinterpret_cast<const float4 *>(sT + t * FP + 8 * j + 4);
+                const float tv[8] = {t0.x, t0.y, t0.z, t0.w, t1.x, t1.y, t1.z, t1.w};
+                float f[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) f[i] = (8 * j + i <= t) ? tv[i] * scl[i] : 0.f;
+                *reinterpret_cast<uint4 *>(sm + OFF_TT + blk_off(R, 8 * j)) = pack8(f);
+            }
+            PHASE(5);
+            // the carry group must be done with chunk c-1's MMAs before PM, K~, A1, U are rewritten
+            if (c > 0 && !mbar_wait_sleep(bar_m2, (c - 1) & 1)) to = true;
+            tc_fence_after();
+            PHASE(6);
+            if (q4 >= 2) {  // Pm rows (TMEM, fp32) -> rows 64 + t of the bf16 [0; Pm] operand
+                float v[32];
+                tmem_ld32(tmem + TM_GPW + lane_base + 32 * hf, v);
+                tmem_ld_wait();
+                const int t = row - 64;
+#pragma unroll
+                for (int j = 0; j < 32; ++j) v[j] = (32 * hf + j <= t) ? v[j] : 0.f;
 #pragma unroll
                 for (int c8 = 0; c8 < 4; ++c8)
-                    *reinterpret_cast<uint4 *>(sm + OFF_PM + blk_off(64 + t, 32 * hf + 8 * c8)) = pack8(&pm[8 * c8]);
+                    *reinterpret_cast<uint4 *>(sm + OFF_PM + blk_off(64 + t, 32 * hf + 8 * c8)) = pack8(&v[8 * c8]);
             }
-        }
-        tc_fence_before();
-        __syncthreads();
-        // ---- a3: T = (I + A)^{-1}, then [T diag(beta); T diag(c_W)] as a bf16 operand ----
-        solve_unit_lower(sA, sT, sX, tid);
-        for (int e = tid; e < 128 * 8; e += NT) {
-            const int R = e >> 3, j = e & 7, t = R & 63;
-            const float *scl = R < 64 ? sBeta : sCw;
-            float f[8];
+            fence_proxy_async_smem();
+            tc_fence_before();
+            if (named_sync_or(BAR_PREP, NGRP, to)) break;
+            tc_fence_after();
+            PHASE(7);
+            // ---- a4: W (rows 64..127 of TT K) and U (rows 0..63 of TT V) ----
+            if (p == 0) {
+                const uint32_t id = idesc_bf16(128, 128, false, true);
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const int s = 8 * j + i;
-                f[i] = s <= t ? sT[t * FP + s] * scl[s] : 0.f;
+                for (int k = 0; k < 4; ++k) {
+                    const uint64_t ad = sdesc_sw128(sbase + OFF_TT + k * 32, 16, 1024);
+                    mma_bf16(tmem + TM_GPW, ad, sdesc_sw128(sbase + OFF_K0 + k * 2048, 16384, 1024), id, k > 0);
+                    mma_bf16(tmem + TM_U, ad, sdesc_sw128(sbase + OFF_V0 + k * 2048, 8192, 1024), id, k > 0);
+                }
+                mma_commit(bar_wu);
             }
-            *reinterpret_cast<uint4 *>(sm + OFF_TT + blk_off(R, 8 * j)) = pack8(f);
-        }
-        fence_proxy_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        tc_fence_after();
-        // ---- a4: W (rows 64..127 of T'K) and U (rows 0..63 of T'V) ----
-        if (tid == 0) {
-            const uint32_t id = idesc_bf16(128, 128, false, true);
+            // meanwhile: X_g rows (64..127 of A1) and K~ from the staged q/k tiles
+            for (int e = p; e < 2 * 64 * 16; e += NGRP) {
+                const int isk = e >> 10, r = (e >> 4) & 63, blk = (e >> 3) & 1, ch = e & 7;
+                const uint32_t rb = (r >> 3) * 1024u + (r & 7) * 128u + ch * 16u;  // same swizzle phase (row % 8)
+                float f[8];
+                if (isk) {
+                    unpack8(*reinterpret_cast<const uint4 *>(sm + OFF_K0 + blk * 16384 + rb), f);
+                    const float sc = vTail[r];
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const uint64_t ad = sdesc_sw128(sbase + OFF_TT + k * 32, 16, 1024);
-                mma_bf16(tmem + TM_WD, ad, sdesc_sw128(sbase + OFF_K0 + k * 2048, 16384, 1024), id, k > 0);
-                mma_bf16(tmem + TM_U, ad, sdesc_sw128(sbase + OFF_V0 + k * 2048, 8192, 1024), id, k > 0);
+                    for (int i = 0; i < 8; ++i) f[i] *= sc;
+                    *reinterpret_cast<uint4 *>(sm + OFF_KT + blk * 8192 + rb) = pack8(f);
+                } else {
+                    unpack8(*reinterpret_cast<const uint4 *>(sm + OFF_Q0 + blk * 16384 + rb), f);
+                    const float sc = vEG[r] * vRq[r];
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) f[i] *= sc;
+                    *reinterpret_cast<uint4 *>(sm + OFF_A1 + blk * 16384 + 8192 + rb) = pack8(f);
+                }
             }
-            mma_commit(bar_mma);
-        }
-        // meanwhile: X_g rows (64..127 of A1) and K~ from the staged q/k tiles
-        for (int e = tid; e < 2 * 64 * 16; e += NT) {
-            const int isk = e >> 10, r = (e >> 4) & 63, blk = (e >> 3) & 1, ch = e & 7;
-            const uint32_t rb = (r >> 3) * 1024u + (r & 7) * 128u + ch * 16u;  // same swizzle phase (row % 8)
-            float f[8];
-            if (isk) {
-                unpack8(*reinterpret_cast<const uint4 *>(sm + (blk ? OFF_K1 : OFF_K0) + rb), f);
-                const float sc = r < n ? sTail[r] : 0.f;
+            wait_ok(bar_wu, par);
+            tc_fence_after();
+            if (named_sync_or(BAR_PREP, NGRP, to)) break;  // staged tiles fully consumed
+            PHASE(8);
+            if (p == 0 && c + 1 < nvalid) issue_loads(c + 1);
+            if (q4 >= 2) {  // W rows -> rows 0..63 of A1
+                const int t = row - 64;
 #pragma unroll
-                for (int i = 0; i < 8; ++i) f[i] *= sc;
-                *reinterpret_cast<uint4 *>(sm + OFF_KT + blk * 8192 + rb) = pack8(f);
-            } else {
-                unpack8(*reinterpret_cast<const uint4 *>(sm + (blk ? OFF_Q1 : OFF_Q0) + rb), f);
-                const float sc = r < n ? sEG[r] * sRq[r] : 0.f;
+                for (int half = 0; half < 2; ++half) {
+                    float v[32];
+                    tmem_ld32(tmem + TM_GPW + lane_base + 64 * hf + 32 * half, v);
+                    tmem_ld_wait();
 #pragma unroll
-                for (int i = 0; i < 8; ++i) f[i] *= sc;
-                *reinterpret_cast<uint4 *>(sm + OFF_A1 + blk * 16384 + 8192 + rb) = pack8(f);
+                    for (int c8 = 0; c8 < 4; ++c8)
+                        *reinterpret_cast<uint4 *>(sm + OFF_A1 + hf * 16384 + blk_off(t, 32 * half + 8 * c8)) =
+                            pack8(&v[8 * c8]);
+                }
             }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            named_sync(BAR_PREP, NGRP);
+            if (p == 0) mbar_arrive(bar_a1);
+            PHASE(9);
         }
-        fence_proxy_async_smem();
-        if (!__syncthreads_and(mma_wait())) { ok = false; break; }
-        if (q4 >= 2) {  // W rows -> rows 0..63 of A1
-            const int t = (q4 - 2) * 32 + lane;
+        if (to && p == 0) *s_abort = 1;
+    } else {
+        // =============================== carry group ==============================
+        bool to = false;  // a wait of this thread timed out
+        bool stop = false;
+        auto wait_ok = [&](uint64_t *bar, uint32_t parity) {
+            if (!mbar_wait(bar, parity)) to = true;
+        };
+        for (int c = 0; c < nvalid; ++c) {
+            const uint32_t par = c & 1;
+            const float *vec = vecs + (c & 1) * 8 * 64;
+            if (!mbar_wait_sleep(bar_a1, par)) to = true;
+            if (named_sync_or(BAR_CARRY, NGRP, to)) { stop = true; break; }
+            tc_fence_after();
+            PHASE(16);
+            const int n = (int)vec[V_N * 64];
+            const float eL = vec[V_EG * 64 + C - 1];
+            // ---- R = [W; X_g] S ----
+            if (tid == 0) {
+                const uint32_t id = idesc_bf16(128, 128, false, true);
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    const uint64_t ad = sdesc_sw128(sbase + OFF_A1 + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024);
+                    const uint64_t bd = sdesc_sw128(sbase + OFF_S + k * 2048, 16384, 1024);
+                    mma_bf16(tmem + TM_R, ad, bd, id, k > 0);
+                }
+                mma_commit(bar_m1);
+            }
+            // meanwhile: S <- e^{G_last} S in TMEM (MMA2 accumulates onto it)
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
                 float v[32];
-                tmem_ld32(tmem + TM_WD + lane_base + 64 * hf + 32 * half, v);
+                const uint32_t ta = tmem + TM_S + lane_base + 64 * hf + 32 * half;
+                tmem_ld32(ta, v);
+                tmem_ld_wait();
+#pragma unroll
+                for (int j = 0; j < 32; ++j) v[j] *= eL;
+                tmem_st32(ta, v);
+            }
+            tmem_st_wait();
+            wait_ok(bar_m1, par);
+            if (tid == 0) bulk_wait_read0();  // the previous out tile (same buffer as v_new) is read
+            tc_fence_before();
+            if (named_sync_or(BAR_CARRY, NGRP, to)) { stop = true; break; }
+            tc_fence_after();
+            PHASE(17);
+            if (q4 < 2) {  // v_new = U - W S for token t, dv columns [64 hf, +64)
+                const int t = row;
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
+                    float u[32], r[32];
+                    tmem_ld32(tmem + TM_U + lane_base + 64 * hf + 32 * half, u);
+                    tmem_ld32(tmem + TM_R + lane_base + 64 * hf + 32 * half, r);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) u[j] = t < n ? u[j] - r[j] : 0.f;
+#pragma unroll
+                    for (int c8 = 0; c8 < 4; ++c8)
+                        *reinterpret_cast<uint4 *>(sm + OFF_VO + hf * 8192 + blk_off(t, 32 * half + 8 * c8)) =
+                            pack8(&u[8 * c8]);
+                }
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            named_sync(BAR_CARRY, NGRP);
+            tc_fence_after();
+            PHASE(18);
+            // ---- S += K~^T v_new ;  R[64:128] += Pm v_new ----
+            if (tid == 0) {
+                const uint32_t id_s = idesc_bf16(128, 128, true, true);
+                const uint32_t id_o = idesc_bf16(128, 128, false, true);
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const uint64_t bd = sdesc_sw128(sbase + OFF_VO + k * 2048, 8192, 1024);
+                    mma_bf16(tmem + TM_S, sdesc_sw128(sbase + OFF_KT + k * 2048, 8192, 1024), bd, id_s, 1);
+                }
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const uint64_t bd = sdesc_sw128(sbase + OFF_VO + k * 2048, 8192, 1024);
+                    mma_bf16(tmem + TM_R, sdesc_sw128(sbase + OFF_PM + k * 32, 16, 1024), bd, id_o, 1);
+                }
+                mma_commit(bar_m2);
+            }
+            wait_ok(bar_m2, par);
+            tc_fence_after();
+            if (named_sync_or(BAR_CARRY, NGRP, to)) { stop = true; break; }
+            PHASE(19);
+            // ---- S (fp32, TMEM) -> bf16 operand tile;  o rows -> out tile ----
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                float v[32];
+                tmem_ld32(tmem + TM_S + lane_base + 64 * hf + 32 * half, v);
                 tmem_ld_wait();
 #pragma unroll
                 for (int c8 = 0; c8 < 4; ++c8)
-                    *reinterpret_cast<uint4 *>(sm + OFF_A1 + hf * 16384 + blk_off(t, 32 * half + 8 * c8)) =
+                    *reinterpret_cast<uint4 *>(sm + OFF_S + hf * 16384 + blk_off(row, 32 * half + 8 * c8)) =
                         pack8(&v[8 * c8]);
             }
-        }
-        fence_proxy_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        tc_fence_after();
-        // ---- a5: R = [W; X_g] S; the staged tiles are free: prefetch the next chunk ----
-        if (tid == 0) {
-            if (c + 1 < nvalid) issue_loads(c + 1);
-            const uint32_t id = idesc_bf16(128, 128, false, true);
-#pragma unroll
-            for (int k = 0; k < 8; ++k) {
-                const uint64_t ad = sdesc_sw128(sbase + OFF_A1 + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024);
-                const uint64_t bd = sdesc_sw128(sbase + OFF_S + k * 2048, 16384, 1024);
-                mma_bf16(tmem + TM_R, ad, bd, id, k > 0);
-            }
-            mma_commit(bar_mma);
-        }
-        if (!__syncthreads_and(mma_wait())) { ok = false; break; }
-        if (q4 < 2) {  // v_new = U - W S for token t, dv columns [64 hf, +64)
-            const int t = q4 * 32 + lane;
-#pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                float u[32], r[32];
-                tmem_ld32(tmem + TM_U + lane_base + 64 * hf + 32 * half, u);
-                tmem_ld32(tmem + TM_R + lane_base + 64 * hf + 32 * half, r);
-                tmem_ld_wait();
-#pragma unroll
-                for (int j = 0; j < 32; ++j) u[j] = t < n ? u[j] - r[j] : 0.f;
-#pragma unroll
-                for (int c8 = 0; c8 < 4; ++c8)
-                    *reinterpret_cast<uint4 *>(sm + OFF_VN + hf * 8192 + blk_off(t, 32 * half + 8 * c8)) =
-                        pack8(&u[8 * c8]);
-            }
-        }
-        if (tid == 0) bulk_wait_read0();  // the previous out tile has been read by its store
-        fence_proxy_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        tc_fence_after();
-        // ---- dS = K~^T v_new ;  R[64:128] += Pm v_new ----
-        if (tid == 0) {
-            const uint32_t id_s = idesc_bf16(128, 128, true, true);
-            const uint32_t id_o = idesc_bf16(128, 128, false, true);
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const uint64_t bd = sdesc_sw128(sbase + OFF_VN + k * 2048, 8192, 1024);
-                mma_bf16(tmem + TM_WD, sdesc_sw128(sbase + OFF_KT + k * 2048, 8192, 1024), bd, id_s, k > 0);
-            }
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const uint64_t bd = sdesc_sw128(sbase + OFF_VN + k * 2048, 8192, 1024);
-                mma_bf16(tmem + TM_R, sdesc_sw128(sbase + OFF_PM + k * 32, 16, 1024), bd, id_o, 1);
-            }
-            mma_commit(bar_mma);
-        }
-        if (!__syncthreads_and(mma_wait())) { ok = false; break; }
-        {
-            const float eL = sEG[C - 1];
-#pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                float d[32];
-                tmem_ld32(tmem + TM_WD + lane_base + 64 * hf + 32 * half, d);
-                tmem_ld_wait();
-#pragma unroll
-                for (int j = 0; j < 32; ++j) st[32 * half + j] = fmaf(eL, st[32 * half + j], d[j]);
-#pragma unroll
-                for (int c8 = 0; c8 < 4; ++c8)
-                    *reinterpret_cast<uint4 *>(sm + OFF_S + hf * 16384 + blk_off(srow, 32 * half + 8 * c8)) =
-                        pack8(&st[32 * half + 8 * c8]);
-            }
-            if (q4 >= 2) {  // o rows -> out tile
-                const int t = (q4 - 2) * 32 + lane;
+            if (q4 >= 2) {
+                const int t = row - 64;
 #pragma unroll
                 for (int half = 0; half < 2; ++half) {
                     float o[32];
@@ -492,48 +639,58 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     for (int j = 0; j < 32; ++j) o[j] = t < n ? o[j] : 0.f;
 #pragma unroll
                     for (int c8 = 0; c8 < 4; ++c8)
-                        *reinterpret_cast<uint4 *>(sm + OFF_O + hf * 8192 + blk_off(t, 32 * half + 8 * c8)) =
+                        *reinterpret_cast<uint4 *>(sm + OFF_VO + hf * 8192 + blk_off(t, 32 * half + 8 * c8)) =
                             pack8(&o[8 * c8]);
                 }
             }
-        }
-        fence_proxy_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        tc_fence_after();
-        if (tid == 0) {
-            tma_store_3d(&tm_o, sm + OFF_O, 0, t0, bh);
-            tma_store_3d(&tm_o, sm + OFF_O + 8192, 64, t0, bh);
-            bulk_commit();
-        }
-    }
-    if (!ok) {
-        if (tid == 0) raise_device_error(a.err, kTimeoutBit);
-    } else {
-        // chunks past the length: zero rows
-        if (nvalid < ntotal) {
-            if (tid == 0) bulk_wait_read0();
-            __syncthreads();
-            for (int e = tid; e < 16384 / 16; e += NT) reinterpret_cast<uint4 *>(sm + OFF_O)[e] = make_uint4(0, 0, 0, 0);
             fence_proxy_async_smem();
-            __syncthreads();
+            tc_fence_before();
+            named_sync(BAR_CARRY, NGRP);
+            tc_fence_after();
             if (tid == 0) {
-                for (int c = nvalid; c < ntotal; ++c) {
-                    tma_store_3d(&tm_o, sm + OFF_O, 0, c * C, bh);
-                    tma_store_3d(&tm_o, sm + OFF_O + 8192, 64, c * C, bh);
-                }
+                tma_store_3d(&tm_o, sm + OFF_VO, 0, c * C, bh);
+                tma_store_3d(&tm_o, sm + OFF_VO + 8192, 64, c * C, bh);
                 bulk_commit();
             }
+            PHASE(20);
         }
-        if (a.final_state) {
-            __nv_bfloat16 *fs = reinterpret_cast<__nv_bfloat16 *>(a.final_state) + ((size_t)bh * D + srow) * D + 64 * hf;
+        if (stop && tid == 0) *s_abort = 1;
+        if (!stop) {
+            // chunks past the length: zero rows
+            if (nvalid < ntotal) {
+                if (tid == 0) bulk_wait_read0();
+                named_sync(BAR_CARRY, NGRP);
+                for (int e = tid; e < 16384 / 16; e += NGRP)
+                    reinterpret_cast<uint4 *>(sm + OFF_VO)[e] = make_uint4(0, 0, 0, 0);
+                fence_proxy_async_smem();
+                named_sync(BAR_CARRY, NGRP);
+                if (tid == 0) {
+                    for (int c = nvalid; c < ntotal; ++c) {
+                        tma_store_3d(&tm_o, sm + OFF_VO, 0, c * C, bh);
+                        tma_store_3d(&tm_o, sm + OFF_VO + 8192, 64, c * C, bh);
+                    }
+                    bulk_commit();
+                }
+            }
+            if (a.final_state) {
+                __nv_bfloat16 *fs =
+                    reinterpret_cast<__nv_bfloat16 *>(a.final_state) + ((size_t)bh * D + row) * D + 64 * hf;
 #pragma unroll
-            for (int c8 = 0; c8 < 8; ++c8) *reinterpret_cast<uint4 *>(fs + 8 * c8) = pack8(&st[8 * c8]);
+                for (int half = 0; half < 2; ++half) {
+                    float v[32];
+                    tmem_ld32(tmem + TM_S + lane_base + 64 * hf + 32 * half, v);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int c8 = 0; c8 < 4; ++c8)
+                        *reinterpret_cast<uint4 *>(fs + 32 * half + 8 * c8) = pack8(&v[8 * c8]);
+                }
+            }
         }
+        if (tid == 0) bulk_wait0();
     }
-    if (tid == 0) bulk_wait0();
     tc_fence_before();
     __syncthreads();
+    if (tid == 0 && *s_abort) raise_device_error(a.err, kTimeoutBit);
     if (warp == 0) tmem_dealloc(tmem, TM_COLS);
 }
 
@@ -569,6 +726,16 @@ bool make_map(CUtensorMap *m, const void *base, int S, long long Z) {
 }
 
 }  // namespace
+
+#ifdef GDR_PHASE_TIMERS
+extern "C" int gdr_phase_timers_read(unsigned long long *out) {
+    cudaDeviceSynchronize();
+    cudaMemcpyFromSymbol(out, g_phase, sizeof(unsigned long long) * 64);
+    unsigned long long z[64] = {0};
+    cudaMemcpyToSymbol(g_phase, z, sizeof(z));
+    return 0;
+}
+#endif
 
 bool chunk_tc_supported(int Dk, int Dv, gdr_dtype dt, int S) { return dt == GDR_BF16 && Dk == D && Dv == D && S > 0; }
 
