@@ -24,7 +24,6 @@ from __future__ import annotations
 
 import argparse
 import json
-import math
 import os
 import statistics
 import sys
@@ -89,8 +88,6 @@ def profiled_traffic(kernel: str):
     p = os.path.join(ROOT, "profiles", "dram_traffic.txt")
     if not os.path.exists(p):
         return None
-    srcs = {"chunk": ["gated_deltanet_gdr_b200/csrc/chunk_tc.cu", "gated_deltanet_gdr_b200/csrc/chunk_simt.cu"],
-            "decode": ["gated_deltanet_gdr_b200/csrc/decode.cu"]}
     for line in open(p):
         parts = line.split()
         if len(parts) >= 4 and parts[0] == kernel and not line.startswith("#"):
@@ -256,32 +253,25 @@ def f32_dev(x):
     return torch.from_numpy(np.ascontiguousarray(np.asarray(x, np.float32))).cuda()
 
 
-def run_ours(args, world, rank, local):
-    import gated_deltanet_gdr_b200 as gdr
-    gdr.lib()  # fails loudly if the library is missing
-    peaks = measured_peaks()
-    stream = torch.cuda.current_stream()
-    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda")
-
-    # ---------------- prefill (the headline) ----------------
+def bench_prefill(gdr, args, world, rank, clk, flush, stream, peaks):
+    """The headline: prefill with the fused prologue; returns (line fields, workload, tensors)."""
     w = workloads.generate("prefill", seed=2 + 1000 * rank)
-    q, k, v, b = bf16_dev(w.q), bf16_dev(w.k), bf16_dev(w.v), bf16_dev(w.b)
-    a = f32_dev(w.a)
-    s0 = bf16_dev(w.initial_state)
-    pro = gdr.Prologue(l2norm_qk=True, eps=1e-6, beta_logits=True, A_log=f32_dev(w.A_log), dt_bias=f32_dev(w.dt_bias))
-    out = torch.empty((w.B, w.Nv, w.S, w.Dv), dtype=torch.bfloat16, device="cuda")
-    fin = torch.empty_like(s0)
+    t = dict(q=bf16_dev(w.q), k=bf16_dev(w.k), v=bf16_dev(w.v), b=bf16_dev(w.b), a=f32_dev(w.a),
+             s0=bf16_dev(w.initial_state))
+    pro = gdr.Prologue(l2norm_qk=True, eps=1e-6, beta_logits=True, A_log=f32_dev(w.A_log),
+                       dt_bias=f32_dev(w.dt_bias))
+    t["out"] = torch.empty((w.B, w.Nv, w.S, w.Dv), dtype=torch.bfloat16, device="cuda")
+    t["fin"] = torch.empty_like(t["s0"])
 
-    def step():
-        gdr.chunk_fwd(q, k, v, b, a, s0, None, w.scale, prologue=pro, out=out, final_state=fin)
+    # argument checks and marshalling happen once; each step is one C-ABI call
+    step = gdr.prepare_chunk_fwd(t["q"], t["k"], t["v"], t["b"], t["a"], t["s0"], None, w.scale, prologue=pro,
+                                 out=t["out"], final_state=t["fin"])
 
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
     if gdr.get_error() != 0:
         raise RuntimeError("device error word set during warm-up")
-
-    clk = ClockSampler(local).__enter__()
     barrier(world)
     torch.cuda.synchronize()
     clk.active = True
@@ -291,96 +281,135 @@ def run_ours(args, world, rank, local):
     total_ms = all_max(sum(times), world)
     ms_per_step = total_ms / args.steps
     tokens = int(w.lengths.sum())
-    value = world * tokens * args.steps / (total_ms / 1e3)
     alg_bytes = algorithmic_prefill_bytes(w)
     achieved = alg_bytes / (ms_per_step / 1e3) / 1e9
-    traffic = profiled_traffic("chunk")
-    roofline = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": achieved / peaks["hbm_gbs"], "traffic": traffic,
-                "peak_source": peaks["source"], "algorithmic_bytes_per_launch": alg_bytes,
-                "kernel": "gdr_chunk_fwd (fused prologue)"}
+    fields = {
+        "value": world * tokens * args.steps / (total_ms / 1e3), "ms_per_step": ms_per_step,
+        "config": {"workload": f"prefill B={w.B} S={w.S} Nk={w.Nk} Nv={w.Nv} Dk=Dv={w.Dk} bf16, fused prologue, "
+                               "equal lengths", "global_batch": w.B * world, "seq_len": w.S,
+                   "parallelism": f"dp{world} (independent batches per GPU)",
+                   "l2": "inputs larger than L2, plus a 256 MiB flush before every timed step"},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": achieved / peaks["hbm_gbs"], "traffic": profiled_traffic("chunk"),
+                     "peak_source": peaks["source"], "algorithmic_bytes_per_launch": alg_bytes,
+                     "kernel": "gdr_chunk_fwd (fused prologue)"},
+        "gpu_launches": args.steps,
+    }
+    return fields, w, t, pro, step
 
-    # ---------------- e2e through the public call with host buffers ----------------
-    hq, hk, hv, hb = (t.cpu().pin_memory() for t in (q, k, v, b))
-    ha, hs0 = a.cpu().pin_memory(), s0.cpu().pin_memory()
-    hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-    hfin = torch.empty(fin.shape, dtype=fin.dtype).pin_memory()
-    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hb, ha, hs0))
+
+def bench_e2e(gdr, args, world, w, t, pro, flush, stream):
+    """Same metric through the public call with host buffers: pinned H2D copies of the
+    step's inputs, the call, D2H of out and the final state, all inside the timed region."""
+    names = ("q", "k", "v", "b", "a", "s0")
+    host = {n: t[n].cpu().pin_memory() for n in names}
+    hout = torch.empty(t["out"].shape, dtype=t["out"].dtype).pin_memory()
+    hfin = torch.empty(t["fin"].shape, dtype=t["fin"].dtype).pin_memory()
+    h2d = sum(x.numel() * x.element_size() for x in host.values())
     d2h = hout.numel() * hout.element_size() + hfin.numel() * hfin.element_size()
 
-    def e2e_step():
-        for d, h in ((q, hq), (k, hk), (v, hv), (b, hb), (a, ha), (s0, hs0)):
-            d.copy_(h, non_blocking=True)
-        gdr.chunk_fwd(q, k, v, b, a, s0, None, w.scale, prologue=pro, out=out, final_state=fin)
-        hout.copy_(out, non_blocking=True)
-        hfin.copy_(fin, non_blocking=True)
+    call = gdr.prepare_chunk_fwd(t["q"], t["k"], t["v"], t["b"], t["a"], t["s0"], None, w.scale, prologue=pro,
+                                 out=t["out"], final_state=t["fin"])
 
-    e2e_steps = max(3, min(args.steps, 10))
+    def e2e_step():
+        for n in names:
+            t[n].copy_(host[n], non_blocking=True)
+        call()
+        hout.copy_(t["out"], non_blocking=True)
+        hfin.copy_(t["fin"], non_blocking=True)
+
+    steps = max(3, min(args.steps, 10))
     for _ in range(2):
         e2e_step()
     barrier(world)
     torch.cuda.synchronize()
-    e2e_times = timed_steps(e2e_step, e2e_steps, flush, stream)
+    times = timed_steps(e2e_step, steps, flush, stream)
     barrier(world)
-    e2e_ms = all_max(sum(e2e_times), world) / e2e_steps
-    e2e = {"value": world * tokens / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
-           "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
-    del hq, hk, hv, hb, ha, hs0, hout, hfin
+    ms = all_max(sum(times), world) / steps
+    tokens = int(w.lengths.sum())
+    return {"value": world * tokens / (ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "ms_per_step": ms, "steps": steps}, steps
 
-    # ---------------- decode row ----------------
+
+def bench_decode(gdr, name, args, world, rank, clk, flush, stream, peaks, rotate: int = 4):
+    """One decode call per step.  The state a call touches (67 MB for the decode workload)
+    fits in L2, so instead of a flush the steps rotate over `rotate` separate copies of the
+    pool: each call reads fresh state and pays the write-back of the previous call's state,
+    as a serving loop does."""
+    wd = workloads.generate(name, seed=(1 if name == "decode" else 4) + 1000 * rank)
+    dq, dk, dv, db = bf16_dev(wd.q), bf16_dev(wd.k), bf16_dev(wd.v), bf16_dev(wd.b)
+    dg = f32_dev(wd.g)
+    dgk = f32_dev(wd.gk) if wd.gk is not None else None
+    pools = [bf16_dev(wd.pool) for _ in range(rotate)]
+    idx = torch.from_numpy(wd.indices).cuda()
+    lens = torch.from_numpy(wd.lengths).cuda()
+    acc = torch.from_numpy(wd.accepted).cuda()
+    dout = torch.empty((wd.B, wd.Nv, wd.S, wd.Dv), dtype=torch.bfloat16, device="cuda")
+    dpro = gdr.Prologue(l2norm_qk=True, eps=1e-6, beta_logits=True)
+    calls = [gdr.prepare_recurrent_step(dq, dk, dv, db, dg, dgk, pool, idx, lens, acc, wd.scale, prologue=dpro,
+                                        out=dout) for pool in pools]
+    for i in range(args.warmup):
+        calls[i % rotate]()
+    barrier(world)
+    torch.cuda.synchronize()
+    evs = []
+    clk.active = True
+    with torch.cuda.stream(stream):
+        for i in range(args.steps):
+            s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            s.record(stream)
+            calls[i % rotate]()
+            e.record(stream)
+            evs.append((s, e))
+    torch.cuda.synchronize()
+    clk.active = False
+    barrier(world)
+    times = [s.elapsed_time(e) for s, e in evs]
+    d_ms = all_max(sum(times), world) / args.steps
+    nb = algorithmic_decode_bytes(wd)
+    gbs = nb["state"] / (d_ms / 1e3) / 1e9
+    tot = (nb["state"] + nb["io"]) / (d_ms / 1e3) / 1e9
+    return {"workload": f"B={wd.B} S={wd.S} Nk={wd.Nk} Nv={wd.Nv} D={wd.Dk} bf16, pool of {wd.pool.shape[0]} slots"
+                        + (", per-key gate" if wd.gk is not None else "") + ", fused prologue",
+            "l2": f"{rotate} rotating pool copies (fresh state every call), no flush",
+            "us_per_call": d_ms * 1e3, "steps_per_s": world * 1e3 / d_ms,
+            "state_GBps": gbs, "state_frac_of_hbm": gbs / peaks["hbm_gbs"],
+            "roofline": {"bound": "hbm", "achieved": tot, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": tot / peaks["hbm_gbs"], "traffic": profiled_traffic("decode"),
+                         "algorithmic_bytes_per_launch": nb["state"] + nb["io"]}}, args.steps
+
+
+def run_ours(args, world, rank, local):
+    import gated_deltanet_gdr_b200 as gdr
+    gdr.lib()  # fails loudly if the library is missing
+    peaks = measured_peaks()
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    clk = ClockSampler(local).__enter__()
+    line = {"metric": METRIC, "value": None, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": None, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic"}
+    launches = 0
+    if args.only in ("all", "prefill"):
+        fields, w, t, pro, _ = bench_prefill(gdr, args, world, rank, clk, flush, stream, peaks)
+        line.update(fields)
+        launches += fields.pop("gpu_launches")
+        if not args.no_e2e:
+            line["e2e"], n = bench_e2e(gdr, args, world, w, t, pro, flush, stream)
+        del t
     decode = {}
-    launches = args.steps
     for name in ("decode", "decode_gk"):
-        wd = workloads.generate(name, seed=(1 if name == "decode" else 4) + 1000 * rank)
-        dq, dk, dv, db = bf16_dev(wd.q), bf16_dev(wd.k), bf16_dev(wd.v), bf16_dev(wd.b)
-        dg = f32_dev(wd.g)
-        dgk = f32_dev(wd.gk) if wd.gk is not None else None
-        pool = bf16_dev(wd.pool)
-        idx = torch.from_numpy(wd.indices).cuda()
-        lens = torch.from_numpy(wd.lengths).cuda()
-        acc = torch.from_numpy(wd.accepted).cuda()
-        dout = torch.empty((wd.B, wd.Nv, wd.S, wd.Dv), dtype=torch.bfloat16, device="cuda")
-        dpro = gdr.Prologue(l2norm_qk=True, eps=1e-6, beta_logits=True)
-
-        def dstep():
-            gdr.recurrent_step(dq, dk, dv, db, dg, dgk, pool, idx, lens, acc, wd.scale, prologue=dpro, out=dout)
-
-        for _ in range(args.warmup):
-            dstep()
-        barrier(world)
-        torch.cuda.synchronize()
-        clk.active = True
-        dt_ms = timed_steps(dstep, args.steps, flush, stream)
-        clk.active = False
-        barrier(world)
-        d_ms = all_max(sum(dt_ms), world) / args.steps
-        nb = algorithmic_decode_bytes(wd)
-        launches += args.steps
-        gbs = nb["state"] / (d_ms / 1e3) / 1e9
-        tot = (nb["state"] + nb["io"]) / (d_ms / 1e3) / 1e9
-        decode[name] = {"workload": f"B={wd.B} S={wd.S} Nk={wd.Nk} Nv={wd.Nv} D={wd.Dk} bf16 pool of "
-                                    f"{wd.pool.shape[0]} slots" + (", per-key gate" if wd.gk is not None else ""),
-                        "us_per_call": d_ms * 1e3, "steps_per_s": world * 1e3 / d_ms,
-                        "state_GBps": gbs, "state_frac_of_hbm": gbs / peaks["hbm_gbs"],
-                        "roofline": {"bound": "hbm", "achieved": tot, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                                     "frac": tot / peaks["hbm_gbs"], "traffic": profiled_traffic("decode"),
-                                     "algorithmic_bytes_per_launch": nb["state"] + nb["io"]}}
-        del pool
-
+        if args.only in ("all", name):
+            decode[name], n = bench_decode(gdr, name, args, world, rank, clk, flush, stream, peaks)
+            launches += n
+    if decode:
+        line["decode"] = decode
     clk.__exit__(None, None, None)
     if gdr.get_error() != 0:
         raise RuntimeError("device error word set during the benchmark")
-
-    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": f"prefill B={w.B} S={w.S} Nk={w.Nk} Nv={w.Nv} Dk=Dv={w.Dk} bf16, fused prologue, "
-                                   "equal lengths", "global_batch": w.B * world, "seq_len": w.S,
-                       "parallelism": f"dp{world} (independent batches per GPU)",
-                       "l2": "inputs larger than L2, plus a 256 MiB flush before every timed step"},
-            "roofline": roofline, "e2e": e2e, "decode": decode, "gpu_launches": launches,
-            "clocks": clk.summary()}
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    line["gpu_launches"] = launches
+    line["clocks"] = clk.summary()
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and args.only in ("all", "prefill"):
         tps, dt, thr = cpu_oracle_sample(workloads.generate("prefill", B=1))
         line["cpu_baseline"] = {"value": tps, "unit": UNIT, "cores": thr, "kind": "oracle",
                                 "sample": f"1 sequence x 4096 tokens x 32 value heads, prologue included, {dt:.1f} s"}
@@ -395,6 +424,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing (for profiling runs)")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg (profiling runs)")
+    ap.add_argument("--only", choices=["all", "prefill", "decode", "decode_gk"], default="all",
+                    help="run one workload only (profiling runs); the default runs all")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

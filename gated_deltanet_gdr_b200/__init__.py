@@ -131,16 +131,14 @@ def _stream(stream) -> ctypes.c_void_p:
     return ctypes.c_void_p(s.cuda_stream)
 
 
-def chunk_fwd(q, k, v, beta, g=None, initial_state=None, actual_seq_lengths=None, scale: float = 1.0, *,
-              prologue: Optional[Prologue] = None, out=None, final_state=None, output_final_state: bool = True,
-              stream=None):
-    """Chunked prefill (``gdr_chunk_fwd``).  Returns (out, final_state or None)."""
+def _chunk_checked(q, k, v, beta, g, initial_state, actual_seq_lengths, prologue, out, final_state,
+                   output_final_state):
     if q.dim() != 4 or v.dim() != 4:
         raise ValueError("q, k must be (B, Nk, S, Dk) and v (B, Nv, S, Dv)")
     B, Nk, S, Dk = q.shape
     Nv, Dv = v.shape[1], v.shape[3]
     dt = q.dtype
-    code = _dtype_code(dt)
+    _dtype_code(dt)
     _dev(q, "q", dt)
     _dev(k, "k", dt, (B, Nk, S, Dk))
     _dev(v, "v", dt, (B, Nv, S, Dv))
@@ -154,30 +152,38 @@ def chunk_fwd(q, k, v, beta, g=None, initial_state=None, actual_seq_lengths=None
     if output_final_state and final_state is None:
         final_state = torch.empty((B, Nv, Dk, Dv), dtype=dt, device=q.device)
     _dev(final_state, "final_state", dt, (B, Nv, Dk, Dv))
-    pro = prologue.as_struct() if prologue is not None else None
     if prologue is not None:
         _dev(prologue.A_log, "A_log", torch.float32, (Nv,))
         _dev(prologue.dt_bias, "dt_bias", torch.float32, (Nv,))
+    return out, final_state
+
+
+def chunk_fwd(q, k, v, beta, g=None, initial_state=None, actual_seq_lengths=None, scale: float = 1.0, *,
+              prologue: Optional[Prologue] = None, out=None, final_state=None, output_final_state: bool = True,
+              stream=None):
+    """Chunked prefill (``gdr_chunk_fwd``).  Returns (out, final_state or None)."""
+    out, final_state = _chunk_checked(q, k, v, beta, g, initial_state, actual_seq_lengths, prologue, out,
+                                      final_state, output_final_state)
+    B, Nk, S, Dk = q.shape
+    Nv, Dv = v.shape[1], v.shape[3]
+    pro = prologue.as_struct() if prologue is not None else None
     st = lib().gdr_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(g), _ptr(initial_state),
-                             _ptr(actual_seq_lengths), float(scale), B, Nk, Nv, S, Dk, Dv, code,
+                             _ptr(actual_seq_lengths), float(scale), B, Nk, Nv, S, Dk, Dv, _dtype_code(q.dtype),
                              ctypes.byref(pro) if pro is not None else None, _ptr(out), _ptr(final_state),
                              _stream(stream))
     _check(st, "gdr_chunk_fwd")
     return out, final_state
 
 
-def recurrent_step(q, k, v, beta, g, gk, state_pool, ssm_state_indices, actual_seq_lengths,
-                   num_accepted_tokens=None, scale: float = 1.0, *, prologue: Optional[Prologue] = None, out=None,
-                   stream=None):
-    """Recurrent decode over a slot pool (``gdr_recurrent_step``), updating
-    ``state_pool`` in place.  Returns (out, state_pool)."""
+def _decode_checked(q, k, v, beta, g, gk, state_pool, ssm_state_indices, actual_seq_lengths, num_accepted_tokens,
+                    out):
     if q.dim() != 4 or v.dim() != 4 or state_pool.dim() != 4:
         raise ValueError("q, k (B, Nk, S, Dk), v (B, Nv, S, Dv), state_pool (slots, Nv, Dk, Dv)")
     B, Nk, S, Dk = q.shape
     Nv, Dv = v.shape[1], v.shape[3]
     dt = q.dtype
-    code = _dtype_code(dt)
-    scode = _dtype_code(state_pool.dtype)
+    _dtype_code(dt)
+    _dtype_code(state_pool.dtype)
     _dev(q, "q", dt)
     _dev(k, "k", dt, (B, Nk, S, Dk))
     _dev(v, "v", dt, (B, Nv, S, Dv))
@@ -193,13 +199,79 @@ def recurrent_step(q, k, v, beta, g, gk, state_pool, ssm_state_indices, actual_s
     if out is None:
         out = torch.empty((B, Nv, S, Dv), dtype=dt, device=q.device)
     _dev(out, "out", dt, (B, Nv, S, Dv))
+    return out
+
+
+def recurrent_step(q, k, v, beta, g, gk, state_pool, ssm_state_indices, actual_seq_lengths,
+                   num_accepted_tokens=None, scale: float = 1.0, *, prologue: Optional[Prologue] = None, out=None,
+                   stream=None):
+    """Recurrent decode over a slot pool (``gdr_recurrent_step``), updating
+    ``state_pool`` in place.  Returns (out, state_pool)."""
+    out = _decode_checked(q, k, v, beta, g, gk, state_pool, ssm_state_indices, actual_seq_lengths,
+                          num_accepted_tokens, out)
+    B, Nk, S, Dk = q.shape
+    Nv, Dv = v.shape[1], v.shape[3]
     pro = prologue.as_struct() if prologue is not None else None
     st = lib().gdr_recurrent_step(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(g), _ptr(gk), _ptr(state_pool),
                                   int(state_pool.shape[0]), _ptr(ssm_state_indices), _ptr(actual_seq_lengths),
-                                  _ptr(num_accepted_tokens), float(scale), B, Nk, Nv, S, Dk, Dv, code, scode,
+                                  _ptr(num_accepted_tokens), float(scale), B, Nk, Nv, S, Dk, Dv,
+                                  _dtype_code(q.dtype), _dtype_code(state_pool.dtype),
                                   ctypes.byref(pro) if pro is not None else None, _ptr(out), _stream(stream))
     _check(st, "gdr_recurrent_step")
     return out, state_pool
+
+
+class PreparedCall:
+    """A C-ABI call with its arguments checked and marshalled once.
+
+    Calling the object launches the library's kernels again on the same buffers
+    (which the caller keeps alive and may refill in place) with no Python-side
+    argument work, for serving loops and for timing the kernels alone.  Raises
+    like the one-shot functions if the library reports an error.
+    """
+
+    def __init__(self, fn, args, what, result):
+        self._fn, self._args, self._what, self.result = fn, args, what, result
+
+    def __call__(self):
+        st = self._fn(*self._args)
+        if st != GDR_OK:
+            _check(st, self._what)
+        return self.result
+
+
+def prepare_chunk_fwd(q, k, v, beta, g=None, initial_state=None, actual_seq_lengths=None, scale: float = 1.0, *,
+                      prologue: Optional[Prologue] = None, out=None, final_state=None, stream=None) -> PreparedCall:
+    """Check and marshal a gdr_chunk_fwd call once; see chunk_fwd for the arguments."""
+    out, final_state = _chunk_checked(q, k, v, beta, g, initial_state, actual_seq_lengths, prologue, out,
+                                      final_state, True)
+    B, Nk, S, Dk = q.shape
+    Nv, Dv = v.shape[1], v.shape[3]
+    pro = prologue.as_struct() if prologue is not None else None
+    args = (_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(g), _ptr(initial_state), _ptr(actual_seq_lengths),
+            ctypes.c_float(scale), B, Nk, Nv, S, Dk, Dv, _dtype_code(q.dtype),
+            ctypes.pointer(pro) if pro is not None else None, _ptr(out), _ptr(final_state), _stream(stream))
+    call = PreparedCall(lib().gdr_chunk_fwd, args, "gdr_chunk_fwd", (out, final_state))
+    call._keep = (pro, prologue)
+    return call
+
+
+def prepare_recurrent_step(q, k, v, beta, g, gk, state_pool, ssm_state_indices, actual_seq_lengths,
+                           num_accepted_tokens=None, scale: float = 1.0, *, prologue: Optional[Prologue] = None,
+                           out=None, stream=None) -> PreparedCall:
+    """Check and marshal a gdr_recurrent_step call once; see recurrent_step for the arguments."""
+    out = _decode_checked(q, k, v, beta, g, gk, state_pool, ssm_state_indices, actual_seq_lengths,
+                          num_accepted_tokens, out)
+    B, Nk, S, Dk = q.shape
+    Nv, Dv = v.shape[1], v.shape[3]
+    pro = prologue.as_struct() if prologue is not None else None
+    args = (_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(g), _ptr(gk), _ptr(state_pool), int(state_pool.shape[0]),
+            _ptr(ssm_state_indices), _ptr(actual_seq_lengths), _ptr(num_accepted_tokens), ctypes.c_float(scale), B,
+            Nk, Nv, S, Dk, Dv, _dtype_code(q.dtype), _dtype_code(state_pool.dtype),
+            ctypes.pointer(pro) if pro is not None else None, _ptr(out), _stream(stream))
+    call = PreparedCall(lib().gdr_recurrent_step, args, "gdr_recurrent_step", (out, state_pool))
+    call._keep = (pro, prologue)
+    return call
 
 
 def prologue(q=None, k=None, b=None, a=None, A_log=None, dt_bias=None, eps: float = 1e-6, *, stream=None):
