@@ -165,14 +165,21 @@ class ClockSampler:
 
 
 def dist_setup():
+    """One process per GPU (torchrun's RANK/LOCAL_RANK/WORLD_SIZE/MASTER_*): NCCL when CUDA is
+    present, gloo otherwise (the CPU tests of this plumbing).  The process group carries only
+    the barrier and the max-over-ranks of the timings: the ranks' batches are independent."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if world > 1:
         import datetime
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=torch.device("cuda", local))
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                    device_id=torch.device("cuda", local))
+        else:
+            dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=60))
     elif torch.cuda.is_available():
         torch.cuda.set_device(local)
     return world, rank, local
@@ -185,12 +192,20 @@ def barrier(world):
 
 
 def all_max(x: float, world: int) -> float:
+    """Max over ranks (the slowest rank sets the job's time)."""
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def weak_scaling_rate(units_per_rank_per_step: int, steps: int, max_total_ms: float, world: int) -> float:
+    """Whole-job throughput: every rank processes its own units each step; the job takes as
+    long as its slowest rank."""
+    return world * units_per_rank_per_step * steps / (max_total_ms / 1e3)
 
 
 def timed_steps(fn, K, flush, stream):
@@ -284,7 +299,7 @@ def bench_prefill(gdr, args, world, rank, clk, flush, stream, peaks):
     alg_bytes = algorithmic_prefill_bytes(w)
     achieved = alg_bytes / (ms_per_step / 1e3) / 1e9
     fields = {
-        "value": world * tokens * args.steps / (total_ms / 1e3), "ms_per_step": ms_per_step,
+        "value": weak_scaling_rate(tokens, args.steps, total_ms, world), "ms_per_step": ms_per_step,
         "config": {"workload": f"prefill B={w.B} S={w.S} Nk={w.Nk} Nv={w.Nv} Dk=Dv={w.Dk} bf16, fused prologue, "
                                "equal lengths", "global_batch": w.B * world, "seq_len": w.S,
                    "parallelism": f"dp{world} (independent batches per GPU)",
