@@ -92,7 +92,7 @@ template <int DK, int DV, typename TI, typename TS> struct DecodeCfg {
         l.stage = l.off_gk + (gk ? S * DK * 4 : 0);
         l.stage = (l.stage + 127) & ~127;
         l.off_meta = 2 * l.stage;
-        l.smem = l.off_meta + 2 * (2 + 3 * kDecodeMaxTokens) * 4;
+        l.smem = l.off_meta + 3 * (2 + 3 * kDecodeMaxTokens) * 4;  // three scalar sets (see the kernel)
         return l;
     }
 };
@@ -207,10 +207,13 @@ decode_kernel(const DecodeArgs a, const int ntiles) {
     issue(tile, s_meta, 0);
     if (tile + (int)gridDim.x < ntiles) prefetch_meta<TI>(a, tile + gridDim.x, Cf::NSPLIT, tid, pre);
 
+    // Stages alternate between two buffers; the scalar sets rotate over three, so a warp that has
+    // finished tile j can already publish the scalars of tile j+1's successor while slower warps
+    // still read tile j's: the only block barrier per tile is the one that makes the copies visible.
     for (int j = 0; tile < ntiles; ++j, tile += gridDim.x) {
         const int stg = j & 1;
         const int nxt = tile + gridDim.x;
-        int *mn = s_meta + (stg ^ 1) * META_INTS;
+        int *mn = s_meta + ((j + 1) % 3) * META_INTS;
         if (nxt < ntiles) put_meta(mn, tid, pre);
         cp_async_wait0();  // the current tile's copies (the only ones in flight)
         __syncthreads();
@@ -220,7 +223,7 @@ decode_kernel(const DecodeArgs a, const int ntiles) {
         }
 
         // ---------------- process the current tile (each warp independently) ----------------
-        const int *mm = s_meta + stg * META_INTS;
+        const int *mm = s_meta + (j % 3) * META_INTS;
         const int split = tile % Cf::NSPLIT, bh = tile / Cf::NSPLIT, h = bh % a.Nv;
         const int col0 = split * DVC;
         const int status = tile_status(mm, S, a.slots);
@@ -347,30 +350,18 @@ decode_kernel(const DecodeArgs a, const int ntiles) {
                     for (int p = 0; p < 4; ++p) sv[r][p] = fma2(k2, pk2(d[2 * p], d[2 * p + 1]), sv[r][p]);
                 }
                 if (t < A && (t == A - 1 || mm[2 + t + 1] != mm[2 + t])) {
-                    // commit: the slab goes back through shared memory so HBM sees whole lines
+                    // commit straight from registers (each store covers 16 rows x 32 bytes per warp)
+                    TS *dst = reinterpret_cast<TS *>(a.pool) + ((size_t)mm[2 + t] * a.Nv + h) * tile_elems + col0 + col;
 #pragma unroll
                     for (int r = 0; r < RPT; ++r) {
                         float f[8];
 #pragma unroll
                         for (int p = 0; p < 4; ++p) up2(sv[r][p], f[2 * p], f[2 * p + 1]);
-                        Vec8<TS>::store(reinterpret_cast<TS *>(slot(r)), f);
+                        Vec8<TS>::store(dst + (size_t)(rg + 16 * r) * DV, f);
                     }
-                    __syncthreads();
-                    uint8_t *dst = reinterpret_cast<uint8_t *>(reinterpret_cast<TS *>(a.pool) +
-                                                               ((size_t)mm[2 + t] * a.Nv + h) * tile_elems + col0);
-#pragma unroll
-                    for (int i = 0; i < Cf::COPY_ITERS; ++i) {
-                        const int e = i * NT + tid, row = e / CPR, pc = e % CPR;
-                        *reinterpret_cast<uint4 *>(dst + (size_t)row * DV * sizeof(TS) + pc * 16) =
-                            *reinterpret_cast<const uint4 *>(st + row * RS + pc * 16);
-                    }
-                    // another commit of this tile would rewrite the slab; the last one is covered by
-                    // the barrier that ends the tile
-                    if (t + 1 < A) __syncthreads();
                 }
             }
         }
-        __syncthreads();  // the stage and its scalars are rewritten for the tile after next
     }
     cp_async_wait0();
 }
