@@ -39,21 +39,37 @@ namespace gdr {
 using namespace sm100;
 
 #ifdef GDR_PHASE_TIMERS
-// Development aid, compiled only with -DGDR_PHASE_TIMERS: accumulated clock64() cycles per
-// phase of CTA 0 (slots 0..15 prep group, 16..31 carry group), read by gdr_phase_timers_read.
+// Development aid, compiled only with -DGDR_PHASE_TIMERS: clock64() cycles per phase, summed
+// in shared memory (so that taking a time stalls nothing) and added to g_phase by CTA 0 at
+// the end; slots 0..15 prep group, 16..31 carry group; read by gdr_phase_timers_read.
 __device__ unsigned long long g_phase[64];
 #define PHASE(slot)                                                            \
     do {                                                                       \
-        if (blockIdx.x == 0 && (tid == 0 || tid == NGRP)) {                    \
+        if (tid == 0 || tid == NGRP) {                                         \
             const unsigned long long now_ = clock64();                         \
-            g_phase[(slot)] += now_ - t_prev_;                                 \
+            s_phase_[(slot)] += now_ - t_prev_;                                \
             t_prev_ = now_;                                                    \
         }                                                                      \
     } while (0)
+// cycles one thread spends in the statements, accumulated into `slot`
+#define TIMED(slot, ...)                                                       \
+    do {                                                                       \
+        const unsigned long long t0_ = clock64();                              \
+        __VA_ARGS__;                                                           \
+        s_phase_[(slot)] += clock64() - t0_;                                   \
+    } while (0)
+#define SOLVE_TIMER_ARGS , unsigned long long &t_prev_, int tid, unsigned long long *s_phase_
+#define SOLVE_TIMER_PASS , t_prev_, tid, s_phase_
 #else
 #define PHASE(slot) \
     do {            \
     } while (0)
+#define TIMED(slot, ...) \
+    do {                 \
+        __VA_ARGS__;     \
+    } while (0)
+#define SOLVE_TIMER_ARGS
+#define SOLVE_TIMER_PASS
 #endif
 
 namespace {
@@ -61,6 +77,8 @@ namespace {
 constexpr int C = 64, D = 128, NT = 512, NGRP = 256;
 constexpr int BAR_CARRY = 1, BAR_PREP = 2;
 constexpr uint32_t kTimeoutBit = 0x4u;
+// carry thread that issues the out-tile TMA stores (thread 0 issues the carry's MMAs)
+constexpr int kStorer = 32;
 
 // ---- shared memory map (bytes from a 1024-aligned base) ----
 // input stage: [K_b0 | Q_b0 | K_b1 | Q_b1 | V_b0 | V_b1], each 64 rows x 128 B (64 bf16)
@@ -71,20 +89,19 @@ constexpr uint32_t OFF_S = 81920;    // S bf16, MN-major (K = dk rows, N = dv): 
 constexpr uint32_t OFF_KT = 114688;  // K~ MN-major (M = dk, K = tok): dk blocks at +0, +8K
 constexpr uint32_t OFF_PM = 131072;  // [0; Pm] K-major 128 x 64
 constexpr uint32_t OFF_VO = 147456;  // v_new (MN-major, K = tok, N = dv) then the out tile: dv blocks +0, +8K
-constexpr int FP = 68;               // row stride (floats) of T and E: 16-byte aligned rows for float4 access
+constexpr int FP = 68;               // row stride (floats) of T: 16-byte aligned rows for float4 access
 constexpr int FA = 65;               // row stride of A: odd, so the row-per-thread stores are conflict-free
 constexpr int XP = 36;               // row stride of the merge scratch
 constexpr uint32_t OFF_AF = 163840;  // A (fp32); after the solve it holds TT = [T diag(beta); T diag(c_W)]
 constexpr uint32_t OFF_TT = OFF_AF;
 constexpr uint32_t OFF_TF = OFF_AF + 64 * FA * 4;  // T (fp32)
-constexpr uint32_t OFF_E = OFF_TF + 64 * FP * 4;   // E[t][s] = e^{G_t - G_s} (s <= t), fp32
-constexpr uint32_t OFF_X = OFF_E + 64 * FP * 4;
+constexpr uint32_t OFF_X = OFF_TF + 64 * FP * 4;
 constexpr uint32_t OFF_VEC = OFF_X + 32 * XP * 4;  // 2 sets x 8 vectors x 64 floats
 constexpr uint32_t OFF_BAR = OFF_VEC + 2 * 8 * 64 * 4;
 constexpr uint32_t SMEM_USED = OFF_BAR + 128;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;  // + alignment slack
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
-static_assert(OFF_TF % 16 == 0 && OFF_E % 16 == 0 && OFF_X % 16 == 0, "float4 alignment");
+static_assert(OFF_TF % 16 == 0 && OFF_X % 16 == 0, "float4 alignment");
 static_assert(OFF_TF >= OFF_TT + 16384, "TT must fit inside the A matrix area");
 
 // TMEM columns (all 128 lanes): [G;P] then W, U, R = [W S; o], the fp32 state S
@@ -128,7 +145,7 @@ __device__ __forceinline__ uint4 pack8(const float *f) {
 // T = (I + A)^{-1} for a strictly lower 64 x 64 A (fp32, row stride FA; T row stride FP), by the 256 prep
 // threads (p = 0..255).  Writes the lower triangle of T and zeros in the upper 16 x 16
 // blocks that the merges read.
-__device__ __forceinline__ void solve_unit_lower(const float *sA, float *sT, float *sX, int p) {
+__device__ __forceinline__ void solve_unit_lower(const float *sA, float *sT, float *sX, int p SOLVE_TIMER_ARGS) {
     if (p < 64) {  // 16 x 16 diagonal blocks, one column per thread
         const int base = (p >> 4) * 16, j = p & 15;
         float x[16];
@@ -154,6 +171,7 @@ __device__ __forceinline__ void solve_unit_lower(const float *sA, float *sT, flo
         }
     }
     named_sync(BAR_PREP, NGRP);
+    PHASE(13);
     // 16 -> 32: X_b = A21 T11, then T21 = -T22 X_b, for the blocks at rows 32b+16, cols 32b
     {
         const int blk = p >> 7, r = (p >> 3) & 15, c2 = (p & 7) * 2, r0 = 32 * blk + 16, c0 = 32 * blk;
@@ -178,6 +196,7 @@ __device__ __forceinline__ void solve_unit_lower(const float *sA, float *sT, flo
         *reinterpret_cast<float2 *>(sT + (r0 + r) * FP + c0 + c2) = make_float2(-y0, -y1);
     }
     named_sync(BAR_PREP, NGRP);
+    PHASE(14);
     // 32 -> 64: X = A21 T11, T21 = -T22 X with 32 x 32 blocks; one row x 4 columns per thread
     {
         const int r = p >> 3, c4 = (p & 7) * 4;
@@ -211,8 +230,10 @@ __device__ __forceinline__ void solve_unit_lower(const float *sA, float *sT, flo
 __global__ void __launch_bounds__(NT, 1)
 chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o, const TcArgs a) {
-    extern __shared__ uint8_t smraw[];
-    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smraw) + 1023) & ~uintptr_t(1023));
+    extern __shared__ __align__(1024) uint8_t smraw[];
+    // 1024-byte aligned base, derived from smraw by pointer arithmetic (not through an
+    // integer) so that the compiler keeps every access below in the shared address space
+    uint8_t *sm = smraw + ((1024u - (smem_u32(smraw) & 1023u)) & 1023u);
     const uint32_t sbase = smem_u32(sm);
     float *vecs = reinterpret_cast<float *>(sm + OFF_VEC);
     uint64_t *bar_ld = reinterpret_cast<uint64_t *>(sm + OFF_BAR);
@@ -222,7 +243,6 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     volatile int *s_abort = reinterpret_cast<volatile int *>(s_tmem + 1);
     float *sA = reinterpret_cast<float *>(sm + OFF_AF), *sT = reinterpret_cast<float *>(sm + OFF_TF);
     float *sX = reinterpret_cast<float *>(sm + OFF_X);
-    float *sE = reinterpret_cast<float *>(sm + OFF_E);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, q4 = warp & 3, hf = (warp >> 2) & 1;
     const bool carry = warp < 8;
@@ -285,10 +305,17 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 
 #ifdef GDR_PHASE_TIMERS
     unsigned long long t_prev_ = clock64();
+    __shared__ unsigned long long s_phase_[64];
+    if (tid < 64) s_phase_[tid] = 0;
+    __syncthreads();
 #endif
     if (!carry) {
         // =============================== prep group ===============================
         const int p = tid - NGRP;
+        // One thread issues the MMAs and nothing else, another the TMA loads and L2 prefetches:
+        // an MMA issued by a thread with global loads or bulk copies still outstanding was seen
+        // to wait for them.
+        const bool issuer = (p == 64), loader = (p == 96);
         const float gA = (a.A_log && a.g) ? a.A_log[h] : 0.f, gB = (a.A_log && a.g) ? a.dt_bias[h] : 0.f;
         const __nv_bfloat16 *bg = reinterpret_cast<const __nv_bfloat16 *>(a.beta) + (size_t)bh * S;
         const float *gg = a.g ? a.g + (size_t)bh * S : nullptr;
@@ -301,6 +328,15 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 nb = __bfloat162float(bg[t]);
                 if (gg) ng = gg[t];
             }
+        };
+        auto prefetch_l2 = [&](int chunk) {
+            const int y = chunk * C;
+            tma_prefetch_3d(&tm_k, 0, y, zq);
+            tma_prefetch_3d(&tm_k, 64, y, zq);
+            tma_prefetch_3d(&tm_q, 0, y, zq);
+            tma_prefetch_3d(&tm_q, 64, y, zq);
+            tma_prefetch_3d(&tm_v, 0, y, bh);
+            tma_prefetch_3d(&tm_v, 64, y, bh);
         };
         auto issue_loads = [&](int chunk) {
             const int y = chunk * C;
@@ -316,7 +352,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         auto wait_ok = [&](uint64_t *bar, uint32_t parity) {
             if (!mbar_wait(bar, parity)) to = true;
         };
-        if (p == 0 && nvalid > 0) issue_loads(0);
+        if (loader && nvalid > 0) issue_loads(0);
         fetch(0);
         for (int c = 0; c < nvalid; ++c) {
             const uint32_t par = c & 1;
@@ -330,6 +366,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 vGam[p] = valid ? (a.A_log ? gate_from_raw(ng, gA, gB) : ng) : 0.f;
             }
             fetch(c + 1);
+            if (loader && c + 1 < nvalid) prefetch_l2(c + 1);
             wait_ok(bar_ld, par);
             if (named_sync_or(BAR_PREP, NGRP, to)) break;
             PHASE(0);
@@ -342,15 +379,17 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             }
             named_sync(BAR_PREP, NGRP);
             // ---- a2: [G; P] = [K; Q] K^T, issued first; the scalar work below overlaps it ----
-            if (p == 0) {
+            if (issuer) {
                 tc_fence_after();
                 const uint32_t id = idesc_bf16(128, 64, false, false);
-#pragma unroll
-                for (int k = 0; k < 8; ++k) {
-                    const uint32_t addr = sbase + OFF_K0 + (k >> 2) * 16384 + (k & 3) * 32;
-                    mma_bf16(tmem + TM_GPW, sdesc_sw128(addr, 16, 1024), sdesc_sw128(addr, 16, 1024), id, k > 0);
-                }
-                mma_commit(bar_gp);
+                TIMED(21, {
+                    _Pragma("unroll")
+                    for (int k = 0; k < 8; ++k) {
+                        const uint32_t addr = sbase + OFF_K0 + (k >> 2) * 16384 + (k & 3) * 32;
+                        mma_bf16(tmem + TM_GPW, sdesc_sw128(addr, 16, 1024), sdesc_sw128(addr, 16, 1024), id, k > 0);
+                    }
+                    mma_commit(bar_gp);
+                });
             }
             PHASE(10);
             if (p < 32) {  // inclusive scan of the gate over the chunk (warp 8)
@@ -366,15 +405,21 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 vGam[2 * p] = excl + x0;
                 vGam[2 * p + 1] = excl + x1;
             }
+#ifdef GDR_PHASE_TIMERS
+            const unsigned long long tn0_ = clock64();
+#endif
             {  // row norms of k and q: 4 threads per row, 32 elements each
                 const int r = p >> 2, part = p & 3;
                 const uint32_t off = (part >> 1) * 16384 + r * 128 + (part & 1) * 64;
                 float sk = 0.f, sq = 0.f;
 #pragma unroll
                 for (int ch = 0; ch < 4; ++ch) {
+                    // the order of the row's chunks does not matter for the sum; rotating it by
+                    // the row spreads the warp's 8 rows over all banks
+                    const uint32_t o = off + ((ch + r) & 3) * 16;
                     float fk[8], fq[8];
-                    unpack8(*reinterpret_cast<const uint4 *>(sm + OFF_K0 + off + ch * 16), fk);
-                    unpack8(*reinterpret_cast<const uint4 *>(sm + OFF_Q0 + off + ch * 16), fq);
+                    unpack8(*reinterpret_cast<const uint4 *>(sm + OFF_K0 + o), fk);
+                    unpack8(*reinterpret_cast<const uint4 *>(sm + OFF_Q0 + o), fq);
 #pragma unroll
                     for (int i = 0; i < 8; ++i) {
                         sk = fmaf(fk[i], fk[i], sk);
@@ -390,19 +435,11 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     vRq[r] = r < n ? a.scale * (a.l2norm ? rsqrtf(sq + a.eps) : 1.f) : 0.f;
                 }
             }
+#ifdef GDR_PHASE_TIMERS
+            if (lane == 0) s_phase_[40 + warp - 8] += clock64() - tn0_;
+#endif
             named_sync(BAR_PREP, NGRP);
             PHASE(11);
-            {  // decay matrix E[t][s] = e^{G_t - G_s} for s <= t, 16 entries per thread
-                const int t = p >> 2, s0 = (p & 3) * 16;
-                const float gt = vGam[t];
-                float e[16];
-#pragma unroll
-                for (int i = 0; i < 16; ++i) e[i] = (s0 + i <= t) ? __expf(gt - vGam[s0 + i]) : 0.f;
-#pragma unroll
-                for (int i = 0; i < 4; ++i)
-                    *reinterpret_cast<float4 *>(sE + t * FP + s0 + 4 * i) =
-                        make_float4(e[4 * i], e[4 * i + 1], e[4 * i + 2], e[4 * i + 3]);
-            }
             if (p < C) {
                 const float gl = vGam[C - 1], gt = vGam[p];
                 vEG[p] = __expf(gt);
@@ -415,34 +452,47 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             wait_ok(bar_gp, par);
             tc_fence_after();
             PHASE(2);
-            {  // A rows (from G, lanes 0..63) and Pm rows (from P, lanes 64..127; parked in TMEM as fp32)
+            // A rows (from G, lanes 0..63) and Pm rows (from P, lanes 64..127; parked in TMEM as
+            // fp32), with the decay e^{G_t - G_s} taken per entry.  Columns s > t are never read
+            // (the solve reads the strict lower triangle, the Pm conversion masks), so the warps
+            // whose 32 x 32 block lies wholly above the diagonal skip it.
+#ifdef GDR_PHASE_TIMERS
+            const unsigned long long tb0_ = clock64();
+#endif
+            if (!((q4 & 1) == 0 && hf == 1)) {
                 float v[32];
                 const uint32_t ta = tmem + TM_GPW + lane_base + 32 * hf;
                 tmem_ld32(ta, v);
                 tmem_ld_wait();
                 PHASE(12);
                 const int t = row & 63;
-                const float *et = sE + t * FP + 32 * hf;
+                const float gt = vGam[t];
                 if (q4 < 2) {
                     const float rb = t < n ? vBeta[t] * vRk[t] : 0.f;
 #pragma unroll
                     for (int j = 0; j < 32; ++j) {
                         const int s = 32 * hf + j;
-                        sA[t * FA + s] = s < t ? rb * vRk[s] * v[j] * et[j] : 0.f;
+                        sA[t * FA + s] = s < t ? rb * vRk[s] * v[j] * __expf(gt - vGam[s]) : 0.f;
                     }
                 } else {
                     const float rq = t < n ? vRq[t] : 0.f;
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) v[j] = rq * vRk[32 * hf + j] * v[j] * et[j];
+                    for (int j = 0; j < 32; ++j) {
+                        const int s = 32 * hf + j;
+                        v[j] = s <= t ? rq * vRk[s] * v[j] * __expf(gt - vGam[s]) : 0.f;
+                    }
                     tmem_st32(ta, v);
                     tmem_st_wait();
                 }
             }
+#ifdef GDR_PHASE_TIMERS
+            if (lane == 0) s_phase_[32 + warp - 8] += clock64() - tb0_;
+#endif
             tc_fence_before();
             if (named_sync_or(BAR_PREP, NGRP, to)) break;
             PHASE(3);
             // ---- a3: T = (I + A)^{-1} and the bf16 operand [T diag(beta); T diag(c_W)] ----
-            solve_unit_lower(sA, sT, sX, p);
+            solve_unit_lower(sA, sT, sX, p SOLVE_TIMER_PASS);
             PHASE(4);
             for (int e = p; e < 128 * 8; e += NGRP) {
                 const int R = e >> 3, j = e & 7, t = R & 63;
@@ -477,15 +527,17 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             tc_fence_after();
             PHASE(7);
             // ---- a4: W (rows 64..127 of TT K) and U (rows 0..63 of TT V) ----
-            if (p == 0) {
+            if (issuer) {
                 const uint32_t id = idesc_bf16(128, 128, false, true);
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    const uint64_t ad = sdesc_sw128(sbase + OFF_TT + k * 32, 16, 1024);
-                    mma_bf16(tmem + TM_GPW, ad, sdesc_sw128(sbase + OFF_K0 + k * 2048, 16384, 1024), id, k > 0);
-                    mma_bf16(tmem + TM_U, ad, sdesc_sw128(sbase + OFF_V0 + k * 2048, 8192, 1024), id, k > 0);
-                }
-                mma_commit(bar_wu);
+                TIMED(22, {
+                    _Pragma("unroll")
+                    for (int k = 0; k < 4; ++k) {
+                        const uint64_t ad = sdesc_sw128(sbase + OFF_TT + k * 32, 16, 1024);
+                        mma_bf16(tmem + TM_GPW, ad, sdesc_sw128(sbase + OFF_K0 + k * 2048, 16384, 1024), id, k > 0);
+                        mma_bf16(tmem + TM_U, ad, sdesc_sw128(sbase + OFF_V0 + k * 2048, 8192, 1024), id, k > 0);
+                    }
+                    mma_commit(bar_wu);
+                });
             }
             // meanwhile: X_g rows (64..127 of A1) and K~ from the staged q/k tiles
             for (int e = p; e < 2 * 64 * 16; e += NGRP) {
@@ -510,7 +562,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             tc_fence_after();
             if (named_sync_or(BAR_PREP, NGRP, to)) break;  // staged tiles fully consumed
             PHASE(8);
-            if (p == 0 && c + 1 < nvalid) issue_loads(c + 1);
+            if (loader && c + 1 < nvalid) issue_loads(c + 1);
             if (q4 >= 2) {  // W rows -> rows 0..63 of A1
                 const int t = row - 64;
 #pragma unroll
@@ -550,13 +602,15 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             // ---- R = [W; X_g] S ----
             if (tid == 0) {
                 const uint32_t id = idesc_bf16(128, 128, false, true);
-#pragma unroll
-                for (int k = 0; k < 8; ++k) {
-                    const uint64_t ad = sdesc_sw128(sbase + OFF_A1 + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024);
-                    const uint64_t bd = sdesc_sw128(sbase + OFF_S + k * 2048, 16384, 1024);
-                    mma_bf16(tmem + TM_R, ad, bd, id, k > 0);
-                }
-                mma_commit(bar_m1);
+                TIMED(23, {
+                    _Pragma("unroll")
+                    for (int k = 0; k < 8; ++k) {
+                        const uint64_t ad = sdesc_sw128(sbase + OFF_A1 + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024);
+                        const uint64_t bd = sdesc_sw128(sbase + OFF_S + k * 2048, 16384, 1024);
+                        mma_bf16(tmem + TM_R, ad, bd, id, k > 0);
+                    }
+                    mma_commit(bar_m1);
+                });
             }
             // meanwhile: S <- e^{G_last} S in TMEM (MMA2 accumulates onto it)
 #pragma unroll
@@ -571,7 +625,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             }
             tmem_st_wait();
             wait_ok(bar_m1, par);
-            if (tid == 0) bulk_wait_read0();  // the previous out tile (same buffer as v_new) is read
+            if (tid == kStorer) bulk_wait_read0();  // the previous out tile (same buffer as v_new) is read
             tc_fence_before();
             if (named_sync_or(BAR_CARRY, NGRP, to)) { stop = true; break; }
             tc_fence_after();
@@ -601,17 +655,19 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             if (tid == 0) {
                 const uint32_t id_s = idesc_bf16(128, 128, true, true);
                 const uint32_t id_o = idesc_bf16(128, 128, false, true);
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    const uint64_t bd = sdesc_sw128(sbase + OFF_VO + k * 2048, 8192, 1024);
-                    mma_bf16(tmem + TM_S, sdesc_sw128(sbase + OFF_KT + k * 2048, 8192, 1024), bd, id_s, 1);
-                }
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    const uint64_t bd = sdesc_sw128(sbase + OFF_VO + k * 2048, 8192, 1024);
-                    mma_bf16(tmem + TM_R, sdesc_sw128(sbase + OFF_PM + k * 32, 16, 1024), bd, id_o, 1);
-                }
-                mma_commit(bar_m2);
+                TIMED(24, {
+                    _Pragma("unroll")
+                    for (int k = 0; k < 4; ++k) {
+                        const uint64_t bd = sdesc_sw128(sbase + OFF_VO + k * 2048, 8192, 1024);
+                        mma_bf16(tmem + TM_S, sdesc_sw128(sbase + OFF_KT + k * 2048, 8192, 1024), bd, id_s, 1);
+                    }
+                    _Pragma("unroll")
+                    for (int k = 0; k < 4; ++k) {
+                        const uint64_t bd = sdesc_sw128(sbase + OFF_VO + k * 2048, 8192, 1024);
+                        mma_bf16(tmem + TM_R, sdesc_sw128(sbase + OFF_PM + k * 32, 16, 1024), bd, id_o, 1);
+                    }
+                    mma_commit(bar_m2);
+                });
             }
             wait_ok(bar_m2, par);
             tc_fence_after();
@@ -647,7 +703,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             tc_fence_before();
             named_sync(BAR_CARRY, NGRP);
             tc_fence_after();
-            if (tid == 0) {
+            if (tid == kStorer) {
                 tma_store_3d(&tm_o, sm + OFF_VO, 0, c * C, bh);
                 tma_store_3d(&tm_o, sm + OFF_VO + 8192, 64, c * C, bh);
                 bulk_commit();
@@ -658,13 +714,13 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         if (!stop) {
             // chunks past the length: zero rows
             if (nvalid < ntotal) {
-                if (tid == 0) bulk_wait_read0();
+                if (tid == kStorer) bulk_wait_read0();
                 named_sync(BAR_CARRY, NGRP);
                 for (int e = tid; e < 16384 / 16; e += NGRP)
                     reinterpret_cast<uint4 *>(sm + OFF_VO)[e] = make_uint4(0, 0, 0, 0);
                 fence_proxy_async_smem();
                 named_sync(BAR_CARRY, NGRP);
-                if (tid == 0) {
+                if (tid == kStorer) {
                     for (int c = nvalid; c < ntotal; ++c) {
                         tma_store_3d(&tm_o, sm + OFF_VO, 0, c * C, bh);
                         tma_store_3d(&tm_o, sm + OFF_VO + 8192, 64, c * C, bh);
@@ -686,11 +742,14 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 }
             }
         }
-        if (tid == 0) bulk_wait0();
+        if (tid == kStorer) bulk_wait0();
     }
     tc_fence_before();
     __syncthreads();
     if (tid == 0 && *s_abort) raise_device_error(a.err, kTimeoutBit);
+#ifdef GDR_PHASE_TIMERS
+    if (blockIdx.x == 0 && tid < 64) g_phase[tid] += s_phase_[tid];
+#endif
     if (warp == 0) tmem_dealloc(tmem, TM_COLS);
 }
 
