@@ -74,8 +74,11 @@ __device__ unsigned long long g_phase[64];
 
 namespace {
 
-constexpr int C = 64, D = 128, NT = 512, NGRP = 256;
-constexpr int BAR_CARRY = 1, BAR_PREP = 2;
+// warps 0-7 carry, 8-15 prep, 16 control (TMA loads and the prep MMAs)
+constexpr int C = 64, D = 128, NGRP = 256, NT = 2 * NGRP + 32, NPC = NGRP + 32;
+constexpr int CTL_WARP = 16;
+// BAR_PCTL: the prep warps and the control warp, at the hand-offs between them
+constexpr int BAR_CARRY = 1, BAR_PREP = 2, BAR_PCTL = 3;
 constexpr uint32_t kTimeoutBit = 0x4u;
 // carry thread that issues the out-tile TMA stores (thread 0 issues the carry's MMAs)
 constexpr int kStorer = 32;
@@ -90,14 +93,15 @@ constexpr uint32_t OFF_KT = 114688;  // K~ MN-major (M = dk, K = tok): dk blocks
 constexpr uint32_t OFF_PM = 131072;  // [0; Pm] K-major 128 x 64
 constexpr uint32_t OFF_VO = 147456;  // v_new (MN-major, K = tok, N = dv) then the out tile: dv blocks +0, +8K
 constexpr int FP = 68;               // row stride (floats) of T: 16-byte aligned rows for float4 access
-constexpr int FA = 65;               // row stride of A: odd, so the row-per-thread stores are conflict-free
+constexpr int FA = 68;               // row stride of A: each quarter-warp's 16-byte row stores hit distinct banks
 constexpr int XP = 36;               // row stride of the merge scratch
 constexpr uint32_t OFF_AF = 163840;  // A (fp32); after the solve it holds TT = [T diag(beta); T diag(c_W)]
 constexpr uint32_t OFF_TT = OFF_AF;
 constexpr uint32_t OFF_TF = OFF_AF + 64 * FA * 4;  // T (fp32)
 constexpr uint32_t OFF_X = OFF_TF + 64 * FP * 4;
-constexpr uint32_t OFF_VEC = OFF_X + 32 * XP * 4;  // 2 sets x 8 vectors x 64 floats
-constexpr uint32_t OFF_BAR = OFF_VEC + 2 * 8 * 64 * 4;
+constexpr int NVEC = 10;             // per-chunk vectors of 64 floats (enum below)
+constexpr uint32_t OFF_VEC = OFF_X + 32 * XP * 4;  // 2 sets x NVEC vectors x 64 floats
+constexpr uint32_t OFF_BAR = OFF_VEC + 2 * NVEC * 64 * 4;
 constexpr uint32_t SMEM_USED = OFF_BAR + 128;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;  // + alignment slack
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
@@ -107,7 +111,10 @@ static_assert(OFF_TF >= OFF_TT + 16384, "TT must fit inside the A matrix area");
 // TMEM columns (all 128 lanes): [G;P] then W, U, R = [W S; o], the fp32 state S
 constexpr uint32_t TM_GPW = 0, TM_U = 128, TM_R = 256, TM_S = 384, TM_COLS = 512;
 
-enum { V_BETA = 0, V_GAM, V_EG, V_TAIL, V_RK, V_RQ, V_CW, V_N };
+// V_G2 = G log2(e); V_LAM = V_G2 - log2(1/|k|), so that e^{G_t - G_s} / |k_s| = 2^{V_G2[t] - V_LAM[s]};
+// V_N holds the chunk's valid-token count in its first entry.
+enum { V_BETA = 0, V_GAM, V_EG, V_TAIL, V_RK, V_RQ, V_CW, V_G2, V_LAM, V_N };
+static_assert(V_N < NVEC, "vector slots");
 
 struct TcArgs {
     const void *beta;
@@ -126,6 +133,18 @@ struct TcArgs {
 
 __device__ __forceinline__ uint32_t blk_off(uint32_t row, uint32_t col) {  // within a 128-B-row block
     return (row >> 3) * 1024u + sw128_offset(row & 7u, col);
+}
+
+// 2^x and log2(x) on the special-function unit (PTX ex2.approx / lg2.approx, flush to zero)
+__device__ __forceinline__ float ex2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+__device__ __forceinline__ float lg2_approx(float x) {
+    float y;
+    asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
 }
 
 __device__ __forceinline__ void unpack8(uint4 u, float (&f)[8]) {
@@ -245,7 +264,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     float *sX = reinterpret_cast<float *>(sm + OFF_X);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, q4 = warp & 3, hf = (warp >> 2) & 1;
-    const bool carry = warp < 8;
+    const bool carry = warp < 8, control = warp == CTL_WARP;
     const int bh = blockIdx.x, h = bh % a.Nv, b = bh / a.Nv, kh = h / (a.Nv / a.Nk);
     const int S = a.S;
     int L = a.lengths ? a.lengths[b] : S;
@@ -309,26 +328,13 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     if (tid < 64) s_phase_[tid] = 0;
     __syncthreads();
 #endif
-    if (!carry) {
-        // =============================== prep group ===============================
-        const int p = tid - NGRP;
-        // One thread issues the MMAs and nothing else, another the TMA loads and L2 prefetches:
-        // an MMA issued by a thread with global loads or bulk copies still outstanding was seen
-        // to wait for them.
-        const bool issuer = (p == 64), loader = (p == 96);
-        const float gA = (a.A_log && a.g) ? a.A_log[h] : 0.f, gB = (a.A_log && a.g) ? a.dt_bias[h] : 0.f;
-        const __nv_bfloat16 *bg = reinterpret_cast<const __nv_bfloat16 *>(a.beta) + (size_t)bh * S;
-        const float *gg = a.g ? a.g + (size_t)bh * S : nullptr;
-        float nb = 0.f, ng = 0.f;  // prefetched raw beta / gate of the next chunk (threads p < 64)
-        auto fetch = [&](int chunk) {
-            nb = 0.f;
-            ng = 0.f;
-            const int t = chunk * C + p;
-            if (p < C && chunk < nvalid && t < L) {
-                nb = __bfloat162float(bg[t]);
-                if (gg) ng = gg[t];
-            }
-        };
+    if (control) {
+        // ============================== control warp ==============================
+        // Lane 0 issues the prep MMAs and nothing else, lane 1 the TMA loads and L2 prefetches
+        // (an MMA issued by a thread with copies of its own outstanding was seen to wait for
+        // them).  Having a warp of its own, neither blocks a prep warp while the tensor pipe is
+        // busy.  The warp follows the prep group's hand-off barriers (BAR_PCTL) and leaves
+        // at the same barrier as the prep group when a wait timed out.
         auto prefetch_l2 = [&](int chunk) {
             const int y = chunk * C;
             tma_prefetch_3d(&tm_k, 0, y, zq);
@@ -348,15 +354,63 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             tma_load_3d(sm + OFF_V0, &tm_v, bar_ld, 0, y, bh);
             tma_load_3d(sm + OFF_V0 + 8192, &tm_v, bar_ld, 64, y, bh);
         };
+        if (lane == 1 && nvalid > 0) {
+            issue_loads(0);
+            if (nvalid > 1) prefetch_l2(1);
+        }
+        for (int c = 0; c < nvalid; ++c) {
+            if (named_sync_or(BAR_PCTL, NPC, false)) break;  // H0: chunk c staged (or a timeout)
+            if (lane == 1 && c + 2 < nvalid) prefetch_l2(c + 2);
+            named_sync(BAR_PCTL, NPC);  // H1: padding rows zeroed
+            if (lane == 0) {  // a2: [G; P] = [K; Q] K^T
+                tc_fence_after();
+                const uint32_t id = idesc_bf16(128, 64, false, false);
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    const uint32_t addr = sbase + OFF_K0 + (k >> 2) * 16384 + (k & 3) * 32;
+                    mma_bf16(tmem + TM_GPW, sdesc_sw128(addr, 16, 1024), sdesc_sw128(addr, 16, 1024), id, k > 0);
+                }
+                mma_commit(bar_gp);
+            }
+            if (named_sync_or(BAR_PCTL, NPC, false)) break;  // H2: TT operand and Pm in place
+            if (lane == 0) {  // a4: W (rows 64..127 of TT K) and U (rows 0..63 of TT V)
+                tc_fence_after();
+                const uint32_t id = idesc_bf16(128, 128, false, true);
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const uint64_t ad = sdesc_sw128(sbase + OFF_TT + k * 32, 16, 1024);
+                    mma_bf16(tmem + TM_GPW, ad, sdesc_sw128(sbase + OFF_K0 + k * 2048, 16384, 1024), id, k > 0);
+                    mma_bf16(tmem + TM_U, ad, sdesc_sw128(sbase + OFF_V0 + k * 2048, 8192, 1024), id, k > 0);
+                }
+                mma_commit(bar_wu);
+            }
+            if (named_sync_or(BAR_PCTL, NPC, false)) break;  // H3: staged tiles fully consumed
+            if (lane == 1 && c + 1 < nvalid) issue_loads(c + 1);
+        }
+    } else if (!carry) {
+        // =============================== prep group ===============================
+        const int p = tid - NGRP;
+        const float gA = (a.A_log && a.g) ? a.A_log[h] : 0.f, gB = (a.A_log && a.g) ? a.dt_bias[h] : 0.f;
+        const __nv_bfloat16 *bg = reinterpret_cast<const __nv_bfloat16 *>(a.beta) + (size_t)bh * S;
+        const float *gg = a.g ? a.g + (size_t)bh * S : nullptr;
+        float nb = 0.f, ng = 0.f;  // prefetched raw beta / gate of the next chunk (threads p < 64)
+        auto fetch = [&](int chunk) {
+            nb = 0.f;
+            ng = 0.f;
+            const int t = chunk * C + p;
+            if (p < C && chunk < nvalid && t < L) {
+                nb = __bfloat162float(bg[t]);
+                if (gg) ng = gg[t];
+            }
+        };
         bool to = false;  // a wait of this thread timed out
         auto wait_ok = [&](uint64_t *bar, uint32_t parity) {
             if (!mbar_wait(bar, parity)) to = true;
         };
-        if (loader && nvalid > 0) issue_loads(0);
         fetch(0);
         for (int c = 0; c < nvalid; ++c) {
             const uint32_t par = c & 1;
-            float *vec = vecs + (c & 1) * 8 * 64;
+            float *vec = vecs + (c & 1) * NVEC * 64;
             float *vBeta = vec + V_BETA * 64, *vGam = vec + V_GAM * 64, *vEG = vec + V_EG * 64;
             float *vTail = vec + V_TAIL * 64, *vRk = vec + V_RK * 64, *vRq = vec + V_RQ * 64, *vCw = vec + V_CW * 64;
             const int n = min(C, L - c * C);
@@ -366,9 +420,8 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 vGam[p] = valid ? (a.A_log ? gate_from_raw(ng, gA, gB) : ng) : 0.f;
             }
             fetch(c + 1);
-            if (loader && c + 1 < nvalid) prefetch_l2(c + 1);
             wait_ok(bar_ld, par);
-            if (named_sync_or(BAR_PREP, NGRP, to)) break;
+            if (named_sync_or(BAR_PCTL, NPC, to)) break;  // H0
             PHASE(0);
             if (n < C) {  // padding rows of the last chunk: zero them so no padding value reaches a product
                 for (int e = p; e < (C - n) * 48; e += NGRP) {
@@ -377,20 +430,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 }
                 fence_proxy_async_smem();
             }
-            named_sync(BAR_PREP, NGRP);
-            // ---- a2: [G; P] = [K; Q] K^T, issued first; the scalar work below overlaps it ----
-            if (issuer) {
-                tc_fence_after();
-                const uint32_t id = idesc_bf16(128, 64, false, false);
-                TIMED(21, {
-                    _Pragma("unroll")
-                    for (int k = 0; k < 8; ++k) {
-                        const uint32_t addr = sbase + OFF_K0 + (k >> 2) * 16384 + (k & 3) * 32;
-                        mma_bf16(tmem + TM_GPW, sdesc_sw128(addr, 16, 1024), sdesc_sw128(addr, 16, 1024), id, k > 0);
-                    }
-                    mma_commit(bar_gp);
-                });
-            }
+            named_sync(BAR_PCTL, NPC);  // H1: the control warp issues [G; P] = [K; Q] K^T
             PHASE(10);
             if (p < 32) {  // inclusive scan of the gate over the chunk (warp 8)
                 float x0 = vGam[2 * p], x1 = vGam[2 * p + 1];
@@ -445,6 +485,10 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 vEG[p] = __expf(gt);
                 vTail[p] = __expf(gl - gt) * vRk[p];
                 vCw[p] = vBeta[p] * __expf(gt) * vRk[p];
+                const float g2 = gt * 1.4426950408889634f;
+                vec[V_G2 * 64 + p] = g2;
+                // padding rows have 1/|k| = 0, so their lambda is +inf and their entries vanish
+                vec[V_LAM * 64 + p] = g2 - lg2_approx(vRk[p]);
                 if (p == 0) vec[V_N * 64] = (float)n;
             }
             named_sync(BAR_PREP, NGRP);
@@ -463,24 +507,29 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 float v[32];
                 const uint32_t ta = tmem + TM_GPW + lane_base + 32 * hf;
                 tmem_ld32(ta, v);
+                const int t = row & 63;
+                const float g2t = vec[V_G2 * 64 + t];
+                // row factor: beta_t / |k_t| for A, scale / |q_t| for Pm (zero past the length)
+                const float rf = t < n ? (q4 < 2 ? vBeta[t] * vRk[t] : vRq[t]) : 0.f;
+                const float4 *lam4 = reinterpret_cast<const float4 *>(vec + V_LAM * 64 + 32 * hf);
                 tmem_ld_wait();
                 PHASE(12);
-                const int t = row & 63;
-                const float gt = vGam[t];
+#pragma unroll
+                for (int j4 = 0; j4 < 8; ++j4) {
+                    const float4 l = lam4[j4];
+                    v[4 * j4 + 0] *= rf * ex2_approx(g2t - l.x);
+                    v[4 * j4 + 1] *= rf * ex2_approx(g2t - l.y);
+                    v[4 * j4 + 2] *= rf * ex2_approx(g2t - l.z);
+                    v[4 * j4 + 3] *= rf * ex2_approx(g2t - l.w);
+                }
                 if (q4 < 2) {
-                    const float rb = t < n ? vBeta[t] * vRk[t] : 0.f;
+                    // entries on or above the diagonal are never read by the solve
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) {
-                        const int s = 32 * hf + j;
-                        sA[t * FA + s] = s < t ? rb * vRk[s] * v[j] * __expf(gt - vGam[s]) : 0.f;
-                    }
+                    for (int j4 = 0; j4 < 8; ++j4)
+                        *reinterpret_cast<float4 *>(sA + t * FA + 32 * hf + 4 * j4) =
+                            make_float4(v[4 * j4], v[4 * j4 + 1], v[4 * j4 + 2], v[4 * j4 + 3]);
                 } else {
-                    const float rq = t < n ? vRq[t] : 0.f;
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) {
-                        const int s = 32 * hf + j;
-                        v[j] = s <= t ? rq * vRk[s] * v[j] * __expf(gt - vGam[s]) : 0.f;
-                    }
+                    // entries above the diagonal are masked when Pm is converted to bf16
                     tmem_st32(ta, v);
                     tmem_st_wait();
                 }
@@ -489,7 +538,9 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             if (lane == 0) s_phase_[32 + warp - 8] += clock64() - tb0_;
 #endif
             tc_fence_before();
-            if (named_sync_or(BAR_PREP, NGRP, to)) break;
+            // a timed-out wait is carried to the next hand-off barrier, where the control warp
+            // learns of it too
+            named_sync(BAR_PREP, NGRP);
             PHASE(3);
             // ---- a3: T = (I + A)^{-1} and the bf16 operand [T diag(beta); T diag(c_W)] ----
             solve_unit_lower(sA, sT, sX, p SOLVE_TIMER_PASS);
@@ -523,22 +574,10 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             }
             fence_proxy_async_smem();
             tc_fence_before();
-            if (named_sync_or(BAR_PREP, NGRP, to)) break;
+            // H2: the control warp issues W and U (rows 64..127 of TT K, rows 0..63 of TT V)
+            if (named_sync_or(BAR_PCTL, NPC, to)) break;
             tc_fence_after();
             PHASE(7);
-            // ---- a4: W (rows 64..127 of TT K) and U (rows 0..63 of TT V) ----
-            if (issuer) {
-                const uint32_t id = idesc_bf16(128, 128, false, true);
-                TIMED(22, {
-                    _Pragma("unroll")
-                    for (int k = 0; k < 4; ++k) {
-                        const uint64_t ad = sdesc_sw128(sbase + OFF_TT + k * 32, 16, 1024);
-                        mma_bf16(tmem + TM_GPW, ad, sdesc_sw128(sbase + OFF_K0 + k * 2048, 16384, 1024), id, k > 0);
-                        mma_bf16(tmem + TM_U, ad, sdesc_sw128(sbase + OFF_V0 + k * 2048, 8192, 1024), id, k > 0);
-                    }
-                    mma_commit(bar_wu);
-                });
-            }
             // meanwhile: X_g rows (64..127 of A1) and K~ from the staged q/k tiles
             for (int e = p; e < 2 * 64 * 16; e += NGRP) {
                 const int isk = e >> 10, r = (e >> 4) & 63, blk = (e >> 3) & 1, ch = e & 7;
@@ -560,9 +599,8 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             }
             wait_ok(bar_wu, par);
             tc_fence_after();
-            if (named_sync_or(BAR_PREP, NGRP, to)) break;  // staged tiles fully consumed
+            if (named_sync_or(BAR_PCTL, NPC, to)) break;  // H3: staged tiles fully consumed
             PHASE(8);
-            if (loader && c + 1 < nvalid) issue_loads(c + 1);
             if (q4 >= 2) {  // W rows -> rows 0..63 of A1
                 const int t = row - 64;
 #pragma unroll
@@ -592,7 +630,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         };
         for (int c = 0; c < nvalid; ++c) {
             const uint32_t par = c & 1;
-            const float *vec = vecs + (c & 1) * 8 * 64;
+            const float *vec = vecs + (c & 1) * NVEC * 64;
             if (!mbar_wait_sleep(bar_a1, par)) to = true;
             if (named_sync_or(BAR_CARRY, NGRP, to)) { stop = true; break; }
             tc_fence_after();
