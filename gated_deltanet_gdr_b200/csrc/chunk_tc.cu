@@ -79,41 +79,50 @@ constexpr int C = 64, D = 128, NGRP = 256, NT = 2 * NGRP + 32, NPC = NGRP + 32;
 constexpr int CTL_WARP = 16;
 // BAR_PCTL: the prep warps and the control warp, at the hand-offs between them
 constexpr int BAR_CARRY = 1, BAR_PREP = 2, BAR_PCTL = 3;
+// BAR_SOLVE: prep warps 8 and 9, which move the merge products of the solve between TMEM and shared memory
+constexpr int BAR_SOLVE = 4;
 constexpr uint32_t kTimeoutBit = 0x4u;
 // carry thread that issues the out-tile TMA stores (thread 0 issues the carry's MMAs)
 constexpr int kStorer = 32;
 
 // ---- shared memory map (bytes from a 1024-aligned base) ----
-// input stage: [K_b0 | Q_b0 | K_b1 | Q_b1 | V_b0 | V_b1], each 64 rows x 128 B (64 bf16)
+// input stage of the prep group: [K_b0 | Q_b0 | K_b1 | Q_b1 | V_b0 | V_b1], 64 rows x 128 B (64 bf16) each
 constexpr uint32_t OFF_K0 = 0, OFF_Q0 = 8192, OFF_K1 = 16384, OFF_Q1 = 24576, OFF_V0 = 32768;
 constexpr uint32_t STAGE_BYTES = 49152;
-constexpr uint32_t OFF_A1 = 49152;   // [W; X_g] K-major 128 x 128: dk blocks at +0, +16K
-constexpr uint32_t OFF_S = 81920;    // S bf16, MN-major (K = dk rows, N = dv): dv blocks at +0, +16K
-constexpr uint32_t OFF_KT = 114688;  // K~ MN-major (M = dk, K = tok): dk blocks at +0, +8K
-constexpr uint32_t OFF_PM = 131072;  // [0; Pm] K-major 128 x 64
-constexpr uint32_t OFF_VO = 147456;  // v_new (MN-major, K = tok, N = dv) then the out tile: dv blocks +0, +8K
-constexpr int FP = 68;               // row stride (floats) of T: 16-byte aligned rows for float4 access
-constexpr int FA = 68;               // row stride of A: each quarter-warp's 16-byte row stores hit distinct banks
-constexpr int XP = 36;               // row stride of the merge scratch
-constexpr uint32_t OFF_AF = 163840;  // A (fp32); after the solve it holds TT = [T diag(beta); T diag(c_W)]
+// operands of the carry group for the chunk it runs
+constexpr uint32_t OFF_A1 = 49152;   // [W; Q] K-major 128 x 128: dk blocks at +0, +16K (Q rows by TMA)
+constexpr uint32_t OFF_KT = 81920;   // raw K tile by TMA, MN-major (M = dk, K = tok): dk blocks at +0, +8K
+constexpr uint32_t OFF_S = 98304;    // S bf16, MN-major (K = dk rows, N = dv): dv blocks at +0, +16K
+constexpr uint32_t OFF_VS = 131072;  // diag(tail) v_new (MN-major, K = tok, N = dv): dv blocks at +0, +8K
+// Pm (K-major 64 x 64), two buffers; the o MMA reads 128 rows starting 8 KB before the buffer so that
+// Pm forms rows 64..127 (rows 0..63 are whatever precedes it and land in dead accumulator lanes)
+constexpr uint32_t OFF_PM0 = 147456, OFF_PM1 = 155648;
+constexpr uint32_t OFF_VO = 163840;  // v_new (MN-major, K = tok, N = dv), then the out tile: dv blocks +0, +8K
+// fp32 64 x 64 matrices of the solve, A and T, in the layout of f32_off() (tf32 MMA operands)
+constexpr uint32_t OFF_AF = 180224;  // A; once the solve has read it, TT = [T diag(beta); T diag(c_W)] (bf16)
 constexpr uint32_t OFF_TT = OFF_AF;
-constexpr uint32_t OFF_TF = OFF_AF + 64 * FA * 4;  // T (fp32)
-constexpr uint32_t OFF_X = OFF_TF + 64 * FP * 4;
-constexpr int NVEC = 10;             // per-chunk vectors of 64 floats (enum below)
-constexpr uint32_t OFF_VEC = OFF_X + 32 * XP * 4;  // 2 sets x NVEC vectors x 64 floats
+constexpr uint32_t OFF_TF = OFF_AF + 16384;  // T
+constexpr uint32_t OFF_XB = OFF_TF + 16384;  // X = A21 T11 of the merges (fp32, b32_off layout, 32 rows)
+// the blocks of T the merges read as their MN-major operand, in the b32_off layout: T(0:32, 0:32) at +0,
+// T(32:48, 32:48) at +4 KB
+constexpr uint32_t OFF_TB = OFF_XB + 4096;
+constexpr int NVEC = 12;             // per-chunk vectors of 64 floats (enum below)
+constexpr uint32_t OFF_VEC = OFF_TB + 6144;  // 2 sets x NVEC vectors x 64 floats
 constexpr uint32_t OFF_BAR = OFF_VEC + 2 * NVEC * 64 * 4;
 constexpr uint32_t SMEM_USED = OFF_BAR + 128;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;  // + alignment slack
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
-static_assert(OFF_TF % 16 == 0 && OFF_X % 16 == 0, "float4 alignment");
-static_assert(OFF_TF >= OFF_TT + 16384, "TT must fit inside the A matrix area");
+static_assert(OFF_AF % 1024 == 0 && OFF_TF % 1024 == 0 && OFF_XB % 1024 == 0 && OFF_TB % 1024 == 0, "swizzle atoms");
+static_assert(OFF_PM0 >= 8192 && OFF_PM1 == OFF_PM0 + 8192, "Pm buffers");
 
-// TMEM columns (all 128 lanes): [G;P] then W, U, R = [W S; o], the fp32 state S
+// TMEM columns (all 128 lanes): the Gram [K; Q][K; Q]^T then W (lanes 64..127), U (lanes 0..63),
+// R = [W S; o] (lanes 0..63 / 64..127), the fp32 state S
 constexpr uint32_t TM_GPW = 0, TM_U = 128, TM_R = 256, TM_S = 384, TM_COLS = 512;
 
 // V_G2 = G log2(e); V_LAM = V_G2 - log2(1/|k|), so that e^{G_t - G_s} / |k_s| = 2^{V_G2[t] - V_LAM[s]};
-// V_N holds the chunk's valid-token count in its first entry.
-enum { V_BETA = 0, V_GAM, V_EG, V_TAIL, V_RK, V_RQ, V_CW, V_G2, V_LAM, V_N };
+// V_XS = e^G scale / |q| (row factor of Q S); V_N holds the chunk's valid-token count in its first entry.
+// V_ET = e^{G_last - G}; V_TAIL = V_ET / |k|.
+enum { V_BETA = 0, V_GAM, V_EG, V_TAIL, V_RK, V_RQ, V_CW, V_G2, V_LAM, V_XS, V_ET, V_N };
 static_assert(V_N < NVEC, "vector slots");
 
 struct TcArgs {
@@ -161,89 +170,56 @@ __device__ __forceinline__ uint4 pack8(const float *f) {
                       pack_bf16x2(f[6], f[7]));
 }
 
-// T = (I + A)^{-1} for a strictly lower 64 x 64 A (fp32, row stride FA; T row stride FP), by the 256 prep
-// threads (p = 0..255).  Writes the lower triangle of T and zeros in the upper 16 x 16
-// blocks that the merges read.
-__device__ __forceinline__ void solve_unit_lower(const float *sA, float *sT, float *sX, int p SOLVE_TIMER_ARGS) {
-    if (p < 64) {  // 16 x 16 diagonal blocks, one column per thread
+// Byte offset of element (r, s) of a 64 x 64 fp32 matrix stored as two column blocks (s < 32 at +0,
+// s >= 32 at +8 KB), each 64 rows of 128 bytes in the 128-byte-swizzled canonical layout (16-byte chunk
+// index XOR r % 8), so that kind::tf32 MMAs read row blocks as K-major and column blocks as MN-major operands.
+__device__ __forceinline__ uint32_t f32_off(int r, int s) {
+    return (uint32_t)((s >> 5) * 8192 + (r >> 3) * 1024 + (r & 7) * 128 + ((((s >> 2) & 7) ^ (r & 7)) << 4) +
+                      (s & 3) * 4);
+}
+
+// Byte offset of element (k, n) (K-row k, column n < 32) of an MN-major kind::tf32 operand in the layout
+// that tcgen05 requires for it: rows of 128 bytes, 4-row groups of 512 bytes, 32-byte granules XORed with
+// k % 4 (descriptor layout type 1, sdesc_sw128_32b with sbo = 512).
+__device__ __forceinline__ uint32_t b32_off(int k, int n) {
+    return (uint32_t)((k >> 2) * 512 + (k & 3) * 128 + ((((n >> 3) ^ (k & 3))) << 5) + (n & 7) * 4);
+}
+
+// First step of T = (I + A)^{-1} (A strictly lower, 64 x 64, fp32 in the f32_off layout), by the 256 prep
+// threads p = 0..255: the four 16 x 16 diagonal blocks of T by forward substitution (one column per thread,
+// the whole column written, zeros above the diagonal), and zeros in the upper 16 x 16 blocks of the two
+// 32 x 32 diagonal blocks, which the tensor-core merges read.
+__device__ __forceinline__ void solve_diag16(const uint8_t *sA, uint8_t *sT, uint8_t *sTB, int p) {
+    if (p < 64) {
         const int base = (p >> 4) * 16, j = p & 15;
         float x[16];
 #pragma unroll
         for (int t = 0; t < 16; ++t) x[t] = (t == j) ? 1.f : 0.f;
 #pragma unroll
         for (int t = 1; t < 16; ++t) {
-            const float *ar = sA + (base + t) * FA + base;
             float a0 = 0.f, a1 = 0.f;
 #pragma unroll
             for (int s = 0; s < t; ++s) {
-                if (s & 1) a1 = fmaf(ar[s], x[s], a1);
-                else a0 = fmaf(ar[s], x[s], a0);
+                const float as = *reinterpret_cast<const float *>(sA + f32_off(base + t, base + s));
+                if (s & 1) a1 = fmaf(as, x[s], a1);
+                else a0 = fmaf(as, x[s], a0);
             }
             if (t > j) x[t] = -(a0 + a1);
         }
 #pragma unroll
-        for (int t = 0; t < 16; ++t) sT[(base + t) * FP + base + j] = x[t];
-    } else {  // zero the upper 16 x 16 blocks inside the two 32 x 32 diagonal blocks
-        for (int e = p - 64; e < 512; e += NGRP - 64) {
-            const int blk = e >> 8, r = (e >> 4) & 15, c = e & 15;
-            sT[(32 * blk + r) * FP + 32 * blk + 16 + c] = 0.f;
+        for (int t = 0; t < 16; ++t) *reinterpret_cast<float *>(sT + f32_off(base + t, base + j)) = x[t];
+        // blocks 0, 1 (T11) and 2 are also MN-major operands of the merges
+        if (base < 48) {
+            uint8_t *tb = sTB + (base >= 32 ? 4096 : 0);
+            const int b0 = base & 31;
+#pragma unroll
+            for (int t = 0; t < 16; ++t) *reinterpret_cast<float *>(tb + b32_off(b0 + t, b0 + j)) = x[t];
         }
+    } else if (p < 192) {
+        const int e = p - 64, blk = e >> 6, r = (e >> 2) & 15, c4 = (e & 3) * 4;
+        *reinterpret_cast<float4 *>(sT + f32_off(32 * blk + r, 32 * blk + 16 + c4)) = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (blk == 0) *reinterpret_cast<float4 *>(sTB + b32_off(r, 16 + c4)) = make_float4(0.f, 0.f, 0.f, 0.f);
     }
-    named_sync(BAR_PREP, NGRP);
-    PHASE(13);
-    // 16 -> 32: X_b = A21 T11, then T21 = -T22 X_b, for the blocks at rows 32b+16, cols 32b
-    {
-        const int blk = p >> 7, r = (p >> 3) & 15, c2 = (p & 7) * 2, r0 = 32 * blk + 16, c0 = 32 * blk;
-        float x0 = 0.f, x1 = 0.f;
-#pragma unroll
-        for (int k = 0; k < 16; ++k) {
-            const float a = sA[(r0 + r) * FA + c0 + k];
-            const float2 t = *reinterpret_cast<const float2 *>(sT + (c0 + k) * FP + c0 + c2);
-            x0 = fmaf(a, t.x, x0);
-            x1 = fmaf(a, t.y, x1);
-        }
-        *reinterpret_cast<float2 *>(sX + (blk * 16 + r) * XP + c2) = make_float2(x0, x1);
-        named_sync(BAR_PREP, NGRP);
-        float y0 = 0.f, y1 = 0.f;
-#pragma unroll
-        for (int k = 0; k < 16; ++k) {
-            const float t = sT[(r0 + r) * FP + r0 + k];
-            const float2 xx = *reinterpret_cast<const float2 *>(sX + (blk * 16 + k) * XP + c2);
-            y0 = fmaf(t, xx.x, y0);
-            y1 = fmaf(t, xx.y, y1);
-        }
-        *reinterpret_cast<float2 *>(sT + (r0 + r) * FP + c0 + c2) = make_float2(-y0, -y1);
-    }
-    named_sync(BAR_PREP, NGRP);
-    PHASE(14);
-    // 32 -> 64: X = A21 T11, T21 = -T22 X with 32 x 32 blocks; one row x 4 columns per thread
-    {
-        const int r = p >> 3, c4 = (p & 7) * 4;
-        float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-        for (int k = 0; k < 32; ++k) {
-            const float a = sA[(32 + r) * FA + k];
-            const float4 t = *reinterpret_cast<const float4 *>(sT + k * FP + c4);
-            x.x = fmaf(a, t.x, x.x);
-            x.y = fmaf(a, t.y, x.y);
-            x.z = fmaf(a, t.z, x.z);
-            x.w = fmaf(a, t.w, x.w);
-        }
-        *reinterpret_cast<float4 *>(sX + r * XP + c4) = x;
-        named_sync(BAR_PREP, NGRP);
-        float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-        for (int k = 0; k < 32; ++k) {
-            const float t = sT[(32 + r) * FP + 32 + k];
-            const float4 xx = *reinterpret_cast<const float4 *>(sX + k * XP + c4);
-            y.x = fmaf(t, xx.x, y.x);
-            y.y = fmaf(t, xx.y, y.y);
-            y.z = fmaf(t, xx.z, y.z);
-            y.w = fmaf(t, xx.w, y.w);
-        }
-        *reinterpret_cast<float4 *>(sT + (32 + r) * FP + c4) = make_float4(-y.x, -y.y, -y.z, -y.w);
-    }
-    named_sync(BAR_PREP, NGRP);
 }
 
 __global__ void __launch_bounds__(NT, 1)
@@ -255,13 +231,17 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     uint8_t *sm = smraw + ((1024u - (smem_u32(smraw) & 1023u)) & 1023u);
     const uint32_t sbase = smem_u32(sm);
     float *vecs = reinterpret_cast<float *>(sm + OFF_VEC);
-    uint64_t *bar_ld = reinterpret_cast<uint64_t *>(sm + OFF_BAR);
-    uint64_t *bar_gp = bar_ld + 1, *bar_wu = bar_ld + 2, *bar_m1 = bar_ld + 3, *bar_m2 = bar_ld + 4;
-    uint64_t *bar_a1 = bar_ld + 5;
-    uint32_t *s_tmem = reinterpret_cast<uint32_t *>(bar_ld + 8);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + OFF_BAR);
+    // bar_ld: input stage landed; bar_gp / bar_wu: the prep MMAs completed; bar_m1 / bar_m2: the carry MMAs
+    // completed; bar_a1: the prep group handed chunk c to the carry group; bar_cq / bar_ck: the raw Q rows
+    // of A1 / the raw K tile landed; bar_pf[i]: the carry group is done with Pm buffer i and vector set i
+    uint64_t *bar_ld = bars, *bar_gp = bars + 1, *bar_wu = bars + 2, *bar_m1 = bars + 3, *bar_m2 = bars + 4;
+    uint64_t *bar_a1 = bars + 5, *bar_cq = bars + 6, *bar_ck = bars + 7, *bar_pf = bars + 8;
+    // the tensor-core merges of the solve: rounds 0..2 on bar_sv (three phases per chunk), round 3 on bar_sv3
+    uint64_t *bar_sv = bars + 10, *bar_sv3 = bars + 11;
+    constexpr int kNumBars = 12;
+    uint32_t *s_tmem = reinterpret_cast<uint32_t *>(bars + kNumBars);
     volatile int *s_abort = reinterpret_cast<volatile int *>(s_tmem + 1);
-    float *sA = reinterpret_cast<float *>(sm + OFF_AF), *sT = reinterpret_cast<float *>(sm + OFF_TF);
-    float *sX = reinterpret_cast<float *>(sm + OFF_X);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, q4 = warp & 3, hf = (warp >> 2) & 1;
     const bool carry = warp < 8, control = warp == CTL_WARP;
@@ -275,18 +255,33 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const uint32_t lane_base = (uint32_t)(q4 * 32) << 16;
     const int row = q4 * 32 + lane;  // TMEM lane of this thread
 
+    // raw Q rows of A1 and the raw K tile of chunk c, for the carry group (issued by carry thread 0)
+    auto load_carry_q = [&](int chunk) {
+        mbar_arrive_expect_tx(bar_cq, 16384);
+        tma_load_3d(sm + OFF_A1 + 8192, &tm_q, bar_cq, 0, chunk * C, zq);
+        tma_load_3d(sm + OFF_A1 + 16384 + 8192, &tm_q, bar_cq, 64, chunk * C, zq);
+    };
+    auto load_carry_k = [&](int chunk) {
+        mbar_arrive_expect_tx(bar_ck, 16384);
+        tma_load_3d(sm + OFF_KT, &tm_k, bar_ck, 0, chunk * C, zq);
+        tma_load_3d(sm + OFF_KT + 8192, &tm_k, bar_ck, 64, chunk * C, zq);
+    };
+
     if (tid == 0) {
         if (bad_len) raise_device_error(a.err, GDR_DEVERR_LENGTH);
-        for (int i = 0; i < 6; ++i) mbar_init(bar_ld + i, 1);
+        for (int i = 0; i < kNumBars; ++i) mbar_init(bars + i, 1);
         *s_abort = 0;
         fence_mbar_init();
         prefetch_tmap(&tm_q);
         prefetch_tmap(&tm_k);
         prefetch_tmap(&tm_v);
         prefetch_tmap(&tm_o);
+        if (nvalid > 0) {
+            load_carry_q(0);
+            load_carry_k(0);
+        }
     }
     if (warp == 0) tmem_alloc(s_tmem, TM_COLS);
-    for (int e = tid; e < 8192 / 16; e += NT) reinterpret_cast<uint4 *>(sm + OFF_PM)[e] = make_uint4(0, 0, 0, 0);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -330,11 +325,11 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 #endif
     if (control) {
         // ============================== control warp ==============================
-        // Lane 0 issues the prep MMAs and nothing else, lane 1 the TMA loads and L2 prefetches
-        // (an MMA issued by a thread with copies of its own outstanding was seen to wait for
-        // them).  Having a warp of its own, neither blocks a prep warp while the tensor pipe is
-        // busy.  The warp follows the prep group's hand-off barriers (BAR_PCTL) and leaves
-        // at the same barrier as the prep group when a wait timed out.
+        // Lane 0 issues the prep MMAs and nothing else, lane 1 the input-stage TMA loads and L2
+        // prefetches (an MMA issued by a thread with copies of its own outstanding was seen to wait
+        // for them).  Having a warp of its own, neither blocks a prep warp while the tensor pipe is
+        // busy.  The warp follows the prep group's hand-off barriers (BAR_PCTL) and leaves at the
+        // same barrier as the prep group when a wait timed out.
         auto prefetch_l2 = [&](int chunk) {
             const int y = chunk * C;
             tma_prefetch_3d(&tm_k, 0, y, zq);
@@ -354,17 +349,63 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             tma_load_3d(sm + OFF_V0, &tm_v, bar_ld, 0, y, bh);
             tma_load_3d(sm + OFF_V0 + 8192, &tm_v, bar_ld, 64, y, bh);
         };
+        // The gate and beta vectors of a chunk, which need no Gram: beta (from logits), the cumulative
+        // gate G (from the raw gate), e^G, G log2(e), e^{G_last - G} and the valid-token count; two
+        // tokens per lane, the scan over the chunk by warp shuffles.
+        const float gA = (a.A_log && a.g) ? a.A_log[h] : 0.f, gB = (a.A_log && a.g) ? a.dt_bias[h] : 0.f;
+        const __nv_bfloat16 *bg = reinterpret_cast<const __nv_bfloat16 *>(a.beta) + (size_t)bh * S;
+        const float *gg = a.g ? a.g + (size_t)bh * S : nullptr;
+        auto chunk_vectors = [&](int chunk) {
+            float *vec = vecs + (chunk & 1) * NVEC * 64;
+            const int n = min(C, L - chunk * C);
+            float bv[2], gv[2];
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+                const int tt = 2 * lane + i, t = chunk * C + tt;
+                float rb = 0.f, rg = 0.f;
+                if (tt < n) {
+                    rb = __bfloat162float(bg[t]);
+                    if (gg) rg = gg[t];
+                }
+                bv[i] = tt < n ? (a.beta_logits ? sigmoid_f32(rb) : rb) : 0.f;
+                gv[i] = tt < n ? (a.A_log ? gate_from_raw(rg, gA, gB) : rg) : 0.f;
+            }
+            const float x1 = gv[0] + gv[1];
+            float sc = x1;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const float y = __shfl_up_sync(0xffffffffu, sc, o);
+                if (lane >= o) sc += y;
+            }
+            const float gl = __shfl_sync(0xffffffffu, sc, 31);
+            const float G[2] = {sc - x1 + gv[0], sc};
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+                const int tt = 2 * lane + i;
+                vec[V_BETA * 64 + tt] = bv[i];
+                vec[V_GAM * 64 + tt] = G[i];
+                vec[V_EG * 64 + tt] = __expf(G[i]);
+                vec[V_G2 * 64 + tt] = G[i] * 1.4426950408889634f;
+                vec[V_ET * 64 + tt] = __expf(gl - G[i]);
+            }
+            if (lane == 0) vec[V_N * 64] = (float)n;
+        };
+        bool to = false;
+        if (nvalid > 0) chunk_vectors(0);
         if (lane == 1 && nvalid > 0) {
             issue_loads(0);
             if (nvalid > 1) prefetch_l2(1);
         }
+        __syncwarp();
         for (int c = 0; c < nvalid; ++c) {
-            if (named_sync_or(BAR_PCTL, NPC, false)) break;  // H0: chunk c staged (or a timeout)
+            const uint32_t par = c & 1;
+            if (named_sync_or(BAR_PCTL, NPC, to)) break;  // H0: chunk c staged (or a timeout)
             if (lane == 1 && c + 2 < nvalid) prefetch_l2(c + 2);
+            __syncwarp();
             named_sync(BAR_PCTL, NPC);  // H1: padding rows zeroed
-            if (lane == 0) {  // a2: [G; P] = [K; Q] K^T
+            if (lane == 0) {  // a2: the Gram [K; Q][K; Q]^T (its diagonal gives the row norms)
                 tc_fence_after();
-                const uint32_t id = idesc_bf16(128, 64, false, false);
+                const uint32_t id = idesc_bf16(128, 128, false, false);
 #pragma unroll
                 for (int k = 0; k < 8; ++k) {
                     const uint32_t addr = sbase + OFF_K0 + (k >> 2) * 16384 + (k & 3) * 32;
@@ -372,7 +413,15 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 }
                 mma_commit(bar_gp);
             }
-            if (named_sync_or(BAR_PCTL, NPC, false)) break;  // H2: TT operand and Pm in place
+            __syncwarp();
+            // while the prep group solves chunk c: the vectors of chunk c+1, into the set that chunk c-1
+            // used (free once the carry's MMA2 of chunk c-1 completed)
+            if (c + 1 < nvalid) {
+                if (c >= 1 && !mbar_wait_sleep(bar_pf + ((c + 1) & 1), ((c - 1) >> 1) & 1)) to = true;
+                chunk_vectors(c + 1);
+            }
+            __syncwarp();
+            if (named_sync_or(BAR_PCTL, NPC, to)) break;  // H2: TT operand in place, TMEM U free
             if (lane == 0) {  // a4: W (rows 64..127 of TT K) and U (rows 0..63 of TT V)
                 tc_fence_after();
                 const uint32_t id = idesc_bf16(128, 128, false, true);
@@ -384,44 +433,30 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 }
                 mma_commit(bar_wu);
             }
-            if (named_sync_or(BAR_PCTL, NPC, false)) break;  // H3: staged tiles fully consumed
-            if (lane == 1 && c + 1 < nvalid) issue_loads(c + 1);
+            if (lane == 1 && c + 1 < nvalid) {  // the stage is consumed once W and U are done
+                if (mbar_wait(bar_wu, par)) issue_loads(c + 1);
+                else to = true;
+            }
+            __syncwarp();
         }
     } else if (!carry) {
         // =============================== prep group ===============================
         const int p = tid - NGRP;
-        const float gA = (a.A_log && a.g) ? a.A_log[h] : 0.f, gB = (a.A_log && a.g) ? a.dt_bias[h] : 0.f;
-        const __nv_bfloat16 *bg = reinterpret_cast<const __nv_bfloat16 *>(a.beta) + (size_t)bh * S;
-        const float *gg = a.g ? a.g + (size_t)bh * S : nullptr;
-        float nb = 0.f, ng = 0.f;  // prefetched raw beta / gate of the next chunk (threads p < 64)
-        auto fetch = [&](int chunk) {
-            nb = 0.f;
-            ng = 0.f;
-            const int t = chunk * C + p;
-            if (p < C && chunk < nvalid && t < L) {
-                nb = __bfloat162float(bg[t]);
-                if (gg) ng = gg[t];
-            }
-        };
         bool to = false;  // a wait of this thread timed out
         auto wait_ok = [&](uint64_t *bar, uint32_t parity) {
             if (!mbar_wait(bar, parity)) to = true;
         };
-        fetch(0);
         for (int c = 0; c < nvalid; ++c) {
             const uint32_t par = c & 1;
-            float *vec = vecs + (c & 1) * NVEC * 64;
-            float *vBeta = vec + V_BETA * 64, *vGam = vec + V_GAM * 64, *vEG = vec + V_EG * 64;
-            float *vTail = vec + V_TAIL * 64, *vRk = vec + V_RK * 64, *vRq = vec + V_RQ * 64, *vCw = vec + V_CW * 64;
+            float *vec = vecs + par * NVEC * 64;
+            float *vBeta = vec + V_BETA * 64, *vEG = vec + V_EG * 64;
+            float *vRk = vec + V_RK * 64, *vRq = vec + V_RQ * 64, *vCw = vec + V_CW * 64;
+            uint8_t *pm = sm + (par ? OFF_PM1 : OFF_PM0);
             const int n = min(C, L - c * C);
-            if (p < C) {
-                const bool valid = p < n;
-                vBeta[p] = valid ? (a.beta_logits ? sigmoid_f32(nb) : nb) : 0.f;
-                vGam[p] = valid ? (a.A_log ? gate_from_raw(ng, gA, gB) : ng) : 0.f;
-            }
-            fetch(c + 1);
+            // Pm buffer `par` and the norm vectors of set `par` were last read for chunk c-2, before its MMA2
+            if (c >= 2 && !mbar_wait_sleep(bar_pf + par, ((c >> 1) + 1) & 1)) to = true;
             wait_ok(bar_ld, par);
-            if (named_sync_or(BAR_PCTL, NPC, to)) break;  // H0
+            if (named_sync_or(BAR_PCTL, NPC, to)) break;  // H0 (the vectors of chunk c were written before H2 of c-1)
             PHASE(0);
             if (n < C) {  // padding rows of the last chunk: zero them so no padding value reaches a product
                 for (int e = p; e < (C - n) * 48; e += NGRP) {
@@ -430,195 +465,271 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 }
                 fence_proxy_async_smem();
             }
-            named_sync(BAR_PCTL, NPC);  // H1: the control warp issues [G; P] = [K; Q] K^T
-            PHASE(10);
-            if (p < 32) {  // inclusive scan of the gate over the chunk (warp 8)
-                float x0 = vGam[2 * p], x1 = vGam[2 * p + 1];
-                x1 += x0;
-                float s = x1;
-#pragma unroll
-                for (int o = 1; o < 32; o <<= 1) {
-                    const float y = __shfl_up_sync(0xffffffffu, s, o);
-                    if (p >= o) s += y;
-                }
-                const float excl = s - x1;
-                vGam[2 * p] = excl + x0;
-                vGam[2 * p + 1] = excl + x1;
-            }
-#ifdef GDR_PHASE_TIMERS
-            const unsigned long long tn0_ = clock64();
-#endif
-            {  // row norms of k and q: 4 threads per row, 32 elements each
-                const int r = p >> 2, part = p & 3;
-                const uint32_t off = (part >> 1) * 16384 + r * 128 + (part & 1) * 64;
-                float sk = 0.f, sq = 0.f;
-#pragma unroll
-                for (int ch = 0; ch < 4; ++ch) {
-                    // the order of the row's chunks does not matter for the sum; rotating it by
-                    // the row spreads the warp's 8 rows over all banks
-                    const uint32_t o = off + ((ch + r) & 3) * 16;
-                    float fk[8], fq[8];
-                    unpack8(*reinterpret_cast<const uint4 *>(sm + OFF_K0 + o), fk);
-                    unpack8(*reinterpret_cast<const uint4 *>(sm + OFF_Q0 + o), fq);
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        sk = fmaf(fk[i], fk[i], sk);
-                        sq = fmaf(fq[i], fq[i], sq);
-                    }
-                }
-                sk += __shfl_xor_sync(0xffffffffu, sk, 1);
-                sq += __shfl_xor_sync(0xffffffffu, sq, 1);
-                sk += __shfl_xor_sync(0xffffffffu, sk, 2);
-                sq += __shfl_xor_sync(0xffffffffu, sq, 2);
-                if (part == 0) {
-                    vRk[r] = r < n ? (a.l2norm ? rsqrtf(sk + a.eps) : 1.f) : 0.f;
-                    vRq[r] = r < n ? a.scale * (a.l2norm ? rsqrtf(sq + a.eps) : 1.f) : 0.f;
-                }
-            }
-#ifdef GDR_PHASE_TIMERS
-            if (lane == 0) s_phase_[40 + warp - 8] += clock64() - tn0_;
-#endif
-            named_sync(BAR_PREP, NGRP);
-            PHASE(11);
-            if (p < C) {
-                const float gl = vGam[C - 1], gt = vGam[p];
-                vEG[p] = __expf(gt);
-                vTail[p] = __expf(gl - gt) * vRk[p];
-                vCw[p] = vBeta[p] * __expf(gt) * vRk[p];
-                const float g2 = gt * 1.4426950408889634f;
-                vec[V_G2 * 64 + p] = g2;
-                // padding rows have 1/|k| = 0, so their lambda is +inf and their entries vanish
-                vec[V_LAM * 64 + p] = g2 - lg2_approx(vRk[p]);
-                if (p == 0) vec[V_N * 64] = (float)n;
-            }
-            named_sync(BAR_PREP, NGRP);
+            named_sync(BAR_PCTL, NPC);  // H1: the control warp issues the Gram
             PHASE(1);
             wait_ok(bar_gp, par);
             tc_fence_after();
-            PHASE(2);
-            // A rows (from G, lanes 0..63) and Pm rows (from P, lanes 64..127; parked in TMEM as
-            // fp32), with the decay e^{G_t - G_s} taken per entry.  Columns s > t are never read
-            // (the solve reads the strict lower triangle, the Pm conversion masks), so the warps
-            // whose 32 x 32 block lies wholly above the diagonal skip it.
-#ifdef GDR_PHASE_TIMERS
-            const unsigned long long tb0_ = clock64();
-#endif
-            if (!((q4 & 1) == 0 && hf == 1)) {
-                float v[32];
-                const uint32_t ta = tmem + TM_GPW + lane_base + 32 * hf;
-                tmem_ld32(ta, v);
-                const int t = row & 63;
-                const float g2t = vec[V_G2 * 64 + t];
-                // row factor: beta_t / |k_t| for A, scale / |q_t| for Pm (zero past the length)
-                const float rf = t < n ? (q4 < 2 ? vBeta[t] * vRk[t] : vRq[t]) : 0.f;
-                const float4 *lam4 = reinterpret_cast<const float4 *>(vec + V_LAM * 64 + 32 * hf);
-                tmem_ld_wait();
-                PHASE(12);
-#pragma unroll
-                for (int j4 = 0; j4 < 8; ++j4) {
-                    const float4 l = lam4[j4];
-                    v[4 * j4 + 0] *= rf * ex2_approx(g2t - l.x);
-                    v[4 * j4 + 1] *= rf * ex2_approx(g2t - l.y);
-                    v[4 * j4 + 2] *= rf * ex2_approx(g2t - l.z);
-                    v[4 * j4 + 3] *= rf * ex2_approx(g2t - l.w);
-                }
-                if (q4 < 2) {
-                    // entries on or above the diagonal are never read by the solve
-#pragma unroll
-                    for (int j4 = 0; j4 < 8; ++j4)
-                        *reinterpret_cast<float4 *>(sA + t * FA + 32 * hf + 4 * j4) =
-                            make_float4(v[4 * j4], v[4 * j4 + 1], v[4 * j4 + 2], v[4 * j4 + 3]);
-                } else {
-                    // entries above the diagonal are masked when Pm is converted to bf16
-                    tmem_st32(ta, v);
-                    tmem_st_wait();
-                }
-            }
-#ifdef GDR_PHASE_TIMERS
-            if (lane == 0) s_phase_[32 + warp - 8] += clock64() - tb0_;
-#endif
-            tc_fence_before();
-            // a timed-out wait is carried to the next hand-off barrier, where the control warp
-            // learns of it too
-            named_sync(BAR_PREP, NGRP);
             PHASE(3);
-            // ---- a3: T = (I + A)^{-1} and the bf16 operand [T diag(beta); T diag(c_W)] ----
-            solve_unit_lower(sA, sT, sX, p SOLVE_TIMER_PASS);
-            PHASE(4);
-            for (int e = p; e < 128 * 8; e += NGRP) {
-                const int R = e >> 3, j = e & 7, t = R & 63;
-                const float *scl = (R < 64 ? vBeta : vCw) + 8 * j;
-                const float4 t0 = *reinterpret_cast<const float4 *>(sT + t * FP + 8 * j);
-                const float4 t1 = *reinterpret_cast<const float4 *>(sT + t * FP + 8 * j + 4);
-                const float tv[8] = {t0.x, t0.y, t0.z, t0.w, t1.x, t1.y, t1.z, t1.w};
-                float f[8];
+            // Each thread takes its Gram row's 32 columns of [K; Q] K^T (lanes 0..63: k_t.k_s, lanes
+            // 64..127: q_t.k_s); the blocks wholly above the diagonal are never read.  The diagonal
+            // gives |k_t|^2 and (from the q_t.q_s columns) |q_t|^2.
+            const bool need = !((q4 & 1) == 0 && hf == 1);
+            if ((q4 < 2 && hf == q4) || (q4 >= 2 && hf == q4 - 2)) {
+                // |k_t|^2 at column t (lanes 0..63), |q_t|^2 at column 64 + t (lanes 64..127): the diagonal
+                // element of this thread's row is entry `lane` of the 32 columns its warp loads
+                float d32[32];
+                tmem_ld32(tmem + TM_GPW + lane_base + (q4 >= 2 ? 64 : 0) + 32 * hf, d32);
+                tmem_ld_wait();
+                float d = 0.f;
 #pragma unroll
-                for (int i = 0; i < 8; ++i) f[i] = (8 * j + i <= t) ? tv[i] * scl[i] : 0.f;
-                *reinterpret_cast<uint4 *>(sm + OFF_TT + blk_off(R, 8 * j)) = pack8(f);
+                for (int j = 0; j < 32; ++j) d = (j == lane) ? d32[j] : d;
+                const int t = row & 63;
+                const float r = t < n ? (a.l2norm ? rsqrtf(d + a.eps) : 1.f) : 0.f;
+                if (q4 < 2) {
+                    vRk[t] = r;
+                    vec[V_TAIL * 64 + t] = vec[V_ET * 64 + t] * r;
+                    vCw[t] = vBeta[t] * vEG[t] * r;
+                    // padding rows have 1/|k| = 0, so their lambda is +inf and their entries vanish
+                    vec[V_LAM * 64 + t] = vec[V_G2 * 64 + t] - lg2_approx(r);
+                } else {
+                    vRq[t] = a.scale * r;
+                    vec[V_XS * 64 + t] = vEG[t] * a.scale * r;
+                }
             }
+            named_sync(BAR_PREP, NGRP);
+            PHASE(4);
+            // A rows (lanes 0..63, fp32 for the solve) and Pm rows (lanes 64..127, bf16 operand of the
+            // carry's o MMA), with the decay e^{G_t - G_s} taken per entry
+            {
+                const int t = row & 63;
+                if (need) {
+                    float v[32];
+                    tmem_ld32(tmem + TM_GPW + lane_base + 32 * hf, v);
+                    const float g2t = vec[V_G2 * 64 + t];
+                    // row factor: beta_t / |k_t| for A, scale / |q_t| for Pm (zero past the length)
+                    const float rf = t < n ? (q4 < 2 ? vBeta[t] * vRk[t] : vRq[t]) : 0.f;
+                    const float4 *lam4 = reinterpret_cast<const float4 *>(vec + V_LAM * 64 + 32 * hf);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int j4 = 0; j4 < 8; ++j4) {
+                        const float4 l = lam4[j4];
+                        v[4 * j4 + 0] *= rf * ex2_approx(g2t - l.x);
+                        v[4 * j4 + 1] *= rf * ex2_approx(g2t - l.y);
+                        v[4 * j4 + 2] *= rf * ex2_approx(g2t - l.z);
+                        v[4 * j4 + 3] *= rf * ex2_approx(g2t - l.w);
+                    }
+                    if (q4 < 2) {
+                        // entries on or above the diagonal are never read by the solve
+#pragma unroll
+                        for (int j4 = 0; j4 < 8; ++j4)
+                            *reinterpret_cast<float4 *>(sm + OFF_AF + f32_off(t, 32 * hf + 4 * j4)) =
+                                make_float4(v[4 * j4], v[4 * j4 + 1], v[4 * j4 + 2], v[4 * j4 + 3]);
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) v[j] = (32 * hf + j <= t) ? v[j] : 0.f;
+#pragma unroll
+                        for (int c8 = 0; c8 < 4; ++c8)
+                            *reinterpret_cast<uint4 *>(pm + blk_off(t, 32 * hf + 8 * c8)) = pack8(&v[8 * c8]);
+                    }
+                } else if (q4 >= 2) {  // Pm rows 0..31, columns 32..63: above the diagonal
+#pragma unroll
+                    for (int c8 = 0; c8 < 4; ++c8)
+                        *reinterpret_cast<uint4 *>(pm + blk_off(t, 32 + 8 * c8)) = make_uint4(0, 0, 0, 0);
+                }
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            named_sync(BAR_PREP, NGRP);
             PHASE(5);
-            // the carry group must be done with chunk c-1's MMAs before PM, K~, A1, U are rewritten
-            if (c > 0 && !mbar_wait_sleep(bar_m2, (c - 1) & 1)) to = true;
+            // ---- a3: T = (I + A)^{-1} and the bf16 operand [T diag(beta); T diag(c_W)] ----
+            // Diagonal 16 x 16 blocks on the CUDA cores, then the off-diagonal blocks T21 = -T22 (A21 T11) on
+            // the tensor core (kind::tf32, M = 128 over rows 0..127 of the operand: rows past the matrix land
+            // in TMEM lanes nobody reads), 16 -> 32 for both 32 x 32 blocks at once, then 32 -> 64.  Warp 8
+            // (lanes 0..31) and warp 9 (lanes 32..63) carry the products through TMEM columns 0..127 of the
+            // Gram area (free until the W MMA); thread p == 0 issues the MMAs.
+            solve_diag16(sm + OFF_AF, sm + OFF_TF, sm + OFF_TB, p);
+            fence_proxy_async_smem();
+            tc_fence_before();
+            named_sync(BAR_PREP, NGRP);
+            PHASE(13);
+            if (warp == 8 || warp == 9) {
+                const uint32_t sA_ = sbase + OFF_AF, sT_ = sbase + OFF_TF, sX_ = sbase + OFF_XB, sTB_ = sbase + OFF_TB;
+                // round 0: X = A21 T11 (16 x 16) for the blocks at rows 16.. and 48.. -> TMEM cols 0.., 32..
+                // (N = 32, one whole swizzle atom of the MN-major operand; columns 16..31 of each product are
+                // not read)
+                if (p == 0) {
+                    tc_fence_after();
+                    const uint32_t id = idesc_tf32(128, 32, false, true, false);
+#pragma unroll
+                    for (int k = 0; k < 2; ++k) {
+                        mma_tf32(tmem + TM_GPW, sdesc_sw128(sA_ + k * 32, 16, 1024),
+                                 sdesc_sw128_32b(sTB_ + k * 1024, 512), id, k > 0);
+                        mma_tf32(tmem + TM_GPW + 32, sdesc_sw128(sA_ + 8192 + k * 32, 16, 1024),
+                                 sdesc_sw128_32b(sTB_ + 4096 + k * 1024, 512), id, k > 0);
+                    }
+                    mma_commit(bar_sv);
+                }
+                __syncwarp();
+                wait_ok(bar_sv, (3 * c) & 1);
+                tc_fence_after();
+                {  // lanes 16..31 (warp 8) / 48..63 (warp 9) hold the 16 rows of X; X -> sX rows 0..15 / 16..31
+                    float xv[32];
+                    tmem_ld32(tmem + TM_GPW + lane_base + 32 * (warp - 8), xv);
+                    tmem_ld_wait();
+                    if (lane >= 16) {
+                        const int kk = lane - 16 + 16 * (warp - 8);
+#pragma unroll
+                        for (int c4 = 0; c4 < 4; ++c4)
+                            *reinterpret_cast<float4 *>(sm + OFF_XB + b32_off(kk, 4 * c4)) =
+                                make_float4(xv[4 * c4], xv[4 * c4 + 1], xv[4 * c4 + 2], xv[4 * c4 + 3]);
+                    }
+                }
+                fence_proxy_async_smem();
+                tc_fence_before();
+                named_sync(BAR_SOLVE, 64);
+                // round 1: T21 = -T22 X (16 x 16) -> TMEM cols 64.., 96.. (N = 32 as above)
+                if (p == 0) {
+                    tc_fence_after();
+                    const uint32_t id = idesc_tf32(128, 32, false, true, true);
+#pragma unroll
+                    for (int k = 0; k < 2; ++k) {
+                        mma_tf32(tmem + TM_GPW + 64, sdesc_sw128(sT_ + 64 + k * 32, 16, 1024),
+                                 sdesc_sw128_32b(sX_ + k * 1024, 512), id, k > 0);
+                        mma_tf32(tmem + TM_GPW + 96, sdesc_sw128(sT_ + 8192 + 64 + k * 32, 16, 1024),
+                                 sdesc_sw128_32b(sX_ + 2048 + k * 1024, 512), id, k > 0);
+                    }
+                    mma_commit(bar_sv);
+                }
+                __syncwarp();
+                wait_ok(bar_sv, (3 * c + 1) & 1);
+                tc_fence_after();
+                {  // T rows 16..31, cols 0..15 (warp 8) and rows 48..63, cols 32..47 (warp 9)
+                    float tv[32];
+                    tmem_ld32(tmem + TM_GPW + lane_base + 64 + 32 * (warp - 8), tv);
+                    tmem_ld_wait();
+                    if (lane >= 16) {
+                        const int r = row, c0 = 32 * (warp - 8);
+#pragma unroll
+                        for (int c4 = 0; c4 < 4; ++c4) {
+                            const float4 t4 = make_float4(tv[4 * c4], tv[4 * c4 + 1], tv[4 * c4 + 2], tv[4 * c4 + 3]);
+                            *reinterpret_cast<float4 *>(sm + OFF_TF + f32_off(r, c0 + 4 * c4)) = t4;
+                            // rows 16..31 belong to T11, the MN-major operand of round 2
+                            if (warp == 8) *reinterpret_cast<float4 *>(sm + OFF_TB + b32_off(r, 4 * c4)) = t4;
+                        }
+                    }
+                }
+                fence_proxy_async_smem();
+                tc_fence_before();
+                named_sync(BAR_SOLVE, 64);
+                // round 2: X = A21 T11 (32 x 32) -> TMEM cols 0..31 (lanes 32..63)
+                if (p == 0) {
+                    tc_fence_after();
+                    const uint32_t id = idesc_tf32(128, 32, false, true, false);
+#pragma unroll
+                    for (int k = 0; k < 4; ++k)
+                        mma_tf32(tmem + TM_GPW, sdesc_sw128(sA_ + k * 32, 16, 1024),
+                                 sdesc_sw128_32b(sTB_ + k * 1024, 512), id, k > 0);
+                    mma_commit(bar_sv);
+                }
+                __syncwarp();
+                if (warp == 9) {
+                    wait_ok(bar_sv, (3 * c + 2) & 1);
+                    tc_fence_after();
+                    float xv[32];
+                    tmem_ld32(tmem + TM_GPW + lane_base, xv);
+                    tmem_ld_wait();
+                    const int kk = lane;
+#pragma unroll
+                    for (int c4 = 0; c4 < 8; ++c4)
+                        *reinterpret_cast<float4 *>(sm + OFF_XB + b32_off(kk, 4 * c4)) =
+                            make_float4(xv[4 * c4], xv[4 * c4 + 1], xv[4 * c4 + 2], xv[4 * c4 + 3]);
+                    fence_proxy_async_smem();
+                    tc_fence_before();
+                }
+                named_sync(BAR_SOLVE, 64);
+                // round 3: T21 = -T22 X (32 x 32) -> TMEM cols 32..63 (lanes 32..63)
+                if (p == 0) {
+                    tc_fence_after();
+                    const uint32_t id = idesc_tf32(128, 32, false, true, true);
+#pragma unroll
+                    for (int k = 0; k < 4; ++k)
+                        mma_tf32(tmem + TM_GPW + 32, sdesc_sw128(sT_ + 8192 + k * 32, 16, 1024),
+                                 sdesc_sw128_32b(sX_ + k * 1024, 512), id, k > 0);
+                    mma_commit(bar_sv3);
+                }
+                __syncwarp();
+            }
+            PHASE(14);
+            // every prep warp: the last merge (and with it every read of A) has completed
+            wait_ok(bar_sv3, par);
             tc_fence_after();
             PHASE(6);
-            if (q4 >= 2) {  // Pm rows (TMEM, fp32) -> rows 64 + t of the bf16 [0; Pm] operand
-                float v[32];
-                tmem_ld32(tmem + TM_GPW + lane_base + 32 * hf, v);
+            if (q4 == 1) {  // TT rows 32 + r (beta, warp 9) / 96 + r (c_W, warp 13), columns 0..31 from T21
+                const int r = lane;
+                float tv[32];
+                tmem_ld32(tmem + TM_GPW + lane_base + 32, tv);
+                const float *scl = hf ? vCw : vBeta;
                 tmem_ld_wait();
-                const int t = row - 64;
 #pragma unroll
-                for (int j = 0; j < 32; ++j) v[j] = (32 * hf + j <= t) ? v[j] : 0.f;
+                for (int j = 0; j < 32; ++j) tv[j] *= scl[j];
 #pragma unroll
                 for (int c8 = 0; c8 < 4; ++c8)
-                    *reinterpret_cast<uint4 *>(sm + OFF_PM + blk_off(64 + t, 32 * hf + 8 * c8)) = pack8(&v[8 * c8]);
+                    *reinterpret_cast<uint4 *>(sm + OFF_TT + blk_off(32 + 64 * hf + r, 8 * c8)) = pack8(&tv[8 * c8]);
+            } else {  // the rest of TT from T11 and T22 in shared memory (zeros above the diagonal)
+                const int pi = (q4 == 0 ? 0 : q4 - 1) * 64 + hf * 32 + lane;  // 0..191
+                for (int e = pi; e < 768; e += 192) {
+                    // items (R, j): rows R with t = R % 64 < 32 take all 8 column chunks, rows with t >= 32 take
+                    // chunks 4..7 (chunks 0..3 are T21, from TMEM)
+                    int R, j;
+                    if (e < 512) { R = (e >> 3) & 31; R += (e >> 8) * 64; j = e & 7; }
+                    else { const int f = e - 512; R = 32 + ((f >> 2) & 31) + (f >> 7) * 64; j = 4 + (f & 3); }
+                    const int t = R & 63;
+                    const float *scl = (R < 64 ? vBeta : vCw) + 8 * j;
+                    float f8[8];
+                    if (8 * j <= t) {
+                        const float4 t0 = *reinterpret_cast<const float4 *>(sm + OFF_TF + f32_off(t, 8 * j));
+                        const float4 t1 = *reinterpret_cast<const float4 *>(sm + OFF_TF + f32_off(t, 8 * j + 4));
+                        const float tv[8] = {t0.x, t0.y, t0.z, t0.w, t1.x, t1.y, t1.z, t1.w};
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) f8[i] = (8 * j + i <= t) ? tv[i] * scl[i] : 0.f;
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) f8[i] = 0.f;
+                    }
+                    *reinterpret_cast<uint4 *>(sm + OFF_TT + blk_off(R, 8 * j)) = pack8(f8);
+                }
             }
+            PHASE(7);
+            // TMEM U is free once the carry group read U of chunk c-1 (its v_new epilogue precedes MMA2)
+            if (c > 0 && !mbar_wait_sleep(bar_m2, (c - 1) & 1)) to = true;
             fence_proxy_async_smem();
             tc_fence_before();
             // H2: the control warp issues W and U (rows 64..127 of TT K, rows 0..63 of TT V)
             if (named_sync_or(BAR_PCTL, NPC, to)) break;
-            tc_fence_after();
-            PHASE(7);
-            // meanwhile: X_g rows (64..127 of A1) and K~ from the staged q/k tiles
-            for (int e = p; e < 2 * 64 * 16; e += NGRP) {
-                const int isk = e >> 10, r = (e >> 4) & 63, blk = (e >> 3) & 1, ch = e & 7;
-                const uint32_t rb = (r >> 3) * 1024u + (r & 7) * 128u + ch * 16u;  // same swizzle phase (row % 8)
-                float f[8];
-                if (isk) {
-                    unpack8(*reinterpret_cast<const uint4 *>(sm + OFF_K0 + blk * 16384 + rb), f);
-                    const float sc = vTail[r];
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) f[i] *= sc;
-                    *reinterpret_cast<uint4 *>(sm + OFF_KT + blk * 8192 + rb) = pack8(f);
-                } else {
-                    unpack8(*reinterpret_cast<const uint4 *>(sm + OFF_Q0 + blk * 16384 + rb), f);
-                    const float sc = vEG[r] * vRq[r];
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) f[i] *= sc;
-                    *reinterpret_cast<uint4 *>(sm + OFF_A1 + blk * 16384 + 8192 + rb) = pack8(f);
-                }
-            }
-            wait_ok(bar_wu, par);
-            tc_fence_after();
-            if (named_sync_or(BAR_PCTL, NPC, to)) break;  // H3: staged tiles fully consumed
             PHASE(8);
+            wait_ok(bar_wu, par);
+            // rows 0..63 of A1 are free once the carry's MMA1 of chunk c-1 completed
+            if (c > 0) wait_ok(bar_m1, (c - 1) & 1);
+            tc_fence_after();
+            PHASE(9);
             if (q4 >= 2) {  // W rows -> rows 0..63 of A1
                 const int t = row - 64;
 #pragma unroll
                 for (int half = 0; half < 2; ++half) {
-                    float v[32];
-                    tmem_ld32(tmem + TM_GPW + lane_base + 64 * hf + 32 * half, v);
+                    float w[32];
+                    tmem_ld32(tmem + TM_GPW + lane_base + 64 * hf + 32 * half, w);
                     tmem_ld_wait();
 #pragma unroll
                     for (int c8 = 0; c8 < 4; ++c8)
                         *reinterpret_cast<uint4 *>(sm + OFF_A1 + hf * 16384 + blk_off(t, 32 * half + 8 * c8)) =
-                            pack8(&v[8 * c8]);
+                            pack8(&w[8 * c8]);
                 }
             }
             fence_proxy_async_smem();
             tc_fence_before();
             named_sync(BAR_PREP, NGRP);
             if (p == 0) mbar_arrive(bar_a1);
-            PHASE(9);
+            PHASE(10);
         }
         if (to && p == 0) *s_abort = 1;
     } else {
@@ -630,14 +741,15 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         };
         for (int c = 0; c < nvalid; ++c) {
             const uint32_t par = c & 1;
-            const float *vec = vecs + (c & 1) * NVEC * 64;
+            const float *vec = vecs + par * NVEC * 64;
             if (!mbar_wait_sleep(bar_a1, par)) to = true;
+            wait_ok(bar_cq, par);
             if (named_sync_or(BAR_CARRY, NGRP, to)) { stop = true; break; }
             tc_fence_after();
             PHASE(16);
             const int n = (int)vec[V_N * 64];
             const float eL = vec[V_EG * 64 + C - 1];
-            // ---- R = [W; X_g] S ----
+            // ---- R = [W; Q] S ----
             if (tid == 0) {
                 const uint32_t id = idesc_bf16(128, 128, false, true);
                 TIMED(23, {
@@ -663,13 +775,15 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             }
             tmem_st_wait();
             wait_ok(bar_m1, par);
+            if (tid == 0 && c + 1 < nvalid) load_carry_q(c + 1);  // the Q rows of A1 are read
             if (tid == kStorer) bulk_wait_read0();  // the previous out tile (same buffer as v_new) is read
             tc_fence_before();
             if (named_sync_or(BAR_CARRY, NGRP, to)) { stop = true; break; }
             tc_fence_after();
             PHASE(17);
-            if (q4 < 2) {  // v_new = U - W S for token t, dv columns [64 hf, +64)
+            if (q4 < 2) {  // v_new = U - W S for token t, dv columns [64 hf, +64); also diag(tail) v_new
                 const int t = row;
+                const float tl = vec[V_TAIL * 64 + t];
 #pragma unroll
                 for (int half = 0; half < 2; ++half) {
                     float u[32], r[32];
@@ -682,32 +796,61 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     for (int c8 = 0; c8 < 4; ++c8)
                         *reinterpret_cast<uint4 *>(sm + OFF_VO + hf * 8192 + blk_off(t, 32 * half + 8 * c8)) =
                             pack8(&u[8 * c8]);
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) u[j] *= tl;
+#pragma unroll
+                    for (int c8 = 0; c8 < 4; ++c8)
+                        *reinterpret_cast<uint4 *>(sm + OFF_VS + hf * 8192 + blk_off(t, 32 * half + 8 * c8)) =
+                            pack8(&u[8 * c8]);
+                }
+            } else {  // rows of Q S: scale by e^{G_t} scale / |q_t| before Pm v_new accumulates onto them
+                const float xs = vec[V_XS * 64 + row - 64];
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
+                    float r[32];
+                    const uint32_t ta = tmem + TM_R + lane_base + 64 * hf + 32 * half;
+                    tmem_ld32(ta, r);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) r[j] *= xs;
+                    tmem_st32(ta, r);
+                }
+                tmem_st_wait();
+            }
+            wait_ok(bar_ck, par);
+            if (n < C) {  // rows of the raw K tile past the length (any content) must not reach S
+                for (int e = tid; e < (C - n) * 16; e += NGRP) {
+                    const int r = n + (e >> 4), blk = (e >> 3) & 1, ch = e & 7;
+                    *reinterpret_cast<uint4 *>(sm + OFF_KT + blk * 8192 + r * 128 + ch * 16) = make_uint4(0, 0, 0, 0);
                 }
             }
             fence_proxy_async_smem();
             tc_fence_before();
-            named_sync(BAR_CARRY, NGRP);
+            if (named_sync_or(BAR_CARRY, NGRP, to)) { stop = true; break; }
             tc_fence_after();
             PHASE(18);
-            // ---- S += K~^T v_new ;  R[64:128] += Pm v_new ----
+            // ---- S += K^T (diag(tail) v_new) ;  R[64:128] += Pm v_new ----
             if (tid == 0) {
                 const uint32_t id_s = idesc_bf16(128, 128, true, true);
                 const uint32_t id_o = idesc_bf16(128, 128, false, true);
+                const uint32_t pm_rows = sbase + (par ? OFF_PM1 : OFF_PM0) - 8192;
                 TIMED(24, {
                     _Pragma("unroll")
                     for (int k = 0; k < 4; ++k) {
-                        const uint64_t bd = sdesc_sw128(sbase + OFF_VO + k * 2048, 8192, 1024);
+                        const uint64_t bd = sdesc_sw128(sbase + OFF_VS + k * 2048, 8192, 1024);
                         mma_bf16(tmem + TM_S, sdesc_sw128(sbase + OFF_KT + k * 2048, 8192, 1024), bd, id_s, 1);
                     }
                     _Pragma("unroll")
                     for (int k = 0; k < 4; ++k) {
                         const uint64_t bd = sdesc_sw128(sbase + OFF_VO + k * 2048, 8192, 1024);
-                        mma_bf16(tmem + TM_R, sdesc_sw128(sbase + OFF_PM + k * 32, 16, 1024), bd, id_o, 1);
+                        mma_bf16(tmem + TM_R, sdesc_sw128(pm_rows + k * 32, 16, 1024), bd, id_o, 1);
                     }
                     mma_commit(bar_m2);
+                    mma_commit(bar_pf + par);
                 });
             }
             wait_ok(bar_m2, par);
+            if (tid == 0 && c + 1 < nvalid) load_carry_k(c + 1);  // the raw K tile is read
             tc_fence_after();
             if (named_sync_or(BAR_CARRY, NGRP, to)) { stop = true; break; }
             PHASE(19);
