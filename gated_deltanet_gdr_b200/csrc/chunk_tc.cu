@@ -98,21 +98,29 @@ constexpr uint32_t OFF_VS = 131072;  // diag(tail) v_new (MN-major, K = tok, N =
 // Pm forms rows 64..127 (rows 0..63 are whatever precedes it and land in dead accumulator lanes)
 constexpr uint32_t OFF_PM0 = 147456, OFF_PM1 = 155648;
 constexpr uint32_t OFF_VO = 163840;  // v_new (MN-major, K = tok, N = dv), then the out tile: dv blocks +0, +8K
-// fp32 64 x 64 matrices of the solve, A and T, in the layout of f32_off() (tf32 MMA operands)
-constexpr uint32_t OFF_AF = 180224;  // A; once the solve has read it, TT = [T diag(beta); T diag(c_W)] (bf16)
-constexpr uint32_t OFF_TT = OFF_AF;
-constexpr uint32_t OFF_TF = OFF_AF + 16384;  // T
-constexpr uint32_t OFF_XB = OFF_TF + 16384;  // X = A21 T11 of the merges (fp32, b32_off layout, 32 rows)
-// the blocks of T the merges read as their MN-major operand, in the b32_off layout: T(0:32, 0:32) at +0,
-// T(32:48, 32:48) at +4 KB
-constexpr uint32_t OFF_TB = OFF_XB + 4096;
+// the solve T = (I + A)^{-1} (see solve_diag16_merge and the prep group's a3 step)
+constexpr int SP = 36;                 // row stride (floats) of the plain 32 x 32 blocks: 16-byte aligned rows
+constexpr uint32_t OFF_TT = 180224;   // TT = [T diag(beta); T diag(c_W)], bf16, K-major 128 x 64; until it is
+                                      // written it holds the diagonal blocks of A (plain) and the merge scratch
+constexpr uint32_t OFF_AP = OFF_TT;              // A11, A22 (plain, 2 x 32 rows of SP floats)
+constexpr uint32_t OFF_XP = OFF_TT + 64 * SP * 4;  // 16 x 16 merge scratch (2 x 16 rows of SP floats)
+constexpr uint32_t OFF_TP = 196608;   // T11, T22 (plain, 2 x 32 rows of SP floats)
+constexpr uint32_t OFF_A21 = 205824;  // A rows 32..63, columns 0..31 (fp32, f32_off layout, 32 rows)
+constexpr uint32_t OFF_T22 = 209920;  // T22 (fp32, f32_off layout, 32 rows)
+constexpr uint32_t OFF_T11 = 214016;  // T11 (fp32, b32_off layout)
+constexpr uint32_t OFF_XB = 218112;   // X = A21 T11 (fp32, b32_off layout)
+static_assert(OFF_XP + 32 * SP * 4 <= OFF_TT + 16384, "plain A and the merge scratch fit in the TT area");
+static_assert(OFF_TP + 64 * SP * 4 <= OFF_A21, "plain T");
 constexpr int NVEC = 12;             // per-chunk vectors of 64 floats (enum below)
-constexpr uint32_t OFF_VEC = OFF_TB + 6144;  // 2 sets x NVEC vectors x 64 floats
+constexpr uint32_t OFF_VEC = OFF_XB + 4096;  // 2 sets x NVEC vectors x 64 floats
 constexpr uint32_t OFF_BAR = OFF_VEC + 2 * NVEC * 64 * 4;
 constexpr uint32_t SMEM_USED = OFF_BAR + 128;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;  // + alignment slack
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
-static_assert(OFF_AF % 1024 == 0 && OFF_TF % 1024 == 0 && OFF_XB % 1024 == 0 && OFF_TB % 1024 == 0, "swizzle atoms");
+static_assert(OFF_TT % 1024 == 0 && OFF_A21 % 1024 == 0 && OFF_T22 % 1024 == 0 && OFF_T11 % 1024 == 0 &&
+                  OFF_XB % 1024 == 0, "swizzle atoms");
+// the M = 128 merge MMAs read 96 rows of 128 bytes past A21 and T22 (their output lanes are not used)
+static_assert(OFF_T22 + 16384 <= SMEM_USED, "merge operand over-read stays in shared memory");
 static_assert(OFF_PM0 >= 8192 && OFF_PM1 == OFF_PM0 + 8192, "Pm buffers");
 
 // TMEM columns (all 128 lanes): the Gram [K; Q][K; Q]^T then W (lanes 64..127), U (lanes 0..63),
@@ -185,41 +193,64 @@ __device__ __forceinline__ uint32_t b32_off(int k, int n) {
     return (uint32_t)((k >> 2) * 512 + (k & 3) * 128 + ((((n >> 3) ^ (k & 3))) << 5) + (n & 7) * 4);
 }
 
-// First step of T = (I + A)^{-1} (A strictly lower, 64 x 64, fp32 in the f32_off layout), by the 256 prep
-// threads p = 0..255: the four 16 x 16 diagonal blocks of T by forward substitution (one column per thread,
-// the whole column written, zeros above the diagonal), and zeros in the upper 16 x 16 blocks of the two
-// 32 x 32 diagonal blocks, which the tensor-core merges read.
-__device__ __forceinline__ void solve_diag16(const uint8_t *sA, uint8_t *sT, uint8_t *sTB, int p) {
+// Element (r, c) of a 32 x 32 diagonal block (r and c in the same 32-block) in the plain layout.
+__device__ __forceinline__ int pl(int r, int c) { return ((r >> 5) * 32 + (r & 31)) * SP + (c & 31); }
+
+// T = (I + A)^{-1}, first part, by the 256 prep threads p: the two 32 x 32 diagonal blocks T11 and T22
+// (A strictly lower; its diagonal blocks plain in sA).  The four 16 x 16 diagonal blocks by forward
+// substitution (one column per thread, zeros above the diagonal), then for each 32-block the lower-left
+// 16 x 16 block T21 = -T22 (A21 T11) with the CUDA cores.
+__device__ __forceinline__ void solve_diag16_merge(const float *sA, float *sT, float *sX, int p) {
     if (p < 64) {
         const int base = (p >> 4) * 16, j = p & 15;
         float x[16];
 #pragma unroll
         for (int t = 0; t < 16; ++t) x[t] = (t == j) ? 1.f : 0.f;
+        const float *a0p = sA + pl(base, base);
 #pragma unroll
         for (int t = 1; t < 16; ++t) {
             float a0 = 0.f, a1 = 0.f;
 #pragma unroll
-            for (int s = 0; s < t; ++s) {
-                const float as = *reinterpret_cast<const float *>(sA + f32_off(base + t, base + s));
-                if (s & 1) a1 = fmaf(as, x[s], a1);
-                else a0 = fmaf(as, x[s], a0);
+            for (int sv = 0; sv < t; ++sv) {
+                if (sv & 1) a1 = fmaf(a0p[t * SP + sv], x[sv], a1);
+                else a0 = fmaf(a0p[t * SP + sv], x[sv], a0);
             }
             if (t > j) x[t] = -(a0 + a1);
         }
+        float *t0p = sT + pl(base, base) + j;
 #pragma unroll
-        for (int t = 0; t < 16; ++t) *reinterpret_cast<float *>(sT + f32_off(base + t, base + j)) = x[t];
-        // blocks 0, 1 (T11) and 2 are also MN-major operands of the merges
-        if (base < 48) {
-            uint8_t *tb = sTB + (base >= 32 ? 4096 : 0);
-            const int b0 = base & 31;
-#pragma unroll
-            for (int t = 0; t < 16; ++t) *reinterpret_cast<float *>(tb + b32_off(b0 + t, b0 + j)) = x[t];
+        for (int t = 0; t < 16; ++t) t0p[t * SP] = x[t];
+    } else {  // zero the upper 16 x 16 block inside each 32 x 32 diagonal block
+        for (int e = p - 64; e < 512; e += 192) {
+            const int blk = e >> 8, r = (e >> 4) & 15, c = e & 15;
+            sT[(32 * blk + r) * SP + 16 + c] = 0.f;
         }
-    } else if (p < 192) {
-        const int e = p - 64, blk = e >> 6, r = (e >> 2) & 15, c4 = (e & 3) * 4;
-        *reinterpret_cast<float4 *>(sT + f32_off(32 * blk + r, 32 * blk + 16 + c4)) = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (blk == 0) *reinterpret_cast<float4 *>(sTB + b32_off(r, 16 + c4)) = make_float4(0.f, 0.f, 0.f, 0.f);
     }
+    named_sync(BAR_PREP, NGRP);
+    // 16 -> 32: X = A21 T11, then T21 = -T22 X, for the blocks at rows 32 b + 16, columns 32 b
+    const int blk = p >> 7, r = (p >> 3) & 15, c2 = (p & 7) * 2;
+    const float *ab = sA + blk * 32 * SP;
+    float *tb = sT + blk * 32 * SP;
+    float x0 = 0.f, x1 = 0.f;
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+        const float a = ab[(16 + r) * SP + k];
+        const float2 t = *reinterpret_cast<const float2 *>(tb + k * SP + c2);
+        x0 = fmaf(a, t.x, x0);
+        x1 = fmaf(a, t.y, x1);
+    }
+    *reinterpret_cast<float2 *>(sX + (blk * 16 + r) * SP + c2) = make_float2(x0, x1);
+    named_sync(BAR_PREP, NGRP);
+    float y0 = 0.f, y1 = 0.f;
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+        const float t = tb[(16 + r) * SP + 16 + k];
+        const float2 xx = *reinterpret_cast<const float2 *>(sX + (blk * 16 + k) * SP + c2);
+        y0 = fmaf(t, xx.x, y0);
+        y1 = fmaf(t, xx.y, y1);
+    }
+    *reinterpret_cast<float2 *>(tb + (16 + r) * SP + c2) = make_float2(-y0, -y1);
+    named_sync(BAR_PREP, NGRP);
 }
 
 __global__ void __launch_bounds__(NT, 1)
@@ -518,11 +549,17 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                         v[4 * j4 + 2] *= rf * ex2_approx(g2t - l.z);
                         v[4 * j4 + 3] *= rf * ex2_approx(g2t - l.w);
                     }
-                    if (q4 < 2) {
-                        // entries on or above the diagonal are never read by the solve
+                    if (q4 < 2 && hf == q4) {
+                        // a diagonal 32 x 32 block, plain (entries on or above the diagonal are never read)
+                        float *ap = reinterpret_cast<float *>(sm + OFF_AP) + pl(t, 0);
 #pragma unroll
                         for (int j4 = 0; j4 < 8; ++j4)
-                            *reinterpret_cast<float4 *>(sm + OFF_AF + f32_off(t, 32 * hf + 4 * j4)) =
+                            *reinterpret_cast<float4 *>(ap + 4 * j4) =
+                                make_float4(v[4 * j4], v[4 * j4 + 1], v[4 * j4 + 2], v[4 * j4 + 3]);
+                    } else if (q4 < 2) {  // A21 (rows 32..63, columns 0..31), operand of the tf32 merge
+#pragma unroll
+                        for (int j4 = 0; j4 < 8; ++j4)
+                            *reinterpret_cast<float4 *>(sm + OFF_A21 + f32_off(t - 32, 4 * j4)) =
                                 make_float4(v[4 * j4], v[4 * j4 + 1], v[4 * j4 + 2], v[4 * j4 + 3]);
                     } else {
 #pragma unroll
@@ -541,164 +578,92 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             tc_fence_before();
             named_sync(BAR_PREP, NGRP);
             PHASE(5);
-            // ---- a3: T = (I + A)^{-1} and the bf16 operand [T diag(beta); T diag(c_W)] ----
-            // Diagonal 16 x 16 blocks on the CUDA cores, then the off-diagonal blocks T21 = -T22 (A21 T11) on
-            // the tensor core (kind::tf32, M = 128 over rows 0..127 of the operand: rows past the matrix land
-            // in TMEM lanes nobody reads), 16 -> 32 for both 32 x 32 blocks at once, then 32 -> 64.  Warp 8
-            // (lanes 0..31) and warp 9 (lanes 32..63) carry the products through TMEM columns 0..127 of the
-            // Gram area (free until the W MMA); thread p == 0 issues the MMAs.
-            solve_diag16(sm + OFF_AF, sm + OFF_TF, sm + OFF_TB, p);
+            // ---- a3: T = (I + A)^{-1} and the bf16 operand TT = [T diag(beta); T diag(c_W)] ----
+            // T = [[T11, 0], [T21, T22]]: the diagonal 32 x 32 blocks on the CUDA cores (solve_diag16_merge),
+            // then one pass that writes them into TT and into the operand layouts of the tensor-core merge
+            // T21 = -T22 (A21 T11): two kind::tf32 MMAs (M = 128 over 32 operand rows: the other lanes are
+            // not read), thread p == 0 issuing them, warp 8 moving X = A21 T11 from TMEM to shared memory,
+            // warps 8 and 12 (TMEM lanes 0..31) scaling T21 into TT.
+            solve_diag16_merge(reinterpret_cast<const float *>(sm + OFF_AP), reinterpret_cast<float *>(sm + OFF_TP),
+                               reinterpret_cast<float *>(sm + OFF_XP), p);
+            PHASE(12);
+            {
+                const int blk = p >> 7, t = (p >> 2) & 31, c8 = p & 3, R = 32 * blk + t, col = 32 * blk + 8 * c8;
+                const float *tp = reinterpret_cast<const float *>(sm + OFF_TP) + pl(R, col);
+                const float4 u0 = *reinterpret_cast<const float4 *>(tp), u1 = *reinterpret_cast<const float4 *>(tp + 4);
+                const float tv[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+                if (blk == 0) {  // T11, the MN-major operand of X = A21 T11
+                    *reinterpret_cast<float4 *>(sm + OFF_T11 + b32_off(t, 8 * c8)) = u0;
+                    *reinterpret_cast<float4 *>(sm + OFF_T11 + b32_off(t, 8 * c8 + 4)) = u1;
+                } else {  // T22, the K-major operand of T21 = -T22 X
+                    *reinterpret_cast<float4 *>(sm + OFF_T22 + f32_off(t, 8 * c8)) = u0;
+                    *reinterpret_cast<float4 *>(sm + OFF_T22 + f32_off(t, 8 * c8 + 4)) = u1;
+                }
+                float fb[8], fw[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    fb[i] = tv[i] * vBeta[col + i];
+                    fw[i] = tv[i] * vCw[col + i];
+                }
+                *reinterpret_cast<uint4 *>(sm + OFF_TT + blk_off(R, col)) = pack8(fb);
+                *reinterpret_cast<uint4 *>(sm + OFF_TT + blk_off(64 + R, col)) = pack8(fw);
+                // zeros: TT rows 0..31 and 64..95, columns 32..63 (above the diagonal)
+                const int Rz = (p >> 2) + ((p >> 7) << 5), cz = 4 + (p & 3);
+                *reinterpret_cast<uint4 *>(sm + OFF_TT + blk_off(Rz, 8 * cz)) = make_uint4(0, 0, 0, 0);
+            }
             fence_proxy_async_smem();
             tc_fence_before();
             named_sync(BAR_PREP, NGRP);
             PHASE(13);
-            if (warp == 8 || warp == 9) {
-                const uint32_t sA_ = sbase + OFF_AF, sT_ = sbase + OFF_TF, sX_ = sbase + OFF_XB, sTB_ = sbase + OFF_TB;
-                // round 0: X = A21 T11 (16 x 16) for the blocks at rows 16.. and 48.. -> TMEM cols 0.., 32..
-                // (N = 32, one whole swizzle atom of the MN-major operand; columns 16..31 of each product are
-                // not read)
-                if (p == 0) {
-                    tc_fence_after();
-                    const uint32_t id = idesc_tf32(128, 32, false, true, false);
-#pragma unroll
-                    for (int k = 0; k < 2; ++k) {
-                        mma_tf32(tmem + TM_GPW, sdesc_sw128(sA_ + k * 32, 16, 1024),
-                                 sdesc_sw128_32b(sTB_ + k * 1024, 512), id, k > 0);
-                        mma_tf32(tmem + TM_GPW + 32, sdesc_sw128(sA_ + 8192 + k * 32, 16, 1024),
-                                 sdesc_sw128_32b(sTB_ + 4096 + k * 1024, 512), id, k > 0);
-                    }
-                    mma_commit(bar_sv);
-                }
-                __syncwarp();
-                wait_ok(bar_sv, (3 * c) & 1);
+            if (p == 0) {  // X = A21 T11 -> TMEM lanes 0..31, columns 0..31
                 tc_fence_after();
-                {  // lanes 16..31 (warp 8) / 48..63 (warp 9) hold the 16 rows of X; X -> sX rows 0..15 / 16..31
-                    float xv[32];
-                    tmem_ld32(tmem + TM_GPW + lane_base + 32 * (warp - 8), xv);
-                    tmem_ld_wait();
-                    if (lane >= 16) {
-                        const int kk = lane - 16 + 16 * (warp - 8);
+                const uint32_t id = idesc_tf32(128, 32, false, true, false);
 #pragma unroll
-                        for (int c4 = 0; c4 < 4; ++c4)
-                            *reinterpret_cast<float4 *>(sm + OFF_XB + b32_off(kk, 4 * c4)) =
-                                make_float4(xv[4 * c4], xv[4 * c4 + 1], xv[4 * c4 + 2], xv[4 * c4 + 3]);
-                    }
-                }
+                for (int k = 0; k < 4; ++k)
+                    mma_tf32(tmem + TM_GPW, sdesc_sw128(sbase + OFF_A21 + k * 32, 16, 1024),
+                             sdesc_sw128_32b(sbase + OFF_T11 + k * 1024, 512), id, k > 0);
+                mma_commit(bar_sv);
+            }
+            if (warp == 8) {
+                __syncwarp();
+                wait_ok(bar_sv, par);
+                tc_fence_after();
+                float xv[32];
+                tmem_ld32(tmem + TM_GPW + lane_base, xv);
+                tmem_ld_wait();
+#pragma unroll
+                for (int c4 = 0; c4 < 8; ++c4)
+                    *reinterpret_cast<float4 *>(sm + OFF_XB + b32_off(lane, 4 * c4)) =
+                        make_float4(xv[4 * c4], xv[4 * c4 + 1], xv[4 * c4 + 2], xv[4 * c4 + 3]);
                 fence_proxy_async_smem();
                 tc_fence_before();
-                named_sync(BAR_SOLVE, 64);
-                // round 1: T21 = -T22 X (16 x 16) -> TMEM cols 64.., 96.. (N = 32 as above)
-                if (p == 0) {
-                    tc_fence_after();
-                    const uint32_t id = idesc_tf32(128, 32, false, true, true);
-#pragma unroll
-                    for (int k = 0; k < 2; ++k) {
-                        mma_tf32(tmem + TM_GPW + 64, sdesc_sw128(sT_ + 64 + k * 32, 16, 1024),
-                                 sdesc_sw128_32b(sX_ + k * 1024, 512), id, k > 0);
-                        mma_tf32(tmem + TM_GPW + 96, sdesc_sw128(sT_ + 8192 + 64 + k * 32, 16, 1024),
-                                 sdesc_sw128_32b(sX_ + 2048 + k * 1024, 512), id, k > 0);
-                    }
-                    mma_commit(bar_sv);
-                }
                 __syncwarp();
-                wait_ok(bar_sv, (3 * c + 1) & 1);
-                tc_fence_after();
-                {  // T rows 16..31, cols 0..15 (warp 8) and rows 48..63, cols 32..47 (warp 9)
-                    float tv[32];
-                    tmem_ld32(tmem + TM_GPW + lane_base + 64 + 32 * (warp - 8), tv);
-                    tmem_ld_wait();
-                    if (lane >= 16) {
-                        const int r = row, c0 = 32 * (warp - 8);
-#pragma unroll
-                        for (int c4 = 0; c4 < 4; ++c4) {
-                            const float4 t4 = make_float4(tv[4 * c4], tv[4 * c4 + 1], tv[4 * c4 + 2], tv[4 * c4 + 3]);
-                            *reinterpret_cast<float4 *>(sm + OFF_TF + f32_off(r, c0 + 4 * c4)) = t4;
-                            // rows 16..31 belong to T11, the MN-major operand of round 2
-                            if (warp == 8) *reinterpret_cast<float4 *>(sm + OFF_TB + b32_off(r, 4 * c4)) = t4;
-                        }
-                    }
-                }
-                fence_proxy_async_smem();
-                tc_fence_before();
-                named_sync(BAR_SOLVE, 64);
-                // round 2: X = A21 T11 (32 x 32) -> TMEM cols 0..31 (lanes 32..63)
-                if (p == 0) {
-                    tc_fence_after();
-                    const uint32_t id = idesc_tf32(128, 32, false, true, false);
-#pragma unroll
-                    for (int k = 0; k < 4; ++k)
-                        mma_tf32(tmem + TM_GPW, sdesc_sw128(sA_ + k * 32, 16, 1024),
-                                 sdesc_sw128_32b(sTB_ + k * 1024, 512), id, k > 0);
-                    mma_commit(bar_sv);
-                }
-                __syncwarp();
-                if (warp == 9) {
-                    wait_ok(bar_sv, (3 * c + 2) & 1);
-                    tc_fence_after();
-                    float xv[32];
-                    tmem_ld32(tmem + TM_GPW + lane_base, xv);
-                    tmem_ld_wait();
-                    const int kk = lane;
-#pragma unroll
-                    for (int c4 = 0; c4 < 8; ++c4)
-                        *reinterpret_cast<float4 *>(sm + OFF_XB + b32_off(kk, 4 * c4)) =
-                            make_float4(xv[4 * c4], xv[4 * c4 + 1], xv[4 * c4 + 2], xv[4 * c4 + 3]);
-                    fence_proxy_async_smem();
-                    tc_fence_before();
-                }
-                named_sync(BAR_SOLVE, 64);
-                // round 3: T21 = -T22 X (32 x 32) -> TMEM cols 32..63 (lanes 32..63)
-                if (p == 0) {
+                if (lane == 0) {  // T21 = -T22 X -> TMEM lanes 0..31, columns 32..63
                     tc_fence_after();
                     const uint32_t id = idesc_tf32(128, 32, false, true, true);
 #pragma unroll
                     for (int k = 0; k < 4; ++k)
-                        mma_tf32(tmem + TM_GPW + 32, sdesc_sw128(sT_ + 8192 + k * 32, 16, 1024),
-                                 sdesc_sw128_32b(sX_ + k * 1024, 512), id, k > 0);
+                        mma_tf32(tmem + TM_GPW + 32, sdesc_sw128(sbase + OFF_T22 + k * 32, 16, 1024),
+                                 sdesc_sw128_32b(sbase + OFF_XB + k * 1024, 512), id, k > 0);
                     mma_commit(bar_sv3);
                 }
                 __syncwarp();
             }
             PHASE(14);
-            // every prep warp: the last merge (and with it every read of A) has completed
-            wait_ok(bar_sv3, par);
-            tc_fence_after();
-            PHASE(6);
-            if (q4 == 1) {  // TT rows 32 + r (beta, warp 9) / 96 + r (c_W, warp 13), columns 0..31 from T21
-                const int r = lane;
+            if (warp == 8 || warp == 12) {  // TT rows 32 + r (beta) / 96 + r (c_W), columns 0..31 from T21
+                wait_ok(bar_sv3, par);
+                tc_fence_after();
                 float tv[32];
-                tmem_ld32(tmem + TM_GPW + lane_base + 32, tv);
+                tmem_ld32(tmem + TM_GPW + 32, tv);
                 const float *scl = hf ? vCw : vBeta;
                 tmem_ld_wait();
 #pragma unroll
-                for (int j = 0; j < 32; ++j) tv[j] *= scl[j];
+                for (int jj = 0; jj < 32; ++jj) tv[jj] *= scl[jj];
 #pragma unroll
                 for (int c8 = 0; c8 < 4; ++c8)
-                    *reinterpret_cast<uint4 *>(sm + OFF_TT + blk_off(32 + 64 * hf + r, 8 * c8)) = pack8(&tv[8 * c8]);
-            } else {  // the rest of TT from T11 and T22 in shared memory (zeros above the diagonal)
-                const int pi = (q4 == 0 ? 0 : q4 - 1) * 64 + hf * 32 + lane;  // 0..191
-                for (int e = pi; e < 768; e += 192) {
-                    // items (R, j): rows R with t = R % 64 < 32 take all 8 column chunks, rows with t >= 32 take
-                    // chunks 4..7 (chunks 0..3 are T21, from TMEM)
-                    int R, j;
-                    if (e < 512) { R = (e >> 3) & 31; R += (e >> 8) * 64; j = e & 7; }
-                    else { const int f = e - 512; R = 32 + ((f >> 2) & 31) + (f >> 7) * 64; j = 4 + (f & 3); }
-                    const int t = R & 63;
-                    const float *scl = (R < 64 ? vBeta : vCw) + 8 * j;
-                    float f8[8];
-                    if (8 * j <= t) {
-                        const float4 t0 = *reinterpret_cast<const float4 *>(sm + OFF_TF + f32_off(t, 8 * j));
-                        const float4 t1 = *reinterpret_cast<const float4 *>(sm + OFF_TF + f32_off(t, 8 * j + 4));
-                        const float tv[8] = {t0.x, t0.y, t0.z, t0.w, t1.x, t1.y, t1.z, t1.w};
-#pragma unroll
-                        for (int i = 0; i < 8; ++i) f8[i] = (8 * j + i <= t) ? tv[i] * scl[i] : 0.f;
-                    } else {
-#pragma unroll
-                        for (int i = 0; i < 8; ++i) f8[i] = 0.f;
-                    }
-                    *reinterpret_cast<uint4 *>(sm + OFF_TT + blk_off(R, 8 * j)) = pack8(f8);
-                }
+                    *reinterpret_cast<uint4 *>(sm + OFF_TT + blk_off(32 + 64 * hf + lane, 8 * c8)) = pack8(&tv[8 * c8]);
             }
+            PHASE(6);
             PHASE(7);
             // TMEM U is free once the carry group read U of chunk c-1 (its v_new epilogue precedes MMA2)
             if (c > 0 && !mbar_wait_sleep(bar_m2, (c - 1) & 1)) to = true;
