@@ -431,8 +431,6 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         for (int c = 0; c < nvalid; ++c) {
             const uint32_t par = c & 1;
             if (named_sync_or(BAR_PCTL, NPC, to)) break;  // H0: chunk c staged (or a timeout)
-            if (lane == 1 && c + 2 < nvalid) prefetch_l2(c + 2);
-            __syncwarp();
             named_sync(BAR_PCTL, NPC);  // H1: padding rows zeroed
             if (lane == 0) {  // a2: the Gram [K; Q][K; Q]^T (its diagonal gives the row norms)
                 tc_fence_after();
@@ -465,8 +463,12 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 mma_commit(bar_wu);
             }
             if (lane == 1 && c + 1 < nvalid) {  // the stage is consumed once W and U are done
-                if (mbar_wait(bar_wu, par)) issue_loads(c + 1);
-                else to = true;
+                if (mbar_wait(bar_wu, par)) {
+                    issue_loads(c + 1);
+                    if (c + 2 < nvalid) prefetch_l2(c + 2);
+                } else {
+                    to = true;
+                }
             }
             __syncwarp();
         }
@@ -727,18 +729,21 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     mma_commit(bar_m1);
                 });
             }
-            // meanwhile: S <- e^{G_last} S in TMEM (MMA2 accumulates onto it)
+            // S <- e^{G_last} S in TMEM, onto which MMA2 accumulates (for c > 0 the previous chunk's
+            // epilogue already wrote the scaled state back)
+            if (c == 0) {
 #pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                float v[32];
-                const uint32_t ta = tmem + TM_S + lane_base + 64 * hf + 32 * half;
-                tmem_ld32(ta, v);
-                tmem_ld_wait();
+                for (int half = 0; half < 2; ++half) {
+                    float v[32];
+                    const uint32_t ta = tmem + TM_S + lane_base + 64 * hf + 32 * half;
+                    tmem_ld32(ta, v);
+                    tmem_ld_wait();
 #pragma unroll
-                for (int j = 0; j < 32; ++j) v[j] *= eL;
-                tmem_st32(ta, v);
+                    for (int j = 0; j < 32; ++j) v[j] *= eL;
+                    tmem_st32(ta, v);
+                }
+                tmem_st_wait();
             }
-            tmem_st_wait();
             wait_ok(bar_m1, par);
             if (tid == 0 && c + 1 < nvalid) load_carry_q(c + 1);  // the Q rows of A1 are read
             if (tid == kStorer) bulk_wait_read0();  // the previous out tile (same buffer as v_new) is read
@@ -819,17 +824,27 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             tc_fence_after();
             if (named_sync_or(BAR_CARRY, NGRP, to)) { stop = true; break; }
             PHASE(19);
-            // ---- S (fp32, TMEM) -> bf16 operand tile;  o rows -> out tile ----
+            // ---- S (fp32, TMEM) -> bf16 operand tile, and back to TMEM scaled by e^{G_last} of the next
+            // chunk (its gate vectors were written before this chunk was handed over);  o rows -> out tile ----
+            const bool more = c + 1 < nvalid;
+            const float eLn = more ? vecs[(par ^ 1) * NVEC * 64 + V_EG * 64 + C - 1] : 1.f;
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
                 float v[32];
-                tmem_ld32(tmem + TM_S + lane_base + 64 * hf + 32 * half, v);
+                const uint32_t ta = tmem + TM_S + lane_base + 64 * hf + 32 * half;
+                tmem_ld32(ta, v);
                 tmem_ld_wait();
 #pragma unroll
                 for (int c8 = 0; c8 < 4; ++c8)
                     *reinterpret_cast<uint4 *>(sm + OFF_S + hf * 16384 + blk_off(row, 32 * half + 8 * c8)) =
                         pack8(&v[8 * c8]);
+                if (more) {
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) v[j] *= eLn;
+                    tmem_st32(ta, v);
+                }
             }
+            if (more) tmem_st_wait();
             if (q4 >= 2) {
                 const int t = row - 64;
 #pragma unroll
