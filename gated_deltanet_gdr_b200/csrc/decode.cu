@@ -54,6 +54,38 @@ __device__ __forceinline__ f2_t fma2(f2_t a, f2_t b, f2_t c) {
     return d;
 }
 
+// explicit shared-memory loads (32-bit shared addresses), so that every operand read of the decode loop
+// is a shared-memory access
+__device__ __forceinline__ uint4 lds128(uint32_t a) {
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
+    return v;
+}
+__device__ __forceinline__ float lds_f32(uint32_t a) {
+    float v;
+    asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(a));
+    return v;
+}
+__device__ __forceinline__ float lds_bf16(uint32_t a) {
+    unsigned short v;
+    asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(a));
+    return __uint_as_float((uint32_t)v << 16);
+}
+template <typename T> __device__ __forceinline__ float lds_elem(uint32_t a);
+template <> __device__ __forceinline__ float lds_elem<float>(uint32_t a) { return lds_f32(a); }
+template <> __device__ __forceinline__ float lds_elem<__nv_bfloat16>(uint32_t a) { return lds_bf16(a); }
+__device__ __forceinline__ int lds_s32(uint32_t a) {
+    int v;
+    asm volatile("ld.shared.s32 %0, [%1];" : "=r"(v) : "r"(a));
+    return v;
+}
+
+// 2^x on the special-function unit (PTX ex2.approx.ftz.f32)
+__device__ __forceinline__ float exp2f_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
 __device__ __forceinline__ void cp_async16(void *smem, const void *gmem) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(sm100::smem_u32(smem)), "l"(gmem) : "memory");
 }
@@ -366,6 +398,383 @@ decode_kernel(const DecodeArgs a, const int ntiles) {
     cp_async_wait0();
 }
 
+// ------------------------------------------------------------------------------------------------
+// Dk = Dv = 128: one tile is a whole (sequence, value head) state.  A persistent CTA of four warps
+// keeps up to NSTAGE tiles in flight (one TMA copy of the state slab plus one bulk copy per token
+// array, on the stage's mbarrier) and computes one; warp w owns state columns [32 w, 32 w + 32),
+// lane (rg = lane / 4, cv = lane % 4) rows rg + 8 r (r = 0..15) and columns 32 w + 8 cv .. + 7, so a
+// thread holds 128 state values and the per-token work (norms, gate, reductions) is spread over twice
+// as many elements as in the general kernel.  The gate e^g and beta are computed once per tile by
+// the scalar threads.  After the three-level reduce-scatter over the row groups, lane (rg, cv) holds
+// both readouts k^T S' and q^T S' of column 32 w + 8 cv + rg, so it computes that column's delta and
+// output directly.
+template <typename TI, typename TS, int NW, int NSTG> struct D128 {
+    static constexpr int D = 128, NT = 32 * NW;
+    static constexpr int NCV = 16 / NW;           // 8-column vectors per warp (lanes per row group)
+    static constexpr int NRG = 32 / NCV;          // row groups per warp
+    static constexpr int RPT = D / NRG;           // state rows per thread (16 or 8)
+    static constexpr int NSTAGE = NSTG;
+    static constexpr int BOXC = 128 / (int)sizeof(TS);  // state columns per 128-byte box row
+    static constexpr int NBOX = D / BOXC;                // boxes per state slab (2 for bf16, 4 for fp32)
+    static constexpr int STATE_BYTES = D * D * (int)sizeof(TS);
+    struct Layout {
+        int off_q, off_k, off_v, off_gk, stage, off_bar, off_meta, smem;
+    };
+    static __host__ __device__ Layout layout(int S, bool gk) {
+        Layout l;
+        l.off_q = STATE_BYTES;
+        l.off_k = l.off_q + S * D * (int)sizeof(TI);
+        l.off_v = l.off_k + S * D * (int)sizeof(TI);
+        l.off_gk = l.off_v + S * D * (int)sizeof(TI);
+        const int end = l.off_gk + (gk ? S * D * 4 : 0);
+        l.stage = (end + 1023) & ~1023;  // the TMA destinations stay 1024-byte aligned
+        l.off_bar = NSTAGE * l.stage;     // NSTAGE "full" then NSTAGE "empty" mbarriers
+        l.off_meta = l.off_bar + 64;
+        l.smem = l.off_meta + 4 * META_INTS * 4 + 1024;  // four scalar sets, + alignment slack
+        return l;
+    }
+};
+
+// Raw per-tile scalars, prefetched one tile ahead into registers by threads 0..T+1 (no branch on a
+// loaded value): thread t < T: idx[b S + t], raw beta, raw gate, A_log[h], dt_bias[h]; thread T: L;
+// thread T+1: A.
+template <typename TI>
+__device__ __forceinline__ void prefetch_meta128(const DecodeArgs &a, int bh, int tid, int (&r)[5]) {
+    const int b = bh / a.Nv, h = bh % a.Nv, S = a.S;
+    r[0] = r[1] = r[2] = r[3] = r[4] = 0;
+    if (tid < T) {
+        if (tid < S) {
+            r[0] = a.idx[(size_t)b * S + tid];
+            r[1] = __float_as_int(to_f32(reinterpret_cast<const TI *>(a.beta)[(size_t)bh * S + tid]));
+            if (a.g) r[2] = __float_as_int(a.g[(size_t)bh * S + tid]);
+            if (a.A_log) {
+                r[3] = __float_as_int(a.A_log[h]);
+                r[4] = __float_as_int(a.dt_bias[h]);
+            }
+        }
+    } else if (tid == T) {
+        r[0] = a.lengths[b];
+    } else if (tid == T + 1) {
+        r[0] = a.accepted ? a.accepted[b] : a.lengths[b];
+    }
+}
+// The set layout of put_meta (L, A, idx[T], beta[T], g[T]), with beta and the decay e^g final.
+__device__ __forceinline__ void put_meta128(const DecodeArgs &a, int *mm, int tid, const int (&r)[5]) {
+    if (tid < T) {
+        mm[2 + tid] = r[0];
+        const float braw = __int_as_float(r[1]), graw = __int_as_float(r[2]);
+        mm[2 + T + tid] = __float_as_int(a.beta_logits ? sigmoid_f32(braw) : braw);
+        const float g = a.A_log ? gate_from_raw(graw, __int_as_float(r[3]), __int_as_float(r[4])) : graw;
+        mm[2 + 2 * T + tid] = __float_as_int(a.g ? expf(g) : 1.f);
+    } else if (tid == T) {
+        mm[0] = r[0];
+    } else if (tid == T + 1) {
+        mm[1] = r[0];
+    }
+}
+
+template <typename TI, typename TS, int NW, int NSTG, int MINB>
+__global__ void __launch_bounds__(32 * NW, MINB)
+decode128_kernel(const __grid_constant__ CUtensorMap tm_pool, const DecodeArgs a, const int ntiles) {
+    using Cf = D128<TI, TS, NW, NSTG>;
+    constexpr int NCV = Cf::NCV, NRG = Cf::NRG, RPT = Cf::RPT;
+    constexpr int D = Cf::D, NS = Cf::NSTAGE;
+    extern __shared__ __align__(1024) uint8_t smraw[];
+    uint8_t *smem = smraw + ((1024u - (sm100::smem_u32(smraw) & 1023u)) & 1023u);
+    const typename Cf::Layout ly = Cf::layout(a.S, a.gk != nullptr);
+    // full[s]: stage s holds its tile (TMA / bulk transactions); empty[s]: the four warps are done with it
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + ly.off_bar), *empty = full + NS;
+    int *s_meta = reinterpret_cast<int *>(smem + ly.off_meta);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int rg = lane / NCV, cv = lane % NCV;
+    const int c0 = 8 * NCV * warp + 8 * cv;  // first state column of this thread
+    const int S = a.S;
+    // byte offset of this thread's 8 columns of row rg (row rg + NRG r is 128 NRG r further): the 128-byte
+    // swizzle XORs the 16-byte chunk index with the row index modulo 8, which is rg % 8 for every row here
+    const int box = c0 / Cf::BOXC, ch0 = (c0 % Cf::BOXC) * (int)sizeof(TS) / 16, sw = rg & 7;
+    const int soff = box * (D * 128) + rg * 128 + ((ch0 ^ sw) << 4);
+    const int soff2 = box * (D * 128) + rg * 128 + (((ch0 + 1) ^ sw) << 4);  // second chunk (fp32 state)
+
+    // checked copies of a tile into stage `st` (thread 0): the state slab by TMA, the token rows by bulk copies
+    auto issue = [&](int tile, const int *mm, int st) {
+        uint64_t *bar = full + st;
+        uint8_t *base = smem + st * ly.stage;
+        const int status = tile_status(mm, S, a.slots);
+        const int Lc = status ? 0 : mm[0];
+        if (Lc <= 0) {
+            sm100::mbar_arrive(bar);
+            return;
+        }
+        const int h = tile % a.Nv, b = tile / a.Nv, kh = h / (a.Nv / a.Nk);
+        const uint32_t tok = (uint32_t)Lc * D * (uint32_t)sizeof(TI);
+        sm100::mbar_arrive_expect_tx(bar, Cf::STATE_BYTES + 3 * tok + (a.gk ? (uint32_t)Lc * D * 4 : 0));
+        const int z = mm[2] * a.Nv + h;
+#pragma unroll
+        for (int x = 0; x < Cf::NBOX; ++x) sm100::tma_load_3d(base + x * (D * 128), &tm_pool, bar, x * Cf::BOXC, 0, z);
+        const size_t qk_off = ((size_t)b * a.Nk + kh) * S * D, v_off = (size_t)tile * S * D;
+        sm100::bulk_load(base + ly.off_q, reinterpret_cast<const TI *>(a.q) + qk_off, tok, bar);
+        sm100::bulk_load(base + ly.off_k, reinterpret_cast<const TI *>(a.k) + qk_off, tok, bar);
+        sm100::bulk_load(base + ly.off_v, reinterpret_cast<const TI *>(a.v) + v_off, tok, bar);
+        if (a.gk) sm100::bulk_load(base + ly.off_gk, a.gk + v_off, (uint32_t)Lc * D * 4, bar);
+    };
+
+    int tile = blockIdx.x;
+    if (tile >= ntiles) return;
+    if (tid == 0) {
+        for (int i = 0; i < NS; ++i) {
+            sm100::mbar_init(full + i, 1);
+            sm100::mbar_init(empty + i, Cf::NT / 32);
+        }
+        sm100::fence_mbar_init();
+        sm100::prefetch_tmap(&tm_pool);
+    }
+    // prologue: scalars of the first NS + 1 tiles, copies of the first NS
+    int pre[5];
+    for (int i = 0; i <= NS; ++i) {
+        const int ti = tile + i * (int)gridDim.x;
+        if (ti < ntiles) {
+            prefetch_meta128<TI>(a, ti, tid, pre);
+            put_meta128(a, s_meta + (i & 3) * META_INTS, tid, pre);
+        }
+    }
+    __syncthreads();
+    if (tid == 0)
+        for (int i = 0; i < NS; ++i) {
+            const int ti = tile + i * (int)gridDim.x;
+            if (ti < ntiles) issue(ti, s_meta + (i & 3) * META_INTS, i);
+        }
+    // raw scalars of the next two tiles to publish (tiles j + NS + 1 and j + NS + 2 at iteration j), so
+    // that their global loads have a whole tile of time to land before they are used
+    int pre2[5] = {0, 0, 0, 0, 0};
+    {
+        const int ti = tile + (NS + 1) * (int)gridDim.x, ti2 = ti + (int)gridDim.x;
+        if (ti < ntiles) prefetch_meta128<TI>(a, ti, tid, pre);
+        if (ti2 < ntiles) prefetch_meta128<TI>(a, ti2, tid, pre2);
+    }
+    bool timed_out = false;
+
+    for (int j = 0; tile < ntiles; ++j, tile += gridDim.x) {
+        const int st = j % NS;
+        const int *mm = s_meta + (j & 3) * META_INTS;
+        const int h = tile % a.Nv;
+        const int status = tile_status(mm, S, a.slots);
+        const int Lv = status ? 0 : mm[0];
+        const int A = min(mm[1], Lv);
+        if (tid == 0 && status) raise_device_error(a.err, status == 1 ? GDR_DEVERR_LENGTH : GDR_DEVERR_SLOT_INDEX);
+        TI *out = reinterpret_cast<TI *>(a.out) + (size_t)tile * S * D;
+        for (int e = tid; e < (S - Lv) * (D / 8); e += Cf::NT) {
+            const int t = Lv + e / (D / 8), c = (e % (D / 8)) * 8;
+            float zz[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+            Vec8<TI>::store(out + (size_t)t * D + c, zz);
+        }
+        if (!sm100::mbar_wait(full + st, (uint32_t)(j / NS) & 1u)) timed_out = true;
+        if (Lv > 0 && !timed_out) {
+            const uint8_t *base = smem + st * ly.stage;
+            const uint32_t sb = sm100::smem_u32(base);
+            f2_t sv[RPT][4];
+#pragma unroll
+            for (int r = 0; r < RPT; ++r) {
+                float f[8];
+                if (sizeof(TS) == 2) {
+                    const uint4 u = lds128(sb + soff + r * NRG * 128);
+                    const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        f[2 * i] = __uint_as_float(w4[i] << 16);
+                        f[2 * i + 1] = __uint_as_float(w4[i] & 0xffff0000u);
+                    }
+                } else {
+                    const uint4 u0 = lds128(sb + soff + r * NRG * 128), u1 = lds128(sb + soff2 + r * NRG * 128);
+                    f[0] = __uint_as_float(u0.x); f[1] = __uint_as_float(u0.y);
+                    f[2] = __uint_as_float(u0.z); f[3] = __uint_as_float(u0.w);
+                    f[4] = __uint_as_float(u1.x); f[5] = __uint_as_float(u1.y);
+                    f[6] = __uint_as_float(u1.z); f[7] = __uint_as_float(u1.w);
+                }
+#pragma unroll
+                for (int p = 0; p < 4; ++p) sv[r][p] = pk2(f[2 * p], f[2 * p + 1]);
+            }
+            const uint32_t sq = sb + ly.off_q + rg * (int)sizeof(TI), sk = sb + ly.off_k + rg * (int)sizeof(TI);
+            const uint32_t sgk = sb + ly.off_gk + rg * 4, svv = sb + ly.off_v;
+            // the column whose readouts this lane ends up with (with 16 row groups, lanes rg and rg ^ 1 share
+            // a column: rg even holds k^T S', rg odd q^T S', exchanged below)
+            const int own = c0 + (NRG == 8 ? rg : rg >> 1);
+            for (int t = 0; t < Lv; ++t) {
+                const uint32_t qrow = sq + t * D * (int)sizeof(TI), krow = sk + t * D * (int)sizeof(TI);
+                float xq[RPT], xk[RPT];
+                float ss_q = 0.f, ss_k = 0.f, qk = 0.f;
+#pragma unroll
+                for (int r = 0; r < RPT; ++r) {
+                    xq[r] = lds_elem<TI>(qrow + NRG * r * (int)sizeof(TI));
+                    xk[r] = lds_elem<TI>(krow + NRG * r * (int)sizeof(TI));
+                    ss_q = fmaf(xq[r], xq[r], ss_q);
+                    ss_k = fmaf(xk[r], xk[r], ss_k);
+                    qk = fmaf(xq[r], xk[r], qk);
+                }
+#pragma unroll
+                for (int o = NCV; o < 32; o <<= 1) {  // sums over the row groups
+                    ss_q += __shfl_xor_sync(0xffffffffu, ss_q, o);
+                    ss_k += __shfl_xor_sync(0xffffffffu, ss_k, o);
+                    qk += __shfl_xor_sync(0xffffffffu, qk, o);
+                }
+                float qs = a.scale, kn = 1.f;
+                if (a.l2norm) {
+                    qs = a.scale * rsqrtf(ss_q + a.eps);
+                    kn = rsqrtf(ss_k + a.eps);
+                }
+                qk *= qs * kn;
+#pragma unroll
+                for (int r = 0; r < RPT; ++r) {
+                    xq[r] *= qs;
+                    xk[r] *= kn;
+                }
+                const float ag = __int_as_float(mm[2 + 2 * T + t]), bt = __int_as_float(mm[2 + T + t]);
+                // decay (and, with gk, the per-row factor e^{gk} = 2^{gk log2 e} on the special-function
+                // unit), and both column readouts of the decayed state
+                f2_t mk[4], mq[4];
+#pragma unroll
+                for (int p = 0; p < 4; ++p) mk[p] = mq[p] = 0ull;
+                const uint32_t gkrow = sgk + t * D * 4;
+#pragma unroll
+                for (int r = 0; r < RPT; ++r) {
+                    const float dr = a.gk ? ag * exp2f_approx(lds_f32(gkrow + NRG * r * 4) * 1.4426950408889634f) : ag;
+                    const f2_t d2 = pk2(dr, dr), k2 = pk2(xk[r], xk[r]), q2 = pk2(xq[r], xq[r]);
+#pragma unroll
+                    for (int p = 0; p < 4; ++p) {
+                        const f2_t sd = mul2(sv[r][p], d2);
+                        sv[r][p] = sd;
+                        mk[p] = fma2(k2, sd, mk[p]);
+                        mq[p] = fma2(q2, sd, mq[p]);
+                    }
+                }
+                // reduce-scatter over the row groups (lane bits 2..4): value i = 2c + w (column c of the 8,
+                // w = 0: k^T S', 1: q^T S') ends summed in the lane with rg = c
+                float v[16];
+#pragma unroll
+                for (int p = 0; p < 4; ++p) {
+                    up2(mk[p], v[4 * p], v[4 * p + 2]);
+                    up2(mq[p], v[4 * p + 1], v[4 * p + 3]);
+                }
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const bool hi = lane & 16;
+                    const float send = hi ? v[i] : v[8 + i], keep = hi ? v[8 + i] : v[i];
+                    v[i] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
+                }
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const bool hi = lane & 8;
+                    const float send = hi ? v[i] : v[4 + i], keep = hi ? v[4 + i] : v[i];
+                    v[i] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
+                }
+#pragma unroll
+                for (int i = 0; i < 2; ++i) {
+                    const bool hi = lane & 4;
+                    const float send = hi ? v[i] : v[2 + i], keep = hi ? v[2 + i] : v[i];
+                    v[i] = keep + __shfl_xor_sync(0xffffffffu, send, 4);
+                }
+                float rk, rq;
+                if (NRG == 8) {
+                    rk = v[0];
+                    rq = v[1];
+                } else {  // one more level (lane bit 1), then the two halves of the column swap
+                    const bool hi = lane & 2;
+                    const float send = hi ? v[0] : v[1], keep = hi ? v[1] : v[0];
+                    const float mine = keep + __shfl_xor_sync(0xffffffffu, send, 2);
+                    const float other = __shfl_xor_sync(0xffffffffu, mine, 2);
+                    rk = hi ? other : mine;
+                    rq = hi ? mine : other;
+                }
+                const float vc = lds_elem<TI>(svv + (t * D + own) * (int)sizeof(TI));
+                const float dc = bt * (vc - rk);
+                if (NRG == 8 || !(lane & 2)) out[(size_t)t * D + own] = from_f32<TI>(fmaf(qk, dc, rq));
+                float d[8];  // delta for this thread's 8 columns, from the lanes that own them
+#pragma unroll
+                for (int c = 0; c < 8; ++c) d[c] = __shfl_sync(0xffffffffu, dc, 4 * c + cv);
+#pragma unroll
+                for (int r = 0; r < RPT; ++r) {
+                    const f2_t k2 = pk2(xk[r], xk[r]);
+#pragma unroll
+                    for (int p = 0; p < 4; ++p) sv[r][p] = fma2(k2, pk2(d[2 * p], d[2 * p + 1]), sv[r][p]);
+                }
+                if (t < A && (t == A - 1 || mm[2 + t + 1] != mm[2 + t])) {
+                    // commit straight from registers
+                    TS *dst = reinterpret_cast<TS *>(a.pool) + ((size_t)mm[2 + t] * a.Nv + h) * (D * D) + c0;
+#pragma unroll
+                    for (int r = 0; r < RPT; ++r) {
+                        float f[8];
+#pragma unroll
+                        for (int p = 0; p < 4; ++p) up2(sv[r][p], f[2 * p], f[2 * p + 1]);
+                        Vec8<TS>::store(dst + (size_t)(rg + NRG * r) * D, f);
+                    }
+                }
+            }
+        }
+        // Each warp releases the stage (and the tile's scalar set) on its own; only warp 0 waits until all
+        // four are done, then refills the stage with tile j + NS (whose scalars it published an iteration
+        // ago) and publishes the scalars of tile j + NS + 1 into the freed set (four sets: tiles j .. j + NS
+        // are live).  The other warps go straight on to their next tile.
+        __syncwarp();
+        if (lane == 0) sm100::mbar_arrive(empty + st);
+        if (timed_out) break;
+        if (warp == 0) {
+            const int nxt = tile + NS * (int)gridDim.x;
+            if (!sm100::mbar_wait(empty + st, (uint32_t)(j / NS) & 1u)) {
+                timed_out = true;
+                break;
+            }
+            if (nxt + (int)gridDim.x < ntiles) put_meta128(a, s_meta + ((j + NS + 1) & 3) * META_INTS, tid, pre);
+            __syncwarp();
+            if (tid == 0 && nxt < ntiles) issue(nxt, s_meta + ((j + NS) & 3) * META_INTS, st);
+#pragma unroll
+            for (int i = 0; i < 5; ++i) pre[i] = pre2[i];
+            if (nxt + 3 * (int)gridDim.x < ntiles) prefetch_meta128<TI>(a, nxt + 3 * gridDim.x, tid, pre2);
+        }
+    }
+    if (timed_out && tid == 0) raise_device_error(a.err, 0x4u);
+}
+
+template <typename TI, typename TS>
+cudaError_t launch_decode128(const DecodeArgs &a, cudaStream_t stream) {
+#ifndef GDR_DEC_NSTG
+#define GDR_DEC_NSTG 3
+#define GDR_DEC_MINB 2
+#endif
+    constexpr int NW = 4, NSTG = sizeof(TS) == 2 ? GDR_DEC_NSTG : 2, MINB = GDR_DEC_MINB;
+    using Cf = D128<TI, TS, NW, NSTG>;
+    const long long ntiles = (long long)a.B * a.Nv;
+    if (ntiles == 0) return cudaSuccess;
+    EncodeTiledFn enc = tensor_map_encoder();
+    if (!enc) return cudaErrorInvalidValue;
+    CUtensorMap tm;
+    const cuuint64_t dims[3] = {(cuuint64_t)Cf::D, (cuuint64_t)Cf::D, (cuuint64_t)a.slots * (cuuint64_t)a.Nv};
+    const cuuint64_t strides[2] = {(cuuint64_t)Cf::D * sizeof(TS), (cuuint64_t)Cf::D * Cf::D * sizeof(TS)};
+    const cuuint32_t box[3] = {(cuuint32_t)Cf::BOXC, (cuuint32_t)Cf::D, 1}, es[3] = {1, 1, 1};
+    if (enc(&tm, sizeof(TS) == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, a.pool, dims,
+            strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return cudaErrorInvalidValue;
+    auto kern = decode128_kernel<TI, TS, NW, NSTG, MINB>;
+    const int smem = Cf::layout(a.S, a.gk != nullptr).smem;
+    static int attr_smem = 0, cached_smem = -1, grid_cap = 1;
+    if (smem > attr_smem) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e != cudaSuccess) return e;
+        attr_smem = smem;
+    }
+    if (smem != cached_smem) {
+        int dev = 0, nsm = 0, per_sm = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, Cf::NT, smem);
+        grid_cap = max(1, nsm * max(1, per_sm));
+        cached_smem = smem;
+    }
+    const int grid = (int)(ntiles < grid_cap ? ntiles : grid_cap);
+    kern<<<grid, Cf::NT, smem, stream>>>(tm, a, (int)ntiles);
+    return cudaGetLastError();
+}
+
 template <int DK, int DV, typename TI, typename TS>
 cudaError_t launch_decode_t(const DecodeArgs &a, cudaStream_t stream) {
     using Cf = DecodeCfg<DK, DV, TI, TS>;
@@ -397,6 +806,12 @@ cudaError_t launch_decode_t(const DecodeArgs &a, cudaStream_t stream) {
 
 template <int DK, int DV>
 cudaError_t launch_decode_d(const DecodeArgs &a, gdr_dtype dt, gdr_dtype st, cudaStream_t stream) {
+    if (DK == 128 && DV == 128) {
+        if (dt == GDR_BF16 && st == GDR_BF16) return launch_decode128<__nv_bfloat16, __nv_bfloat16>(a, stream);
+        if (dt == GDR_BF16 && st == GDR_F32) return launch_decode128<__nv_bfloat16, float>(a, stream);
+        if (dt == GDR_F32 && st == GDR_BF16) return launch_decode128<float, __nv_bfloat16>(a, stream);
+        return launch_decode128<float, float>(a, stream);
+    }
     if (dt == GDR_BF16 && st == GDR_BF16) return launch_decode_t<DK, DV, __nv_bfloat16, __nv_bfloat16>(a, stream);
     if (dt == GDR_BF16 && st == GDR_F32) return launch_decode_t<DK, DV, __nv_bfloat16, float>(a, stream);
     if (dt == GDR_F32 && st == GDR_BF16) return launch_decode_t<DK, DV, float, __nv_bfloat16>(a, stream);

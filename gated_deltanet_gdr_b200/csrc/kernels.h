@@ -1,6 +1,7 @@
 // kernels.h -- argument blocks and launchers of the device kernels (internal to libgdr.so).
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -41,6 +42,12 @@ struct ChunkArgs {
     const float *A_log, *dt_bias;
     unsigned int *err;
 };
+
+// cuTensorMapEncodeTiled, obtained once through the runtime's driver entry point (NULL if unavailable).
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn tensor_map_encoder();
 
 cudaError_t launch_decode(const DecodeArgs &a, int Dk, int Dv, gdr_dtype dt, gdr_dtype st, cudaStream_t s);
 bool chunk_tc_supported(int Dk, int Dv, gdr_dtype dt, int S);
