@@ -270,7 +270,9 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     uint64_t *bar_a1 = bars + 5, *bar_cq = bars + 6, *bar_ck = bars + 7, *bar_pf = bars + 8;
     // the tensor-core merges of the solve: rounds 0..2 on bar_sv (three phases per chunk), round 3 on bar_sv3
     uint64_t *bar_sv = bars + 10, *bar_sv3 = bars + 11;
-    constexpr int kNumBars = 12;
+    // bar_wr: the carry group has read W of its chunk out of the Gram columns of TMEM
+    uint64_t *bar_wr = bars + 12;
+    constexpr int kNumBars = 13;
     uint32_t *s_tmem = reinterpret_cast<uint32_t *>(bars + kNumBars);
     volatile int *s_abort = reinterpret_cast<volatile int *>(s_tmem + 1);
 
@@ -433,6 +435,8 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             if (named_sync_or(BAR_PCTL, NPC, to)) break;  // H0: chunk c staged (or a timeout)
             named_sync(BAR_PCTL, NPC);  // H1: padding rows zeroed
             if (lane == 0) {  // a2: the Gram [K; Q][K; Q]^T (its diagonal gives the row norms)
+                // the Gram columns hold W of chunk c-1 until the carry group has read it
+                if (c > 0 && !mbar_wait(bar_wr, (c - 1) & 1)) to = true;
                 tc_fence_after();
                 const uint32_t id = idesc_bf16(128, 128, false, false);
 #pragma unroll
@@ -531,6 +535,8 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             }
             named_sync(BAR_PREP, NGRP);
             PHASE(4);
+            // the TT area (which now takes plain A) is free once the W/U MMAs of chunk c-1 completed
+            if (c > 0) wait_ok(bar_wu, (c - 1) & 1);
             // A rows (lanes 0..63, fp32 for the solve) and Pm rows (lanes 64..127, bf16 operand of the
             // carry's o MMA), with the decay e^{G_t - G_s} taken per entry
             {
@@ -671,32 +677,11 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             if (c > 0 && !mbar_wait_sleep(bar_m2, (c - 1) & 1)) to = true;
             fence_proxy_async_smem();
             tc_fence_before();
-            // H2: the control warp issues W and U (rows 64..127 of TT K, rows 0..63 of TT V)
+            // H2: the control warp issues W and U (rows 64..127 of TT K, rows 0..63 of TT V); the chunk is
+            // handed over at once (the carry group waits for W and U itself and moves W into A1)
             if (named_sync_or(BAR_PCTL, NPC, to)) break;
-            PHASE(8);
-            wait_ok(bar_wu, par);
-            // rows 0..63 of A1 are free once the carry's MMA1 of chunk c-1 completed
-            if (c > 0) wait_ok(bar_m1, (c - 1) & 1);
-            tc_fence_after();
-            PHASE(9);
-            if (q4 >= 2) {  // W rows -> rows 0..63 of A1
-                const int t = row - 64;
-#pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    float w[32];
-                    tmem_ld32(tmem + TM_GPW + lane_base + 64 * hf + 32 * half, w);
-                    tmem_ld_wait();
-#pragma unroll
-                    for (int c8 = 0; c8 < 4; ++c8)
-                        *reinterpret_cast<uint4 *>(sm + OFF_A1 + hf * 16384 + blk_off(t, 32 * half + 8 * c8)) =
-                            pack8(&w[8 * c8]);
-                }
-            }
-            fence_proxy_async_smem();
-            tc_fence_before();
-            named_sync(BAR_PREP, NGRP);
             if (p == 0) mbar_arrive(bar_a1);
-            PHASE(10);
+            PHASE(8);
         }
         if (to && p == 0) *s_abort = 1;
     } else {
@@ -711,8 +696,27 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             const float *vec = vecs + par * NVEC * 64;
             if (!mbar_wait_sleep(bar_a1, par)) to = true;
             wait_ok(bar_cq, par);
+            wait_ok(bar_wu, par);
             if (named_sync_or(BAR_CARRY, NGRP, to)) { stop = true; break; }
             tc_fence_after();
+            if (q4 >= 2) {  // W rows (TMEM lanes 64..127 of the Gram columns) -> rows 0..63 of A1
+                const int t = row - 64;
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
+                    float w[32];
+                    tmem_ld32(tmem + TM_GPW + lane_base + 64 * hf + 32 * half, w);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int c8 = 0; c8 < 4; ++c8)
+                        *reinterpret_cast<uint4 *>(sm + OFF_A1 + hf * 16384 + blk_off(t, 32 * half + 8 * c8)) =
+                            pack8(&w[8 * c8]);
+                }
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            named_sync(BAR_CARRY, NGRP);
+            tc_fence_after();
+            if (tid == 0) mbar_arrive(bar_wr);
             PHASE(16);
             const int n = (int)vec[V_N * 64];
             const float eL = vec[V_EG * 64 + C - 1];
