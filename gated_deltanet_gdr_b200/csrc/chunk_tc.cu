@@ -86,14 +86,19 @@ constexpr uint32_t kTimeoutBit = 0x4u;
 constexpr int kStorer = 32;
 
 // ---- shared memory map (bytes from a 1024-aligned base) ----
-// input stage of the prep group: [K_b0 | Q_b0 | K_b1 | Q_b1 | V_b0 | V_b1], 64 rows x 128 B (64 bf16) each
-constexpr uint32_t OFF_K0 = 0, OFF_Q0 = 8192, OFF_K1 = 16384, OFF_Q1 = 24576, OFF_V0 = 32768;
-constexpr uint32_t STAGE_BYTES = 49152;
+// input tiles of the prep group, 64 rows x 128 B (64 bf16) each, per dk block b (b = 0, 1) at 24 KB b:
+// [K even chunk | Q | K odd chunk], so that [K; Q] (even chunks) and [Q; K] (odd chunks) are each one
+// 128-row operand for the Gram; the K tile is double-buffered so that the next chunk's K and Q can land
+// during the current chunk.  V (dv blocks at +0, +8K) is single-buffered: it is needed late.
+constexpr uint32_t KQ_BLK = 24576, OFF_V = 49152;
+__host__ __device__ constexpr uint32_t off_k(int par, int blk) { return blk * KQ_BLK + (par ? 16384u : 0u); }
+__host__ __device__ constexpr uint32_t off_q(int blk) { return blk * KQ_BLK + 8192u; }
+__host__ __device__ constexpr uint32_t off_gram(int par, int blk) { return blk * KQ_BLK + (par ? 8192u : 0u); }
 // operands of the carry group for the chunk it runs
-constexpr uint32_t OFF_A1 = 49152;   // [W; Q] K-major 128 x 128: dk blocks at +0, +16K (Q rows by TMA)
-constexpr uint32_t OFF_KT = 81920;   // raw K tile by TMA, MN-major (M = dk, K = tok): dk blocks at +0, +8K
-constexpr uint32_t OFF_S = 98304;    // S bf16, MN-major (K = dk rows, N = dv): dv blocks at +0, +16K
-constexpr uint32_t OFF_VS = 131072;  // diag(tail) v_new (MN-major, K = tok, N = dv): dv blocks at +0, +8K
+constexpr uint32_t OFF_A1 = 65536;   // [W; Q] K-major 128 x 128: dk blocks at +0, +16K (Q rows by TMA)
+constexpr uint32_t OFF_KT = 98304;   // K tile by TMA, scaled in place to diag(tail) K: MN-major (M = dk,
+                                     // K = tok), dk blocks at +0, +8K
+constexpr uint32_t OFF_S = 114688;   // S bf16, MN-major (K = dk rows, N = dv): dv blocks at +0, +16K
 // Pm (K-major 64 x 64), two buffers; the o MMA reads 128 rows starting 8 KB before the buffer so that
 // Pm forms rows 64..127 (rows 0..63 are whatever precedes it and land in dead accumulator lanes)
 constexpr uint32_t OFF_PM0 = 147456, OFF_PM1 = 155648;
@@ -123,8 +128,9 @@ static_assert(OFF_TT % 1024 == 0 && OFF_A21 % 1024 == 0 && OFF_T22 % 1024 == 0 &
 static_assert(OFF_T22 + 16384 <= SMEM_USED, "merge operand over-read stays in shared memory");
 static_assert(OFF_PM0 >= 8192 && OFF_PM1 == OFF_PM0 + 8192, "Pm buffers");
 
-// TMEM columns (all 128 lanes): the Gram [K; Q][K; Q]^T then W (lanes 64..127), U (lanes 0..63),
-// R = [W S; o] (lanes 0..63 / 64..127), the fp32 state S
+// TMEM columns (all 128 lanes): the Gram [K; Q][K; Q]^T (then the solve's merge products); U (lanes
+// 0..63); R: first W of the chunk (lanes 64..127, written while R is otherwise free), then [W S; o]
+// (lanes 0..63 / 64..127); the fp32 state S
 constexpr uint32_t TM_GPW = 0, TM_U = 128, TM_R = 256, TM_S = 384, TM_COLS = 512;
 
 // V_G2 = G log2(e); V_LAM = V_G2 - log2(1/|k|), so that e^{G_t - G_s} / |k_s| = 2^{V_G2[t] - V_LAM[s]};
@@ -263,16 +269,16 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const uint32_t sbase = smem_u32(sm);
     float *vecs = reinterpret_cast<float *>(sm + OFF_VEC);
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + OFF_BAR);
-    // bar_ld: input stage landed; bar_gp / bar_wu: the prep MMAs completed; bar_m1 / bar_m2: the carry MMAs
+    // bar_ld: K and Q of the chunk landed (bar_ldv: V); bar_gp / bar_wu: the prep MMAs completed; bar_m1 / bar_m2: the carry MMAs
     // completed; bar_a1: the prep group handed chunk c to the carry group; bar_cq / bar_ck: the raw Q rows
     // of A1 / the raw K tile landed; bar_pf[i]: the carry group is done with Pm buffer i and vector set i
     uint64_t *bar_ld = bars, *bar_gp = bars + 1, *bar_wu = bars + 2, *bar_m1 = bars + 3, *bar_m2 = bars + 4;
     uint64_t *bar_a1 = bars + 5, *bar_cq = bars + 6, *bar_ck = bars + 7, *bar_pf = bars + 8;
     // the tensor-core merges of the solve: rounds 0..2 on bar_sv (three phases per chunk), round 3 on bar_sv3
     uint64_t *bar_sv = bars + 10, *bar_sv3 = bars + 11;
-    // bar_wr: the carry group has read W of its chunk out of the Gram columns of TMEM
-    uint64_t *bar_wr = bars + 12;
-    constexpr int kNumBars = 13;
+    // bar_rf: the carry group has read the out rows of its chunk from TMEM R (where the next W MMA writes)
+    uint64_t *bar_rf = bars + 12, *bar_ldv = bars + 13;
+    constexpr int kNumBars = 14;
     uint32_t *s_tmem = reinterpret_cast<uint32_t *>(bars + kNumBars);
     volatile int *s_abort = reinterpret_cast<volatile int *>(s_tmem + 1);
 
@@ -372,15 +378,24 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             tma_prefetch_3d(&tm_v, 0, y, bh);
             tma_prefetch_3d(&tm_v, 64, y, bh);
         };
-        auto issue_loads = [&](int chunk) {
+        // K of a chunk into its buffer (this also arms the chunk's K/Q barrier), Q into the single Q buffer,
+        // V into the single V buffer
+        auto issue_k = [&](int chunk) {
+            const int y = chunk * C, pc = chunk & 1;
+            mbar_arrive_expect_tx(bar_ld, 32768);
+            tma_load_3d(sm + off_k(pc, 0), &tm_k, bar_ld, 0, y, zq);
+            tma_load_3d(sm + off_k(pc, 1), &tm_k, bar_ld, 64, y, zq);
+        };
+        auto issue_q = [&](int chunk) {
             const int y = chunk * C;
-            mbar_arrive_expect_tx(bar_ld, STAGE_BYTES);
-            tma_load_3d(sm + OFF_K0, &tm_k, bar_ld, 0, y, zq);
-            tma_load_3d(sm + OFF_K1, &tm_k, bar_ld, 64, y, zq);
-            tma_load_3d(sm + OFF_Q0, &tm_q, bar_ld, 0, y, zq);
-            tma_load_3d(sm + OFF_Q1, &tm_q, bar_ld, 64, y, zq);
-            tma_load_3d(sm + OFF_V0, &tm_v, bar_ld, 0, y, bh);
-            tma_load_3d(sm + OFF_V0 + 8192, &tm_v, bar_ld, 64, y, bh);
+            tma_load_3d(sm + off_q(0), &tm_q, bar_ld, 0, y, zq);
+            tma_load_3d(sm + off_q(1), &tm_q, bar_ld, 64, y, zq);
+        };
+        auto issue_v = [&](int chunk) {
+            const int y = chunk * C;
+            mbar_arrive_expect_tx(bar_ldv, 16384);
+            tma_load_3d(sm + OFF_V, &tm_v, bar_ldv, 0, y, bh);
+            tma_load_3d(sm + OFF_V + 8192, &tm_v, bar_ldv, 64, y, bh);
         };
         // The gate and beta vectors of a chunk, which need no Gram: beta (from logits), the cumulative
         // gate G (from the raw gate), e^G, G log2(e), e^{G_last - G} and the valid-token count; two
@@ -426,7 +441,9 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         bool to = false;
         if (nvalid > 0) chunk_vectors(0);
         if (lane == 1 && nvalid > 0) {
-            issue_loads(0);
+            issue_k(0);
+            issue_q(0);
+            issue_v(0);
             if (nvalid > 1) prefetch_l2(1);
         }
         __syncwarp();
@@ -434,17 +451,29 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             const uint32_t par = c & 1;
             if (named_sync_or(BAR_PCTL, NPC, to)) break;  // H0: chunk c staged (or a timeout)
             named_sync(BAR_PCTL, NPC);  // H1: padding rows zeroed
-            if (lane == 0) {  // a2: the Gram [K; Q][K; Q]^T (its diagonal gives the row norms)
-                // the Gram columns hold W of chunk c-1 until the carry group has read it
-                if (c > 0 && !mbar_wait(bar_wr, (c - 1) & 1)) to = true;
+            if (lane == 0) {  // a2: the Gram [K; Q][K; Q]^T ([Q; K][Q; K]^T for odd chunks); its diagonal gives
+                              // the row norms
                 tc_fence_after();
                 const uint32_t id = idesc_bf16(128, 128, false, false);
 #pragma unroll
                 for (int k = 0; k < 8; ++k) {
-                    const uint32_t addr = sbase + OFF_K0 + (k >> 2) * 16384 + (k & 3) * 32;
+                    const uint32_t addr = sbase + off_gram(par, k >> 2) + (k & 3) * 32;
                     mma_bf16(tmem + TM_GPW, sdesc_sw128(addr, 16, 1024), sdesc_sw128(addr, 16, 1024), id, k > 0);
                 }
                 mma_commit(bar_gp);
+            }
+            if (lane == 1) {
+                // V and the other K buffer were last read by the W/U MMAs of chunk c-1, issued a whole chunk
+                // ago; V of this chunk is needed only at its own W/U MMAs, K and Q of the next chunk at its
+                // Gram.  Q is free once this chunk's Gram has read it.
+                if (c > 0 && !mbar_wait(bar_wu, (c - 1) & 1)) to = true;
+                if (c > 0) issue_v(c);
+                if (c + 1 < nvalid) {
+                    issue_k(c + 1);
+                    if (mbar_wait(bar_gp, par)) issue_q(c + 1);
+                    else to = true;
+                    if (c + 2 < nvalid) prefetch_l2(c + 2);
+                }
             }
             __syncwarp();
             // while the prep group solves chunk c: the vectors of chunk c+1, into the set that chunk c-1
@@ -455,24 +484,19 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             }
             __syncwarp();
             if (named_sync_or(BAR_PCTL, NPC, to)) break;  // H2: TT operand in place, TMEM U free
-            if (lane == 0) {  // a4: W (rows 64..127 of TT K) and U (rows 0..63 of TT V)
+            if (lane == 0) {  // a4: W (rows 64..127 of TT K, into TMEM R) and U (rows 0..63 of TT V)
+                if (!mbar_wait(bar_ldv, par)) to = true;
+                // R holds the out rows of chunk c-1 until the carry group has read them
+                if (c > 0 && !mbar_wait(bar_rf, (c - 1) & 1)) to = true;
                 tc_fence_after();
                 const uint32_t id = idesc_bf16(128, 128, false, true);
 #pragma unroll
                 for (int k = 0; k < 4; ++k) {
                     const uint64_t ad = sdesc_sw128(sbase + OFF_TT + k * 32, 16, 1024);
-                    mma_bf16(tmem + TM_GPW, ad, sdesc_sw128(sbase + OFF_K0 + k * 2048, 16384, 1024), id, k > 0);
-                    mma_bf16(tmem + TM_U, ad, sdesc_sw128(sbase + OFF_V0 + k * 2048, 8192, 1024), id, k > 0);
+                    mma_bf16(tmem + TM_R, ad, sdesc_sw128(sbase + off_k(par, 0) + k * 2048, KQ_BLK, 1024), id, k > 0);
+                    mma_bf16(tmem + TM_U, ad, sdesc_sw128(sbase + OFF_V + k * 2048, 8192, 1024), id, k > 0);
                 }
                 mma_commit(bar_wu);
-            }
-            if (lane == 1 && c + 1 < nvalid) {  // the stage is consumed once W and U are done
-                if (mbar_wait(bar_wu, par)) {
-                    issue_loads(c + 1);
-                    if (c + 2 < nvalid) prefetch_l2(c + 2);
-                } else {
-                    to = true;
-                }
             }
             __syncwarp();
         }
@@ -495,10 +519,11 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             wait_ok(bar_ld, par);
             if (named_sync_or(BAR_PCTL, NPC, to)) break;  // H0 (the vectors of chunk c were written before H2 of c-1)
             PHASE(0);
-            if (n < C) {  // padding rows of the last chunk: zero them so no padding value reaches a product
-                for (int e = p; e < (C - n) * 48; e += NGRP) {
-                    const int r = n + e / 48, k = e % 48;
-                    *reinterpret_cast<uint4 *>(sm + (k >> 3) * 8192 + r * 128 + (k & 7) * 16) = make_uint4(0, 0, 0, 0);
+            if (n < C) {  // padding rows of the last chunk's K and Q: zero them so no padding value reaches a product
+                for (int e = p; e < (C - n) * 32; e += NGRP) {
+                    const int r = n + e / 32, k = e % 32, tile = k >> 3;
+                    const uint32_t base = (tile & 1) ? off_q(tile >> 1) : off_k(par, tile >> 1);
+                    *reinterpret_cast<uint4 *>(sm + base + r * 128 + (k & 7) * 16) = make_uint4(0, 0, 0, 0);
                 }
                 fence_proxy_async_smem();
             }
@@ -510,19 +535,24 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             // Each thread takes its Gram row's 32 columns of [K; Q] K^T (lanes 0..63: k_t.k_s, lanes
             // 64..127: q_t.k_s); the blocks wholly above the diagonal are never read.  The diagonal
             // gives |k_t|^2 and (from the q_t.q_s columns) |q_t|^2.
-            const bool need = !((q4 & 1) == 0 && hf == 1);
-            if ((q4 < 2 && hf == q4) || (q4 >= 2 && hf == q4 - 2)) {
-                // |k_t|^2 at column t (lanes 0..63), |q_t|^2 at column 64 + t (lanes 64..127): the diagonal
-                // element of this thread's row is entry `lane` of the 32 columns its warp loads
+            // Even chunks: TMEM lanes 0..63 hold the k rows and 64..127 the q rows, columns 0..63 the k
+            // columns; odd chunks ([Q; K]) swap both.  A warp of the "k role" builds rows of A, one of the
+            // "q role" rows of Pm; qa is the 32-row block of the chunk its lanes cover.
+            const bool krole = (q4 >> 1) == (int)par;
+            const int qa = q4 & 1, kcol = par ? 64 : 0, qcol = par ? 0 : 64;
+            const bool need = !(qa == 0 && hf == 1);
+            if (qa == hf) {
+                // |k_t|^2 / |q_t|^2 is the diagonal entry of this thread's row: entry `lane` of the 32 columns
+                // its warp loads
                 float d32[32];
-                tmem_ld32(tmem + TM_GPW + lane_base + (q4 >= 2 ? 64 : 0) + 32 * hf, d32);
+                tmem_ld32(tmem + TM_GPW + lane_base + (krole ? kcol : qcol) + 32 * hf, d32);
                 tmem_ld_wait();
                 float d = 0.f;
 #pragma unroll
                 for (int j = 0; j < 32; ++j) d = (j == lane) ? d32[j] : d;
                 const int t = row & 63;
                 const float r = t < n ? (a.l2norm ? rsqrtf(d + a.eps) : 1.f) : 0.f;
-                if (q4 < 2) {
+                if (krole) {
                     vRk[t] = r;
                     vec[V_TAIL * 64 + t] = vec[V_ET * 64 + t] * r;
                     vCw[t] = vBeta[t] * vEG[t] * r;
@@ -537,16 +567,16 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             PHASE(4);
             // the TT area (which now takes plain A) is free once the W/U MMAs of chunk c-1 completed
             if (c > 0) wait_ok(bar_wu, (c - 1) & 1);
-            // A rows (lanes 0..63, fp32 for the solve) and Pm rows (lanes 64..127, bf16 operand of the
-            // carry's o MMA), with the decay e^{G_t - G_s} taken per entry
+            // A rows (k role, fp32 for the solve) and Pm rows (q role, bf16 operand of the carry's o MMA), with
+            // the decay e^{G_t - G_s} taken per entry
             {
                 const int t = row & 63;
                 if (need) {
                     float v[32];
-                    tmem_ld32(tmem + TM_GPW + lane_base + 32 * hf, v);
+                    tmem_ld32(tmem + TM_GPW + lane_base + kcol + 32 * hf, v);
                     const float g2t = vec[V_G2 * 64 + t];
                     // row factor: beta_t / |k_t| for A, scale / |q_t| for Pm (zero past the length)
-                    const float rf = t < n ? (q4 < 2 ? vBeta[t] * vRk[t] : vRq[t]) : 0.f;
+                    const float rf = t < n ? (krole ? vBeta[t] * vRk[t] : vRq[t]) : 0.f;
                     const float4 *lam4 = reinterpret_cast<const float4 *>(vec + V_LAM * 64 + 32 * hf);
                     tmem_ld_wait();
 #pragma unroll
@@ -557,14 +587,14 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                         v[4 * j4 + 2] *= rf * ex2_approx(g2t - l.z);
                         v[4 * j4 + 3] *= rf * ex2_approx(g2t - l.w);
                     }
-                    if (q4 < 2 && hf == q4) {
+                    if (krole && hf == qa) {
                         // a diagonal 32 x 32 block, plain (entries on or above the diagonal are never read)
                         float *ap = reinterpret_cast<float *>(sm + OFF_AP) + pl(t, 0);
 #pragma unroll
                         for (int j4 = 0; j4 < 8; ++j4)
                             *reinterpret_cast<float4 *>(ap + 4 * j4) =
                                 make_float4(v[4 * j4], v[4 * j4 + 1], v[4 * j4 + 2], v[4 * j4 + 3]);
-                    } else if (q4 < 2) {  // A21 (rows 32..63, columns 0..31), operand of the tf32 merge
+                    } else if (krole) {  // A21 (rows 32..63, columns 0..31), operand of the tf32 merge
 #pragma unroll
                         for (int j4 = 0; j4 < 8; ++j4)
                             *reinterpret_cast<float4 *>(sm + OFF_A21 + f32_off(t - 32, 4 * j4)) =
@@ -576,7 +606,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                         for (int c8 = 0; c8 < 4; ++c8)
                             *reinterpret_cast<uint4 *>(pm + blk_off(t, 32 * hf + 8 * c8)) = pack8(&v[8 * c8]);
                     }
-                } else if (q4 >= 2) {  // Pm rows 0..31, columns 32..63: above the diagonal
+                } else if (!krole) {  // Pm rows 0..31, columns 32..63: above the diagonal
 #pragma unroll
                     for (int c8 = 0; c8 < 4; ++c8)
                         *reinterpret_cast<uint4 *>(pm + blk_off(t, 32 + 8 * c8)) = make_uint4(0, 0, 0, 0);
@@ -673,6 +703,13 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             }
             PHASE(6);
             PHASE(7);
+            if (n < C) {  // padding rows of the last chunk's V, once it has landed
+                wait_ok(bar_ldv, par);
+                for (int e = p; e < (C - n) * 16; e += NGRP) {
+                    const int r = n + e / 16, k = e % 16;
+                    *reinterpret_cast<uint4 *>(sm + OFF_V + (k >> 3) * 8192 + r * 128 + (k & 7) * 16) = make_uint4(0, 0, 0, 0);
+                }
+            }
             // TMEM U is free once the carry group read U of chunk c-1 (its v_new epilogue precedes MMA2)
             if (c > 0 && !mbar_wait_sleep(bar_m2, (c - 1) & 1)) to = true;
             fence_proxy_async_smem();
@@ -699,12 +736,12 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             wait_ok(bar_wu, par);
             if (named_sync_or(BAR_CARRY, NGRP, to)) { stop = true; break; }
             tc_fence_after();
-            if (q4 >= 2) {  // W rows (TMEM lanes 64..127 of the Gram columns) -> rows 0..63 of A1
+            if (q4 >= 2) {  // W rows (TMEM lanes 64..127 of R) -> rows 0..63 of A1
                 const int t = row - 64;
 #pragma unroll
                 for (int half = 0; half < 2; ++half) {
                     float w[32];
-                    tmem_ld32(tmem + TM_GPW + lane_base + 64 * hf + 32 * half, w);
+                    tmem_ld32(tmem + TM_R + lane_base + 64 * hf + 32 * half, w);
                     tmem_ld_wait();
 #pragma unroll
                     for (int c8 = 0; c8 < 4; ++c8)
@@ -716,7 +753,6 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             tc_fence_before();
             named_sync(BAR_CARRY, NGRP);
             tc_fence_after();
-            if (tid == 0) mbar_arrive(bar_wr);
             PHASE(16);
             const int n = (int)vec[V_N * 64];
             const float eL = vec[V_EG * 64 + C - 1];
@@ -748,6 +784,24 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 }
                 tmem_st_wait();
             }
+            // meanwhile: the K tile -> K~ = diag(e^{G_last - G} / |k|) K in place (rows past the length, whatever
+            // they hold, become zero), the A operand of the state update
+            wait_ok(bar_ck, par);
+            {
+                const float *vtail = vec + V_TAIL * 64;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int e = tid + i * NGRP, t = (e >> 3) & 63;
+                    uint4 *pk = reinterpret_cast<uint4 *>(sm + OFF_KT + (e >> 9) * 8192 + t * 128 + (e & 7) * 16);
+                    float f[8];
+                    unpack8(*pk, f);
+                    const float sc = vtail[t];
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) f[j] = t < n ? f[j] * sc : 0.f;
+                    *pk = pack8(f);
+                }
+            }
+            fence_proxy_async_smem();
             wait_ok(bar_m1, par);
             if (tid == 0 && c + 1 < nvalid) load_carry_q(c + 1);  // the Q rows of A1 are read
             if (tid == kStorer) bulk_wait_read0();  // the previous out tile (same buffer as v_new) is read
@@ -755,9 +809,8 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             if (named_sync_or(BAR_CARRY, NGRP, to)) { stop = true; break; }
             tc_fence_after();
             PHASE(17);
-            if (q4 < 2) {  // v_new = U - W S for token t, dv columns [64 hf, +64); also diag(tail) v_new
+            if (q4 < 2) {  // v_new = U - W S for token t, dv columns [64 hf, +64)
                 const int t = row;
-                const float tl = vec[V_TAIL * 64 + t];
 #pragma unroll
                 for (int half = 0; half < 2; ++half) {
                     float u[32], r[32];
@@ -769,12 +822,6 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 #pragma unroll
                     for (int c8 = 0; c8 < 4; ++c8)
                         *reinterpret_cast<uint4 *>(sm + OFF_VO + hf * 8192 + blk_off(t, 32 * half + 8 * c8)) =
-                            pack8(&u[8 * c8]);
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) u[j] *= tl;
-#pragma unroll
-                    for (int c8 = 0; c8 < 4; ++c8)
-                        *reinterpret_cast<uint4 *>(sm + OFF_VS + hf * 8192 + blk_off(t, 32 * half + 8 * c8)) =
                             pack8(&u[8 * c8]);
                 }
             } else {  // rows of Q S: scale by e^{G_t} scale / |q_t| before Pm v_new accumulates onto them
@@ -791,19 +838,12 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 }
                 tmem_st_wait();
             }
-            wait_ok(bar_ck, par);
-            if (n < C) {  // rows of the raw K tile past the length (any content) must not reach S
-                for (int e = tid; e < (C - n) * 16; e += NGRP) {
-                    const int r = n + (e >> 4), blk = (e >> 3) & 1, ch = e & 7;
-                    *reinterpret_cast<uint4 *>(sm + OFF_KT + blk * 8192 + r * 128 + ch * 16) = make_uint4(0, 0, 0, 0);
-                }
-            }
             fence_proxy_async_smem();
             tc_fence_before();
             if (named_sync_or(BAR_CARRY, NGRP, to)) { stop = true; break; }
             tc_fence_after();
             PHASE(18);
-            // ---- S += K^T (diag(tail) v_new) ;  R[64:128] += Pm v_new ----
+            // ---- S += K~^T v_new ;  R[64:128] += Pm v_new ----
             if (tid == 0) {
                 const uint32_t id_s = idesc_bf16(128, 128, true, true);
                 const uint32_t id_o = idesc_bf16(128, 128, false, true);
@@ -811,7 +851,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 TIMED(24, {
                     _Pragma("unroll")
                     for (int k = 0; k < 4; ++k) {
-                        const uint64_t bd = sdesc_sw128(sbase + OFF_VS + k * 2048, 8192, 1024);
+                        const uint64_t bd = sdesc_sw128(sbase + OFF_VO + k * 2048, 8192, 1024);
                         mma_bf16(tmem + TM_S, sdesc_sw128(sbase + OFF_KT + k * 2048, 8192, 1024), bd, id_s, 1);
                     }
                     _Pragma("unroll")
@@ -868,6 +908,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             tc_fence_before();
             named_sync(BAR_CARRY, NGRP);
             tc_fence_after();
+            if (tid == 0) mbar_arrive(bar_rf);  // R is read: the W MMA of chunk c+1 may write it
             if (tid == kStorer) {
                 tma_store_3d(&tm_o, sm + OFF_VO, 0, c * C, bh);
                 tma_store_3d(&tm_o, sm + OFF_VO + 8192, 64, c * C, bh);
