@@ -390,7 +390,7 @@ def bench_decode(gdr, name, args, world, rank, clk, flush, stream, peaks, rotate
             "us_per_call": d_ms * 1e3, "steps_per_s": world * 1e3 / d_ms,
             "state_GBps": gbs, "state_frac_of_hbm": gbs / peaks["hbm_gbs"],
             "roofline": {"bound": "hbm", "achieved": tot, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                         "frac": tot / peaks["hbm_gbs"], "traffic": profiled_traffic("decode"),
+                         "frac": tot / peaks["hbm_gbs"], "traffic": profiled_traffic(name),
                          "algorithmic_bytes_per_launch": nb["state"] + nb["io"]}}, args.steps
 
 
