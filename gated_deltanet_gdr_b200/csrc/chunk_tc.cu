@@ -276,8 +276,8 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     uint64_t *bar_a1 = bars + 5, *bar_cq = bars + 6, *bar_ck = bars + 7, *bar_pf = bars + 8;
     // the tensor-core merges of the solve: rounds 0..2 on bar_sv (three phases per chunk), round 3 on bar_sv3
     uint64_t *bar_sv = bars + 10, *bar_sv3 = bars + 11;
-    // bar_rf: the carry group has read the out rows of its chunk from TMEM R (where the next W MMA writes)
-    uint64_t *bar_rf = bars + 12, *bar_ldv = bars + 13;
+    // bar_vr: the control warp has written the gate vectors of the next chunk (one phase per chunk)
+    uint64_t *bar_vr = bars + 12, *bar_ldv = bars + 13;
     constexpr int kNumBars = 14;
     uint32_t *s_tmem = reinterpret_cast<uint32_t *>(bars + kNumBars);
     volatile int *s_abort = reinterpret_cast<volatile int *>(s_tmem + 1);
@@ -449,10 +449,11 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         __syncwarp();
         for (int c = 0; c < nvalid; ++c) {
             const uint32_t par = c & 1;
-            if (named_sync_or(BAR_PCTL, NPC, to)) break;  // H0: chunk c staged (or a timeout)
-            named_sync(BAR_PCTL, NPC);  // H1: padding rows zeroed
+            // H0: the prep group is at chunk c (and, for a last partial chunk, has zeroed its padding rows)
+            if (named_sync_or(BAR_PCTL, NPC, to)) break;
             if (lane == 0) {  // a2: the Gram [K; Q][K; Q]^T ([Q; K][Q; K]^T for odd chunks); its diagonal gives
                               // the row norms
+                if (!mbar_wait(bar_ld, par)) to = true;
                 tc_fence_after();
                 const uint32_t id = idesc_bf16(128, 128, false, false);
 #pragma unroll
@@ -469,6 +470,9 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 if (c > 0 && !mbar_wait(bar_wu, (c - 1) & 1)) to = true;
                 if (c > 0) issue_v(c);
                 if (c + 1 < nvalid) {
+                    // the K/Q barrier is armed for chunk c+1 only after its phase for chunk c has completed (an
+                    // arrival on a phase still pending would count towards that phase)
+                    if (!mbar_wait(bar_ld, par)) to = true;
                     issue_k(c + 1);
                     if (mbar_wait(bar_gp, par)) issue_q(c + 1);
                     else to = true;
@@ -483,22 +487,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 chunk_vectors(c + 1);
             }
             __syncwarp();
-            if (named_sync_or(BAR_PCTL, NPC, to)) break;  // H2: TT operand in place, TMEM U free
-            if (lane == 0) {  // a4: W (rows 64..127 of TT K, into TMEM R) and U (rows 0..63 of TT V)
-                if (!mbar_wait(bar_ldv, par)) to = true;
-                // R holds the out rows of chunk c-1 until the carry group has read them
-                if (c > 0 && !mbar_wait(bar_rf, (c - 1) & 1)) to = true;
-                tc_fence_after();
-                const uint32_t id = idesc_bf16(128, 128, false, true);
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    const uint64_t ad = sdesc_sw128(sbase + OFF_TT + k * 32, 16, 1024);
-                    mma_bf16(tmem + TM_R, ad, sdesc_sw128(sbase + off_k(par, 0) + k * 2048, KQ_BLK, 1024), id, k > 0);
-                    mma_bf16(tmem + TM_U, ad, sdesc_sw128(sbase + OFF_V + k * 2048, 8192, 1024), id, k > 0);
-                }
-                mma_commit(bar_wu);
-            }
-            __syncwarp();
+            if (lane == 0 && c + 1 < nvalid) mbar_arrive(bar_vr);
         }
     } else if (!carry) {
         // =============================== prep group ===============================
@@ -515,11 +504,11 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             uint8_t *pm = sm + (par ? OFF_PM1 : OFF_PM0);
             const int n = min(C, L - c * C);
             // Pm buffer `par` and the norm vectors of set `par` were last read for chunk c-2, before its MMA2
-            if (c >= 2 && !mbar_wait_sleep(bar_pf + par, ((c >> 1) + 1) & 1)) to = true;
-            wait_ok(bar_ld, par);
-            if (named_sync_or(BAR_PCTL, NPC, to)) break;  // H0 (the vectors of chunk c were written before H2 of c-1)
-            PHASE(0);
+            // Pm buffer `par` and the norm vectors of set `par` were last read for chunk c-2, before its MMA2;
+            // the control warp waited for that MMA2 before it wrote chunk c's gate vectors, ahead of H0.
+            PHASE(26);
             if (n < C) {  // padding rows of the last chunk's K and Q: zero them so no padding value reaches a product
+                wait_ok(bar_ld, par);
                 for (int e = p; e < (C - n) * 32; e += NGRP) {
                     const int r = n + e / 32, k = e % 32, tile = k >> 3;
                     const uint32_t base = (tile & 1) ? off_q(tile >> 1) : off_k(par, tile >> 1);
@@ -527,8 +516,9 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 }
                 fence_proxy_async_smem();
             }
-            named_sync(BAR_PCTL, NPC);  // H1: the control warp issues the Gram
-            PHASE(1);
+            // H0: the control warp (which wrote chunk c's gate vectors during chunk c-1) issues the Gram
+            if (named_sync_or(BAR_PCTL, NPC, to)) break;
+            PHASE(0);
             wait_ok(bar_gp, par);
             tc_fence_after();
             PHASE(3);
@@ -563,10 +553,10 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     vec[V_XS * 64 + t] = vEG[t] * a.scale * r;
                 }
             }
+            // the TT area (which takes plain A next) is free once the W/U MMAs of chunk c-1 completed
+            if (p == 0 && c > 0) wait_ok(bar_wu, (c - 1) & 1);
             named_sync(BAR_PREP, NGRP);
             PHASE(4);
-            // the TT area (which now takes plain A) is free once the W/U MMAs of chunk c-1 completed
-            if (c > 0) wait_ok(bar_wu, (c - 1) & 1);
             // A rows (k role, fp32 for the solve) and Pm rows (q role, bf16 operand of the carry's o MMA), with
             // the decay e^{G_t - G_s} taken per entry
             {
@@ -710,13 +700,11 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     *reinterpret_cast<uint4 *>(sm + OFF_V + (k >> 3) * 8192 + r * 128 + (k & 7) * 16) = make_uint4(0, 0, 0, 0);
                 }
             }
-            // TMEM U is free once the carry group read U of chunk c-1 (its v_new epilogue precedes MMA2)
-            if (c > 0 && !mbar_wait_sleep(bar_m2, (c - 1) & 1)) to = true;
+            // hand the chunk over: the carry group issues W and U from TT (it owns TMEM R and U, so they are
+            // free in its own program order), waits for them and moves W into A1
             fence_proxy_async_smem();
             tc_fence_before();
-            // H2: the control warp issues W and U (rows 64..127 of TT K, rows 0..63 of TT V); the chunk is
-            // handed over at once (the carry group waits for W and U itself and moves W into A1)
-            if (named_sync_or(BAR_PCTL, NPC, to)) break;
+            named_sync(BAR_PREP, NGRP);
             if (p == 0) mbar_arrive(bar_a1);
             PHASE(8);
         }
@@ -733,8 +721,20 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             const float *vec = vecs + par * NVEC * 64;
             if (!mbar_wait_sleep(bar_a1, par)) to = true;
             wait_ok(bar_cq, par);
-            wait_ok(bar_wu, par);
             if (named_sync_or(BAR_CARRY, NGRP, to)) { stop = true; break; }
+            if (tid == 0) {  // a4: W (rows 64..127 of TT K, into TMEM R) and U (rows 0..63 of TT V)
+                if (!mbar_wait(bar_ldv, par)) to = true;
+                tc_fence_after();
+                const uint32_t id = idesc_bf16(128, 128, false, true);
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const uint64_t ad = sdesc_sw128(sbase + OFF_TT + k * 32, 16, 1024);
+                    mma_bf16(tmem + TM_R, ad, sdesc_sw128(sbase + off_k(par, 0) + k * 2048, KQ_BLK, 1024), id, k > 0);
+                    mma_bf16(tmem + TM_U, ad, sdesc_sw128(sbase + OFF_V + k * 2048, 8192, 1024), id, k > 0);
+                }
+                mma_commit(bar_wu);
+            }
+            wait_ok(bar_wu, par);
             tc_fence_after();
             if (q4 >= 2) {  // W rows (TMEM lanes 64..127 of R) -> rows 0..63 of A1
                 const int t = row - 64;
@@ -838,6 +838,14 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 }
                 tmem_st_wait();
             }
+            // e^{G_last} of the next chunk (for the state written back after MMA2), read before this chunk's MMA2:
+            // the control warp cannot get two chunks ahead of it then
+            const bool more = c + 1 < nvalid;
+            float eLn = 1.f;
+            if (more) {
+                wait_ok(bar_vr, par);
+                eLn = vecs[(par ^ 1) * NVEC * 64 + V_EG * 64 + C - 1];
+            }
             fence_proxy_async_smem();
             tc_fence_before();
             if (named_sync_or(BAR_CARRY, NGRP, to)) { stop = true; break; }
@@ -870,8 +878,6 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             PHASE(19);
             // ---- S (fp32, TMEM) -> bf16 operand tile, and back to TMEM scaled by e^{G_last} of the next
             // chunk (its gate vectors were written before this chunk was handed over);  o rows -> out tile ----
-            const bool more = c + 1 < nvalid;
-            const float eLn = more ? vecs[(par ^ 1) * NVEC * 64 + V_EG * 64 + C - 1] : 1.f;
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
                 float v[32];
@@ -908,7 +914,6 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             tc_fence_before();
             named_sync(BAR_CARRY, NGRP);
             tc_fence_after();
-            if (tid == 0) mbar_arrive(bar_rf);  // R is read: the W MMA of chunk c+1 may write it
             if (tid == kStorer) {
                 tma_store_3d(&tm_o, sm + OFF_VO, 0, c * C, bh);
                 tma_store_3d(&tm_o, sm + OFF_VO + 8192, 64, c * C, bh);
