@@ -7,9 +7,10 @@
 //
 //   a1  G_t = cumulative log-gate (tokens past the length count 0).
 //   a2  [G; P] = [K; Q] K^T                       tcgen05.mma  M=128 N=64  K=128
-//   a3  A = strictLower(beta_t k_t.k_s e^{G_t-G_s});  T = (I + A)^{-1} in fp32 on the CUDA
-//       cores: 16x16 diagonal blocks by forward substitution, merged 16 -> 32 -> 64 with
-//       T21 = -T22 A21 T11 (register-blocked, fully unrolled).
+//   a3  A = strictLower(beta_t k_t.k_s e^{G_t-G_s});  T = (I + A)^{-1}: 16x16 diagonal blocks by
+//       forward substitution and the 16 -> 32 merges T21 = -T22 A21 T11 in fp32 on the CUDA
+//       cores, the 32 -> 64 merge with warp-level tf32 tensor-core MMAs (mma.sync m16n8k8,
+//       operands and products in registers).
 //   a4  W = T diag(beta e^G) K,  U = T diag(beta) V        tcgen05.mma  M=128 N=128 K=64
 //   a5  R = [W; diag(e^G) X] S                    tcgen05.mma  M=128 N=128 K=128
 //       v_new = U - R[0:64]
@@ -79,8 +80,6 @@ constexpr int C = 64, D = 128, NGRP = 256, NT = 2 * NGRP + 32, NPC = NGRP + 32;
 constexpr int CTL_WARP = 16;
 // BAR_PCTL: the prep warps and the control warp, at the hand-offs between them
 constexpr int BAR_CARRY = 1, BAR_PREP = 2, BAR_PCTL = 3;
-// BAR_SOLVE: prep warps 8 and 9, which move the merge products of the solve between TMEM and shared memory
-constexpr int BAR_SOLVE = 4;
 constexpr uint32_t kTimeoutBit = 0x4u;
 // carry thread that issues the out-tile TMA stores (thread 0 issues the carry's MMAs)
 constexpr int kStorer = 32;
@@ -110,22 +109,18 @@ constexpr uint32_t OFF_TT = 180224;   // TT = [T diag(beta); T diag(c_W)], bf16,
 constexpr uint32_t OFF_AP = OFF_TT;              // A11, A22 (plain, 2 x 32 rows of SP floats)
 constexpr uint32_t OFF_XP = OFF_TT + 64 * SP * 4;  // 16 x 16 merge scratch (2 x 16 rows of SP floats)
 constexpr uint32_t OFF_TP = 196608;   // T11, T22 (plain, 2 x 32 rows of SP floats)
-constexpr uint32_t OFF_A21 = 205824;  // A rows 32..63, columns 0..31 (fp32, f32_off layout, 32 rows)
-constexpr uint32_t OFF_T22 = 209920;  // T22 (fp32, f32_off layout, 32 rows)
-constexpr uint32_t OFF_T11 = 214016;  // T11 (fp32, b32_off layout)
-constexpr uint32_t OFF_XB = 218112;   // X = A21 T11 (fp32, b32_off layout)
+constexpr uint32_t OFF_A21 = 205824;  // A rows 32..63, columns 0..31 (plain, 32 rows of SP floats)
+constexpr uint32_t OFF_XM = 210432;   // X = A21 T11 of the 32 -> 64 merge (plain, 32 rows of SP floats)
 static_assert(OFF_XP + 32 * SP * 4 <= OFF_TT + 16384, "plain A and the merge scratch fit in the TT area");
-static_assert(OFF_TP + 64 * SP * 4 <= OFF_A21, "plain T");
+static_assert(OFF_TP + 64 * SP * 4 <= OFF_A21 && OFF_A21 + 32 * SP * 4 <= OFF_XM, "plain T, A21");
 constexpr int NVEC = 12;             // per-chunk vectors of 64 floats (enum below)
-constexpr uint32_t OFF_VEC = OFF_XB + 4096;  // 2 sets x NVEC vectors x 64 floats
+constexpr uint32_t OFF_VEC = 215040;  // 2 sets x NVEC vectors x 64 floats
+static_assert(OFF_XM + 32 * SP * 4 <= OFF_VEC, "merge product");
 constexpr uint32_t OFF_BAR = OFF_VEC + 2 * NVEC * 64 * 4;
 constexpr uint32_t SMEM_USED = OFF_BAR + 128;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;  // + alignment slack
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
-static_assert(OFF_TT % 1024 == 0 && OFF_A21 % 1024 == 0 && OFF_T22 % 1024 == 0 && OFF_T11 % 1024 == 0 &&
-                  OFF_XB % 1024 == 0, "swizzle atoms");
-// the M = 128 merge MMAs read 96 rows of 128 bytes past A21 and T22 (their output lanes are not used)
-static_assert(OFF_T22 + 16384 <= SMEM_USED, "merge operand over-read stays in shared memory");
+static_assert(OFF_TT % 1024 == 0, "swizzle atoms");
 static_assert(OFF_PM0 >= 8192 && OFF_PM1 == OFF_PM0 + 8192, "Pm buffers");
 
 // TMEM columns (all 128 lanes): the Gram [K; Q][K; Q]^T (then the solve's merge products); U (lanes
@@ -184,19 +179,37 @@ __device__ __forceinline__ uint4 pack8(const float *f) {
                       pack_bf16x2(f[6], f[7]));
 }
 
-// Byte offset of element (r, s) of a 64 x 64 fp32 matrix stored as two column blocks (s < 32 at +0,
-// s >= 32 at +8 KB), each 64 rows of 128 bytes in the 128-byte-swizzled canonical layout (16-byte chunk
-// index XOR r % 8), so that kind::tf32 MMAs read row blocks as K-major and column blocks as MN-major operands.
-__device__ __forceinline__ uint32_t f32_off(int r, int s) {
-    return (uint32_t)((s >> 5) * 8192 + (r >> 3) * 1024 + (r & 7) * 128 + ((((s >> 2) & 7) ^ (r & 7)) << 4) +
-                      (s & 3) * 4);
+// D (16 x 8) += A (16 x 8) B (8 x 8) with tf32 operands and fp32 accumulation: one warp-level tensor-core MMA.
+// Thread l of the warp (g = l / 4, i = l % 4) holds a = {A[g][i], A[g+8][i], A[g][i+4], A[g+8][i+4]},
+// b = {B[i][g], B[i+4][g]} and d = {D[g][2i], D[g][2i+1], D[g+8][2i], D[g+8][2i+1]}.
+__device__ __forceinline__ void mma_16x8x8_tf32(float (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
+    asm volatile("mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+                 "{%0, %1, %2, %3};"
+                 : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+                 : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+// fp32 -> tf32, rounded to nearest (ties away from zero)
+__device__ __forceinline__ uint32_t to_tf32(float x) {
+    uint32_t y;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(y) : "f"(x));
+    return y;
 }
 
-// Byte offset of element (k, n) (K-row k, column n < 32) of an MN-major kind::tf32 operand in the layout
-// that tcgen05 requires for it: rows of 128 bytes, 4-row groups of 512 bytes, 32-byte granules XORed with
-// k % 4 (descriptor layout type 1, sdesc_sw128_32b with sbo = 512).
-__device__ __forceinline__ uint32_t b32_off(int k, int n) {
-    return (uint32_t)((k >> 2) * 512 + (k & 3) * 128 + ((((n >> 3) ^ (k & 3))) << 5) + (n & 7) * 4);
+// One 16 x 8 tile of D = A B (32 x 32 operands, plain layouts with row stride SP floats) for k-steps
+// [ks0, ks1): thread fragments as in mma_16x8x8_tf32.
+__device__ __forceinline__ void gemm32_tile(float (&d)[4], const float *A, const float *B, int rt, int ct, int ks0,
+                                            int ks1, int lane) {
+    const int g = lane >> 2, i = lane & 3;
+    d[0] = d[1] = d[2] = d[3] = 0.f;
+#pragma unroll
+    for (int ks = 0; ks < 4; ++ks) {
+        if (ks < ks0 || ks >= ks1) continue;
+        const float *ar = A + (16 * rt + g) * SP + 8 * ks + i;
+        const float *br = B + (8 * ks + i) * SP + 8 * ct + g;
+        const uint32_t a[4] = {to_tf32(ar[0]), to_tf32(ar[8 * SP]), to_tf32(ar[4]), to_tf32(ar[8 * SP + 4])};
+        const uint32_t b[2] = {to_tf32(br[0]), to_tf32(br[4 * SP])};
+        mma_16x8x8_tf32(d, a, b);
+    }
 }
 
 // Element (r, c) of a 32 x 32 diagonal block (r and c in the same 32-block) in the plain layout.
@@ -274,11 +287,9 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     // of A1 / the raw K tile landed; bar_pf[i]: the carry group is done with Pm buffer i and vector set i
     uint64_t *bar_ld = bars, *bar_gp = bars + 1, *bar_wu = bars + 2, *bar_m1 = bars + 3, *bar_m2 = bars + 4;
     uint64_t *bar_a1 = bars + 5, *bar_cq = bars + 6, *bar_ck = bars + 7, *bar_pf = bars + 8;
-    // the tensor-core merges of the solve: rounds 0..2 on bar_sv (three phases per chunk), round 3 on bar_sv3
-    uint64_t *bar_sv = bars + 10, *bar_sv3 = bars + 11;
     // bar_vr: the control warp has written the gate vectors of the next chunk (one phase per chunk)
-    uint64_t *bar_vr = bars + 12, *bar_ldv = bars + 13;
-    constexpr int kNumBars = 14;
+    uint64_t *bar_vr = bars + 10, *bar_ldv = bars + 11;
+    constexpr int kNumBars = 12;
     uint32_t *s_tmem = reinterpret_cast<uint32_t *>(bars + kNumBars);
     volatile int *s_abort = reinterpret_cast<volatile int *>(s_tmem + 1);
 
@@ -403,20 +414,26 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         const float gA = (a.A_log && a.g) ? a.A_log[h] : 0.f, gB = (a.A_log && a.g) ? a.dt_bias[h] : 0.f;
         const __nv_bfloat16 *bg = reinterpret_cast<const __nv_bfloat16 *>(a.beta) + (size_t)bh * S;
         const float *gg = a.g ? a.g + (size_t)bh * S : nullptr;
-        auto chunk_vectors = [&](int chunk) {
+        // raw beta and gate values of a chunk's tokens (two per lane), loaded a chunk before they are used so
+        // that their memory latency stays off the hand-offs
+        auto load_raw = [&](int chunk, float (&rb)[2], float (&rg)[2]) {
+            const int n = min(C, L - chunk * C);
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+                const int tt = 2 * lane + i, t = chunk * C + tt;
+                rb[i] = tt < n ? __bfloat162float(bg[t]) : 0.f;
+                rg[i] = (tt < n && gg) ? gg[t] : 0.f;
+            }
+        };
+        auto chunk_vectors = [&](int chunk, const float (&rb)[2], const float (&rg)[2]) {
             float *vec = vecs + (chunk & 1) * NVEC * 64;
             const int n = min(C, L - chunk * C);
             float bv[2], gv[2];
 #pragma unroll
             for (int i = 0; i < 2; ++i) {
-                const int tt = 2 * lane + i, t = chunk * C + tt;
-                float rb = 0.f, rg = 0.f;
-                if (tt < n) {
-                    rb = __bfloat162float(bg[t]);
-                    if (gg) rg = gg[t];
-                }
-                bv[i] = tt < n ? (a.beta_logits ? sigmoid_f32(rb) : rb) : 0.f;
-                gv[i] = tt < n ? (a.A_log ? gate_from_raw(rg, gA, gB) : rg) : 0.f;
+                const int tt = 2 * lane + i;
+                bv[i] = tt < n ? (a.beta_logits ? sigmoid_f32(rb[i]) : rb[i]) : 0.f;
+                gv[i] = tt < n ? (a.A_log ? gate_from_raw(rg[i], gA, gB) : rg[i]) : 0.f;
             }
             const float x1 = gv[0] + gv[1];
             float sc = x1;
@@ -439,7 +456,11 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             if (lane == 0) vec[V_N * 64] = (float)n;
         };
         bool to = false;
-        if (nvalid > 0) chunk_vectors(0);
+        float rbN[2] = {0.f, 0.f}, rgN[2] = {0.f, 0.f};
+        if (nvalid > 0) {
+            load_raw(0, rbN, rgN);
+            chunk_vectors(0, rbN, rgN);
+        }
         if (lane == 1 && nvalid > 0) {
             issue_k(0);
             issue_q(0);
@@ -449,6 +470,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         __syncwarp();
         for (int c = 0; c < nvalid; ++c) {
             const uint32_t par = c & 1;
+            if (c + 1 < nvalid) load_raw(c + 1, rbN, rgN);
             // H0: the prep group is at chunk c (and, for a last partial chunk, has zeroed its padding rows)
             if (named_sync_or(BAR_PCTL, NPC, to)) break;
             if (lane == 0) {  // a2: the Gram [K; Q][K; Q]^T ([Q; K][Q; K]^T for odd chunks); its diagonal gives
@@ -484,7 +506,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             // used (free once the carry's MMA2 of chunk c-1 completed)
             if (c + 1 < nvalid) {
                 if (c >= 1 && !mbar_wait_sleep(bar_pf + ((c + 1) & 1), ((c - 1) >> 1) & 1)) to = true;
-                chunk_vectors(c + 1);
+                chunk_vectors(c + 1, rbN, rgN);
             }
             __syncwarp();
             if (lane == 0 && c + 1 < nvalid) mbar_arrive(bar_vr);
@@ -584,10 +606,11 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                         for (int j4 = 0; j4 < 8; ++j4)
                             *reinterpret_cast<float4 *>(ap + 4 * j4) =
                                 make_float4(v[4 * j4], v[4 * j4 + 1], v[4 * j4 + 2], v[4 * j4 + 3]);
-                    } else if (krole) {  // A21 (rows 32..63, columns 0..31), operand of the tf32 merge
+                    } else if (krole) {  // A21 (rows 32..63, columns 0..31), operand of the 32 -> 64 merge
+                        float *ap = reinterpret_cast<float *>(sm + OFF_A21) + (t - 32) * SP;
 #pragma unroll
                         for (int j4 = 0; j4 < 8; ++j4)
-                            *reinterpret_cast<float4 *>(sm + OFF_A21 + f32_off(t - 32, 4 * j4)) =
+                            *reinterpret_cast<float4 *>(ap + 4 * j4) =
                                 make_float4(v[4 * j4], v[4 * j4 + 1], v[4 * j4 + 2], v[4 * j4 + 3]);
                     } else {
 #pragma unroll
@@ -607,26 +630,28 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             named_sync(BAR_PREP, NGRP);
             PHASE(5);
             // ---- a3: T = (I + A)^{-1} and the bf16 operand TT = [T diag(beta); T diag(c_W)] ----
-            // T = [[T11, 0], [T21, T22]]: the diagonal 32 x 32 blocks on the CUDA cores (solve_diag16_merge),
-            // then one pass that writes them into TT and into the operand layouts of the tensor-core merge
-            // T21 = -T22 (A21 T11): two kind::tf32 MMAs (M = 128 over 32 operand rows: the other lanes are
-            // not read), thread p == 0 issuing them, warp 8 moving X = A21 T11 from TMEM to shared memory,
-            // warps 8 and 12 (TMEM lanes 0..31) scaling T21 into TT.
+            // T = [[T11, 0], [T21, T22]]: the diagonal 32 x 32 blocks on the CUDA cores (solve_diag16_merge), then
+            // T21 = -T22 (A21 T11) by the eight prep warps, one 16 x 8 tile each of X = A21 T11 and then of T21,
+            // on warp-level tf32 MMAs; the diagonal blocks go into TT meanwhile.
             solve_diag16_merge(reinterpret_cast<const float *>(sm + OFF_AP), reinterpret_cast<float *>(sm + OFF_TP),
                                reinterpret_cast<float *>(sm + OFF_XP), p);
             PHASE(12);
+            const float *tpl = reinterpret_cast<const float *>(sm + OFF_TP);
+            float *xm = reinterpret_cast<float *>(sm + OFF_XM);
+            const int pw = p >> 5, rt = pw >> 2, ct = pw & 3, gq = lane >> 2, iq = lane & 3;
             {
+                // X tile (rows 16 rt.., columns 8 ct..); T11 is lower triangular, so k-steps before ct add nothing
+                float d[4];
+                gemm32_tile(d, reinterpret_cast<const float *>(sm + OFF_A21), tpl, rt, ct, ct, 4, lane);
+                *reinterpret_cast<float2 *>(xm + (16 * rt + gq) * SP + 8 * ct + 2 * iq) = make_float2(d[0], d[1]);
+                *reinterpret_cast<float2 *>(xm + (16 * rt + gq + 8) * SP + 8 * ct + 2 * iq) = make_float2(d[2], d[3]);
+            }
+            {
+                // TT rows of the diagonal blocks (and zeros above them), while other warps finish X
                 const int blk = p >> 7, t = (p >> 2) & 31, c8 = p & 3, R = 32 * blk + t, col = 32 * blk + 8 * c8;
-                const float *tp = reinterpret_cast<const float *>(sm + OFF_TP) + pl(R, col);
+                const float *tp = tpl + pl(R, col);
                 const float4 u0 = *reinterpret_cast<const float4 *>(tp), u1 = *reinterpret_cast<const float4 *>(tp + 4);
                 const float tv[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
-                if (blk == 0) {  // T11, the MN-major operand of X = A21 T11
-                    *reinterpret_cast<float4 *>(sm + OFF_T11 + b32_off(t, 8 * c8)) = u0;
-                    *reinterpret_cast<float4 *>(sm + OFF_T11 + b32_off(t, 8 * c8 + 4)) = u1;
-                } else {  // T22, the K-major operand of T21 = -T22 X
-                    *reinterpret_cast<float4 *>(sm + OFF_T22 + f32_off(t, 8 * c8)) = u0;
-                    *reinterpret_cast<float4 *>(sm + OFF_T22 + f32_off(t, 8 * c8 + 4)) = u1;
-                }
                 float fb[8], fw[8];
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
@@ -639,58 +664,24 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 const int Rz = (p >> 2) + ((p >> 7) << 5), cz = 4 + (p & 3);
                 *reinterpret_cast<uint4 *>(sm + OFF_TT + blk_off(Rz, 8 * cz)) = make_uint4(0, 0, 0, 0);
             }
-            fence_proxy_async_smem();
-            tc_fence_before();
             named_sync(BAR_PREP, NGRP);
             PHASE(13);
-            if (p == 0) {  // X = A21 T11 -> TMEM lanes 0..31, columns 0..31
-                tc_fence_after();
-                const uint32_t id = idesc_tf32(128, 32, false, true, false);
+            {
+                // T21 tile = -(T22 X): T22 is lower triangular, so rows 16 rt.. need k-steps up to 2 rt + 1 only;
+                // straight into TT rows 32 + r (times beta_s) and 96 + r (times c_W,s), columns s < 32
+                float d[4];
+                gemm32_tile(d, tpl + 32 * SP, xm, rt, ct, 0, 2 * rt + 2, lane);
+                const int s0 = 8 * ct + 2 * iq;
+                const float b0 = vBeta[s0], b1 = vBeta[s0 + 1], w0 = vCw[s0], w1 = vCw[s0 + 1];
 #pragma unroll
-                for (int k = 0; k < 4; ++k)
-                    mma_tf32(tmem + TM_GPW, sdesc_sw128(sbase + OFF_A21 + k * 32, 16, 1024),
-                             sdesc_sw128_32b(sbase + OFF_T11 + k * 1024, 512), id, k > 0);
-                mma_commit(bar_sv);
-            }
-            if (warp == 8) {
-                __syncwarp();
-                wait_ok(bar_sv, par);
-                tc_fence_after();
-                float xv[32];
-                tmem_ld32(tmem + TM_GPW + lane_base, xv);
-                tmem_ld_wait();
-#pragma unroll
-                for (int c4 = 0; c4 < 8; ++c4)
-                    *reinterpret_cast<float4 *>(sm + OFF_XB + b32_off(lane, 4 * c4)) =
-                        make_float4(xv[4 * c4], xv[4 * c4 + 1], xv[4 * c4 + 2], xv[4 * c4 + 3]);
-                fence_proxy_async_smem();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) {  // T21 = -T22 X -> TMEM lanes 0..31, columns 32..63
-                    tc_fence_after();
-                    const uint32_t id = idesc_tf32(128, 32, false, true, true);
-#pragma unroll
-                    for (int k = 0; k < 4; ++k)
-                        mma_tf32(tmem + TM_GPW + 32, sdesc_sw128(sbase + OFF_T22 + k * 32, 16, 1024),
-                                 sdesc_sw128_32b(sbase + OFF_XB + k * 1024, 512), id, k > 0);
-                    mma_commit(bar_sv3);
+                for (int hh = 0; hh < 2; ++hh) {
+                    const int r = 16 * rt + gq + 8 * hh;
+                    const float t0 = -d[2 * hh], t1 = -d[2 * hh + 1];
+                    *reinterpret_cast<uint32_t *>(sm + OFF_TT + blk_off(32 + r, s0)) = pack_bf16x2(t0 * b0, t1 * b1);
+                    *reinterpret_cast<uint32_t *>(sm + OFF_TT + blk_off(96 + r, s0)) = pack_bf16x2(t0 * w0, t1 * w1);
                 }
-                __syncwarp();
             }
             PHASE(14);
-            if (warp == 8 || warp == 12) {  // TT rows 32 + r (beta) / 96 + r (c_W), columns 0..31 from T21
-                wait_ok(bar_sv3, par);
-                tc_fence_after();
-                float tv[32];
-                tmem_ld32(tmem + TM_GPW + 32, tv);
-                const float *scl = hf ? vCw : vBeta;
-                tmem_ld_wait();
-#pragma unroll
-                for (int jj = 0; jj < 32; ++jj) tv[jj] *= scl[jj];
-#pragma unroll
-                for (int c8 = 0; c8 < 4; ++c8)
-                    *reinterpret_cast<uint4 *>(sm + OFF_TT + blk_off(32 + 64 * hf + lane, 8 * c8)) = pack8(&tv[8 * c8]);
-            }
             PHASE(6);
             PHASE(7);
             if (n < C) {  // padding rows of the last chunk's V, once it has landed
@@ -722,6 +713,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             if (!mbar_wait_sleep(bar_a1, par)) to = true;
             wait_ok(bar_cq, par);
             if (named_sync_or(BAR_CARRY, NGRP, to)) { stop = true; break; }
+            PHASE(21);
             if (tid == 0) {  // a4: W (rows 64..127 of TT K, into TMEM R) and U (rows 0..63 of TT V)
                 if (!mbar_wait(bar_ldv, par)) to = true;
                 tc_fence_after();
@@ -736,6 +728,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             }
             wait_ok(bar_wu, par);
             tc_fence_after();
+            PHASE(22);
             if (q4 >= 2) {  // W rows (TMEM lanes 64..127 of R) -> rows 0..63 of A1
                 const int t = row - 64;
 #pragma unroll
