@@ -75,11 +75,12 @@ __device__ unsigned long long g_phase[64];
 
 namespace {
 
-// warps 0-7 carry, 8-15 prep, 16 control (TMA loads and the prep MMAs)
-constexpr int C = 64, D = 128, NGRP = 256, NT = 2 * NGRP + 32, NPC = NGRP + 32;
+// warps 0-7 carry, 8-15 prep, 16 control (TMA loads and the prep MMAs), 17-19 helpers (the K~ operand).  The
+// register file is allocated to warps in groups of four, so the helpers cost no registers per thread.
+constexpr int C = 64, D = 128, NGRP = 256, NHELP = 96, NT = 2 * NGRP + 32 + NHELP, NPC = NGRP + 32;
 constexpr int CTL_WARP = 16;
-// BAR_PCTL: the prep warps and the control warp, at the hand-offs between them
-constexpr int BAR_CARRY = 1, BAR_PREP = 2, BAR_PCTL = 3;
+// BAR_PCTL: the prep warps and the control warp, at the hand-offs between them; BAR_HELP: the helper warps
+constexpr int BAR_CARRY = 1, BAR_PREP = 2, BAR_PCTL = 3, BAR_HELP = 4;
 constexpr uint32_t kTimeoutBit = 0x4u;
 // carry thread that issues the out-tile TMA stores (thread 0 issues the carry's MMAs)
 constexpr int kStorer = 32;
@@ -289,12 +290,15 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     uint64_t *bar_a1 = bars + 5, *bar_cq = bars + 6, *bar_ck = bars + 7, *bar_pf = bars + 8;
     // bar_vr: the control warp has written the gate vectors of the next chunk (one phase per chunk)
     uint64_t *bar_vr = bars + 10, *bar_ldv = bars + 11;
-    constexpr int kNumBars = 12;
+    // bar_go: the carry group has taken chunk c over (its tail factors are in place); bar_kt: the helper warps
+    // have scaled chunk c's K tile into K~ (one phase per chunk each)
+    uint64_t *bar_go = bars + 12, *bar_kt = bars + 13;
+    constexpr int kNumBars = 14;
     uint32_t *s_tmem = reinterpret_cast<uint32_t *>(bars + kNumBars);
     volatile int *s_abort = reinterpret_cast<volatile int *>(s_tmem + 1);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, q4 = warp & 3, hf = (warp >> 2) & 1;
-    const bool carry = warp < 8, control = warp == CTL_WARP;
+    const bool carry = warp < 8, control = warp == CTL_WARP, helper = warp > CTL_WARP;
     const int bh = blockIdx.x, h = bh % a.Nv, b = bh / a.Nv, kh = h / (a.Nv / a.Nk);
     const int S = a.S;
     int L = a.lengths ? a.lengths[b] : S;
@@ -511,6 +515,39 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             __syncwarp();
             if (lane == 0 && c + 1 < nvalid) mbar_arrive(bar_vr);
         }
+    } else if (helper) {
+        // ============================== helper warps ==============================
+        // K~ = diag(e^{G_last - G} / |k|) K of each chunk, in place in the carry's raw K tile (rows past the
+        // length, whatever they hold, become zero): the A operand of the state update, made off the carry's
+        // serial chain.  The tile of chunk c lands after MMA2 of chunk c-1 and is needed at MMA2 of chunk c.
+        const int hp = tid - (CTL_WARP + 1) * 32;
+        bool to = false;
+        for (int c = 0; c < nvalid; ++c) {
+            const uint32_t par = c & 1;
+            const float *vec = vecs + par * NVEC * 64;
+            // bar_go of chunk c+1 follows bar_kt of chunk c, and the K tile of chunk c+1 is loaded after MMA2 of
+            // chunk c, which waits for bar_kt of chunk c: neither wait can be a phase behind
+            if (!mbar_wait(bar_go, par)) to = true;
+            if (!mbar_wait(bar_ck, par)) to = true;
+            if (!to) {
+                const int n = (int)vec[V_N * 64];
+                const float *vtail = vec + V_TAIL * 64;
+                for (int e = hp; e < 1024; e += NHELP) {
+                    const int t = (e >> 3) & 63;
+                    uint4 *pk = reinterpret_cast<uint4 *>(sm + OFF_KT + (e >> 9) * 8192 + t * 128 + (e & 7) * 16);
+                    float f[8];
+                    unpack8(*pk, f);
+                    const float sc = vtail[t];
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) f[j] = t < n ? f[j] * sc : 0.f;
+                    *pk = pack8(f);
+                }
+            }
+            fence_proxy_async_smem();
+            if (named_sync_or(BAR_HELP, NHELP, to)) break;
+            if (hp == 0) mbar_arrive(bar_kt);
+        }
+        if (to && hp == 0) *s_abort = 1;
     } else if (!carry) {
         // =============================== prep group ===============================
         const int p = tid - NGRP;
@@ -714,6 +751,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             wait_ok(bar_cq, par);
             if (named_sync_or(BAR_CARRY, NGRP, to)) { stop = true; break; }
             PHASE(21);
+            if (tid == 0) mbar_arrive(bar_go);
             if (tid == 0) {  // a4: W (rows 64..127 of TT K, into TMEM R) and U (rows 0..63 of TT V)
                 if (!mbar_wait(bar_ldv, par)) to = true;
                 tc_fence_after();
@@ -777,24 +815,6 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 }
                 tmem_st_wait();
             }
-            // meanwhile: the K tile -> K~ = diag(e^{G_last - G} / |k|) K in place (rows past the length, whatever
-            // they hold, become zero), the A operand of the state update
-            wait_ok(bar_ck, par);
-            {
-                const float *vtail = vec + V_TAIL * 64;
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const int e = tid + i * NGRP, t = (e >> 3) & 63;
-                    uint4 *pk = reinterpret_cast<uint4 *>(sm + OFF_KT + (e >> 9) * 8192 + t * 128 + (e & 7) * 16);
-                    float f[8];
-                    unpack8(*pk, f);
-                    const float sc = vtail[t];
-#pragma unroll
-                    for (int j = 0; j < 8; ++j) f[j] = t < n ? f[j] * sc : 0.f;
-                    *pk = pack8(f);
-                }
-            }
-            fence_proxy_async_smem();
             wait_ok(bar_m1, par);
             if (tid == 0 && c + 1 < nvalid) load_carry_q(c + 1);  // the Q rows of A1 are read
             if (tid == kStorer) bulk_wait_read0();  // the previous out tile (same buffer as v_new) is read
@@ -846,6 +866,8 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             PHASE(18);
             // ---- S += K~^T v_new ;  R[64:128] += Pm v_new ----
             if (tid == 0) {
+                if (!mbar_wait(bar_kt, par)) to = true;  // K~ of this chunk (helper warps)
+                tc_fence_after();
                 const uint32_t id_s = idesc_bf16(128, 128, true, true);
                 const uint32_t id_o = idesc_bf16(128, 128, false, true);
                 const uint32_t pm_rows = sbase + (par ? OFF_PM1 : OFF_PM0) - 8192;
