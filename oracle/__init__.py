@@ -7,7 +7,8 @@ import it.  It shares no code with the CUDA path and never calls it.
 ``gdr_oracle.c`` holds the token-by-token definition (compiled here with gcc,
 no fast-math); ``forms.py`` holds independent formulations from the pages
 (the chunked WY form, the pseudo-value form, gated linear attention by brute
-force) used to pin it.  Every function here is pinned by
+force) used to pin it.  ``gated_rmsnorm`` is the layer's output epilogue, written
+out from its definition and pinned by closed forms.  Every function here is pinned by
 ``tests/test_oracle_pins.py`` (closed forms, worked examples printed on the
 pages, independent formulations, brute force, invariants); none is left
 unpinned.
@@ -28,7 +29,7 @@ _LIB_PATH = os.path.join(_BUILD, "libgdr_oracle.so")
 _lock = threading.Lock()
 _lib = None
 
-__all__ = ["build", "lib", "prologue", "chunk_fwd", "recurrent_step", "threads"]
+__all__ = ["build", "lib", "prologue", "chunk_fwd", "recurrent_step", "gated_rmsnorm", "threads"]
 
 
 def build(force: bool = False) -> str:
@@ -179,3 +180,30 @@ def recurrent_step(q, k, v, beta, g, gk, state_pool, ssm_state_indices, actual_s
     if rc != 0:
         raise ValueError(f"oracle recurrent_step rejected the arguments (code {rc})")
     return out, pool
+
+
+def gated_rmsnorm(o, z, norm_w, eps: float, actual_seq_lengths=None):
+    """fp64 output epilogue of the layer: per head and token, the row o (length Dv) becomes
+
+        o / sqrt(mean_j o_j^2 + eps) * w * silu(z),   silu(z) = z / (1 + e^{-z}),
+
+    with one weight vector w (Dv) shared by all heads.  Rows t >= L_b (padding) are returned
+    unchanged (the calls leave them zero).
+
+    Source: the gated RMSNorm applied per head after the recurrence in deltanet.rs (mean of the
+    squares over the head's Dv outputs, eps inside the square root, times norm_w and silu of the
+    head's z slice) and the same arithmetic in the WGSL core shader of that crate; the blog
+    "gated-delta-net" page applies it as self.norm(core_attn_out, z) on rows of length d_v.  Its
+    comment names the gate sigmoid(z); both code listings use silu, which is the reading taken.
+
+    o, z: (B, Nv, S, Dv); norm_w: (Dv,); actual_seq_lengths: (B,) or None (all S).
+    """
+    oa, za, wa = _f64(o), _f64(z), _f64(norm_w)
+    if oa.shape != za.shape or wa.shape != (oa.shape[-1],):
+        raise ValueError("o and z must have the same shape and norm_w the length of their last axis")
+    B, S = oa.shape[0], oa.shape[2]
+    L = np.full(B, S, np.int64) if actual_seq_lengths is None else np.asarray(actual_seq_lengths, np.int64)
+    inv = 1.0 / np.sqrt(np.mean(oa * oa, axis=-1, keepdims=True) + float(eps))
+    y = oa * inv * wa * (za / (1.0 + np.exp(-za)))
+    t = np.arange(S)[None, None, :, None]
+    return np.where(t < L[:, None, None, None], y, oa)

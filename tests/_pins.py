@@ -275,3 +275,63 @@ def check_store_and_recall(impl):
 ALL_CHECKS = [check_worked_examples, check_matrix_form, check_readback, check_beta_zero, check_chunked_forms,
               check_gla_orthogonal, check_teaching_form, check_split_resume, check_gqa, check_padding,
               check_state_bounded, check_store_and_recall]
+
+
+# ---- the output epilogue: rmsnorm(o) * w * silu(z) ----
+
+def check_epi_constant_row(impl):
+    """o = 3 in every entry, eps = 16: the mean square is 9, so the row factor is 3/5 exactly;
+    z = ln 3 gives sigmoid(z) = 3/4 and silu(z) = (3/4) ln 3 (a gate of sigmoid(z) would give 3/4)."""
+    Dv = 8
+    w = np.arange(1, Dv + 1, dtype=np.float64) * 0.5
+    o = np.full((1, 2, 3, Dv), 3.0)
+    z = np.full_like(o, math.log(3.0))
+    got = impl(o, z, w, 16.0)
+    want = 0.6 * 0.75 * math.log(3.0) * w
+    assert np.allclose(got, np.broadcast_to(want, got.shape), rtol=0, atol=1e-15)
+
+
+def check_epi_row_mean(impl):
+    """One non-zero entry 3 in a row of Dv = 4 with eps = 3/4: mean square 9/4, plus eps = 3, so the
+    entry becomes 3 / sqrt(3) = sqrt(3) (a sum instead of a mean would give 3 / sqrt(9.75))."""
+    o = np.zeros((1, 1, 1, 4))
+    o[..., 0] = 3.0
+    z = np.full_like(o, 50.0)  # silu(50) = 50 to double precision
+    got = impl(o, z, np.ones(4), 0.75)
+    assert abs(got[0, 0, 0, 0] - math.sqrt(3.0) * 50.0) < 1e-12
+    assert np.all(got[0, 0, 0, 1:] == 0.0)
+
+
+def check_epi_invariants(impl):
+    """z = 0 closes the gate exactly; with eps = 0 the result does not depend on the scale of o
+    and is odd in o; with w = 1 and silu(z) = 1 the output row has mean square ms / (ms + eps)."""
+    rng = np.random.default_rng(7)
+    o = rng.standard_normal((2, 3, 5, 16))
+    w = rng.uniform(0.5, 1.5, 16)
+    z = rng.standard_normal(o.shape)
+    assert np.all(impl(o, np.zeros_like(o), w, 1e-6) == 0.0)
+    base = impl(o, z, w, 0.0)
+    assert np.allclose(impl(7.5 * o, z, w, 0.0), base, rtol=1e-13, atol=0)
+    assert np.allclose(impl(-o, z, w, 0.0), -base, rtol=1e-13, atol=0)
+    # silu(z1) = 1 at the root of z = 1 + e^{-z}, found by bisection
+    lo, hi = 1.0, 2.0
+    for _ in range(200):
+        mid = 0.5 * (lo + hi)
+        lo, hi = (mid, hi) if mid / (1.0 + math.exp(-mid)) < 1.0 else (lo, mid)
+    eps = 0.3
+    out = impl(o, np.full_like(o, lo), np.ones(16), eps)
+    ms = np.mean(o * o, axis=-1)
+    assert np.allclose(np.mean(out * out, axis=-1), ms / (ms + eps), rtol=1e-12, atol=0)
+
+
+def check_epi_padding(impl):
+    """Rows t >= L_b are passed through untouched (the calls keep them zero)."""
+    rng = np.random.default_rng(8)
+    o = rng.standard_normal((2, 1, 6, 8))
+    z = rng.standard_normal(o.shape)
+    got = impl(o, z, np.ones(8), 1e-6, np.array([4, 0]))
+    assert np.array_equal(got[0, :, 4:], o[0, :, 4:]) and np.array_equal(got[1], o[1])
+    assert not np.allclose(got[0, :, :4], o[0, :, :4])
+
+
+EPILOGUE_CHECKS = [check_epi_constant_row, check_epi_row_mean, check_epi_invariants, check_epi_padding]

@@ -215,3 +215,9 @@ def test_oracle_is_thread_count_independent():
     assert np.array_equal(o1, o2) and np.array_equal(f1, f2)
     assert oracle.threads() >= 1
     assert math.isfinite(float(np.abs(o1).max()))
+
+
+
+@pytest.mark.parametrize("check", _pins.EPILOGUE_CHECKS, ids=lambda c: c.__name__)
+def test_gated_rmsnorm_oracle_pin(check):
+    check(oracle.gated_rmsnorm)

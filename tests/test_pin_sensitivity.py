@@ -78,3 +78,46 @@ def test_planted_mistake_is_caught(mutation):
         except (AssertionError, ValueError, IndexError):
             failed.append(check.__name__)
     assert failed, f"no pin caught the planted mistake {mutation!r}"
+
+
+def make_epilogue(mutation=None):
+    """A plain copy of rmsnorm(o) * w * silu(z) per row, with planted mistakes."""
+    def impl(o, z, w, eps, lengths=None):
+        o, z, w = (np.asarray(x, np.float64) for x in (o, z, w))
+        B, S = o.shape[0], o.shape[2]
+        out = o.copy()
+        for b in range(B):
+            L = S if lengths is None else int(lengths[b])
+            for t in range(S if mutation == "epi_pads_too" else L):
+                r = o[b, :, t]
+                ms = np.sum(r * r, -1, keepdims=True) if mutation == "epi_sum" else np.mean(r * r, -1, keepdims=True)
+                if mutation == "epi_eps_outside":
+                    inv = 1.0 / np.sqrt(ms) + eps
+                else:
+                    inv = 1.0 / np.sqrt(ms + eps)
+                zz = z[b, :, t]
+                gate = 1.0 / (1.0 + np.exp(-zz)) if mutation == "epi_sigmoid" else zz / (1.0 + np.exp(-zz))
+                wv = 1.0 if mutation == "epi_no_weight" else w
+                out[b, :, t] = r * inv * wv * gate
+        return out
+    return impl
+
+
+EPI_MUTATIONS = ["epi_sum", "epi_eps_outside", "epi_sigmoid", "epi_no_weight", "epi_pads_too"]
+
+
+def test_unmodified_epilogue_copy_passes_every_pin():
+    for check in _pins.EPILOGUE_CHECKS:
+        check(make_epilogue())
+
+
+@pytest.mark.parametrize("mutation", EPI_MUTATIONS)
+def test_planted_epilogue_mistake_is_caught(mutation):
+    impl = make_epilogue(mutation)
+    caught = 0
+    for check in _pins.EPILOGUE_CHECKS:
+        try:
+            check(impl)
+        except AssertionError:
+            caught += 1
+    assert caught > 0, mutation
