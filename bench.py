@@ -313,6 +313,37 @@ def bench_prefill(gdr, args, world, rank, clk, flush, stream, peaks):
     return fields, w, t, pro, step
 
 
+def bench_prefill_epilogue(gdr, args, world, w, t, pro, flush, stream, peaks):
+    """The same prefill call with the fused gated RMSNorm output epilogue (z and norm_w of the layer's
+    output gate); returns (fields, launches)."""
+    z, nw = workloads.epilogue_inputs(w)
+    epi = gdr.Epilogue(z=bf16_dev(z), norm_w=f32_dev(nw), eps=1e-6)
+    del z
+    step = gdr.prepare_chunk_fwd(t["q"], t["k"], t["v"], t["b"], t["a"], t["s0"], None, w.scale, prologue=pro,
+                                 epilogue=epi, out=t["out"], final_state=t["fin"])
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if gdr.get_error() != 0:
+        raise RuntimeError("device error word set during warm-up")
+    barrier(world)
+    torch.cuda.synchronize()
+    times = timed_steps(step, args.steps, flush, stream)
+    barrier(world)
+    total_ms = all_max(sum(times), world)
+    ms_per_step = total_ms / args.steps
+    tokens = int(w.lengths.sum())
+    # the prefill's bytes plus z (one bf16 row per valid token and value head) and norm_w
+    alg_bytes = algorithmic_prefill_bytes(w) + tokens * w.Nv * w.Dv * 2 + w.Dv * 4
+    achieved = alg_bytes / (ms_per_step / 1e3) / 1e9
+    return {"workload": f"prefill B={w.B} S={w.S} Nk={w.Nk} Nv={w.Nv} Dk=Dv={w.Dk} bf16, fused prologue and "
+                        "gated RMSNorm epilogue (eps 1e-6)",
+            "ms_per_step": ms_per_step, "tokens_per_s": weak_scaling_rate(tokens, args.steps, total_ms, world),
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": achieved / peaks["hbm_gbs"], "traffic": None, "algorithmic_bytes_per_launch":
+                         alg_bytes, "kernel": "gdr_chunk_fwd (fused prologue and epilogue)"}}, args.steps
+
+
 def bench_e2e(gdr, args, world, w, t, pro, flush, stream):
     """Same metric through the public call with host buffers: pinned H2D copies of the
     step's inputs, the call, D2H of out and the final state, all inside the timed region."""
@@ -411,6 +442,9 @@ def run_ours(args, world, rank, local):
         launches += fields.pop("gpu_launches")
         if not args.no_e2e:
             line["e2e"], n = bench_e2e(gdr, args, world, w, t, pro, flush, stream)
+        if not args.no_epilogue:
+            line["prefill_epilogue"], n = bench_prefill_epilogue(gdr, args, world, w, t, pro, flush, stream, peaks)
+            launches += n
         del t
     decode = {}
     for name in ("decode", "decode_gk"):
@@ -440,6 +474,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing (for profiling runs)")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg (profiling runs)")
+    ap.add_argument("--no-epilogue", action="store_true",
+                    help="skip the prefill line with the fused gated RMSNorm epilogue (profiling runs)")
     ap.add_argument("--only", choices=["all", "prefill", "decode", "decode_gk"], default="all",
                     help="run one workload only (profiling runs); the default runs all")
     args = ap.parse_args()

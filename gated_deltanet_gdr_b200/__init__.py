@@ -40,6 +40,10 @@ class GdrPrologueStruct(ctypes.Structure):
                 ("A_log", ctypes.c_void_p), ("dt_bias", ctypes.c_void_p)]
 
 
+class GdrEpilogueStruct(ctypes.Structure):
+    _fields_ = [("z", ctypes.c_void_p), ("norm_w", ctypes.c_void_p), ("eps", ctypes.c_float)]
+
+
 _lib = None
 _lock = threading.Lock()
 
@@ -57,10 +61,11 @@ def lib() -> ctypes.CDLL:
         vp, i32, f32 = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
         L.gdr_chunk_fwd.restype = i32
         L.gdr_chunk_fwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, f32, i32, i32, i32, i32, i32, i32, i32,
-                                    ctypes.POINTER(GdrPrologueStruct), vp, vp, vp]
+                                    ctypes.POINTER(GdrPrologueStruct), ctypes.POINTER(GdrEpilogueStruct), vp, vp, vp]
         L.gdr_recurrent_step.restype = i32
         L.gdr_recurrent_step.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, vp, vp, vp, f32, i32, i32, i32, i32, i32,
-                                         i32, i32, i32, ctypes.POINTER(GdrPrologueStruct), vp, vp]
+                                         i32, i32, i32, ctypes.POINTER(GdrPrologueStruct),
+                                         ctypes.POINTER(GdrEpilogueStruct), vp, vp]
         L.gdr_prologue_apply.restype = i32
         L.gdr_prologue_apply.argtypes = [vp, vp, vp, vp, vp, vp, f32, i32, i32, i32, i32, i32, i32, vp, vp, vp, vp,
                                          vp]
@@ -87,6 +92,26 @@ class Prologue:
     def as_struct(self) -> GdrPrologueStruct:
         return GdrPrologueStruct(int(self.l2norm_qk), float(self.eps), int(self.beta_logits), _ptr(self.A_log),
                                  _ptr(self.dt_bias))
+
+
+@dataclass
+class Epilogue:
+    """Fused output epilogue (see ``gdr_epilogue`` in include/gdr.h): each valid out row o
+    becomes o / sqrt(mean(o^2) + eps) * norm_w * silu(z) (the layer's gated RMSNorm)."""
+    z: torch.Tensor  # (B, Nv, S, Dv), the dtype of q
+    norm_w: torch.Tensor  # (Dv,) fp32
+    eps: float = 1e-6
+
+    def as_struct(self) -> GdrEpilogueStruct:
+        return GdrEpilogueStruct(_ptr(self.z), _ptr(self.norm_w), float(self.eps))
+
+
+def _check_epilogue(epi, B, Nv, S, Dv, dt):
+    if epi is None:
+        return None
+    _dev(epi.z, "epilogue.z", dt, (B, Nv, S, Dv))
+    _dev(epi.norm_w, "epilogue.norm_w", torch.float32, (Dv,))
+    return epi.as_struct()
 
 
 def _check(status: int, what: str):
@@ -159,17 +184,19 @@ def _chunk_checked(q, k, v, beta, g, initial_state, actual_seq_lengths, prologue
 
 
 def chunk_fwd(q, k, v, beta, g=None, initial_state=None, actual_seq_lengths=None, scale: float = 1.0, *,
-              prologue: Optional[Prologue] = None, out=None, final_state=None, output_final_state: bool = True,
-              stream=None):
+              prologue: Optional[Prologue] = None, epilogue: Optional[Epilogue] = None, out=None, final_state=None,
+              output_final_state: bool = True, stream=None):
     """Chunked prefill (``gdr_chunk_fwd``).  Returns (out, final_state or None)."""
     out, final_state = _chunk_checked(q, k, v, beta, g, initial_state, actual_seq_lengths, prologue, out,
                                       final_state, output_final_state)
     B, Nk, S, Dk = q.shape
     Nv, Dv = v.shape[1], v.shape[3]
     pro = prologue.as_struct() if prologue is not None else None
+    epi = _check_epilogue(epilogue, B, Nv, S, Dv, q.dtype)
     st = lib().gdr_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(g), _ptr(initial_state),
                              _ptr(actual_seq_lengths), float(scale), B, Nk, Nv, S, Dk, Dv, _dtype_code(q.dtype),
-                             ctypes.byref(pro) if pro is not None else None, _ptr(out), _ptr(final_state),
+                             ctypes.byref(pro) if pro is not None else None,
+                             ctypes.byref(epi) if epi is not None else None, _ptr(out), _ptr(final_state),
                              _stream(stream))
     _check(st, "gdr_chunk_fwd")
     return out, final_state
@@ -203,8 +230,8 @@ def _decode_checked(q, k, v, beta, g, gk, state_pool, ssm_state_indices, actual_
 
 
 def recurrent_step(q, k, v, beta, g, gk, state_pool, ssm_state_indices, actual_seq_lengths,
-                   num_accepted_tokens=None, scale: float = 1.0, *, prologue: Optional[Prologue] = None, out=None,
-                   stream=None):
+                   num_accepted_tokens=None, scale: float = 1.0, *, prologue: Optional[Prologue] = None,
+                   epilogue: Optional[Epilogue] = None, out=None, stream=None):
     """Recurrent decode over a slot pool (``gdr_recurrent_step``), updating
     ``state_pool`` in place.  Returns (out, state_pool)."""
     out = _decode_checked(q, k, v, beta, g, gk, state_pool, ssm_state_indices, actual_seq_lengths,
@@ -212,11 +239,13 @@ def recurrent_step(q, k, v, beta, g, gk, state_pool, ssm_state_indices, actual_s
     B, Nk, S, Dk = q.shape
     Nv, Dv = v.shape[1], v.shape[3]
     pro = prologue.as_struct() if prologue is not None else None
+    epi = _check_epilogue(epilogue, B, Nv, S, Dv, q.dtype)
     st = lib().gdr_recurrent_step(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(g), _ptr(gk), _ptr(state_pool),
                                   int(state_pool.shape[0]), _ptr(ssm_state_indices), _ptr(actual_seq_lengths),
                                   _ptr(num_accepted_tokens), float(scale), B, Nk, Nv, S, Dk, Dv,
                                   _dtype_code(q.dtype), _dtype_code(state_pool.dtype),
-                                  ctypes.byref(pro) if pro is not None else None, _ptr(out), _stream(stream))
+                                  ctypes.byref(pro) if pro is not None else None,
+                                  ctypes.byref(epi) if epi is not None else None, _ptr(out), _stream(stream))
     _check(st, "gdr_recurrent_step")
     return out, state_pool
 
@@ -241,36 +270,41 @@ class PreparedCall:
 
 
 def prepare_chunk_fwd(q, k, v, beta, g=None, initial_state=None, actual_seq_lengths=None, scale: float = 1.0, *,
-                      prologue: Optional[Prologue] = None, out=None, final_state=None, stream=None) -> PreparedCall:
+                      prologue: Optional[Prologue] = None, epilogue: Optional[Epilogue] = None, out=None,
+                      final_state=None, stream=None) -> PreparedCall:
     """Check and marshal a gdr_chunk_fwd call once; see chunk_fwd for the arguments."""
     out, final_state = _chunk_checked(q, k, v, beta, g, initial_state, actual_seq_lengths, prologue, out,
                                       final_state, True)
     B, Nk, S, Dk = q.shape
     Nv, Dv = v.shape[1], v.shape[3]
     pro = prologue.as_struct() if prologue is not None else None
+    epi = _check_epilogue(epilogue, B, Nv, S, Dv, q.dtype)
     args = (_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(g), _ptr(initial_state), _ptr(actual_seq_lengths),
             ctypes.c_float(scale), B, Nk, Nv, S, Dk, Dv, _dtype_code(q.dtype),
-            ctypes.pointer(pro) if pro is not None else None, _ptr(out), _ptr(final_state), _stream(stream))
+            ctypes.pointer(pro) if pro is not None else None, ctypes.pointer(epi) if epi is not None else None,
+            _ptr(out), _ptr(final_state), _stream(stream))
     call = PreparedCall(lib().gdr_chunk_fwd, args, "gdr_chunk_fwd", (out, final_state))
-    call._keep = (pro, prologue)
+    call._keep = (pro, prologue, epi, epilogue)
     return call
 
 
 def prepare_recurrent_step(q, k, v, beta, g, gk, state_pool, ssm_state_indices, actual_seq_lengths,
                            num_accepted_tokens=None, scale: float = 1.0, *, prologue: Optional[Prologue] = None,
-                           out=None, stream=None) -> PreparedCall:
+                           epilogue: Optional[Epilogue] = None, out=None, stream=None) -> PreparedCall:
     """Check and marshal a gdr_recurrent_step call once; see recurrent_step for the arguments."""
     out = _decode_checked(q, k, v, beta, g, gk, state_pool, ssm_state_indices, actual_seq_lengths,
                           num_accepted_tokens, out)
     B, Nk, S, Dk = q.shape
     Nv, Dv = v.shape[1], v.shape[3]
     pro = prologue.as_struct() if prologue is not None else None
+    epi = _check_epilogue(epilogue, B, Nv, S, Dv, q.dtype)
     args = (_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(g), _ptr(gk), _ptr(state_pool), int(state_pool.shape[0]),
             _ptr(ssm_state_indices), _ptr(actual_seq_lengths), _ptr(num_accepted_tokens), ctypes.c_float(scale), B,
             Nk, Nv, S, Dk, Dv, _dtype_code(q.dtype), _dtype_code(state_pool.dtype),
-            ctypes.pointer(pro) if pro is not None else None, _ptr(out), _stream(stream))
+            ctypes.pointer(pro) if pro is not None else None, ctypes.pointer(epi) if epi is not None else None,
+            _ptr(out), _stream(stream))
     call = PreparedCall(lib().gdr_recurrent_step, args, "gdr_recurrent_step", (out, state_pool))
-    call._keep = (pro, prologue)
+    call._keep = (pro, prologue, epi, epilogue)
     return call
 
 

@@ -75,6 +75,14 @@ int check_prologue(const gdr_prologue *p, const float *g) {
     return GDR_OK;
 }
 
+int check_epilogue(const gdr_epilogue *e) {
+    if (!e) return GDR_OK;
+    if (!e->z || !e->norm_w) return GDR_ERR_NULL;
+    if (!(e->eps >= 0.f)) return GDR_ERR_SHAPE;
+    if (!aligned16(e->z) || !aligned16(e->norm_w)) return GDR_ERR_ALIGN;
+    return GDR_OK;
+}
+
 }  // namespace
 }  // namespace gdr
 
@@ -83,10 +91,11 @@ using namespace gdr;
 extern "C" int gdr_chunk_fwd(const void *q, const void *k, const void *v, const void *beta, const float *g,
                              const void *initial_state, const int32_t *actual_seq_lengths, float scale, int B,
                              int Nk, int Nv, int S, int Dk, int Dv, gdr_dtype dtype, const gdr_prologue *prologue,
-                             void *out, void *final_state, gdr_stream_t stream) {
+                             const gdr_epilogue *epilogue, void *out, void *final_state, gdr_stream_t stream) {
     int st = check_common(B, Nk, Nv, S, Dk, Dv, dtype);
     if (st) return st;
     if ((st = check_prologue(prologue, g))) return st;
+    if ((st = check_epilogue(epilogue))) return st;
     if ((long long)B * S > 0 && (!q || !k || !v || !beta || !out)) return GDR_ERR_NULL;
     const void *ptrs[] = {q, k, v, beta, g, initial_state, actual_seq_lengths, out, final_state};
     for (const void *p : ptrs)
@@ -109,7 +118,20 @@ extern "C" int gdr_chunk_fwd(const void *q, const void *k, const void *v, const 
     a.dt_bias = prologue ? prologue->dt_bias : nullptr;
     a.err = err;
     cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
-    cudaError_t e = chunk_tc_supported(Dk, Dv, dtype, S) ? launch_chunk_tc(a, cs) : launch_chunk_simt(a, Dk, Dv, dtype, cs);
+    cudaError_t e;
+    if (chunk_tc_supported(Dk, Dv, dtype, S)) {
+        if (epilogue) {  // fused into the tensor-core kernel's out epilogue
+            a.epi_z = epilogue->z;
+            a.epi_w = epilogue->norm_w;
+            a.epi_eps = epilogue->eps;
+        }
+        e = launch_chunk_tc(a, cs);
+    } else {
+        e = launch_chunk_simt(a, Dk, Dv, dtype, cs);
+        if (e == cudaSuccess && epilogue && S > 0)
+            e = launch_gated_rmsnorm(out, epilogue->z, epilogue->norm_w, epilogue->eps, actual_seq_lengths, B, Nv,
+                                     S, Dv, dtype, cs);
+    }
     return e == cudaSuccess ? GDR_OK : GDR_ERR_LAUNCH;
 }
 
@@ -117,13 +139,14 @@ extern "C" int gdr_recurrent_step(const void *q, const void *k, const void *v, c
                                   const float *gk, void *state_pool, int slots, const int32_t *ssm_state_indices,
                                   const int32_t *actual_seq_lengths, const int32_t *num_accepted_tokens,
                                   float scale, int B, int Nk, int Nv, int S, int Dk, int Dv, gdr_dtype dtype,
-                                  gdr_dtype state_dtype, const gdr_prologue *prologue, void *out,
-                                  gdr_stream_t stream) {
+                                  gdr_dtype state_dtype, const gdr_prologue *prologue,
+                                  const gdr_epilogue *epilogue, void *out, gdr_stream_t stream) {
     int st = check_common(B, Nk, Nv, S, Dk, Dv, dtype);
     if (st) return st;
     if (state_dtype != GDR_F32 && state_dtype != GDR_BF16) return GDR_ERR_DTYPE;
     if (S < 1 || S > kDecodeMaxTokens || slots < 1) return GDR_ERR_SHAPE;
     if ((st = check_prologue(prologue, g))) return st;
+    if ((st = check_epilogue(epilogue))) return st;
     if (B > 0 && (!q || !k || !v || !beta || !out || !state_pool || !ssm_state_indices || !actual_seq_lengths))
         return GDR_ERR_NULL;
     const void *ptrs[] = {q, k, v, beta, g, gk, state_pool, ssm_state_indices, actual_seq_lengths,
@@ -147,7 +170,11 @@ extern "C" int gdr_recurrent_step(const void *q, const void *k, const void *v, c
     a.A_log = prologue ? prologue->A_log : nullptr;
     a.dt_bias = prologue ? prologue->dt_bias : nullptr;
     a.err = err;
-    cudaError_t e = launch_decode(a, Dk, Dv, dtype, state_dtype, reinterpret_cast<cudaStream_t>(stream));
+    cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = launch_decode(a, Dk, Dv, dtype, state_dtype, cs);
+    if (e == cudaSuccess && epilogue)
+        e = launch_gated_rmsnorm(out, epilogue->z, epilogue->norm_w, epilogue->eps, actual_seq_lengths, B, Nv, S, Dv,
+                                 dtype, cs);
     return e == cudaSuccess ? GDR_OK : GDR_ERR_LAUNCH;
 }
 

@@ -18,7 +18,8 @@
 //       S += (diag(e^{G_last-G}) K)^T v_new       tcgen05.mma  accumulate into the TMEM state
 //       R[64:128] += Pm v_new,  Pm = (X K^T) e^{G_t-G_s} (causal)  -> o
 //   a6  o -> bf16 -> TMA store; padding rows and chunks are zero; the final state is
-//       written once from TMEM.
+//       written once from TMEM.  With the optional epilogue each o row first becomes
+//       o / sqrt(mean o^2 + eps) * norm_w * silu(z) in fp32 (the layer's gated RMSNorm).
 //
 // X = scale * q / |q| (the fused l2norm and the 1/|k| factors are folded into row and
 // column scalings, so the raw q/k tiles feed the tensor cores directly).
@@ -80,7 +81,8 @@ namespace {
 constexpr int C = 64, D = 128, NGRP = 256, NHELP = 96, NT = 2 * NGRP + 32 + NHELP, NPC = NGRP + 32;
 constexpr int CTL_WARP = 16;
 // BAR_PCTL: the prep warps and the control warp, at the hand-offs between them; BAR_HELP: the helper warps
-constexpr int BAR_CARRY = 1, BAR_PREP = 2, BAR_PCTL = 3, BAR_HELP = 4;
+// BAR_EPI: the carry warps that hold o rows (TMEM lanes 64..127), at the epilogue's row-norm exchange
+constexpr int BAR_CARRY = 1, BAR_PREP = 2, BAR_PCTL = 3, BAR_HELP = 4, BAR_EPI = 5;
 constexpr uint32_t kTimeoutBit = 0x4u;
 // carry thread that issues the out-tile TMA stores (thread 0 issues the carry's MMAs)
 constexpr int kStorer = 32;
@@ -118,7 +120,8 @@ constexpr int NVEC = 12;             // per-chunk vectors of 64 floats (enum bel
 constexpr uint32_t OFF_VEC = 215040;  // 2 sets x NVEC vectors x 64 floats
 static_assert(OFF_XM + 32 * SP * 4 <= OFF_VEC, "merge product");
 constexpr uint32_t OFF_BAR = OFF_VEC + 2 * NVEC * 64 * 4;
-constexpr uint32_t SMEM_USED = OFF_BAR + 128;
+constexpr uint32_t OFF_EPI = OFF_BAR + 128;  // epilogue: partial squared norms of the o rows (2 x 64 floats)
+constexpr uint32_t SMEM_USED = OFF_EPI + 512;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;  // + alignment slack
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 static_assert(OFF_TT % 1024 == 0, "swizzle atoms");
@@ -148,10 +151,22 @@ struct TcArgs {
     int beta_logits;
     const float *A_log, *dt_bias;
     unsigned int *err;
+    const __nv_bfloat16 *epi_z;  // NULL: no epilogue
+    const float *epi_w;
+    float epi_eps;
 };
 
 __device__ __forceinline__ uint32_t blk_off(uint32_t row, uint32_t col) {  // within a 128-B-row block
     return (row >> 3) * 1024u + sw128_offset(row & 7u, col);
+}
+
+// silu(x) = x sigmoid(x) with sigmoid(x) = (1 + tanh(x / 2)) / 2 and tanh on the special-function unit (PTX
+// tanh.approx, relative error about 2^-11): one special-function operation per element; the result is rounded
+// to bf16 (2^-9) right after
+__device__ __forceinline__ float silu_fast(float x) {
+    float t;
+    asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(0.5f * x));
+    return x * fmaf(0.5f, t, 0.5f);
 }
 
 // 2^x and log2(x) on the special-function unit (PTX ex2.approx / lg2.approx, flush to zero)
@@ -392,6 +407,12 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             tma_prefetch_3d(&tm_q, 64, y, zq);
             tma_prefetch_3d(&tm_v, 0, y, bh);
             tma_prefetch_3d(&tm_v, 64, y, bh);
+            if (a.epi_z) {  // the chunk's z rows of the epilogue: one contiguous block of valid rows
+                const int rows = min(C, L - y);
+                asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(a.epi_z + ((size_t)bh * S + y) * D),
+                             "r"((uint32_t)(rows * D * 2))
+                             : "memory");
+            }
         };
         // K of a chunk into its buffer (this also arms the chunk's K/Q barrier), Q into the single Q buffer,
         // V into the single V buffer
@@ -838,6 +859,9 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                             pack8(&u[8 * c8]);
                 }
             } else {  // rows of Q S: scale by e^{G_t} scale / |q_t| before Pm v_new accumulates onto them
+                if (a.epi_z && row - 64 < n)  // this thread's half row of z, for the epilogue
+                    asm volatile("prefetch.global.L1 [%0];" ::"l"(a.epi_z + ((size_t)bh * S + (size_t)c * C + row - 64) *
+                                                                        D + 64 * hf));
                 const float xs = vec[V_XS * 64 + row - 64];
 #pragma unroll
                 for (int half = 0; half < 2; ++half) {
@@ -912,11 +936,45 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             if (more) tmem_st_wait();
             if (q4 >= 2) {
                 const int t = row - 64;
+                // epilogue: the row's squared norm from its two halves (this thread and the one of the other hf
+                // warp with the same lane), then o * inv * norm_w * silu(z) for this thread's 64 columns
+                const bool epi = a.epi_z != nullptr;
+                float inv = 1.f;
+                const __nv_bfloat16 *zr = nullptr;
+                if (epi) {
+                    float ss = 0.f;
+#pragma unroll
+                    for (int half = 0; half < 2; ++half) {
+                        float o[32];
+                        tmem_ld32(tmem + TM_R + lane_base + 64 * hf + 32 * half, o);
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) ss = fmaf(o[j], o[j], ss);
+                    }
+                    float *eps2 = reinterpret_cast<float *>(sm + OFF_EPI);
+                    eps2[hf * 64 + t] = ss;
+                    if (t < n) zr = a.epi_z + ((size_t)bh * S + (size_t)c * C + t) * D + 64 * hf;  // rows past the
+                                                                                                   // length: unread
+                    named_sync(BAR_EPI, 128);
+                    inv = rsqrtf((eps2[t] + eps2[64 + t]) * (1.f / D) + a.epi_eps);
+                }
 #pragma unroll
                 for (int half = 0; half < 2; ++half) {
                     float o[32];
                     tmem_ld32(tmem + TM_R + lane_base + 64 * hf + 32 * half, o);
                     tmem_ld_wait();
+                    if (epi && t < n) {
+#pragma unroll
+                        for (int c8 = 0; c8 < 4; ++c8) {
+                            float zf[8];
+                            unpack8(*reinterpret_cast<const uint4 *>(zr + 32 * half + 8 * c8), zf);
+                            const float4 *wp = reinterpret_cast<const float4 *>(a.epi_w + 64 * hf + 32 * half + 8 * c8);
+                            const float4 w0 = wp[0], w1 = wp[1];
+                            const float wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+#pragma unroll
+                            for (int i = 0; i < 8; ++i) o[8 * c8 + i] *= inv * wv[i] * silu_fast(zf[i]);
+                        }
+                    }
 #pragma unroll
                     for (int j = 0; j < 32; ++j) o[j] = t < n ? o[j] : 0.f;
 #pragma unroll
@@ -1015,6 +1073,7 @@ cudaError_t launch_chunk_tc(const ChunkArgs &ca, cudaStream_t stream) {
     a.B = ca.B; a.Nk = ca.Nk; a.Nv = ca.Nv; a.S = ca.S; a.final_state = ca.final_state;
     a.l2norm = ca.l2norm; a.eps = ca.eps; a.beta_logits = ca.beta_logits; a.A_log = ca.A_log;
     a.dt_bias = ca.dt_bias; a.err = ca.err;
+    a.epi_z = static_cast<const __nv_bfloat16 *>(ca.epi_z); a.epi_w = ca.epi_w; a.epi_eps = ca.epi_eps;
     static bool attr_set = false;
     if (!attr_set) {
         cudaError_t e = cudaFuncSetAttribute(chunk_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);

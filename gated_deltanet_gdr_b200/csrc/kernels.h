@@ -41,6 +41,10 @@ struct ChunkArgs {
     int beta_logits;
     const float *A_log, *dt_bias;
     unsigned int *err;
+    // fused gated RMSNorm epilogue (tensor-core path only): z (B, Nv, S, Dv) in the input dtype, norm_w (Dv)
+    const void *epi_z;
+    const float *epi_w;
+    float epi_eps;
 };
 
 // cuTensorMapEncodeTiled, obtained once through the runtime's driver entry point (NULL if unavailable).
@@ -53,6 +57,9 @@ cudaError_t launch_decode(const DecodeArgs &a, int Dk, int Dv, gdr_dtype dt, gdr
 bool chunk_tc_supported(int Dk, int Dv, gdr_dtype dt, int S);
 cudaError_t launch_chunk_tc(const ChunkArgs &a, cudaStream_t s);
 cudaError_t launch_chunk_simt(const ChunkArgs &a, int Dk, int Dv, gdr_dtype dt, cudaStream_t s);
+// out rows t < L_b <- rmsnorm(out row) * norm_w * silu(z row), in place (the unfused epilogue)
+cudaError_t launch_gated_rmsnorm(void *out, const void *z, const float *norm_w, float eps, const int32_t *lengths,
+                                 int B, int Nv, int S, int Dv, gdr_dtype dt, cudaStream_t s);
 cudaError_t launch_prologue(const void *q, const void *k, const void *b, const float *a, const float *A_log,
                             const float *dt_bias, float eps, int B, int Nk, int Nv, int S, int Dk, gdr_dtype dt,
                             void *q_hat, void *k_hat, void *beta, float *g, cudaStream_t stream);

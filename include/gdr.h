@@ -94,6 +94,33 @@ typedef struct gdr_prologue {
 } gdr_prologue;
 
 /*
+ * Optional output epilogue: the gated RMSNorm the layer applies to each head's
+ * output row before its output projection, fused into the call.  Source: the
+ * per-head gated RMSNorm of deltanet.rs and of its WGSL core shader (mean of
+ * the squares over the head's Dv outputs, eps inside the square root, times the
+ * norm weight and silu of the head's slice of z), applied by the transformers
+ * layer as self.norm(core_attn_out, z) (blog "gated-delta-net" page; its
+ * comment names the gate sigmoid(z), both code listings use silu).
+ *
+ *   z        device (B, Nv, S, Dv) in dtype: the layer's output gate branch
+ *   norm_w   device fp32 (Dv): the RMSNorm weight, shared by all heads
+ *   eps      added to the mean square inside the square root (>= 0)
+ *
+ * With it, out row (b, h, t) for t < L_b holds, computed in fp32 and rounded
+ * once to dtype:
+ *     o / sqrt(mean_j o_j^2 + eps) * norm_w * silu(z),  silu(x) = x / (1 + e^{-x})
+ * where o is the row the rule produces; padding rows stay zero.  The bf16
+ * tensor-core prefill applies it to the fp32 row before rounding; the other
+ * paths apply it to the row already stored in dtype (for bf16 that rounds o
+ * once more, within the bf16 tolerance).  z and norm_w must be 16-byte aligned.
+ */
+typedef struct gdr_epilogue {
+    const void *z;
+    const float *norm_w;
+    float eps;
+} gdr_epilogue;
+
+/*
  * Chunked prefill.  Source: lite_boost chunk_gated_delta_rule (arguments,
  * BNSD layout, GQA, variable lengths with padding written as zero, optional
  * gate, final state) and torch_chunk_gated_delta_rule (chunk size 64,
@@ -110,17 +137,20 @@ typedef struct gdr_prologue {
  *                          non-finite values) and out rows t >= L_b are zero.
  *                          L_b = 0 gives final_state = initial_state exactly.
  *   scale                  multiplies q before the rule (1/sqrt(Dk) in the layer)
+ *   epilogue               NULL, or the fused gated RMSNorm of the out rows
+ *                          (see gdr_epilogue)
  *   out                    device (B, Nv, S, Dv), written in full
  *   final_state            device (B, Nv, Dk, Dv) or NULL: not written.  It
  *                          may alias initial_state (in-place update).
  * Constraints: B, S >= 0; Nk, Nv >= 1; Nv % Nk == 0; Dk, Dv in {16,32,64,128};
- * every pointer 16-byte aligned.  bf16 with Dk = Dv = 128 runs on the
+ * every pointer 16-byte aligned.  An epilogue with a NULL z or norm_w returns
+ * GDR_ERR_NULL, one with eps < 0 (or NaN) GDR_ERR_SHAPE.  bf16 with Dk = Dv = 128 runs on the
  * tensor-core (tcgen05) path; other shapes and fp32 run the CUDA-core path.
  */
 int gdr_chunk_fwd(const void *q, const void *k, const void *v, const void *beta, const float *g,
                   const void *initial_state, const int32_t *actual_seq_lengths, float scale, int B, int Nk,
-                  int Nv, int S, int Dk, int Dv, gdr_dtype dtype, const gdr_prologue *prologue, void *out,
-                  void *final_state, gdr_stream_t stream);
+                  int Nv, int S, int Dk, int Dv, gdr_dtype dtype, const gdr_prologue *prologue,
+                  const gdr_epilogue *epilogue, void *out, void *final_state, gdr_stream_t stream);
 
 /*
  * Recurrent decode over a pool of state slots.  Source: lite_boost
@@ -139,6 +169,8 @@ int gdr_chunk_fwd(const void *q, const void *k, const void *v, const void *beta,
  *   actual_seq_lengths     device int32 (B): tokens processed for sequence b,
  *                          in [0, S]; out rows t >= L_b are zero
  *   num_accepted_tokens    device int32 (B), or NULL (= actual_seq_lengths)
+ *   epilogue               NULL, or the gated RMSNorm of the out rows (see
+ *                          gdr_epilogue)
  *   out                    device (B, Nv, S, Dv), written in full
  * Reading of num_accepted_tokens (the operator defines it only as the count of
  * accepted tokens, equal to the lengths in plain inference): the chain starts
@@ -154,7 +186,8 @@ int gdr_recurrent_step(const void *q, const void *k, const void *v, const void *
                        const float *gk, void *state_pool, int slots, const int32_t *ssm_state_indices,
                        const int32_t *actual_seq_lengths, const int32_t *num_accepted_tokens, float scale, int B,
                        int Nk, int Nv, int S, int Dk, int Dv, gdr_dtype dtype, gdr_dtype state_dtype,
-                       const gdr_prologue *prologue, void *out, gdr_stream_t stream);
+                       const gdr_prologue *prologue, const gdr_epilogue *epilogue, void *out,
+                       gdr_stream_t stream);
 
 /*
  * Stand-alone prologue (the same arithmetic the fused prologue applies), for

@@ -50,19 +50,20 @@ NUL = None
 
 def chunk(L, **kw):
     a = dict(q=P, k=P, v=P, beta=P, g=NUL, s0=NUL, lens=NUL, scale=1.0, B=1, Nk=2, Nv=4, S=8, Dk=128, Dv=128,
-             dt=gdr.GDR_BF16, pro=None, out=P, fin=NUL)
+             dt=gdr.GDR_BF16, pro=None, epi=None, out=P, fin=NUL)
     a.update(kw)
     return L.gdr_chunk_fwd(a["q"], a["k"], a["v"], a["beta"], a["g"], a["s0"], a["lens"], a["scale"], a["B"],
-                           a["Nk"], a["Nv"], a["S"], a["Dk"], a["Dv"], a["dt"], a["pro"], a["out"], a["fin"], None)
+                           a["Nk"], a["Nv"], a["S"], a["Dk"], a["Dv"], a["dt"], a["pro"], a["epi"], a["out"], a["fin"],
+                           None)
 
 
 def decode(L, **kw):
     a = dict(q=P, k=P, v=P, beta=P, g=NUL, gk=NUL, pool=P, slots=4, idx=P, lens=P, acc=NUL, scale=1.0, B=1, Nk=2,
-             Nv=4, S=1, Dk=128, Dv=128, dt=gdr.GDR_BF16, sdt=gdr.GDR_BF16, pro=None, out=P)
+             Nv=4, S=1, Dk=128, Dv=128, dt=gdr.GDR_BF16, sdt=gdr.GDR_BF16, pro=None, epi=None, out=P)
     a.update(kw)
     return L.gdr_recurrent_step(a["q"], a["k"], a["v"], a["beta"], a["g"], a["gk"], a["pool"], a["slots"], a["idx"],
                                 a["lens"], a["acc"], a["scale"], a["B"], a["Nk"], a["Nv"], a["S"], a["Dk"], a["Dv"],
-                                a["dt"], a["sdt"], a["pro"], a["out"], None)
+                                a["dt"], a["sdt"], a["pro"], a["epi"], a["out"], None)
 
 
 def test_chunk_host_validation(L):
@@ -83,6 +84,14 @@ def test_chunk_host_validation(L):
     assert chunk(L, pro=ctypes.byref(pro)) == gdr.GDR_ERR_NULL
     pro = gdr.GdrPrologueStruct(1, -1.0, 0, None, None)  # negative eps
     assert chunk(L, pro=ctypes.byref(pro)) == gdr.GDR_ERR_SHAPE
+    epi = gdr.GdrEpilogueStruct(4096, None, 1e-6)  # epilogue without norm_w
+    assert chunk(L, epi=ctypes.byref(epi)) == gdr.GDR_ERR_NULL
+    epi = gdr.GdrEpilogueStruct(None, 4096, 1e-6)  # epilogue without z
+    assert chunk(L, epi=ctypes.byref(epi)) == gdr.GDR_ERR_NULL
+    epi = gdr.GdrEpilogueStruct(4096, 4096, -1.0)  # negative eps
+    assert chunk(L, epi=ctypes.byref(epi)) == gdr.GDR_ERR_SHAPE
+    epi = gdr.GdrEpilogueStruct(4104, 4096, 1e-6)  # misaligned z
+    assert chunk(L, epi=ctypes.byref(epi)) == gdr.GDR_ERR_ALIGN
     # nothing to do: B == 0 returns OK without touching a device
     assert chunk(L, B=0, q=NUL, k=NUL, v=NUL, beta=NUL, out=NUL) == gdr.GDR_OK
 
@@ -98,6 +107,10 @@ def test_decode_host_validation(L):
     assert decode(L, lens=NUL) == gdr.GDR_ERR_NULL
     assert decode(L, gk=ctypes.c_void_p(4100)) == gdr.GDR_ERR_ALIGN
     assert decode(L, Dk=48) == gdr.GDR_ERR_UNSUPPORTED
+    epi = gdr.GdrEpilogueStruct(4096, None, 1e-6)
+    assert decode(L, epi=ctypes.byref(epi)) == gdr.GDR_ERR_NULL
+    epi = gdr.GdrEpilogueStruct(4096, 4096, float("nan"))
+    assert decode(L, epi=ctypes.byref(epi)) == gdr.GDR_ERR_SHAPE
     assert decode(L, B=0) == gdr.GDR_OK
 
 

@@ -108,7 +108,7 @@ def generate(name: str, *, B=None, S=None, Nk=None, Nv=None, D=None, seed=None, 
     v = _normal(rng, (B, Nv, S, D), dtype=fd)
     b = _normal(rng, (B, Nv, S), dtype=fd)
     w = Workload(name=name, B=B, Nk=Nk, Nv=Nv, S=S, Dk=D, Dv=D, dtype=dt, scale=1.0 / math.sqrt(D),
-                 q=q, k=k, v=v, b=b, lengths=np.full(B, S, np.int32))
+                 q=q, k=k, v=v, b=b, lengths=np.full(B, S, np.int32), meta={"seed": seed, "fd": fd})
     if name in ("tiny", "decode", "decode_gk"):
         w.g = _loguniform_gate(rng, (B, Nv, S), 0.9, 0.999, np.float32 if dt == "bf16" else fd)
     else:
@@ -153,7 +153,8 @@ def random_case(*, B, Nk, Nv, S, Dk, Dv, seed, gate="loguniform", lengths=None, 
     v = _normal(rng, (B, Nv, S, Dv), dtype=fd)
     b = _normal(rng, (B, Nv, S), dtype=fd)
     w = Workload(name=f"case{seed}", B=B, Nk=Nk, Nv=Nv, S=S, Dk=Dk, Dv=Dv, dtype="f32",
-                 scale=1.0 / math.sqrt(Dk), q=q, k=k, v=v, b=b, lengths=np.full(B, S, np.int32))
+                 scale=1.0 / math.sqrt(Dk), q=q, k=k, v=v, b=b, lengths=np.full(B, S, np.int32),
+                 meta={"seed": seed, "fd": fd})
     if gate == "loguniform":
         w.g = _loguniform_gate(rng, (B, Nv, S), 0.9, 0.999, fd)
     elif gate == "strong":
@@ -177,3 +178,13 @@ def random_case(*, B, Nk, Nv, S, Dk, Dv, seed, gate="loguniform", lengths=None, 
             w.indices = rng.permutation(slots)[:B * S].astype(np.int32)
         w.accepted = np.array([rng.integers(0, L, endpoint=True) if L > 0 else 0 for L in w.lengths], np.int32)
     return w
+
+
+def epilogue_inputs(w: Workload):
+    """The output gate branch z ~ N(0, 1), shape (B, Nv, S, Dv), and the RMSNorm weight
+    norm_w ~ U(0.5, 1.5), shape (Dv,), of the layer's output epilogue.  Drawn from a stream of
+    their own (seeded by the workload's seed and 1), so the workload's other draws are unchanged."""
+    rng = np.random.default_rng([int(w.meta["seed"]), 1])
+    z = _normal(rng, (w.B, w.Nv, w.S, w.Dv), dtype=w.meta.get("fd", np.float32))
+    norm_w = rng.uniform(0.5, 1.5, size=w.Dv).astype(np.float32)
+    return z, norm_w
