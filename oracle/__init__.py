@@ -7,8 +7,9 @@ import it.  It shares no code with the CUDA path and never calls it.
 ``gdr_oracle.c`` holds the token-by-token definition (compiled here with gcc,
 no fast-math); ``forms.py`` holds independent formulations from the pages
 (the chunked WY form, the pseudo-value form, gated linear attention by brute
-force) used to pin it.  ``gated_rmsnorm`` is the layer's output epilogue, written
-out from its definition and pinned by closed forms.  Every function here is pinned by
+force) used to pin it.  ``gated_rmsnorm`` is the layer's output epilogue and
+``causal_conv1d`` the depthwise causal convolution before the rule, each written
+out from its definition and pinned by closed forms and library routines.  Every function here is pinned by
 ``tests/test_oracle_pins.py`` (closed forms, worked examples printed on the
 pages, independent formulations, brute force, invariants); none is left
 unpinned.
@@ -29,7 +30,7 @@ _LIB_PATH = os.path.join(_BUILD, "libgdr_oracle.so")
 _lock = threading.Lock()
 _lib = None
 
-__all__ = ["build", "lib", "prologue", "chunk_fwd", "recurrent_step", "gated_rmsnorm", "threads"]
+__all__ = ["build", "lib", "prologue", "chunk_fwd", "recurrent_step", "gated_rmsnorm", "causal_conv1d", "threads"]
 
 
 def build(force: bool = False) -> str:
@@ -207,3 +208,41 @@ def gated_rmsnorm(o, z, norm_w, eps: float, actual_seq_lengths=None):
     y = oa * inv * wa * (za / (1.0 + np.exp(-za)))
     t = np.arange(S)[None, None, :, None]
     return np.where(t < L[:, None, None, None], y, oa)
+
+
+def causal_conv1d(x, weight, bias=None, conv_state=None, actual_seq_lengths=None):
+    """fp64 depthwise causal convolution with SiLU over the fused q/k/v channels, and its state.
+
+    For sequence b with L = L_b valid positions, channel c, taps w[c, 0..K-1] oldest first:
+
+        y[t, c] = silu(bias[c] + sum_j w[c, j] * x[t - K + 1 + j, c]),   0 <= t < L,
+
+    where the positions before 0 are the K inputs held in the state (newest last; zeros without one).
+    The state afterwards holds the last K inputs of that history (the state followed by x[0..L-1]).
+    Rows t >= L are zero.
+
+    Source: the layer's conv over mixed_qkv = cat(q, k, v) with causal_conv1d_fn / causal_conv1d_update
+    and conv_state = F.pad(mixed_qkv, (K - L, 0)) (blog "gated-delta-net" page), and deltanet.rs's
+    per-channel ring of the last K inputs (shift, append, dot with the taps oldest first, silu) with its
+    WGSL twin.
+
+    x: (B, S, C) channels last; weight: (C, K); bias: (C,) or None; conv_state: (B, C, K) or None;
+    actual_seq_lengths: (B,) or None (all S).  Returns (y (B, S, C), new_state (B, C, K)).
+    """
+    xa, wa = _f64(x), _f64(weight)
+    B, S, C = xa.shape
+    K = wa.shape[1]
+    if wa.shape != (C, K):
+        raise ValueError("weight must be (C, K)")
+    ba = np.zeros(C) if bias is None else _f64(bias)
+    st = np.zeros((B, C, K)) if conv_state is None else _f64(conv_state)
+    L = np.full(B, S, np.int64) if actual_seq_lengths is None else np.asarray(actual_seq_lengths, np.int64)
+    y = np.zeros((B, S, C))
+    new = np.empty((B, C, K))
+    for b in range(B):
+        hist = np.concatenate([st[b].T, xa[b, :L[b]]], axis=0)  # (K + L, C): the K state inputs, then x
+        for t in range(L[b]):
+            acc = ba + np.sum(wa.T * hist[t + 1:t + 1 + K], axis=0)
+            y[b, t] = acc / (1.0 + np.exp(-acc))
+        new[b] = hist[L[b]:L[b] + K].T
+    return y, new

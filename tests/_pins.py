@@ -335,3 +335,83 @@ def check_epi_padding(impl):
 
 
 EPILOGUE_CHECKS = [check_epi_constant_row, check_epi_row_mean, check_epi_invariants, check_epi_padding]
+
+
+# ---- the depthwise causal conv1d + SiLU before the rule: impl(x, w, bias, state, lengths) -> (y, state) ----
+
+def check_conv_special_taps(impl):
+    """One-hot taps with inputs whose silu is exact: 0 (silu 0), ln 3 (silu = (3/4) ln 3) and 50 (silu = 50
+    to double precision).  The newest tap passes x through; the oldest delays it by K - 1 positions, with
+    the zero history in front."""
+    K = 4
+    vals = np.array([0.0, math.log(3.0), 50.0, 0.0, 50.0, math.log(3.0), 50.0])
+    silu = {0.0: 0.0, math.log(3.0): 0.75 * math.log(3.0), 50.0: 50.0}
+    x = vals.reshape(1, -1, 1)
+    newest = np.zeros((1, K)); newest[0, K - 1] = 1.0
+    y, _ = impl(x, newest, None, None, None)
+    assert np.allclose(y[0, :, 0], [silu[v] for v in vals], rtol=0, atol=1e-14)
+    oldest = np.zeros((1, K)); oldest[0, 0] = 1.0
+    y, _ = impl(x, oldest, None, None, None)
+    want = [0.0] * (K - 1) + [silu[v] for v in vals[:len(vals) - K + 1]]
+    assert np.allclose(y[0, :, 0], want, rtol=0, atol=1e-14)
+
+
+def check_conv_against_library_convolution(impl):
+    """The pre-activation of every channel equals numpy's full convolution of the channel with its taps in
+    reverse order (taps are stored oldest first), truncated to the sequence; checked through
+    silu^-1 of the output on a monotone range (|pre| < 2 keeps silu invertible by bisection)."""
+    rng = np.random.default_rng(21)
+    B, S, C, K = 2, 19, 5, 4
+    x = rng.uniform(-0.3, 0.3, (B, S, C))
+    w = rng.uniform(-0.5, 0.5, (C, K))
+    bias = rng.uniform(-0.2, 0.2, C)
+    y, _ = impl(x, w, bias, None, None)
+    for b in range(B):
+        for c in range(C):
+            pre = np.convolve(x[b, :, c], w[c, ::-1])[:S] + bias[c]
+            lo, hi = np.full(S, -1.2), np.full(S, 2.0)  # silu is increasing on [-1.2, inf)
+            for _ in range(80):
+                mid = 0.5 * (lo + hi)
+                f = mid / (1.0 + np.exp(-mid))
+                lo, hi = np.where(f < y[b, :, c], mid, lo), np.where(f < y[b, :, c], hi, mid)
+            assert np.allclose(lo, pre, rtol=0, atol=1e-12)
+
+
+def check_conv_state_handoff(impl):
+    """Running [0, s) and then [s, S) with the state carried equals one run over [0, S), for every split
+    (s = 1, 2 and 3 are shorter than the window: the history then comes partly from the state), and the
+    final state holds the last K inputs."""
+    rng = np.random.default_rng(22)
+    B, S, C, K = 2, 11, 3, 4
+    x = rng.standard_normal((B, S, C))
+    w = rng.standard_normal((C, K))
+    bias = rng.standard_normal(C)
+    s0 = rng.standard_normal((B, C, K))
+    y_all, st_all = impl(x, w, bias, s0, None)
+    assert np.array_equal(st_all, np.transpose(x[:, S - K:], (0, 2, 1)))
+    for s in range(1, S):
+        y1, st1 = impl(x[:, :s], w, bias, s0, None)
+        y2, st2 = impl(x[:, s:], w, bias, st1, None)
+        assert np.allclose(np.concatenate([y1, y2], 1), y_all, rtol=0, atol=1e-13)
+        assert np.allclose(st2, st_all, rtol=0, atol=0)
+
+
+def check_conv_lengths(impl):
+    """Rows t >= L are zero and do not reach the state: L = 0 keeps the state, L = 1 shifts it by one, and a
+    padded batch row equals the unpadded run."""
+    rng = np.random.default_rng(23)
+    B, S, C, K = 3, 7, 4, 3
+    x = rng.standard_normal((B, S, C))
+    w = rng.standard_normal((C, K))
+    s0 = rng.standard_normal((B, C, K))
+    L = np.array([0, 1, 5])
+    y, st = impl(x, w, None, s0, L)
+    assert np.all(y[0] == 0) and np.all(y[1, 1:] == 0) and np.all(y[2, 5:] == 0)
+    assert np.array_equal(st[0], s0[0])
+    assert np.array_equal(st[1], np.concatenate([s0[1][:, 1:], x[1, :1].T], axis=1))
+    y2, st2 = impl(x[2:, :5], w, None, s0[2:], None)
+    assert np.allclose(y[2, :5], y2[0], rtol=0, atol=1e-15) and np.array_equal(st[2], st2[0])
+
+
+CONV_CHECKS = [check_conv_special_taps, check_conv_against_library_convolution, check_conv_state_handoff,
+               check_conv_lengths]

@@ -221,3 +221,12 @@ def test_oracle_is_thread_count_independent():
 @pytest.mark.parametrize("check", _pins.EPILOGUE_CHECKS, ids=lambda c: c.__name__)
 def test_gated_rmsnorm_oracle_pin(check):
     check(oracle.gated_rmsnorm)
+
+
+def conv_impl(x, w, bias, state, lengths):
+    return oracle.causal_conv1d(x, w, bias, state, lengths)
+
+
+@pytest.mark.parametrize("check", _pins.CONV_CHECKS, ids=lambda c: c.__name__)
+def test_causal_conv1d_oracle_pin(check):
+    check(conv_impl)

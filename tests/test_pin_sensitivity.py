@@ -121,3 +121,50 @@ def test_planted_epilogue_mistake_is_caught(mutation):
         except AssertionError:
             caught += 1
     assert caught > 0, mutation
+
+
+def make_conv(mutation=None):
+    """A plain copy of the depthwise causal conv + SiLU with its state, with planted mistakes."""
+    def impl(x, w, bias, state, lengths):
+        x, w = np.asarray(x, np.float64), np.asarray(w, np.float64)
+        B, S, C = x.shape
+        K = w.shape[1]
+        bias = np.zeros(C) if bias is None or mutation == "conv_no_bias" else np.asarray(bias, np.float64)
+        st = np.zeros((B, C, K)) if state is None or mutation == "conv_state_ignored" else np.asarray(state)
+        taps = w[:, ::-1] if mutation == "conv_taps_reversed" else w
+        y = np.zeros((B, S, C))
+        new = np.empty((B, C, K))
+        for b in range(B):
+            L = S if lengths is None else int(lengths[b])
+            hist = np.concatenate([st[b].T, x[b, :L]], axis=0)
+            off = 0 if mutation == "conv_window_late" else 1
+            for t in range(L):
+                win = hist[t + off:t + off + K]
+                acc = bias + np.sum(taps.T * win, axis=0)
+                y[b, t] = 1.0 / (1.0 + np.exp(-acc)) if mutation == "conv_sigmoid" else acc / (1.0 + np.exp(-acc))
+            keep = hist[L:L + K] if mutation != "conv_state_short" else np.concatenate([np.zeros((1, C)),
+                                                                                         hist[L + 1:L + K]], 0)
+            new[b] = keep.T
+        return y, new
+    return impl
+
+
+CONV_MUTATIONS = ["conv_no_bias", "conv_state_ignored", "conv_taps_reversed", "conv_window_late", "conv_sigmoid",
+                  "conv_state_short"]
+
+
+def test_unmodified_conv_copy_passes_every_pin():
+    for check in _pins.CONV_CHECKS:
+        check(make_conv())
+
+
+@pytest.mark.parametrize("mutation", CONV_MUTATIONS)
+def test_planted_conv_mistake_is_caught(mutation):
+    impl = make_conv(mutation)
+    caught = 0
+    for check in _pins.CONV_CHECKS:
+        try:
+            check(impl)
+        except (AssertionError, IndexError, ValueError):
+            caught += 1
+    assert caught > 0, mutation
