@@ -344,6 +344,40 @@ def bench_prefill_epilogue(gdr, args, world, w, t, pro, flush, stream, peaks):
                          alg_bytes, "kernel": "gdr_chunk_fwd (fused prologue and epilogue)"}}, args.steps
 
 
+def bench_conv1d(gdr, args, world, rank, flush, stream, peaks):
+    """The depthwise causal conv1d + SiLU before the rule on the prefill workload's layout (C = 2 Nk Dk +
+    Nv Dv = 8192 channels, K = 4, bf16, with bias and input state), writing q, k, v and the new state."""
+    w = workloads.generate("prefill", seed=2 + 1000 * rank)
+    x, wt, bias, st = workloads.conv_inputs(w, 4)
+    x, wt, bias, st = bf16_dev(x), bf16_dev(wt), bf16_dev(bias), bf16_dev(st)
+    B, S, C = x.shape
+    q = torch.empty((B, w.Nk, S, w.Dk), dtype=torch.bfloat16, device="cuda")
+    k, v = torch.empty_like(q), torch.empty((B, w.Nv, S, w.Dv), dtype=torch.bfloat16, device="cuda")
+    ns = torch.empty_like(st)
+    step = gdr.prepare_conv1d(x, wt, bias, st, None, Nk=w.Nk, Nv=w.Nv, Dk=w.Dk, Dv=w.Dv, q=q, k=k, v=v,
+                              conv_state_out=ns)
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if gdr.get_error() != 0:
+        raise RuntimeError("device error word set during warm-up")
+    barrier(world)
+    torch.cuda.synchronize()
+    times = timed_steps(step, args.steps, flush, stream)
+    barrier(world)
+    total_ms = all_max(sum(times), world)
+    ms = total_ms / args.steps
+    alg = 2 * B * S * C * 2 + C * 4 * 2 + C * 2 + 2 * B * C * 4 * 2  # x in, q/k/v out, taps, bias, state in/out
+    achieved = alg / (ms / 1e3) / 1e9
+    # one conv launch per step; with S > 64 the state is written by a second, small launch
+    return {"workload": f"conv1d B={B} S={S} C={C} (Nk={w.Nk} Nv={w.Nv} D={w.Dk}) K=4 bf16, bias and state",
+            "ms_per_step": ms, "tokens_per_s": weak_scaling_rate(B * S, args.steps, total_ms, world),
+            "l2": "inputs larger than L2, plus a 256 MiB flush before every timed step",
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": achieved / peaks["hbm_gbs"], "traffic": profiled_traffic("conv1d"),
+                         "algorithmic_bytes_per_launch": alg, "kernel": "gdr_conv1d"}}, 2 * args.steps
+
+
 def bench_e2e(gdr, args, world, w, t, pro, flush, stream):
     """Same metric through the public call with host buffers: pinned H2D copies of the
     step's inputs, the call, D2H of out and the final state, all inside the timed region."""
@@ -446,6 +480,9 @@ def run_ours(args, world, rank, local):
             line["prefill_epilogue"], n = bench_prefill_epilogue(gdr, args, world, w, t, pro, flush, stream, peaks)
             launches += n
         del t
+    if args.only in ("all", "conv1d"):
+        line["conv1d"], n = bench_conv1d(gdr, args, world, rank, flush, stream, peaks)
+        launches += n
     decode = {}
     for name in ("decode", "decode_gk"):
         if args.only in ("all", name):
@@ -476,7 +513,7 @@ def main():
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg (profiling runs)")
     ap.add_argument("--no-epilogue", action="store_true",
                     help="skip the prefill line with the fused gated RMSNorm epilogue (profiling runs)")
-    ap.add_argument("--only", choices=["all", "prefill", "decode", "decode_gk"], default="all",
+    ap.add_argument("--only", choices=["all", "prefill", "decode", "decode_gk", "conv1d"], default="all",
                     help="run one workload only (profiling runs); the default runs all")
     args = ap.parse_args()
     if args.warmup < 3:

@@ -31,8 +31,8 @@ GDR_F32, GDR_BF16 = 0, 1
 DEVERR_SLOT_INDEX, DEVERR_LENGTH = 0x1, 0x2
 
 # Every symbol the C header declares (checked by the ABI test).
-EXPORTED = ("gdr_chunk_fwd", "gdr_recurrent_step", "gdr_prologue_apply", "gdr_get_error", "gdr_status_string",
-            "gdr_version")
+EXPORTED = ("gdr_chunk_fwd", "gdr_recurrent_step", "gdr_conv1d", "gdr_prologue_apply", "gdr_get_error",
+            "gdr_status_string", "gdr_version")
 
 
 class GdrPrologueStruct(ctypes.Structure):
@@ -66,6 +66,8 @@ def lib() -> ctypes.CDLL:
         L.gdr_recurrent_step.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, vp, vp, vp, f32, i32, i32, i32, i32, i32,
                                          i32, i32, i32, ctypes.POINTER(GdrPrologueStruct),
                                          ctypes.POINTER(GdrEpilogueStruct), vp, vp]
+        L.gdr_conv1d.restype = i32
+        L.gdr_conv1d.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, i32, vp, vp, vp, vp, vp]
         L.gdr_prologue_apply.restype = i32
         L.gdr_prologue_apply.argtypes = [vp, vp, vp, vp, vp, vp, f32, i32, i32, i32, i32, i32, i32, vp, vp, vp, vp,
                                          vp]
@@ -306,6 +308,55 @@ def prepare_recurrent_step(q, k, v, beta, g, gk, state_pool, ssm_state_indices, 
     call = PreparedCall(lib().gdr_recurrent_step, args, "gdr_recurrent_step", (out, state_pool))
     call._keep = (pro, prologue, epi, epilogue)
     return call
+
+
+def _conv1d_checked(x, weight, bias, conv_state, actual_seq_lengths, Nk, Nv, Dk, Dv, q, k, v, conv_state_out,
+                    output_state, stream):
+    if x.dim() != 3 or weight.dim() != 2:
+        raise ValueError("x must be (B, S, C) and weight (C, K)")
+    B, S, C = x.shape
+    K = weight.shape[1]
+    if C != 2 * Nk * Dk + Nv * Dv:
+        raise ValueError(f"x has {C} channels; 2 * Nk * Dk + Nv * Dv = {2 * Nk * Dk + Nv * Dv}")
+    dt = x.dtype
+    code = _dtype_code(dt)
+    _dev(x, "x", dt)
+    _dev(weight, "weight", dt, (C, K))
+    _dev(bias, "bias", dt, (C,))
+    _dev(conv_state, "conv_state", dt, (B, C, K))
+    _dev(actual_seq_lengths, "actual_seq_lengths", torch.int32, (B,))
+    outs = []
+    for name, t, shape in (("q", q, (B, Nk, S, Dk)), ("k", k, (B, Nk, S, Dk)), ("v", v, (B, Nv, S, Dv))):
+        t = torch.empty(shape, dtype=dt, device=x.device) if t is None else t
+        outs.append(_dev(t, name, dt, shape))
+    if output_state and conv_state_out is None:
+        conv_state_out = torch.empty((B, C, K), dtype=dt, device=x.device)
+    _dev(conv_state_out, "conv_state_out", dt, (B, C, K))
+    args = (_ptr(x), _ptr(weight), _ptr(bias), _ptr(conv_state), _ptr(actual_seq_lengths), B, S, Nk, Nv, Dk, Dv, K,
+            code, _ptr(outs[0]), _ptr(outs[1]), _ptr(outs[2]), _ptr(conv_state_out), _stream(stream))
+    return args, (outs[0], outs[1], outs[2], conv_state_out)
+
+
+def conv1d(x, weight, bias=None, conv_state=None, actual_seq_lengths=None, *, Nk: int, Nv: int, Dk: int, Dv: int,
+           q=None, k=None, v=None, conv_state_out=None, output_state: bool = True, stream=None):
+    """Depthwise causal conv1d + SiLU over the fused q/k/v channels (``gdr_conv1d``).
+
+    x (B, S, C) channels last with C = 2 * Nk * Dk + Nv * Dv, weight (C, K) taps oldest first, bias (C,) or
+    None, conv_state (B, C, K) or None (zeros).  Returns (q (B, Nk, S, Dk), k, v (B, Nv, S, Dv), new state
+    (B, C, K) or None).  Pass ``conv_state_out=conv_state`` to update the state in place (decode)."""
+    args, res = _conv1d_checked(x, weight, bias, conv_state, actual_seq_lengths, Nk, Nv, Dk, Dv, q, k, v,
+                                conv_state_out, output_state, stream)
+    _check(lib().gdr_conv1d(*args), "gdr_conv1d")
+    return res
+
+
+def prepare_conv1d(x, weight, bias=None, conv_state=None, actual_seq_lengths=None, *, Nk: int, Nv: int, Dk: int,
+                   Dv: int, q=None, k=None, v=None, conv_state_out=None, output_state: bool = True,
+                   stream=None) -> "PreparedCall":
+    """Check and marshal a gdr_conv1d call once; see conv1d for the arguments."""
+    args, res = _conv1d_checked(x, weight, bias, conv_state, actual_seq_lengths, Nk, Nv, Dk, Dv, q, k, v,
+                                conv_state_out, output_state, stream)
+    return PreparedCall(lib().gdr_conv1d, args, "gdr_conv1d", res)
 
 
 def prologue(q=None, k=None, b=None, a=None, A_log=None, dt_bias=None, eps: float = 1e-6, *, stream=None):

@@ -178,6 +178,27 @@ extern "C" int gdr_recurrent_step(const void *q, const void *k, const void *v, c
     return e == cudaSuccess ? GDR_OK : GDR_ERR_LAUNCH;
 }
 
+extern "C" int gdr_conv1d(const void *x, const void *weight, const void *bias, const void *conv_state_in,
+                          const int32_t *actual_seq_lengths, int B, int S, int Nk, int Nv, int Dk, int Dv, int K,
+                          gdr_dtype dtype, void *q, void *k, void *v, void *conv_state_out, gdr_stream_t stream) {
+    int st = check_common(B, Nk, Nv, S, Dk, Dv, dtype);
+    if (st) return st;
+    if (K < 1 || K > 8) return GDR_ERR_SHAPE;
+    // grid: (channel groups, 64-step time tiles, B)
+    if (B > 65535 || (long long)S > 65535LL * 64) return GDR_ERR_SHAPE;
+    if ((long long)B * S > 0 && (!x || !weight || !q || !k || !v)) return GDR_ERR_NULL;
+    if (B > 0 && conv_state_out && !weight) return GDR_ERR_NULL;
+    const void *ptrs[] = {x, weight, bias, conv_state_in, actual_seq_lengths, q, k, v, conv_state_out};
+    for (const void *p : ptrs)
+        if (!aligned16(p)) return GDR_ERR_ALIGN;
+    if (B == 0 || (S == 0 && !conv_state_out)) return GDR_OK;
+    unsigned int *err = nullptr;
+    if ((st = device_setup(&err))) return st;
+    cudaError_t e = launch_conv1d(x, weight, bias, conv_state_in, actual_seq_lengths, B, S, Nk, Nv, Dk, Dv, K, dtype,
+                                  q, k, v, conv_state_out, err, reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? GDR_OK : GDR_ERR_LAUNCH;
+}
+
 extern "C" int gdr_prologue_apply(const void *q, const void *k, const void *b, const float *a, const float *A_log,
                                   const float *dt_bias, float eps, int B, int Nk, int Nv, int S, int Dk,
                                   gdr_dtype dtype, void *q_hat, void *k_hat, void *beta, float *g,

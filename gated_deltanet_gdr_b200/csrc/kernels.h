@@ -60,6 +60,10 @@ cudaError_t launch_chunk_simt(const ChunkArgs &a, int Dk, int Dv, gdr_dtype dt, 
 // out rows t < L_b <- rmsnorm(out row) * norm_w * silu(z row), in place (the unfused epilogue)
 cudaError_t launch_gated_rmsnorm(void *out, const void *z, const float *norm_w, float eps, const int32_t *lengths,
                                  int B, int Nv, int S, int Dv, gdr_dtype dt, cudaStream_t s);
+// depthwise causal conv1d + SiLU over the fused q/k/v channels into q, k, v, and its state (gdr_conv1d)
+cudaError_t launch_conv1d(const void *x, const void *weight, const void *bias, const void *state_in,
+                          const int32_t *lengths, int B, int S, int Nk, int Nv, int Dk, int Dv, int K, gdr_dtype dt,
+                          void *q, void *k, void *v, void *state_out, unsigned int *err, cudaStream_t s);
 cudaError_t launch_prologue(const void *q, const void *k, const void *b, const float *a, const float *A_log,
                             const float *dt_bias, float eps, int B, int Nk, int Nv, int S, int Dk, gdr_dtype dt,
                             void *q_hat, void *k_hat, void *beta, float *g, cudaStream_t stream);

@@ -190,6 +190,41 @@ int gdr_recurrent_step(const void *q, const void *k, const void *v, const void *
                        gdr_stream_t stream);
 
 /*
+ * Depthwise causal conv1d + SiLU over the fused q/k/v channels, with its state:
+ * the step before the rule, writing the rule's q, k and v.  Source: the layer's
+ * conv over mixed_qkv = cat(q, k, v) with causal_conv1d_fn (prefill) and
+ * causal_conv1d_update (decode), conv_state = F.pad(mixed_qkv, (K - L, 0))
+ * (blog "gated-delta-net" page), and the per-channel ring of the last K inputs
+ * in deltanet.rs and its WGSL twin (shift, append, dot with the taps oldest
+ * first, silu).
+ *
+ * For sequence b (L = L_b valid positions) and channel c:
+ *     y[t, c] = silu(bias[c] + sum_{j<K} weight[c, j] * x[t - K + 1 + j, c]),  t < L
+ * where the K positions before 0 come from conv_state_in (newest last; zeros
+ * when it is NULL).  Computed in fp32, rounded once to dtype.
+ *
+ *   x                    device (B, S, C) channels last, C = 2*Nk*Dk + Nv*Dv: the
+ *                        q channels (Nk heads of Dk), then k (Nk x Dk), then v (Nv x Dv)
+ *   weight               device (C, K), taps oldest first
+ *   bias                 device (C) or NULL: no bias
+ *   conv_state_in        device (B, C, K) or NULL: zeros
+ *   actual_seq_lengths   device int32 (B) or NULL: all S; positions t >= L_b are padding
+ *   q, k, v              device outputs (B, Nk, S, Dk), (B, Nk, S, Dk), (B, Nv, S, Dv):
+ *                        y split by channel and head; padding rows are zero
+ *   conv_state_out       device (B, C, K) or NULL: the last K inputs of the history
+ *                        (conv_state_in followed by x[0..L_b-1]); it may alias
+ *                        conv_state_in (the in-place update of decode)
+ * x, weight, bias, the states and the outputs are in dtype (GDR_F32 or
+ * GDR_BF16).  Constraints: B, S >= 0; Nk, Nv >= 1; Dk, Dv in {16,32,64,128};
+ * 1 <= K <= 8 (4 in the layer); every pointer 16-byte aligned.  A length
+ * outside [0, S] skips the sequence (outputs zero, state untouched) and sets
+ * GDR_DEVERR_LENGTH.
+ */
+int gdr_conv1d(const void *x, const void *weight, const void *bias, const void *conv_state_in,
+               const int32_t *actual_seq_lengths, int B, int S, int Nk, int Nv, int Dk, int Dv, int K,
+               gdr_dtype dtype, void *q, void *k, void *v, void *conv_state_out, gdr_stream_t stream);
+
+/*
  * Stand-alone prologue (the same arithmetic the fused prologue applies), for
  * callers that want the normalised tensors materialised.  Source: as for
  * gdr_prologue.

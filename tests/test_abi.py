@@ -114,6 +114,29 @@ def test_decode_host_validation(L):
     assert decode(L, B=0) == gdr.GDR_OK
 
 
+def conv(L, **kw):
+    a = dict(x=P, w=P, bias=NUL, s0=NUL, lens=NUL, B=1, S=8, Nk=2, Nv=4, Dk=128, Dv=128, K=4, dt=gdr.GDR_BF16,
+             q=P, k=P, v=P, s1=NUL)
+    a.update(kw)
+    return L.gdr_conv1d(a["x"], a["w"], a["bias"], a["s0"], a["lens"], a["B"], a["S"], a["Nk"], a["Nv"], a["Dk"],
+                        a["Dv"], a["K"], a["dt"], a["q"], a["k"], a["v"], a["s1"], None)
+
+
+def test_conv1d_host_validation(L):
+    assert conv(L, K=0) == gdr.GDR_ERR_SHAPE
+    assert conv(L, K=9) == gdr.GDR_ERR_SHAPE
+    assert conv(L, Nv=3) == gdr.GDR_ERR_SHAPE
+    assert conv(L, B=70000) == gdr.GDR_ERR_SHAPE  # grid z limit
+    assert conv(L, dt=4) == gdr.GDR_ERR_DTYPE
+    assert conv(L, Dv=48) == gdr.GDR_ERR_UNSUPPORTED
+    assert conv(L, x=NUL) == gdr.GDR_ERR_NULL
+    assert conv(L, v=NUL) == gdr.GDR_ERR_NULL
+    assert conv(L, S=0, w=NUL, s1=P) == gdr.GDR_ERR_NULL  # a state update needs the taps' shape
+    assert conv(L, bias=ctypes.c_void_p(4098)) == gdr.GDR_ERR_ALIGN
+    assert conv(L, B=0) == gdr.GDR_OK
+    assert conv(L, S=0, x=NUL, q=NUL, k=NUL, v=NUL) == gdr.GDR_OK  # nothing to compute, no state asked for
+
+
 def test_prologue_host_validation(L):
     f = L.gdr_prologue_apply
     assert f(P, NUL, NUL, NUL, NUL, NUL, 1e-6, 1, 1, 1, 4, 16, 5, P, NUL, NUL, NUL, None) == gdr.GDR_ERR_DTYPE

@@ -188,3 +188,18 @@ def epilogue_inputs(w: Workload):
     z = _normal(rng, (w.B, w.Nv, w.S, w.Dv), dtype=w.meta.get("fd", np.float32))
     norm_w = rng.uniform(0.5, 1.5, size=w.Dv).astype(np.float32)
     return z, norm_w
+
+
+def conv_inputs(w: Workload, K: int = 4, with_state: bool = True, with_bias: bool = True):
+    """Inputs of the depthwise causal conv1d before the rule, for a workload's head layout: the fused
+    projection x ~ N(0, 1) of shape (B, S, C), C = 2 Nk Dk + Nv Dv (channels last), taps ~ U(-0.5, 0.5) of
+    shape (C, K), bias ~ N(0, 0.1^2) of shape (C,) and a state ~ N(0, 1) of shape (B, C, K).  Drawn from a
+    stream of their own (the workload's seed and 2)."""
+    rng = np.random.default_rng([int(w.meta["seed"]), 2])
+    C = 2 * w.Nk * w.Dk + w.Nv * w.Dv
+    fd = w.meta.get("fd", np.float32)
+    x = _normal(rng, (w.B, w.S, C), dtype=fd)
+    weight = rng.uniform(-0.5, 0.5, size=(C, K)).astype(fd)
+    bias = _normal(rng, (C,), std=0.1, dtype=fd) if with_bias else None
+    state = _normal(rng, (w.B, C, K), dtype=fd) if with_state else None
+    return x, weight, bias, state
