@@ -60,8 +60,8 @@ def lib() -> ctypes.CDLL:
             L.gdr_oracle_chunk_fwd.argtypes = [dp, dp, dp, dp, dp, dp, ip, c_double, c_int, c_int, c_int, c_int,
                                                c_int, c_int, dp, dp]
             L.gdr_oracle_recurrent_step.restype = c_int
-            L.gdr_oracle_recurrent_step.argtypes = [dp, dp, dp, dp, dp, dp, dp, c_int, ip, ip, ip, c_double, c_int,
-                                                    c_int, c_int, c_int, c_int, c_int, dp]
+            L.gdr_oracle_recurrent_step.argtypes = [dp, dp, dp, dp, dp, dp, dp, c_int, ip, ip, ip, c_int, c_double,
+                                                    c_int, c_int, c_int, c_int, c_int, c_int, dp]
             L.gdr_oracle_threads.restype = c_int
             L.gdr_oracle_threads.argtypes = []
             _lib = L
@@ -160,12 +160,14 @@ def chunk_fwd(q, k, v, beta, g=None, initial_state=None, actual_seq_lengths=None
 
 
 def recurrent_step(q, k, v, beta, g, gk, state_pool, ssm_state_indices, actual_seq_lengths,
-                   num_accepted_tokens=None, scale: float = 1.0):
+                   num_accepted_tokens=None, scale: float = 1.0, per_token: bool = False):
     """fp64 semantics of the decode call over a slot pool.
 
     Returns (out (B,Nv,S,Dv), new_pool (slots,Nv,Dk,Dv)); the input pool is
-    not modified (a copy is updated).  See gdr_oracle.c for the reading of
-    num_accepted_tokens.
+    not modified (a copy is updated).  See gdr_oracle.c for the two readings of
+    num_accepted_tokens (per_token False: commit the first A states; True: the
+    speculative-decoding reading, start from the slot of token A - 1 and commit
+    every token's state to its own slot).
     """
     qa, ka, va, ba = _f64(q), _f64(k), _f64(v), _f64(beta)
     B, Nk, S, Dk = qa.shape
@@ -177,7 +179,8 @@ def recurrent_step(q, k, v, beta, g, gk, state_pool, ssm_state_indices, actual_s
     A = _i32(num_accepted_tokens)
     out = np.empty((B, Nv, S, Dv), np.float64)
     rc = lib().gdr_oracle_recurrent_step(_dp(qa), _dp(ka), _dp(va), _dp(ba), _dp(ga), _dp(gka), _dp(pool), slots,
-                                         _ip(idx), _ip(L), _ip(A), float(scale), B, Nk, Nv, S, Dk, Dv, _dp(out))
+                                         _ip(idx), _ip(L), _ip(A), int(bool(per_token)), float(scale), B, Nk, Nv,
+                                         S, Dk, Dv, _dp(out))
     if rc != 0:
         raise ValueError(f"oracle recurrent_step rejected the arguments (code {rc})")
     return out, pool

@@ -215,10 +215,15 @@ int gdr_oracle_chunk_fwd(const double *q, const double *k, const double *v,
  *   out         (B, Nv, S, Dv); rows t >= L_b are zero
  *
  * Reading of num_accepted_tokens (the page defines it only as the number of
- * accepted tokens, equal to the lengths in plain inference): the chain starts
- * from pool[indices[b*S]]; all L_b tokens are processed and output; the state
- * after token t is written to pool[indices[b*S + t]] only when
- * t < min(A_b, L_b).  A sequence with L_b = 0 leaves the pool untouched.
+ * accepted tokens, equal to the lengths in plain inference), per_token = 0:
+ * the chain starts from pool[indices[b*S]]; all L_b tokens are processed and
+ * output; the state after token t is written to pool[indices[b*S + t]] only
+ * when t < min(A_b, L_b).  per_token = 1 (the speculative-decoding reading):
+ * A_b counts the tokens of the previous step that were accepted, whose states
+ * went to their own slots, so the chain starts from pool[indices[b*S + A_b - 1]]
+ * and the state after every token t < L_b is written to pool[indices[b*S + t]];
+ * A_b must lie in [1, S] (ORACLE_BAD_SHAPE otherwise; NULL accepted means 1).
+ * A sequence with L_b = 0 leaves the pool untouched.
  * Returns ORACLE_BAD_INDEX for a referenced slot outside [0, slots), and
  * ORACLE_BAD_SHAPE for bad sizes or lengths outside [0, S].  Two sequences
  * must not share a slot (their chains would race; the result is undefined).
@@ -227,14 +232,20 @@ int gdr_oracle_recurrent_step(const double *q, const double *k, const double *v,
                               const double *beta, const double *g,
                               const double *gk, double *pool, int slots,
                               const int32_t *indices, const int32_t *lengths,
-                              const int32_t *accepted, double scale, int B,
-                              int Nk, int Nv, int S, int Dk, int Dv,
+                              const int32_t *accepted, int per_token, double scale,
+                              int B, int Nk, int Nv, int S, int Dk, int Dv,
                               double *out) {
     if (B < 0 || Nk <= 0 || Nv <= 0 || S < 0 || Dk <= 0 || Dv <= 0 || slots < 0)
         return ORACLE_BAD_SHAPE;
     if (Nv % Nk != 0) return ORACLE_BAD_SHAPE;
     for (int b = 0; b < B; ++b) {
         if (lengths[b] < 0 || lengths[b] > S) return ORACLE_BAD_SHAPE;
+        if (per_token && lengths[b] > 0) {
+            int A = accepted ? accepted[b] : 1;
+            if (A < 1 || A > S) return ORACLE_BAD_SHAPE;
+            int s = indices[(size_t)b * S + A - 1];
+            if (s < 0 || s >= slots) return ORACLE_BAD_INDEX;
+        }
         for (int t = 0; t < lengths[b]; ++t) {
             int s = indices[(size_t)b * S + t];
             if (s < 0 || s >= slots) return ORACLE_BAD_INDEX;
@@ -246,8 +257,10 @@ int gdr_oracle_recurrent_step(const double *q, const double *k, const double *v,
     for (int bh = 0; bh < B * Nv; ++bh) {
         int b = bh / Nv, h = bh % Nv, kh = h / group;
         int L = lengths[b];
-        int A = accepted ? accepted[b] : L;
-        if (A > L) A = L;
+        int A = accepted ? accepted[b] : (per_token ? 1 : L);
+        /* commits: tokens t < ncommit; the chain starts from the slot of token `first` */
+        int ncommit = per_token ? L : (A < L ? A : L);
+        int first = per_token ? A - 1 : 0;
         size_t sd = (size_t)Dk * Dv;
         for (int t = L; t < S; ++t) {
             double *o = out + ((size_t)bh * S + t) * Dv;
@@ -263,7 +276,7 @@ int gdr_oracle_recurrent_step(const double *q, const double *k, const double *v,
             status = ORACLE_NO_MEMORY;
             continue;
         }
-        int s0 = indices[(size_t)b * S];
+        int s0 = indices[(size_t)b * S + first];
         memcpy(St, pool + ((size_t)s0 * Nv + h) * sd, sd * sizeof(double));
         for (int t = 0; t < L; ++t) {
             const double *qr = q + (((size_t)b * Nk + kh) * S + t) * Dk;
@@ -274,7 +287,7 @@ int gdr_oracle_recurrent_step(const double *q, const double *k, const double *v,
             double *o = out + gi * Dv;
             for (int i = 0; i < Dk; ++i) x[i] = scale * qr[i];
             token_step(St, x, kr, vr, beta[gi], g ? g[gi] : 0.0, gkr, Dk, Dv, m, o);
-            if (t < A) {
+            if (t < ncommit) {
                 int st = indices[(size_t)b * S + t];
                 memcpy(pool + ((size_t)st * Nv + h) * sd, St, sd * sizeof(double));
             }

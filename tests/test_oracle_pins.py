@@ -230,3 +230,64 @@ def conv_impl(x, w, bias, state, lengths):
 @pytest.mark.parametrize("check", _pins.CONV_CHECKS, ids=lambda c: c.__name__)
 def test_causal_conv1d_oracle_pin(check):
     check(conv_impl)
+
+
+# ---- the speculative-decoding reading of num_accepted_tokens (per-token state slots) ----
+
+def _spec_case(seed, B=3, S=4, Nk=2, Nv=4, D=8):
+    rng = np.random.default_rng(seed)
+    q = rng.standard_normal((B, Nk, S, D))
+    k = rng.standard_normal((B, Nk, S, D))
+    k /= np.linalg.norm(k, axis=-1, keepdims=True)
+    v = rng.standard_normal((B, Nv, S, D))
+    beta = rng.uniform(0.1, 0.9, (B, Nv, S))
+    g = np.log(rng.uniform(0.8, 0.99, (B, Nv, S)))
+    return q, k, v, beta, g
+
+
+def test_spec_reading_with_one_accepted_equals_committing_every_token():
+    """A = 1 starts from the slot of token 0, as the other reading does; with every token committed both
+    write the same states to the same per-token slots."""
+    q, k, v, beta, g = _spec_case(31)
+    B, S = q.shape[0], q.shape[2]
+    rng = np.random.default_rng(32)
+    pool = rng.standard_normal((B * S + 2, 4, 8, 8))
+    idx = rng.permutation(B * S + 2)[:B * S].astype(np.int32)
+    L = np.array([4, 2, 3], np.int32)
+    o1, p1 = oracle.recurrent_step(q, k, v, beta, g, None, pool, idx, L, np.ones(B, np.int32), 0.5, per_token=True)
+    o2, p2 = oracle.recurrent_step(q, k, v, beta, g, None, pool, idx, L, L, 0.5)
+    assert np.array_equal(o1, o2) and np.array_equal(p1, p2)
+
+
+def test_spec_two_steps_equal_the_chain_over_accepted_tokens():
+    """Step 1 verifies 4 draft tokens from slot s0 and writes each token's state to its own slot; 2 are
+    accepted.  Step 2 starts from the state after the second token (slot of token A - 1) and processes 4
+    new tokens: its outputs and states equal the prefill oracle's chain over x1, x2, y1..y4."""
+    q1, k1, v1, b1, g1 = _spec_case(33, B=1)
+    q2, k2, v2, b2, g2 = _spec_case(34, B=1)
+    S = 4
+    rng = np.random.default_rng(35)
+    pool = rng.standard_normal((6, 4, 8, 8))
+    slots = np.array([5, 1, 3, 0], np.int32)
+    _, p1 = oracle.recurrent_step(q1, k1, v1, b1, g1, None, pool, slots, np.array([S], np.int32),
+                                  np.array([1], np.int32), 0.5, per_token=True)
+    A = 2
+    o2, p2 = oracle.recurrent_step(q2, k2, v2, b2, g2, None, p1, slots, np.array([S], np.int32),
+                                   np.array([A], np.int32), 0.5, per_token=True)
+    cat = lambda a1, a2: np.concatenate([a1[:, :, :A], a2], axis=2)
+    s0 = pool[slots[0]][None]  # the chain's state before x1
+    oc, fc = oracle.chunk_fwd(cat(q1, q2), cat(k1, k2), cat(v1, v2), cat(b1, b2), cat(g1, g2), s0, None, 0.5)
+    assert np.allclose(o2, oc[:, :, A:], rtol=1e-12, atol=1e-12)
+    assert np.allclose(p2[slots[S - 1]], fc[0], rtol=1e-12, atol=1e-12)
+    untouched = [s for s in range(6) if s not in slots]
+    assert np.array_equal(p2[untouched], pool[untouched])
+
+
+def test_spec_reading_rejects_accepted_outside_range():
+    q, k, v, beta, g = _spec_case(36, B=1)
+    pool = np.zeros((4, 4, 8, 8))
+    idx = np.arange(4, dtype=np.int32)
+    for A in (0, 5):
+        with pytest.raises(ValueError):
+            oracle.recurrent_step(q, k, v, beta, g, None, pool, idx, np.array([4], np.int32),
+                                  np.array([A], np.int32), 0.5, per_token=True)
