@@ -416,7 +416,15 @@ def bench_decode(gdr, name, args, world, rank, clk, flush, stream, peaks, rotate
     fits in L2, so instead of a flush the steps rotate over `rotate` separate copies of the
     pool: each call reads fresh state and pays the write-back of the previous call's state,
     as a serving loop does."""
-    wd = workloads.generate(name, seed=(1 if name == "decode" else 4) + 1000 * rank)
+    spec = name == "decode_spec"
+    if spec:
+        # speculative decoding: 64 sequences verify 4 draft tokens each, every token with its own slot (the
+        # previous step's A of them accepted); gdr_recurrent_step_spec
+        wd = workloads.random_case(B=64, Nk=16, Nv=32, S=4, Dk=128, Dv=128, seed=6 + 1000 * rank, slots=64 * 4 + 64,
+                                   share_slot=False, fd=np.float32)
+        wd.accepted = np.random.default_rng([6 + 1000 * rank, 3]).integers(1, 5, size=64).astype(np.int32)
+    else:
+        wd = workloads.generate(name, seed=(1 if name == "decode" else 4) + 1000 * rank)
     dq, dk, dv, db = bf16_dev(wd.q), bf16_dev(wd.k), bf16_dev(wd.v), bf16_dev(wd.b)
     dg = f32_dev(wd.g)
     dgk = f32_dev(wd.gk) if wd.gk is not None else None
@@ -427,7 +435,7 @@ def bench_decode(gdr, name, args, world, rank, clk, flush, stream, peaks, rotate
     dout = torch.empty((wd.B, wd.Nv, wd.S, wd.Dv), dtype=torch.bfloat16, device="cuda")
     dpro = gdr.Prologue(l2norm_qk=True, eps=1e-6, beta_logits=True)
     calls = [gdr.prepare_recurrent_step(dq, dk, dv, db, dg, dgk, pool, idx, lens, acc, wd.scale, prologue=dpro,
-                                        out=dout) for pool in pools]
+                                        out=dout, per_token=spec) for pool in pools]
     for i in range(args.warmup):
         calls[i % rotate]()
     barrier(world)
@@ -447,10 +455,13 @@ def bench_decode(gdr, name, args, world, rank, clk, flush, stream, peaks, rotate
     times = [s.elapsed_time(e) for s, e in evs]
     d_ms = all_max(sum(times), world) / args.steps
     nb = algorithmic_decode_bytes(wd)
+    if spec:  # one state read per sequence and head, one state written per processed token
+        nb["state"] = int((1 + wd.lengths).sum()) * wd.Nv * wd.Dk * wd.Dv * 2
     gbs = nb["state"] / (d_ms / 1e3) / 1e9
     tot = (nb["state"] + nb["io"]) / (d_ms / 1e3) / 1e9
     return {"workload": f"B={wd.B} S={wd.S} Nk={wd.Nk} Nv={wd.Nv} D={wd.Dk} bf16, pool of {wd.pool.shape[0]} slots"
-                        + (", per-key gate" if wd.gk is not None else "") + ", fused prologue",
+                        + (", per-key gate" if wd.gk is not None else "") + ", fused prologue"
+                        + (", per-token slots, accepted ~ U[1, 4] (speculative decoding)" if spec else ""),
             "l2": f"{rotate} rotating pool copies (fresh state every call), no flush",
             "us_per_call": d_ms * 1e3, "steps_per_s": world * 1e3 / d_ms,
             "state_GBps": gbs, "state_frac_of_hbm": gbs / peaks["hbm_gbs"],
@@ -484,7 +495,7 @@ def run_ours(args, world, rank, local):
         line["conv1d"], n = bench_conv1d(gdr, args, world, rank, flush, stream, peaks)
         launches += n
     decode = {}
-    for name in ("decode", "decode_gk"):
+    for name in ("decode", "decode_gk", "decode_spec"):
         if args.only in ("all", name):
             decode[name], n = bench_decode(gdr, name, args, world, rank, clk, flush, stream, peaks)
             launches += n
@@ -513,7 +524,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg (profiling runs)")
     ap.add_argument("--no-epilogue", action="store_true",
                     help="skip the prefill line with the fused gated RMSNorm epilogue (profiling runs)")
-    ap.add_argument("--only", choices=["all", "prefill", "decode", "decode_gk", "conv1d"], default="all",
+    ap.add_argument("--only", choices=["all", "prefill", "decode", "decode_gk", "decode_spec", "conv1d"],
+                    default="all",
                     help="run one workload only (profiling runs); the default runs all")
     args = ap.parse_args()
     if args.warmup < 3:

@@ -31,8 +31,8 @@ GDR_F32, GDR_BF16 = 0, 1
 DEVERR_SLOT_INDEX, DEVERR_LENGTH = 0x1, 0x2
 
 # Every symbol the C header declares (checked by the ABI test).
-EXPORTED = ("gdr_chunk_fwd", "gdr_recurrent_step", "gdr_conv1d", "gdr_prologue_apply", "gdr_get_error",
-            "gdr_status_string", "gdr_version")
+EXPORTED = ("gdr_chunk_fwd", "gdr_recurrent_step", "gdr_recurrent_step_spec", "gdr_conv1d", "gdr_prologue_apply",
+            "gdr_get_error", "gdr_status_string", "gdr_version")
 
 
 class GdrPrologueStruct(ctypes.Structure):
@@ -66,6 +66,8 @@ def lib() -> ctypes.CDLL:
         L.gdr_recurrent_step.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, vp, vp, vp, f32, i32, i32, i32, i32, i32,
                                          i32, i32, i32, ctypes.POINTER(GdrPrologueStruct),
                                          ctypes.POINTER(GdrEpilogueStruct), vp, vp]
+        L.gdr_recurrent_step_spec.restype = i32
+        L.gdr_recurrent_step_spec.argtypes = L.gdr_recurrent_step.argtypes
         L.gdr_conv1d.restype = i32
         L.gdr_conv1d.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, i32, vp, vp, vp, vp, vp]
         L.gdr_prologue_apply.restype = i32
@@ -233,22 +235,25 @@ def _decode_checked(q, k, v, beta, g, gk, state_pool, ssm_state_indices, actual_
 
 def recurrent_step(q, k, v, beta, g, gk, state_pool, ssm_state_indices, actual_seq_lengths,
                    num_accepted_tokens=None, scale: float = 1.0, *, prologue: Optional[Prologue] = None,
-                   epilogue: Optional[Epilogue] = None, out=None, stream=None):
+                   epilogue: Optional[Epilogue] = None, out=None, per_token: bool = False, stream=None):
     """Recurrent decode over a slot pool (``gdr_recurrent_step``), updating
-    ``state_pool`` in place.  Returns (out, state_pool)."""
+    ``state_pool`` in place.  Returns (out, state_pool).  ``per_token=True`` calls
+    ``gdr_recurrent_step_spec`` (speculative decoding: start from the slot of token
+    A - 1, every token's state to its own slot)."""
     out = _decode_checked(q, k, v, beta, g, gk, state_pool, ssm_state_indices, actual_seq_lengths,
                           num_accepted_tokens, out)
     B, Nk, S, Dk = q.shape
     Nv, Dv = v.shape[1], v.shape[3]
     pro = prologue.as_struct() if prologue is not None else None
     epi = _check_epilogue(epilogue, B, Nv, S, Dv, q.dtype)
-    st = lib().gdr_recurrent_step(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(g), _ptr(gk), _ptr(state_pool),
+    fn = lib().gdr_recurrent_step_spec if per_token else lib().gdr_recurrent_step
+    st = fn(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(g), _ptr(gk), _ptr(state_pool),
                                   int(state_pool.shape[0]), _ptr(ssm_state_indices), _ptr(actual_seq_lengths),
                                   _ptr(num_accepted_tokens), float(scale), B, Nk, Nv, S, Dk, Dv,
                                   _dtype_code(q.dtype), _dtype_code(state_pool.dtype),
                                   ctypes.byref(pro) if pro is not None else None,
                                   ctypes.byref(epi) if epi is not None else None, _ptr(out), _stream(stream))
-    _check(st, "gdr_recurrent_step")
+    _check(st, "gdr_recurrent_step_spec" if per_token else "gdr_recurrent_step")
     return out, state_pool
 
 
@@ -292,7 +297,8 @@ def prepare_chunk_fwd(q, k, v, beta, g=None, initial_state=None, actual_seq_leng
 
 def prepare_recurrent_step(q, k, v, beta, g, gk, state_pool, ssm_state_indices, actual_seq_lengths,
                            num_accepted_tokens=None, scale: float = 1.0, *, prologue: Optional[Prologue] = None,
-                           epilogue: Optional[Epilogue] = None, out=None, stream=None) -> PreparedCall:
+                           epilogue: Optional[Epilogue] = None, out=None, per_token: bool = False,
+                           stream=None) -> PreparedCall:
     """Check and marshal a gdr_recurrent_step call once; see recurrent_step for the arguments."""
     out = _decode_checked(q, k, v, beta, g, gk, state_pool, ssm_state_indices, actual_seq_lengths,
                           num_accepted_tokens, out)
@@ -305,7 +311,8 @@ def prepare_recurrent_step(q, k, v, beta, g, gk, state_pool, ssm_state_indices, 
             Nk, Nv, S, Dk, Dv, _dtype_code(q.dtype), _dtype_code(state_pool.dtype),
             ctypes.pointer(pro) if pro is not None else None, ctypes.pointer(epi) if epi is not None else None,
             _ptr(out), _stream(stream))
-    call = PreparedCall(lib().gdr_recurrent_step, args, "gdr_recurrent_step", (out, state_pool))
+    name = "gdr_recurrent_step_spec" if per_token else "gdr_recurrent_step"
+    call = PreparedCall(getattr(lib(), name), args, name, (out, state_pool))
     call._keep = (pro, prologue, epi, epilogue)
     return call
 

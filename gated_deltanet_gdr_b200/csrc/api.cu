@@ -135,12 +135,12 @@ extern "C" int gdr_chunk_fwd(const void *q, const void *k, const void *v, const 
     return e == cudaSuccess ? GDR_OK : GDR_ERR_LAUNCH;
 }
 
-extern "C" int gdr_recurrent_step(const void *q, const void *k, const void *v, const void *beta, const float *g,
-                                  const float *gk, void *state_pool, int slots, const int32_t *ssm_state_indices,
-                                  const int32_t *actual_seq_lengths, const int32_t *num_accepted_tokens,
-                                  float scale, int B, int Nk, int Nv, int S, int Dk, int Dv, gdr_dtype dtype,
-                                  gdr_dtype state_dtype, const gdr_prologue *prologue,
-                                  const gdr_epilogue *epilogue, void *out, gdr_stream_t stream) {
+namespace {
+int recurrent_step(const void *q, const void *k, const void *v, const void *beta, const float *g, const float *gk,
+                   void *state_pool, int slots, const int32_t *ssm_state_indices, const int32_t *actual_seq_lengths,
+                   const int32_t *num_accepted_tokens, float scale, int B, int Nk, int Nv, int S, int Dk, int Dv,
+                   gdr_dtype dtype, gdr_dtype state_dtype, const gdr_prologue *prologue, const gdr_epilogue *epilogue,
+                   void *out, gdr_stream_t stream, int per_token) {
     int st = check_common(B, Nk, Nv, S, Dk, Dv, dtype);
     if (st) return st;
     if (state_dtype != GDR_F32 && state_dtype != GDR_BF16) return GDR_ERR_DTYPE;
@@ -170,12 +170,37 @@ extern "C" int gdr_recurrent_step(const void *q, const void *k, const void *v, c
     a.A_log = prologue ? prologue->A_log : nullptr;
     a.dt_bias = prologue ? prologue->dt_bias : nullptr;
     a.err = err;
+    a.per_token = per_token;
     cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
     cudaError_t e = launch_decode(a, Dk, Dv, dtype, state_dtype, cs);
     if (e == cudaSuccess && epilogue)
         e = launch_gated_rmsnorm(out, epilogue->z, epilogue->norm_w, epilogue->eps, actual_seq_lengths, B, Nv, S, Dv,
                                  dtype, cs);
     return e == cudaSuccess ? GDR_OK : GDR_ERR_LAUNCH;
+}
+}  // namespace
+
+extern "C" int gdr_recurrent_step(const void *q, const void *k, const void *v, const void *beta, const float *g,
+                                  const float *gk, void *state_pool, int slots, const int32_t *ssm_state_indices,
+                                  const int32_t *actual_seq_lengths, const int32_t *num_accepted_tokens,
+                                  float scale, int B, int Nk, int Nv, int S, int Dk, int Dv, gdr_dtype dtype,
+                                  gdr_dtype state_dtype, const gdr_prologue *prologue,
+                                  const gdr_epilogue *epilogue, void *out, gdr_stream_t stream) {
+    return recurrent_step(q, k, v, beta, g, gk, state_pool, slots, ssm_state_indices, actual_seq_lengths,
+                          num_accepted_tokens, scale, B, Nk, Nv, S, Dk, Dv, dtype, state_dtype, prologue, epilogue,
+                          out, stream, 0);
+}
+
+extern "C" int gdr_recurrent_step_spec(const void *q, const void *k, const void *v, const void *beta,
+                                       const float *g, const float *gk, void *state_pool, int slots,
+                                       const int32_t *ssm_state_indices, const int32_t *actual_seq_lengths,
+                                       const int32_t *num_accepted_tokens, float scale, int B, int Nk, int Nv, int S,
+                                       int Dk, int Dv, gdr_dtype dtype, gdr_dtype state_dtype,
+                                       const gdr_prologue *prologue, const gdr_epilogue *epilogue, void *out,
+                                       gdr_stream_t stream) {
+    return recurrent_step(q, k, v, beta, g, gk, state_pool, slots, ssm_state_indices, actual_seq_lengths,
+                          num_accepted_tokens, scale, B, Nk, Nv, S, Dk, Dv, dtype, state_dtype, prologue, epilogue,
+                          out, stream, 1);
 }
 
 extern "C" int gdr_conv1d(const void *x, const void *weight, const void *bias, const void *conv_state_in,

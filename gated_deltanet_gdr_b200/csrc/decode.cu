@@ -148,7 +148,7 @@ __device__ __forceinline__ void prefetch_meta(const DecodeArgs &a, int tile, int
     } else if (tid == T) {
         r[0] = a.lengths[b];
     } else if (tid == T + 1) {
-        r[0] = a.accepted ? a.accepted[b] : a.lengths[b];
+        r[0] = a.accepted ? a.accepted[b] : (a.per_token ? 1 : a.lengths[b]);
     }
 }
 __device__ __forceinline__ void put_meta(int *mm, int tid, const int (&r)[3]) {
@@ -162,15 +162,28 @@ __device__ __forceinline__ void put_meta(int *mm, int tid, const int (&r)[3]) {
         mm[1] = r[0];
     }
 }
-// 0 = process, 1 = bad length, 2 = a referenced slot index out of range (same answer in every thread)
-__device__ __forceinline__ int tile_status(const int *mm, int S, int slots) {
+// 0 = process, 1 = bad length (or, per-token reading, an accepted count outside [1, S]), 2 = a referenced slot
+// index out of range (same answer in every thread).  mm = (L, A, idx[T], ...).
+__device__ __forceinline__ int tile_status(const int *mm, int S, int slots, int per_token) {
     const int L = mm[0], A = mm[1];
     if (L < 0 || L > S) return 1;
+    if (per_token && L > 0) {  // the start slot is that of token A - 1; every processed token commits
+        if (A < 1 || A > S) return 1;
+        if (mm[2 + A - 1] < 0 || mm[2 + A - 1] >= slots) return 2;
+        for (int t = 0; t < L; ++t)
+            if (mm[2 + t] < 0 || mm[2 + t] >= slots) return 2;
+        return 0;
+    }
     int nref = min(L, A);
     if (L > 0 && nref < 1) nref = 1;
     for (int t = 0; t < nref; ++t)
         if (mm[2 + t] < 0 || mm[2 + t] >= slots) return 2;
     return 0;
+}
+// slot the chain starts from, and the number of leading tokens whose states are committed (a valid tile)
+__device__ __forceinline__ int start_slot(const int *mm, int per_token) { return mm[2 + (per_token ? mm[1] - 1 : 0)]; }
+__device__ __forceinline__ int commit_count(const int *mm, int Lv, int per_token) {
+    return per_token ? Lv : min(mm[1], Lv);
 }
 
 template <int DK, int DV, typename TI, typename TS>
@@ -193,10 +206,11 @@ decode_kernel(const DecodeArgs a, const int ntiles) {
         uint8_t *st = smem + stage * ly.stage;
         const int split = tile % Cf::NSPLIT, bh = tile / Cf::NSPLIT, h = bh % a.Nv, b = bh / a.Nv;
         const int kh = h / (a.Nv / a.Nk), col0 = split * DVC;
-        const int Lc = tile_status(mm, S, a.slots) ? 0 : mm[0];
+        const int Lc = tile_status(mm, S, a.slots, a.per_token) ? 0 : mm[0];
         if (Lc > 0) {
             const uint8_t *src = reinterpret_cast<const uint8_t *>(
-                reinterpret_cast<const TS *>(a.pool) + ((size_t)mm[2] * a.Nv + h) * tile_elems + col0);
+                reinterpret_cast<const TS *>(a.pool) + ((size_t)start_slot(mm, a.per_token) * a.Nv + h) * tile_elems +
+                col0);
 #pragma unroll
             for (int i = 0; i < Cf::COPY_ITERS; ++i) {
                 const int e = i * NT + tid, row = e / CPR, pc = e % CPR;
@@ -258,9 +272,9 @@ decode_kernel(const DecodeArgs a, const int ntiles) {
         const int *mm = s_meta + (j % 3) * META_INTS;
         const int split = tile % Cf::NSPLIT, bh = tile / Cf::NSPLIT, h = bh % a.Nv;
         const int col0 = split * DVC;
-        const int status = tile_status(mm, S, a.slots);
+        const int status = tile_status(mm, S, a.slots, a.per_token);
         const int Lv = status ? 0 : mm[0];
-        const int A = min(mm[1], Lv);
+        const int A = commit_count(mm, Lv, a.per_token);
         if (tid == 0 && status) raise_device_error(a.err, status == 1 ? GDR_DEVERR_LENGTH : GDR_DEVERR_SLOT_INDEX);
         TI *out = reinterpret_cast<TI *>(a.out) + (size_t)bh * S * DV + col0;
         for (int e = tid; e < (S - Lv) * (DVC / 8); e += NT) {
@@ -455,7 +469,7 @@ __device__ __forceinline__ void prefetch_meta128(const DecodeArgs &a, int bh, in
     } else if (tid == T) {
         r[0] = a.lengths[b];
     } else if (tid == T + 1) {
-        r[0] = a.accepted ? a.accepted[b] : a.lengths[b];
+        r[0] = a.accepted ? a.accepted[b] : (a.per_token ? 1 : a.lengths[b]);
     }
 }
 // The set layout of put_meta (L, A, idx[T], beta[T], g[T]), with beta and the decay e^g final.
@@ -500,7 +514,7 @@ decode128_kernel(const __grid_constant__ CUtensorMap tm_pool, const DecodeArgs a
     auto issue = [&](int tile, const int *mm, int st) {
         uint64_t *bar = full + st;
         uint8_t *base = smem + st * ly.stage;
-        const int status = tile_status(mm, S, a.slots);
+        const int status = tile_status(mm, S, a.slots, a.per_token);
         const int Lc = status ? 0 : mm[0];
         if (Lc <= 0) {
             sm100::mbar_arrive(bar);
@@ -509,7 +523,7 @@ decode128_kernel(const __grid_constant__ CUtensorMap tm_pool, const DecodeArgs a
         const int h = tile % a.Nv, b = tile / a.Nv, kh = h / (a.Nv / a.Nk);
         const uint32_t tok = (uint32_t)Lc * D * (uint32_t)sizeof(TI);
         sm100::mbar_arrive_expect_tx(bar, Cf::STATE_BYTES + 3 * tok + (a.gk ? (uint32_t)Lc * D * 4 : 0));
-        const int z = mm[2] * a.Nv + h;
+        const int z = start_slot(mm, a.per_token) * a.Nv + h;
 #pragma unroll
         for (int x = 0; x < Cf::NBOX; ++x) sm100::tma_load_3d(base + x * (D * 128), &tm_pool, bar, x * Cf::BOXC, 0, z);
         const size_t qk_off = ((size_t)b * a.Nk + kh) * S * D, v_off = (size_t)tile * S * D;
@@ -558,9 +572,9 @@ decode128_kernel(const __grid_constant__ CUtensorMap tm_pool, const DecodeArgs a
         const int st = j % NS;
         const int *mm = s_meta + (j & 3) * META_INTS;
         const int h = tile % a.Nv;
-        const int status = tile_status(mm, S, a.slots);
+        const int status = tile_status(mm, S, a.slots, a.per_token);
         const int Lv = status ? 0 : mm[0];
-        const int A = min(mm[1], Lv);
+        const int A = commit_count(mm, Lv, a.per_token);
         if (tid == 0 && status) raise_device_error(a.err, status == 1 ? GDR_DEVERR_LENGTH : GDR_DEVERR_SLOT_INDEX);
         TI *out = reinterpret_cast<TI *>(a.out) + (size_t)tile * S * D;
         for (int e = tid; e < (S - Lv) * (D / 8); e += Cf::NT) {

@@ -26,6 +26,7 @@ struct DecodeArgs {
     int beta_logits;
     const float *A_log, *dt_bias;
     unsigned int *err;
+    int per_token;  // num_accepted_tokens read per token (speculative decoding): see gdr_recurrent_step_spec
 };
 
 struct ChunkArgs {

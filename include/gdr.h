@@ -190,6 +190,26 @@ int gdr_recurrent_step(const void *q, const void *k, const void *v, const void *
                        gdr_stream_t stream);
 
 /*
+ * The decode call with the speculative-decoding reading of num_accepted_tokens:
+ * per-token state slots.  Source: the recurrent_gated_delta_rule operator
+ * (lite_boost) gives num_accepted_tokens only as the number of accepted
+ * tokens; in speculative decoding the previous step wrote the state after each
+ * of its tokens to that token's own slot and A_b of them were accepted.  So
+ * here the chain of sequence b starts from pool[ssm_state_indices[b*S + A_b - 1]]
+ * and the state after every processed token t < L_b is written to
+ * pool[ssm_state_indices[b*S + t]].  A_b must lie in [1, S] for a sequence with
+ * L_b > 0 (otherwise the sequence is skipped, its out rows are zero and
+ * GDR_DEVERR_LENGTH is set); num_accepted_tokens == NULL means A_b = 1.
+ * Arguments, layouts and the other errors are those of gdr_recurrent_step.
+ */
+int gdr_recurrent_step_spec(const void *q, const void *k, const void *v, const void *beta, const float *g,
+                            const float *gk, void *state_pool, int slots, const int32_t *ssm_state_indices,
+                            const int32_t *actual_seq_lengths, const int32_t *num_accepted_tokens, float scale,
+                            int B, int Nk, int Nv, int S, int Dk, int Dv, gdr_dtype dtype, gdr_dtype state_dtype,
+                            const gdr_prologue *prologue, const gdr_epilogue *epilogue, void *out,
+                            gdr_stream_t stream);
+
+/*
  * Depthwise causal conv1d + SiLU over the fused q/k/v channels, with its state:
  * the step before the rule, writing the rule's q, k and v.  Source: the layer's
  * conv over mixed_qkv = cat(q, k, v) with causal_conv1d_fn (prefill) and
