@@ -378,6 +378,53 @@ def bench_conv1d(gdr, args, world, rank, flush, stream, peaks):
                          "algorithmic_bytes_per_launch": alg, "kernel": "gdr_conv1d"}}, 2 * args.steps
 
 
+def bench_f16(gdr, args, world, rank, flush, stream, peaks):
+    """fp16 inputs: the prefill workload (fused prologue; the tensor-core kernel with fp16 operands) and the decode
+    workload with an fp32 state (the general decode kernel).  Returns (fields, launches)."""
+    h = lambda x: torch.from_numpy(np.ascontiguousarray(x)).to(torch.float16).cuda()
+    w = workloads.generate("prefill", seed=2 + 1000 * rank)
+    pro = gdr.Prologue(l2norm_qk=True, eps=1e-6, beta_logits=True, A_log=f32_dev(w.A_log), dt_bias=f32_dev(w.dt_bias))
+    out = torch.empty((w.B, w.Nv, w.S, w.Dv), dtype=torch.float16, device="cuda")
+    s0 = h(w.initial_state)
+    fin = torch.empty_like(s0)
+    step = gdr.prepare_chunk_fwd(h(w.q), h(w.k), h(w.v), h(w.b), f32_dev(w.a), s0, None, w.scale, prologue=pro,
+                                 out=out, final_state=fin)
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    barrier(world)
+    times = timed_steps(step, args.steps, flush, stream)
+    barrier(world)
+    p_ms = all_max(sum(times), world) / args.steps
+    alg = algorithmic_prefill_bytes(w)
+    wd = workloads.generate("decode", seed=1 + 1000 * rank)
+    pool = f32_dev(wd.pool)
+    dout = torch.empty((wd.B, wd.Nv, wd.S, wd.Dv), dtype=torch.float16, device="cuda")
+    dstep = gdr.prepare_recurrent_step(h(wd.q), h(wd.k), h(wd.v), h(wd.b), f32_dev(wd.g), None, pool,
+                                       torch.from_numpy(wd.indices).cuda(), torch.from_numpy(wd.lengths).cuda(),
+                                       torch.from_numpy(wd.accepted).cuda(), wd.scale,
+                                       prologue=gdr.Prologue(l2norm_qk=True, eps=1e-6, beta_logits=True), out=dout)
+    for _ in range(args.warmup):
+        dstep()
+    torch.cuda.synchronize()
+    barrier(world)
+    dtimes = timed_steps(dstep, args.steps, flush, stream)
+    barrier(world)
+    d_ms = all_max(sum(dtimes), world) / args.steps
+    nb = algorithmic_decode_bytes(wd)
+    nb_state = nb["state"] * 2  # the fp32 state moves twice the bytes of the bf16 one counted there
+    d_gbs = (nb_state + nb["io"]) / (d_ms / 1e3) / 1e9
+    return {"prefill": {"workload": "prefill B=4 S=4096 Nk=16 Nv=32 D=128 fp16, fused prologue (tensor-core kernel)",
+                        "ms_per_step": p_ms, "tokens_per_s": weak_scaling_rate(int(w.lengths.sum()), args.steps,
+                                                                              p_ms * args.steps, world),
+                        "roofline": {"bound": "hbm", "achieved": alg / (p_ms / 1e3) / 1e9, "peak": peaks["hbm_gbs"],
+                                     "unit": "GB/s", "frac": alg / (p_ms / 1e3) / 1e9 / peaks["hbm_gbs"]}},
+            "decode": {"workload": "decode B=64 S=1 fp16 inputs, fp32 state (general decode kernel), L2 flush",
+                       "us_per_call": d_ms * 1e3,
+                       "roofline": {"bound": "hbm", "achieved": d_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                                    "frac": d_gbs / peaks["hbm_gbs"]}}}, 2 * args.steps
+
+
 def bench_e2e(gdr, args, world, w, t, pro, flush, stream):
     """Same metric through the public call with host buffers: pinned H2D copies of the
     step's inputs, the call, D2H of out and the final state, all inside the timed region."""
@@ -494,6 +541,9 @@ def run_ours(args, world, rank, local):
     if args.only in ("all", "conv1d"):
         line["conv1d"], n = bench_conv1d(gdr, args, world, rank, flush, stream, peaks)
         launches += n
+    if args.only in ("all", "f16"):
+        line["f16"], n = bench_f16(gdr, args, world, rank, flush, stream, peaks)
+        launches += n
     decode = {}
     for name in ("decode", "decode_gk", "decode_spec"):
         if args.only in ("all", name):
@@ -524,7 +574,7 @@ def main():
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg (profiling runs)")
     ap.add_argument("--no-epilogue", action="store_true",
                     help="skip the prefill line with the fused gated RMSNorm epilogue (profiling runs)")
-    ap.add_argument("--only", choices=["all", "prefill", "decode", "decode_gk", "decode_spec", "conv1d"],
+    ap.add_argument("--only", choices=["all", "prefill", "decode", "decode_gk", "decode_spec", "conv1d", "f16"],
                     default="all",
                     help="run one workload only (profiling runs); the default runs all")
     args = ap.parse_args()

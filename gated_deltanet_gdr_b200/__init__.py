@@ -27,7 +27,7 @@ LIB_PATH = os.path.join(_PKG, "libgdr.so")
 
 GDR_OK, GDR_ERR_SHAPE, GDR_ERR_DTYPE, GDR_ERR_NULL, GDR_ERR_ALIGN, GDR_ERR_UNSUPPORTED, GDR_ERR_DEVICE, \
     GDR_ERR_LAUNCH = range(8)
-GDR_F32, GDR_BF16 = 0, 1
+GDR_F32, GDR_BF16, GDR_F16 = 0, 1, 2
 DEVERR_SLOT_INDEX, DEVERR_LENGTH = 0x1, 0x2
 
 # Every symbol the C header declares (checked by the ABI test).
@@ -136,7 +136,9 @@ def _dtype_code(dt: torch.dtype) -> int:
         return GDR_F32
     if dt == torch.bfloat16:
         return GDR_BF16
-    raise RuntimeError(f"unsupported dtype {dt}; use torch.float32 or torch.bfloat16")
+    if dt == torch.float16:
+        return GDR_F16
+    raise RuntimeError(f"unsupported dtype {dt}; use torch.float32, torch.bfloat16 or torch.float16")
 
 
 def _dev(t: torch.Tensor, name: str, dtype=None, shape=None):

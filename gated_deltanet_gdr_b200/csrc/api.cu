@@ -59,7 +59,7 @@ int device_setup(unsigned int **err) {
 }
 
 int check_common(int B, int Nk, int Nv, int S, int Dk, int Dv, int dtype) {
-    if (dtype != GDR_F32 && dtype != GDR_BF16) return GDR_ERR_DTYPE;
+    if (dtype != GDR_F32 && dtype != GDR_BF16 && dtype != GDR_F16) return GDR_ERR_DTYPE;
     if (B < 0 || S < 0 || Nk < 1 || Nv < 1 || Dk < 1 || Dv < 1) return GDR_ERR_SHAPE;
     if (Nv % Nk != 0) return GDR_ERR_SHAPE;
     if (!supported_head(Dk) || !supported_head(Dv)) return GDR_ERR_UNSUPPORTED;
@@ -125,7 +125,7 @@ extern "C" int gdr_chunk_fwd(const void *q, const void *k, const void *v, const 
             a.epi_w = epilogue->norm_w;
             a.epi_eps = epilogue->eps;
         }
-        e = launch_chunk_tc(a, cs);
+        e = launch_chunk_tc(a, dtype, cs);
     } else {
         e = launch_chunk_simt(a, Dk, Dv, dtype, cs);
         if (e == cudaSuccess && epilogue && S > 0)
@@ -143,7 +143,10 @@ int recurrent_step(const void *q, const void *k, const void *v, const void *beta
                    void *out, gdr_stream_t stream, int per_token) {
     int st = check_common(B, Nk, Nv, S, Dk, Dv, dtype);
     if (st) return st;
-    if (state_dtype != GDR_F32 && state_dtype != GDR_BF16) return GDR_ERR_DTYPE;
+    if (state_dtype != GDR_F32 && state_dtype != GDR_BF16 && state_dtype != GDR_F16) return GDR_ERR_DTYPE;
+    // fp16 inputs take an fp16 or fp32 state; an fp16 state takes fp16 inputs
+    if ((dtype == GDR_F16 && state_dtype == GDR_BF16) || (state_dtype == GDR_F16 && dtype != GDR_F16))
+        return GDR_ERR_DTYPE;
     if (S < 1 || S > kDecodeMaxTokens || slots < 1) return GDR_ERR_SHAPE;
     if ((st = check_prologue(prologue, g))) return st;
     if ((st = check_epilogue(epilogue))) return st;
@@ -228,7 +231,7 @@ extern "C" int gdr_prologue_apply(const void *q, const void *k, const void *b, c
                                   const float *dt_bias, float eps, int B, int Nk, int Nv, int S, int Dk,
                                   gdr_dtype dtype, void *q_hat, void *k_hat, void *beta, float *g,
                                   gdr_stream_t stream) {
-    if (dtype != GDR_F32 && dtype != GDR_BF16) return GDR_ERR_DTYPE;
+    if (dtype != GDR_F32 && dtype != GDR_BF16 && dtype != GDR_F16) return GDR_ERR_DTYPE;
     if (B < 0 || S < 0 || Nk < 1 || Nv < 1 || Dk < 1) return GDR_ERR_SHAPE;
     if (!(eps >= 0.f)) return GDR_ERR_SHAPE;
     if ((q && !q_hat) || (k && !k_hat) || (b && !beta) || (a && (!g || !A_log || !dt_bias))) return GDR_ERR_NULL;

@@ -228,6 +228,14 @@ static cudaError_t launch_simt_k(const ChunkArgs &a, int DV, cudaStream_t s) {
 }
 
 cudaError_t launch_chunk_simt(const ChunkArgs &a, int Dk, int Dv, gdr_dtype dt, cudaStream_t s) {
+    if (dt == GDR_F16) {
+        switch (Dk) {
+            case 16: return launch_simt_k<16, __half>(a, Dv, s);
+            case 32: return launch_simt_k<32, __half>(a, Dv, s);
+            case 64: return launch_simt_k<64, __half>(a, Dv, s);
+            default: return launch_simt_k<128, __half>(a, Dv, s);
+        }
+    }
     if (dt == GDR_BF16) {
         switch (Dk) {
             case 16: return launch_simt_k<16, __nv_bfloat16>(a, Dv, s);

@@ -1,8 +1,8 @@
 // chunk_tc.cu -- chunked prefill of the gated delta rule on the sm_100a tensor cores.
 //
 // The chunked (WY / UT transform) form of torch_chunk_gated_delta_rule (blog
-// "gated-delta-net" page, steps 1-8), chunk C = 64, head size Dk = Dv = 128, bf16 in
-// and out, fp32 accumulation and an fp32 state.  One CTA owns one (b, value head)
+// "gated-delta-net" page, steps 1-8), chunk C = 64, head size Dk = Dv = 128, bf16 or fp16
+// in and out (the MMA operand copies in the same type), fp32 accumulation and an fp32 state.  One CTA owns one (b, value head)
 // chain.  Per chunk:
 //
 //   a1  G_t = cumulative log-gate (tokens past the length count 0).
@@ -151,7 +151,7 @@ struct TcArgs {
     int beta_logits;
     const float *A_log, *dt_bias;
     unsigned int *err;
-    const __nv_bfloat16 *epi_z;  // NULL: no epilogue
+    const void *epi_z;  // NULL: no epilogue
     const float *epi_w;
     float epi_eps;
 };
@@ -160,14 +160,17 @@ __device__ __forceinline__ uint32_t blk_off(uint32_t row, uint32_t col) {  // wi
     return (row >> 3) * 1024u + sw128_offset(row & 7u, col);
 }
 
-// silu(x) = x sigmoid(x) with sigmoid(x) = (1 + tanh(x / 2)) / 2 and tanh on the special-function unit (PTX
-// tanh.approx, relative error about 2^-11): one special-function operation per element; the result is rounded
-// to bf16 (2^-9) right after
-__device__ __forceinline__ float silu_fast(float x) {
+// silu(x) = x sigmoid(x).  For bf16 outputs sigmoid(x) = (1 + tanh(x / 2)) / 2 with tanh on the special-function
+// unit (PTX tanh.approx, relative error about 2^-11, below the bf16 rounding of 2^-9 that follows): one
+// special-function operation per element.  For fp16 outputs (rounding 2^-11) x / (1 + e^{-x}) with the fast
+// division (about 1e-6).
+template <typename T> __device__ __forceinline__ float silu_out(float x);
+template <> __device__ __forceinline__ float silu_out<__nv_bfloat16>(float x) {
     float t;
     asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(0.5f * x));
     return x * fmaf(0.5f, t, 0.5f);
 }
+template <> __device__ __forceinline__ float silu_out<__half>(float x) { return __fdividef(x, 1.f + __expf(-x)); }
 
 // 2^x and log2(x) on the special-function unit (PTX ex2.approx / lg2.approx, flush to zero)
 __device__ __forceinline__ float ex2_approx(float x) {
@@ -181,18 +184,44 @@ __device__ __forceinline__ float lg2_approx(float x) {
     return y;
 }
 
-__device__ __forceinline__ void unpack8(uint4 u, float (&f)[8]) {
-    const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&u);
+// The element type of the inputs, the operand copies and the outputs: bf16 or fp16 (tcgen05 kind::f16 takes
+// either, A and B of the same type).  TMA data type, descriptor operand format, and pairs packed / unpacked.
+template <typename T> struct TcT;
+template <> struct TcT<__nv_bfloat16> {
+    static constexpr CUtensorMapDataType kMap = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    static constexpr uint32_t kFmt = 1;
+    static __device__ __forceinline__ uint32_t pack2(float lo, float hi) { return pack_bf16x2(lo, hi); }
+    static __device__ __forceinline__ float2 unpack2(uint32_t u) {
+        return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u));
+    }
+};
+template <> struct TcT<__half> {
+    static constexpr CUtensorMapDataType kMap = CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+    static constexpr uint32_t kFmt = 0;
+    static __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
+        const __half2 h = __floats2half2_rn(lo, hi);
+        return *reinterpret_cast<const uint32_t *>(&h);
+    }
+    static __device__ __forceinline__ float2 unpack2(uint32_t u) {
+        return __half22float2(*reinterpret_cast<const __half2 *>(&u));
+    }
+};
+template <typename T> __host__ __device__ constexpr uint32_t idesc_t(int M, int N, bool a_mn_major, bool b_mn_major) {
+    return idesc_f16kind(M, N, a_mn_major, b_mn_major, TcT<T>::kFmt);
+}
+
+template <typename T> __device__ __forceinline__ void unpack8(uint4 u, float (&f)[8]) {
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-        float2 x = __bfloat1622float2(h[i]);
+        const float2 x = TcT<T>::unpack2(w[i]);
         f[2 * i] = x.x;
         f[2 * i + 1] = x.y;
     }
 }
-__device__ __forceinline__ uint4 pack8(const float *f) {
-    return make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]), pack_bf16x2(f[4], f[5]),
-                      pack_bf16x2(f[6], f[7]));
+template <typename T> __device__ __forceinline__ uint4 pack8(const float *f) {
+    return make_uint4(TcT<T>::pack2(f[0], f[1]), TcT<T>::pack2(f[2], f[3]), TcT<T>::pack2(f[4], f[5]),
+                      TcT<T>::pack2(f[6], f[7]));
 }
 
 // D (16 x 8) += A (16 x 8) B (8 x 8) with tf32 operands and fp32 accumulation: one warp-level tensor-core MMA.
@@ -288,6 +317,7 @@ __device__ __forceinline__ void solve_diag16_merge(const float *sA, float *sT, f
     named_sync(BAR_PREP, NGRP);
 }
 
+template <typename T>
 __global__ void __launch_bounds__(NT, 1)
 chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o, const TcArgs a) {
@@ -358,7 +388,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 
     if (carry) {
         // ---- initial state into TMEM (fp32) and the bf16 operand tile ----
-        const __nv_bfloat16 *s0 = reinterpret_cast<const __nv_bfloat16 *>(a.initial_state);
+        const T *s0 = reinterpret_cast<const T *>(a.initial_state);
         const size_t off = ((size_t)bh * D + row) * D + 64 * hf;
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
@@ -367,7 +397,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             for (int c8 = 0; c8 < 4; ++c8) {
                 float f[8];
                 if (s0) {
-                    unpack8(*reinterpret_cast<const uint4 *>(s0 + off + 32 * half + 8 * c8), f);
+                    unpack8<T>(*reinterpret_cast<const uint4 *>(s0 + off + 32 * half + 8 * c8), f);
                 } else {
 #pragma unroll
                     for (int i = 0; i < 8; ++i) f[i] = 0.f;
@@ -375,7 +405,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 #pragma unroll
                 for (int i = 0; i < 8; ++i) v[8 * c8 + i] = f[i];
                 *reinterpret_cast<uint4 *>(sm + OFF_S + hf * 16384 + blk_off(row, 32 * half + 8 * c8)) =
-                    pack8(&v[8 * c8]);
+                    pack8<T>(&v[8 * c8]);
             }
             tmem_st32(tmem + TM_S + lane_base + 64 * hf + 32 * half, v);
         }
@@ -409,7 +439,8 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             tma_prefetch_3d(&tm_v, 64, y, bh);
             if (a.epi_z) {  // the chunk's z rows of the epilogue: one contiguous block of valid rows
                 const int rows = min(C, L - y);
-                asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(a.epi_z + ((size_t)bh * S + y) * D),
+                asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;"
+                             ::"l"(static_cast<const T *>(a.epi_z) + ((size_t)bh * S + y) * D),
                              "r"((uint32_t)(rows * D * 2))
                              : "memory");
             }
@@ -437,7 +468,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         // gate G (from the raw gate), e^G, G log2(e), e^{G_last - G} and the valid-token count; two
         // tokens per lane, the scan over the chunk by warp shuffles.
         const float gA = (a.A_log && a.g) ? a.A_log[h] : 0.f, gB = (a.A_log && a.g) ? a.dt_bias[h] : 0.f;
-        const __nv_bfloat16 *bg = reinterpret_cast<const __nv_bfloat16 *>(a.beta) + (size_t)bh * S;
+        const T *bg = reinterpret_cast<const T *>(a.beta) + (size_t)bh * S;
         const float *gg = a.g ? a.g + (size_t)bh * S : nullptr;
         // raw beta and gate values of a chunk's tokens (two per lane), loaded a chunk before they are used so
         // that their memory latency stays off the hand-offs
@@ -446,7 +477,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 #pragma unroll
             for (int i = 0; i < 2; ++i) {
                 const int tt = 2 * lane + i, t = chunk * C + tt;
-                rb[i] = tt < n ? __bfloat162float(bg[t]) : 0.f;
+                rb[i] = tt < n ? to_f32(bg[t]) : 0.f;
                 rg[i] = (tt < n && gg) ? gg[t] : 0.f;
             }
         };
@@ -502,7 +533,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                               // the row norms
                 if (!mbar_wait(bar_ld, par)) to = true;
                 tc_fence_after();
-                const uint32_t id = idesc_bf16(128, 128, false, false);
+                const uint32_t id = idesc_t<T>(128, 128, false, false);
 #pragma unroll
                 for (int k = 0; k < 8; ++k) {
                     const uint32_t addr = sbase + off_gram(par, k >> 2) + (k & 3) * 32;
@@ -557,11 +588,11 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     const int t = (e >> 3) & 63;
                     uint4 *pk = reinterpret_cast<uint4 *>(sm + OFF_KT + (e >> 9) * 8192 + t * 128 + (e & 7) * 16);
                     float f[8];
-                    unpack8(*pk, f);
+                    unpack8<T>(*pk, f);
                     const float sc = vtail[t];
 #pragma unroll
                     for (int j = 0; j < 8; ++j) f[j] = t < n ? f[j] * sc : 0.f;
-                    *pk = pack8(f);
+                    *pk = pack8<T>(f);
                 }
             }
             fence_proxy_async_smem();
@@ -675,7 +706,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                         for (int j = 0; j < 32; ++j) v[j] = (32 * hf + j <= t) ? v[j] : 0.f;
 #pragma unroll
                         for (int c8 = 0; c8 < 4; ++c8)
-                            *reinterpret_cast<uint4 *>(pm + blk_off(t, 32 * hf + 8 * c8)) = pack8(&v[8 * c8]);
+                            *reinterpret_cast<uint4 *>(pm + blk_off(t, 32 * hf + 8 * c8)) = pack8<T>(&v[8 * c8]);
                     }
                 } else if (!krole) {  // Pm rows 0..31, columns 32..63: above the diagonal
 #pragma unroll
@@ -716,8 +747,8 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     fb[i] = tv[i] * vBeta[col + i];
                     fw[i] = tv[i] * vCw[col + i];
                 }
-                *reinterpret_cast<uint4 *>(sm + OFF_TT + blk_off(R, col)) = pack8(fb);
-                *reinterpret_cast<uint4 *>(sm + OFF_TT + blk_off(64 + R, col)) = pack8(fw);
+                *reinterpret_cast<uint4 *>(sm + OFF_TT + blk_off(R, col)) = pack8<T>(fb);
+                *reinterpret_cast<uint4 *>(sm + OFF_TT + blk_off(64 + R, col)) = pack8<T>(fw);
                 // zeros: TT rows 0..31 and 64..95, columns 32..63 (above the diagonal)
                 const int Rz = (p >> 2) + ((p >> 7) << 5), cz = 4 + (p & 3);
                 *reinterpret_cast<uint4 *>(sm + OFF_TT + blk_off(Rz, 8 * cz)) = make_uint4(0, 0, 0, 0);
@@ -735,8 +766,8 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 for (int hh = 0; hh < 2; ++hh) {
                     const int r = 16 * rt + gq + 8 * hh;
                     const float t0 = -d[2 * hh], t1 = -d[2 * hh + 1];
-                    *reinterpret_cast<uint32_t *>(sm + OFF_TT + blk_off(32 + r, s0)) = pack_bf16x2(t0 * b0, t1 * b1);
-                    *reinterpret_cast<uint32_t *>(sm + OFF_TT + blk_off(96 + r, s0)) = pack_bf16x2(t0 * w0, t1 * w1);
+                    *reinterpret_cast<uint32_t *>(sm + OFF_TT + blk_off(32 + r, s0)) = TcT<T>::pack2(t0 * b0, t1 * b1);
+                    *reinterpret_cast<uint32_t *>(sm + OFF_TT + blk_off(96 + r, s0)) = TcT<T>::pack2(t0 * w0, t1 * w1);
                 }
             }
             PHASE(14);
@@ -776,7 +807,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             if (tid == 0) {  // a4: W (rows 64..127 of TT K, into TMEM R) and U (rows 0..63 of TT V)
                 if (!mbar_wait(bar_ldv, par)) to = true;
                 tc_fence_after();
-                const uint32_t id = idesc_bf16(128, 128, false, true);
+                const uint32_t id = idesc_t<T>(128, 128, false, true);
 #pragma unroll
                 for (int k = 0; k < 4; ++k) {
                     const uint64_t ad = sdesc_sw128(sbase + OFF_TT + k * 32, 16, 1024);
@@ -798,7 +829,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 #pragma unroll
                     for (int c8 = 0; c8 < 4; ++c8)
                         *reinterpret_cast<uint4 *>(sm + OFF_A1 + hf * 16384 + blk_off(t, 32 * half + 8 * c8)) =
-                            pack8(&w[8 * c8]);
+                            pack8<T>(&w[8 * c8]);
                 }
             }
             fence_proxy_async_smem();
@@ -810,7 +841,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             const float eL = vec[V_EG * 64 + C - 1];
             // ---- R = [W; Q] S ----
             if (tid == 0) {
-                const uint32_t id = idesc_bf16(128, 128, false, true);
+                const uint32_t id = idesc_t<T>(128, 128, false, true);
                 TIMED(23, {
                     _Pragma("unroll")
                     for (int k = 0; k < 8; ++k) {
@@ -856,12 +887,13 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 #pragma unroll
                     for (int c8 = 0; c8 < 4; ++c8)
                         *reinterpret_cast<uint4 *>(sm + OFF_VO + hf * 8192 + blk_off(t, 32 * half + 8 * c8)) =
-                            pack8(&u[8 * c8]);
+                            pack8<T>(&u[8 * c8]);
                 }
             } else {  // rows of Q S: scale by e^{G_t} scale / |q_t| before Pm v_new accumulates onto them
                 if (a.epi_z && row - 64 < n)  // this thread's half row of z, for the epilogue
-                    asm volatile("prefetch.global.L1 [%0];" ::"l"(a.epi_z + ((size_t)bh * S + (size_t)c * C + row - 64) *
-                                                                        D + 64 * hf));
+                    asm volatile("prefetch.global.L1 [%0];" ::"l"(static_cast<const T *>(a.epi_z) +
+                                                                    ((size_t)bh * S + (size_t)c * C + row - 64) * D +
+                                                                    64 * hf));
                 const float xs = vec[V_XS * 64 + row - 64];
 #pragma unroll
                 for (int half = 0; half < 2; ++half) {
@@ -892,8 +924,8 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             if (tid == 0) {
                 if (!mbar_wait(bar_kt, par)) to = true;  // K~ of this chunk (helper warps)
                 tc_fence_after();
-                const uint32_t id_s = idesc_bf16(128, 128, true, true);
-                const uint32_t id_o = idesc_bf16(128, 128, false, true);
+                const uint32_t id_s = idesc_t<T>(128, 128, true, true);
+                const uint32_t id_o = idesc_t<T>(128, 128, false, true);
                 const uint32_t pm_rows = sbase + (par ? OFF_PM1 : OFF_PM0) - 8192;
                 TIMED(24, {
                     _Pragma("unroll")
@@ -926,7 +958,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 #pragma unroll
                 for (int c8 = 0; c8 < 4; ++c8)
                     *reinterpret_cast<uint4 *>(sm + OFF_S + hf * 16384 + blk_off(row, 32 * half + 8 * c8)) =
-                        pack8(&v[8 * c8]);
+                        pack8<T>(&v[8 * c8]);
                 if (more) {
 #pragma unroll
                     for (int j = 0; j < 32; ++j) v[j] *= eLn;
@@ -940,7 +972,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 // warp with the same lane), then o * inv * norm_w * silu(z) for this thread's 64 columns
                 const bool epi = a.epi_z != nullptr;
                 float inv = 1.f;
-                const __nv_bfloat16 *zr = nullptr;
+                const T *zr = nullptr;
                 if (epi) {
                     float ss = 0.f;
 #pragma unroll
@@ -953,8 +985,8 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     }
                     float *eps2 = reinterpret_cast<float *>(sm + OFF_EPI);
                     eps2[hf * 64 + t] = ss;
-                    if (t < n) zr = a.epi_z + ((size_t)bh * S + (size_t)c * C + t) * D + 64 * hf;  // rows past the
-                                                                                                   // length: unread
+                    if (t < n)  // rows past the length are never read
+                        zr = static_cast<const T *>(a.epi_z) + ((size_t)bh * S + (size_t)c * C + t) * D + 64 * hf;
                     named_sync(BAR_EPI, 128);
                     inv = rsqrtf((eps2[t] + eps2[64 + t]) * (1.f / D) + a.epi_eps);
                 }
@@ -967,12 +999,12 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 #pragma unroll
                         for (int c8 = 0; c8 < 4; ++c8) {
                             float zf[8];
-                            unpack8(*reinterpret_cast<const uint4 *>(zr + 32 * half + 8 * c8), zf);
+                            unpack8<T>(*reinterpret_cast<const uint4 *>(zr + 32 * half + 8 * c8), zf);
                             const float4 *wp = reinterpret_cast<const float4 *>(a.epi_w + 64 * hf + 32 * half + 8 * c8);
                             const float4 w0 = wp[0], w1 = wp[1];
                             const float wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
 #pragma unroll
-                            for (int i = 0; i < 8; ++i) o[8 * c8 + i] *= inv * wv[i] * silu_fast(zf[i]);
+                            for (int i = 0; i < 8; ++i) o[8 * c8 + i] *= inv * wv[i] * silu_out<T>(zf[i]);
                         }
                     }
 #pragma unroll
@@ -980,7 +1012,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 #pragma unroll
                     for (int c8 = 0; c8 < 4; ++c8)
                         *reinterpret_cast<uint4 *>(sm + OFF_VO + hf * 8192 + blk_off(t, 32 * half + 8 * c8)) =
-                            pack8(&o[8 * c8]);
+                            pack8<T>(&o[8 * c8]);
                 }
             }
             fence_proxy_async_smem();
@@ -1013,8 +1045,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 }
             }
             if (a.final_state) {
-                __nv_bfloat16 *fs =
-                    reinterpret_cast<__nv_bfloat16 *>(a.final_state) + ((size_t)bh * D + row) * D + 64 * hf;
+                T *fs = reinterpret_cast<T *>(a.final_state) + ((size_t)bh * D + row) * D + 64 * hf;
 #pragma unroll
                 for (int half = 0; half < 2; ++half) {
                     float v[32];
@@ -1022,7 +1053,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     tmem_ld_wait();
 #pragma unroll
                     for (int c8 = 0; c8 < 4; ++c8)
-                        *reinterpret_cast<uint4 *>(fs + 32 * half + 8 * c8) = pack8(&v[8 * c8]);
+                        *reinterpret_cast<uint4 *>(fs + 32 * half + 8 * c8) = pack8<T>(&v[8 * c8]);
                 }
             }
         }
@@ -1037,14 +1068,14 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     if (warp == 0) tmem_dealloc(tmem, TM_COLS);
 }
 
-// (D, S, Z) bf16 tensor, 64 x 64 boxes, 128-byte swizzle.
-bool make_map(CUtensorMap *m, const void *base, int S, long long Z) {
+// (D, S, Z) tensor of 2-byte elements (bf16 or fp16), 64 x 64 boxes, 128-byte swizzle.
+bool make_map(CUtensorMap *m, const void *base, int S, long long Z, CUtensorMapDataType type) {
     EncodeTiledFn enc = tensor_map_encoder();
     if (!enc) return false;
     cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)S, (cuuint64_t)Z};
     cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)S * D * 2};
     cuuint32_t box[3] = {64, 64, 1}, es[3] = {1, 1, 1};
-    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, es,
+    return enc(m, type, 3, const_cast<void *>(base), dims, strides, box, es,
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -1061,29 +1092,42 @@ extern "C" int gdr_phase_timers_read(unsigned long long *out) {
 }
 #endif
 
-bool chunk_tc_supported(int Dk, int Dv, gdr_dtype dt, int S) { return dt == GDR_BF16 && Dk == D && Dv == D && S > 0; }
+bool chunk_tc_supported(int Dk, int Dv, gdr_dtype dt, int S) {
+    return (dt == GDR_BF16 || dt == GDR_F16) && Dk == D && Dv == D && S > 0;
+}
 
-cudaError_t launch_chunk_tc(const ChunkArgs &ca, cudaStream_t stream) {
+namespace {
+template <typename T>
+cudaError_t launch_tc_t(const ChunkArgs &ca, cudaStream_t stream) {
+    constexpr CUtensorMapDataType ty = TcT<T>::kMap;
     CUtensorMap mq, mk, mv, mo;
-    if (!make_map(&mq, ca.q, ca.S, (long long)ca.B * ca.Nk) || !make_map(&mk, ca.k, ca.S, (long long)ca.B * ca.Nk) ||
-        !make_map(&mv, ca.v, ca.S, (long long)ca.B * ca.Nv) || !make_map(&mo, ca.out, ca.S, (long long)ca.B * ca.Nv))
+    if (!make_map(&mq, ca.q, ca.S, (long long)ca.B * ca.Nk, ty) ||
+        !make_map(&mk, ca.k, ca.S, (long long)ca.B * ca.Nk, ty) ||
+        !make_map(&mv, ca.v, ca.S, (long long)ca.B * ca.Nv, ty) ||
+        !make_map(&mo, ca.out, ca.S, (long long)ca.B * ca.Nv, ty))
         return cudaErrorInvalidValue;
     TcArgs a{};
     a.beta = ca.beta; a.g = ca.g; a.initial_state = ca.initial_state; a.lengths = ca.lengths; a.scale = ca.scale;
     a.B = ca.B; a.Nk = ca.Nk; a.Nv = ca.Nv; a.S = ca.S; a.final_state = ca.final_state;
     a.l2norm = ca.l2norm; a.eps = ca.eps; a.beta_logits = ca.beta_logits; a.A_log = ca.A_log;
     a.dt_bias = ca.dt_bias; a.err = ca.err;
-    a.epi_z = static_cast<const __nv_bfloat16 *>(ca.epi_z); a.epi_w = ca.epi_w; a.epi_eps = ca.epi_eps;
-    static bool attr_set = false;
+    a.epi_z = ca.epi_z; a.epi_w = ca.epi_w; a.epi_eps = ca.epi_eps;
+    static bool attr_set = false;  // one per element type
     if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(chunk_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+        cudaError_t e =
+            cudaFuncSetAttribute(chunk_tc_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
         if (e != cudaSuccess) return e;
         attr_set = true;
     }
     const long long blocks = (long long)ca.B * ca.Nv;
     if (blocks == 0) return cudaSuccess;
-    chunk_tc_kernel<<<(unsigned)blocks, NT, SMEM_BYTES, stream>>>(mq, mk, mv, mo, a);
+    chunk_tc_kernel<T><<<(unsigned)blocks, NT, SMEM_BYTES, stream>>>(mq, mk, mv, mo, a);
     return cudaGetLastError();
+}
+}  // namespace
+
+cudaError_t launch_chunk_tc(const ChunkArgs &ca, gdr_dtype dt, cudaStream_t stream) {
+    return dt == GDR_F16 ? launch_tc_t<__half>(ca, stream) : launch_tc_t<__nv_bfloat16>(ca, stream);
 }
 
 }  // namespace gdr

@@ -43,6 +43,20 @@ template <> struct ConvV<__nv_bfloat16> {
         *reinterpret_cast<uint2 *>(p) = *reinterpret_cast<const uint2 *>(h);
     }
 };
+template <> struct ConvV<__half> {
+    static constexpr int V = 4;
+    using Raw = uint2;
+    static __device__ __forceinline__ Raw zero() { return make_uint2(0, 0); }
+    static __device__ __forceinline__ void unpack(uint2 u, float (&x)[4]) {
+        const __half2 *h = reinterpret_cast<const __half2 *>(&u);
+        const float2 f0 = __half22float2(h[0]), f1 = __half22float2(h[1]);
+        x[0] = f0.x; x[1] = f0.y; x[2] = f1.x; x[3] = f1.y;
+    }
+    static __device__ __forceinline__ void store(__half *p, const float (&x)[4]) {
+        __half2 h[2] = {__floats2half2_rn(x[0], x[1]), __floats2half2_rn(x[2], x[3])};
+        *reinterpret_cast<uint2 *>(p) = *reinterpret_cast<const uint2 *>(h);
+    }
+};
 template <> struct ConvV<float> {
     static constexpr int V = 4;
     using Raw = uint4;
@@ -228,7 +242,9 @@ cudaError_t launch_conv1d(const void *x, const void *weight, const void *bias, c
     a.q = q; a.k = k; a.v = v; a.state_out = state_out;
     a.S = S; a.C = 2 * Nk * Dk + Nv * Dv; a.Nk = Nk; a.Nv = Nv; a.Dk = Dk; a.Dv = Dv; a.err = err;
     if (B == 0) return cudaSuccess;
-    return dt == GDR_BF16 ? launch_t<__nv_bfloat16>(a, B, K, s) : launch_t<float>(a, B, K, s);
+    if (dt == GDR_BF16) return launch_t<__nv_bfloat16>(a, B, K, s);
+    if (dt == GDR_F16) return launch_t<__half>(a, B, K, s);
+    return launch_t<float>(a, B, K, s);
 }
 
 }  // namespace gdr

@@ -820,6 +820,12 @@ cudaError_t launch_decode_t(const DecodeArgs &a, cudaStream_t stream) {
 
 template <int DK, int DV>
 cudaError_t launch_decode_d(const DecodeArgs &a, gdr_dtype dt, gdr_dtype st, cudaStream_t stream) {
+    // fp16 inputs (with an fp16 or fp32 state) run the general kernel at every head size
+    if (dt == GDR_F16) {
+        if (st == GDR_F16) return launch_decode_t<DK, DV, __half, __half>(a, stream);
+        if (st == GDR_F32) return launch_decode_t<DK, DV, __half, float>(a, stream);
+        return cudaErrorInvalidValue;
+    }
     if (DK == 128 && DV == 128) {
         if (dt == GDR_BF16 && st == GDR_BF16) return launch_decode128<__nv_bfloat16, __nv_bfloat16>(a, stream);
         if (dt == GDR_BF16 && st == GDR_F32) return launch_decode128<__nv_bfloat16, float>(a, stream);

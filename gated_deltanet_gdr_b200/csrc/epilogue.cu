@@ -71,6 +71,9 @@ cudaError_t launch_gated_rmsnorm(void *out, const void *z, const float *norm_w, 
     if (dt == GDR_BF16)
         return launch_t(static_cast<__nv_bfloat16 *>(out), static_cast<const __nv_bfloat16 *>(z), norm_w, eps,
                         lengths, B, Nv, S, Dv, s);
+    if (dt == GDR_F16)
+        return launch_t(static_cast<__half *>(out), static_cast<const __half *>(z), norm_w, eps, lengths, B, Nv, S,
+                        Dv, s);
     return launch_t(static_cast<float *>(out), static_cast<const float *>(z), norm_w, eps, lengths, B, Nv, S, Dv, s);
 }
 

@@ -56,7 +56,7 @@ EncodeTiledFn tensor_map_encoder();
 
 cudaError_t launch_decode(const DecodeArgs &a, int Dk, int Dv, gdr_dtype dt, gdr_dtype st, cudaStream_t s);
 bool chunk_tc_supported(int Dk, int Dv, gdr_dtype dt, int S);
-cudaError_t launch_chunk_tc(const ChunkArgs &a, cudaStream_t s);
+cudaError_t launch_chunk_tc(const ChunkArgs &a, gdr_dtype dt, cudaStream_t s);
 cudaError_t launch_chunk_simt(const ChunkArgs &a, int Dk, int Dv, gdr_dtype dt, cudaStream_t s);
 // out rows t < L_b <- rmsnorm(out row) * norm_w * silu(z row), in place (the unfused epilogue)
 cudaError_t launch_gated_rmsnorm(void *out, const void *z, const float *norm_w, float eps, const int32_t *lengths,

@@ -67,6 +67,9 @@ cudaError_t launch_prologue(const void *q, const void *k, const void *b, const f
     if (dt == GDR_BF16)
         return launch_prologue_t<__nv_bfloat16>(q, k, b, a, A_log, dt_bias, eps, B, Nk, Nv, S, Dk, q_hat, k_hat,
                                                 beta, g, stream);
+    if (dt == GDR_F16)
+        return launch_prologue_t<__half>(q, k, b, a, A_log, dt_bias, eps, B, Nk, Nv, S, Dk, q_hat, k_hat, beta, g,
+                                         stream);
     return launch_prologue_t<float>(q, k, b, a, A_log, dt_bias, eps, B, Nk, Nv, S, Dk, q_hat, k_hat, beta, g,
                                     stream);
 }

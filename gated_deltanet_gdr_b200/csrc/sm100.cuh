@@ -201,9 +201,14 @@ __device__ __forceinline__ void mma_commit(uint64_t *bar) {
 // Instruction descriptor, kind::f16: bf16 A and B, fp32 D, dense.
 //   [4,6) D format (1 = f32), [7,10) A format (1 = bf16), [10,13) B format (1 = bf16),
 //   [15] A major (0 = K, 1 = MN), [16] B major, [17,23) N >> 3, [24,29) M >> 4.
-__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn_major, bool b_mn_major) {
-    return (1u << 4) | (1u << 7) | (1u << 10) | ((a_mn_major ? 1u : 0u) << 15) | ((b_mn_major ? 1u : 0u) << 16) |
+// kind::f16 instruction descriptor: fp32 accumulator, A and B of operand format fmt (0 = fp16, 1 = bf16; both the
+// same), K-major unless *_mn_major
+__host__ __device__ constexpr uint32_t idesc_f16kind(int M, int N, bool a_mn_major, bool b_mn_major, uint32_t fmt) {
+    return (1u << 4) | (fmt << 7) | (fmt << 10) | ((a_mn_major ? 1u : 0u) << 15) | ((b_mn_major ? 1u : 0u) << 16) |
            ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn_major, bool b_mn_major) {
+    return idesc_f16kind(M, N, a_mn_major, b_mn_major, 1u);
 }
 
 // Instruction descriptor, kind::tf32: tf32 A and B (format 2), fp32 D, dense; `negate_a` negates A.

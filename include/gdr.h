@@ -27,8 +27,13 @@
  *       state_pool     (slots, Nv, Dk, Dv)
  *   - Grouped heads: Nv must be a multiple of Nk; value head h reads key head
  *     h / (Nv / Nk) (contiguous groups, the repeat_interleave grouping).
- *   - dtype names the type of q, k, v, beta, the state and out: GDR_F32 or
- *     GDR_BF16.  g, gk and the prologue's a, A_log, dt_bias are always fp32.
+ *   - dtype names the type of q, k, v, beta, the state and out: GDR_F32,
+ *     GDR_BF16 or GDR_F16 (the chunk_gated_delta_rule operator lists fp16 and
+ *     bf16 inputs).  g, gk and the prologue's a, A_log, dt_bias are always fp32.
+ *     bf16 prefill with Dk = Dv = 128 runs on the tensor cores; fp16 and fp32
+ *     prefill run the CUDA-core kernel (fp32 arithmetic, one rounding of each
+ *     output), fp16 decode the general decode kernel with an fp16 or fp32
+ *     state (an fp16 state needs fp16 inputs; other pairs: GDR_ERR_DTYPE).
  *     Index arrays are int32.  Stores to bf16 round to nearest even, once.
  *   - The caller owns every buffer.  The library allocates no device memory
  *     and keeps no pointer after a call returns.  Work is enqueued on
@@ -71,7 +76,7 @@ typedef enum gdr_status {
     GDR_ERR_LAUNCH = 7       /* a kernel launch or a CUDA call failed */
 } gdr_status;
 
-typedef enum gdr_dtype { GDR_F32 = 0, GDR_BF16 = 1 } gdr_dtype;
+typedef enum gdr_dtype { GDR_F32 = 0, GDR_BF16 = 1, GDR_F16 = 2 } gdr_dtype;
 
 /* Bits of the device error word (gdr_get_error). */
 #define GDR_DEVERR_SLOT_INDEX 0x1u /* a referenced slot index was outside [0, slots) */

@@ -16,11 +16,17 @@ import oracle
 
 # Tolerances of the parity bar: fp32 inputs, max-abs <= 1e-4 on out and state;
 # bf16 inputs and state, rel-L2 <= 2e-2 per tensor against the fp64 oracle fed the
-# same bf16-rounded inputs.
+# same bf16-rounded inputs.  fp16 (not fixed by the pages): rel-L2 <= 2e-3, derived from
+# the arithmetic -- the fp16 paths compute in fp32 from the rounded inputs the oracle also
+# sees; the CUDA-core kernels round each output once to fp16 (2^-11 relative) and the
+# tensor-core prefill also rounds its MMA operand copies (T, W, the state, v_new, P) to fp16,
+# the same number of roundings at which its bf16 (2^-9) twin stays near 3e-3, i.e. near
+# 8e-4 for fp16.
 F32_MAX_ABS = 1e-4
 BF16_REL_L2 = 2e-2
+F16_REL_L2 = 2e-3
 
-TORCH_DT = {"f32": torch.float32, "bf16": torch.bfloat16}
+TORCH_DT = {"f32": torch.float32, "bf16": torch.bfloat16, "f16": torch.float16}
 
 
 def rnd(x, dt: str) -> np.ndarray:
@@ -72,7 +78,8 @@ def assert_close(x, ref, dt: str, what: str):
         assert err <= F32_MAX_ABS, f"{what}: max-abs {err:.3e} > {F32_MAX_ABS}"
     else:
         err = rel_l2(x, ref)
-        assert err <= BF16_REL_L2, f"{what}: rel-L2 {err:.3e} > {BF16_REL_L2}"
+        bar = F16_REL_L2 if dt == "f16" else BF16_REL_L2
+        assert err <= bar, f"{what}: rel-L2 {err:.3e} > {bar}"
     return err
 
 

@@ -107,6 +107,8 @@ def test_decode_host_validation(L):
     assert decode(L, lens=NUL) == gdr.GDR_ERR_NULL
     assert decode(L, gk=ctypes.c_void_p(4100)) == gdr.GDR_ERR_ALIGN
     assert decode(L, Dk=48) == gdr.GDR_ERR_UNSUPPORTED
+    assert decode(L, dt=gdr.GDR_F16, sdt=gdr.GDR_BF16) == gdr.GDR_ERR_DTYPE  # fp16 inputs: fp16 or fp32 state
+    assert decode(L, dt=gdr.GDR_BF16, sdt=gdr.GDR_F16) == gdr.GDR_ERR_DTYPE  # an fp16 state needs fp16 inputs
     epi = gdr.GdrEpilogueStruct(4096, None, 1e-6)
     assert decode(L, epi=ctypes.byref(epi)) == gdr.GDR_ERR_NULL
     epi = gdr.GdrEpilogueStruct(4096, 4096, float("nan"))
@@ -159,7 +161,8 @@ def test_binding_rejects_host_tensors_and_bad_dtypes():
     q = torch.zeros(1, 1, 4, 16)
     with pytest.raises(RuntimeError):
         gdr.chunk_fwd(q, q, q, torch.zeros(1, 1, 4))
+    assert gdr._dtype_code(torch.float16) == gdr.GDR_F16
     with pytest.raises(RuntimeError):
-        gdr._dtype_code(torch.float16)
+        gdr._dtype_code(torch.float64)
     with pytest.raises(ValueError):
         gdr.chunk_fwd(torch.zeros(4, 16), q, q, q)
