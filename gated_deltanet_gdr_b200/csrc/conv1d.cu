@@ -138,55 +138,73 @@ __global__ void __launch_bounds__(kThreads, min_blocks(K)) conv1d_kernel(const C
     int row;
     T *op = out_base<T>(a, b, c0, row);
 
-    float w[K][V], bs[V];
+    // taps, bias and the window as channel pairs (f32x2 arithmetic)
+    constexpr int V2 = V / 2;
+    f2_t w2[K][V2], b2[V2];
 #pragma unroll
-    for (int i = 0; i < V; ++i) {
-        bs[i] = a.bias ? to_f32(static_cast<const T *>(a.bias)[c0 + i]) : 0.f;
+    for (int p = 0; p < V2; ++p) {
+        const T *b_ = static_cast<const T *>(a.bias);
+        b2[p] = pk2(b_ ? to_f32(b_[c0 + 2 * p]) : 0.f, b_ ? to_f32(b_[c0 + 2 * p + 1]) : 0.f);
 #pragma unroll
-        for (int j = 0; j < K; ++j) w[j][i] = to_f32(static_cast<const T *>(a.w)[(size_t)(c0 + i) * K + j]);
+        for (int j = 0; j < K; ++j)
+            w2[j][p] = pk2(to_f32(static_cast<const T *>(a.w)[(size_t)(c0 + 2 * p) * K + j]),
+                           to_f32(static_cast<const T *>(a.w)[(size_t)(c0 + 2 * p + 1) * K + j]));
     }
     // window: win[j] holds position t - K + 1 + j for the step at t; the K - 1 positions before the tile
-    float win[K][V];
+    f2_t win[K][V2];
 #pragma unroll
     for (int j = 0; j < K - 1; ++j)
 #pragma unroll
-        for (int i = 0; i < V; ++i)  // history index = position + K
-            win[j][i] = t0 < L ? hist_at<T, K>(a, b, c0 + i, t0 + 1 + j) : 0.f;
+        for (int p = 0; p < V2; ++p)  // history index = position + K
+            win[j][p] = t0 < L ? pk2(hist_at<T, K>(a, b, c0 + 2 * p, t0 + 1 + j),
+                                     hist_at<T, K>(a, b, c0 + 2 * p + 1, t0 + 1 + j))
+                               : pk2(0.f, 0.f);
 
     using Raw = typename ConvV<T>::Raw;
-    const Raw *xp = reinterpret_cast<const Raw *>(static_cast<const T *>(a.x) + (size_t)b * a.S * a.C + c0);
-    const size_t xstep = (size_t)a.C * sizeof(T) / sizeof(Raw);  // one time step, in access units
-    const int tl = min(t1, L);                           // valid steps of this tile end here
-    for (int tb = t0; tb < t1; tb += kBatch) {
+    const unsigned xstep = (unsigned)((size_t)a.C * sizeof(T) / sizeof(Raw));  // one time step, in access units
+    const Raw *xq = reinterpret_cast<const Raw *>(static_cast<const T *>(a.x) + ((size_t)b * a.S + t0) * a.C + c0);
+    T *oq = op + (size_t)t0 * row;
+    const int nv = min(t1, L) - t0;  // valid steps of this tile (may be <= 0)
+    const int nt = t1 - t0;          // steps of this tile
+    // (unrolling the whole tile, so that the window shifts become register renames, measured slower: the
+    // batch loop stays rolled)
+#pragma unroll 1
+    for (int tb = 0; tb < kTile; tb += kBatch) {
+        if (tb >= nt) break;
         // the batch's inputs first (read-only path, so they need not wait for this thread's earlier stores)
         Raw raw[kBatch];
 #pragma unroll
-        for (int u = 0; u < kBatch; ++u)
-            raw[u] = tb + u < tl ? __ldg(xp + (size_t)(tb + u) * xstep) : ConvV<T>::zero();
+        for (int u = 0; u < kBatch; ++u) raw[u] = tb + u < nv ? __ldg(xq + u * xstep) : ConvV<T>::zero();
 #pragma unroll
         for (int u = 0; u < kBatch; ++u) {
-            const int t = tb + u;
-            if (t >= t1) break;
+            if (tb + u >= nt) break;
             float y[V];
-            if (t < L) {
-                ConvV<T>::unpack(raw[u], win[K - 1]);
+            if (tb + u < nv) {
+                float x[V];
+                ConvV<T>::unpack(raw[u], x);
 #pragma unroll
-                for (int i = 0; i < V; ++i) {
-                    float acc = bs[i];
+                for (int p = 0; p < V2; ++p) win[K - 1][p] = pk2(x[2 * p], x[2 * p + 1]);
 #pragma unroll
-                    for (int j = 0; j < K; ++j) acc = fmaf(w[j][i], win[j][i], acc);
-                    y[i] = silu_fast(acc);
+                for (int p = 0; p < V2; ++p) {
+                    f2_t acc = b2[p];
+#pragma unroll
+                    for (int j = 0; j < K; ++j) acc = fma2(w2[j][p], win[j][p], acc);
+                    up2(acc, y[2 * p], y[2 * p + 1]);
                 }
+#pragma unroll
+                for (int i = 0; i < V; ++i) y[i] = silu_fast(y[i]);
 #pragma unroll
                 for (int j = 0; j < K - 1; ++j)
 #pragma unroll
-                    for (int i = 0; i < V; ++i) win[j][i] = win[j + 1][i];
+                    for (int p = 0; p < V2; ++p) win[j][p] = win[j + 1][p];
             } else {
 #pragma unroll
                 for (int i = 0; i < V; ++i) y[i] = 0.f;
             }
-            ConvV<T>::store(op + (size_t)t * row, y);
+            ConvV<T>::store(oq + u * row, y);
         }
+        xq += kBatch * xstep;
+        oq += kBatch * row;
     }
     if (state_here && a.state_out && Lr >= 0) write_state<T, K, V>(a, b, c0, L);
 }

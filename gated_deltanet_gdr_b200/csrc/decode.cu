@@ -35,25 +35,6 @@ namespace {
 
 constexpr int T = kDecodeMaxTokens;
 
-// packed fp32 pairs (sm_100 f32x2 arithmetic): one instruction updates two state columns
-typedef unsigned long long f2_t;
-__device__ __forceinline__ f2_t pk2(float lo, float hi) {
-    f2_t d;
-    asm("mov.b64 %0, {%1, %2};" : "=l"(d) : "f"(lo), "f"(hi));
-    return d;
-}
-__device__ __forceinline__ void up2(f2_t v, float &lo, float &hi) { asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v)); }
-__device__ __forceinline__ f2_t mul2(f2_t a, f2_t b) {
-    f2_t d;
-    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-    return d;
-}
-__device__ __forceinline__ f2_t fma2(f2_t a, f2_t b, f2_t c) {
-    f2_t d;
-    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
-    return d;
-}
-
 // explicit shared-memory loads (32-bit shared addresses), so that every operand read of the decode loop
 // is a shared-memory access
 __device__ __forceinline__ uint4 lds128(uint32_t a) {
