@@ -116,7 +116,7 @@ constexpr uint32_t OFF_A21 = 205824;  // A rows 32..63, columns 0..31 (plain, 32
 constexpr uint32_t OFF_XM = 210432;   // X = A21 T11 of the 32 -> 64 merge (plain, 32 rows of SP floats)
 static_assert(OFF_XP + 32 * SP * 4 <= OFF_TT + 16384, "plain A and the merge scratch fit in the TT area");
 static_assert(OFF_TP + 64 * SP * 4 <= OFF_A21 && OFF_A21 + 32 * SP * 4 <= OFF_XM, "plain T, A21");
-constexpr int NVEC = 12;             // per-chunk vectors of 64 floats (enum below)
+constexpr int NVEC = 11;             // per-chunk vectors of 64 floats (enum below)
 constexpr uint32_t OFF_VEC = 215040;  // 2 sets x NVEC vectors x 64 floats
 static_assert(OFF_XM + 32 * SP * 4 <= OFF_VEC, "merge product");
 constexpr uint32_t OFF_BAR = OFF_VEC + 2 * NVEC * 64 * 4;
@@ -135,7 +135,7 @@ constexpr uint32_t TM_GPW = 0, TM_U = 128, TM_R = 256, TM_S = 384, TM_COLS = 512
 // V_G2 = G log2(e); V_LAM = V_G2 - log2(1/|k|), so that e^{G_t - G_s} / |k_s| = 2^{V_G2[t] - V_LAM[s]};
 // V_XS = e^G scale / |q| (row factor of Q S); V_N holds the chunk's valid-token count in its first entry.
 // V_ET = e^{G_last - G}; V_TAIL = V_ET / |k|.
-enum { V_BETA = 0, V_GAM, V_EG, V_TAIL, V_RK, V_RQ, V_CW, V_G2, V_LAM, V_XS, V_ET, V_N };
+enum { V_BETA = 0, V_EG, V_TAIL, V_RK, V_RQ, V_CW, V_G2, V_LAM, V_XS, V_ET, V_N };
 static_assert(V_N < NVEC, "vector slots");
 
 struct TcArgs {
@@ -504,7 +504,6 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             for (int i = 0; i < 2; ++i) {
                 const int tt = 2 * lane + i;
                 vec[V_BETA * 64 + tt] = bv[i];
-                vec[V_GAM * 64 + tt] = G[i];
                 vec[V_EG * 64 + tt] = __expf(G[i]);
                 vec[V_G2 * 64 + tt] = G[i] * 1.4426950408889634f;
                 vec[V_ET * 64 + tt] = __expf(gl - G[i]);

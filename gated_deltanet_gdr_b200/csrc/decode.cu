@@ -55,11 +55,6 @@ __device__ __forceinline__ float lds_bf16(uint32_t a) {
 template <typename T> __device__ __forceinline__ float lds_elem(uint32_t a);
 template <> __device__ __forceinline__ float lds_elem<float>(uint32_t a) { return lds_f32(a); }
 template <> __device__ __forceinline__ float lds_elem<__nv_bfloat16>(uint32_t a) { return lds_bf16(a); }
-__device__ __forceinline__ int lds_s32(uint32_t a) {
-    int v;
-    asm volatile("ld.shared.s32 %0, [%1];" : "=r"(v) : "r"(a));
-    return v;
-}
 
 // 2^x on the special-function unit (PTX ex2.approx.ftz.f32)
 __device__ __forceinline__ float exp2f_approx(float x) {

@@ -182,39 +182,22 @@ __device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a_desc, uint6
         "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
         : "memory");
 }
-// D[tmem] (+)= A[smem] * B[smem], kind::tf32 (fp32 operands read as tf32, fp32 accumulate), one CTA.
-__device__ __forceinline__ void mma_tf32(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
-                                         uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
 // Arrive (once) on an mbarrier when all previously issued tcgen05.mma of this thread complete.
 __device__ __forceinline__ void mma_commit(uint64_t *bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
                  : "memory");
 }
 
-// Instruction descriptor, kind::f16: bf16 A and B, fp32 D, dense.
-//   [4,6) D format (1 = f32), [7,10) A format (1 = bf16), [10,13) B format (1 = bf16),
-//   [15] A major (0 = K, 1 = MN), [16] B major, [17,23) N >> 3, [24,29) M >> 4.
-// kind::f16 instruction descriptor: fp32 accumulator, A and B of operand format fmt (0 = fp16, 1 = bf16; both the
-// same), K-major unless *_mn_major
+// Instruction descriptor, kind::f16: fp32 D, A and B of operand format fmt (0 = fp16, 1 = bf16; both the same),
+// dense, K-major unless *_mn_major.
+//   [4,6) D format (1 = f32), [7,10) A format, [10,13) B format, [15] A major (0 = K, 1 = MN), [16] B major,
+//   [17,23) N >> 3, [24,29) M >> 4.
 __host__ __device__ constexpr uint32_t idesc_f16kind(int M, int N, bool a_mn_major, bool b_mn_major, uint32_t fmt) {
     return (1u << 4) | (fmt << 7) | (fmt << 10) | ((a_mn_major ? 1u : 0u) << 15) | ((b_mn_major ? 1u : 0u) << 16) |
            ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn_major, bool b_mn_major) {
     return idesc_f16kind(M, N, a_mn_major, b_mn_major, 1u);
-}
-
-// Instruction descriptor, kind::tf32: tf32 A and B (format 2), fp32 D, dense; `negate_a` negates A.
-__host__ __device__ constexpr uint32_t idesc_tf32(int M, int N, bool a_mn_major, bool b_mn_major, bool negate_a) {
-    return (1u << 4) | (2u << 7) | (2u << 10) | ((negate_a ? 1u : 0u) << 13) | ((a_mn_major ? 1u : 0u) << 15) |
-           ((b_mn_major ? 1u : 0u) << 16) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
 // Shared-memory matrix descriptor for a 128-byte-swizzled canonical layout.
@@ -231,20 +214,6 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t smem_addr, uint32_t lbo
     d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
     d |= (uint64_t)1u << 46;
     d |= (uint64_t)2u << 61;
-    return d;
-}
-
-// Shared-memory matrix descriptor for the MN-major kind::tf32 operand layout: 128-byte rows along MN
-// (32 fp32), groups of 4 K-rows (512 bytes) every `sbo` bytes, 32-byte granules XORed with the row index
-// modulo 4 (layout type 1, "128-byte swizzle with 32-byte atoms"; the plain 128-byte swizzle is not valid
-// for an MN-major tf32 operand).
-__device__ __forceinline__ uint64_t sdesc_sw128_32b(uint32_t smem_addr, uint32_t sbo) {
-    uint64_t d = 0;
-    d |= (uint64_t)((smem_addr >> 4) & 0x3FFFu);
-    d |= (uint64_t)((8192u >> 4) & 0x3FFFu) << 16;
-    d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
-    d |= (uint64_t)1u << 46;
-    d |= (uint64_t)1u << 61;
     return d;
 }
 
