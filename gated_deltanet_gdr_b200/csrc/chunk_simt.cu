@@ -212,7 +212,8 @@ static cudaError_t launch_simt_t(const ChunkArgs &a, int DV, cudaStream_t stream
     const long long blocks = (long long)a.B * a.Nv * (DV / VC);
     if (blocks == 0) return cudaSuccess;
     auto kern = chunk_simt_kernel<DK, VC, TI>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Ly::bytes);
+    static LaunchCache cache(reinterpret_cast<const void *>(kern));
+    cudaError_t e = cache.allow_smem((int)Ly::bytes);
     if (e != cudaSuccess) return e;
     kern<<<(unsigned)blocks, 256, Ly::bytes, stream>>>(a, DV);
     return cudaGetLastError();

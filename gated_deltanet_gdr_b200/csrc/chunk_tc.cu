@@ -1111,13 +1111,9 @@ cudaError_t launch_tc_t(const ChunkArgs &ca, cudaStream_t stream) {
     a.l2norm = ca.l2norm; a.eps = ca.eps; a.beta_logits = ca.beta_logits; a.A_log = ca.A_log;
     a.dt_bias = ca.dt_bias; a.err = ca.err;
     a.epi_z = ca.epi_z; a.epi_w = ca.epi_w; a.epi_eps = ca.epi_eps;
-    static bool attr_set = false;  // one per element type
-    if (!attr_set) {
-        cudaError_t e =
-            cudaFuncSetAttribute(chunk_tc_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
-        if (e != cudaSuccess) return e;
-        attr_set = true;
-    }
+    static LaunchCache cache(reinterpret_cast<const void *>(chunk_tc_kernel<T>));
+    cudaError_t e = cache.allow_smem((int)SMEM_BYTES);
+    if (e != cudaSuccess) return e;
     const long long blocks = (long long)ca.B * ca.Nv;
     if (blocks == 0) return cudaSuccess;
     chunk_tc_kernel<T><<<(unsigned)blocks, NT, SMEM_BYTES, stream>>>(mq, mk, mv, mo, a);

@@ -746,20 +746,12 @@ cudaError_t launch_decode128(const DecodeArgs &a, cudaStream_t stream) {
         return cudaErrorInvalidValue;
     auto kern = decode128_kernel<TI, TS, NW, NSTG, MINB>;
     const int smem = Cf::layout(a.S, a.gk != nullptr).smem;
-    static int attr_smem = 0, cached_smem = -1, grid_cap = 1;
-    if (smem > attr_smem) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-        if (e != cudaSuccess) return e;
-        attr_smem = smem;
-    }
-    if (smem != cached_smem) {
-        int dev = 0, nsm = 0, per_sm = 0;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, Cf::NT, smem);
-        grid_cap = max(1, nsm * max(1, per_sm));
-        cached_smem = smem;
-    }
+    static LaunchCache cache(reinterpret_cast<const void *>(kern));
+    cudaError_t e = cache.allow_smem(smem);
+    if (e != cudaSuccess) return e;
+    int grid_cap = 1;
+    e = cache.resident_grid(Cf::NT, smem, &grid_cap);
+    if (e != cudaSuccess) return e;
     const int grid = (int)(ntiles < grid_cap ? ntiles : grid_cap);
     kern<<<grid, Cf::NT, smem, stream>>>(tm, a, (int)ntiles);
     return cudaGetLastError();
@@ -772,23 +764,14 @@ cudaError_t launch_decode_t(const DecodeArgs &a, cudaStream_t stream) {
     if (ntiles == 0) return cudaSuccess;
     auto kern = decode_kernel<DK, DV, TI, TS>;
     const int smem = Cf::layout(a.S, a.gk != nullptr).smem;
-    // resident CTAs on the device for this shared-memory size (all B200s have the same count),
-    // cached per instantiation and size; an overestimate would only queue extra CTAs, since
-    // tiles are independent
-    static int attr_smem = 0, cached_smem = -1, grid_cap = 1;
-    if (smem > attr_smem) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-        if (e != cudaSuccess) return e;
-        attr_smem = smem;
-    }
-    if (smem != cached_smem) {
-        int dev = 0, nsm = 0, per_sm = 0;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, Cf::NT, smem);
-        grid_cap = max(1, nsm * max(1, per_sm));
-        cached_smem = smem;
-    }
+    // a persistent grid of the CTAs resident at once for this shared-memory size (tiles are independent, so
+    // an overestimate would only queue extra CTAs)
+    static LaunchCache cache(reinterpret_cast<const void *>(kern));
+    cudaError_t e = cache.allow_smem(smem);
+    if (e != cudaSuccess) return e;
+    int grid_cap = 1;
+    e = cache.resident_grid(Cf::NT, smem, &grid_cap);
+    if (e != cudaSuccess) return e;
     const int grid = (int)(ntiles < grid_cap ? ntiles : grid_cap);
     kern<<<grid, Cf::NT, smem, stream>>>(a, (int)ntiles);
     return cudaGetLastError();

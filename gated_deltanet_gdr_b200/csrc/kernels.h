@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <mutex>
+
 #include "../../include/gdr.h"
 
 namespace gdr {
@@ -53,6 +55,26 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t
                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 EncodeTiledFn tensor_map_encoder();
+
+// Launch facts of one kernel, kept per device: the dynamic shared-memory size its attribute allows, and the number
+// of CTAs resident at once for a block shape.  Function attributes and occupancy belong to a device, so a process
+// that drives several devices sets and asks them on each; the record is guarded for use from several host threads.
+class LaunchCache {
+  public:
+    explicit LaunchCache(const void *func) : func_(func) {}
+    // make `smem` bytes of dynamic shared memory launchable on the current device
+    cudaError_t allow_smem(int smem);
+    // CTAs of `threads` threads with `smem` bytes that the current device holds at once (at least 1)
+    cudaError_t resident_grid(int threads, int smem, int *grid);
+
+  private:
+    static constexpr int kMaxDevices = 64;  // devices past this count are served without a record
+    const void *func_;
+    std::mutex mu_;
+    int smem_[kMaxDevices] = {};
+    int grid_key_[kMaxDevices] = {};  // (threads << 20) | smem of the recorded grid, 0 = none
+    int grid_[kMaxDevices] = {};
+};
 
 cudaError_t launch_decode(const DecodeArgs &a, int Dk, int Dv, gdr_dtype dt, gdr_dtype st, cudaStream_t s);
 bool chunk_tc_supported(int Dk, int Dv, gdr_dtype dt, int S);
