@@ -28,7 +28,7 @@ LIB_PATH = os.path.join(_PKG, "libgdr.so")
 GDR_OK, GDR_ERR_SHAPE, GDR_ERR_DTYPE, GDR_ERR_NULL, GDR_ERR_ALIGN, GDR_ERR_UNSUPPORTED, GDR_ERR_DEVICE, \
     GDR_ERR_LAUNCH = range(8)
 GDR_F32, GDR_BF16, GDR_F16 = 0, 1, 2
-DEVERR_SLOT_INDEX, DEVERR_LENGTH = 0x1, 0x2
+DEVERR_SLOT_INDEX, DEVERR_LENGTH, DEVERR_TIMEOUT = 0x1, 0x2, 0x4
 
 # Every symbol the C header declares (checked by the ABI test).
 EXPORTED = ("gdr_chunk_fwd", "gdr_recurrent_step", "gdr_recurrent_step_spec", "gdr_conv1d", "gdr_prologue_apply",

@@ -83,7 +83,6 @@ constexpr int CTL_WARP = 16;
 // BAR_PCTL: the prep warps and the control warp, at the hand-offs between them; BAR_HELP: the helper warps
 // BAR_EPI: the carry warps that hold o rows (TMEM lanes 64..127), at the epilogue's row-norm exchange
 constexpr int BAR_CARRY = 1, BAR_PREP = 2, BAR_PCTL = 3, BAR_HELP = 4, BAR_EPI = 5;
-constexpr uint32_t kTimeoutBit = 0x4u;
 // carry thread that issues the out-tile TMA stores (thread 0 issues the carry's MMAs)
 constexpr int kStorer = 32;
 
@@ -1060,7 +1059,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     }
     tc_fence_before();
     __syncthreads();
-    if (tid == 0 && *s_abort) raise_device_error(a.err, kTimeoutBit);
+    if (tid == 0 && *s_abort) raise_device_error(a.err, GDR_DEVERR_TIMEOUT);
 #ifdef GDR_PHASE_TIMERS
     if (blockIdx.x == 0 && tid < 64) g_phase[tid] += s_phase_[tid];
 #endif

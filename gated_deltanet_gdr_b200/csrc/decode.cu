@@ -721,7 +721,7 @@ decode128_kernel(const __grid_constant__ CUtensorMap tm_pool, const DecodeArgs a
             if (nxt + 3 * (int)gridDim.x < ntiles) prefetch_meta128<TI>(a, nxt + 3 * gridDim.x, tid, pre2);
         }
     }
-    if (timed_out && tid == 0) raise_device_error(a.err, 0x4u);
+    if (timed_out && tid == 0) raise_device_error(a.err, GDR_DEVERR_TIMEOUT);
 }
 
 template <typename TI, typename TS>

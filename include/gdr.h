@@ -30,10 +30,12 @@
  *   - dtype names the type of q, k, v, beta, the state and out: GDR_F32,
  *     GDR_BF16 or GDR_F16 (the chunk_gated_delta_rule operator lists fp16 and
  *     bf16 inputs).  g, gk and the prologue's a, A_log, dt_bias are always fp32.
- *     bf16 prefill with Dk = Dv = 128 runs on the tensor cores; fp16 and fp32
- *     prefill run the CUDA-core kernel (fp32 arithmetic, one rounding of each
- *     output), fp16 decode the general decode kernel with an fp16 or fp32
- *     state (an fp16 state needs fp16 inputs; other pairs: GDR_ERR_DTYPE).
+ *     bf16 and fp16 prefill with Dk = Dv = 128 run on the tensor cores (fp32
+ *     accumulation and state, MMA operand copies in the input type); other
+ *     head sizes and fp32 run the CUDA-core kernel (fp32 arithmetic, one
+ *     rounding of each output).  Decode takes a state of GDR_F32, GDR_BF16 or
+ *     GDR_F16 (an fp16 state needs fp16 inputs, fp16 inputs an fp16 or fp32
+ *     state; other pairs: GDR_ERR_DTYPE).
  *     Index arrays are int32.  Stores to bf16 round to nearest even, once.
  *   - The caller owns every buffer.  The library allocates no device memory
  *     and keeps no pointer after a call returns.  Work is enqueued on
@@ -81,6 +83,9 @@ typedef enum gdr_dtype { GDR_F32 = 0, GDR_BF16 = 1, GDR_F16 = 2 } gdr_dtype;
 /* Bits of the device error word (gdr_get_error). */
 #define GDR_DEVERR_SLOT_INDEX 0x1u /* a referenced slot index was outside [0, slots) */
 #define GDR_DEVERR_LENGTH 0x2u     /* a length was outside [0, S] */
+#define GDR_DEVERR_TIMEOUT 0x4u    /* a kernel's bounded wait for its own copies or for another of its warp
+                                      groups ran out: it released what it held and returned early, so the
+                                      call's outputs are incomplete (not expected in normal operation) */
 
 /*
  * Optional fused prologue (the layer's pre-processing, computed in fp32
@@ -114,10 +119,10 @@ typedef struct gdr_prologue {
  * With it, out row (b, h, t) for t < L_b holds, computed in fp32 and rounded
  * once to dtype:
  *     o / sqrt(mean_j o_j^2 + eps) * norm_w * silu(z),  silu(x) = x / (1 + e^{-x})
- * where o is the row the rule produces; padding rows stay zero.  The bf16
- * tensor-core prefill applies it to the fp32 row before rounding; the other
- * paths apply it to the row already stored in dtype (for bf16 that rounds o
- * once more, within the bf16 tolerance).  z and norm_w must be 16-byte aligned.
+ * where o is the row the rule produces; padding rows stay zero.  The
+ * tensor-core prefill (bf16 or fp16, Dk = Dv = 128) applies it to the fp32 row
+ * before rounding; the other paths apply it to the row already stored in
+ * dtype (for a 16-bit dtype that rounds o once more, within its tolerance).  z and norm_w must be 16-byte aligned.
  */
 typedef struct gdr_epilogue {
     const void *z;
@@ -149,8 +154,9 @@ typedef struct gdr_epilogue {
  *                          may alias initial_state (in-place update).
  * Constraints: B, S >= 0; Nk, Nv >= 1; Nv % Nk == 0; Dk, Dv in {16,32,64,128};
  * every pointer 16-byte aligned.  An epilogue with a NULL z or norm_w returns
- * GDR_ERR_NULL, one with eps < 0 (or NaN) GDR_ERR_SHAPE.  bf16 with Dk = Dv = 128 runs on the
- * tensor-core (tcgen05) path; other shapes and fp32 run the CUDA-core path.
+ * GDR_ERR_NULL, one with eps < 0 (or NaN) GDR_ERR_SHAPE.  bf16 or fp16 with
+ * Dk = Dv = 128 runs on the tensor-core (tcgen05) path; other shapes and fp32
+ * run the CUDA-core path.
  */
 int gdr_chunk_fwd(const void *q, const void *k, const void *v, const void *beta, const float *g,
                   const void *initial_state, const int32_t *actual_seq_lengths, float scale, int B, int Nk,
@@ -185,7 +191,7 @@ int gdr_chunk_fwd(const void *q, const void *k, const void *v, const void *beta,
  * must not reference the same slot (their updates would race).
  * Constraints: 1 <= S <= 8 (the operator is decode-only), slots >= 1, other
  * constraints as for gdr_chunk_fwd.  state_dtype may be GDR_F32 or GDR_BF16
- * independently of dtype.
+ * with GDR_F32 or GDR_BF16 inputs; fp16 inputs take GDR_F16 or GDR_F32.
  */
 int gdr_recurrent_step(const void *q, const void *k, const void *v, const void *beta, const float *g,
                        const float *gk, void *state_pool, int slots, const int32_t *ssm_state_indices,
@@ -239,8 +245,8 @@ int gdr_recurrent_step_spec(const void *q, const void *k, const void *v, const v
  *   conv_state_out       device (B, C, K) or NULL: the last K inputs of the history
  *                        (conv_state_in followed by x[0..L_b-1]); it may alias
  *                        conv_state_in (the in-place update of decode)
- * x, weight, bias, the states and the outputs are in dtype (GDR_F32 or
- * GDR_BF16).  Constraints: B, S >= 0; Nk, Nv >= 1; Dk, Dv in {16,32,64,128};
+ * x, weight, bias, the states and the outputs are in dtype (GDR_F32,
+ * GDR_BF16 or GDR_F16).  Constraints: B, S >= 0; Nk, Nv >= 1; Dk, Dv in {16,32,64,128};
  * 1 <= K <= 8 (4 in the layer); every pointer 16-byte aligned.  A length
  * outside [0, S] skips the sequence (outputs zero, state untouched) and sets
  * GDR_DEVERR_LENGTH.

@@ -37,6 +37,19 @@ def test_exports_every_declared_symbol(L):
         assert hasattr(L, n), f"libgdr.so does not export {n}"
 
 
+def test_header_codes_match_the_binding():
+    """The status codes, dtype codes and device error bits the header defines are the values the Python
+    binding uses."""
+    src = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    enums = dict((n, int(v)) for n, v in re.findall(r"\b(GDR_[A-Z0-9_]+)\s*=\s*(\d+)", src))
+    defines = dict((n, int(v, 16)) for n, v in re.findall(r"#define\s+(GDR_DEVERR_[A-Z_]+)\s+(0x[0-9a-fA-F]+)u", src))
+    for name in ("GDR_OK", "GDR_ERR_SHAPE", "GDR_ERR_DTYPE", "GDR_ERR_NULL", "GDR_ERR_ALIGN", "GDR_ERR_UNSUPPORTED",
+                 "GDR_ERR_DEVICE", "GDR_ERR_LAUNCH", "GDR_F32", "GDR_BF16", "GDR_F16"):
+        assert enums[name] == getattr(gdr, name), name
+    assert defines == {"GDR_DEVERR_SLOT_INDEX": gdr.DEVERR_SLOT_INDEX, "GDR_DEVERR_LENGTH": gdr.DEVERR_LENGTH,
+                       "GDR_DEVERR_TIMEOUT": gdr.DEVERR_TIMEOUT}, defines
+
+
 def test_status_strings_and_version(L):
     for s in range(8):
         assert L.gdr_status_string(s)
