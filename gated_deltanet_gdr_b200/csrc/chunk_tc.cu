@@ -120,7 +120,10 @@ constexpr uint32_t OFF_VEC = 215040;  // 2 sets x NVEC vectors x 64 floats
 static_assert(OFF_XM + 32 * SP * 4 <= OFF_VEC, "merge product");
 constexpr uint32_t OFF_BAR = OFF_VEC + 2 * NVEC * 64 * 4;
 constexpr uint32_t OFF_EPI = OFF_BAR + 128;  // epilogue: partial squared norms of the o rows (2 x 64 floats)
-constexpr uint32_t SMEM_USED = OFF_EPI + 512;
+// the order of the chains (see order_chain): the B lengths, then the selected sequence
+constexpr int kRankMaxB = 1024;
+constexpr uint32_t OFF_LEN = OFF_EPI + 512;
+constexpr uint32_t SMEM_USED = OFF_LEN + kRankMaxB * 4 + 16;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;  // + alignment slack
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 static_assert(OFF_TT % 1024 == 0, "swizzle atoms");
@@ -316,6 +319,35 @@ __device__ __forceinline__ void solve_diag16_merge(const float *sA, float *sT, f
     named_sync(BAR_PREP, NGRP);
 }
 
+// The sequence a CTA runs, longest first.  A CTA holds an SM for its whole chain and CTAs start in index
+// order as SMs free up, so with more chains than SMs a long chain that starts late sets the end of the launch
+// (longest-processing-time-first list scheduling).  CTA i takes the sequence whose valid length ranks
+// i / Nv-th (longest first, ties by index; an invalid length counts as 0); its value head stays i % Nv.
+// Without lengths, or with more than kRankMaxB sequences, the order is the index order.  Called by all
+// threads of the CTA before anything else touches shared memory.
+__device__ __forceinline__ int order_chain(const TcArgs &a, int tid, uint8_t *sm) {
+    const int seq = blockIdx.x / a.Nv;
+    if (!a.lengths || a.B <= 1 || a.B > kRankMaxB) return seq;
+    int *s_len = reinterpret_cast<int *>(sm + OFF_LEN);
+    volatile int *s_sel = s_len + kRankMaxB;
+    for (int i = tid; i < a.B; i += NT) {
+        const int L = a.lengths[i];
+        s_len[i] = (L < 0 || L > a.S) ? 0 : L;
+    }
+    __syncthreads();
+    for (int i = tid; i < a.B; i += NT) {  // the ranks are a permutation of 0..B-1: one i matches
+        const int Li = s_len[i];
+        int r = 0;
+        for (int j = 0; j < a.B; ++j) {
+            const int Lj = s_len[j];
+            r += (Lj > Li) || (Lj == Li && j < i);
+        }
+        if (r == seq) *s_sel = i;
+    }
+    __syncthreads();
+    return *s_sel;
+}
+
 template <typename T>
 __global__ void __launch_bounds__(NT, 1)
 chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -343,7 +375,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, q4 = warp & 3, hf = (warp >> 2) & 1;
     const bool carry = warp < 8, control = warp == CTL_WARP, helper = warp > CTL_WARP;
-    const int bh = blockIdx.x, h = bh % a.Nv, b = bh / a.Nv, kh = h / (a.Nv / a.Nk);
+    const int h = blockIdx.x % a.Nv, b = order_chain(a, tid, sm), bh = b * a.Nv + h, kh = h / (a.Nv / a.Nk);
     const int S = a.S;
     int L = a.lengths ? a.lengths[b] : S;
     const bool bad_len = (L < 0 || L > S);
