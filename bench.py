@@ -313,6 +313,39 @@ def bench_prefill(gdr, args, world, rank, clk, flush, stream, peaks):
     return fields, w, t, pro, step
 
 
+def bench_varlen(gdr, args, world, rank, flush, stream, peaks):
+    """The variable-length prefill workload (B=8, padded S=8192, lengths ~ U[512, 8192] with one 0), fused
+    prologue; a parity-test configuration, timed only on request (--only varlen), not in the default line.
+    256 chains on 148 SMs: the kernel starts the longest sequences first."""
+    w = workloads.generate("varlen", seed=3 + 1000 * rank)
+    t = dict(q=bf16_dev(w.q), k=bf16_dev(w.k), v=bf16_dev(w.v), b=bf16_dev(w.b), a=f32_dev(w.a),
+             s0=bf16_dev(w.initial_state))
+    pro = gdr.Prologue(l2norm_qk=True, eps=1e-6, beta_logits=True, A_log=f32_dev(w.A_log),
+                       dt_bias=f32_dev(w.dt_bias))
+    lens = torch.from_numpy(w.lengths).cuda()
+    step = gdr.prepare_chunk_fwd(t["q"], t["k"], t["v"], t["b"], t["a"], t["s0"], lens, w.scale, prologue=pro)
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if gdr.get_error() != 0:
+        raise RuntimeError("device error word set during warm-up")
+    barrier(world)
+    torch.cuda.synchronize()
+    times = timed_steps(step, args.steps, flush, stream)
+    barrier(world)
+    ms = all_max(sum(times), world) / args.steps
+    tokens = int(w.lengths.sum())
+    nb = algorithmic_prefill_bytes(w)
+    achieved = nb / (ms / 1e3) / 1e9
+    return {"workload": f"varlen B={w.B} padded S={w.S} Nk={w.Nk} Nv={w.Nv} D={w.Dk} bf16, lengths "
+                        f"{w.lengths.tolist()}, fused prologue", "ms_per_step": ms,
+            "tokens_per_s": weak_scaling_rate(tokens, args.steps, ms * args.steps, world),
+            "l2": "inputs larger than L2, plus a 256 MiB flush before every timed step",
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": achieved / peaks["hbm_gbs"], "traffic": None, "algorithmic_bytes_per_launch": nb}}, \
+        args.steps
+
+
 def bench_prefill_epilogue(gdr, args, world, w, t, pro, flush, stream, peaks):
     """The same prefill call with the fused gated RMSNorm output epilogue (z and norm_w of the layer's
     output gate); returns (fields, launches)."""
@@ -569,6 +602,9 @@ def run_ours(args, world, rank, local):
             line["prefill_epilogue"], n = bench_prefill_epilogue(gdr, args, world, w, t, pro, flush, stream, peaks)
             launches += n
         del t
+    if args.only == "varlen":  # a parity-test configuration: timed on request only
+        line["varlen"], n = bench_varlen(gdr, args, world, rank, flush, stream, peaks)
+        launches += n
     if args.only in ("all", "conv1d"):
         line["conv1d"], n = bench_conv1d(gdr, args, world, rank, flush, stream, peaks)
         launches += n
@@ -605,9 +641,10 @@ def main():
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg (profiling runs)")
     ap.add_argument("--no-epilogue", action="store_true",
                     help="skip the prefill line with the fused gated RMSNorm epilogue (profiling runs)")
-    ap.add_argument("--only", choices=["all", "prefill", "decode", "decode_gk", "decode_spec", "conv1d", "f16"],
-                    default="all",
-                    help="run one workload only (profiling runs); the default runs all")
+    ap.add_argument("--only", choices=["all", "prefill", "decode", "decode_gk", "decode_spec", "conv1d", "f16",
+                                       "varlen"], default="all",
+                    help="run one workload only (profiling runs); the default runs all but varlen, a "
+                         "parity-test configuration timed on request")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

@@ -121,7 +121,7 @@ static_assert(OFF_XM + 32 * SP * 4 <= OFF_VEC, "merge product");
 constexpr uint32_t OFF_BAR = OFF_VEC + 2 * NVEC * 64 * 4;
 constexpr uint32_t OFF_EPI = OFF_BAR + 128;  // epilogue: partial squared norms of the o rows (2 x 64 floats)
 // the order of the chains (see order_chain): the B lengths, then the selected sequence
-constexpr int kRankMaxB = 1024;
+constexpr int kRankMaxB = 256;
 constexpr uint32_t OFF_LEN = OFF_EPI + 512;
 constexpr uint32_t SMEM_USED = OFF_LEN + kRankMaxB * 4 + 16;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;  // + alignment slack
@@ -324,7 +324,9 @@ __device__ __forceinline__ void solve_diag16_merge(const float *sA, float *sT, f
 // (longest-processing-time-first list scheduling).  CTA i takes the sequence whose valid length ranks
 // i / Nv-th (longest first, ties by index; an invalid length counts as 0); its value head stays i % Nv.
 // Without lengths, or with more than kRankMaxB sequences, the order is the index order.  Called by all
-// threads of the CTA before anything else touches shared memory.
+// threads of the CTA before anything else touches shared memory.  The kernel's ordered instantiation runs
+// it, and the host launches that one only when the chains outnumber the resident CTAs: its sequence index
+// lives in a register, where the index order's is recomputed from blockIdx, and in one wave order is moot.
 __device__ __forceinline__ int order_chain(const TcArgs &a, int tid, uint8_t *sm) {
     const int seq = blockIdx.x / a.Nv;
     if (!a.lengths || a.B <= 1 || a.B > kRankMaxB) return seq;
@@ -348,7 +350,7 @@ __device__ __forceinline__ int order_chain(const TcArgs &a, int tid, uint8_t *sm
     return *s_sel;
 }
 
-template <typename T>
+template <typename T, bool kOrdered>
 __global__ void __launch_bounds__(NT, 1)
 chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o, const TcArgs a) {
@@ -375,7 +377,9 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, q4 = warp & 3, hf = (warp >> 2) & 1;
     const bool carry = warp < 8, control = warp == CTL_WARP, helper = warp > CTL_WARP;
-    const int h = blockIdx.x % a.Nv, b = order_chain(a, tid, sm), bh = b * a.Nv + h, kh = h / (a.Nv / a.Nk);
+    const int h = blockIdx.x % a.Nv;
+    const int b = kOrdered ? order_chain(a, tid, sm) : (int)blockIdx.x / a.Nv;
+    const int bh = kOrdered ? b * a.Nv + h : (int)blockIdx.x, kh = h / (a.Nv / a.Nk);
     const int S = a.S;
     int L = a.lengths ? a.lengths[b] : S;
     const bool bad_len = (L < 0 || L > S);
@@ -1142,12 +1146,24 @@ cudaError_t launch_tc_t(const ChunkArgs &ca, cudaStream_t stream) {
     a.l2norm = ca.l2norm; a.eps = ca.eps; a.beta_logits = ca.beta_logits; a.A_log = ca.A_log;
     a.dt_bias = ca.dt_bias; a.err = ca.err;
     a.epi_z = ca.epi_z; a.epi_w = ca.epi_w; a.epi_eps = ca.epi_eps;
-    static LaunchCache cache(reinterpret_cast<const void *>(chunk_tc_kernel<T>));
-    cudaError_t e = cache.allow_smem((int)SMEM_BYTES);
-    if (e != cudaSuccess) return e;
+    static LaunchCache plain(reinterpret_cast<const void *>(chunk_tc_kernel<T, false>));
+    static LaunchCache ordered(reinterpret_cast<const void *>(chunk_tc_kernel<T, true>));
     const long long blocks = (long long)ca.B * ca.Nv;
     if (blocks == 0) return cudaSuccess;
-    chunk_tc_kernel<T><<<(unsigned)blocks, NT, SMEM_BYTES, stream>>>(mq, mk, mv, mo, a);
+    // longest sequences first only when the chains do not all start at once
+    bool order = false;
+    if (ca.lengths && ca.B > 1 && ca.B <= kRankMaxB) {
+        int resident = 0;
+        cudaError_t e = ordered.resident_grid(NT, (int)SMEM_BYTES, &resident);
+        if (e != cudaSuccess) return e;
+        order = blocks > resident;
+    }
+    cudaError_t e = (order ? ordered : plain).allow_smem((int)SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    if (order)
+        chunk_tc_kernel<T, true><<<(unsigned)blocks, NT, SMEM_BYTES, stream>>>(mq, mk, mv, mo, a);
+    else
+        chunk_tc_kernel<T, false><<<(unsigned)blocks, NT, SMEM_BYTES, stream>>>(mq, mk, mv, mo, a);
     return cudaGetLastError();
 }
 }  // namespace

@@ -129,6 +129,26 @@ def test_varlen_padding_zero_and_empty_sequence():
         assert np.array_equal(gf[0], ins["initial_state"][0])
 
 
+@pytest.mark.parametrize("dt", ["bf16", "f16"])
+def test_varlen_more_chains_than_sms_longest_first(dt):
+    """B = 40 sequences x Nv = 4 heads = 160 chains, more than the 148 SMs hold at once, so the tensor-core
+    kernel starts the longest sequences first: ragged lengths with ties, zeros and a full-length one, every
+    output row and final state against the oracle (padding rows zero, L = 0 states bit for bit)."""
+    B, S = 40, 130
+    L = np.random.default_rng(77).integers(0, S + 1, size=B).astype(np.int32)
+    L[:4] = [S, 0, 70, 70]
+    w = workloads.random_case(B=B, Nk=2, Nv=4, S=S, Dk=128, Dv=128, seed=78, lengths=L)
+    ins = unfused_inputs(w, dt)
+    go, gf = gpu_chunk(ins, w, dt, lengths=L)
+    ro, rf = ref_chunk(ins, w, lengths=L)
+    assert_close(go, ro, dt, "out")
+    assert_close(gf, rf, dt, "final_state")
+    for b in range(B):
+        assert np.all(go[b, :, L[b]:] == 0.0)
+        if L[b] == 0:
+            assert np.array_equal(gf[b], ins["initial_state"][b])
+
+
 def test_no_gate_no_initial_state_and_empty_sequence_axis():
     w = workloads.random_case(B=2, Nk=2, Nv=2, S=70, Dk=32, Dv=32, seed=70, gate="none", initial_state=False)
     ins = unfused_inputs(w, "f32")
