@@ -238,6 +238,15 @@ def cpu_oracle_sample(w):
     return w.S / dt, dt, oracle.threads()
 
 
+def prefill_config(world: int) -> dict:
+    """The `config` of the headline line (both arms)."""
+    p = workloads.spec("prefill")
+    return {"workload": f"prefill B={p['B']} S={p['S']} Nk={p['Nk']} Nv={p['Nv']} Dk=Dv={p['D']} bf16, fused "
+                        "prologue, equal lengths", "global_batch": p["B"] * world, "seq_len": p["S"],
+            "parallelism": f"dp{world} (independent batches per GPU)",
+            "l2": "inputs larger than L2, plus a 256 MiB flush before every timed step"}
+
+
 def run_reference(args, world, rank):
     if rank != 0:
         return
@@ -249,12 +258,12 @@ def run_reference(args, world, rank):
             vals.append(dt)
     tot = sum(vals)
     value = w.S * len(vals) / tot
-    sample = f"1 sequence x 4096 tokens x 32 value heads of the prefill workload per step, prologue included"
+    sample = (f"1 of the workload's {workloads.spec('prefill')['B']} sequences per step (4096 tokens x 32 value "
+              "heads, prologue included), on the host cores; the oracle in fp64")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot / len(vals),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": "prefill B=4 S=4096 Nk=16 Nv=32 Dk=Dv=128 (oracle sample: B=1)",
-                       "global_batch": 1, "seq_len": 4096, "parallelism": "host cores"},
+            "config": prefill_config(world),
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": thr, "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -300,10 +309,7 @@ def bench_prefill(gdr, args, world, rank, clk, flush, stream, peaks):
     achieved = alg_bytes / (ms_per_step / 1e3) / 1e9
     fields = {
         "value": weak_scaling_rate(tokens, args.steps, total_ms, world), "ms_per_step": ms_per_step,
-        "config": {"workload": f"prefill B={w.B} S={w.S} Nk={w.Nk} Nv={w.Nv} Dk=Dv={w.Dk} bf16, fused prologue, "
-                               "equal lengths", "global_batch": w.B * world, "seq_len": w.S,
-                   "parallelism": f"dp{world} (independent batches per GPU)",
-                   "l2": "inputs larger than L2, plus a 256 MiB flush before every timed step"},
+        "config": prefill_config(world),
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                      "frac": achieved / peaks["hbm_gbs"], "traffic": profiled_traffic("chunk"),
                      "peak_source": peaks["source"], "algorithmic_bytes_per_launch": alg_bytes,

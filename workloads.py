@@ -82,18 +82,26 @@ def _loguniform_gate(rng, shape, lo, hi, dtype):
     return np.log(rng.uniform(lo, hi, size=shape)).astype(dtype)
 
 
+_SPECS = {
+    "tiny": dict(B=1, S=64, Nk=2, Nv=2, D=32, seed=0, dtype="f32"),
+    "decode": dict(B=64, S=1, Nk=16, Nv=32, D=128, seed=1, dtype="bf16"),
+    "prefill": dict(B=4, S=4096, Nk=16, Nv=32, D=128, seed=2, dtype="bf16"),
+    "varlen": dict(B=8, S=8192, Nk=16, Nv=32, D=128, seed=3, dtype="bf16"),
+    "decode_gk": dict(B=256, S=4, Nk=16, Nv=32, D=128, seed=4, dtype="bf16"),
+}
+
+
+def spec(name: str) -> dict:
+    """The sizes, seed and dtype of a named workload, without drawing it."""
+    if name not in NAMES:
+        raise ValueError(f"unknown workload {name!r}; choose from {NAMES}")
+    return dict(_SPECS[name])
+
+
 def generate(name: str, *, B=None, S=None, Nk=None, Nv=None, D=None, seed=None, fdtype=None) -> Workload:
     """Draw one of the named workloads.  Keyword overrides shrink it (for
     parity tests at small sizes) while keeping the same distributions."""
-    if name not in NAMES:
-        raise ValueError(f"unknown workload {name!r}; choose from {NAMES}")
-    base = {
-        "tiny": dict(B=1, S=64, Nk=2, Nv=2, D=32, seed=0, dtype="f32"),
-        "decode": dict(B=64, S=1, Nk=16, Nv=32, D=128, seed=1, dtype="bf16"),
-        "prefill": dict(B=4, S=4096, Nk=16, Nv=32, D=128, seed=2, dtype="bf16"),
-        "varlen": dict(B=8, S=8192, Nk=16, Nv=32, D=128, seed=3, dtype="bf16"),
-        "decode_gk": dict(B=256, S=4, Nk=16, Nv=32, D=128, seed=4, dtype="bf16"),
-    }[name]
+    base = spec(name)
     B = base["B"] if B is None else B
     S = base["S"] if S is None else S
     Nk = base["Nk"] if Nk is None else Nk
