@@ -86,6 +86,16 @@ def test_decode_head_sizes_f32(Dk, Dv):
     check_decode(w, go, gp, ro, rp, p0, "f32")
 
 
+@pytest.mark.parametrize("dt,sdt", [("bf16", "bf16"), ("bf16", "f32")])
+def test_decode_max_tokens_per_key_gate(dt, sdt):
+    """S = 8, the most tokens one decode call takes, with the per-key gate at D = 128: the largest stage of
+    the decode kernel.  Ragged lengths (one empty), accepted counts drawn in [0, L]."""
+    w = workloads.random_case(B=12, Nk=2, Nv=4, S=8, Dk=128, Dv=128, seed=44, slots=16, with_gk=True,
+                              lengths=[8, 8, 7, 1, 0, 8, 5, 8, 2, 8, 8, 3])
+    go, gp, ro, rp, p0 = run_decode(w, dt, sdt)
+    check_decode(w, go, gp, ro, rp, p0, dt, sdt)
+
+
 def test_decode_distinct_slots_per_token():
     """One slot per token: the state after token t lands in slot idx[t] for t < A."""
     w = workloads.random_case(B=4, Nk=2, Nv=4, S=4, Dk=64, Dv=64, seed=43, slots=20, share_slot=False,

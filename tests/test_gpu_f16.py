@@ -12,7 +12,8 @@ pytestmark = pytest.mark.gpu
 
 @pytest.mark.parametrize("D,S", [(128, 200), (64, 65), (32, 40)])
 def test_chunk_f16(D, S):
-    """fp16 prefill (the CUDA-core kernel) with ragged lengths, one empty sequence and an initial state."""
+    """fp16 prefill (the tensor-core kernel at D = 128, the CUDA-core kernel otherwise) with ragged lengths, one
+    empty sequence and an initial state."""
     lengths = np.array([S, max(S - 29, 1), 0], np.int32)
     w = workloads.random_case(B=3, Nk=2, Nv=4, S=S, Dk=D, Dv=D, seed=600 + S + D, lengths=lengths)
     ins = unfused_inputs(w, "f16")
