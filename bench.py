@@ -604,6 +604,7 @@ def run_ours(args, world, rank, local):
         launches += fields.pop("gpu_launches")
         if not args.no_e2e:
             line["e2e"], n = bench_e2e(gdr, args, world, w, t, pro, flush, stream)
+            launches += n  # one prefill kernel per step
         if not args.no_epilogue:
             line["prefill_epilogue"], n = bench_prefill_epilogue(gdr, args, world, w, t, pro, flush, stream, peaks)
             launches += n
