@@ -148,6 +148,9 @@ def _dev(t: torch.Tensor, name: str, dtype=None, shape=None):
         raise RuntimeError(f"{name} must be a torch.Tensor")
     if not t.is_cuda:
         raise RuntimeError(f"{name} must be a CUDA tensor")
+    cur = torch.cuda.current_device()
+    if t.device.index != cur:  # the kernels run on the current device and would read this pointer there
+        raise RuntimeError(f"{name} is on {t.device}, but the call runs on the current device cuda:{cur}")
     if dtype is not None and t.dtype != dtype:
         raise RuntimeError(f"{name} must have dtype {dtype}, got {t.dtype}")
     if shape is not None and tuple(t.shape) != tuple(shape):
@@ -159,6 +162,9 @@ def _dev(t: torch.Tensor, name: str, dtype=None, shape=None):
 
 def _stream(stream) -> ctypes.c_void_p:
     s = stream if stream is not None else torch.cuda.current_stream()
+    if s.device.index != torch.cuda.current_device():
+        raise RuntimeError(f"the stream is on {s.device}, but the call runs on the current device "
+                           f"cuda:{torch.cuda.current_device()}")
     return ctypes.c_void_p(s.cuda_stream)
 
 
