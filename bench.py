@@ -223,19 +223,72 @@ def timed_steps(fn, K, flush, stream):
     return [s.elapsed_time(e) for s, e in evs]
 
 
-def cpu_oracle_sample(w):
+def cpu_oracle_sample(w, heads=None):
     """The fp64 oracle as it stands on one sequence of the prefill workload (all
-    value heads, all 4096 tokens), prologue included.  Returns (tokens/s, seconds, threads)."""
+    value heads, or the first `heads` of them, all 4096 tokens), prologue included.
+    Returns (tokens/s for all the workload's value heads, seconds, threads)."""
     import oracle
     sl = slice(0, 1)
+    hv = w.Nv if heads is None else heads
+    hk = max(1, hv * w.Nk // w.Nv)
     to_bf16 = lambda x: torch.from_numpy(np.ascontiguousarray(x)).to(torch.bfloat16).double().numpy()
-    q, k, v, b = (to_bf16(x[sl]) for x in (w.q, w.k, w.v, w.b))
-    s0 = to_bf16(w.initial_state[sl])
+    q, k = (to_bf16(x[sl, :hk]) for x in (w.q, w.k))
+    v, b = (to_bf16(x[sl, :hv]) for x in (w.v, w.b))
+    s0 = to_bf16(w.initial_state[sl, :hv])
     t0 = time.perf_counter()
-    p = oracle.prologue(q=q, k=k, b=b, a=w.a[sl], A_log=w.A_log, dt_bias=w.dt_bias)
+    p = oracle.prologue(q=q, k=k, b=b, a=w.a[sl, :hv], A_log=w.A_log[:hv], dt_bias=w.dt_bias[:hv])
     oracle.chunk_fwd(p["q_hat"], p["k_hat"], v, p["beta"], p["g"], s0, None, w.scale)
     dt = time.perf_counter() - t0
-    return w.S / dt, dt, oracle.threads()
+    return w.S * hv / w.Nv / dt, dt, oracle.threads()
+
+
+def cpu_model() -> str:
+    """The host CPU's model name (lscpu, else /proc/cpuinfo)."""
+    import subprocess
+    try:
+        out = subprocess.run(["lscpu"], capture_output=True, text=True, timeout=10).stdout
+        for line in out.splitlines():
+            if line.strip().startswith("Model name:"):
+                return line.split(":", 1)[1].strip()
+    except Exception:
+        pass
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except Exception:
+        pass
+    return "unknown"
+
+
+def cpu_baseline_fields() -> dict:
+    """The oracle on the host cores: one prefill sequence on all threads (the headline's unit), the first 4 value
+    heads of it on one thread, and one call of the decode workload (B=64, one token, 32 value heads)."""
+    import oracle
+    wp = workloads.generate("prefill", B=1)
+    tps, dt, thr = cpu_oracle_sample(wp)
+    oracle.set_threads(1)
+    try:
+        tps1, dt1, _ = cpu_oracle_sample(wp, heads=4)
+        wd = workloads.generate("decode")
+        to_bf16 = lambda x: torch.from_numpy(np.ascontiguousarray(x)).to(torch.bfloat16).double().numpy()
+        q, k, v, b, pool = (to_bf16(x) for x in (wd.q, wd.k, wd.v, wd.b, wd.pool))
+        g = np.asarray(wd.g, np.float32).astype(np.float64)
+        t0 = time.perf_counter()
+        p = oracle.prologue(q=q, k=k, b=b)
+        oracle.recurrent_step(p["q_hat"], p["k_hat"], v, p["beta"], g, None, pool, wd.indices, wd.lengths,
+                              wd.accepted, wd.scale)
+        dtd = time.perf_counter() - t0
+    finally:
+        oracle.set_threads(thr)
+    state = algorithmic_decode_bytes(wd)["state"]
+    return {"value": tps, "unit": UNIT, "cores": thr, "kind": "oracle", "cpu_model": cpu_model(),
+            "sample": f"1 sequence x 4096 tokens x 32 value heads, prologue included, {dt:.1f} s on {thr} threads",
+            "single_thread": {"value": tps1, "unit": UNIT, "cores": 1,
+                              "sample": f"the first 4 value heads of that sequence on 1 thread, {dt1:.1f} s, "
+                                        "scaled to 32 heads"},
+            "decode": {"us_per_call": dtd * 1e6, "state_GBps": state / dtd / 1e9, "cores": 1,
+                       "sample": "one call of the decode workload (B=64, one token, 32 value heads), 1 thread"}}
 
 
 def prefill_config(world: int) -> dict:
@@ -314,15 +367,14 @@ def bench_prefill(gdr, args, world, rank, clk, flush, stream, peaks):
                      "frac": achieved / peaks["hbm_gbs"], "traffic": profiled_traffic("chunk"),
                      "peak_source": peaks["source"], "algorithmic_bytes_per_launch": alg_bytes,
                      "kernel": "gdr_chunk_fwd (fused prologue)"},
-        "gpu_launches": args.steps,
+        "gpu_launches": 2 * args.steps,  # the WY pass and the chain kernel per call
     }
     return fields, w, t, pro, step
 
 
 def bench_varlen(gdr, args, world, rank, flush, stream, peaks):
     """The variable-length prefill workload (B=8, padded S=8192, lengths ~ U[512, 8192] with one 0), fused
-    prologue; a parity-test configuration, timed only on request (--only varlen), not in the default line.
-    256 chains on 148 SMs: the kernel starts the longest sequences first."""
+    prologue.  256 chains on 148 SMs: the chain kernel starts the longest sequences first."""
     w = workloads.generate("varlen", seed=3 + 1000 * rank)
     t = dict(q=bf16_dev(w.q), k=bf16_dev(w.k), v=bf16_dev(w.v), b=bf16_dev(w.b), a=f32_dev(w.a),
              s0=bf16_dev(w.initial_state))
@@ -349,7 +401,35 @@ def bench_varlen(gdr, args, world, rank, flush, stream, peaks):
             "l2": "inputs larger than L2, plus a 256 MiB flush before every timed step",
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                          "frac": achieved / peaks["hbm_gbs"], "traffic": None, "algorithmic_bytes_per_launch": nb}}, \
-        args.steps
+        2 * args.steps
+
+
+def bench_prefill_no_gate(gdr, args, world, w, t, flush, stream, peaks):
+    """The prefill workload without a gate (g = NULL, hasGamma = 0 of the chunk operator): the build of the WY pass
+    and the chain kernel without the gate arithmetic; l2norm and beta logits fused."""
+    pro = gdr.Prologue(l2norm_qk=True, eps=1e-6, beta_logits=True)
+    step = gdr.prepare_chunk_fwd(t["q"], t["k"], t["v"], t["b"], None, t["s0"], None, w.scale, prologue=pro,
+                                 out=t["out"], final_state=t["fin"])
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if gdr.get_error() != 0:
+        raise RuntimeError("device error word set during warm-up")
+    barrier(world)
+    torch.cuda.synchronize()
+    times = timed_steps(step, args.steps, flush, stream)
+    barrier(world)
+    total_ms = all_max(sum(times), world)
+    ms = total_ms / args.steps
+    tokens = int(w.lengths.sum())
+    alg = algorithmic_prefill_bytes(w) - tokens * w.Nv * 4  # no gate input
+    achieved = alg / (ms / 1e3) / 1e9
+    return {"workload": f"prefill B={w.B} S={w.S} Nk={w.Nk} Nv={w.Nv} Dk=Dv={w.Dk} bf16, no gate (g = NULL), "
+                        "fused l2norm and beta", "ms_per_step": ms,
+            "tokens_per_s": weak_scaling_rate(tokens, args.steps, total_ms, world),
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": achieved / peaks["hbm_gbs"], "traffic": None, "algorithmic_bytes_per_launch": alg,
+                         "kernel": "gdr_chunk_fwd without gate"}}, 2 * args.steps
 
 
 def bench_prefill_epilogue(gdr, args, world, w, t, pro, flush, stream, peaks):
@@ -380,7 +460,7 @@ def bench_prefill_epilogue(gdr, args, world, w, t, pro, flush, stream, peaks):
             "ms_per_step": ms_per_step, "tokens_per_s": weak_scaling_rate(tokens, args.steps, total_ms, world),
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                          "frac": achieved / peaks["hbm_gbs"], "traffic": None, "algorithmic_bytes_per_launch":
-                         alg_bytes, "kernel": "gdr_chunk_fwd (fused prologue and epilogue)"}}, args.steps
+                         alg_bytes, "kernel": "gdr_chunk_fwd (fused prologue and epilogue)"}}, 2 * args.steps
 
 
 def bench_conv1d(gdr, args, world, rank, flush, stream, peaks):
@@ -461,7 +541,7 @@ def bench_f16(gdr, args, world, rank, flush, stream, peaks):
             "decode": {"workload": "decode B=64 S=1 fp16 inputs, fp32 state (general decode kernel), L2 flush",
                        "us_per_call": d_ms * 1e3,
                        "roofline": {"bound": "hbm", "achieved": d_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                                    "frac": d_gbs / peaks["hbm_gbs"]}}}, 2 * args.steps
+                                    "frac": d_gbs / peaks["hbm_gbs"]}}}, 3 * args.steps
 
 
 def bench_e2e(gdr, args, world, w, t, pro, flush, stream):
@@ -567,10 +647,21 @@ def bench_decode(gdr, name, args, world, rank, clk, flush, stream, peaks, rotate
             e.record(stream)
             evs.append((s, e))
     torch.cuda.synchronize()
-    clk.active = False
     barrier(world)
     times = [s.elapsed_time(e) for s, e in evs]
-    d_ms = all_max(sum(times), world) / args.steps
+    single_ms = all_max(sum(times), world) / args.steps
+    # the serving loop: the same calls back to back inside one event pair (no host gap inside the region)
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record(stream)
+        for i in range(args.steps):
+            calls[i % rotate]()
+        e.record(stream)
+    torch.cuda.synchronize()
+    clk.active = False
+    barrier(world)
+    d_ms = all_max(s.elapsed_time(e), world) / args.steps
     nb = algorithmic_decode_bytes(wd)
     if spec:  # one state read per sequence and head, one state written per processed token
         nb["state"] = int((1 + wd.lengths).sum()) * wd.Nv * wd.Dk * wd.Dv * 2
@@ -580,11 +671,13 @@ def bench_decode(gdr, name, args, world, rank, clk, flush, stream, peaks, rotate
                         + (", per-key gate" if wd.gk is not None else "") + ", fused prologue"
                         + (", per-token slots, accepted ~ U[1, 4] (speculative decoding)" if spec else ""),
             "l2": f"{rotate} rotating pool copies (fresh state every call), no flush",
-            "us_per_call": d_ms * 1e3, "steps_per_s": world * 1e3 / d_ms,
+            "timing": f"{args.steps} calls back to back inside one event pair; us_per_call_single: each call inside "
+                      "its own event pair",
+            "us_per_call": d_ms * 1e3, "us_per_call_single": single_ms * 1e3, "steps_per_s": world * 1e3 / d_ms,
             "state_GBps": gbs, "state_frac_of_hbm": gbs / peaks["hbm_gbs"],
             "roofline": {"bound": "hbm", "achieved": tot, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                          "frac": tot / peaks["hbm_gbs"], "traffic": profiled_traffic(name),
-                         "algorithmic_bytes_per_launch": nb["state"] + nb["io"]}}, args.steps
+                         "algorithmic_bytes_per_launch": nb["state"] + nb["io"]}}, 2 * args.steps
 
 
 def run_ours(args, world, rank, local):
@@ -604,12 +697,14 @@ def run_ours(args, world, rank, local):
         launches += fields.pop("gpu_launches")
         if not args.no_e2e:
             line["e2e"], n = bench_e2e(gdr, args, world, w, t, pro, flush, stream)
-            launches += n  # one prefill kernel per step
+            launches += 2 * n  # two prefill kernels per step
         if not args.no_epilogue:
             line["prefill_epilogue"], n = bench_prefill_epilogue(gdr, args, world, w, t, pro, flush, stream, peaks)
             launches += n
+        line["prefill_no_gate"], n = bench_prefill_no_gate(gdr, args, world, w, t, flush, stream, peaks)
+        launches += n
         del t
-    if args.only == "varlen":  # a parity-test configuration: timed on request only
+    if args.only in ("all", "varlen"):
         line["varlen"], n = bench_varlen(gdr, args, world, rank, flush, stream, peaks)
         launches += n
     if args.only in ("all", "conv1d"):
@@ -631,9 +726,7 @@ def run_ours(args, world, rank, local):
     line["gpu_launches"] = launches
     line["clocks"] = clk.summary()
     if rank == 0 and world == 1 and not args.no_cpu_baseline and args.only in ("all", "prefill"):
-        tps, dt, thr = cpu_oracle_sample(workloads.generate("prefill", B=1))
-        line["cpu_baseline"] = {"value": tps, "unit": UNIT, "cores": thr, "kind": "oracle",
-                                "sample": f"1 sequence x 4096 tokens x 32 value heads, prologue included, {dt:.1f} s"}
+        line["cpu_baseline"] = cpu_baseline_fields()
     if rank == 0:
         print(json.dumps(line), flush=True)
 
@@ -650,8 +743,7 @@ def main():
                     help="skip the prefill line with the fused gated RMSNorm epilogue (profiling runs)")
     ap.add_argument("--only", choices=["all", "prefill", "decode", "decode_gk", "decode_spec", "conv1d", "f16",
                                        "varlen"], default="all",
-                    help="run one workload only (profiling runs); the default runs all but varlen, a "
-                         "parity-test configuration timed on request")
+                    help="run one workload only (profiling runs); the default runs all")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

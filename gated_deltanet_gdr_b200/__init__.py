@@ -26,13 +26,14 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libgdr.so")
 
 GDR_OK, GDR_ERR_SHAPE, GDR_ERR_DTYPE, GDR_ERR_NULL, GDR_ERR_ALIGN, GDR_ERR_UNSUPPORTED, GDR_ERR_DEVICE, \
-    GDR_ERR_LAUNCH = range(8)
+    GDR_ERR_LAUNCH, GDR_ERR_WORKSPACE = range(9)
 GDR_F32, GDR_BF16, GDR_F16 = 0, 1, 2
 DEVERR_SLOT_INDEX, DEVERR_LENGTH, DEVERR_TIMEOUT = 0x1, 0x2, 0x4
 
 # Every symbol the C header declares (checked by the ABI test).
-EXPORTED = ("gdr_chunk_fwd", "gdr_recurrent_step", "gdr_recurrent_step_spec", "gdr_conv1d", "gdr_prologue_apply",
-            "gdr_get_error", "gdr_status_string", "gdr_version")
+EXPORTED = ("gdr_chunk_fwd_workspace", "gdr_chunk_fwd", "gdr_recurrent_step", "gdr_recurrent_step_spec", "gdr_conv1d",
+            "gdr_prologue_apply", "gdr_get_error", "gdr_debug_set_wait_limit", "gdr_debug_timeout_site",
+            "gdr_status_string", "gdr_version")
 
 
 class GdrPrologueStruct(ctypes.Structure):
@@ -59,9 +60,12 @@ def lib() -> ctypes.CDLL:
                                "`python -m gated_deltanet_gdr_b200.build` -- there is no fallback path")
         L = ctypes.CDLL(LIB_PATH)
         vp, i32, f32 = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+        L.gdr_chunk_fwd_workspace.restype = ctypes.c_size_t
+        L.gdr_chunk_fwd_workspace.argtypes = [i32, i32, i32, i32, i32, i32, i32]
         L.gdr_chunk_fwd.restype = i32
         L.gdr_chunk_fwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, f32, i32, i32, i32, i32, i32, i32, i32,
-                                    ctypes.POINTER(GdrPrologueStruct), ctypes.POINTER(GdrEpilogueStruct), vp, vp, vp]
+                                    ctypes.POINTER(GdrPrologueStruct), ctypes.POINTER(GdrEpilogueStruct), vp, vp, vp,
+                                    ctypes.c_size_t, vp]
         L.gdr_recurrent_step.restype = i32
         L.gdr_recurrent_step.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, vp, vp, vp, f32, i32, i32, i32, i32, i32,
                                          i32, i32, i32, ctypes.POINTER(GdrPrologueStruct),
@@ -75,6 +79,10 @@ def lib() -> ctypes.CDLL:
                                          vp]
         L.gdr_get_error.restype = i32
         L.gdr_get_error.argtypes = [vp, ctypes.POINTER(ctypes.c_int)]
+        L.gdr_debug_set_wait_limit.restype = i32
+        L.gdr_debug_set_wait_limit.argtypes = [ctypes.c_ulonglong]
+        L.gdr_debug_timeout_site.restype = i32
+        L.gdr_debug_timeout_site.argtypes = [ctypes.POINTER(ctypes.c_uint)]
         L.gdr_status_string.restype = ctypes.c_char_p
         L.gdr_status_string.argtypes = [i32]
         L.gdr_version.restype = i32
@@ -195,21 +203,41 @@ def _chunk_checked(q, k, v, beta, g, initial_state, actual_seq_lengths, prologue
     return out, final_state
 
 
+def chunk_fwd_workspace_bytes(B: int, Nk: int, Nv: int, S: int, Dk: int, Dv: int, dtype: torch.dtype) -> int:
+    """Bytes of workspace ``gdr_chunk_fwd`` needs for these sizes (``gdr_chunk_fwd_workspace``)."""
+    return int(lib().gdr_chunk_fwd_workspace(B, Nk, Nv, S, Dk, Dv, _dtype_code(dtype)))
+
+
+def _workspace(q, v, workspace):
+    """The caller's workspace (a CUDA uint8 tensor), or a new one of the size the call needs."""
+    B, Nk, S, Dk = q.shape
+    Nv, Dv = v.shape[1], v.shape[3]
+    need = chunk_fwd_workspace_bytes(B, Nk, Nv, S, Dk, Dv, q.dtype)
+    if workspace is None:
+        return torch.empty(need, dtype=torch.uint8, device=q.device) if need else None
+    _dev(workspace, "workspace", torch.uint8)
+    if workspace.numel() < need:
+        raise ValueError(f"workspace holds {workspace.numel()} bytes; the call needs {need}")
+    return workspace
+
+
 def chunk_fwd(q, k, v, beta, g=None, initial_state=None, actual_seq_lengths=None, scale: float = 1.0, *,
               prologue: Optional[Prologue] = None, epilogue: Optional[Epilogue] = None, out=None, final_state=None,
-              output_final_state: bool = True, stream=None):
-    """Chunked prefill (``gdr_chunk_fwd``).  Returns (out, final_state or None)."""
+              output_final_state: bool = True, workspace=None, stream=None):
+    """Chunked prefill (``gdr_chunk_fwd``).  Returns (out, final_state or None).  ``workspace`` (uint8, at least
+    ``chunk_fwd_workspace_bytes`` bytes) is allocated per call when not given."""
     out, final_state = _chunk_checked(q, k, v, beta, g, initial_state, actual_seq_lengths, prologue, out,
                                       final_state, output_final_state)
     B, Nk, S, Dk = q.shape
     Nv, Dv = v.shape[1], v.shape[3]
     pro = prologue.as_struct() if prologue is not None else None
     epi = _check_epilogue(epilogue, B, Nv, S, Dv, q.dtype)
+    ws = _workspace(q, v, workspace)
     st = lib().gdr_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(g), _ptr(initial_state),
                              _ptr(actual_seq_lengths), float(scale), B, Nk, Nv, S, Dk, Dv, _dtype_code(q.dtype),
                              ctypes.byref(pro) if pro is not None else None,
                              ctypes.byref(epi) if epi is not None else None, _ptr(out), _ptr(final_state),
-                             _stream(stream))
+                             _ptr(ws), 0 if ws is None else ws.numel(), _stream(stream))
     _check(st, "gdr_chunk_fwd")
     return out, final_state
 
@@ -286,20 +314,23 @@ class PreparedCall:
 
 def prepare_chunk_fwd(q, k, v, beta, g=None, initial_state=None, actual_seq_lengths=None, scale: float = 1.0, *,
                       prologue: Optional[Prologue] = None, epilogue: Optional[Epilogue] = None, out=None,
-                      final_state=None, stream=None) -> PreparedCall:
-    """Check and marshal a gdr_chunk_fwd call once; see chunk_fwd for the arguments."""
+                      final_state=None, workspace=None, stream=None) -> PreparedCall:
+    """Check and marshal a gdr_chunk_fwd call once; see chunk_fwd for the arguments (the workspace, if not given,
+    is allocated once here and kept by the prepared call)."""
     out, final_state = _chunk_checked(q, k, v, beta, g, initial_state, actual_seq_lengths, prologue, out,
                                       final_state, True)
     B, Nk, S, Dk = q.shape
     Nv, Dv = v.shape[1], v.shape[3]
     pro = prologue.as_struct() if prologue is not None else None
     epi = _check_epilogue(epilogue, B, Nv, S, Dv, q.dtype)
+    ws = _workspace(q, v, workspace)
     args = (_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(g), _ptr(initial_state), _ptr(actual_seq_lengths),
             ctypes.c_float(scale), B, Nk, Nv, S, Dk, Dv, _dtype_code(q.dtype),
             ctypes.pointer(pro) if pro is not None else None, ctypes.pointer(epi) if epi is not None else None,
-            _ptr(out), _ptr(final_state), _stream(stream))
+            _ptr(out), _ptr(final_state), _ptr(ws), ctypes.c_size_t(0 if ws is None else ws.numel()),
+            _stream(stream))
     call = PreparedCall(lib().gdr_chunk_fwd, args, "gdr_chunk_fwd", (out, final_state))
-    call._keep = (pro, prologue, epi, epilogue)
+    call._keep = (pro, prologue, epi, epilogue, ws)
     return call
 
 
@@ -415,3 +446,19 @@ def get_error(stream=None) -> int:
 
 def version() -> int:
     return int(lib().gdr_version())
+
+
+def take_timeout_site() -> dict:
+    """Diagnostic: the first bounded wait of the tensor-core prefill that ran out since the last read (cleared by
+    the read), as {"warp", "barrier", "parity", "cta"}, or {} if none."""
+    v = ctypes.c_uint(0)
+    _check(lib().gdr_debug_timeout_site(ctypes.byref(v)), "gdr_debug_timeout_site")
+    x = v.value
+    if not x:
+        return {}
+    return {"warp": (x >> 24) & 0x3F, "barrier": (x >> 16) & 0xFF, "parity": (x >> 15) & 1, "cta": x & 0x7FFF}
+
+
+def set_wait_limit_ns(ns: int) -> None:
+    """Diagnostic: the limit of the tensor-core prefill's bounded waits for later calls (0: the default, 1 s)."""
+    _check(lib().gdr_debug_set_wait_limit(int(ns)), "gdr_debug_set_wait_limit")

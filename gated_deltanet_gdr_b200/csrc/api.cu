@@ -6,7 +6,10 @@
 
 #include <cstdint>
 #include <cstdlib>
+#include <cstring>
 #include <mutex>
+#include <unordered_map>
+#include <vector>
 
 #include "../../include/gdr.h"
 #include "kernels.h"
@@ -15,6 +18,13 @@ namespace gdr {
 
 // The device error word (GDR_DEVERR_* bits) of this library, one per device.
 __device__ unsigned int g_device_error = 0;
+// Snapshots of the error word taken by gdr_get_error, one slot per concurrent call (a call takes the next slot
+// round-robin, so calls on different streams or host threads do not share one).
+constexpr int kErrSlots = 64;
+__device__ unsigned int g_error_snapshot[kErrSlots];
+
+// Reads and clears the error word in one atomic step, so no bit raised meanwhile by another stream's kernel is lost.
+__global__ void take_error_kernel(unsigned int *err, unsigned int *slot) { *slot = atomicExch(err, 0u); }
 
 namespace {
 
@@ -22,6 +32,8 @@ constexpr int kMaxDevices = 64;
 std::mutex g_mu;
 int g_dev_checked[kMaxDevices];        // 0 unknown, 1 sm_100, -1 unusable
 unsigned int *g_err_ptr[kMaxDevices];  // device address of g_device_error per device
+unsigned int *g_snap_ptr[kMaxDevices]; // device address of g_error_snapshot per device
+unsigned int g_snap_next = 0;          // next snapshot slot (under g_mu)
 
 bool supported_head(int d) { return d == 16 || d == 32 || d == 64 || d == 128; }
 bool aligned16(const void *p) { return p == nullptr || (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -51,6 +63,11 @@ int device_setup(unsigned int **err) {
             return GDR_ERR_LAUNCH;
         }
         g_err_ptr[dev] = static_cast<unsigned int *>(p);
+        if (cudaGetSymbolAddress(&p, g_error_snapshot) != cudaSuccess) {
+            cudaGetLastError();
+            return GDR_ERR_LAUNCH;
+        }
+        g_snap_ptr[dev] = static_cast<unsigned int *>(p);
         g_dev_checked[dev] = 1;
     }
     if (g_dev_checked[dev] < 0) return GDR_ERR_DEVICE;
@@ -75,6 +92,69 @@ int check_prologue(const gdr_prologue *p, const float *g) {
     return GDR_OK;
 }
 
+// ---- checked mode (environment variable GDR_CHECKS=1): host-side validation of the index and length arrays ----
+// The kernels never trap on bad lengths or slots (they skip the sequence and flag the error word), and two
+// sequences that share a slot race silently.  In checked mode the library copies the arrays to the host before
+// launching (a synchronisation on the caller's stream, so for debugging only) and rejects such calls with
+// GDR_ERR_SHAPE.
+bool checks_enabled() {
+    const char *v = std::getenv("GDR_CHECKS");
+    return v && v[0] && std::strcmp(v, "0") != 0;
+}
+
+bool copy_i32(std::vector<int32_t> &h, const int32_t *d, size_t n, cudaStream_t s) {
+    h.assign(n, 0);
+    if (n == 0 || !d) return true;
+    if (cudaMemcpyAsync(h.data(), d, n * sizeof(int32_t), cudaMemcpyDeviceToHost, s) != cudaSuccess) return false;
+    return cudaStreamSynchronize(s) == cudaSuccess;
+}
+
+// lengths within [0, S]
+int check_lengths_host(const int32_t *lengths, int B, int S, cudaStream_t s) {
+    if (!lengths) return GDR_OK;
+    std::vector<int32_t> L;
+    if (!copy_i32(L, lengths, (size_t)B, s)) return GDR_ERR_LAUNCH;
+    for (int b = 0; b < B; ++b)
+        if (L[b] < 0 || L[b] > S) return GDR_ERR_SHAPE;
+    return GDR_OK;
+}
+
+// Decode: lengths in [0, S], accepted counts in range, every slot a sequence reads or writes in [0, slots), and
+// no slot touched by two sequences.  per_token selects the speculative-decoding reading (the chain starts at token
+// A - 1's slot and every processed token's state goes to its own slot); otherwise the chain starts at token 0's
+// slot and the first min(A, L) states are committed.
+int check_decode_host(const int32_t *idx, const int32_t *lengths, const int32_t *accepted, int B, int S, int slots,
+                      int per_token, cudaStream_t s) {
+    std::vector<int32_t> I, L, A;
+    if (!copy_i32(I, idx, (size_t)B * S, s) || !copy_i32(L, lengths, (size_t)B, s) ||
+        !copy_i32(A, accepted, accepted ? (size_t)B : 0, s))
+        return GDR_ERR_LAUNCH;
+    std::unordered_map<int32_t, int> owner;
+    for (int b = 0; b < B; ++b) {
+        const int Lb = L[b];
+        if (Lb < 0 || Lb > S) return GDR_ERR_SHAPE;
+        if (Lb == 0) continue;
+        int Ab = accepted ? A[b] : (per_token ? 1 : Lb);
+        std::vector<int32_t> touched;
+        if (per_token) {
+            if (Ab < 1 || Ab > S) return GDR_ERR_SHAPE;
+            touched.push_back(I[(size_t)b * S + Ab - 1]);
+            for (int t = 0; t < Lb; ++t) touched.push_back(I[(size_t)b * S + t]);
+        } else {
+            if (Ab < 0) return GDR_ERR_SHAPE;
+            touched.push_back(I[(size_t)b * S]);
+            for (int t = 0; t < (Ab < Lb ? Ab : Lb); ++t) touched.push_back(I[(size_t)b * S + t]);
+        }
+        for (int32_t x : touched) {
+            if (x < 0 || x >= slots) return GDR_ERR_SHAPE;
+            auto it = owner.find(x);
+            if (it != owner.end() && it->second != b) return GDR_ERR_SHAPE;
+            owner[x] = b;
+        }
+    }
+    return GDR_OK;
+}
+
 int check_epilogue(const gdr_epilogue *e) {
     if (!e) return GDR_OK;
     if (!e->z || !e->norm_w) return GDR_ERR_NULL;
@@ -88,18 +168,28 @@ int check_epilogue(const gdr_epilogue *e) {
 
 using namespace gdr;
 
+extern "C" size_t gdr_chunk_fwd_workspace(int B, int Nk, int Nv, int S, int Dk, int Dv, gdr_dtype dtype) {
+    if (check_common(B, Nk, Nv, S, Dk, Dv, dtype) != GDR_OK) return 0;
+    if ((long long)B * S == 0 || !chunk_tc_supported(Dk, Dv, dtype, S)) return 0;
+    return chunk_tc_workspace(B, Nv, S);
+}
+
 extern "C" int gdr_chunk_fwd(const void *q, const void *k, const void *v, const void *beta, const float *g,
                              const void *initial_state, const int32_t *actual_seq_lengths, float scale, int B,
                              int Nk, int Nv, int S, int Dk, int Dv, gdr_dtype dtype, const gdr_prologue *prologue,
-                             const gdr_epilogue *epilogue, void *out, void *final_state, gdr_stream_t stream) {
+                             const gdr_epilogue *epilogue, void *out, void *final_state, void *workspace,
+                             size_t ws_bytes, gdr_stream_t stream) {
     int st = check_common(B, Nk, Nv, S, Dk, Dv, dtype);
     if (st) return st;
     if ((st = check_prologue(prologue, g))) return st;
     if ((st = check_epilogue(epilogue))) return st;
     if ((long long)B * S > 0 && (!q || !k || !v || !beta || !out)) return GDR_ERR_NULL;
-    const void *ptrs[] = {q, k, v, beta, g, initial_state, actual_seq_lengths, out, final_state};
+    const void *ptrs[] = {q, k, v, beta, g, initial_state, actual_seq_lengths, out, final_state, workspace};
     for (const void *p : ptrs)
         if (!aligned16(p)) return GDR_ERR_ALIGN;
+    const size_t need = gdr_chunk_fwd_workspace(B, Nk, Nv, S, Dk, Dv, dtype);
+    if (need > 0 && !workspace) return GDR_ERR_NULL;
+    if (ws_bytes < need) return GDR_ERR_WORKSPACE;
     if (B == 0 || (S == 0 && !final_state)) return GDR_OK;
     unsigned int *err = nullptr;
     if ((st = device_setup(&err))) return st;
@@ -117,7 +207,9 @@ extern "C" int gdr_chunk_fwd(const void *q, const void *k, const void *v, const 
     a.A_log = prologue ? prologue->A_log : nullptr;
     a.dt_bias = prologue ? prologue->dt_bias : nullptr;
     a.err = err;
+    a.workspace = workspace;
     cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+    if (checks_enabled() && (st = check_lengths_host(actual_seq_lengths, B, S, cs))) return st;
     cudaError_t e;
     if (chunk_tc_supported(Dk, Dv, dtype, S)) {
         if (epilogue) {  // fused into the tensor-core kernel's out epilogue
@@ -148,6 +240,8 @@ int recurrent_step(const void *q, const void *k, const void *v, const void *beta
     if ((dtype == GDR_F16 && state_dtype == GDR_BF16) || (state_dtype == GDR_F16 && dtype != GDR_F16))
         return GDR_ERR_DTYPE;
     if (S < 1 || S > kDecodeMaxTokens || slots < 1) return GDR_ERR_SHAPE;
+    // the kernels address the pool by (slot, head) tile in 32-bit arithmetic
+    if ((long long)slots * Nv >= (1LL << 31)) return GDR_ERR_SHAPE;
     if ((st = check_prologue(prologue, g))) return st;
     if ((st = check_epilogue(epilogue))) return st;
     if (B > 0 && (!q || !k || !v || !beta || !out || !state_pool || !ssm_state_indices || !actual_seq_lengths))
@@ -175,6 +269,10 @@ int recurrent_step(const void *q, const void *k, const void *v, const void *beta
     a.err = err;
     a.per_token = per_token;
     cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+    if (checks_enabled() &&
+        (st = check_decode_host(ssm_state_indices, actual_seq_lengths, num_accepted_tokens, B, S, slots, per_token,
+                                cs)))
+        return st;
     cudaError_t e = launch_decode(a, Dk, Dv, dtype, state_dtype, cs);
     if (e == cudaSuccess && epilogue)
         e = launch_gated_rmsnorm(out, epilogue->z, epilogue->norm_w, epilogue->eps, actual_seq_lengths, B, Nv, S, Dv,
@@ -254,10 +352,17 @@ extern "C" int gdr_get_error(gdr_stream_t stream, int *device_error) {
     int st = device_setup(&err);
     if (st) return st;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    unsigned int *slot = nullptr;
+    {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        std::lock_guard<std::mutex> lk(g_mu);
+        slot = g_snap_ptr[dev] + (g_snap_next++ % kErrSlots);
+    }
     unsigned int host = 0;
-    if (cudaStreamSynchronize(s) != cudaSuccess) return GDR_ERR_LAUNCH;
-    if (cudaMemcpyAsync(&host, err, sizeof(host), cudaMemcpyDeviceToHost, s) != cudaSuccess) return GDR_ERR_LAUNCH;
-    if (cudaMemsetAsync(err, 0, sizeof(unsigned int), s) != cudaSuccess) return GDR_ERR_LAUNCH;
+    take_error_kernel<<<1, 1, 0, s>>>(err, slot);
+    if (cudaGetLastError() != cudaSuccess) return GDR_ERR_LAUNCH;
+    if (cudaMemcpyAsync(&host, slot, sizeof(host), cudaMemcpyDeviceToHost, s) != cudaSuccess) return GDR_ERR_LAUNCH;
     if (cudaStreamSynchronize(s) != cudaSuccess) return GDR_ERR_LAUNCH;
     *device_error = (int)host;
     return GDR_OK;
@@ -273,8 +378,23 @@ extern "C" const char *gdr_status_string(int status) {
         case GDR_ERR_UNSUPPORTED: return "head size not built (Dk and Dv must be 16, 32, 64 or 128)";
         case GDR_ERR_DEVICE: return "no usable sm_100 CUDA device";
         case GDR_ERR_LAUNCH: return "a CUDA call or kernel launch failed";
+        case GDR_ERR_WORKSPACE: return "workspace smaller than gdr_chunk_fwd_workspace() returns";
         default: return "unknown status";
     }
 }
 
-extern "C" int gdr_version(void) { return 100; }
+extern "C" int gdr_version(void) { return 200; }
+
+extern "C" int gdr_debug_set_wait_limit(unsigned long long ns) {
+    chunk_tc_set_wait_ns(ns);
+    return GDR_OK;
+}
+
+extern "C" int gdr_debug_timeout_site(unsigned int *site) {
+    if (!site) return GDR_ERR_NULL;
+    *site = 0;
+    unsigned int *err = nullptr;
+    int st = device_setup(&err);
+    if (st) return st;
+    return chunk_tc_take_timeout_site(site) == cudaSuccess ? GDR_OK : GDR_ERR_LAUNCH;
+}

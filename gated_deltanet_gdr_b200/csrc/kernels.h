@@ -48,6 +48,8 @@ struct ChunkArgs {
     const void *epi_z;
     const float *epi_w;
     float epi_eps;
+    // caller-owned scratch of the tensor-core path (chunk_tc_workspace bytes, 16-byte aligned)
+    void *workspace;
 };
 
 // cuTensorMapEncodeTiled, obtained once through the runtime's driver entry point (NULL if unavailable).
@@ -78,7 +80,14 @@ class LaunchCache {
 
 cudaError_t launch_decode(const DecodeArgs &a, int Dk, int Dv, gdr_dtype dt, gdr_dtype st, cudaStream_t s);
 bool chunk_tc_supported(int Dk, int Dv, gdr_dtype dt, int S);
+// bytes of workspace the tensor-core prefill needs: per (b, value head, 64-token chunk) the 64 x 64 16-bit T' and
+// six vectors of 64 floats
+size_t chunk_tc_workspace(int B, int Nv, int S);
 cudaError_t launch_chunk_tc(const ChunkArgs &a, gdr_dtype dt, cudaStream_t s);
+// limit of the tensor-core prefill's bounded waits, in ns (0: the default of one second)
+void chunk_tc_set_wait_ns(unsigned long long ns);
+// reads and clears the record of the first bounded wait of the tensor-core prefill that ran out (synchronous)
+cudaError_t chunk_tc_take_timeout_site(unsigned int *site);
 cudaError_t launch_chunk_simt(const ChunkArgs &a, int Dk, int Dv, gdr_dtype dt, cudaStream_t s);
 // out rows t < L_b <- rmsnorm(out row) * norm_w * silu(z row), in place (the unfused epilogue)
 cudaError_t launch_gated_rmsnorm(void *out, const void *z, const float *norm_w, float eps, const int32_t *lengths,

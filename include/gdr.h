@@ -38,7 +38,9 @@
  *     state; other pairs: GDR_ERR_DTYPE).
  *     Index arrays are int32.  Stores to bf16 round to nearest even, once.
  *   - The caller owns every buffer.  The library allocates no device memory
- *     and keeps no pointer after a call returns.  Work is enqueued on
+ *     and keeps no pointer after a call returns; the tensor-core prefill's
+ *     scratch is a caller-owned workspace sized by gdr_chunk_fwd_workspace().
+ *     Work is enqueued on
  *     `stream` (a cudaStream_t; NULL = the legacy default stream) and runs
  *     asynchronously: the call returns before the kernels finish.
  *   - Host-side argument checks run before anything is launched; on a non-zero
@@ -75,7 +77,8 @@ typedef enum gdr_status {
     GDR_ERR_ALIGN = 4,       /* a pointer is not 16-byte aligned */
     GDR_ERR_UNSUPPORTED = 5, /* valid per the API but not built: Dk or Dv not in {16,32,64,128} */
     GDR_ERR_DEVICE = 6,      /* no usable device, or it is not sm_100 */
-    GDR_ERR_LAUNCH = 7       /* a kernel launch or a CUDA call failed */
+    GDR_ERR_LAUNCH = 7,      /* a kernel launch or a CUDA call failed */
+    GDR_ERR_WORKSPACE = 8    /* ws_bytes is smaller than gdr_chunk_fwd_workspace() returns */
 } gdr_status;
 
 typedef enum gdr_dtype { GDR_F32 = 0, GDR_BF16 = 1, GDR_F16 = 2 } gdr_dtype;
@@ -131,6 +134,20 @@ typedef struct gdr_epilogue {
 } gdr_epilogue;
 
 /*
+ * Bytes of device workspace a gdr_chunk_fwd call with these sizes needs (0 if
+ * it needs none).  The tensor-core path (bf16 or fp16, Dk = Dv = 128) first
+ * solves the WY transform of every 64-token chunk at once and keeps, per
+ * (b, value head, chunk), the 64 x 64 matrix (I + A)^{-1} diag(beta) in the
+ * input dtype and six vectors of 64 floats (the chunk's gate and norm
+ * factors): B * Nv * ceil(S / 64) * (8192 + 1536) bytes.  Invalid sizes give
+ * 0 (the call itself reports them).  Source: the lite_boost
+ * chunk_gated_delta_rule operator (caller-owned buffers) and the order of
+ * torch_chunk_gated_delta_rule, which forms every chunk's attn/T solve before
+ * the inter-chunk loop.
+ */
+size_t gdr_chunk_fwd_workspace(int B, int Nk, int Nv, int S, int Dk, int Dv, gdr_dtype dtype);
+
+/*
  * Chunked prefill.  Source: lite_boost chunk_gated_delta_rule (arguments,
  * BNSD layout, GQA, variable lengths with padding written as zero, optional
  * gate, final state) and torch_chunk_gated_delta_rule (chunk size 64,
@@ -152,16 +169,26 @@ typedef struct gdr_epilogue {
  *   out                    device (B, Nv, S, Dv), written in full
  *   final_state            device (B, Nv, Dk, Dv) or NULL: not written.  It
  *                          may alias initial_state (in-place update).
+ *   workspace, ws_bytes    device scratch of at least
+ *                          gdr_chunk_fwd_workspace(B, Nk, Nv, S, Dk, Dv, dtype)
+ *                          bytes, owned by the caller, 16-byte aligned; NULL and
+ *                          0 when that is 0.  Its contents on entry do not
+ *                          matter and on return are unspecified; two calls in
+ *                          flight at once need separate workspaces.
  * Constraints: B, S >= 0; Nk, Nv >= 1; Nv % Nk == 0; Dk, Dv in {16,32,64,128};
  * every pointer 16-byte aligned.  An epilogue with a NULL z or norm_w returns
- * GDR_ERR_NULL, one with eps < 0 (or NaN) GDR_ERR_SHAPE.  bf16 or fp16 with
- * Dk = Dv = 128 runs on the tensor-core (tcgen05) path; other shapes and fp32
- * run the CUDA-core path.
+ * GDR_ERR_NULL, one with eps < 0 (or NaN) GDR_ERR_SHAPE.  A NULL workspace
+ * where one is needed returns GDR_ERR_NULL, a short one GDR_ERR_WORKSPACE.
+ * bf16 or fp16 with Dk = Dv = 128 runs on the tensor-core (tcgen05) path: the
+ * WY pass over all chunks, then one CTA per (b, value head) for the carry.
+ * Other shapes and fp32 run the CUDA-core path.  Without g (NULL, the
+ * operator's hasGamma = 0) a build without the gate arithmetic runs.
  */
 int gdr_chunk_fwd(const void *q, const void *k, const void *v, const void *beta, const float *g,
                   const void *initial_state, const int32_t *actual_seq_lengths, float scale, int B, int Nk,
                   int Nv, int S, int Dk, int Dv, gdr_dtype dtype, const gdr_prologue *prologue,
-                  const gdr_epilogue *epilogue, void *out, void *final_state, gdr_stream_t stream);
+                  const gdr_epilogue *epilogue, void *out, void *final_state, void *workspace, size_t ws_bytes,
+                  gdr_stream_t stream);
 
 /*
  * Recurrent decode over a pool of state slots.  Source: lite_boost
@@ -272,13 +299,36 @@ int gdr_prologue_apply(const void *q, const void *k, const void *b, const float 
                        void *q_hat, void *k_hat, void *beta, float *g, gdr_stream_t stream);
 
 /*
- * Waits for `stream`, then returns in *device_error the device error word
- * (GDR_DEVERR_* bits accumulated by every kernel of this library on the
- * current device since the last call) and clears it.  Returns GDR_OK or
- * GDR_ERR_LAUNCH if a CUDA call failed (including an earlier asynchronous
- * kernel fault on the stream).
+ * Returns in *device_error the device error word and clears it, in one atomic
+ * step on `stream` (after the work already enqueued there), then waits for
+ * the stream.  The word is one per device: it holds the GDR_DEVERR_* bits
+ * raised by every kernel of this library on the current device since it was
+ * last cleared, including kernels on other streams or from other host
+ * threads, so a caller that needs per-call attribution serialises its calls.
+ * Returns GDR_OK, or GDR_ERR_LAUNCH if a CUDA call failed (including an
+ * earlier asynchronous kernel fault on the stream).
  */
 int gdr_get_error(gdr_stream_t stream, int *device_error);
+
+/*
+ * Diagnostic hook for the bounded waits of the tensor-core prefill: their limit
+ * in nanoseconds for the calls that follow in this process (0 restores the
+ * default of one second).  A limit shorter than the kernel needs makes its
+ * waits run out: the kernel then drains its own copies and MMAs, returns early
+ * and sets GDR_DEVERR_TIMEOUT (outputs incomplete).  Used by the tests of that
+ * path; not for production use.  Always returns GDR_OK.
+ */
+int gdr_debug_set_wait_limit(unsigned long long ns);
+
+/*
+ * Diagnostic: waits for the device, then returns in *site (and clears) the
+ * record of the first bounded wait of the tensor-core prefill that ran out on
+ * the current device since the last read: 0 if none, else bit 31 set, the
+ * warp in bits 24-29, the kernel's barrier index in bits 16-23, the awaited
+ * phase parity in bit 15 and the CTA index (low 15 bits) in bits 0-14.
+ * Returns GDR_OK, GDR_ERR_NULL, GDR_ERR_DEVICE or GDR_ERR_LAUNCH.
+ */
+int gdr_debug_timeout_site(unsigned int *site);
 
 /* Static description of a status code; never NULL. */
 const char *gdr_status_string(int status);

@@ -30,7 +30,8 @@ _LIB_PATH = os.path.join(_BUILD, "libgdr_oracle.so")
 _lock = threading.Lock()
 _lib = None
 
-__all__ = ["build", "lib", "prologue", "chunk_fwd", "recurrent_step", "gated_rmsnorm", "causal_conv1d", "threads"]
+__all__ = ["build", "lib", "prologue", "chunk_fwd", "recurrent_step", "gated_rmsnorm", "causal_conv1d", "threads",
+           "set_threads"]
 
 
 def build(force: bool = False) -> str:
@@ -64,6 +65,8 @@ def lib() -> ctypes.CDLL:
                                                     c_int, c_int, c_int, c_int, c_int, c_int, dp]
             L.gdr_oracle_threads.restype = c_int
             L.gdr_oracle_threads.argtypes = []
+            L.gdr_oracle_set_threads.restype = None
+            L.gdr_oracle_set_threads.argtypes = [c_int]
             _lib = L
     return _lib
 
@@ -95,6 +98,11 @@ def _ip(a):
 def threads() -> int:
     """OpenMP threads the C oracle runs with."""
     return int(lib().gdr_oracle_threads())
+
+
+def set_threads(n: int) -> None:
+    """OpenMP threads of later oracle calls (the results do not depend on it)."""
+    lib().gdr_oracle_set_threads(int(n))
 
 
 def prologue(q=None, k=None, b=None, a=None, A_log=None, dt_bias=None, eps: float = 1e-6):

@@ -297,6 +297,17 @@ int gdr_oracle_recurrent_step(const double *q, const double *k, const double *v,
     return status;
 }
 
+/* Sets the number of OpenMP threads of later calls (for a single-thread timing); n < 1 is ignored.  The
+ * results do not depend on it: every chain is computed in the same fixed order. */
+void gdr_oracle_set_threads(int n) {
+#ifdef _OPENMP
+    extern void omp_set_num_threads(int);
+    if (n >= 1) omp_set_num_threads(n);
+#else
+    (void)n;
+#endif
+}
+
 /* Number of OpenMP threads the oracle will use (reported with timings). */
 int gdr_oracle_threads(void) {
 #ifdef _OPENMP

@@ -44,17 +44,17 @@ def test_header_codes_match_the_binding():
     enums = dict((n, int(v)) for n, v in re.findall(r"\b(GDR_[A-Z0-9_]+)\s*=\s*(\d+)", src))
     defines = dict((n, int(v, 16)) for n, v in re.findall(r"#define\s+(GDR_DEVERR_[A-Z_]+)\s+(0x[0-9a-fA-F]+)u", src))
     for name in ("GDR_OK", "GDR_ERR_SHAPE", "GDR_ERR_DTYPE", "GDR_ERR_NULL", "GDR_ERR_ALIGN", "GDR_ERR_UNSUPPORTED",
-                 "GDR_ERR_DEVICE", "GDR_ERR_LAUNCH", "GDR_F32", "GDR_BF16", "GDR_F16"):
+                 "GDR_ERR_DEVICE", "GDR_ERR_LAUNCH", "GDR_ERR_WORKSPACE", "GDR_F32", "GDR_BF16", "GDR_F16"):
         assert enums[name] == getattr(gdr, name), name
     assert defines == {"GDR_DEVERR_SLOT_INDEX": gdr.DEVERR_SLOT_INDEX, "GDR_DEVERR_LENGTH": gdr.DEVERR_LENGTH,
                        "GDR_DEVERR_TIMEOUT": gdr.DEVERR_TIMEOUT}, defines
 
 
 def test_status_strings_and_version(L):
-    for s in range(8):
-        assert L.gdr_status_string(s)
+    for s in range(9):
+        assert L.gdr_status_string(s) and b"unknown" not in L.gdr_status_string(s)
     assert b"unknown" in L.gdr_status_string(99)
-    assert gdr.version() == 100
+    assert gdr.version() == 200
 
 
 P = ctypes.c_void_p(4096)  # placeholder: aligned, non-NULL, never dereferenced (every call is rejected first)
@@ -63,11 +63,11 @@ NUL = None
 
 def chunk(L, **kw):
     a = dict(q=P, k=P, v=P, beta=P, g=NUL, s0=NUL, lens=NUL, scale=1.0, B=1, Nk=2, Nv=4, S=8, Dk=128, Dv=128,
-             dt=gdr.GDR_BF16, pro=None, epi=None, out=P, fin=NUL)
+             dt=gdr.GDR_BF16, pro=None, epi=None, out=P, fin=NUL, ws=P, ws_bytes=1 << 40)
     a.update(kw)
     return L.gdr_chunk_fwd(a["q"], a["k"], a["v"], a["beta"], a["g"], a["s0"], a["lens"], a["scale"], a["B"],
                            a["Nk"], a["Nv"], a["S"], a["Dk"], a["Dv"], a["dt"], a["pro"], a["epi"], a["out"], a["fin"],
-                           None)
+                           a["ws"], a["ws_bytes"], None)
 
 
 def decode(L, **kw):
@@ -105,8 +105,25 @@ def test_chunk_host_validation(L):
     assert chunk(L, epi=ctypes.byref(epi)) == gdr.GDR_ERR_SHAPE
     epi = gdr.GdrEpilogueStruct(4104, 4096, 1e-6)  # misaligned z
     assert chunk(L, epi=ctypes.byref(epi)) == gdr.GDR_ERR_ALIGN
+    # the tensor-core path's workspace: required, large enough, aligned
+    assert chunk(L, ws=NUL) == gdr.GDR_ERR_NULL
+    need = L.gdr_chunk_fwd_workspace(1, 2, 4, 8, 128, 128, gdr.GDR_BF16)
+    assert chunk(L, ws_bytes=need - 1) == gdr.GDR_ERR_WORKSPACE
+    assert chunk(L, ws=ctypes.c_void_p(4104)) == gdr.GDR_ERR_ALIGN
     # nothing to do: B == 0 returns OK without touching a device
-    assert chunk(L, B=0, q=NUL, k=NUL, v=NUL, beta=NUL, out=NUL) == gdr.GDR_OK
+    assert chunk(L, B=0, q=NUL, k=NUL, v=NUL, beta=NUL, out=NUL, ws=NUL, ws_bytes=0) == gdr.GDR_OK
+
+
+def test_workspace_size(L):
+    """Per (b, value head, 64-token chunk): the 64 x 64 16-bit T' and six vectors of 64 floats, for the tensor-core
+    path only (bf16 or fp16, Dk = Dv = 128); zero for the CUDA-core path and for invalid sizes."""
+    per = 64 * 64 * 2 + 6 * 64 * 4
+    assert L.gdr_chunk_fwd_workspace(4, 16, 32, 4096, 128, 128, gdr.GDR_BF16) == 4 * 32 * 64 * per
+    assert L.gdr_chunk_fwd_workspace(2, 1, 3, 65, 128, 128, gdr.GDR_F16) == 2 * 3 * 2 * per
+    assert L.gdr_chunk_fwd_workspace(2, 1, 3, 65, 128, 128, gdr.GDR_F32) == 0
+    assert L.gdr_chunk_fwd_workspace(2, 1, 3, 65, 64, 64, gdr.GDR_BF16) == 0
+    assert L.gdr_chunk_fwd_workspace(0, 1, 3, 65, 128, 128, gdr.GDR_BF16) == 0
+    assert L.gdr_chunk_fwd_workspace(2, 2, 3, 65, 128, 128, gdr.GDR_BF16) == 0  # Nv % Nk != 0
 
 
 def test_decode_host_validation(L):
@@ -118,6 +135,9 @@ def test_decode_host_validation(L):
     assert decode(L, pool=NUL) == gdr.GDR_ERR_NULL
     assert decode(L, idx=NUL) == gdr.GDR_ERR_NULL
     assert decode(L, lens=NUL) == gdr.GDR_ERR_NULL
+    # the pool's (slot, head) tiles are addressed in 32-bit arithmetic
+    assert decode(L, slots=(1 << 31) // 4, Nv=4, Nk=2) == gdr.GDR_ERR_SHAPE
+    assert decode(L, slots=(1 << 31) // 4 - 1, Nv=4, Nk=2, pool=NUL) == gdr.GDR_ERR_NULL
     assert decode(L, gk=ctypes.c_void_p(4100)) == gdr.GDR_ERR_ALIGN
     assert decode(L, Dk=48) == gdr.GDR_ERR_UNSUPPORTED
     assert decode(L, dt=gdr.GDR_F16, sdt=gdr.GDR_BF16) == gdr.GDR_ERR_DTYPE  # fp16 inputs: fp16 or fp32 state
