@@ -31,7 +31,7 @@ GDR_F32, GDR_BF16, GDR_F16 = 0, 1, 2
 DEVERR_SLOT_INDEX, DEVERR_LENGTH, DEVERR_TIMEOUT = 0x1, 0x2, 0x4
 
 # Every symbol the C header declares (checked by the ABI test).
-EXPORTED = ("gdr_chunk_fwd_workspace", "gdr_chunk_fwd", "gdr_recurrent_step", "gdr_recurrent_step_spec", "gdr_conv1d",
+EXPORTED = ("gdr_chunk_fwd_workspace", "gdr_chunk_fwd", "gdr_chunk_fwd_noalloc", "gdr_recurrent_step", "gdr_recurrent_step_spec", "gdr_conv1d",
             "gdr_prologue_apply", "gdr_get_error", "gdr_debug_set_wait_limit", "gdr_debug_timeout_site",
             "gdr_status_string", "gdr_version")
 
@@ -66,6 +66,10 @@ def lib() -> ctypes.CDLL:
         L.gdr_chunk_fwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, f32, i32, i32, i32, i32, i32, i32, i32,
                                     ctypes.POINTER(GdrPrologueStruct), ctypes.POINTER(GdrEpilogueStruct), vp, vp, vp,
                                     ctypes.c_size_t, vp]
+        L.gdr_chunk_fwd_noalloc.restype = i32
+        L.gdr_chunk_fwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, f32, i32, i32, i32, i32, i32, i32, i32,
+                                            ctypes.POINTER(GdrPrologueStruct), ctypes.POINTER(GdrEpilogueStruct),
+                                            vp, vp, vp]
         L.gdr_recurrent_step.restype = i32
         L.gdr_recurrent_step.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, vp, vp, vp, f32, i32, i32, i32, i32, i32,
                                          i32, i32, i32, ctypes.POINTER(GdrPrologueStruct),

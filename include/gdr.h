@@ -191,6 +191,36 @@ int gdr_chunk_fwd(const void *q, const void *k, const void *v, const void *beta,
                   gdr_stream_t stream);
 
 /*
+ * The chunked prefill for callers that cannot allocate device memory: code in
+ * a framework hook or plug-in that only receives one operation's tensors, a
+ * serving loop whose memory is all reserved by its own pool, a runtime with no
+ * allocator to call on this path.  It takes the arguments of gdr_chunk_fwd
+ * without workspace and ws_bytes, and computes the same result; the scratch
+ * the tensor-core path needs is instead a fixed 16 MiB array compiled into the
+ * library (one per GPU that loads the library, held until the process exits).
+ * No passage of the operator pages corresponds to this entry point: it exists
+ * for the memory discipline of such callers.
+ *   - It allocates nothing: no cudaMalloc, cudaFree or allocating library call.
+ *   - Sizes whose workspace (gdr_chunk_fwd_workspace) exceeds 16 MiB, that is
+ *     B * Nv * ceil(S / 64) > 1724 on the tensor-core path, return
+ *     GDR_ERR_WORKSPACE without launching anything.  The CUDA-core path needs
+ *     no scratch and has no such limit.
+ *   - Every call shares the one array per device, so two calls that overlap on
+ *     the GPU (on different streams, or from different host threads, without
+ *     ordering between them) race and give wrong results.  Calls ordered on one
+ *     stream are fine; the array keeps the last call's contents, which no later
+ *     call depends on.
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture.
+ * Other arguments, checks, layouts and errors are those of gdr_chunk_fwd.
+ */
+int gdr_chunk_fwd_noalloc(const void *q, const void *k, const void *v, const void *beta, const float *g,
+                          const void *initial_state, const int32_t *actual_seq_lengths, float scale, int B, int Nk,
+                          int Nv, int S, int Dk, int Dv, gdr_dtype dtype, const gdr_prologue *prologue,
+                          const gdr_epilogue *epilogue, void *out, void *final_state, gdr_stream_t stream);
+
+/*
  * Recurrent decode over a pool of state slots.  Source: lite_boost
  * recurrent_gated_delta_rule (state pool, ssm_state_indices with one slot per
  * flattened token, gk, num_accepted_tokens, S <= 8, the decay
