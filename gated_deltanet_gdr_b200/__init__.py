@@ -33,6 +33,7 @@ DEVERR_SLOT_INDEX, DEVERR_LENGTH, DEVERR_TIMEOUT = 0x1, 0x2, 0x4
 # Every symbol the C header declares (checked by the ABI test).
 EXPORTED = ("gdr_chunk_fwd_workspace", "gdr_chunk_fwd", "gdr_chunk_fwd_noalloc", "gdr_recurrent_step", "gdr_recurrent_step_spec", "gdr_conv1d",
             "gdr_prologue_apply", "gdr_get_error", "gdr_debug_set_wait_limit", "gdr_debug_timeout_site",
+            "gdr_debug_set_chunk_schedule",
             "gdr_status_string", "gdr_version")
 
 
@@ -87,6 +88,8 @@ def lib() -> ctypes.CDLL:
         L.gdr_debug_set_wait_limit.argtypes = [ctypes.c_ulonglong]
         L.gdr_debug_timeout_site.restype = i32
         L.gdr_debug_timeout_site.argtypes = [ctypes.POINTER(ctypes.c_uint)]
+        L.gdr_debug_set_chunk_schedule.restype = i32
+        L.gdr_debug_set_chunk_schedule.argtypes = [i32]
         L.gdr_status_string.restype = ctypes.c_char_p
         L.gdr_status_string.argtypes = [i32]
         L.gdr_version.restype = i32
@@ -208,7 +211,8 @@ def _chunk_checked(q, k, v, beta, g, initial_state, actual_seq_lengths, prologue
 
 
 def chunk_fwd_workspace_bytes(B: int, Nk: int, Nv: int, S: int, Dk: int, Dv: int, dtype: torch.dtype) -> int:
-    """Bytes of workspace ``gdr_chunk_fwd`` needs for these sizes (``gdr_chunk_fwd_workspace``)."""
+    """Bytes of workspace the fastest schedule of ``gdr_chunk_fwd`` wants for these sizes
+    (``gdr_chunk_fwd_workspace``; 0 when it wants none)."""
     return int(lib().gdr_chunk_fwd_workspace(B, Nk, Nv, S, Dk, Dv, _dtype_code(dtype)))
 
 
@@ -229,7 +233,7 @@ def chunk_fwd(q, k, v, beta, g=None, initial_state=None, actual_seq_lengths=None
               prologue: Optional[Prologue] = None, epilogue: Optional[Epilogue] = None, out=None, final_state=None,
               output_final_state: bool = True, workspace=None, stream=None):
     """Chunked prefill (``gdr_chunk_fwd``).  Returns (out, final_state or None).  ``workspace`` (uint8, at least
-    ``chunk_fwd_workspace_bytes`` bytes) is allocated per call when not given."""
+    ``chunk_fwd_workspace_bytes`` bytes) is allocated per call when not given and the sizes ask for one."""
     out, final_state = _chunk_checked(q, k, v, beta, g, initial_state, actual_seq_lengths, prologue, out,
                                       final_state, output_final_state)
     B, Nk, S, Dk = q.shape
@@ -461,6 +465,16 @@ def take_timeout_site() -> dict:
     if not x:
         return {}
     return {"warp": (x >> 24) & 0x3F, "barrier": (x >> 16) & 0xFF, "parity": (x >> 15) & 1, "cta": x & 0x7FFF}
+
+
+# schedules of the tensor-core prefill for ``set_chunk_schedule``
+SCHEDULE_AUTO, SCHEDULE_ONE_KERNEL, SCHEDULE_TWO_KERNELS = 0, 1, 2
+
+
+def set_chunk_schedule(schedule: int) -> None:
+    """Diagnostic: which schedule of the tensor-core prefill the workspace query sizes for later calls
+    (``gdr_debug_set_chunk_schedule``): SCHEDULE_AUTO by shape, or one of the two always."""
+    _check(lib().gdr_debug_set_chunk_schedule(int(schedule)), "gdr_debug_set_chunk_schedule")
 
 
 def set_wait_limit_ns(ns: int) -> None:

@@ -35,7 +35,40 @@ unsigned int *g_err_ptr[kMaxDevices];  // device address of g_device_error per d
 unsigned int *g_snap_ptr[kMaxDevices]; // device address of g_error_snapshot per device
 unsigned int g_snap_next = 0;          // next snapshot slot (under g_mu)
 
+int g_sm_count[kMaxDevices];           // multiprocessors per device (0 until first asked)
+int g_chunk_schedule = 0;              // tensor-core prefill schedule: 0 by shape, 1 one kernel, 2 two kernels
+
 bool supported_head(int d) { return d == 16 || d == 32 || d == 64 || d == 128; }
+
+// Multiprocessors of the current device; 148 (a full B200) when no device can be asked, so that the workspace
+// query answers the same on a machine without a GPU.
+int sm_count() {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+        cudaGetLastError();
+        return 148;
+    }
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (g_sm_count[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
+            cudaGetLastError();
+            return 148;
+        }
+        g_sm_count[dev] = n;
+    }
+    return g_sm_count[dev];
+}
+
+// The tensor-core prefill's two-kernel schedule (a WY pass over every chunk on every SM, then the chains) pays
+// off when the (b, value head) chains occupy at most a third of the SMs: the one-kernel schedule would leave the
+// rest idle while each chain solves its chunks' WY systems in turn.  With more chains the one-kernel schedule,
+// which needs no workspace, is faster.
+bool two_kernel_schedule(int B, int Nv) {
+    if (g_chunk_schedule == 1) return false;
+    if (g_chunk_schedule == 2) return true;
+    return (long long)B * Nv * 3 <= sm_count();
+}
 bool aligned16(const void *p) { return p == nullptr || (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 // Checks the current device once (sm_100 family) and fetches the address of the error
@@ -171,7 +204,7 @@ using namespace gdr;
 extern "C" size_t gdr_chunk_fwd_workspace(int B, int Nk, int Nv, int S, int Dk, int Dv, gdr_dtype dtype) {
     if (check_common(B, Nk, Nv, S, Dk, Dv, dtype) != GDR_OK) return 0;
     if ((long long)B * S == 0 || !chunk_tc_supported(Dk, Dv, dtype, S)) return 0;
-    return chunk_tc_workspace(B, Nv, S);
+    return two_kernel_schedule(B, Nv) ? chunk_wy_workspace(B, Nv, S) : 0;
 }
 
 extern "C" int gdr_chunk_fwd(const void *q, const void *k, const void *v, const void *beta, const float *g,
@@ -187,9 +220,10 @@ extern "C" int gdr_chunk_fwd(const void *q, const void *k, const void *v, const 
     const void *ptrs[] = {q, k, v, beta, g, initial_state, actual_seq_lengths, out, final_state, workspace};
     for (const void *p : ptrs)
         if (!aligned16(p)) return GDR_ERR_ALIGN;
+    // a workspace of at least the queried size selects the two-kernel schedule where the query asks for one; no
+    // workspace runs the one-kernel schedule, which needs none
     const size_t need = gdr_chunk_fwd_workspace(B, Nk, Nv, S, Dk, Dv, dtype);
-    if (need > 0 && !workspace) return GDR_ERR_NULL;
-    if (ws_bytes < need) return GDR_ERR_WORKSPACE;
+    if (workspace && ws_bytes < need) return GDR_ERR_WORKSPACE;
     if (B == 0 || (S == 0 && !final_state)) return GDR_OK;
     unsigned int *err = nullptr;
     if ((st = device_setup(&err))) return st;
@@ -217,7 +251,7 @@ extern "C" int gdr_chunk_fwd(const void *q, const void *k, const void *v, const 
             a.epi_w = epilogue->norm_w;
             a.epi_eps = epilogue->eps;
         }
-        e = launch_chunk_tc(a, dtype, cs);
+        e = (need > 0 && workspace) ? launch_chunk_wy(a, dtype, cs) : launch_chunk_tc(a, dtype, cs);
     } else {
         e = launch_chunk_simt(a, Dk, Dv, dtype, cs);
         if (e == cudaSuccess && epilogue && S > 0)
@@ -396,5 +430,15 @@ extern "C" int gdr_debug_timeout_site(unsigned int *site) {
     unsigned int *err = nullptr;
     int st = device_setup(&err);
     if (st) return st;
-    return chunk_tc_take_timeout_site(site) == cudaSuccess ? GDR_OK : GDR_ERR_LAUNCH;
+    unsigned int one = 0, two = 0;
+    if (chunk_tc_take_timeout_site(&one) != cudaSuccess || chunk_wy_take_timeout_site(&two) != cudaSuccess)
+        return GDR_ERR_LAUNCH;
+    *site = one ? one : two;
+    return GDR_OK;
+}
+
+extern "C" int gdr_debug_set_chunk_schedule(int schedule) {
+    if (schedule < 0 || schedule > 2) return GDR_ERR_SHAPE;
+    g_chunk_schedule = schedule;
+    return GDR_OK;
 }

@@ -1,45 +1,38 @@
-// chunk_tc.cu -- chunked prefill of the gated delta rule on the sm_100a tensor cores (bf16 or fp16 in and out,
-// Dk = Dv = 128, chunk C = 64), in two kernels.
+// chunk_tc.cu -- chunked prefill of the gated delta rule on the sm_100a tensor cores.
 //
-// The chunked (WY / UT transform) form of torch_chunk_gated_delta_rule (blog "gated-delta-net" page, steps
-// 1-8).  Everything that does not depend on the state is independent per chunk, so it runs first, over all
-// chunks at once; only the state carry is serial.
+// The chunked (WY / UT transform) form of torch_chunk_gated_delta_rule (blog
+// "gated-delta-net" page, steps 1-8), chunk C = 64, head size Dk = Dv = 128, bf16 or fp16
+// in and out (the MMA operand copies in the same type), fp32 accumulation and an fp32 state.  One CTA owns one (b, value head)
+// chain.  Per chunk:
 //
-//   wy_kernel (one CTA per (sequence, key head, chunk), every SM, several CTAs per SM):
-//     a0  the fused prologue: beta = sigmoid(b), g = -e^{A_log} softplus(a + dt_bias), 1/|k| (eps inside the
-//         root, from the diagonal of the Gram)
-//     a1  G_t = cumulative log-gate inside the chunk (tokens past the length count 0)
-//     a2  Gram K K^T of the raw keys (warp-level bf16/fp16 tensor-core MMAs, fp32 accumulation)
-//     a3  A = strictLower(beta_t k_t.k_s e^{G_t-G_s}) with unit keys;  T = (I + A)^{-1}: 16 x 16 diagonal
-//         blocks by forward substitution, the 16 -> 32 merges on the CUDA cores, the 32 -> 64 merge on tf32
-//         warp MMAs
-//     and writes, per (b, value head, chunk), into the caller's workspace: T' = T diag(beta) (16-bit,
-//     row-major 64 x 64) and six vectors of 64 floats (e^G, e^G/|k|, e^{G_last-G}/|k|, G log2 e,
-//     G log2 e - log2(1/|k|), and [e^{G_last}, valid count]).
+//   a1  G_t = cumulative log-gate (tokens past the length count 0).
+//   a2  [G; P] = [K; Q] K^T                       tcgen05.mma  M=128 N=64  K=128
+//   a3  A = strictLower(beta_t k_t.k_s e^{G_t-G_s});  T = (I + A)^{-1}: 16x16 diagonal blocks by
+//       forward substitution and the 16 -> 32 merges T21 = -T22 A21 T11 in fp32 on the CUDA
+//       cores, the 32 -> 64 merge with warp-level tf32 tensor-core MMAs (mma.sync m16n8k8,
+//       operands and products in registers).
+//   a4  W = T diag(beta e^G) K,  U = T diag(beta) V        tcgen05.mma  M=128 N=128 K=64
+//   a5  R = [W; diag(e^G) X] S                    tcgen05.mma  M=128 N=128 K=128
+//       v_new = U - R[0:64]
+//       S <- e^{G_last} S  (in TMEM, while R is computed)
+//       S += (diag(e^{G_last-G}) K)^T v_new       tcgen05.mma  accumulate into the TMEM state
+//       R[64:128] += Pm v_new,  Pm = (X K^T) e^{G_t-G_s} (causal)  -> o
+//   a6  o -> bf16 -> TMA store; padding rows and chunks are zero; the final state is
+//       written once from TMEM.  With the optional epilogue each o row first becomes
+//       o / sqrt(mean o^2 + eps) * norm_w * silu(z) in fp32 (the layer's gated RMSNorm).
 //
-//   chain_kernel (one CTA per (b, value head) chain): per chunk, with the state held TRANSPOSED in tensor
-//   memory (lane = value column j, columns = key row i, fp32) so that the state and v_new are the A operand
-//   of the tensor core straight from TMEM:
-//     a4  U^T = V^T T'^T                                     tcgen05 M=128 (dv) N=64 (t) K=64
-//         W^T = K^T (T' diag(e^G/|k|))^T                     tcgen05 M=128 (dk) N=64 K=64
-//     a5  v_new^T = U^T - S^T W^T                            tcgen05, A = S^T (bf16 copy in TMEM)
-//         o^T     = S^T Q~^T + v_new^T Pm^T                  Q~ = diag(e^G) Q, Pm = causal
-//                                                            q_t.k_s/|k_s| e^{G_t-G_s}; the row factor
-//                                                            scale/|q_t| is applied to o afterwards
-//         S^T     = e^{G_last} S^T + (v_new diag(c))^T K     c_t = e^{G_last-G_t}/|k_t| folded into the
-//                                                            16-bit copy of v_new (A from TMEM), K raw
-//     a6  o -> dtype -> TMA store (padding rows and chunks zero); the final state written once from TMEM.
-//   The serial chain per chunk is MMA -> v_new (TMEM -> registers -> TMEM) -> MMA -> S (TMEM -> registers ->
-//   TMEM): no shared-memory round trip and no proxy fence on it.  The other products run on the tensor pipe
-//   while the carry warps convert.
+// X = scale * q / |q| (the fused l2norm and the 1/|k| factors are folded into row and
+// column scalings, so the raw q/k tiles feed the tensor cores directly).
 //
-// Warp roles of chain_kernel: warps 0-7 carry (the two conversions of the chain, the initial and final
-// state), 8-11 out (1/|q| and Q~ of the next chunk; o rows -> out tile, the optional gated RMSNorm epilogue,
-// TMA stores), 12-15 prep (W^T, Pm and T' diag(e^G/|k|) of the next chunk, padding rows), 16 MMA issue (one
-// thread issues every tcgen05.mma; the products of the next chunk go in when their operands are ready, never
-// ahead of the chain's own), 17 TMA loads.  Hand-offs are mbarriers; every wait is bounded by elapsed time and gives up
-// when another group has stopped, after which the CTA drains its own copies and MMAs, sets the timeout bit
-// of the device error word, releases TMEM and returns.
+// Warp roles: warps 0-7 ("carry") run the serial chain of chunk c -- the three MMAs that
+// touch the state and their epilogues; warps 8-15 ("prep") meanwhile prepare chunk c+1
+// (tile loads, norms, gate scan, [G; P], the solve, W and U, the X_g and K~ operands).
+// They hand over through mbarriers: a1_ready (prep -> carry: operands of chunk c are in
+// place) and mma2_done (carry -> prep: the MMAs of chunk c-1 that read the shared
+// operand buffers have completed).  Every wait is bounded by elapsed time and gives up early once another group
+// has stopped; then the CTA waits for its own copies and MMAs still in flight, sets the timeout bit of the device
+// error word, releases TMEM and returns.  Stop decisions inside a group are collective (bar.red.or at the group's
+// hand-offs), so every member leaves its loop at the same barrier.
 #include <cuda.h>
 
 #include "common.cuh"
@@ -49,54 +42,151 @@
 namespace gdr {
 using namespace sm100;
 
-// The first bounded wait of the chain kernel that ran out since the word was last read (0: none): bit 31 set,
-// the warp in bits 24-29, the barrier in bits 16-23, its phase parity in bit 15, the CTA in bits 0-14.
+namespace {
+// The first bounded wait of the one-kernel schedule that ran out since the word was last read (0: none): bit 31
+// set, the warp in bits 24-29, the barrier in bits 16-23, its phase parity in bit 15, the CTA in bits 0-14.
 __device__ unsigned int g_timeout_site = 0;
+constexpr uint64_t kDefaultWaitNs = 1000000000ull;  // a bounded wait gives up after 1 s
+constexpr uint64_t kDrainWaitNs = 1000000000ull;    // waits for the CTA's own copies and MMAs at the exit
+unsigned long long g_wait_ns = 0;                   // 0: the default limit (a test may shorten it)
+}  // namespace
+
+void chunk_tc_set_wait_ns(unsigned long long ns) { g_wait_ns = ns; }
+unsigned long long chunk_wait_ns() { return g_wait_ns ? g_wait_ns : kDefaultWaitNs; }
+cudaError_t chunk_tc_take_timeout_site(unsigned int *site) {
+    unsigned int zero = 0;
+    cudaError_t e = cudaMemcpyFromSymbol(site, g_timeout_site, sizeof(unsigned int));
+    if (e == cudaSuccess) e = cudaMemcpyToSymbol(g_timeout_site, &zero, sizeof(unsigned int));
+    return e;
+}
 
 #ifdef GDR_PHASE_TIMERS
-// Development aid, compiled only with -DGDR_PHASE_TIMERS (never in the library the package builds): cycles the
-// first thread of each role of CTA 0 spends blocked in each barrier wait, [role][barrier] with roles carry, out,
-// prep, MMA, TMA; then the CTA's total cycles and its chunk count.  Read by gdr_phase_timers_read.
-constexpr int kTimerSlots = 5 * 36 + 2;
-__device__ unsigned long long g_phase[kTimerSlots];
-// and a timeline of chunks kEvC0 .. kEvC0 + kEvN - 1 of CTA 0: clock64 at 16 hand-off / issue events per chunk
-constexpr int kEvC0 = 8, kEvN = 8, kEvK = 16;
-__device__ long long g_events[kEvN * kEvK];
-#define EVENT(chunk, k)                                                                       \
-    do {                                                                                      \
-        if (blockIdx.x == 0 && (chunk) >= kEvC0 && (chunk) < kEvC0 + kEvN)                    \
-            g_events[((chunk) - kEvC0) * kEvK + (k)] = clock64();                             \
+// Development aid, compiled only with -DGDR_PHASE_TIMERS: clock64() cycles per phase, summed
+// in shared memory (so that taking a time stalls nothing) and added to g_phase by CTA 0 at
+// the end; slots 0..15 prep group, 16..31 carry group; read by gdr_phase_timers_read.
+__device__ unsigned long long g_phase[64];
+#define PHASE(slot)                                                            \
+    do {                                                                       \
+        if (tid == 0 || tid == NGRP) {                                         \
+            const unsigned long long now_ = clock64();                         \
+            s_phase_[(slot)] += now_ - t_prev_;                                \
+            t_prev_ = now_;                                                    \
+        }                                                                      \
     } while (0)
+// cycles one thread spends in the statements, accumulated into `slot`
+#define TIMED(slot, ...)                                                       \
+    do {                                                                       \
+        const unsigned long long t0_ = clock64();                              \
+        __VA_ARGS__;                                                           \
+        s_phase_[(slot)] += clock64() - t0_;                                   \
+    } while (0)
+#define SOLVE_TIMER_ARGS , unsigned long long &t_prev_, int tid, unsigned long long *s_phase_
+#define SOLVE_TIMER_PASS , t_prev_, tid, s_phase_
 #else
-#define EVENT(chunk, k) \
-    do {                \
+#define PHASE(slot) \
+    do {            \
     } while (0)
+#define TIMED(slot, ...) \
+    do {                 \
+        __VA_ARGS__;     \
+    } while (0)
+#define SOLVE_TIMER_ARGS
+#define SOLVE_TIMER_PASS
 #endif
 
 namespace {
 
-constexpr int C = 64, D = 128;
-constexpr uint64_t kDefaultWaitNs = 1000000000ull;  // a bounded wait gives up after 1 s
-constexpr uint64_t kDrainWaitNs = 1000000000ull;    // waits for the CTA's own copies and MMAs when it stops
+// warps 0-7 carry, 8-15 prep, 16 control (TMA loads and the prep MMAs), 17-19 helpers (the K~ operand).  The
+// register file is allocated to warps in groups of four, so the helpers cost no registers per thread.
+constexpr int C = 64, D = 128, NGRP = 256, NHELP = 96, NT = 2 * NGRP + 32 + NHELP, NPC = NGRP + 32;
+constexpr int CTL_WARP = 16;
+// BAR_PCTL: the prep warps and the control warp, at the hand-offs between them; BAR_HELP: the helper warps
+// BAR_EPI: the carry warps that hold o rows (TMEM lanes 64..127), at the epilogue's row-norm exchange
+constexpr int BAR_CARRY = 1, BAR_PREP = 2, BAR_PCTL = 3, BAR_HELP = 4, BAR_EPI = 5;
+// carry thread that issues the out-tile TMA stores (thread 0 issues the carry's MMAs)
+constexpr int kStorer = 32;
 
-// ---- workspace (per (b, value head, chunk): T' then, in a second region, the vectors) ----
-constexpr size_t kTpBytes = (size_t)C * C * 2;
-constexpr int kNumVec = 6;
-constexpr size_t kVecBytes = (size_t)kNumVec * C * 4;
-// V_EG = e^{G_t}; V_CW = e^{G_t}/|k_t| (column factor of T' for W); V_CT = e^{G_last - G_t}/|k_t| (row factor
-// of K~); V_G2 = G_t log2 e; V_LAM = V_G2 - log2(1/|k_t|) (so that e^{G_t - G_s}/|k_s| = 2^{V_G2[t] - V_LAM[s]});
-// V_MISC[0] = e^{G_last}, V_MISC[1] = the chunk's valid-token count.  Entries past the length: 1/|k| = 0.
-enum { V_EG = 0, V_CW, V_CT, V_G2, V_LAM, V_MISC };
+// ---- shared memory map (bytes from a 1024-aligned base) ----
+// input tiles of the prep group, 64 rows x 128 B (64 bf16) each, per dk block b (b = 0, 1) at 24 KB b:
+// [K even chunk | Q | K odd chunk], so that [K; Q] (even chunks) and [Q; K] (odd chunks) are each one
+// 128-row operand for the Gram; the K tile is double-buffered so that the next chunk's K and Q can land
+// during the current chunk.  V (dv blocks at +0, +8K) is single-buffered: it is needed late.
+constexpr uint32_t KQ_BLK = 24576, OFF_V = 49152;
+__host__ __device__ constexpr uint32_t off_k(int par, int blk) { return blk * KQ_BLK + (par ? 16384u : 0u); }
+__host__ __device__ constexpr uint32_t off_q(int blk) { return blk * KQ_BLK + 8192u; }
+__host__ __device__ constexpr uint32_t off_gram(int par, int blk) { return blk * KQ_BLK + (par ? 8192u : 0u); }
+// operands of the carry group for the chunk it runs
+constexpr uint32_t OFF_A1 = 65536;   // [W; Q] K-major 128 x 128: dk blocks at +0, +16K (Q rows by TMA)
+constexpr uint32_t OFF_KT = 98304;   // K tile by TMA, scaled in place to diag(tail) K: MN-major (M = dk,
+                                     // K = tok), dk blocks at +0, +8K
+constexpr uint32_t OFF_S = 114688;   // S bf16, MN-major (K = dk rows, N = dv): dv blocks at +0, +16K
+// Pm (K-major 64 x 64), two buffers; the o MMA reads 128 rows starting 8 KB before the buffer so that
+// Pm forms rows 64..127 (rows 0..63 are whatever precedes it and land in dead accumulator lanes)
+constexpr uint32_t OFF_PM0 = 147456, OFF_PM1 = 155648;
+constexpr uint32_t OFF_VO = 163840;  // v_new (MN-major, K = tok, N = dv), then the out tile: dv blocks +0, +8K
+// the solve T = (I + A)^{-1} (see solve_diag16_merge and the prep group's a3 step)
+constexpr int SP = 36;                 // row stride (floats) of the plain 32 x 32 blocks: 16-byte aligned rows
+constexpr uint32_t OFF_TT = 180224;   // TT = [T diag(beta); T diag(c_W)], bf16, K-major 128 x 64; until it is
+                                      // written it holds the diagonal blocks of A (plain) and the merge scratch
+constexpr uint32_t OFF_AP = OFF_TT;              // A11, A22 (plain, 2 x 32 rows of SP floats)
+constexpr uint32_t OFF_XP = OFF_TT + 64 * SP * 4;  // 16 x 16 merge scratch (2 x 16 rows of SP floats)
+constexpr uint32_t OFF_TP = 196608;   // T11, T22 (plain, 2 x 32 rows of SP floats)
+constexpr uint32_t OFF_A21 = 205824;  // A rows 32..63, columns 0..31 (plain, 32 rows of SP floats)
+constexpr uint32_t OFF_XM = 210432;   // X = A21 T11 of the 32 -> 64 merge (plain, 32 rows of SP floats)
+static_assert(OFF_XP + 32 * SP * 4 <= OFF_TT + 16384, "plain A and the merge scratch fit in the TT area");
+static_assert(OFF_TP + 64 * SP * 4 <= OFF_A21 && OFF_A21 + 32 * SP * 4 <= OFF_XM, "plain T, A21");
+constexpr int NVEC = 11;             // per-chunk vectors of 64 floats (enum below)
+constexpr uint32_t OFF_VEC = 215040;  // 2 sets x NVEC vectors x 64 floats
+static_assert(OFF_XM + 32 * SP * 4 <= OFF_VEC, "merge product");
+constexpr uint32_t OFF_BAR = OFF_VEC + 2 * NVEC * 64 * 4;
+constexpr uint32_t OFF_EPI = OFF_BAR + 128;  // epilogue: partial squared norms of the o rows (2 x 64 floats)
+// the order of the chains (see order_chain): the B lengths, then the selected sequence
+constexpr int kRankMaxB = 256;
+constexpr uint32_t OFF_LEN = OFF_EPI + 512;
+constexpr uint32_t SMEM_USED = OFF_LEN + kRankMaxB * 4 + 16;
+constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;  // + alignment slack
+static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+static_assert(OFF_TT % 1024 == 0, "swizzle atoms");
+static_assert(OFF_PM0 >= 8192 && OFF_PM1 == OFF_PM0 + 8192, "Pm buffers");
 
-__host__ __device__ constexpr size_t vec_offset(size_t nch) { return nch * kTpBytes; }
+// TMEM columns (all 128 lanes): the Gram [K; Q][K; Q]^T (then the solve's merge products); U (lanes
+// 0..63); R: first W of the chunk (lanes 64..127, written while R is otherwise free), then [W S; o]
+// (lanes 0..63 / 64..127); the fp32 state S
+constexpr uint32_t TM_GPW = 0, TM_U = 128, TM_R = 256, TM_S = 384, TM_COLS = 512;
 
-__device__ __forceinline__ uint32_t blk_off(uint32_t row, uint32_t col) {  // within a 128-B-row swizzled block
+// V_G2 = G log2(e); V_LAM = V_G2 - log2(1/|k|), so that e^{G_t - G_s} / |k_s| = 2^{V_G2[t] - V_LAM[s]};
+// V_XS = e^G scale / |q| (row factor of Q S); V_N holds the chunk's valid-token count in its first entry.
+// V_ET = e^{G_last - G}; V_TAIL = V_ET / |k|.
+enum { V_BETA = 0, V_EG, V_TAIL, V_RK, V_RQ, V_CW, V_G2, V_LAM, V_XS, V_ET, V_N };
+static_assert(V_N < NVEC, "vector slots");
+
+struct TcArgs {
+    const void *beta;
+    const float *g;
+    const void *initial_state;
+    const int32_t *lengths;
+    float scale;
+    int B, Nk, Nv, S;
+    void *final_state;
+    int l2norm;
+    float eps;
+    int beta_logits;
+    const float *A_log, *dt_bias;
+    unsigned int *err;
+    const void *epi_z;  // NULL: no epilogue
+    const float *epi_w;
+    float epi_eps;
+    uint64_t wait_ns;  // limit of each bounded wait
+};
+
+__device__ __forceinline__ uint32_t blk_off(uint32_t row, uint32_t col) {  // within a 128-B-row block
     return (row >> 3) * 1024u + sw128_offset(row & 7u, col);
 }
 
 // silu(x) = x sigmoid(x).  For bf16 outputs sigmoid(x) = (1 + tanh(x / 2)) / 2 with tanh on the special-function
-// unit (PTX tanh.approx, relative error about 2^-11, below the bf16 rounding of 2^-9 that follows); for fp16
-// outputs (rounding 2^-11) x / (1 + e^{-x}) with the fast division (about 1e-6).
+// unit (PTX tanh.approx, relative error about 2^-11, below the bf16 rounding of 2^-9 that follows): one
+// special-function operation per element.  For fp16 outputs (rounding 2^-11) x / (1 + e^{-x}) with the fast
+// division (about 1e-6).
 template <typename T> __device__ __forceinline__ float silu_out(float x);
 template <> __device__ __forceinline__ float silu_out<__nv_bfloat16>(float x) {
     float t;
@@ -118,8 +208,7 @@ __device__ __forceinline__ float lg2_approx(float x) {
 }
 
 // The element type of the inputs, the operand copies and the outputs: bf16 or fp16 (tcgen05 kind::f16 takes
-// either, A and B of the same type).  TMA data type, descriptor operand format, pairs packed / unpacked, and the
-// warp-level MMA of the Gram.
+// either, A and B of the same type).  TMA data type, descriptor operand format, and pairs packed / unpacked.
 template <typename T> struct TcT;
 template <> struct TcT<__nv_bfloat16> {
     static constexpr CUtensorMapDataType kMap = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
@@ -127,13 +216,6 @@ template <> struct TcT<__nv_bfloat16> {
     static __device__ __forceinline__ uint32_t pack2(float lo, float hi) { return pack_bf16x2(lo, hi); }
     static __device__ __forceinline__ float2 unpack2(uint32_t u) {
         return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u));
-    }
-    // D (16 x 8, fp32) += A (16 x 16) B (16 x 8): m16n8k16, operands in the mma.sync fragment layout
-    static __device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
-        asm volatile("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
-                     "{%8, %9}, {%0, %1, %2, %3};"
-                     : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-                     : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
     }
 };
 template <> struct TcT<__half> {
@@ -145,12 +227,6 @@ template <> struct TcT<__half> {
     }
     static __device__ __forceinline__ float2 unpack2(uint32_t u) {
         return __half22float2(*reinterpret_cast<const __half2 *>(&u));
-    }
-    static __device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
-        asm volatile("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
-                     "{%8, %9}, {%0, %1, %2, %3};"
-                     : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-                     : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
     }
 };
 template <typename T> __host__ __device__ constexpr uint32_t idesc_t(int M, int N, bool a_mn_major, bool b_mn_major) {
@@ -170,21 +246,6 @@ template <typename T> __device__ __forceinline__ uint4 pack8(const float *f) {
     return make_uint4(TcT<T>::pack2(f[0], f[1]), TcT<T>::pack2(f[2], f[3]), TcT<T>::pack2(f[4], f[5]),
                       TcT<T>::pack2(f[6], f[7]));
 }
-
-// four 8 x 8 16-bit matrices from shared memory into the mma.sync fragment layout (lane l supplies the address of
-// row l % 8 of matrix l / 8)
-__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], uint32_t addr) {
-    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-                 : "r"(addr));
-}
-
-// ============================================================================================================
-// The WY solve T = (I + A)^{-1} (A strictly lower triangular, 64 x 64, fp32), by 256 threads.
-// ============================================================================================================
-
-constexpr int SP = 36;  // row stride (floats) of the plain 32 x 32 blocks: 16-byte aligned rows
-constexpr int BAR_SOLVE = 1;
 
 // D (16 x 8) += A (16 x 8) B (8 x 8) with tf32 operands and fp32 accumulation: one warp-level tensor-core MMA.
 // Thread l of the warp (g = l / 4, i = l % 4) holds a = {A[g][i], A[g+8][i], A[g][i+4], A[g+8][i+4]},
@@ -222,10 +283,10 @@ __device__ __forceinline__ void gemm32_tile(float (&d)[4], const float *A, const
 // Element (r, c) of a 32 x 32 diagonal block (r and c in the same 32-block) in the plain layout.
 __device__ __forceinline__ int pl(int r, int c) { return ((r >> 5) * 32 + (r & 31)) * SP + (c & 31); }
 
-// T = (I + A)^{-1}, first part, by 256 threads p: the two 32 x 32 diagonal blocks T11 and T22 (A strictly lower;
-// its diagonal blocks plain in sA).  The four 16 x 16 diagonal blocks by forward substitution (one column per
-// thread, zeros above the diagonal), then for each 32-block the lower-left 16 x 16 block T21 = -T22 (A21 T11)
-// with the CUDA cores.
+// T = (I + A)^{-1}, first part, by the 256 prep threads p: the two 32 x 32 diagonal blocks T11 and T22
+// (A strictly lower; its diagonal blocks plain in sA).  The four 16 x 16 diagonal blocks by forward
+// substitution (one column per thread, zeros above the diagonal), then for each 32-block the lower-left
+// 16 x 16 block T21 = -T22 (A21 T11) with the CUDA cores.
 __device__ __forceinline__ void solve_diag16_merge(const float *sA, float *sT, float *sX, int p) {
     if (p < 64) {
         const int base = (p >> 4) * 16, j = p & 15;
@@ -252,7 +313,7 @@ __device__ __forceinline__ void solve_diag16_merge(const float *sA, float *sT, f
             sT[(32 * blk + r) * SP + 16 + c] = 0.f;
         }
     }
-    named_sync(BAR_SOLVE, 256);
+    named_sync(BAR_PREP, NGRP);
     // 16 -> 32: X = A21 T11, then T21 = -T22 X, for the blocks at rows 32 b + 16, columns 32 b
     const int blk = p >> 7, r = (p >> 3) & 15, c2 = (p & 7) * 2;
     const float *ab = sA + blk * 32 * SP;
@@ -266,7 +327,7 @@ __device__ __forceinline__ void solve_diag16_merge(const float *sA, float *sT, f
         x1 = fmaf(a, t.y, x1);
     }
     *reinterpret_cast<float2 *>(sX + (blk * 16 + r) * SP + c2) = make_float2(x0, x1);
-    named_sync(BAR_SOLVE, 256);
+    named_sync(BAR_PREP, NGRP);
     float y0 = 0.f, y1 = 0.f;
 #pragma unroll
     for (int k = 0; k < 16; ++k) {
@@ -276,306 +337,28 @@ __device__ __forceinline__ void solve_diag16_merge(const float *sA, float *sT, f
         y1 = fmaf(t, xx.y, y1);
     }
     *reinterpret_cast<float2 *>(tb + (16 + r) * SP + c2) = make_float2(-y0, -y1);
-    named_sync(BAR_SOLVE, 256);
+    named_sync(BAR_PREP, NGRP);
 }
 
-// ============================================================================================================
-// wy_kernel: per (b, key head, chunk), for each value head of the group: T' = (I + A)^{-1} diag(beta) and the
-// chunk's vectors, into the workspace.
-// ============================================================================================================
-
-struct WyArgs {
-    const void *k;
-    const void *beta;
-    const float *g;
-    const int32_t *lengths;
-    int B, Nk, Nv, S, NC;
-    int l2norm;
-    float eps;
-    int beta_logits;
-    const float *A_log, *dt_bias;
-    void *tp;    // workspace: T' (16-bit), (B Nv NC) x 64 x 64
-    float *vec;  // workspace: vectors, (B Nv NC) x kNumVec x 64
-};
-
-constexpr int WY_THREADS = 256;
-constexpr int KST = 136;  // K tile row stride in elements (272 B: the 8 rows of an ldmatrix hit distinct banks)
-constexpr int GST = 65;   // Gram row stride (floats)
-constexpr uint32_t WY_OFF_K = 0;                             // 64 x KST 16-bit; after the Gram: A (diag blocks), X
-constexpr uint32_t WY_OFF_G = 17408;                         // Gram, 64 x GST fp32
-constexpr uint32_t WY_OFF_TP = WY_OFF_G + 64 * GST * 4;      // T diagonal blocks, 64 x SP
-constexpr uint32_t WY_OFF_A21 = WY_OFF_TP + 64 * SP * 4;     // A21, then T21: 32 x SP
-constexpr uint32_t WY_OFF_XM = WY_OFF_A21 + 32 * SP * 4;     // X = A21 T11 of the 32 -> 64 merge: 32 x SP
-constexpr uint32_t WY_OFF_VEC = WY_OFF_XM + 32 * SP * 4;     // kNumVec vectors, then beta, then 1/|k|
-constexpr uint32_t WY_SMEM = WY_OFF_VEC + (kNumVec + 2) * 64 * 4;
-static_assert(64 * KST * 2 <= WY_OFF_G, "K tile");
-static_assert(64 * SP * 4 + 32 * SP * 4 <= WY_OFF_G, "A diagonal blocks and the merge scratch fit in the K tile");
-constexpr int WV_BETA = kNumVec, WV_RK = kNumVec + 1;
-
-template <typename T, bool kGate>
-__global__ void __launch_bounds__(WY_THREADS, 4) wy_kernel(const WyArgs a) {
-    extern __shared__ __align__(16) uint8_t wsm[];
-    T *Ks = reinterpret_cast<T *>(wsm + WY_OFF_K);
-    float *sAP = reinterpret_cast<float *>(wsm + WY_OFF_K);  // reuses the K tile after the Gram
-    float *sXP = sAP + 64 * SP;
-    float *Gs = reinterpret_cast<float *>(wsm + WY_OFF_G);
-    float *sTP = reinterpret_cast<float *>(wsm + WY_OFF_TP);
-    float *sA21 = reinterpret_cast<float *>(wsm + WY_OFF_A21);
-    float *sXM = reinterpret_cast<float *>(wsm + WY_OFF_XM);
-    float *sv = reinterpret_cast<float *>(wsm + WY_OFF_VEC);
-
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int c = blockIdx.x % a.NC;
-    const int rest = blockIdx.x / a.NC;
-    const int kh = rest % a.Nk, b = rest / a.Nk;
-    int L = a.lengths ? a.lengths[b] : a.S;
-    if (L < 0 || L > a.S) L = 0;  // the chain kernel reports the bad length
-    const int n = min(C, L - c * C);
-    if (n <= 0) return;
-
-    // ---- the raw K tile (rows past the length zero) ----
-    const T *kp = static_cast<const T *>(a.k) + ((size_t)(b * a.Nk + kh) * a.S + (size_t)c * C) * D;
-    for (int e = tid; e < C * (D / 8); e += WY_THREADS) {
-        const int t = e >> 4, c8 = e & 15;
-        uint4 u = make_uint4(0, 0, 0, 0);
-        if (t < n) u = __ldg(reinterpret_cast<const uint4 *>(kp + (size_t)t * D + 8 * c8));
-        *reinterpret_cast<uint4 *>(Ks + t * KST + 8 * c8) = u;
-    }
-    __syncthreads();
-
-    // ---- a2: the Gram K K^T, lower 16 x 16 blocks (bi >= bj), warp-level MMAs ----
-    {
-        const int g = lane >> 2, i4 = lane & 3;
-        const int r = (lane & 7) + ((lane >> 3) & 1) * 8, cofs = (lane >> 4) * 8;
-        for (int blk = warp; blk < 10; blk += WY_THREADS / 32) {
-            const int bi = blk < 1 ? 0 : blk < 3 ? 1 : blk < 6 ? 2 : 3;
-            const int bj = blk - bi * (bi + 1) / 2;
-            float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-            const uint32_t abase = smem_u32(Ks + (16 * bi + r) * KST + cofs);
-            const uint32_t bbase = smem_u32(Ks + (16 * bj + r) * KST + cofs);
-#pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk) {
-                uint32_t af[4], bf[4];
-                ldsm_x4(af, abase + kk * 32);
-                ldsm_x4(bf, bbase + kk * 32);
-                TcT<T>::mma16816(acc[0], af, bf[0], bf[2]);
-                TcT<T>::mma16816(acc[1], af, bf[1], bf[3]);
-            }
-#pragma unroll
-            for (int nt = 0; nt < 2; ++nt) {
-                const int col = 16 * bj + 8 * nt + 2 * i4;
-                float *g0 = Gs + (16 * bi + g) * GST + col;
-                g0[0] = acc[nt][0];
-                g0[1] = acc[nt][1];
-                g0[8 * GST] = acc[nt][2];
-                g0[8 * GST + 1] = acc[nt][3];
-            }
-        }
-    }
-    __syncthreads();
-    if (tid < C) {  // 1/|k_t| from the Gram diagonal (0 past the length)
-        const float d = Gs[tid * GST + tid];
-        sv[WV_RK * 64 + tid] = tid < n ? (a.l2norm ? rsqrtf(d + a.eps) : 1.f) : 0.f;
-    }
-
-    const int grp = a.Nv / a.Nk;
-    for (int hh = 0; hh < grp; ++hh) {
-        const int h = kh * grp + hh;
-        const size_t bh = (size_t)b * a.Nv + h;
-        const size_t ch = bh * a.NC + c;
-        __syncthreads();  // the previous head's solve and stores are done with the shared buffers
-        // ---- a0/a1: beta, the gate, the cumulative gate and the vectors (warp 0, two tokens per lane) ----
-        if (warp == 0) {
-            const T *bp = static_cast<const T *>(a.beta) + bh * a.S + (size_t)c * C;
-            const float *gp = a.g ? a.g + bh * a.S + (size_t)c * C : nullptr;
-            const float gA = (kGate && a.A_log) ? a.A_log[h] : 0.f, gB = (kGate && a.A_log) ? a.dt_bias[h] : 0.f;
-            float bv[2], gv[2];
-#pragma unroll
-            for (int i = 0; i < 2; ++i) {
-                const int t = 2 * lane + i;
-                const float rb = t < n ? to_f32(bp[t]) : 0.f;
-                bv[i] = t < n ? (a.beta_logits ? sigmoid_f32(rb) : rb) : 0.f;
-                gv[i] = 0.f;
-                if (kGate && t < n) gv[i] = a.A_log ? gate_from_raw(gp[t], gA, gB) : gp[t];
-            }
-            float G[2] = {0.f, 0.f}, gl = 0.f;
-            if (kGate) {
-                const float x1 = gv[0] + gv[1];
-                float sc = x1;
-#pragma unroll
-                for (int o = 1; o < 32; o <<= 1) {
-                    const float y = __shfl_up_sync(0xffffffffu, sc, o);
-                    if (lane >= o) sc += y;
-                }
-                gl = __shfl_sync(0xffffffffu, sc, 31);
-                G[0] = sc - x1 + gv[0];
-                G[1] = sc;
-            }
-#pragma unroll
-            for (int i = 0; i < 2; ++i) {
-                const int t = 2 * lane + i;
-                const float rk = sv[WV_RK * 64 + t];
-                const float eg = kGate ? __expf(G[i]) : 1.f;
-                const float g2 = G[i] * 1.4426950408889634f;
-                sv[V_EG * 64 + t] = eg;
-                sv[V_CW * 64 + t] = eg * rk;
-                sv[V_CT * 64 + t] = (kGate ? __expf(gl - G[i]) : 1.f) * rk;
-                sv[V_G2 * 64 + t] = g2;
-                sv[V_LAM * 64 + t] = g2 - lg2_approx(rk);  // +inf past the length: those entries vanish
-                sv[V_MISC * 64 + t] = t == 0 ? (kGate ? __expf(gl) : 1.f) : (t == 1 ? (float)n : 0.f);
-                sv[WV_BETA * 64 + t] = bv[i];
-            }
-            __syncwarp();
-            float4 *vo = reinterpret_cast<float4 *>(a.vec + ch * (kVecBytes / 4));
-            const float4 *vi = reinterpret_cast<const float4 *>(sv);
-#pragma unroll
-            for (int e = 0; e < 3; ++e) vo[lane + 32 * e] = vi[lane + 32 * e];
-        }
-        __syncthreads();
-        // ---- a3: A (strictly lower) into the solve's plain layouts ----
-        {
-            const int t = tid >> 2, s0 = (tid & 3) * 16;
-            if (s0 < t) {
-                const float rowf = sv[WV_BETA * 64 + t] * sv[WV_RK * 64 + t];
-                const float g2t = sv[V_G2 * 64 + t];
-#pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    const int s = s0 + j;
-                    float v = 0.f;
-                    if (s < t)
-                        v = Gs[t * GST + s] * rowf *
-                            (kGate ? ex2_approx(g2t - sv[V_LAM * 64 + s]) : sv[WV_RK * 64 + s]);
-                    if ((t >> 5) == (s >> 5)) sAP[pl(t, s)] = v;
-                    else sA21[(t - 32) * SP + s] = v;
-                }
-            }
-        }
-        __syncthreads();
-        solve_diag16_merge(sAP, sTP, sXP, tid);
-        {
-            // 32 -> 64: X = A21 T11 (T11 lower triangular: k-steps before ct add nothing), then T21 = -(T22 X)
-            // (T22 lower triangular: rows 16 rt.. need k-steps up to 2 rt + 1), written over A21
-            const int rt = warp >> 2, ct = warp & 3, gq = lane >> 2, iq = lane & 3;
-            float d[4];
-            gemm32_tile(d, sA21, sTP, rt, ct, ct, 4, lane);
-            *reinterpret_cast<float2 *>(sXM + (16 * rt + gq) * SP + 8 * ct + 2 * iq) = make_float2(d[0], d[1]);
-            *reinterpret_cast<float2 *>(sXM + (16 * rt + gq + 8) * SP + 8 * ct + 2 * iq) = make_float2(d[2], d[3]);
-            __syncthreads();
-            gemm32_tile(d, sTP + 32 * SP, sXM, rt, ct, 0, 2 * rt + 2, lane);
-            *reinterpret_cast<float2 *>(sA21 + (16 * rt + gq) * SP + 8 * ct + 2 * iq) = make_float2(-d[0], -d[1]);
-            *reinterpret_cast<float2 *>(sA21 + (16 * rt + gq + 8) * SP + 8 * ct + 2 * iq) = make_float2(-d[2], -d[3]);
-        }
-        __syncthreads();
-        // ---- T' = T diag(beta), 16-bit, row-major, coalesced ----
-        T *tpo = static_cast<T *>(a.tp) + ch * (C * C);
-        for (int e = tid; e < C * C / 8; e += WY_THREADS) {
-            const int t = e >> 3, s8 = (e & 7) * 8;
-            float f[8];
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const int s = s8 + j;
-                float tv = 0.f;
-                if (s <= t) tv = ((t >> 5) == (s >> 5)) ? sTP[pl(t, s)] : sA21[(t - 32) * SP + s];
-                f[j] = tv * sv[WV_BETA * 64 + s];
-            }
-            *reinterpret_cast<uint4 *>(tpo + t * C + s8) = pack8<T>(f);
-        }
-    }
-}
-
-// ============================================================================================================
-// chain_kernel: the serial carry of one (b, value head) chain.
-// ============================================================================================================
-
-constexpr int NCARRY = 256, NOUTW = 128, NPREP = 128;
-constexpr int W_OUT0 = 8, W_PREP0 = 12, W_MMA = 16, W_TMA = 17;
-constexpr int CH_THREADS = 18 * 32;
-constexpr int BAR_CARRY = 1, BAR_OUT = 2, BAR_PREP = 3;
-
-// ---- shared memory map (bytes from a 1024-aligned base); every tile is 64 rows x 128 B, 128-byte swizzle ----
-constexpr int NKQ = 3, NVS = 2, NAX = 2;
-constexpr uint32_t KQ_STAGE = 32768;                      // [Q dk 0-63 | K dk 0-63 | Q dk 64-127 | K dk 64-127]
-constexpr uint32_t OFF_KQ = 0;
-constexpr uint32_t OFF_V = OFF_KQ + NKQ * KQ_STAGE;       // V stages: [dv 0-63 | dv 64-127]
-constexpr uint32_t OFF_TPS = OFF_V + NVS * 16384;         // T' stages (K-major [t][s])
-constexpr uint32_t OFF_TW = OFF_TPS + NAX * 8192;         // T' diag(e^G/|k|): B operand of the W product
-constexpr uint32_t OFF_WT = OFF_TW + 8192;                // -W^T, MN-major B operand [dk][t] of the v_new product
-constexpr uint32_t OFF_PM = OFF_WT + 16384;               // Pm, two buffers, K-major [t][s]
-constexpr uint32_t OFF_OUT = OFF_PM + 2 * 8192;           // out tile [t][dv] (two 64-column boxes)
-constexpr uint32_t OFF_Z = OFF_OUT + 16384;               // epilogue z tile; with OFF_OUT: the initial state
-constexpr uint32_t OFF_VECS = OFF_Z + 16384;              // vector stages
-constexpr uint32_t OFF_RED = OFF_VECS + NAX * kVecBytes;  // epilogue: 4 x 64 partial sums, then 64 factors
-constexpr uint32_t OFF_RQ = OFF_RED + 5 * 64 * 4;         // scale / |q_t|, two chunks (out warps)
-constexpr uint32_t OFF_BARS = OFF_RQ + 2 * 64 * 4;
-constexpr int kNumBars = 36;
-constexpr uint32_t OFF_MISC = OFF_BARS + kNumBars * 8;    // TMEM base, abort flag, selected sequence
-constexpr int kRankMaxB = 256;
-constexpr uint32_t OFF_LEN = OFF_MISC + 16;               // the B lengths, for the longest-first order
-constexpr uint32_t CH_SMEM_USED = OFF_LEN + kRankMaxB * 4 + 16;
-constexpr uint32_t CH_SMEM = CH_SMEM_USED + 1024;         // + alignment slack
-static_assert(CH_SMEM <= 232448, "shared memory budget");
-static_assert(OFF_TPS % 1024 == 0 && OFF_TW % 1024 == 0 && OFF_WT % 1024 == 0 && OFF_PM % 1024 == 0 &&
-                  OFF_OUT % 1024 == 0 && OFF_Z % 1024 == 0,
-              "swizzle atoms");
-
-// TMEM columns (128 lanes): S^T fp32 (lane = value column j, column = key row i); R = [v_new^T | o^T] fp32 with
-// two 16-bit copies of v_new^T packed over its first columns (plain for o, scaled by c_t for the state); two 16-bit copies of S^T (the A operand of the
-// chunk's v_new and o products, alternating per chunk); W^T fp32 (lane = key row, column = token); the Gram
-// [Q; K] K^T (lanes 0-63: P = Q K^T).
-constexpr uint32_t TM_S = 0, TM_R = 128, TM_SA0 = 256, TM_SA1 = 320, TM_W = 384, TM_P = 448, TM_COLS = 512;
-
-// barrier indices
-enum {
-    B_FULL_KQ = 0,                  // [3] K, Q of a chunk landed (TMA)
-    B_EMPTY_KQ = 3,                 // [3] the chunk's K~ and Q~ are read (MMA commit)
-    B_FULL_V = 6,                   // [2]
-    B_EMPTY_V = 8,                  // [2]
-    B_FULL_AX = 10,                 // [2] T' and the vectors landed
-    B_EMPTY_AX = 12,                // [2] 4 arrivals: the U product read T'; prep, carry and out read the vectors
-    B_KQ_OK = 14, B_V_OK,           // prep: the raw K, Q / V of the chunk may be read (padding rows zeroed)
-    B_TW, B_W_DONE, B_WT,           // T' diag(cw) written; W^T in TMEM; -W^T in shared memory
-    B_P_DONE, B_QK, B_PM,           // Gram in TMEM; Q~ in place (out warps); Pm written (and the Gram read)
-    B_V_DONE, B_VA,                 // v_new^T in TMEM; its 16-bit copy written
-    B_S_DONE, B_SA, B_SD,           // state updated; its 16-bit copy written; the decayed fp32 state written
-    B_O_DONE, B_O_READ,             // o^T complete; o^T read
-    B_S0, B_S0_FREE, B_Z,           // initial state landed; its staging tile is free again; epilogue z tile
-    B_DRAIN,                        // the last MMAs completed (exit)
-    B_COUNT
-};
-static_assert(B_COUNT <= kNumBars, "barriers");
-
-struct ChainArgs {
-    const void *initial_state;
-    void *final_state;
-    const int32_t *lengths;
-    float scale;
-    int B, Nk, Nv, S, NC;
-    int l2norm;
-    float eps;
-    const float *vec;  // workspace vectors
-    unsigned int *err;
-    const void *epi_z;  // NULL: no epilogue
-    const float *epi_w;
-    float epi_eps;
-    unsigned long long wait_ns;
-};
-
-// The sequence a CTA runs, longest first.  A CTA holds an SM for its whole chain and CTAs start in index order as
-// SMs free up, so with more chains than SMs a long chain that starts late sets the end of the launch (longest-
-// processing-time-first list scheduling).  CTA i takes the sequence whose valid length ranks i / Nv-th (longest
-// first, ties by index; an invalid length counts as 0); its value head stays i % Nv.  Without lengths, or with more
-// than kRankMaxB sequences, the order is the index order.  Called by all threads before anything else.
-__device__ __forceinline__ int order_chain(const ChainArgs &a, int tid, uint8_t *sm) {
+// The sequence a CTA runs, longest first.  A CTA holds an SM for its whole chain and CTAs start in index
+// order as SMs free up, so with more chains than SMs a long chain that starts late sets the end of the launch
+// (longest-processing-time-first list scheduling).  CTA i takes the sequence whose valid length ranks
+// i / Nv-th (longest first, ties by index; an invalid length counts as 0); its value head stays i % Nv.
+// Without lengths, or with more than kRankMaxB sequences, the order is the index order.  Called by all
+// threads of the CTA before anything else touches shared memory.  The kernel's ordered instantiation runs
+// it, and the host launches that one only when the chains outnumber the resident CTAs: its sequence index
+// lives in a register, where the index order's is recomputed from blockIdx, and in one wave order is moot.
+__device__ __forceinline__ int order_chain(const TcArgs &a, int tid, uint8_t *sm) {
     const int seq = blockIdx.x / a.Nv;
     if (!a.lengths || a.B <= 1 || a.B > kRankMaxB) return seq;
     int *s_len = reinterpret_cast<int *>(sm + OFF_LEN);
-    volatile int *s_sel = reinterpret_cast<volatile int *>(sm + OFF_MISC + 8);
-    for (int i = tid; i < a.B; i += CH_THREADS) {
+    volatile int *s_sel = s_len + kRankMaxB;
+    for (int i = tid; i < a.B; i += NT) {
         const int L = a.lengths[i];
         s_len[i] = (L < 0 || L > a.S) ? 0 : L;
     }
     __syncthreads();
-    for (int i = tid; i < a.B; i += CH_THREADS) {  // the ranks are a permutation of 0..B-1: one i matches
+    for (int i = tid; i < a.B; i += NT) {  // the ranks are a permutation of 0..B-1: one i matches
         const int Li = s_len[i];
         int r = 0;
         for (int j = 0; j < a.B; ++j) {
@@ -588,34 +371,39 @@ __device__ __forceinline__ int order_chain(const ChainArgs &a, int tid, uint8_t 
     return *s_sel;
 }
 
-// Pairs of 16-bit values across neighbouring lanes: lane l holds x[k] = M[k][col] for its column col = base + l and
-// rows k = 0..63; after this, even lanes hold the word (M[2i][col], M[2i][col+1]) of row 2i and odd lanes the word
-// (M[2i+1][col-1], M[2i+1][col]) of row 2i+1, i = 0..31 (one shuffle per pair of rows).
-template <typename T> __device__ __forceinline__ uint32_t pair_word(float x0, float x1, int lane) {
-    const bool odd = lane & 1;
-    const float send = odd ? x0 : x1;
-    const float recv = __shfl_xor_sync(0xffffffffu, send, 1);
-    return odd ? TcT<T>::pack2(recv, x1) : TcT<T>::pack2(x0, recv);
-}
-
-template <typename T, bool kGate, bool kOrdered>
-__global__ void __launch_bounds__(CH_THREADS, 1)
-chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-             const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
-             const __grid_constant__ CUtensorMap tm_tp, const __grid_constant__ CUtensorMap tm_s0,
-             const __grid_constant__ CUtensorMap tm_fs, const __grid_constant__ CUtensorMap tm_z, const ChainArgs a) {
+template <typename T, bool kOrdered>
+__global__ void __launch_bounds__(NT, 1)
+chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o, const TcArgs a) {
     extern __shared__ __align__(1024) uint8_t smraw[];
+    // 1024-byte aligned base, derived from smraw by pointer arithmetic (not through an
+    // integer) so that the compiler keeps every access below in the shared address space
     uint8_t *sm = smraw + ((1024u - (smem_u32(smraw) & 1023u)) & 1023u);
     const uint32_t sbase = smem_u32(sm);
-    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + OFF_BARS);
-    uint32_t *s_tmem = reinterpret_cast<uint32_t *>(sm + OFF_MISC);
-    volatile int *s_abort = reinterpret_cast<volatile int *>(sm + OFF_MISC + 4);
-    const float *vecs = reinterpret_cast<const float *>(sm + OFF_VECS);
+    float *vecs = reinterpret_cast<float *>(sm + OFF_VEC);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + OFF_BAR);
+    // bar_ld: K and Q of the chunk landed (bar_ldv: V); bar_gp / bar_wu: the prep MMAs completed; bar_m1 / bar_m2: the carry MMAs
+    // completed; bar_a1: the prep group handed chunk c to the carry group; bar_cq / bar_ck: the raw Q rows
+    // of A1 / the raw K tile landed; bar_pf[i]: the carry group is done with Pm buffer i and vector set i
+    uint64_t *bar_ld = bars, *bar_gp = bars + 1, *bar_wu = bars + 2, *bar_m1 = bars + 3, *bar_m2 = bars + 4;
+    uint64_t *bar_a1 = bars + 5, *bar_cq = bars + 6, *bar_ck = bars + 7, *bar_pf = bars + 8;
+    // bar_vr: the control warp has written the gate vectors of the next chunk (one phase per chunk)
+    uint64_t *bar_vr = bars + 10, *bar_ldv = bars + 11;
+    // bar_go: the carry group has taken chunk c over (its tail factors are in place); bar_kt: the helper warps
+    // have scaled chunk c's K tile into K~ (one phase per chunk each)
+    uint64_t *bar_go = bars + 12, *bar_kt = bars + 13;
+    // bar_dr: two commits, every MMA of the control warp and of the carry group completed (exit)
+    uint64_t *bar_dr = bars + 14;
+    constexpr int kNumBars = 15;
+    static_assert(kNumBars * 8 + 8 <= 128, "barriers, TMEM base and abort flag before the epilogue scratch");
+    uint32_t *s_tmem = reinterpret_cast<uint32_t *>(bars + kNumBars);
+    volatile int *s_abort = reinterpret_cast<volatile int *>(s_tmem + 1);
 
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, q4 = warp & 3;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, q4 = warp & 3, hf = (warp >> 2) & 1;
+    const bool carry = warp < 8, control = warp == CTL_WARP, helper = warp > CTL_WARP;
     const int h = blockIdx.x % a.Nv;
     const int b = kOrdered ? order_chain(a, tid, sm) : (int)blockIdx.x / a.Nv;
-    const int bh = b * a.Nv + h, kh = h / (a.Nv / a.Nk);
+    const int bh = kOrdered ? b * a.Nv + h : (int)blockIdx.x, kh = h / (a.Nv / a.Nk);
     const int S = a.S;
     int L = a.lengths ? a.lengths[b] : S;
     const bool bad_len = (L < 0 || L > S);
@@ -623,832 +411,820 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     const int nvalid = (L + C - 1) / C, ntotal = (S + C - 1) / C;
     const int zq = b * a.Nk + kh;  // TMA z coordinate of q/k rows
     const uint32_t lane_base = (uint32_t)(q4 * 32) << 16;
-    const uint64_t wait_ns = a.wait_ns;
-    const size_t ch0 = (size_t)bh * a.NC;  // workspace index of chunk 0
+    const int row = q4 * 32 + lane;  // TMEM lane of this thread
+
+    // a bounded wait: false when it ran out (the first such wait of the launch is recorded) or another group stopped
+    auto bw = [&](uint64_t *bar, uint32_t parity) -> bool {
+        if (mbar_wait_ns(bar, parity, a.wait_ns, s_abort)) return true;
+        if (!*s_abort)
+            atomicCAS(&g_timeout_site, 0u,
+                      0x80000000u | ((uint32_t)warp << 24) | ((uint32_t)(bar - bars) << 16) | (parity << 15) |
+                          (blockIdx.x & 0x7fffu));
+        return false;
+    };
+    // loads issued per barrier by the thread that issues them (one phase each), for the drain at the exit
+    int n_ld = 0, n_ldv = 0, n_cq = 0, n_ck = 0;
+
+    // raw Q rows of A1 and the raw K tile of chunk c, for the carry group (issued by carry thread 0)
+    auto load_carry_q = [&](int chunk) {
+        ++n_cq;
+        mbar_arrive_expect_tx(bar_cq, 16384);
+        tma_load_3d(sm + OFF_A1 + 8192, &tm_q, bar_cq, 0, chunk * C, zq);
+        tma_load_3d(sm + OFF_A1 + 16384 + 8192, &tm_q, bar_cq, 64, chunk * C, zq);
+    };
+    auto load_carry_k = [&](int chunk) {
+        ++n_ck;
+        mbar_arrive_expect_tx(bar_ck, 16384);
+        tma_load_3d(sm + OFF_KT, &tm_k, bar_ck, 0, chunk * C, zq);
+        tma_load_3d(sm + OFF_KT + 8192, &tm_k, bar_ck, 64, chunk * C, zq);
+    };
 
     if (tid == 0) {
         if (bad_len) raise_device_error(a.err, GDR_DEVERR_LENGTH);
-        for (int i = 0; i < B_COUNT; ++i) mbar_init(bars + i, (i == B_EMPTY_AX || i == B_EMPTY_AX + 1) ? 4 : 1);
+        for (int i = 0; i < kNumBars; ++i) mbar_init(bars + i, i == 14 ? 2 : 1);
         *s_abort = 0;
         fence_mbar_init();
+        prefetch_tmap(&tm_q);
+        prefetch_tmap(&tm_k);
+        prefetch_tmap(&tm_v);
+        prefetch_tmap(&tm_o);
+        if (nvalid > 0) {
+            load_carry_q(0);
+            load_carry_k(0);
+        }
     }
     if (warp == 0) tmem_alloc(s_tmem, TM_COLS);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *s_tmem;
-    auto vec_of = [&](int j) { return vecs + (j % NAX) * (kVecBytes / 4); };
-    auto chunk_n = [&](int j) { return min(C, L - j * C); };
-#ifdef GDR_PHASE_TIMERS
-    __shared__ unsigned long long s_wcyc[kTimerSlots];
-    for (int i = tid; i < kTimerSlots; i += CH_THREADS) s_wcyc[i] = 0;
-    __syncthreads();
-    const long long t_start = clock64();
-    const int role = warp < 8 ? 0 : warp < W_PREP0 ? 1 : warp < W_MMA ? 2 : warp == W_MMA ? 3 : 4;
-    const bool rep_thread = tid == 0 || tid == W_OUT0 * 32 || tid == W_PREP0 * 32 || tid == W_MMA * 32 ||
-                            tid == W_TMA * 32;
-#endif
-    auto wait = [&](int idx, uint32_t parity) {
-#ifdef GDR_PHASE_TIMERS
-        const long long t0 = clock64();
-        const bool ok = mbar_wait_ns(bars + idx, parity, wait_ns, s_abort);
-        if (rep_thread) s_wcyc[role * 36 + idx] += (unsigned long long)(clock64() - t0);
-        if (ok) return true;
-#else
-        if (mbar_wait_ns(bars + idx, parity, wait_ns, s_abort)) return true;
-#endif
-        if (!*s_abort)  // this wait ran out (rather than seeing another group stop): record where
-            atomicCAS(&g_timeout_site, 0u,
-                      0x80000000u | ((uint32_t)warp << 24) | ((uint32_t)idx << 16) | (parity << 15) |
-                          (blockIdx.x & 0x7fffu));
-        return false;
-    };
-    auto stop = [&]() { *s_abort = 1; };
 
-    if (warp == W_TMA) {
-        // ================================ TMA loads ================================
-        int issued_kq[NKQ] = {0, 0, 0}, issued_v[NVS] = {0, 0}, issued_ax[NAX] = {0, 0};
-        bool s0_issued = false;
-        if (lane == 0) {
-            prefetch_tmap(&tm_q);
-            prefetch_tmap(&tm_k);
-            prefetch_tmap(&tm_v);
-            prefetch_tmap(&tm_tp);
-            // the initial state: read by the carry (or copied out unchanged for an empty sequence)
-            if (a.initial_state && (nvalid > 0 || a.final_state)) {
-                mbar_arrive_expect_tx(bars + B_S0, 32768);
-                for (int bx = 0; bx < 4; ++bx)  // box (dv block bx / 2, dk block bx % 2)
-                    tma_load_3d(sm + OFF_OUT + bx * 8192, &tm_s0, bars + B_S0, 64 * (bx >> 1), 64 * (bx & 1), bh);
-                s0_issued = true;
+    if (carry) {
+        // ---- initial state into TMEM (fp32) and the bf16 operand tile ----
+        const T *s0 = reinterpret_cast<const T *>(a.initial_state);
+        const size_t off = ((size_t)bh * D + row) * D + 64 * hf;
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+            float v[32];
+#pragma unroll
+            for (int c8 = 0; c8 < 4; ++c8) {
+                float f[8];
+                if (s0) {
+                    unpack8<T>(*reinterpret_cast<const uint4 *>(s0 + off + 32 * half + 8 * c8), f);
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) f[i] = 0.f;
+                }
+#pragma unroll
+                for (int i = 0; i < 8; ++i) v[8 * c8 + i] = f[i];
+                *reinterpret_cast<uint4 *>(sm + OFF_S + hf * 16384 + blk_off(row, 32 * half + 8 * c8)) =
+                    pack8<T>(&v[8 * c8]);
             }
-            for (int j = 0; j < nvalid; ++j) {
-                const int y = j * C;
-                const int sk = j % NKQ, sv = j % NVS, sa = j % NAX;
-                if (j >= NKQ && !wait(B_EMPTY_KQ + sk, ((j / NKQ) - 1) & 1)) { stop(); break; }
-                mbar_arrive_expect_tx(bars + B_FULL_KQ + sk, 32768);
-                uint8_t *st = sm + OFF_KQ + sk * KQ_STAGE;
-                tma_load_3d(st, &tm_q, bars + B_FULL_KQ + sk, 0, y, zq);
-                tma_load_3d(st + 8192, &tm_k, bars + B_FULL_KQ + sk, 0, y, zq);
-                tma_load_3d(st + 16384, &tm_q, bars + B_FULL_KQ + sk, 64, y, zq);
-                tma_load_3d(st + 24576, &tm_k, bars + B_FULL_KQ + sk, 64, y, zq);
-                ++issued_kq[sk];
-                if (j >= NVS && !wait(B_EMPTY_V + sv, ((j / NVS) - 1) & 1)) { stop(); break; }
-                mbar_arrive_expect_tx(bars + B_FULL_V + sv, 16384);
-                tma_load_3d(sm + OFF_V + sv * 16384, &tm_v, bars + B_FULL_V + sv, 0, y, bh);
-                tma_load_3d(sm + OFF_V + sv * 16384 + 8192, &tm_v, bars + B_FULL_V + sv, 64, y, bh);
-                ++issued_v[sv];
-                if (j >= NAX && !wait(B_EMPTY_AX + sa, ((j / NAX) - 1) & 1)) { stop(); break; }
-                mbar_arrive_expect_tx(bars + B_FULL_AX + sa, (uint32_t)(kTpBytes + kVecBytes));
-                tma_load_3d(sm + OFF_TPS + sa * 8192, &tm_tp, bars + B_FULL_AX + sa, 0, 0, (int)(ch0 + j));
-                bulk_load(sm + OFF_VECS + sa * kVecBytes, a.vec + (ch0 + j) * (kVecBytes / 4), (uint32_t)kVecBytes,
-                          bars + B_FULL_AX + sa);
-                ++issued_ax[sa];
-            }
-            // drain: every load this warp issued has landed before the CTA leaves
-            if (s0_issued) mbar_wait_ns(bars + B_S0, 0, kDrainWaitNs);
-            for (int s = 0; s < NKQ; ++s)
-                if (issued_kq[s]) mbar_wait_ns(bars + B_FULL_KQ + s, (issued_kq[s] - 1) & 1, kDrainWaitNs);
-            for (int s = 0; s < NVS; ++s)
-                if (issued_v[s]) mbar_wait_ns(bars + B_FULL_V + s, (issued_v[s] - 1) & 1, kDrainWaitNs);
-            for (int s = 0; s < NAX; ++s)
-                if (issued_ax[s]) mbar_wait_ns(bars + B_FULL_AX + s, (issued_ax[s] - 1) & 1, kDrainWaitNs);
+            tmem_st32(tmem + TM_S + lane_base + 64 * hf + 32 * half, v);
         }
-    } else if (warp == W_MMA) {
-        // ============================== MMA issue ==============================
-        if (lane == 0 && nvalid > 0) {
-            const uint32_t idSS = idesc_t<T>(128, 64, true, false);   // A MN-major smem, B K-major
-            const uint32_t idP = idesc_t<T>(128, 64, false, false);   // A, B K-major smem
-            const uint32_t id1a = idesc_t<T>(128, 64, false, true);   // A TMEM, B MN-major
-            const uint32_t idTK = idesc_t<T>(128, 64, false, false);  // A TMEM, B K-major
-            const uint32_t id2 = idesc_t<T>(128, 128, false, true);   // A TMEM, B MN-major, N = 128
-            auto kq_base = [&](int j) { return sbase + OFF_KQ + (uint32_t)(j % NKQ) * KQ_STAGE; };
-            // the 16-bit copies of v_new^T: tokens 16 kk .. 16 kk + 15 (plain, and scaled by c_t)
-            auto va_col = [&](int kk) { return tmem + TM_R + 32 * (kk >> 1) + 8 * (kk & 1); };
-            auto vs_col = [&](int kk) { return tmem + TM_R + 32 * (kk >> 1) + 16 + 8 * (kk & 1); };
-            auto issue_W = [&](int j) {  // W^T = K^T (T' diag(cw))^T
-                const uint32_t kb = kq_base(j) + 8192;
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    mma_bf16(tmem + TM_W, sdesc_sw128(kb + kk * 2048, 16384, 1024),
-                             sdesc_sw128(sbase + OFF_TW + kk * 32, 16, 1024), idSS, kk > 0);
-            };
-            auto issue_P = [&](int j) {  // [Q; K] K^T
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    const uint32_t ad = kq_base(j) + (kk >> 2) * 16384 + (kk & 3) * 32;
-                    mma_bf16(tmem + TM_P, sdesc_sw128(ad, 16, 1024), sdesc_sw128(ad + 8192, 16, 1024), idP, kk > 0);
-                }
-            };
-            auto issue_U = [&](int j) {  // U^T = V^T T'^T
-                const uint32_t vb = sbase + OFF_V + (uint32_t)(j % NVS) * 16384;
-                const uint32_t tb = sbase + OFF_TPS + (uint32_t)(j % NAX) * 8192;
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    mma_bf16(tmem + TM_R, sdesc_sw128(vb + kk * 2048, 8192, 1024), sdesc_sw128(tb + kk * 32, 16, 1024),
-                             idSS, kk > 0);
-            };
-            // Every wait on a hand-off barrier below comes before this thread's own step that lets the producer
-            // reach its next arrival on that barrier, so no barrier can run two phases ahead of a wait (which a
-            // parity wait would take for the current, incomplete phase).  The prep group's hand-offs of chunk
-            // j + 1 (raw K/Q/V and T' diag(cw)) are therefore all awaited before the W product of chunk j + 1, and
-            // Q~/K~ of chunk j before the Gram of chunk j + 1.
-            bool to = false;
-            const bool ok = wait(B_TW, 0) && wait(B_KQ_OK, 0) && wait(B_V_OK, 0) && wait(B_FULL_KQ, 0) &&
-                            wait(B_FULL_AX, 0) && wait(B_FULL_V, 0);
-            if (ok) {
-                tc_fence_after();
-                issue_W(0);
-                mma_commit(bars + B_W_DONE);
-                issue_P(0);
-                mma_commit(bars + B_P_DONE);
-                issue_U(0);
-                mma_commit(bars + B_EMPTY_V);
-                mma_commit(bars + B_EMPTY_AX);
+        tmem_st_wait();
+        fence_proxy_async_smem();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+
+#ifdef GDR_PHASE_TIMERS
+    unsigned long long t_prev_ = clock64();
+    __shared__ unsigned long long s_phase_[64];
+    if (tid < 64) s_phase_[tid] = 0;
+    __syncthreads();
+#endif
+    if (control) {
+        // ============================== control warp ==============================
+        // Lane 0 issues the prep MMAs and nothing else, lane 1 the input-stage TMA loads and L2
+        // prefetches (an MMA issued by a thread with copies of its own outstanding was seen to wait
+        // for them).  Having a warp of its own, neither blocks a prep warp while the tensor pipe is
+        // busy.  The warp follows the prep group's hand-off barriers (BAR_PCTL) and leaves at the
+        // same barrier as the prep group when a wait timed out.
+        auto prefetch_l2 = [&](int chunk) {
+            const int y = chunk * C;
+            tma_prefetch_3d(&tm_k, 0, y, zq);
+            tma_prefetch_3d(&tm_k, 64, y, zq);
+            tma_prefetch_3d(&tm_q, 0, y, zq);
+            tma_prefetch_3d(&tm_q, 64, y, zq);
+            tma_prefetch_3d(&tm_v, 0, y, bh);
+            tma_prefetch_3d(&tm_v, 64, y, bh);
+            if (a.epi_z) {  // the chunk's z rows of the epilogue: one contiguous block of valid rows
+                const int rows = min(C, L - y);
+                asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;"
+                             ::"l"(static_cast<const T *>(a.epi_z) + ((size_t)bh * S + y) * D),
+                             "r"((uint32_t)(rows * D * 2))
+                             : "memory");
             }
-            if (!ok) to = true;
-            for (int c = 0; !to && c < nvalid; ++c) {
-                const uint32_t par = c & 1;
-                const bool more = c + 1 < nvalid;
-                const int j = c + 1;
-                const uint32_t sa = tmem + (par ? TM_SA1 : TM_SA0);
-                // v_new^T = U^T - S^T W^T (critical)
-                if (!(wait(B_SA, par) && wait(B_WT, par))) { to = true; break; }
-                EVENT(c, 15);
-                tc_fence_after();
+        };
+        // K of a chunk into its buffer (this also arms the chunk's K/Q barrier), Q into the single Q buffer,
+        // V into the single V buffer
+        auto issue_k = [&](int chunk) {
+            const int y = chunk * C, pc = chunk & 1;
+            ++n_ld;
+            mbar_arrive_expect_tx(bar_ld, 32768);
+            tma_load_3d(sm + off_k(pc, 0), &tm_k, bar_ld, 0, y, zq);
+            tma_load_3d(sm + off_k(pc, 1), &tm_k, bar_ld, 64, y, zq);
+        };
+        auto issue_q = [&](int chunk) {
+            const int y = chunk * C;
+            tma_load_3d(sm + off_q(0), &tm_q, bar_ld, 0, y, zq);
+            tma_load_3d(sm + off_q(1), &tm_q, bar_ld, 64, y, zq);
+        };
+        auto issue_v = [&](int chunk) {
+            const int y = chunk * C;
+            ++n_ldv;
+            mbar_arrive_expect_tx(bar_ldv, 16384);
+            tma_load_3d(sm + OFF_V, &tm_v, bar_ldv, 0, y, bh);
+            tma_load_3d(sm + OFF_V + 8192, &tm_v, bar_ldv, 64, y, bh);
+        };
+        // The gate and beta vectors of a chunk, which need no Gram: beta (from logits), the cumulative
+        // gate G (from the raw gate), e^G, G log2(e), e^{G_last - G} and the valid-token count; two
+        // tokens per lane, the scan over the chunk by warp shuffles.
+        const float gA = (a.A_log && a.g) ? a.A_log[h] : 0.f, gB = (a.A_log && a.g) ? a.dt_bias[h] : 0.f;
+        const T *bg = reinterpret_cast<const T *>(a.beta) + (size_t)bh * S;
+        const float *gg = a.g ? a.g + (size_t)bh * S : nullptr;
+        // raw beta and gate values of a chunk's tokens (two per lane), loaded a chunk before they are used so
+        // that their memory latency stays off the hand-offs
+        auto load_raw = [&](int chunk, float (&rb)[2], float (&rg)[2]) {
+            const int n = min(C, L - chunk * C);
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                    mma_ts(tmem + TM_R, sa + 8 * kk, sdesc_sw128(sbase + OFF_WT + kk * 2048, 16384, 1024), id1a, 1);
-                mma_commit(bars + B_V_DONE);
-                EVENT(c, 1);
-                // While the carry converts v_new: W and the Gram of the next chunk, if their operands are already
-                // in place (tested, not waited for: the chain's own product must not queue behind them).  Each
-                // phase is observed once (a successful test counts as the wait).
-                bool w_next = false, p_next = false, qk_seen = false, pm_seen = false;
-                if (more && mbar_test(bars + B_TW, j & 1) && mbar_test(bars + B_KQ_OK, j & 1) &&
-                    mbar_test(bars + B_V_OK, j & 1) && mbar_test(bars + B_FULL_KQ + j % NKQ, (j / NKQ) & 1)) {
-                    tc_fence_after();
-                    issue_W(j);
-                    mma_commit(bars + B_W_DONE);
-                    EVENT(c, 6);
-                    w_next = true;
-                    if (mbar_test(bars + B_QK, par) && mbar_test(bars + B_PM, par)) {
-                        qk_seen = pm_seen = true;
-                        tc_fence_after();
-                        issue_P(j);
-                        mma_commit(bars + B_P_DONE);
-                        EVENT(c, 7);
-                        p_next = true;
-                    }
-                }
-                // S^T = e^{G_last} S^T + (v_new diag(c))^T K (critical)
-                if (!(wait(B_VA, par) && wait(B_SD, par))) { to = true; break; }
-                tc_fence_after();
-                {
-                    const uint32_t kb = kq_base(c) + 8192;
-#pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        mma_ts(tmem + TM_S, vs_col(kk), sdesc_sw128(kb + kk * 2048, 16384, 1024), id2, 1);
-                }
-                mma_commit(bars + B_S_DONE);
-                EVENT(c, 4);
-                // o^T = S^T Q~^T + v_new^T Pm^T, while the carry converts the state
-                if (!qk_seen && !wait(B_QK, par)) { to = true; break; }
-                qk_seen = true;
-                if (c > 0 && !wait(B_O_READ, (c - 1) & 1)) { to = true; break; }
-                tc_fence_after();
-                {
-                    const uint32_t qb = kq_base(c);
-#pragma unroll
-                    for (int kk = 0; kk < 8; ++kk)
-                        mma_ts(tmem + TM_R + 64, sa + 8 * kk, sdesc_sw128(qb + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
-                               idTK, kk > 0);
-                }
-                EVENT(c, 8);
-                if (!pm_seen && !wait(B_PM, par)) { to = true; break; }
-                pm_seen = true;
-                tc_fence_after();
-                {
-                    const uint32_t pb = sbase + OFF_PM + par * 8192;
-#pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        mma_ts(tmem + TM_R + 64, va_col(kk), sdesc_sw128(pb + kk * 32, 16, 1024), idTK, 1);
-                }
-                mma_commit(bars + B_O_DONE);
-                mma_commit(bars + B_EMPTY_KQ + c % NKQ);
-                EVENT(c, 9);
-                if (more) {
-                    if (!w_next) {  // the next chunk's W, waited for now
-                        if (!(wait(B_TW, j & 1) && wait(B_KQ_OK, j & 1) && wait(B_V_OK, j & 1) &&
-                              wait(B_FULL_KQ + j % NKQ, (j / NKQ) & 1))) {
-                            to = true;
-                            break;
-                        }
-                        tc_fence_after();
-                        issue_W(j);
-                        mma_commit(bars + B_W_DONE);
-                        EVENT(c, 6);
-                    }
-                    if (!p_next) {  // the Gram of the next chunk (Q~, Pm of this one are in place: waited above)
-                        tc_fence_after();
-                        issue_P(j);
-                        mma_commit(bars + B_P_DONE);
-                        EVENT(c, 7);
-                    }
-                    // U of the next chunk (v_new of this one is read)
-                    if (!(wait(B_FULL_V + j % NVS, (j / NVS) & 1) && wait(B_FULL_AX + j % NAX, (j / NAX) & 1))) {
-                        to = true;
-                        break;
-                    }
-                    tc_fence_after();
-                    issue_U(j);
-                    mma_commit(bars + B_EMPTY_V + j % NVS);
-                    mma_commit(bars + B_EMPTY_AX + j % NAX);
-                    EVENT(c, 10);
-                }
+            for (int i = 0; i < 2; ++i) {
+                const int tt = 2 * lane + i, t = chunk * C + tt;
+                rb[i] = tt < n ? to_f32(bg[t]) : 0.f;
+                rg[i] = (tt < n && gg) ? gg[t] : 0.f;
             }
-            if (to) stop();
-            // drain: every MMA issued has completed before TMEM is released
-            mma_commit(bars + B_DRAIN);
-            mbar_wait_ns(bars + B_DRAIN, 0, kDrainWaitNs);
-        }
-    } else if (warp >= W_PREP0) {
-        // ================================ prep ================================
-        const int p = tid - W_PREP0 * 32;
+        };
+        auto chunk_vectors = [&](int chunk, const float (&rb)[2], const float (&rg)[2]) {
+            float *vec = vecs + (chunk & 1) * NVEC * 64;
+            const int n = min(C, L - chunk * C);
+            float bv[2], gv[2];
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+                const int tt = 2 * lane + i;
+                bv[i] = tt < n ? (a.beta_logits ? sigmoid_f32(rb[i]) : rb[i]) : 0.f;
+                gv[i] = tt < n ? (a.A_log ? gate_from_raw(rg[i], gA, gB) : rg[i]) : 0.f;
+            }
+            const float x1 = gv[0] + gv[1];
+            float sc = x1;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const float y = __shfl_up_sync(0xffffffffu, sc, o);
+                if (lane >= o) sc += y;
+            }
+            const float gl = __shfl_sync(0xffffffffu, sc, 31);
+            const float G[2] = {sc - x1 + gv[0], sc};
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+                const int tt = 2 * lane + i;
+                vec[V_BETA * 64 + tt] = bv[i];
+                vec[V_EG * 64 + tt] = __expf(G[i]);
+                vec[V_G2 * 64 + tt] = G[i] * 1.4426950408889634f;
+                vec[V_ET * 64 + tt] = __expf(gl - G[i]);
+            }
+            if (lane == 0) vec[V_N * 64] = (float)n;
+        };
         bool to = false;
-        // padding rows of chunk j's raw K, Q and V (zeroed so that no padding value reaches a product), then the
-        // hand-offs that let the MMA warp read them; then T' diag(e^G/|k|) of chunk j
-        auto stage_in = [&](int j) -> bool {
-            const int n = chunk_n(j);
-            bool t2 = !(wait(B_FULL_KQ + j % NKQ, (j / NKQ) & 1) && wait(B_FULL_V + j % NVS, (j / NVS) & 1) &&
-                        wait(B_FULL_AX + j % NAX, (j / NAX) & 1));
-            if (named_sync_or(BAR_PREP, NPREP, t2)) return false;
-            if (n < C) {
-                uint8_t *kq = sm + OFF_KQ + (j % NKQ) * KQ_STAGE;
-                uint8_t *vv = sm + OFF_V + (j % NVS) * 16384;
-                for (int e = p; e < (C - n) * 8 * 6; e += NPREP) {  // 6 tiles x (C - n) rows x 8 chunks
-                    const int tile = e / ((C - n) * 8), r = n + (e / 8) % (C - n), c8 = e & 7;
-                    uint8_t *base = tile < 4 ? kq + tile * 8192 : vv + (tile - 4) * 8192;
-                    *reinterpret_cast<uint4 *>(base + r * 128 + c8 * 16) = make_uint4(0, 0, 0, 0);
+        float rbN[2] = {0.f, 0.f}, rgN[2] = {0.f, 0.f};
+        if (nvalid > 0) {
+            load_raw(0, rbN, rgN);
+            chunk_vectors(0, rbN, rgN);
+        }
+        if (lane == 1 && nvalid > 0) {
+            issue_k(0);
+            issue_q(0);
+            issue_v(0);
+            if (nvalid > 1) prefetch_l2(1);
+        }
+        __syncwarp();
+        for (int c = 0; c < nvalid; ++c) {
+            const uint32_t par = c & 1;
+            if (c + 1 < nvalid) load_raw(c + 1, rbN, rgN);
+            // H0: the prep group is at chunk c (and, for a last partial chunk, has zeroed its padding rows)
+            if (named_sync_or(BAR_PCTL, NPC, to)) break;
+            if (lane == 0) {  // a2: the Gram [K; Q][K; Q]^T ([Q; K][Q; K]^T for odd chunks); its diagonal gives
+                              // the row norms
+                if (!bw(bar_ld, par)) to = true;
+                tc_fence_after();
+                const uint32_t id = idesc_t<T>(128, 128, false, false);
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    const uint32_t addr = sbase + off_gram(par, k >> 2) + (k & 3) * 32;
+                    mma_bf16(tmem + TM_GPW, sdesc_sw128(addr, 16, 1024), sdesc_sw128(addr, 16, 1024), id, k > 0);
+                }
+                mma_commit(bar_gp);
+            }
+            if (lane == 1) {
+                // V and the other K buffer were last read by the W/U MMAs of chunk c-1, issued a whole chunk
+                // ago; V of this chunk is needed only at its own W/U MMAs, K and Q of the next chunk at its
+                // Gram.  Q is free once this chunk's Gram has read it.
+                if (c > 0 && !bw(bar_wu, (c - 1) & 1)) to = true;
+                if (c > 0) issue_v(c);
+                if (c + 1 < nvalid) {
+                    // the K/Q barrier is armed for chunk c+1 only after its phase for chunk c has completed (an
+                    // arrival on a phase still pending would count towards that phase)
+                    if (!bw(bar_ld, par)) to = true;
+                    issue_k(c + 1);
+                    if (bw(bar_gp, par)) issue_q(c + 1);
+                    else to = true;
+                    if (c + 2 < nvalid) prefetch_l2(c + 2);
+                }
+            }
+            __syncwarp();
+            // while the prep group solves chunk c: the vectors of chunk c+1, into the set that chunk c-1
+            // used (free once the carry's MMA2 of chunk c-1 completed)
+            if (c + 1 < nvalid) {
+                if (c >= 1 && !bw(bar_pf + ((c + 1) & 1), ((c - 1) >> 1) & 1)) to = true;
+                chunk_vectors(c + 1, rbN, rgN);
+            }
+            __syncwarp();
+            if (lane == 0 && c + 1 < nvalid) mbar_arrive(bar_vr);
+        }
+    } else if (helper) {
+        // ============================== helper warps ==============================
+        // K~ = diag(e^{G_last - G} / |k|) K of each chunk, in place in the carry's raw K tile (rows past the
+        // length, whatever they hold, become zero): the A operand of the state update, made off the carry's
+        // serial chain.  The tile of chunk c lands after MMA2 of chunk c-1 and is needed at MMA2 of chunk c.
+        const int hp = tid - (CTL_WARP + 1) * 32;
+        bool to = false;
+        for (int c = 0; c < nvalid; ++c) {
+            const uint32_t par = c & 1;
+            const float *vec = vecs + par * NVEC * 64;
+            // bar_go of chunk c+1 follows bar_kt of chunk c, and the K tile of chunk c+1 is loaded after MMA2 of
+            // chunk c, which waits for bar_kt of chunk c: neither wait can be a phase behind
+            if (!bw(bar_go, par)) to = true;
+            if (!bw(bar_ck, par)) to = true;
+            if (!to) {
+                const int n = (int)vec[V_N * 64];
+                const float *vtail = vec + V_TAIL * 64;
+                for (int e = hp; e < 1024; e += NHELP) {
+                    const int t = (e >> 3) & 63;
+                    uint4 *pk = reinterpret_cast<uint4 *>(sm + OFF_KT + (e >> 9) * 8192 + t * 128 + (e & 7) * 16);
+                    float f[8];
+                    unpack8<T>(*pk, f);
+                    const float sc = vtail[t];
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) f[j] = t < n ? f[j] * sc : 0.f;
+                    *pk = pack8<T>(f);
+                }
+            }
+            fence_proxy_async_smem();
+            if (named_sync_or(BAR_HELP, NHELP, to)) break;
+            if (hp == 0) mbar_arrive(bar_kt);
+        }
+        if (to && hp == 0) *s_abort = 1;
+    } else if (!carry) {
+        // =============================== prep group ===============================
+        const int p = tid - NGRP;
+        bool to = false;  // a wait of this thread timed out
+        auto wait_ok = [&](uint64_t *bar, uint32_t parity) {
+            if (!bw(bar, parity)) to = true;
+        };
+        for (int c = 0; c < nvalid; ++c) {
+            const uint32_t par = c & 1;
+            float *vec = vecs + par * NVEC * 64;
+            float *vBeta = vec + V_BETA * 64, *vEG = vec + V_EG * 64;
+            float *vRk = vec + V_RK * 64, *vRq = vec + V_RQ * 64, *vCw = vec + V_CW * 64;
+            uint8_t *pm = sm + (par ? OFF_PM1 : OFF_PM0);
+            const int n = min(C, L - c * C);
+            // Pm buffer `par` and the norm vectors of set `par` were last read for chunk c-2, before its MMA2
+            // Pm buffer `par` and the norm vectors of set `par` were last read for chunk c-2, before its MMA2;
+            // the control warp waited for that MMA2 before it wrote chunk c's gate vectors, ahead of H0.
+            PHASE(26);
+            if (n < C) {  // padding rows of the last chunk's K and Q: zero them so no padding value reaches a product
+                wait_ok(bar_ld, par);
+                for (int e = p; e < (C - n) * 32; e += NGRP) {
+                    const int r = n + e / 32, k = e % 32, tile = k >> 3;
+                    const uint32_t base = (tile & 1) ? off_q(tile >> 1) : off_k(par, tile >> 1);
+                    *reinterpret_cast<uint4 *>(sm + base + r * 128 + (k & 7) * 16) = make_uint4(0, 0, 0, 0);
                 }
                 fence_proxy_async_smem();
             }
-            named_sync(BAR_PREP, NPREP);
-            if (p == 0) {
-                mbar_arrive(bars + B_KQ_OK);
-                mbar_arrive(bars + B_V_OK);
-            }
-            // T' diag(cw): column factors of T' (the B operand of W^T = K^T (T' diag(cw))^T)
-            const uint8_t *tp = sm + OFF_TPS + (j % NAX) * 8192;
-            const float *cw = vec_of(j) + V_CW * 64;
-            for (int e = p; e < 512; e += NPREP) {
-                const int t = e >> 3, pos = e & 7, s0 = ((pos ^ (t & 7)) * 8);
-                float f[8];
-                unpack8<T>(*reinterpret_cast<const uint4 *>(tp + t * 128 + pos * 16), f);
-#pragma unroll
-                for (int i = 0; i < 8; ++i) f[i] *= cw[s0 + i];
-                *reinterpret_cast<uint4 *>(sm + OFF_TW + t * 128 + pos * 16) = pack8<T>(f);
-            }
-            fence_proxy_async_smem();
-            named_sync(BAR_PREP, NPREP);
-            if (p == 0) mbar_arrive(bars + B_TW);
-            return true;
-        };
-        if (nvalid > 0 && !stage_in(0)) to = true;
-        for (int c = 0; !to && c < nvalid; ++c) {
-            const uint32_t par = c & 1;
-            const int n = chunk_n(c);
-            const float *vc = vec_of(c);
-            // ---- -W^T of chunk c into the MN-major B tile [dk][t] ----
-            bool t2 = !wait(B_W_DONE, par);
-            if (named_sync_or(BAR_PREP, NPREP, t2)) { to = true; break; }
+            // H0: the control warp (which wrote chunk c's gate vectors during chunk c-1) issues the Gram
+            if (named_sync_or(BAR_PCTL, NPC, to)) break;
+            PHASE(0);
+            wait_ok(bar_gp, par);
             tc_fence_after();
-            {
-                const int dk = q4 * 32 + lane;
+            PHASE(3);
+            // Each thread takes its Gram row's 32 columns of [K; Q] K^T (lanes 0..63: k_t.k_s, lanes
+            // 64..127: q_t.k_s); the blocks wholly above the diagonal are never read.  The diagonal
+            // gives |k_t|^2 and (from the q_t.q_s columns) |q_t|^2.
+            // Even chunks: TMEM lanes 0..63 hold the k rows and 64..127 the q rows, columns 0..63 the k
+            // columns; odd chunks ([Q; K]) swap both.  A warp of the "k role" builds rows of A, one of the
+            // "q role" rows of Pm; qa is the 32-row block of the chunk its lanes cover.
+            const bool krole = (q4 >> 1) == (int)par;
+            const int qa = q4 & 1, kcol = par ? 64 : 0, qcol = par ? 0 : 64;
+            const bool need = !(qa == 0 && hf == 1);
+            if (qa == hf) {
+                // |k_t|^2 / |q_t|^2 is the diagonal entry of this thread's row: entry `lane` of the 32 columns
+                // its warp loads
+                float d32[32];
+                tmem_ld32(tmem + TM_GPW + lane_base + (krole ? kcol : qcol) + 32 * hf, d32);
+                tmem_ld_wait();
+                float d = 0.f;
 #pragma unroll
-                for (int hv = 0; hv < 2; ++hv) {
-                    float w[32];
-                    tmem_ld32(tmem + TM_W + lane_base + 32 * hv, w);
+                for (int j = 0; j < 32; ++j) d = (j == lane) ? d32[j] : d;
+                const int t = row & 63;
+                const float r = t < n ? (a.l2norm ? rsqrtf(d + a.eps) : 1.f) : 0.f;
+                if (krole) {
+                    vRk[t] = r;
+                    vec[V_TAIL * 64 + t] = vec[V_ET * 64 + t] * r;
+                    vCw[t] = vBeta[t] * vEG[t] * r;
+                    // padding rows have 1/|k| = 0, so their lambda is +inf and their entries vanish
+                    vec[V_LAM * 64 + t] = vec[V_G2 * 64 + t] - lg2_approx(r);
+                } else {
+                    vRq[t] = a.scale * r;
+                    vec[V_XS * 64 + t] = vEG[t] * a.scale * r;
+                }
+            }
+            // the TT area (which takes plain A next) is free once the W/U MMAs of chunk c-1 completed
+            if (p == 0 && c > 0) wait_ok(bar_wu, (c - 1) & 1);
+            named_sync(BAR_PREP, NGRP);
+            PHASE(4);
+            // A rows (k role, fp32 for the solve) and Pm rows (q role, bf16 operand of the carry's o MMA), with
+            // the decay e^{G_t - G_s} taken per entry
+            {
+                const int t = row & 63;
+                if (need) {
+                    float v[32];
+                    tmem_ld32(tmem + TM_GPW + lane_base + kcol + 32 * hf, v);
+                    const float g2t = vec[V_G2 * 64 + t];
+                    // row factor: beta_t / |k_t| for A, scale / |q_t| for Pm (zero past the length)
+                    const float rf = t < n ? (krole ? vBeta[t] * vRk[t] : vRq[t]) : 0.f;
+                    const float4 *lam4 = reinterpret_cast<const float4 *>(vec + V_LAM * 64 + 32 * hf);
                     tmem_ld_wait();
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) w[i] = -w[i];
+                    for (int j4 = 0; j4 < 8; ++j4) {
+                        const float4 l = lam4[j4];
+                        v[4 * j4 + 0] *= rf * ex2_approx(g2t - l.x);
+                        v[4 * j4 + 1] *= rf * ex2_approx(g2t - l.y);
+                        v[4 * j4 + 2] *= rf * ex2_approx(g2t - l.z);
+                        v[4 * j4 + 3] *= rf * ex2_approx(g2t - l.w);
+                    }
+                    if (krole && hf == qa) {
+                        // a diagonal 32 x 32 block, plain (entries on or above the diagonal are never read)
+                        float *ap = reinterpret_cast<float *>(sm + OFF_AP) + pl(t, 0);
+#pragma unroll
+                        for (int j4 = 0; j4 < 8; ++j4)
+                            *reinterpret_cast<float4 *>(ap + 4 * j4) =
+                                make_float4(v[4 * j4], v[4 * j4 + 1], v[4 * j4 + 2], v[4 * j4 + 3]);
+                    } else if (krole) {  // A21 (rows 32..63, columns 0..31), operand of the 32 -> 64 merge
+                        float *ap = reinterpret_cast<float *>(sm + OFF_A21) + (t - 32) * SP;
+#pragma unroll
+                        for (int j4 = 0; j4 < 8; ++j4)
+                            *reinterpret_cast<float4 *>(ap + 4 * j4) =
+                                make_float4(v[4 * j4], v[4 * j4 + 1], v[4 * j4 + 2], v[4 * j4 + 3]);
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) v[j] = (32 * hf + j <= t) ? v[j] : 0.f;
+#pragma unroll
+                        for (int c8 = 0; c8 < 4; ++c8)
+                            *reinterpret_cast<uint4 *>(pm + blk_off(t, 32 * hf + 8 * c8)) = pack8<T>(&v[8 * c8]);
+                    }
+                } else if (!krole) {  // Pm rows 0..31, columns 32..63: above the diagonal
 #pragma unroll
                     for (int c8 = 0; c8 < 4; ++c8)
-                        *reinterpret_cast<uint4 *>(sm + OFF_WT + blk_off(dk, 32 * hv + 8 * c8)) = pack8<T>(&w[8 * c8]);
+                        *reinterpret_cast<uint4 *>(pm + blk_off(t, 32 + 8 * c8)) = make_uint4(0, 0, 0, 0);
                 }
             }
             fence_proxy_async_smem();
             tc_fence_before();
-            named_sync(BAR_PREP, NPREP);
-            if (p == 0) {
-                mbar_arrive(bars + B_WT);
-                EVENT(c, 11);
+            named_sync(BAR_PREP, NGRP);
+            PHASE(5);
+            // ---- a3: T = (I + A)^{-1} and the bf16 operand TT = [T diag(beta); T diag(c_W)] ----
+            // T = [[T11, 0], [T21, T22]]: the diagonal 32 x 32 blocks on the CUDA cores (solve_diag16_merge), then
+            // T21 = -T22 (A21 T11) by the eight prep warps, one 16 x 8 tile each of X = A21 T11 and then of T21,
+            // on warp-level tf32 MMAs; the diagonal blocks go into TT meanwhile.
+            solve_diag16_merge(reinterpret_cast<const float *>(sm + OFF_AP), reinterpret_cast<float *>(sm + OFF_TP),
+                               reinterpret_cast<float *>(sm + OFF_XP), p);
+            PHASE(12);
+            const float *tpl = reinterpret_cast<const float *>(sm + OFF_TP);
+            float *xm = reinterpret_cast<float *>(sm + OFF_XM);
+            const int pw = p >> 5, rt = pw >> 2, ct = pw & 3, gq = lane >> 2, iq = lane & 3;
+            {
+                // X tile (rows 16 rt.., columns 8 ct..); T11 is lower triangular, so k-steps before ct add nothing
+                float d[4];
+                gemm32_tile(d, reinterpret_cast<const float *>(sm + OFF_A21), tpl, rt, ct, ct, 4, lane);
+                *reinterpret_cast<float2 *>(xm + (16 * rt + gq) * SP + 8 * ct + 2 * iq) = make_float2(d[0], d[1]);
+                *reinterpret_cast<float2 *>(xm + (16 * rt + gq + 8) * SP + 8 * ct + 2 * iq) = make_float2(d[2], d[3]);
             }
-            // ---- the Gram of chunk c has landed: Pm (rows t of lanes 0..63; the row factor scale/|q_t| is applied
-            // to o by the out warps) ----
-            t2 = !wait(B_P_DONE, par);
-            if (named_sync_or(BAR_PREP, NPREP, t2)) { to = true; break; }
+            {
+                // TT rows of the diagonal blocks (and zeros above them), while other warps finish X
+                const int blk = p >> 7, t = (p >> 2) & 31, c8 = p & 3, R = 32 * blk + t, col = 32 * blk + 8 * c8;
+                const float *tp = tpl + pl(R, col);
+                const float4 u0 = *reinterpret_cast<const float4 *>(tp), u1 = *reinterpret_cast<const float4 *>(tp + 4);
+                const float tv[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+                float fb[8], fw[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    fb[i] = tv[i] * vBeta[col + i];
+                    fw[i] = tv[i] * vCw[col + i];
+                }
+                *reinterpret_cast<uint4 *>(sm + OFF_TT + blk_off(R, col)) = pack8<T>(fb);
+                *reinterpret_cast<uint4 *>(sm + OFF_TT + blk_off(64 + R, col)) = pack8<T>(fw);
+                // zeros: TT rows 0..31 and 64..95, columns 32..63 (above the diagonal)
+                const int Rz = (p >> 2) + ((p >> 7) << 5), cz = 4 + (p & 3);
+                *reinterpret_cast<uint4 *>(sm + OFF_TT + blk_off(Rz, 8 * cz)) = make_uint4(0, 0, 0, 0);
+            }
+            named_sync(BAR_PREP, NGRP);
+            PHASE(13);
+            {
+                // T21 tile = -(T22 X): T22 is lower triangular, so rows 16 rt.. need k-steps up to 2 rt + 1 only;
+                // straight into TT rows 32 + r (times beta_s) and 96 + r (times c_W,s), columns s < 32
+                float d[4];
+                gemm32_tile(d, tpl + 32 * SP, xm, rt, ct, 0, 2 * rt + 2, lane);
+                const int s0 = 8 * ct + 2 * iq;
+                const float b0 = vBeta[s0], b1 = vBeta[s0 + 1], w0 = vCw[s0], w1 = vCw[s0 + 1];
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    const int r = 16 * rt + gq + 8 * hh;
+                    const float t0 = -d[2 * hh], t1 = -d[2 * hh + 1];
+                    *reinterpret_cast<uint32_t *>(sm + OFF_TT + blk_off(32 + r, s0)) = TcT<T>::pack2(t0 * b0, t1 * b1);
+                    *reinterpret_cast<uint32_t *>(sm + OFF_TT + blk_off(96 + r, s0)) = TcT<T>::pack2(t0 * w0, t1 * w1);
+                }
+            }
+            PHASE(14);
+            PHASE(6);
+            PHASE(7);
+            if (n < C) {  // padding rows of the last chunk's V, once it has landed
+                wait_ok(bar_ldv, par);
+                for (int e = p; e < (C - n) * 16; e += NGRP) {
+                    const int r = n + e / 16, k = e % 16;
+                    *reinterpret_cast<uint4 *>(sm + OFF_V + (k >> 3) * 8192 + r * 128 + (k & 7) * 16) = make_uint4(0, 0, 0, 0);
+                }
+            }
+            // hand the chunk over: the carry group issues W and U from TT (it owns TMEM R and U, so they are
+            // free in its own program order), waits for them and moves W into A1
+            fence_proxy_async_smem();
+            tc_fence_before();
+            named_sync(BAR_PREP, NGRP);
+            if (p == 0) mbar_arrive(bar_a1);
+            PHASE(8);
+        }
+        if (to && p == 0) *s_abort = 1;
+    } else {
+        // =============================== carry group ==============================
+        bool to = false;  // a wait of this thread timed out
+        bool stop = false;
+        auto wait_ok = [&](uint64_t *bar, uint32_t parity) {
+            if (!bw(bar, parity)) to = true;
+        };
+        for (int c = 0; c < nvalid; ++c) {
+            const uint32_t par = c & 1;
+            const float *vec = vecs + par * NVEC * 64;
+            if (!bw(bar_a1, par)) to = true;
+            wait_ok(bar_cq, par);
+            if (named_sync_or(BAR_CARRY, NGRP, to)) { stop = true; break; }
+            PHASE(21);
+            if (tid == 0) mbar_arrive(bar_go);
+            if (tid == 0) {  // a4: W (rows 64..127 of TT K, into TMEM R) and U (rows 0..63 of TT V)
+                if (!bw(bar_ldv, par)) to = true;
+                tc_fence_after();
+                const uint32_t id = idesc_t<T>(128, 128, false, true);
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const uint64_t ad = sdesc_sw128(sbase + OFF_TT + k * 32, 16, 1024);
+                    mma_bf16(tmem + TM_R, ad, sdesc_sw128(sbase + off_k(par, 0) + k * 2048, KQ_BLK, 1024), id, k > 0);
+                    mma_bf16(tmem + TM_U, ad, sdesc_sw128(sbase + OFF_V + k * 2048, 8192, 1024), id, k > 0);
+                }
+                mma_commit(bar_wu);
+            }
+            wait_ok(bar_wu, par);
             tc_fence_after();
-            if (q4 < 2) {
-                const int t = q4 * 32 + lane;
-                const bool valid = t < n;
-                const float g2t = vc[V_G2 * 64 + t];
-                uint8_t *pm = sm + OFF_PM + par * 8192;
+            PHASE(22);
+            if (q4 >= 2) {  // W rows (TMEM lanes 64..127 of R) -> rows 0..63 of A1
+                const int t = row - 64;
 #pragma unroll
-                for (int hv = 0; hv < 2; ++hv) {
+                for (int half = 0; half < 2; ++half) {
+                    float w[32];
+                    tmem_ld32(tmem + TM_R + lane_base + 64 * hf + 32 * half, w);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int c8 = 0; c8 < 4; ++c8)
+                        *reinterpret_cast<uint4 *>(sm + OFF_A1 + hf * 16384 + blk_off(t, 32 * half + 8 * c8)) =
+                            pack8<T>(&w[8 * c8]);
+                }
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            named_sync(BAR_CARRY, NGRP);
+            tc_fence_after();
+            PHASE(16);
+            const int n = (int)vec[V_N * 64];
+            const float eL = vec[V_EG * 64 + C - 1];
+            // ---- R = [W; Q] S ----
+            if (tid == 0) {
+                const uint32_t id = idesc_t<T>(128, 128, false, true);
+                TIMED(23, {
+                    _Pragma("unroll")
+                    for (int k = 0; k < 8; ++k) {
+                        const uint64_t ad = sdesc_sw128(sbase + OFF_A1 + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024);
+                        const uint64_t bd = sdesc_sw128(sbase + OFF_S + k * 2048, 16384, 1024);
+                        mma_bf16(tmem + TM_R, ad, bd, id, k > 0);
+                    }
+                    mma_commit(bar_m1);
+                });
+            }
+            // S <- e^{G_last} S in TMEM, onto which MMA2 accumulates (for c > 0 the previous chunk's
+            // epilogue already wrote the scaled state back)
+            if (c == 0) {
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
                     float v[32];
-                    if (hv == 1 && q4 == 0) {  // rows 0..31, columns 32..63: above the diagonal
+                    const uint32_t ta = tmem + TM_S + lane_base + 64 * hf + 32 * half;
+                    tmem_ld32(ta, v);
+                    tmem_ld_wait();
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) v[i] = 0.f;
-                    } else {
-                        tmem_ld32(tmem + TM_P + lane_base + 32 * hv, v);
+                    for (int j = 0; j < 32; ++j) v[j] *= eL;
+                    tmem_st32(ta, v);
+                }
+                tmem_st_wait();
+            }
+            wait_ok(bar_m1, par);
+            if (tid == 0 && c + 1 < nvalid) load_carry_q(c + 1);  // the Q rows of A1 are read
+            if (tid == kStorer) bulk_wait_read0();  // the previous out tile (same buffer as v_new) is read
+            tc_fence_before();
+            if (named_sync_or(BAR_CARRY, NGRP, to)) { stop = true; break; }
+            tc_fence_after();
+            PHASE(17);
+            if (q4 < 2) {  // v_new = U - W S for token t, dv columns [64 hf, +64)
+                const int t = row;
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
+                    float u[32], r[32];
+                    tmem_ld32(tmem + TM_U + lane_base + 64 * hf + 32 * half, u);
+                    tmem_ld32(tmem + TM_R + lane_base + 64 * hf + 32 * half, r);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) u[j] = t < n ? u[j] - r[j] : 0.f;
+#pragma unroll
+                    for (int c8 = 0; c8 < 4; ++c8)
+                        *reinterpret_cast<uint4 *>(sm + OFF_VO + hf * 8192 + blk_off(t, 32 * half + 8 * c8)) =
+                            pack8<T>(&u[8 * c8]);
+                }
+            } else {  // rows of Q S: scale by e^{G_t} scale / |q_t| before Pm v_new accumulates onto them
+                if (a.epi_z && row - 64 < n)  // this thread's half row of z, for the epilogue
+                    asm volatile("prefetch.global.L1 [%0];" ::"l"(static_cast<const T *>(a.epi_z) +
+                                                                    ((size_t)bh * S + (size_t)c * C + row - 64) * D +
+                                                                    64 * hf));
+                const float xs = vec[V_XS * 64 + row - 64];
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
+                    float r[32];
+                    const uint32_t ta = tmem + TM_R + lane_base + 64 * hf + 32 * half;
+                    tmem_ld32(ta, r);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) r[j] *= xs;
+                    tmem_st32(ta, r);
+                }
+                tmem_st_wait();
+            }
+            // e^{G_last} of the next chunk (for the state written back after MMA2), read before this chunk's MMA2:
+            // the control warp cannot get two chunks ahead of it then
+            const bool more = c + 1 < nvalid;
+            float eLn = 1.f;
+            if (more) {
+                wait_ok(bar_vr, par);
+                eLn = vecs[(par ^ 1) * NVEC * 64 + V_EG * 64 + C - 1];
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            if (named_sync_or(BAR_CARRY, NGRP, to)) { stop = true; break; }
+            tc_fence_after();
+            PHASE(18);
+            // ---- S += K~^T v_new ;  R[64:128] += Pm v_new ----
+            if (tid == 0) {
+                if (!bw(bar_kt, par)) to = true;  // K~ of this chunk (helper warps)
+                tc_fence_after();
+                const uint32_t id_s = idesc_t<T>(128, 128, true, true);
+                const uint32_t id_o = idesc_t<T>(128, 128, false, true);
+                const uint32_t pm_rows = sbase + (par ? OFF_PM1 : OFF_PM0) - 8192;
+                TIMED(24, {
+                    _Pragma("unroll")
+                    for (int k = 0; k < 4; ++k) {
+                        const uint64_t bd = sdesc_sw128(sbase + OFF_VO + k * 2048, 8192, 1024);
+                        mma_bf16(tmem + TM_S, sdesc_sw128(sbase + OFF_KT + k * 2048, 8192, 1024), bd, id_s, 1);
+                    }
+                    _Pragma("unroll")
+                    for (int k = 0; k < 4; ++k) {
+                        const uint64_t bd = sdesc_sw128(sbase + OFF_VO + k * 2048, 8192, 1024);
+                        mma_bf16(tmem + TM_R, sdesc_sw128(pm_rows + k * 32, 16, 1024), bd, id_o, 1);
+                    }
+                    mma_commit(bar_m2);
+                    mma_commit(bar_pf + par);
+                });
+            }
+            wait_ok(bar_m2, par);
+            if (tid == 0 && c + 1 < nvalid) load_carry_k(c + 1);  // the raw K tile is read
+            tc_fence_after();
+            if (named_sync_or(BAR_CARRY, NGRP, to)) { stop = true; break; }
+            PHASE(19);
+            // ---- S (fp32, TMEM) -> bf16 operand tile, and back to TMEM scaled by e^{G_last} of the next
+            // chunk (its gate vectors were written before this chunk was handed over);  o rows -> out tile ----
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                float v[32];
+                const uint32_t ta = tmem + TM_S + lane_base + 64 * hf + 32 * half;
+                tmem_ld32(ta, v);
+                tmem_ld_wait();
+#pragma unroll
+                for (int c8 = 0; c8 < 4; ++c8)
+                    *reinterpret_cast<uint4 *>(sm + OFF_S + hf * 16384 + blk_off(row, 32 * half + 8 * c8)) =
+                        pack8<T>(&v[8 * c8]);
+                if (more) {
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) v[j] *= eLn;
+                    tmem_st32(ta, v);
+                }
+            }
+            if (more) tmem_st_wait();
+            if (q4 >= 2) {
+                const int t = row - 64;
+                // epilogue: the row's squared norm from its two halves (this thread and the one of the other hf
+                // warp with the same lane), then o * inv * norm_w * silu(z) for this thread's 64 columns
+                const bool epi = a.epi_z != nullptr;
+                float inv = 1.f;
+                const T *zr = nullptr;
+                if (epi) {
+                    float ss = 0.f;
+#pragma unroll
+                    for (int half = 0; half < 2; ++half) {
+                        float o[32];
+                        tmem_ld32(tmem + TM_R + lane_base + 64 * hf + 32 * half, o);
                         tmem_ld_wait();
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) {
-                            const int s = 32 * hv + i;
-                            const float dec = kGate ? ex2_approx(g2t - vc[V_LAM * 64 + s]) : vc[V_CT * 64 + s];
-                            v[i] = (valid && s <= t) ? v[i] * dec : 0.f;
+                        for (int j = 0; j < 32; ++j) ss = fmaf(o[j], o[j], ss);
+                    }
+                    float *eps2 = reinterpret_cast<float *>(sm + OFF_EPI);
+                    eps2[hf * 64 + t] = ss;
+                    if (t < n)  // rows past the length are never read
+                        zr = static_cast<const T *>(a.epi_z) + ((size_t)bh * S + (size_t)c * C + t) * D + 64 * hf;
+                    named_sync(BAR_EPI, 128);
+                    inv = rsqrtf((eps2[t] + eps2[64 + t]) * (1.f / D) + a.epi_eps);
+                }
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
+                    float o[32];
+                    tmem_ld32(tmem + TM_R + lane_base + 64 * hf + 32 * half, o);
+                    tmem_ld_wait();
+                    if (epi && t < n) {
+#pragma unroll
+                        for (int c8 = 0; c8 < 4; ++c8) {
+                            float zf[8];
+                            unpack8<T>(*reinterpret_cast<const uint4 *>(zr + 32 * half + 8 * c8), zf);
+                            const float4 *wp = reinterpret_cast<const float4 *>(a.epi_w + 64 * hf + 32 * half + 8 * c8);
+                            const float4 w0 = wp[0], w1 = wp[1];
+                            const float wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+#pragma unroll
+                            for (int i = 0; i < 8; ++i) o[8 * c8 + i] *= inv * wv[i] * silu_out<T>(zf[i]);
                         }
                     }
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) o[j] = t < n ? o[j] : 0.f;
 #pragma unroll
                     for (int c8 = 0; c8 < 4; ++c8)
-                        *reinterpret_cast<uint4 *>(pm + blk_off(t, 32 * hv + 8 * c8)) = pack8<T>(&v[8 * c8]);
+                        *reinterpret_cast<uint4 *>(sm + OFF_VO + hf * 8192 + blk_off(t, 32 * half + 8 * c8)) =
+                            pack8<T>(&o[8 * c8]);
                 }
             }
             fence_proxy_async_smem();
             tc_fence_before();
-            named_sync(BAR_PREP, NPREP);
-            if (p == 0) {
-                EVENT(c, 12);
-                mbar_arrive(bars + B_PM);
-                mbar_arrive(bars + B_EMPTY_AX + c % NAX);  // done with chunk c's vectors
-            }
-            if (c + 1 < nvalid && !stage_in(c + 1)) { to = true; break; }
-        }
-        if (to && p == 0) stop();
-    } else if (warp >= W_OUT0) {
-        // ================================ out ================================
-        const int p = tid - W_OUT0 * 32, dv = q4 * 32 + lane;
-        const bool storer = p == 0;
-        const bool epi = a.epi_z != nullptr;
-        float *red = reinterpret_cast<float *>(sm + OFF_RED);
-        bool to = false;
-        float wdv = 1.f;
-        if (epi) wdv = a.epi_w[dv];
-        auto load_z = [&](int c) {
-            mbar_arrive_expect_tx(bars + B_Z, 16384);
-            tma_load_3d(sm + OFF_Z, &tm_z, bars + B_Z, 0, c * C, bh);
-            tma_load_3d(sm + OFF_Z + 8192, &tm_z, bars + B_Z, 64, c * C, bh);
-        };
-        float *rqs = reinterpret_cast<float *>(sm + OFF_RQ);  // scale / |q_t| of chunks j (set j % 2)
-        // Once the Gram of chunk j has read the raw Q rows: scale / |q_t| (eps inside the root; 0 past the length)
-        // and, with a gate, Q~ = diag(e^{G_t}) Q in place (the B operand of the chunk's o product).  Thread p takes
-        // half of row p / 2.
-        auto make_q = [&](int j) -> bool {
-            const int n = chunk_n(j);
-            bool t2 = !(wait(B_P_DONE, j & 1) && wait(B_FULL_AX + j % NAX, (j / NAX) & 1));
-            if (named_sync_or(BAR_OUT, NOUTW, t2)) return false;
-            const int t = p >> 1, hb = p & 1;
-            uint4 *qrow = reinterpret_cast<uint4 *>(sm + OFF_KQ + (j % NKQ) * KQ_STAGE + hb * 16384 + t * 128);
-            float ss = 0.f;
-#pragma unroll
-            for (int c8 = 0; c8 < 8; ++c8) {
-                float f[8];
-                unpack8<T>(qrow[c8], f);
-#pragma unroll
-                for (int i = 0; i < 8; ++i) ss = fmaf(f[i], f[i], ss);
-            }
-            ss += __shfl_xor_sync(0xffffffffu, ss, 1);
-            if (hb == 0) rqs[(j & 1) * 64 + t] = t < n ? a.scale * (a.l2norm ? rsqrtf(ss + a.eps) : 1.f) : 0.f;
-            if (kGate) {
-                const float eg = t < n ? vec_of(j)[V_EG * 64 + t] : 0.f;
-#pragma unroll
-                for (int c8 = 0; c8 < 8; ++c8) {
-                    float f[8];
-                    unpack8<T>(qrow[c8], f);
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) f[i] *= eg;
-                    qrow[c8] = pack8<T>(f);
-                }
-                fence_proxy_async_smem();
-            }
-            named_sync(BAR_OUT, NOUTW);
-            if (storer) {
-                EVENT(j, 13);
-                mbar_arrive(bars + B_QK);
-                mbar_arrive(bars + B_EMPTY_AX + j % NAX);  // done with chunk j's vectors
-            }
-            return true;
-        };
-        int z_issued = 0;
-        if (epi && nvalid > 0 && storer) {
-            // the z tile shares its space with the initial state: wait until the carry has read it
-            if (a.initial_state && !wait(B_S0_FREE, 0)) to = true;
-            if (!to) {
-                load_z(0);
-                ++z_issued;
-            }
-        }
-        if (nvalid > 0 && !make_q(0)) to = true;
-        for (int c = 0; !to && c < nvalid; ++c) {
-            const uint32_t par = c & 1;
-            const int n = chunk_n(c);
-            if (c + 1 < nvalid && !make_q(c + 1)) { to = true; break; }
-            bool t2 = !wait(B_O_DONE, par);
-            if (named_sync_or(BAR_OUT, NOUTW, t2)) { to = true; break; }
+            named_sync(BAR_CARRY, NGRP);
             tc_fence_after();
-            float o[2][32];  // o[hv][i]: token 32 hv + i of this lane's value column
-            tmem_ld32(tmem + TM_R + 64 + lane_base, o[0]);
-            tmem_ld32(tmem + TM_R + 96 + lane_base, o[1]);
-            tmem_ld_wait();
-            tc_fence_before();
-            if (storer) bulk_wait_read0();  // the previous out tile has been read by its store
-            named_sync(BAR_OUT, NOUTW);
-            if (storer) mbar_arrive(bars + B_O_READ);
-            {
-                const float *rq = rqs + par * 64;
-#pragma unroll
-                for (int t = 0; t < 64; ++t) o[t >> 5][t & 31] *= rq[t];
-            }
-            if (epi) {
-                // sum over the head's Dv outputs of o^2 for each token: reduce-scatter inside the warp (lane l
-                // ends with tokens 2l, 2l+1), then over the four warps through shared memory
-                // (per half of the tokens: lane l ends with token 32 hv + l)
-#pragma unroll
-                for (int hv = 0; hv < 2; ++hv) {
-                    float x[32];
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) x[i] = o[hv][i] * o[hv][i];
-#pragma unroll
-                    for (int w = 16, off = 16; off >= 1; w >>= 1, off >>= 1) {
-                        const bool up = lane & off;
-#pragma unroll
-                        for (int i = 0; i < w; ++i) {
-                            const float send = up ? x[i] : x[i + w];
-                            const float keep = up ? x[i + w] : x[i];
-                            x[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
-                        }
-                    }
-                    red[q4 * 64 + 32 * hv + lane] = x[0];
-                }
-                named_sync(BAR_OUT, NOUTW);
-                if (p < C) {
-                    const float ssq = red[p] + red[64 + p] + red[128 + p] + red[192 + p];
-                    red[256 + p] = rsqrtf(ssq * (1.f / D) + a.epi_eps);
-                }
-                bool t3 = !wait(B_Z, par);
-                if (named_sync_or(BAR_OUT, NOUTW, t3)) { to = true; break; }
-                const uint8_t *zt = sm + OFF_Z + (dv >> 6) * 8192;
-#pragma unroll
-                for (int t = 0; t < 64; ++t) {
-                    const uint16_t zr = *reinterpret_cast<const uint16_t *>(zt + blk_off(t, dv & 63));
-                    const float zf = TcT<T>::unpack2((uint32_t)zr).x;
-                    o[t >> 5][t & 31] *= red[256 + t] * wdv * silu_out<T>(zf);
-                }
-                named_sync(BAR_OUT, NOUTW);  // the z tile and the factors are read
-                if (storer && c + 1 < nvalid) {
-                    load_z(c + 1);
-                    ++z_issued;
-                }
-            }
-            // out rows t < n; zero past the length.  Neighbouring lanes exchange values so that each stores
-            // 32-bit words of one row.
-            uint8_t *ot = sm + OFF_OUT + (dv >> 6) * 8192;
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                const float x0 = 2 * i < n ? o[i >> 4][(2 * i) & 31] : 0.f;
-                const float x1 = 2 * i + 1 < n ? o[i >> 4][(2 * i + 1) & 31] : 0.f;
-                const uint32_t wv = pair_word<T>(x0, x1, lane);
-                const int row = 2 * i + (lane & 1), col = (dv & 63) & ~1;
-                *reinterpret_cast<uint32_t *>(ot + blk_off(row, col)) = wv;
-            }
-            fence_proxy_async_smem();
-            named_sync(BAR_OUT, NOUTW);
-            if (storer) {
-                tma_store_3d(&tm_o, sm + OFF_OUT, 0, c * C, bh);
-                tma_store_3d(&tm_o, sm + OFF_OUT + 8192, 64, c * C, bh);
+            if (tid == kStorer) {
+                tma_store_3d(&tm_o, sm + OFF_VO, 0, c * C, bh);
+                tma_store_3d(&tm_o, sm + OFF_VO + 8192, 64, c * C, bh);
                 bulk_commit();
             }
+            PHASE(20);
         }
-        if (!to && nvalid < ntotal) {  // chunks past the length: zero rows
-            // with no valid chunk the out tile may still hold the initial state: wait until the carry is done
-            bool t2 = false;
-            if (nvalid == 0 && a.initial_state) t2 = !wait(B_S0_FREE, 0);
-            if (storer) bulk_wait_read0();
-            if (!named_sync_or(BAR_OUT, NOUTW, t2)) {
-                for (int e = p; e < 16384 / 16; e += NOUTW)
-                    reinterpret_cast<uint4 *>(sm + OFF_OUT)[e] = make_uint4(0, 0, 0, 0);
+        if (stop && tid == 0) *s_abort = 1;
+        if (!stop) {
+            // chunks past the length: zero rows
+            if (nvalid < ntotal) {
+                if (tid == kStorer) bulk_wait_read0();
+                named_sync(BAR_CARRY, NGRP);
+                for (int e = tid; e < 16384 / 16; e += NGRP)
+                    reinterpret_cast<uint4 *>(sm + OFF_VO)[e] = make_uint4(0, 0, 0, 0);
                 fence_proxy_async_smem();
-                named_sync(BAR_OUT, NOUTW);
-                if (storer) {
+                named_sync(BAR_CARRY, NGRP);
+                if (tid == kStorer) {
                     for (int c = nvalid; c < ntotal; ++c) {
-                        tma_store_3d(&tm_o, sm + OFF_OUT, 0, c * C, bh);
-                        tma_store_3d(&tm_o, sm + OFF_OUT + 8192, 64, c * C, bh);
+                        tma_store_3d(&tm_o, sm + OFF_VO, 0, c * C, bh);
+                        tma_store_3d(&tm_o, sm + OFF_VO + 8192, 64, c * C, bh);
                     }
                     bulk_commit();
                 }
-            } else {
-                to = true;
             }
-        }
-        if (storer) {
-            bulk_wait0();
-            // drain the epilogue loads this warp issued
-            if (z_issued) mbar_wait_ns(bars + B_Z, (z_issued - 1) & 1, kDrainWaitNs);
-        }
-        if (to && storer) stop();
-    } else {
-        // ================================ carry ================================
-        const int hf = warp >> 2;          // key rows [64 hf, 64 hf + 64)
-        const int dv = q4 * 32 + lane;     // this thread's value column = TMEM lane
-        bool to = false;
-        float v[2][32];  // v[hv][i]: key row 64 hf + 32 hv + i of this lane's state column (initial state)
-        // the initial state column dv, rows 64 hf.. (fp32), from the staged tile
-        if (a.initial_state && nvalid > 0) {
-            bool t2 = !wait(B_S0, 0);
-            if (named_sync_or(BAR_CARRY, NCARRY, t2)) to = true;
-            if (!to) {
-                const uint8_t *st = sm + OFF_OUT + ((dv >> 6) * 2 + hf) * 8192;
+            if (a.final_state) {
+                T *fs = reinterpret_cast<T *>(a.final_state) + ((size_t)bh * D + row) * D + 64 * hf;
 #pragma unroll
-                for (int i = 0; i < 64; ++i) {
-                    const uint16_t r = *reinterpret_cast<const uint16_t *>(st + blk_off(i, dv & 63));
-                    v[i >> 5][i & 31] = TcT<T>::unpack2((uint32_t)r).x;
-                }
-            }
-        } else {
-#pragma unroll
-            for (int i = 0; i < 32; ++i) v[0][i] = v[1][i] = 0.f;
-        }
-        // the staged initial state is read (an empty sequence copies it out first, below)
-        if (nvalid > 0) {
-            named_sync(BAR_CARRY, NCARRY);
-            if (tid == 0) mbar_arrive(bars + B_S0_FREE);
-        }
-        // S^T of chunk j (in v): its 16-bit copy (the A operand of chunk j's v_new and o products), then the fp32
-        // state decayed by the chunk's e^{G_last}, onto which the chunk's state update accumulates (without a gate
-        // the fp32 state in TMEM is already the state, except before chunk 0)
-        auto put_state = [&](int j, float (&v)[2][32]) -> bool {
-#pragma unroll
-            for (int hv = 0; hv < 2; ++hv) {
-                uint32_t pk[16];
-#pragma unroll
-                for (int i = 0; i < 16; ++i) pk[i] = TcT<T>::pack2(v[hv][2 * i], v[hv][2 * i + 1]);
-                tmem_st16(tmem + ((j & 1) ? TM_SA1 : TM_SA0) + lane_base + 32 * hf + 16 * hv, pk);
-            }
-            tmem_st_wait();
-            tc_fence_before();
-            named_sync(BAR_CARRY, NCARRY);
-            if (tid == 0) {
-                mbar_arrive(bars + B_SA);
-                EVENT(j, 0);
-            }
-            // chunk j's vectors: e^{G_last} here, c_t at its v_new conversion
-            bool t2 = !wait(B_FULL_AX + j % NAX, (j / NAX) & 1);
-            if (named_sync_or(BAR_CARRY, NCARRY, t2)) return false;
-            if (kGate) {
-                const float eL = vec_of(j)[V_MISC * 64];
-                float w[32];
-#pragma unroll
-                for (int hv = 0; hv < 2; ++hv) {
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) w[i] = v[hv][i] * eL;
-                    tmem_st32(tmem + TM_S + lane_base + 64 * hf + 32 * hv, w);
-                }
-                tmem_st_wait();
-            } else if (j == 0) {
-#pragma unroll
-                for (int hv = 0; hv < 2; ++hv) tmem_st32(tmem + TM_S + lane_base + 64 * hf + 32 * hv, v[hv]);
-                tmem_st_wait();
-            }
-            tc_fence_before();
-            named_sync(BAR_CARRY, NCARRY);
-            if (tid == 0) {
-                mbar_arrive(bars + B_SD);
-                EVENT(j, 14);
-            }
-            return true;
-        };
-        if (!to && nvalid > 0 && !put_state(0, v)) to = true;
-        for (int c = 0; !to && c < nvalid; ++c) {
-            const uint32_t par = c & 1;
-            // ---- v_new^T (fp32, 32 of this lane's token columns) -> its 16-bit copy over the same columns ----
-            bool t2 = !wait(B_V_DONE, par);
-            if (named_sync_or(BAR_CARRY, NCARRY, t2)) { to = true; break; }
-            if (tid == 0) EVENT(c, 2);
-            tc_fence_after();
-            {
-                // tokens 32 hf .. 32 hf + 31: the plain copy (for o) and the copy scaled by
-                // c_t = e^{G_last - G_t}/|k_t| (for the state update), over the fp32 columns just read
-                const float *ct = vec_of(c) + V_CT * 64 + 32 * hf;
-                float u[32];
-                tmem_ld32(tmem + TM_R + lane_base + 32 * hf, u);
-                tmem_ld_wait();
-                uint32_t pk[16], ps[16];
-#pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    pk[i] = TcT<T>::pack2(u[2 * i], u[2 * i + 1]);
-                    ps[i] = TcT<T>::pack2(u[2 * i] * ct[2 * i], u[2 * i + 1] * ct[2 * i + 1]);
-                }
-                tmem_st16(tmem + TM_R + lane_base + 32 * hf, pk);
-                tmem_st16(tmem + TM_R + lane_base + 32 * hf + 16, ps);
-                tmem_st_wait();
-            }
-            tc_fence_before();
-            named_sync(BAR_CARRY, NCARRY);
-            if (tid == 0) {
-                mbar_arrive(bars + B_VA);
-                EVENT(c, 3);
-                mbar_arrive(bars + B_EMPTY_AX + c % NAX);  // done with chunk c's vectors
-            }
-            // ---- the updated state: 16-bit copy for the next chunk, decayed fp32 back ----
-            t2 = !wait(B_S_DONE, par);
-            if (named_sync_or(BAR_CARRY, NCARRY, t2)) { to = true; break; }
-            if (tid == 0) EVENT(c, 5);
-            if (c + 1 == nvalid) break;  // the final state stays in TMEM
-            tc_fence_after();
-            float sv[2][32];
-            tmem_ld32(tmem + TM_S + lane_base + 64 * hf, sv[0]);
-            tmem_ld32(tmem + TM_S + lane_base + 64 * hf + 32, sv[1]);
-            tmem_ld_wait();
-            if (!put_state(c + 1, sv)) { to = true; break; }
-        }
-        // ---- the final state (or the initial one, for an empty sequence) ----
-        if (!to && a.final_state) {
-            // staging: a K/Q stage no load or MMA uses any more (the initial-state tile for an empty sequence)
-            const bool copy = nvalid == 0 && a.initial_state;
-            uint8_t *st = copy ? sm + OFF_OUT : sm + OFF_KQ + (nvalid % NKQ) * KQ_STAGE;
-            bool t2 = copy && !wait(B_S0, 0);
-            if (named_sync_or(BAR_CARRY, NCARRY, t2)) to = true;
-            if (!copy && !to) {
-                float fv[2][32];
-                if (nvalid > 0) {  // S^T after the last chunk, fp32 in TMEM
-                    tc_fence_after();
-                    tmem_ld32(tmem + TM_S + lane_base + 64 * hf, fv[0]);
-                    tmem_ld32(tmem + TM_S + lane_base + 64 * hf + 32, fv[1]);
+                for (int half = 0; half < 2; ++half) {
+                    float v[32];
+                    tmem_ld32(tmem + TM_S + lane_base + 64 * hf + 32 * half, v);
                     tmem_ld_wait();
-                } else {
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) fv[0][i] = fv[1][i] = 0.f;
+                    for (int c8 = 0; c8 < 4; ++c8)
+                        *reinterpret_cast<uint4 *>(fs + 32 * half + 8 * c8) = pack8<T>(&v[8 * c8]);
                 }
-                uint8_t *bx = st + ((dv >> 6) * 2 + hf) * 8192;
-#pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    const uint32_t wv = pair_word<T>(fv[i >> 4][(2 * i) & 31], fv[i >> 4][(2 * i + 1) & 31], lane);
-                    const int row = 2 * i + (lane & 1), col = (dv & 63) & ~1;
-                    *reinterpret_cast<uint32_t *>(bx + blk_off(row, col)) = wv;
-                }
-            }
-            fence_proxy_async_smem();
-            named_sync(BAR_CARRY, NCARRY);
-            if (tid == 0 && !to) {
-                for (int bxi = 0; bxi < 4; ++bxi)
-                    tma_store_3d(&tm_fs, st + bxi * 8192, 64 * (bxi >> 1), 64 * (bxi & 1), bh);
-                bulk_commit();
-                bulk_wait0();
             }
         }
-        if (nvalid == 0 && tid == 0) mbar_arrive(bars + B_S0_FREE);  // the out warps may reuse the staging tile now
-        if (to && tid == 0) stop();
+        if (tid == kStorer) bulk_wait0();
+    }
+    // drain: every copy and MMA the CTA issued has completed before its shared memory and TMEM are released
+    // (normally each was consumed already; after a stop some may still be in flight)
+    if (control && lane == 1) {
+        if (n_ld) mbar_wait_ns(bar_ld, (n_ld - 1) & 1, kDrainWaitNs);
+        if (n_ldv) mbar_wait_ns(bar_ldv, (n_ldv - 1) & 1, kDrainWaitNs);
+    }
+    if (tid == 0) {
+        if (n_cq) mbar_wait_ns(bar_cq, (n_cq - 1) & 1, kDrainWaitNs);
+        if (n_ck) mbar_wait_ns(bar_ck, (n_ck - 1) & 1, kDrainWaitNs);
+    }
+    if ((control && lane == 0) || tid == 0) {
+        mma_commit(bar_dr);
+        mbar_wait_ns(bar_dr, 0, kDrainWaitNs);
     }
     tc_fence_before();
     __syncthreads();
     if (tid == 0 && *s_abort) raise_device_error(a.err, GDR_DEVERR_TIMEOUT);
 #ifdef GDR_PHASE_TIMERS
-    if (blockIdx.x == 0) {
-        if (tid == 0) {
-            s_wcyc[5 * 36] = (unsigned long long)(clock64() - t_start);
-            s_wcyc[5 * 36 + 1] = (unsigned long long)nvalid;
-        }
-        __syncthreads();
-        for (int i = tid; i < kTimerSlots; i += CH_THREADS) g_phase[i] += s_wcyc[i];
-    }
+    if (blockIdx.x == 0 && tid < 64) g_phase[tid] += s_phase_[tid];
 #endif
-    if (warp == 0) {
-        tc_fence_after();
-        tmem_dealloc(tmem, TM_COLS);
-    }
+    if (warp == 0) tmem_dealloc(tmem, TM_COLS);
 }
 
-// (inner, rows, Z) tensor of 2-byte elements (bf16 or fp16), 64 x 64 boxes, 128-byte swizzle.
-bool make_map(CUtensorMap *m, const void *base, int inner, long long rows, long long Z, CUtensorMapDataType type) {
+// (D, S, Z) tensor of 2-byte elements (bf16 or fp16), 64 x 64 boxes, 128-byte swizzle.
+bool make_map(CUtensorMap *m, const void *base, int S, long long Z, CUtensorMapDataType type) {
     EncodeTiledFn enc = tensor_map_encoder();
     if (!enc) return false;
-    cuuint64_t dims[3] = {(cuuint64_t)inner, (cuuint64_t)rows, (cuuint64_t)Z};
-    cuuint64_t strides[2] = {(cuuint64_t)inner * 2, (cuuint64_t)rows * inner * 2};
+    cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)S, (cuuint64_t)Z};
+    cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)S * D * 2};
     cuuint32_t box[3] = {64, 64, 1}, es[3] = {1, 1, 1};
-    return enc(m, type, 3, const_cast<void *>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
-               CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+    return enc(m, type, 3, const_cast<void *>(base), dims, strides, box, es,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 }  // namespace
 
+#ifdef GDR_PHASE_TIMERS
+extern "C" int gdr_phase_timers_read(unsigned long long *out) {
+    cudaDeviceSynchronize();
+    cudaMemcpyFromSymbol(out, g_phase, sizeof(unsigned long long) * 64);
+    unsigned long long z[64] = {0};
+    cudaMemcpyToSymbol(g_phase, z, sizeof(z));
+    return 0;
+}
+#endif
+
 bool chunk_tc_supported(int Dk, int Dv, gdr_dtype dt, int S) {
     return (dt == GDR_BF16 || dt == GDR_F16) && Dk == D && Dv == D && S > 0;
 }
 
-size_t chunk_tc_workspace(int B, int Nv, int S) {
-    const size_t nch = (size_t)B * Nv * (size_t)((S + C - 1) / C);
-    return nch * (kTpBytes + kVecBytes);
-}
-
 namespace {
-unsigned long long g_wait_ns = 0;  // 0: the default limit (a test may shorten it)
-
-template <typename T, bool kGate>
+template <typename T>
 cudaError_t launch_tc_t(const ChunkArgs &ca, cudaStream_t stream) {
     constexpr CUtensorMapDataType ty = TcT<T>::kMap;
-    const int NC = (ca.S + C - 1) / C;
-    const size_t nch = (size_t)ca.B * ca.Nv * NC;
-    if (nch == 0) return cudaSuccess;
-    uint8_t *ws = static_cast<uint8_t *>(ca.workspace);
-    float *vec = reinterpret_cast<float *>(ws + vec_offset(nch));
-
-    // ---- the WY pass over every chunk ----
-    WyArgs w{};
-    w.k = ca.k; w.beta = ca.beta; w.g = ca.g; w.lengths = ca.lengths;
-    w.B = ca.B; w.Nk = ca.Nk; w.Nv = ca.Nv; w.S = ca.S; w.NC = NC;
-    w.l2norm = ca.l2norm; w.eps = ca.eps; w.beta_logits = ca.beta_logits; w.A_log = ca.A_log; w.dt_bias = ca.dt_bias;
-    w.tp = ws;
-    w.vec = vec;
-    static LaunchCache wyc(reinterpret_cast<const void *>(wy_kernel<T, kGate>));
-    cudaError_t e = wyc.allow_smem((int)WY_SMEM);
-    if (e != cudaSuccess) return e;
-    const long long wy_blocks = (long long)ca.B * ca.Nk * NC;
-    if (wy_blocks >= (1LL << 31)) return cudaErrorInvalidValue;
-    wy_kernel<T, kGate><<<(unsigned)wy_blocks, WY_THREADS, WY_SMEM, stream>>>(w);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-
-    // ---- the chains ----
-    CUtensorMap mq, mk, mv, mo, mtp, ms0, mfs, mz;
-    memset(&ms0, 0, sizeof(ms0));
-    memset(&mfs, 0, sizeof(mfs));
-    memset(&mz, 0, sizeof(mz));
-    if (!make_map(&mq, ca.q, D, ca.S, (long long)ca.B * ca.Nk, ty) ||
-        !make_map(&mk, ca.k, D, ca.S, (long long)ca.B * ca.Nk, ty) ||
-        !make_map(&mv, ca.v, D, ca.S, (long long)ca.B * ca.Nv, ty) ||
-        !make_map(&mo, ca.out, D, ca.S, (long long)ca.B * ca.Nv, ty) ||
-        !make_map(&mtp, ws, C, C, (long long)nch, ty))
+    CUtensorMap mq, mk, mv, mo;
+    if (!make_map(&mq, ca.q, ca.S, (long long)ca.B * ca.Nk, ty) ||
+        !make_map(&mk, ca.k, ca.S, (long long)ca.B * ca.Nk, ty) ||
+        !make_map(&mv, ca.v, ca.S, (long long)ca.B * ca.Nv, ty) ||
+        !make_map(&mo, ca.out, ca.S, (long long)ca.B * ca.Nv, ty))
         return cudaErrorInvalidValue;
-    if (ca.initial_state && !make_map(&ms0, ca.initial_state, D, D, (long long)ca.B * ca.Nv, ty))
-        return cudaErrorInvalidValue;
-    if (ca.final_state && !make_map(&mfs, ca.final_state, D, D, (long long)ca.B * ca.Nv, ty))
-        return cudaErrorInvalidValue;
-    if (ca.epi_z && !make_map(&mz, ca.epi_z, D, ca.S, (long long)ca.B * ca.Nv, ty)) return cudaErrorInvalidValue;
-    ChainArgs a{};
-    a.initial_state = ca.initial_state; a.final_state = ca.final_state; a.lengths = ca.lengths; a.scale = ca.scale;
-    a.B = ca.B; a.Nk = ca.Nk; a.Nv = ca.Nv; a.S = ca.S; a.NC = NC;
-    a.l2norm = ca.l2norm; a.eps = ca.eps; a.vec = vec; a.err = ca.err;
+    TcArgs a{};
+    a.beta = ca.beta; a.g = ca.g; a.initial_state = ca.initial_state; a.lengths = ca.lengths; a.scale = ca.scale;
+    a.B = ca.B; a.Nk = ca.Nk; a.Nv = ca.Nv; a.S = ca.S; a.final_state = ca.final_state;
+    a.l2norm = ca.l2norm; a.eps = ca.eps; a.beta_logits = ca.beta_logits; a.A_log = ca.A_log;
+    a.dt_bias = ca.dt_bias; a.err = ca.err;
     a.epi_z = ca.epi_z; a.epi_w = ca.epi_w; a.epi_eps = ca.epi_eps;
-    a.wait_ns = g_wait_ns ? g_wait_ns : kDefaultWaitNs;
-    static LaunchCache plain(reinterpret_cast<const void *>(chain_kernel<T, kGate, false>));
-    static LaunchCache ordered(reinterpret_cast<const void *>(chain_kernel<T, kGate, true>));
+    a.wait_ns = chunk_wait_ns();
+    static LaunchCache plain(reinterpret_cast<const void *>(chunk_tc_kernel<T, false>));
+    static LaunchCache ordered(reinterpret_cast<const void *>(chunk_tc_kernel<T, true>));
     const long long blocks = (long long)ca.B * ca.Nv;
+    if (blocks == 0) return cudaSuccess;
     // longest sequences first only when the chains do not all start at once
     bool order = false;
     if (ca.lengths && ca.B > 1 && ca.B <= kRankMaxB) {
         int resident = 0;
-        if ((e = ordered.resident_grid(CH_THREADS, (int)CH_SMEM, &resident)) != cudaSuccess) return e;
+        cudaError_t e = ordered.resident_grid(NT, (int)SMEM_BYTES, &resident);
+        if (e != cudaSuccess) return e;
         order = blocks > resident;
     }
-    if ((e = (order ? ordered : plain).allow_smem((int)CH_SMEM)) != cudaSuccess) return e;
+    cudaError_t e = (order ? ordered : plain).allow_smem((int)SMEM_BYTES);
+    if (e != cudaSuccess) return e;
     if (order)
-        chain_kernel<T, kGate, true><<<(unsigned)blocks, CH_THREADS, CH_SMEM, stream>>>(mq, mk, mv, mo, mtp, ms0, mfs,
-                                                                                        mz, a);
+        chunk_tc_kernel<T, true><<<(unsigned)blocks, NT, SMEM_BYTES, stream>>>(mq, mk, mv, mo, a);
     else
-        chain_kernel<T, kGate, false><<<(unsigned)blocks, CH_THREADS, CH_SMEM, stream>>>(mq, mk, mv, mo, mtp, ms0,
-                                                                                         mfs, mz, a);
+        chunk_tc_kernel<T, false><<<(unsigned)blocks, NT, SMEM_BYTES, stream>>>(mq, mk, mv, mo, a);
     return cudaGetLastError();
 }
 }  // namespace
 
-void chunk_tc_set_wait_ns(unsigned long long ns) { g_wait_ns = ns; }
-
-#ifdef GDR_PHASE_TIMERS
-extern "C" int gdr_phase_events_read(long long *out) {
-    cudaDeviceSynchronize();
-    cudaMemcpyFromSymbol(out, g_events, sizeof(long long) * kEvN * kEvK);
-    return kEvN * kEvK;
-}
-extern "C" int gdr_phase_timers_read(unsigned long long *out) {
-    cudaDeviceSynchronize();
-    cudaMemcpyFromSymbol(out, g_phase, sizeof(unsigned long long) * kTimerSlots);
-    static unsigned long long z[kTimerSlots];
-    cudaMemcpyToSymbol(g_phase, z, sizeof(z));
-    return kTimerSlots;
-}
-#endif
-
-cudaError_t chunk_tc_take_timeout_site(unsigned int *site) {
-    unsigned int zero = 0;
-    cudaError_t e = cudaMemcpyFromSymbol(site, g_timeout_site, sizeof(unsigned int));
-    if (e == cudaSuccess) e = cudaMemcpyToSymbol(g_timeout_site, &zero, sizeof(unsigned int));
-    return e;
-}
-
 cudaError_t launch_chunk_tc(const ChunkArgs &ca, gdr_dtype dt, cudaStream_t stream) {
-    const bool gate = ca.g != nullptr;
-    if (dt == GDR_F16) return gate ? launch_tc_t<__half, true>(ca, stream) : launch_tc_t<__half, false>(ca, stream);
-    return gate ? launch_tc_t<__nv_bfloat16, true>(ca, stream) : launch_tc_t<__nv_bfloat16, false>(ca, stream);
+    return dt == GDR_F16 ? launch_tc_t<__half>(ca, stream) : launch_tc_t<__nv_bfloat16>(ca, stream);
 }
 
 }  // namespace gdr

@@ -48,7 +48,7 @@ struct ChunkArgs {
     const void *epi_z;
     const float *epi_w;
     float epi_eps;
-    // caller-owned scratch of the tensor-core path (chunk_tc_workspace bytes, 16-byte aligned)
+    // caller-owned scratch of the two-kernel tensor-core schedule (chunk_wy_workspace bytes, 16-byte aligned)
     void *workspace;
 };
 
@@ -79,15 +79,23 @@ class LaunchCache {
 };
 
 cudaError_t launch_decode(const DecodeArgs &a, int Dk, int Dv, gdr_dtype dt, gdr_dtype st, cudaStream_t s);
+// The tensor-core prefill (bf16 / fp16, Dk = Dv = 128) has two schedules:
+//   chunk_tc.cu  one kernel, one CTA per (b, value head) chain that also solves each chunk's WY system; needs no
+//                workspace;
+//   chunk_wy.cu  a WY pass over every chunk on every SM into a caller workspace, then a chain kernel that only
+//                carries the state; for few chains (B Nv at most a third of the SMs).
 bool chunk_tc_supported(int Dk, int Dv, gdr_dtype dt, int S);
-// bytes of workspace the tensor-core prefill needs: per (b, value head, 64-token chunk) the 64 x 64 16-bit T' and
-// six vectors of 64 floats
-size_t chunk_tc_workspace(int B, int Nv, int S);
 cudaError_t launch_chunk_tc(const ChunkArgs &a, gdr_dtype dt, cudaStream_t s);
-// limit of the tensor-core prefill's bounded waits, in ns (0: the default of one second)
+// bytes of workspace the two-kernel schedule needs: per (b, value head, 64-token chunk) the 64 x 64 16-bit T' and
+// six vectors of 64 floats
+size_t chunk_wy_workspace(int B, int Nv, int S);
+cudaError_t launch_chunk_wy(const ChunkArgs &a, gdr_dtype dt, cudaStream_t s);
+// limit of the tensor-core prefill's bounded waits, in ns (0: the default of one second); the value in force
 void chunk_tc_set_wait_ns(unsigned long long ns);
-// reads and clears the record of the first bounded wait of the tensor-core prefill that ran out (synchronous)
+unsigned long long chunk_wait_ns();
+// read and clear the record of the first bounded wait of each schedule that ran out (synchronous)
 cudaError_t chunk_tc_take_timeout_site(unsigned int *site);
+cudaError_t chunk_wy_take_timeout_site(unsigned int *site);
 cudaError_t launch_chunk_simt(const ChunkArgs &a, int Dk, int Dv, gdr_dtype dt, cudaStream_t s);
 // out rows t < L_b <- rmsnorm(out row) * norm_w * silu(z row), in place (the unfused epilogue)
 cudaError_t launch_gated_rmsnorm(void *out, const void *z, const float *norm_w, float eps, const int32_t *lengths,

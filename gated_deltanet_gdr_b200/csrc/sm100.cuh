@@ -86,6 +86,18 @@ __device__ __forceinline__ bool mbar_test(uint64_t *bar, uint32_t parity) {
     return ok != 0;
 }
 
+// One lane of the (fully active) warp is elected, the same one on every call with the full mask: the lane that
+// issues a group of tcgen05.mma must also issue the tcgen05.commit that tracks them.
+__device__ __forceinline__ bool elect_one_sync() {
+    uint32_t pred;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "elect.sync _|p, 0xffffffff;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(pred));
+    return pred != 0;
+}
+
 // Nanoseconds from the GPU's global timer (%globaltimer).
 __device__ __forceinline__ uint64_t global_ns() {
     uint64_t t;

@@ -38,8 +38,9 @@
  *     state; other pairs: GDR_ERR_DTYPE).
  *     Index arrays are int32.  Stores to bf16 round to nearest even, once.
  *   - The caller owns every buffer.  The library allocates no device memory
- *     and keeps no pointer after a call returns; the tensor-core prefill's
- *     scratch is a caller-owned workspace sized by gdr_chunk_fwd_workspace().
+ *     and keeps no pointer after a call returns; the scratch of the
+ *     tensor-core prefill's two-kernel schedule is an optional caller-owned
+ *     workspace sized by gdr_chunk_fwd_workspace().
  *     Work is enqueued on
  *     `stream` (a cudaStream_t; NULL = the legacy default stream) and runs
  *     asynchronously: the call returns before the kernels finish.
@@ -134,16 +135,23 @@ typedef struct gdr_epilogue {
 } gdr_epilogue;
 
 /*
- * Bytes of device workspace a gdr_chunk_fwd call with these sizes needs (0 if
- * it needs none).  The tensor-core path (bf16 or fp16, Dk = Dv = 128) first
- * solves the WY transform of every 64-token chunk at once and keeps, per
- * (b, value head, chunk), the 64 x 64 matrix (I + A)^{-1} diag(beta) in the
- * input dtype and six vectors of 64 floats (the chunk's gate and norm
- * factors): B * Nv * ceil(S / 64) * (8192 + 1536) bytes.  Invalid sizes give
- * 0 (the call itself reports them).  Source: the lite_boost
- * chunk_gated_delta_rule operator (caller-owned buffers) and the order of
- * torch_chunk_gated_delta_rule, which forms every chunk's attn/T solve before
- * the inter-chunk loop.
+ * Bytes of device workspace the fastest schedule of a gdr_chunk_fwd call with
+ * these sizes wants (0 if it wants none).  The tensor-core path (bf16 or fp16,
+ * Dk = Dv = 128) has two schedules:
+ *   - one kernel, one CTA per (b, value head) chain, each chain solving its
+ *     chunks' WY systems itself; needs no workspace;
+ *   - two kernels: the WY transform of every 64-token chunk solved at once on
+ *     every SM, keeping per (b, value head, chunk) the 64 x 64 matrix
+ *     (I + A)^{-1} diag(beta) in the input dtype and six vectors of 64 floats
+ *     (the chunk's gate and norm factors), then the chains.  Workspace:
+ *     B * Nv * ceil(S / 64) * (8192 + 1536) bytes.
+ * The two-kernel schedule is asked for when the chains fill at most a third of
+ * the current device's SMs (B * Nv * 3 <= SMs; a device that cannot be asked
+ * counts as 148), where the one-kernel schedule would leave most SMs idle.
+ * Other shapes, fp32 and invalid sizes give 0 (the call itself reports the
+ * latter).  Source: the lite_boost chunk_gated_delta_rule operator
+ * (caller-owned buffers) and the order of torch_chunk_gated_delta_rule, which
+ * forms every chunk's attn/T solve before the inter-chunk loop.
  */
 size_t gdr_chunk_fwd_workspace(int B, int Nk, int Nv, int S, int Dk, int Dv, gdr_dtype dtype);
 
@@ -169,20 +177,23 @@ size_t gdr_chunk_fwd_workspace(int B, int Nk, int Nv, int S, int Dk, int Dv, gdr
  *   out                    device (B, Nv, S, Dv), written in full
  *   final_state            device (B, Nv, Dk, Dv) or NULL: not written.  It
  *                          may alias initial_state (in-place update).
- *   workspace, ws_bytes    device scratch of at least
+ *   workspace, ws_bytes    NULL and 0, or device scratch of at least
  *                          gdr_chunk_fwd_workspace(B, Nk, Nv, S, Dk, Dv, dtype)
- *                          bytes, owned by the caller, 16-byte aligned; NULL and
- *                          0 when that is 0.  Its contents on entry do not
- *                          matter and on return are unspecified; two calls in
- *                          flight at once need separate workspaces.
+ *                          bytes, owned by the caller, 16-byte aligned.  With
+ *                          it, the schedule the query sized runs; without it
+ *                          (or when the query gives 0) the one-kernel
+ *                          schedule.  Both give the same result up to rounding.
+ *                          Its contents on entry do not matter and on return
+ *                          are unspecified; two calls in flight at once need
+ *                          separate workspaces.
  * Constraints: B, S >= 0; Nk, Nv >= 1; Nv % Nk == 0; Dk, Dv in {16,32,64,128};
  * every pointer 16-byte aligned.  An epilogue with a NULL z or norm_w returns
- * GDR_ERR_NULL, one with eps < 0 (or NaN) GDR_ERR_SHAPE.  A NULL workspace
- * where one is needed returns GDR_ERR_NULL, a short one GDR_ERR_WORKSPACE.
- * bf16 or fp16 with Dk = Dv = 128 runs on the tensor-core (tcgen05) path: the
- * WY pass over all chunks, then one CTA per (b, value head) for the carry.
- * Other shapes and fp32 run the CUDA-core path.  Without g (NULL, the
- * operator's hasGamma = 0) a build without the gate arithmetic runs.
+ * GDR_ERR_NULL, one with eps < 0 (or NaN) GDR_ERR_SHAPE.  A workspace shorter
+ * than the query returns GDR_ERR_WORKSPACE.  bf16 or fp16 with
+ * Dk = Dv = 128 runs on the tensor-core (tcgen05) path in one of the two
+ * schedules above; other shapes and fp32 run the CUDA-core path.  Without g
+ * (NULL, the operator's hasGamma = 0) a build without the gate arithmetic
+ * runs.
  */
 int gdr_chunk_fwd(const void *q, const void *k, const void *v, const void *beta, const float *g,
                   const void *initial_state, const int32_t *actual_seq_lengths, float scale, int B, int Nk,
@@ -202,9 +213,10 @@ int gdr_chunk_fwd(const void *q, const void *k, const void *v, const void *beta,
  * for the memory discipline of such callers.
  *   - It allocates nothing: no cudaMalloc, cudaFree or allocating library call.
  *   - Sizes whose workspace (gdr_chunk_fwd_workspace) exceeds 16 MiB, that is
- *     B * Nv * ceil(S / 64) > 1724 on the tensor-core path, return
- *     GDR_ERR_WORKSPACE without launching anything.  The CUDA-core path needs
- *     no scratch and has no such limit.
+ *     the two-kernel schedule with B * Nv * ceil(S / 64) > 1724, return
+ *     GDR_ERR_WORKSPACE without launching anything.  Sizes whose query is 0
+ *     (the one-kernel schedule, the CUDA-core path) need no scratch and have
+ *     no such limit.
  *   - Every call shares the one array per device, so two calls that overlap on
  *     the GPU (on different streams, or from different host threads, without
  *     ordering between them) race and give wrong results.  Calls ordered on one
@@ -359,6 +371,15 @@ int gdr_debug_set_wait_limit(unsigned long long ns);
  * Returns GDR_OK, GDR_ERR_NULL, GDR_ERR_DEVICE or GDR_ERR_LAUNCH.
  */
 int gdr_debug_timeout_site(unsigned int *site);
+
+/*
+ * Diagnostic: which schedule of the tensor-core prefill gdr_chunk_fwd_workspace
+ * sizes for the calls that follow in this process: 0 by shape (the default), 1
+ * always the one-kernel schedule (the query gives 0), 2 always the two-kernel
+ * schedule.  Lets the tests compare both schedules on the same inputs.
+ * Returns GDR_OK, or GDR_ERR_SHAPE for another value.
+ */
+int gdr_debug_set_chunk_schedule(int schedule);
 
 /* Static description of a status code; never NULL. */
 const char *gdr_status_string(int status);

@@ -105,9 +105,10 @@ def test_chunk_host_validation(L):
     assert chunk(L, epi=ctypes.byref(epi)) == gdr.GDR_ERR_SHAPE
     epi = gdr.GdrEpilogueStruct(4104, 4096, 1e-6)  # misaligned z
     assert chunk(L, epi=ctypes.byref(epi)) == gdr.GDR_ERR_ALIGN
-    # the tensor-core path's workspace: required, large enough, aligned
-    assert chunk(L, ws=NUL) == gdr.GDR_ERR_NULL
+    # the two-kernel schedule's workspace, when given: large enough and aligned (a NULL workspace is valid: the
+    # one-kernel schedule runs, so it is not called here, where every call must be refused before a launch)
     need = L.gdr_chunk_fwd_workspace(1, 2, 4, 8, 128, 128, gdr.GDR_BF16)
+    assert need > 0
     assert chunk(L, ws_bytes=need - 1) == gdr.GDR_ERR_WORKSPACE
     assert chunk(L, ws=ctypes.c_void_p(4104)) == gdr.GDR_ERR_ALIGN
     # nothing to do: B == 0 returns OK without touching a device
@@ -115,15 +116,29 @@ def test_chunk_host_validation(L):
 
 
 def test_workspace_size(L):
-    """Per (b, value head, 64-token chunk): the 64 x 64 16-bit T' and six vectors of 64 floats, for the tensor-core
-    path only (bf16 or fp16, Dk = Dv = 128); zero for the CUDA-core path and for invalid sizes."""
+    """The two-kernel schedule's workspace: per (b, value head, 64-token chunk) the 64 x 64 16-bit T' and six
+    vectors of 64 floats; asked for when B * Nv * 3 <= the SM count (148 where no device answers), else 0 (the
+    one-kernel schedule needs none); zero for the CUDA-core path and for invalid sizes.  The schedule override
+    moves the answer both ways."""
     per = 64 * 64 * 2 + 6 * 64 * 4
-    assert L.gdr_chunk_fwd_workspace(4, 16, 32, 4096, 128, 128, gdr.GDR_BF16) == 4 * 32 * 64 * per
+    assert L.gdr_chunk_fwd_workspace(1, 16, 32, 4096, 128, 128, gdr.GDR_BF16) == 32 * 64 * per  # 32 chains
+    assert L.gdr_chunk_fwd_workspace(4, 16, 32, 4096, 128, 128, gdr.GDR_BF16) == 0  # 128 chains: one kernel
+    assert L.gdr_chunk_fwd_workspace(1, 7, 49, 64, 128, 128, gdr.GDR_BF16) == 49 * per  # 147 <= 148
+    assert L.gdr_chunk_fwd_workspace(2, 5, 25, 64, 128, 128, gdr.GDR_BF16) == 0  # 150 > 148
     assert L.gdr_chunk_fwd_workspace(2, 1, 3, 65, 128, 128, gdr.GDR_F16) == 2 * 3 * 2 * per
     assert L.gdr_chunk_fwd_workspace(2, 1, 3, 65, 128, 128, gdr.GDR_F32) == 0
     assert L.gdr_chunk_fwd_workspace(2, 1, 3, 65, 64, 64, gdr.GDR_BF16) == 0
     assert L.gdr_chunk_fwd_workspace(0, 1, 3, 65, 128, 128, gdr.GDR_BF16) == 0
     assert L.gdr_chunk_fwd_workspace(2, 2, 3, 65, 128, 128, gdr.GDR_BF16) == 0  # Nv % Nk != 0
+    try:
+        assert L.gdr_debug_set_chunk_schedule(2) == gdr.GDR_OK
+        assert L.gdr_chunk_fwd_workspace(4, 16, 32, 4096, 128, 128, gdr.GDR_BF16) == 4 * 32 * 64 * per
+        assert L.gdr_chunk_fwd_workspace(2, 1, 3, 65, 128, 128, gdr.GDR_F32) == 0
+        assert L.gdr_debug_set_chunk_schedule(1) == gdr.GDR_OK
+        assert L.gdr_chunk_fwd_workspace(1, 16, 32, 4096, 128, 128, gdr.GDR_BF16) == 0
+        assert L.gdr_debug_set_chunk_schedule(3) == gdr.GDR_ERR_SHAPE
+    finally:
+        L.gdr_debug_set_chunk_schedule(0)
 
 
 def test_decode_host_validation(L):

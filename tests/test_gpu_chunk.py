@@ -8,7 +8,7 @@ import oracle
 import workloads
 from tests._helpers import (assert_close, dev, dev_i32, fused_inputs, host, rnd, rnd32, unfused_inputs)
 
-pytestmark = pytest.mark.gpu
+pytestmark = [pytest.mark.gpu, pytest.mark.usefixtures("chunk_schedule")]
 
 
 def gpu_chunk(ins, w, dt, lengths=None, fused_raw=None, initial=True):

@@ -23,6 +23,7 @@ def epilogue_for(w, dt):
 
 @pytest.mark.parametrize("dt,D,S", [("bf16", 128, 200), ("bf16", 128, 64), ("bf16", 128, 1), ("f32", 128, 130),
                                     ("f32", 64, 150), ("f32", 16, 40), ("bf16", 64, 100)])
+@pytest.mark.usefixtures("chunk_schedule")
 def test_chunk_epilogue(dt, D, S):
     """bf16 with D = 128 runs the epilogue inside the tensor-core kernel; the other cases run the CUDA-core
     kernel and the row pass.  Lengths are ragged, with one empty sequence."""
@@ -45,6 +46,7 @@ def test_chunk_epilogue(dt, D, S):
         assert np.all(go[b, :, int(lengths[b]):] == 0.0)
 
 
+@pytest.mark.usefixtures("chunk_schedule")
 def test_chunk_epilogue_with_fused_prologue_strong_gate():
     """bf16, D = 128, raw q/k/b/a through the fused prologue and the epilogue in the same call."""
     from tests._helpers import fused_inputs

@@ -10,6 +10,7 @@ from tests._helpers import assert_close, dev, dev_i32, fused_inputs, host, rnd, 
 pytestmark = pytest.mark.gpu
 
 
+@pytest.mark.usefixtures("chunk_schedule")
 @pytest.mark.parametrize("D,S", [(128, 200), (64, 65), (32, 40)])
 def test_chunk_f16(D, S):
     """fp16 prefill (the tensor-core kernel at D = 128, the CUDA-core kernel otherwise) with ragged lengths, one
@@ -28,6 +29,7 @@ def test_chunk_f16(D, S):
     assert bool((out[0, :, S:] == 0).all()) and bool((out[2] == 0).all())
 
 
+@pytest.mark.usefixtures("chunk_schedule")
 def test_chunk_f16_fused_prologue_and_epilogue():
     w = workloads.random_case(B=2, Nk=2, Nv=4, S=130, Dk=128, Dv=128, seed=610, gate="strong")
     raw, ref = fused_inputs(w, "f16")
@@ -95,6 +97,7 @@ def test_conv1d_f16():
     assert_close(host(ns), rs, "f16", "state")
 
 
+@pytest.mark.usefixtures("chunk_schedule")
 @pytest.mark.parametrize("gate", ["loguniform", "none"])
 def test_chunk_f16_tensor_core_weak_gate(gate):
     """fp16 with D = 128 runs the tensor-core kernel (fp16 MMA operand copies); a weak or absent gate makes
@@ -111,6 +114,7 @@ def test_chunk_f16_tensor_core_weak_gate(gate):
     assert_close(host(fin), rf, "f16", "final_state")
 
 
+@pytest.mark.usefixtures("chunk_schedule")
 def test_prefill_workload_full_size_f16_sampled():
     """The prefill workload in fp16 with the fused prologue (the launch the benchmark's fp16 line times):
     sampled chains computed one by one by the oracle."""

@@ -27,11 +27,13 @@ def _call(w, ins):
 
 
 def test_bounded_wait_runs_out_and_the_next_call_is_clean():
-    """With the wait limit cut to 1 ns every wait that is not already satisfied runs out: the kernel drains its own
-    copies and MMAs, releases tensor memory, returns and sets GDR_DEVERR_TIMEOUT, and records which wait ran out.
-    The context stays usable: the next call with the default limit passes parity."""
+    """With the wait limit cut to 1 ns every wait of the two-kernel schedule's chain kernel that is not already
+    satisfied runs out: the kernel drains its own copies and MMAs, releases tensor memory, returns and sets
+    GDR_DEVERR_TIMEOUT, and records which wait ran out.  The context stays usable: the next call with the default
+    limit passes parity."""
     w, ins = _tiny_tc_case()
     assert gdr.get_error() == 0 and gdr.take_timeout_site() == {}
+    gdr.set_chunk_schedule(gdr.SCHEDULE_TWO_KERNELS)
     gdr.set_wait_limit_ns(1)
     try:
         _call(w, ins)
@@ -39,8 +41,9 @@ def test_bounded_wait_runs_out_and_the_next_call_is_clean():
         site = gdr.take_timeout_site()
     finally:
         gdr.set_wait_limit_ns(0)
+        gdr.set_chunk_schedule(gdr.SCHEDULE_AUTO)
     assert err & gdr.DEVERR_TIMEOUT, err
-    assert site and 0 <= site["warp"] < 18 and site["cta"] < w.B * w.Nv, site
+    assert site and 0 <= site["warp"] < 20 and site["cta"] < w.B * w.Nv, site
     out, fin = _call(w, ins)
     assert gdr.get_error() == 0 and gdr.take_timeout_site() == {}
     ro, rf = oracle.chunk_fwd(ins["q"], ins["k"], ins["v"], ins["beta"], ins["g"], ins["initial_state"], None, w.scale)

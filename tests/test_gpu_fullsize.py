@@ -16,7 +16,7 @@ import oracle
 import workloads
 from tests._helpers import BF16_REL_L2, F16_REL_L2, dev, dev_i32, host, rel_l2, rnd, rnd32
 
-pytestmark = pytest.mark.gpu
+pytestmark = [pytest.mark.gpu, pytest.mark.usefixtures("chunk_schedule")]
 
 
 def _run(w, dt, lengths=None, epilogue=None, gate=True):
