@@ -870,6 +870,9 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         auto wait_ok = [&](uint64_t *bar, uint32_t parity) {
             if (!bw(bar, parity)) to = true;
         };
+        // warp 0 issues the carry's MMAs as a whole warp, one elected lane issuing, with warp-uniform operand
+        // addresses (a lone divergent lane issues several times slower)
+        const uint32_t tmu = __shfl_sync(0xffffffffu, tmem, 0), sbu = __shfl_sync(0xffffffffu, sbase, 0);
         for (int c = 0; c < nvalid; ++c) {
             const uint32_t par = c & 1;
             const float *vec = vecs + par * NVEC * 64;
@@ -878,17 +881,20 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             if (named_sync_or(BAR_CARRY, NGRP, to)) { stop = true; break; }
             PHASE(21);
             if (tid == 0) mbar_arrive(bar_go);
-            if (tid == 0) {  // a4: W (rows 64..127 of TT K, into TMEM R) and U (rows 0..63 of TT V)
-                if (!bw(bar_ldv, par)) to = true;
+            if (warp == 0) {  // a4: W (rows 64..127 of TT K, into TMEM R) and U (rows 0..63 of TT V)
+                if (!__all_sync(0xffffffffu, bw(bar_ldv, par))) to = true;
                 tc_fence_after();
                 const uint32_t id = idesc_t<T>(128, 128, false, true);
+                if (elect_one_sync()) {
 #pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    const uint64_t ad = sdesc_sw128(sbase + OFF_TT + k * 32, 16, 1024);
-                    mma_bf16(tmem + TM_R, ad, sdesc_sw128(sbase + off_k(par, 0) + k * 2048, KQ_BLK, 1024), id, k > 0);
-                    mma_bf16(tmem + TM_U, ad, sdesc_sw128(sbase + OFF_V + k * 2048, 8192, 1024), id, k > 0);
+                    for (int k = 0; k < 4; ++k) {
+                        const uint64_t ad = sdesc_sw128(sbu + OFF_TT + k * 32, 16, 1024);
+                        mma_bf16(tmu + TM_R, ad, sdesc_sw128(sbu + off_k(par, 0) + k * 2048, KQ_BLK, 1024), id, k > 0);
+                        mma_bf16(tmu + TM_U, ad, sdesc_sw128(sbu + OFF_V + k * 2048, 8192, 1024), id, k > 0);
+                    }
+                    mma_commit(bar_wu);
                 }
-                mma_commit(bar_wu);
+                __syncwarp();
             }
             wait_ok(bar_wu, par);
             tc_fence_after();
@@ -914,17 +920,20 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             const int n = (int)vec[V_N * 64];
             const float eL = vec[V_EG * 64 + C - 1];
             // ---- R = [W; Q] S ----
-            if (tid == 0) {
+            if (warp == 0) {
                 const uint32_t id = idesc_t<T>(128, 128, false, true);
-                TIMED(23, {
-                    _Pragma("unroll")
-                    for (int k = 0; k < 8; ++k) {
-                        const uint64_t ad = sdesc_sw128(sbase + OFF_A1 + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024);
-                        const uint64_t bd = sdesc_sw128(sbase + OFF_S + k * 2048, 16384, 1024);
-                        mma_bf16(tmem + TM_R, ad, bd, id, k > 0);
-                    }
-                    mma_commit(bar_m1);
-                });
+                if (elect_one_sync()) {
+                    TIMED(23, {
+                        _Pragma("unroll")
+                        for (int k = 0; k < 8; ++k) {
+                            const uint64_t ad = sdesc_sw128(sbu + OFF_A1 + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024);
+                            const uint64_t bd = sdesc_sw128(sbu + OFF_S + k * 2048, 16384, 1024);
+                            mma_bf16(tmu + TM_R, ad, bd, id, k > 0);
+                        }
+                        mma_commit(bar_m1);
+                    });
+                }
+                __syncwarp();
             }
             // S <- e^{G_last} S in TMEM, onto which MMA2 accumulates (for c > 0 the previous chunk's
             // epilogue already wrote the scaled state back)
@@ -995,26 +1004,29 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             tc_fence_after();
             PHASE(18);
             // ---- S += K~^T v_new ;  R[64:128] += Pm v_new ----
-            if (tid == 0) {
-                if (!bw(bar_kt, par)) to = true;  // K~ of this chunk (helper warps)
+            if (warp == 0) {
+                if (!__all_sync(0xffffffffu, bw(bar_kt, par))) to = true;  // K~ of this chunk (helper warps)
                 tc_fence_after();
                 const uint32_t id_s = idesc_t<T>(128, 128, true, true);
                 const uint32_t id_o = idesc_t<T>(128, 128, false, true);
-                const uint32_t pm_rows = sbase + (par ? OFF_PM1 : OFF_PM0) - 8192;
-                TIMED(24, {
-                    _Pragma("unroll")
-                    for (int k = 0; k < 4; ++k) {
-                        const uint64_t bd = sdesc_sw128(sbase + OFF_VO + k * 2048, 8192, 1024);
-                        mma_bf16(tmem + TM_S, sdesc_sw128(sbase + OFF_KT + k * 2048, 8192, 1024), bd, id_s, 1);
-                    }
-                    _Pragma("unroll")
-                    for (int k = 0; k < 4; ++k) {
-                        const uint64_t bd = sdesc_sw128(sbase + OFF_VO + k * 2048, 8192, 1024);
-                        mma_bf16(tmem + TM_R, sdesc_sw128(pm_rows + k * 32, 16, 1024), bd, id_o, 1);
-                    }
-                    mma_commit(bar_m2);
-                    mma_commit(bar_pf + par);
-                });
+                const uint32_t pm_rows = sbu + (par ? OFF_PM1 : OFF_PM0) - 8192;
+                if (elect_one_sync()) {
+                    TIMED(24, {
+                        _Pragma("unroll")
+                        for (int k = 0; k < 4; ++k) {
+                            const uint64_t bd = sdesc_sw128(sbu + OFF_VO + k * 2048, 8192, 1024);
+                            mma_bf16(tmu + TM_S, sdesc_sw128(sbu + OFF_KT + k * 2048, 8192, 1024), bd, id_s, 1);
+                        }
+                        _Pragma("unroll")
+                        for (int k = 0; k < 4; ++k) {
+                            const uint64_t bd = sdesc_sw128(sbu + OFF_VO + k * 2048, 8192, 1024);
+                            mma_bf16(tmu + TM_R, sdesc_sw128(pm_rows + k * 32, 16, 1024), bd, id_o, 1);
+                        }
+                        mma_commit(bar_m2);
+                        mma_commit(bar_pf + par);
+                    });
+                }
+                __syncwarp();
             }
             wait_ok(bar_m2, par);
             if (tid == 0 && c + 1 < nvalid) load_carry_k(c + 1);  // the raw K tile is read
@@ -1143,8 +1155,13 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         if (n_cq) mbar_wait_ns(bar_cq, (n_cq - 1) & 1, kDrainWaitNs);
         if (n_ck) mbar_wait_ns(bar_ck, (n_ck - 1) & 1, kDrainWaitNs);
     }
-    if ((control && lane == 0) || tid == 0) {
+    if (control && lane == 0) {
         mma_commit(bar_dr);
+        mbar_wait_ns(bar_dr, 0, kDrainWaitNs);
+    }
+    if (warp == 0) {  // the carry's MMAs were issued by the lane of warp 0 that elect.sync picks
+        if (elect_one_sync()) mma_commit(bar_dr);
+        __syncwarp();
         mbar_wait_ns(bar_dr, 0, kDrainWaitNs);
     }
     tc_fence_before();
