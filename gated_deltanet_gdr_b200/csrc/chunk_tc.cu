@@ -371,7 +371,9 @@ __device__ __forceinline__ int order_chain(const TcArgs &a, int tid, uint8_t *sm
     return *s_sel;
 }
 
-template <typename T, bool kOrdered>
+// kGate = false: the build for g = NULL (no decay): no gate scan, the A and Pm entries take the column factor
+// 1/|k_s| without an exponential, and the state is never rescaled in TMEM.
+template <typename T, bool kGate, bool kOrdered>
 __global__ void __launch_bounds__(NT, 1)
 chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o, const TcArgs a) {
@@ -544,7 +546,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         // tokens per lane, the scan over the chunk by warp shuffles.
         const float gA = (a.A_log && a.g) ? a.A_log[h] : 0.f, gB = (a.A_log && a.g) ? a.dt_bias[h] : 0.f;
         const T *bg = reinterpret_cast<const T *>(a.beta) + (size_t)bh * S;
-        const float *gg = a.g ? a.g + (size_t)bh * S : nullptr;
+        const float *gg = (kGate && a.g) ? a.g + (size_t)bh * S : nullptr;
         // raw beta and gate values of a chunk's tokens (two per lane), loaded a chunk before they are used so
         // that their memory latency stays off the hand-offs
         auto load_raw = [&](int chunk, float (&rb)[2], float (&rg)[2]) {
@@ -564,7 +566,19 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             for (int i = 0; i < 2; ++i) {
                 const int tt = 2 * lane + i;
                 bv[i] = tt < n ? (a.beta_logits ? sigmoid_f32(rb[i]) : rb[i]) : 0.f;
-                gv[i] = tt < n ? (a.A_log ? gate_from_raw(rg[i], gA, gB) : rg[i]) : 0.f;
+                gv[i] = (kGate && tt < n) ? (a.A_log ? gate_from_raw(rg[i], gA, gB) : rg[i]) : 0.f;
+            }
+            if (!kGate) {
+#pragma unroll
+                for (int i = 0; i < 2; ++i) {
+                    const int tt = 2 * lane + i;
+                    vec[V_BETA * 64 + tt] = bv[i];
+                    vec[V_EG * 64 + tt] = 1.f;
+                    vec[V_G2 * 64 + tt] = 0.f;
+                    vec[V_ET * 64 + tt] = 1.f;
+                }
+                if (lane == 0) vec[V_N * 64] = (float)n;
+                return;
             }
             const float x1 = gv[0] + gv[1];
             float sc = x1;
@@ -754,13 +768,25 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     const float rf = t < n ? (krole ? vBeta[t] * vRk[t] : vRq[t]) : 0.f;
                     const float4 *lam4 = reinterpret_cast<const float4 *>(vec + V_LAM * 64 + 32 * hf);
                     tmem_ld_wait();
+                    if (kGate) {
 #pragma unroll
-                    for (int j4 = 0; j4 < 8; ++j4) {
-                        const float4 l = lam4[j4];
-                        v[4 * j4 + 0] *= rf * ex2_approx(g2t - l.x);
-                        v[4 * j4 + 1] *= rf * ex2_approx(g2t - l.y);
-                        v[4 * j4 + 2] *= rf * ex2_approx(g2t - l.z);
-                        v[4 * j4 + 3] *= rf * ex2_approx(g2t - l.w);
+                        for (int j4 = 0; j4 < 8; ++j4) {
+                            const float4 l = lam4[j4];
+                            v[4 * j4 + 0] *= rf * ex2_approx(g2t - l.x);
+                            v[4 * j4 + 1] *= rf * ex2_approx(g2t - l.y);
+                            v[4 * j4 + 2] *= rf * ex2_approx(g2t - l.z);
+                            v[4 * j4 + 3] *= rf * ex2_approx(g2t - l.w);
+                        }
+                    } else {  // no decay: the column factor 1/|k_s| alone (0 past the length)
+                        const float4 *rk4 = reinterpret_cast<const float4 *>(vRk + 32 * hf);
+#pragma unroll
+                        for (int j4 = 0; j4 < 8; ++j4) {
+                            const float4 l = rk4[j4];
+                            v[4 * j4 + 0] *= rf * l.x;
+                            v[4 * j4 + 1] *= rf * l.y;
+                            v[4 * j4 + 2] *= rf * l.z;
+                            v[4 * j4 + 3] *= rf * l.w;
+                        }
                     }
                     if (krole && hf == qa) {
                         // a diagonal 32 x 32 block, plain (entries on or above the diagonal are never read)
@@ -937,7 +963,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             }
             // S <- e^{G_last} S in TMEM, onto which MMA2 accumulates (for c > 0 the previous chunk's
             // epilogue already wrote the scaled state back)
-            if (c == 0) {
+            if (kGate && c == 0) {
 #pragma unroll
                 for (int half = 0; half < 2; ++half) {
                     float v[32];
@@ -1045,13 +1071,13 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 for (int c8 = 0; c8 < 4; ++c8)
                     *reinterpret_cast<uint4 *>(sm + OFF_S + hf * 16384 + blk_off(row, 32 * half + 8 * c8)) =
                         pack8<T>(&v[8 * c8]);
-                if (more) {
+                if (kGate && more) {
 #pragma unroll
                     for (int j = 0; j < 32; ++j) v[j] *= eLn;
                     tmem_st32(ta, v);
                 }
             }
-            if (more) tmem_st_wait();
+            if (kGate && more) tmem_st_wait();
             if (q4 >= 2) {
                 const int t = row - 64;
                 // epilogue: the row's squared norm from its two halves (this thread and the one of the other hf
@@ -1202,7 +1228,7 @@ bool chunk_tc_supported(int Dk, int Dv, gdr_dtype dt, int S) {
 }
 
 namespace {
-template <typename T>
+template <typename T, bool kGate>
 cudaError_t launch_tc_t(const ChunkArgs &ca, cudaStream_t stream) {
     constexpr CUtensorMapDataType ty = TcT<T>::kMap;
     CUtensorMap mq, mk, mv, mo;
@@ -1218,8 +1244,8 @@ cudaError_t launch_tc_t(const ChunkArgs &ca, cudaStream_t stream) {
     a.dt_bias = ca.dt_bias; a.err = ca.err;
     a.epi_z = ca.epi_z; a.epi_w = ca.epi_w; a.epi_eps = ca.epi_eps;
     a.wait_ns = chunk_wait_ns();
-    static LaunchCache plain(reinterpret_cast<const void *>(chunk_tc_kernel<T, false>));
-    static LaunchCache ordered(reinterpret_cast<const void *>(chunk_tc_kernel<T, true>));
+    static LaunchCache plain(reinterpret_cast<const void *>(chunk_tc_kernel<T, kGate, false>));
+    static LaunchCache ordered(reinterpret_cast<const void *>(chunk_tc_kernel<T, kGate, true>));
     const long long blocks = (long long)ca.B * ca.Nv;
     if (blocks == 0) return cudaSuccess;
     // longest sequences first only when the chains do not all start at once
@@ -1233,15 +1259,17 @@ cudaError_t launch_tc_t(const ChunkArgs &ca, cudaStream_t stream) {
     cudaError_t e = (order ? ordered : plain).allow_smem((int)SMEM_BYTES);
     if (e != cudaSuccess) return e;
     if (order)
-        chunk_tc_kernel<T, true><<<(unsigned)blocks, NT, SMEM_BYTES, stream>>>(mq, mk, mv, mo, a);
+        chunk_tc_kernel<T, kGate, true><<<(unsigned)blocks, NT, SMEM_BYTES, stream>>>(mq, mk, mv, mo, a);
     else
-        chunk_tc_kernel<T, false><<<(unsigned)blocks, NT, SMEM_BYTES, stream>>>(mq, mk, mv, mo, a);
+        chunk_tc_kernel<T, kGate, false><<<(unsigned)blocks, NT, SMEM_BYTES, stream>>>(mq, mk, mv, mo, a);
     return cudaGetLastError();
 }
 }  // namespace
 
 cudaError_t launch_chunk_tc(const ChunkArgs &ca, gdr_dtype dt, cudaStream_t stream) {
-    return dt == GDR_F16 ? launch_tc_t<__half>(ca, stream) : launch_tc_t<__nv_bfloat16>(ca, stream);
+    const bool gate = ca.g != nullptr;
+    if (dt == GDR_F16) return gate ? launch_tc_t<__half, true>(ca, stream) : launch_tc_t<__half, false>(ca, stream);
+    return gate ? launch_tc_t<__nv_bfloat16, true>(ca, stream) : launch_tc_t<__nv_bfloat16, false>(ca, stream);
 }
 
 }  // namespace gdr
