@@ -63,7 +63,7 @@ def algorithmic_decode_bytes(w) -> dict:
     seqs = int((w.lengths > 0).sum())
     state = 2 * seqs * w.Nv * w.Dk * w.Dv * e
     tok = int(w.lengths.sum())
-    io = tok * (2 * w.Nk * w.Dk * e + w.Nv * w.Dv * e + w.Nv * e + w.Nv * 4)
+    io = tok * (2 * w.Nk * w.Dk * e + w.Nv * w.Dv * e + w.Nv * e + (w.Nv * 4 if w.g is not None else 0))
     if w.gk is not None:
         io += tok * w.Nv * w.Dk * 4
     io += w.B * w.S * w.Nv * w.Dv * e  # out, all positions
@@ -614,7 +614,11 @@ def bench_decode(gdr, name, args, world, rank, clk, flush, stream, peaks, rotate
     pool: each call reads fresh state and pays the write-back of the previous call's state,
     as a serving loop does."""
     spec = name == "decode_spec"
-    if spec:
+    if name == "decode_no_gate":
+        # the decode workload with g = NULL (hasGamma = 0): the D = 128 kernel's build without the decay
+        wd = workloads.generate("decode", seed=1 + 1000 * rank)
+        wd.g = None
+    elif spec:
         # speculative decoding: 64 sequences verify 4 draft tokens each, every token with its own slot (the
         # previous step's A of them accepted); gdr_recurrent_step_spec
         wd = workloads.random_case(B=64, Nk=16, Nv=32, S=4, Dk=128, Dv=128, seed=6 + 1000 * rank, slots=64 * 4 + 64,
@@ -623,7 +627,7 @@ def bench_decode(gdr, name, args, world, rank, clk, flush, stream, peaks, rotate
     else:
         wd = workloads.generate(name, seed=(1 if name == "decode" else 4) + 1000 * rank)
     dq, dk, dv, db = bf16_dev(wd.q), bf16_dev(wd.k), bf16_dev(wd.v), bf16_dev(wd.b)
-    dg = f32_dev(wd.g)
+    dg = f32_dev(wd.g) if wd.g is not None else None
     dgk = f32_dev(wd.gk) if wd.gk is not None else None
     pools = [bf16_dev(wd.pool) for _ in range(rotate)]
     idx = torch.from_numpy(wd.indices).cuda()
@@ -668,7 +672,8 @@ def bench_decode(gdr, name, args, world, rank, clk, flush, stream, peaks, rotate
     gbs = nb["state"] / (d_ms / 1e3) / 1e9
     tot = (nb["state"] + nb["io"]) / (d_ms / 1e3) / 1e9
     return {"workload": f"B={wd.B} S={wd.S} Nk={wd.Nk} Nv={wd.Nv} D={wd.Dk} bf16, pool of {wd.pool.shape[0]} slots"
-                        + (", per-key gate" if wd.gk is not None else "") + ", fused prologue"
+                        + (", per-key gate" if wd.gk is not None else "")
+                        + (", no gate (g = NULL)" if wd.g is None else "") + ", fused prologue"
                         + (", per-token slots, accepted ~ U[1, 4] (speculative decoding)" if spec else ""),
             "l2": f"{rotate} rotating pool copies (fresh state every call), no flush",
             "timing": f"{args.steps} calls back to back inside one event pair; us_per_call_single: each call inside "
@@ -714,8 +719,8 @@ def run_ours(args, world, rank, local):
         line["f16"], n = bench_f16(gdr, args, world, rank, flush, stream, peaks)
         launches += n
     decode = {}
-    for name in ("decode", "decode_gk", "decode_spec"):
-        if args.only in ("all", name):
+    for name in ("decode", "decode_gk", "decode_spec", "decode_no_gate"):
+        if args.only in ("all", name) or (name == "decode_no_gate" and args.only == "decode"):
             decode[name], n = bench_decode(gdr, name, args, world, rank, clk, flush, stream, peaks)
             launches += n
     if decode:

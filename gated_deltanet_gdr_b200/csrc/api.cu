@@ -302,6 +302,7 @@ int recurrent_step(const void *q, const void *k, const void *v, const void *beta
     a.dt_bias = prologue ? prologue->dt_bias : nullptr;
     a.err = err;
     a.per_token = per_token;
+    a.wait_ns = chunk_wait_ns();
     cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
     if (checks_enabled() &&
         (st = check_decode_host(ssm_state_indices, actual_seq_lengths, num_accepted_tokens, B, S, slots, per_token,

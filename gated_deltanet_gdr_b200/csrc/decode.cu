@@ -34,6 +34,7 @@ namespace gdr {
 namespace {
 
 constexpr int T = kDecodeMaxTokens;
+constexpr uint64_t kDecodeDrainNs = 1000000000ull;  // bound of the drain after a timed-out wait
 
 // explicit shared-memory loads (32-bit shared addresses), so that every operand read of the decode loop
 // is a shared-memory access
@@ -463,7 +464,8 @@ __device__ __forceinline__ void put_meta128(const DecodeArgs &a, int *mm, int ti
     }
 }
 
-template <typename TI, typename TS, int NW, int NSTG, int MINB>
+// kDecay = false: the build for g = NULL and gk = NULL (no decay), which never rescales the state.
+template <typename TI, typename TS, int NW, int NSTG, int MINB, bool kDecay>
 __global__ void __launch_bounds__(32 * NW, MINB)
 decode128_kernel(const __grid_constant__ CUtensorMap tm_pool, const DecodeArgs a, const int ntiles) {
     using Cf = D128<TI, TS, NW, NSTG>;
@@ -486,9 +488,12 @@ decode128_kernel(const __grid_constant__ CUtensorMap tm_pool, const DecodeArgs a
     const int soff = box * (D * 128) + rg * 128 + ((ch0 ^ sw) << 4);
     const int soff2 = box * (D * 128) + rg * 128 + (((ch0 + 1) ^ sw) << 4);  // second chunk (fp32 state)
 
+    // tiles thread 0 has issued; the i-th went to stage i % NS (for the drain after a timeout)
+    int n_issued = 0;
     // checked copies of a tile into stage `st` (thread 0): the state slab by TMA, the token rows by bulk copies
     auto issue = [&](int tile, const int *mm, int st) {
         uint64_t *bar = full + st;
+        ++n_issued;
         uint8_t *base = smem + st * ly.stage;
         const int status = tile_status(mm, S, a.slots, a.per_token);
         const int Lc = status ? 0 : mm[0];
@@ -558,7 +563,7 @@ decode128_kernel(const __grid_constant__ CUtensorMap tm_pool, const DecodeArgs a
             float zz[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
             Vec8<TI>::store(out + (size_t)t * D + c, zz);
         }
-        if (!sm100::mbar_wait(full + st, (uint32_t)(j / NS) & 1u)) timed_out = true;
+        if (!sm100::mbar_wait_ns(full + st, (uint32_t)(j / NS) & 1u, a.wait_ns)) timed_out = true;
         if (Lv > 0 && !timed_out) {
             const uint8_t *base = smem + st * ly.stage;
             const uint32_t sb = sm100::smem_u32(base);
@@ -627,14 +632,18 @@ decode128_kernel(const __grid_constant__ CUtensorMap tm_pool, const DecodeArgs a
                 const uint32_t gkrow = sgk + t * D * 4;
 #pragma unroll
                 for (int r = 0; r < RPT; ++r) {
-                    const float dr = a.gk ? ag * exp2f_approx(lds_f32(gkrow + NRG * r * 4) * 1.4426950408889634f) : ag;
-                    const f2_t d2 = pk2(dr, dr), k2 = pk2(xk[r], xk[r]), q2 = pk2(xq[r], xq[r]);
+                    const f2_t k2 = pk2(xk[r], xk[r]), q2 = pk2(xq[r], xq[r]);
+                    if (kDecay) {
+                        const float dr =
+                            a.gk ? ag * exp2f_approx(lds_f32(gkrow + NRG * r * 4) * 1.4426950408889634f) : ag;
+                        const f2_t d2 = pk2(dr, dr);
+#pragma unroll
+                        for (int p = 0; p < 4; ++p) sv[r][p] = mul2(sv[r][p], d2);
+                    }
 #pragma unroll
                     for (int p = 0; p < 4; ++p) {
-                        const f2_t sd = mul2(sv[r][p], d2);
-                        sv[r][p] = sd;
-                        mk[p] = fma2(k2, sd, mk[p]);
-                        mq[p] = fma2(q2, sd, mq[p]);
+                        mk[p] = fma2(k2, sv[r][p], mk[p]);
+                        mq[p] = fma2(q2, sv[r][p], mq[p]);
                     }
                 }
                 // reduce-scatter over the row groups (lane bits 2..4): value i = 2c + w (column c of the 8,
@@ -709,7 +718,7 @@ decode128_kernel(const __grid_constant__ CUtensorMap tm_pool, const DecodeArgs a
         if (timed_out) break;
         if (warp == 0) {
             const int nxt = tile + NS * (int)gridDim.x;
-            if (!sm100::mbar_wait(empty + st, (uint32_t)(j / NS) & 1u)) {
+            if (!sm100::mbar_wait_ns(empty + st, (uint32_t)(j / NS) & 1u, a.wait_ns)) {
                 timed_out = true;
                 break;
             }
@@ -721,7 +730,16 @@ decode128_kernel(const __grid_constant__ CUtensorMap tm_pool, const DecodeArgs a
             if (nxt + 3 * (int)gridDim.x < ntiles) prefetch_meta128<TI>(a, nxt + 3 * gridDim.x, tid, pre2);
         }
     }
-    if (timed_out && tid == 0) raise_device_error(a.err, GDR_DEVERR_TIMEOUT);
+    if (timed_out && tid == 0) {
+        // drain: each stage's last armed phase (the only one that can still be in flight) has landed before the
+        // CTA leaves, so no copy writes into the shared memory of a later CTA
+#pragma unroll
+        for (int i = 0; i < NS; ++i) {
+            const int phases = n_issued > i ? (n_issued - 1 - i) / NS + 1 : 0;  // issues that went to stage i
+            if (phases) sm100::mbar_wait_ns(full + i, (uint32_t)(phases - 1) & 1u, kDecodeDrainNs);
+        }
+        raise_device_error(a.err, GDR_DEVERR_TIMEOUT);
+    }
 }
 
 template <typename TI, typename TS>
@@ -744,9 +762,12 @@ cudaError_t launch_decode128(const DecodeArgs &a, cudaStream_t stream) {
             strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
         return cudaErrorInvalidValue;
-    auto kern = decode128_kernel<TI, TS, NW, NSTG, MINB>;
+    auto kern = (a.g || a.gk) ? decode128_kernel<TI, TS, NW, NSTG, MINB, true>
+                              : decode128_kernel<TI, TS, NW, NSTG, MINB, false>;
     const int smem = Cf::layout(a.S, a.gk != nullptr).smem;
-    static LaunchCache cache(reinterpret_cast<const void *>(kern));
+    static LaunchCache cache_decay(reinterpret_cast<const void *>(decode128_kernel<TI, TS, NW, NSTG, MINB, true>));
+    static LaunchCache cache_plain(reinterpret_cast<const void *>(decode128_kernel<TI, TS, NW, NSTG, MINB, false>));
+    LaunchCache &cache = (a.g || a.gk) ? cache_decay : cache_plain;
     cudaError_t e = cache.allow_smem(smem);
     if (e != cudaSuccess) return e;
     int grid_cap = 1;

@@ -29,6 +29,7 @@ struct DecodeArgs {
     const float *A_log, *dt_bias;
     unsigned int *err;
     int per_token;  // num_accepted_tokens read per token (speculative decoding): see gdr_recurrent_step_spec
+    uint64_t wait_ns;  // limit of each bounded wait of the D = 128 kernel (its stage pipeline)
 };
 
 struct ChunkArgs {

@@ -105,15 +105,30 @@ __device__ __forceinline__ uint64_t global_ns() {
     return t;
 }
 
+// try_wait with an explicit suspend-time hint in nanoseconds (an upper bound on one suspension)
+__device__ __forceinline__ bool mbar_try_wait_hint(uint64_t *bar, uint32_t parity, uint32_t hint_ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.b32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return ok != 0;
+}
+
 // Wait for the phase with the given parity for at most `limit_ns` of elapsed time (global timer),
 // giving up early when *abort (a flag in shared memory that another warp group raises when it
-// stops) is set.  Returns false on timeout or abort.
+// stops) is set.  Returns false on timeout or abort.  One suspension lasts at most the smaller of
+// the limit and 65.5 us, so a short limit is honoured.
 __device__ __forceinline__ bool mbar_wait_ns(uint64_t *bar, uint32_t parity, uint64_t limit_ns,
                                              const volatile int *abort = nullptr) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_test(bar, parity)) return true;
+    const uint32_t hint = limit_ns < 0x10000ull ? (uint32_t)limit_ns : 0x10000u;
     const uint64_t t0 = global_ns();
     for (;;) {
-        if (mbar_try_wait(bar, parity)) return true;
+        if (mbar_try_wait_hint(bar, parity, hint)) return true;
         if (abort && *abort) return false;
         if (global_ns() - t0 >= limit_ns) return false;
     }

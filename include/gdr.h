@@ -353,12 +353,13 @@ int gdr_prologue_apply(const void *q, const void *k, const void *b, const float 
 int gdr_get_error(gdr_stream_t stream, int *device_error);
 
 /*
- * Diagnostic hook for the bounded waits of the tensor-core prefill: their limit
- * in nanoseconds for the calls that follow in this process (0 restores the
- * default of one second).  A limit shorter than the kernel needs makes its
- * waits run out: the kernel then drains its own copies and MMAs, returns early
- * and sets GDR_DEVERR_TIMEOUT (outputs incomplete).  Used by the tests of that
- * path; not for production use.  Always returns GDR_OK.
+ * Diagnostic hook for the bounded waits of the tensor-core prefill and of the
+ * D = 128 decode kernel: their limit in nanoseconds for the calls that follow in
+ * this process (0 restores the default of one second).  A limit shorter than a
+ * kernel needs makes its waits run out: the kernel then drains its own copies
+ * (and MMAs), returns early and sets GDR_DEVERR_TIMEOUT (outputs and, for
+ * decode, the state pool incomplete).  Used by the tests of those paths; not
+ * for production use.  Always returns GDR_OK.
  */
 int gdr_debug_set_wait_limit(unsigned long long ns);
 

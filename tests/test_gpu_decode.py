@@ -64,6 +64,15 @@ def test_decode_gk_workload_bf16():
     check_decode(w, *run_decode(w, "bf16"), "bf16")
 
 
+@pytest.mark.parametrize("S,share", [(1, True), (4, False)])
+def test_decode_no_gate_d128(S, share):
+    """g = NULL and gk = NULL (the operator's hasGamma = 0): the D = 128 kernel's build without the decay."""
+    w = workloads.random_case(B=12, Nk=2, Nv=4, S=S, Dk=128, Dv=128, seed=120 + S, gate="none", slots=64,
+                              share_slot=share)
+    assert w.g is None and w.gk is None
+    check_decode(w, *run_decode(w, "bf16"), "bf16")
+
+
 def test_decode_gk_workload_fused_prologue():
     w = workloads.generate("decode_gk", B=32)
     check_decode(w, *run_decode(w, "bf16", fused=True), "bf16")
