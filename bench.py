@@ -367,7 +367,7 @@ def bench_prefill(gdr, args, world, rank, clk, flush, stream, peaks):
                      "frac": achieved / peaks["hbm_gbs"], "traffic": profiled_traffic("chunk"),
                      "peak_source": peaks["source"], "algorithmic_bytes_per_launch": alg_bytes,
                      "kernel": "gdr_chunk_fwd (fused prologue)"},
-        "gpu_launches": 2 * args.steps,  # the WY pass and the chain kernel per call
+        "gpu_launches": prefill_kernels(gdr, w) * args.steps,
     }
     return fields, w, t, pro, step
 
@@ -401,12 +401,51 @@ def bench_varlen(gdr, args, world, rank, flush, stream, peaks):
             "l2": "inputs larger than L2, plus a 256 MiB flush before every timed step",
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                          "frac": achieved / peaks["hbm_gbs"], "traffic": None, "algorithmic_bytes_per_launch": nb}}, \
-        2 * args.steps
+        prefill_kernels(gdr, w) * args.steps
+
+
+def prefill_kernels(gdr, w) -> int:
+    """Kernels one prefill call launches: 2 when the sizes ask for the two-kernel schedule's workspace (the WY
+    pass, then the chains), else 1 (the one-kernel schedule)."""
+    return 2 if gdr.chunk_fwd_workspace_bytes(w.B, w.Nk, w.Nv, w.S, w.Dk, w.Dv, torch.bfloat16) > 0 else 1
+
+
+def bench_prefill_b1(gdr, args, world, rank, flush, stream, peaks):
+    """One sequence of the prefill workload (B=1, S=4096, fused prologue): 32 chains on 148 SMs, where the
+    workspace query asks for the two-kernel schedule (the WY pass over every chunk on every SM, then the
+    chains)."""
+    w = workloads.generate("prefill", B=1, seed=12 + 1000 * rank)
+    t = dict(q=bf16_dev(w.q), k=bf16_dev(w.k), v=bf16_dev(w.v), b=bf16_dev(w.b), a=f32_dev(w.a),
+             s0=bf16_dev(w.initial_state))
+    pro = gdr.Prologue(l2norm_qk=True, eps=1e-6, beta_logits=True, A_log=f32_dev(w.A_log),
+                       dt_bias=f32_dev(w.dt_bias))
+    step = gdr.prepare_chunk_fwd(t["q"], t["k"], t["v"], t["b"], t["a"], t["s0"], None, w.scale, prologue=pro)
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if gdr.get_error() != 0:
+        raise RuntimeError("device error word set during warm-up")
+    barrier(world)
+    torch.cuda.synchronize()
+    times = timed_steps(step, args.steps, flush, stream)
+    barrier(world)
+    total_ms = all_max(sum(times), world)
+    ms = total_ms / args.steps
+    tokens = int(w.lengths.sum())
+    alg = algorithmic_prefill_bytes(w)
+    achieved = alg / (ms / 1e3) / 1e9
+    nk = prefill_kernels(gdr, w)
+    return {"workload": f"prefill B={w.B} S={w.S} Nk={w.Nk} Nv={w.Nv} Dk=Dv={w.Dk} bf16, fused prologue",
+            "schedule": "two kernels (WY pass, then the chains)" if nk == 2 else "one kernel",
+            "ms_per_step": ms, "tokens_per_s": weak_scaling_rate(tokens, args.steps, total_ms, world),
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": achieved / peaks["hbm_gbs"], "traffic": None, "algorithmic_bytes_per_launch": alg,
+                         "kernel": "gdr_chunk_fwd (fused prologue)"}}, nk * args.steps
 
 
 def bench_prefill_no_gate(gdr, args, world, w, t, flush, stream, peaks):
-    """The prefill workload without a gate (g = NULL, hasGamma = 0 of the chunk operator): the build of the WY pass
-    and the chain kernel without the gate arithmetic; l2norm and beta logits fused."""
+    """The prefill workload without a gate (g = NULL, hasGamma = 0 of the chunk operator): the tensor-core
+    prefill's build without the gate arithmetic; l2norm and beta logits fused."""
     pro = gdr.Prologue(l2norm_qk=True, eps=1e-6, beta_logits=True)
     step = gdr.prepare_chunk_fwd(t["q"], t["k"], t["v"], t["b"], None, t["s0"], None, w.scale, prologue=pro,
                                  out=t["out"], final_state=t["fin"])
@@ -429,7 +468,7 @@ def bench_prefill_no_gate(gdr, args, world, w, t, flush, stream, peaks):
             "tokens_per_s": weak_scaling_rate(tokens, args.steps, total_ms, world),
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                          "frac": achieved / peaks["hbm_gbs"], "traffic": None, "algorithmic_bytes_per_launch": alg,
-                         "kernel": "gdr_chunk_fwd without gate"}}, 2 * args.steps
+                         "kernel": "gdr_chunk_fwd without gate"}}, prefill_kernels(gdr, w) * args.steps
 
 
 def bench_prefill_epilogue(gdr, args, world, w, t, pro, flush, stream, peaks):
@@ -460,7 +499,8 @@ def bench_prefill_epilogue(gdr, args, world, w, t, pro, flush, stream, peaks):
             "ms_per_step": ms_per_step, "tokens_per_s": weak_scaling_rate(tokens, args.steps, total_ms, world),
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                          "frac": achieved / peaks["hbm_gbs"], "traffic": None, "algorithmic_bytes_per_launch":
-                         alg_bytes, "kernel": "gdr_chunk_fwd (fused prologue and epilogue)"}}, 2 * args.steps
+                         alg_bytes, "kernel": "gdr_chunk_fwd (fused prologue and epilogue)"}}, \
+        prefill_kernels(gdr, w) * args.steps
 
 
 def bench_conv1d(gdr, args, world, rank, flush, stream, peaks):
@@ -541,7 +581,7 @@ def bench_f16(gdr, args, world, rank, flush, stream, peaks):
             "decode": {"workload": "decode B=64 S=1 fp16 inputs, fp32 state (general decode kernel), L2 flush",
                        "us_per_call": d_ms * 1e3,
                        "roofline": {"bound": "hbm", "achieved": d_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                                    "frac": d_gbs / peaks["hbm_gbs"]}}}, 3 * args.steps
+                                    "frac": d_gbs / peaks["hbm_gbs"]}}}, (prefill_kernels(gdr, w) + 1) * args.steps
 
 
 def bench_e2e(gdr, args, world, w, t, pro, flush, stream):
@@ -702,13 +742,16 @@ def run_ours(args, world, rank, local):
         launches += fields.pop("gpu_launches")
         if not args.no_e2e:
             line["e2e"], n = bench_e2e(gdr, args, world, w, t, pro, flush, stream)
-            launches += 2 * n  # two prefill kernels per step
+            launches += prefill_kernels(gdr, w) * n
         if not args.no_epilogue:
             line["prefill_epilogue"], n = bench_prefill_epilogue(gdr, args, world, w, t, pro, flush, stream, peaks)
             launches += n
         line["prefill_no_gate"], n = bench_prefill_no_gate(gdr, args, world, w, t, flush, stream, peaks)
         launches += n
         del t
+    if args.only in ("all", "prefill_b1"):
+        line["prefill_b1"], n = bench_prefill_b1(gdr, args, world, rank, flush, stream, peaks)
+        launches += n
     if args.only in ("all", "varlen"):
         line["varlen"], n = bench_varlen(gdr, args, world, rank, flush, stream, peaks)
         launches += n
@@ -746,8 +789,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg (profiling runs)")
     ap.add_argument("--no-epilogue", action="store_true",
                     help="skip the prefill line with the fused gated RMSNorm epilogue (profiling runs)")
-    ap.add_argument("--only", choices=["all", "prefill", "decode", "decode_gk", "decode_spec", "conv1d", "f16",
-                                       "varlen"], default="all",
+    ap.add_argument("--only", choices=["all", "prefill", "prefill_b1", "decode", "decode_gk", "decode_spec",
+                                       "conv1d", "f16", "varlen"], default="all",
                     help="run one workload only (profiling runs); the default runs all")
     args = ap.parse_args()
     if args.warmup < 3:
