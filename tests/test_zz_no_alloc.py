@@ -53,6 +53,32 @@ def test_noalloc_matches_the_workspace_entry_point_on_two_calls():
             assert np.all(go[b, :, int(w.lengths[b]):] == 0.0)
 
 
+def test_noalloc_with_the_one_kernel_schedule():
+    """Sizes whose workspace query is 0 (here forced to the one-kernel schedule) run without touching the array;
+    the result is the same call's through gdr_chunk_fwd."""
+    L = gdr.lib()
+    w = workloads.random_case(B=2, Nk=2, Nv=4, S=130, Dk=128, Dv=128, seed=501, lengths=[130, 64])
+    ins = unfused_inputs(w, "bf16")
+    t = dict(q=dev(ins["q"], "bf16"), k=dev(ins["k"], "bf16"), v=dev(ins["v"], "bf16"),
+             beta=dev(ins["beta"], "bf16"), g=dev(ins["g"], "f32"), s0=dev(ins["initial_state"], "bf16"))
+    lens = dev_i32(w.lengths)
+    gdr.set_chunk_schedule(gdr.SCHEDULE_ONE_KERNEL)
+    try:
+        assert gdr.chunk_fwd_workspace_bytes(w.B, w.Nk, w.Nv, w.S, w.Dk, w.Dv, torch.bfloat16) == 0
+        ref_out, ref_fin = gdr.chunk_fwd(t["q"], t["k"], t["v"], t["beta"], t["g"], t["s0"], lens, w.scale)
+        out = torch.full_like(ref_out, float("nan"))
+        fin = torch.full_like(ref_fin, float("nan"))
+        assert _noalloc(L, t, lens, w, out, fin) == gdr.GDR_OK
+        torch.cuda.synchronize()
+    finally:
+        gdr.set_chunk_schedule(gdr.SCHEDULE_AUTO)
+    assert gdr.get_error() == 0
+    go, gf = host(out), host(fin)
+    assert rel_l2(go, host(ref_out)) <= BF16_REL_L2 and rel_l2(gf, host(ref_fin)) <= BF16_REL_L2
+    for b in range(w.B):
+        assert np.all(go[b, :, int(w.lengths[b]):] == 0.0)
+
+
 def test_noalloc_refuses_a_size_beyond_its_array():
     """B * Nv * ceil(S / 64) > 1724 needs more than the 16 MiB array: GDR_ERR_WORKSPACE, nothing launched."""
     L = gdr.lib()
