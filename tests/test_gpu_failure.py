@@ -51,6 +51,34 @@ def test_bounded_wait_runs_out_and_the_next_call_is_clean():
     assert_close(host(fin), rf, "bf16", "final_state")
 
 
+@pytest.mark.timeout(300)
+def test_bounded_wait_runs_out_one_kernel_schedule():
+    """The same with the one-kernel schedule (the prefill workload's): with the limit at 1 ns its waits run out,
+    each warp group stops at its next collective hand-off (bar.red.or, so no group splits at a named barrier),
+    the issuers wait for their copies and MMAs in flight, and the call returns with GDR_DEVERR_TIMEOUT and the
+    first site that ran out.  The next call with the default limit passes parity."""
+    w, ins = _tiny_tc_case()
+    assert gdr.get_error() == 0 and gdr.take_timeout_site() == {}
+    gdr.set_chunk_schedule(gdr.SCHEDULE_ONE_KERNEL)
+    try:
+        gdr.set_wait_limit_ns(1)
+        try:
+            _call(w, ins)
+            err = gdr.get_error()
+            site = gdr.take_timeout_site()
+        finally:
+            gdr.set_wait_limit_ns(0)
+        assert err & gdr.DEVERR_TIMEOUT, err
+        assert site and 0 <= site["warp"] < 20 and site["cta"] < w.B * w.Nv, site
+        out, fin = _call(w, ins)
+        assert gdr.get_error() == 0 and gdr.take_timeout_site() == {}
+    finally:
+        gdr.set_chunk_schedule(gdr.SCHEDULE_AUTO)
+    ro, rf = oracle.chunk_fwd(ins["q"], ins["k"], ins["v"], ins["beta"], ins["g"], ins["initial_state"], None, w.scale)
+    assert_close(host(out), ro, "bf16", "out")
+    assert_close(host(fin), rf, "bf16", "final_state")
+
+
 def _decode_case(B=4, S=2, slots=12):
     w = workloads.random_case(B=B, Nk=1, Nv=2, S=S, Dk=128, Dv=128, seed=92, slots=slots, share_slot=True)
     ins = unfused_inputs(w, "bf16")
