@@ -539,7 +539,7 @@ def bench_conv1d(gdr, args, world, rank, flush, stream, peaks):
 
 def bench_f16(gdr, args, world, rank, flush, stream, peaks):
     """fp16 inputs: the prefill workload (fused prologue; the tensor-core kernel with fp16 operands) and the decode
-    workload with an fp32 state (the general decode kernel).  Returns (fields, launches)."""
+    workload with an fp32 state (the D = 128 decode kernel).  Returns (fields, launches)."""
     h = lambda x: torch.from_numpy(np.ascontiguousarray(x)).to(torch.float16).cuda()
     w = workloads.generate("prefill", seed=2 + 1000 * rank)
     pro = gdr.Prologue(l2norm_qk=True, eps=1e-6, beta_logits=True, A_log=f32_dev(w.A_log), dt_bias=f32_dev(w.dt_bias))
@@ -578,7 +578,7 @@ def bench_f16(gdr, args, world, rank, flush, stream, peaks):
                                                                               p_ms * args.steps, world),
                         "roofline": {"bound": "hbm", "achieved": alg / (p_ms / 1e3) / 1e9, "peak": peaks["hbm_gbs"],
                                      "unit": "GB/s", "frac": alg / (p_ms / 1e3) / 1e9 / peaks["hbm_gbs"]}},
-            "decode": {"workload": "decode B=64 S=1 fp16 inputs, fp32 state (general decode kernel), L2 flush",
+            "decode": {"workload": "decode B=64 S=1 fp16 inputs, fp32 state, L2 flush",
                        "us_per_call": d_ms * 1e3,
                        "roofline": {"bound": "hbm", "achieved": d_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                                     "frac": d_gbs / peaks["hbm_gbs"]}}}, (prefill_kernels(gdr, w) + 1) * args.steps

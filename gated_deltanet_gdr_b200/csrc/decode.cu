@@ -25,6 +25,8 @@
 //   - the column reductions k^T S' and q^T S' of the decayed state are taken in one pass
 //     and finished by a 4-step xor butterfly inside the warp, and the output uses
 //     o = q^T S' + (q . k) d, so no second pass over S is needed.
+#include <type_traits>
+
 #include "common.cuh"
 #include "kernels.h"
 #include "sm100.cuh"
@@ -53,9 +55,27 @@ __device__ __forceinline__ float lds_bf16(uint32_t a) {
     asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(a));
     return __uint_as_float((uint32_t)v << 16);
 }
+__device__ __forceinline__ float lds_f16(uint32_t a) {
+    unsigned short v;
+    asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(a));
+    return __half2float(__ushort_as_half(v));
+}
 template <typename T> __device__ __forceinline__ float lds_elem(uint32_t a);
 template <> __device__ __forceinline__ float lds_elem<float>(uint32_t a) { return lds_f32(a); }
 template <> __device__ __forceinline__ float lds_elem<__nv_bfloat16>(uint32_t a) { return lds_bf16(a); }
+template <> __device__ __forceinline__ float lds_elem<__half>(uint32_t a) { return lds_f16(a); }
+// the two 16-bit values packed in w (low half first) as floats
+template <typename T> __device__ __forceinline__ void unpack2(uint32_t w, float &lo, float &hi);
+template <> __device__ __forceinline__ void unpack2<__nv_bfloat16>(uint32_t w, float &lo, float &hi) {
+    lo = __uint_as_float(w << 16);
+    hi = __uint_as_float(w & 0xffff0000u);
+}
+template <> __device__ __forceinline__ void unpack2<__half>(uint32_t w, float &lo, float &hi) {
+    const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&w));
+    lo = f.x;
+    hi = f.y;
+}
+template <> __device__ __forceinline__ void unpack2<float>(uint32_t, float &, float &) {}
 
 // 2^x on the special-function unit (PTX ex2.approx.ftz.f32)
 __device__ __forceinline__ float exp2f_approx(float x) {
@@ -575,10 +595,7 @@ decode128_kernel(const __grid_constant__ CUtensorMap tm_pool, const DecodeArgs a
                     const uint4 u = lds128(sb + soff + r * NRG * 128);
                     const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        f[2 * i] = __uint_as_float(w4[i] << 16);
-                        f[2 * i + 1] = __uint_as_float(w4[i] & 0xffff0000u);
-                    }
+                    for (int i = 0; i < 4; ++i) unpack2<TS>(w4[i], f[2 * i], f[2 * i + 1]);
                 } else {
                     const uint4 u0 = lds128(sb + soff + r * NRG * 128), u1 = lds128(sb + soff2 + r * NRG * 128);
                     f[0] = __uint_as_float(u0.x); f[1] = __uint_as_float(u0.y);
@@ -758,7 +775,10 @@ cudaError_t launch_decode128(const DecodeArgs &a, cudaStream_t stream) {
     const cuuint64_t dims[3] = {(cuuint64_t)Cf::D, (cuuint64_t)Cf::D, (cuuint64_t)a.slots * (cuuint64_t)a.Nv};
     const cuuint64_t strides[2] = {(cuuint64_t)Cf::D * sizeof(TS), (cuuint64_t)Cf::D * Cf::D * sizeof(TS)};
     const cuuint32_t box[3] = {(cuuint32_t)Cf::BOXC, (cuuint32_t)Cf::D, 1}, es[3] = {1, 1, 1};
-    if (enc(&tm, sizeof(TS) == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, a.pool, dims,
+    const CUtensorMapDataType tmt = sizeof(TS) == 4                        ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
+                                    : std::is_same<TS, __half>::value ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
+                                                                      : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    if (enc(&tm, tmt, 3, a.pool, dims,
             strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
         return cudaErrorInvalidValue;
@@ -800,18 +820,18 @@ cudaError_t launch_decode_t(const DecodeArgs &a, cudaStream_t stream) {
 
 template <int DK, int DV>
 cudaError_t launch_decode_d(const DecodeArgs &a, gdr_dtype dt, gdr_dtype st, cudaStream_t stream) {
-    // fp16 inputs (with an fp16 or fp32 state) run the general kernel at every head size
-    if (dt == GDR_F16) {
-        if (st == GDR_F16) return launch_decode_t<DK, DV, __half, __half>(a, stream);
-        if (st == GDR_F32) return launch_decode_t<DK, DV, __half, float>(a, stream);
-        return cudaErrorInvalidValue;
-    }
+    // fp16 inputs take an fp16 or fp32 state
+    if (dt == GDR_F16 && st != GDR_F16 && st != GDR_F32) return cudaErrorInvalidValue;
     if (DK == 128 && DV == 128) {
+        if (dt == GDR_F16 && st == GDR_F16) return launch_decode128<__half, __half>(a, stream);
+        if (dt == GDR_F16) return launch_decode128<__half, float>(a, stream);
         if (dt == GDR_BF16 && st == GDR_BF16) return launch_decode128<__nv_bfloat16, __nv_bfloat16>(a, stream);
         if (dt == GDR_BF16 && st == GDR_F32) return launch_decode128<__nv_bfloat16, float>(a, stream);
         if (dt == GDR_F32 && st == GDR_BF16) return launch_decode128<float, __nv_bfloat16>(a, stream);
         return launch_decode128<float, float>(a, stream);
     }
+    if (dt == GDR_F16 && st == GDR_F16) return launch_decode_t<DK, DV, __half, __half>(a, stream);
+    if (dt == GDR_F16) return launch_decode_t<DK, DV, __half, float>(a, stream);
     if (dt == GDR_BF16 && st == GDR_BF16) return launch_decode_t<DK, DV, __nv_bfloat16, __nv_bfloat16>(a, stream);
     if (dt == GDR_BF16 && st == GDR_F32) return launch_decode_t<DK, DV, __nv_bfloat16, float>(a, stream);
     if (dt == GDR_F32 && st == GDR_BF16) return launch_decode_t<DK, DV, float, __nv_bfloat16>(a, stream);

@@ -73,6 +73,17 @@ def test_decode_no_gate_d128(S, share):
     check_decode(w, *run_decode(w, "bf16"), "bf16")
 
 
+@pytest.mark.parametrize("sdt", ["f16", "f32"])
+def test_decode_f16_d128_workload_and_no_gate(sdt):
+    """fp16 inputs on the D = 128 kernel: the decode workload (64 sequences, one token, injective slots) with an
+    fp16 or fp32 state, then the same pool stepped without a gate (its build without the decay)."""
+    w = workloads.generate("decode")
+    check_decode(w, *run_decode(w, "f16", sdt), "f16", sdt)
+    w = workloads.random_case(B=12, Nk=2, Nv=4, S=3, Dk=128, Dv=128, seed=125, gate="none", slots=64,
+                              share_slot=True)
+    check_decode(w, *run_decode(w, "f16", sdt), "f16", sdt)
+
+
 def test_decode_gk_workload_fused_prologue():
     w = workloads.generate("decode_gk", B=32)
     check_decode(w, *run_decode(w, "bf16", fused=True), "bf16")

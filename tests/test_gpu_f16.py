@@ -49,8 +49,8 @@ def test_chunk_f16_fused_prologue_and_epilogue():
     assert_close(host(fin), rf, "f16", "final_state")
 
 
-@pytest.mark.parametrize("sdt,D,per_token", [("f16", 128, False), ("f32", 128, False), ("f16", 64, True),
-                                             ("f32", 32, True)])
+@pytest.mark.parametrize("sdt,D,per_token", [("f16", 128, False), ("f32", 128, False), ("f16", 128, True),
+                                             ("f32", 128, True), ("f16", 64, True), ("f32", 32, True)])
 def test_decode_f16(sdt, D, per_token):
     S, B = 4, 5
     w = workloads.random_case(B=B, Nk=2, Nv=4, S=S, Dk=D, Dv=D, seed=620 + D + per_token, with_gk=True,
