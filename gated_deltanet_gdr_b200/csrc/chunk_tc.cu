@@ -373,6 +373,20 @@ __device__ __forceinline__ int order_chain(const TcArgs &a, int tid, uint8_t *sm
 
 // kGate = false: the build for g = NULL (no decay): no gate scan, the A and Pm entries take the column factor
 // 1/|k_s| without an exponential, and the state is never rescaled in TMEM.
+// The part of a bounded wait after its first test failed, out of line: one copy of the polling loop and the
+// timeout record instead of one per call site.  The kernel's code is large (every role's loop is hot at once),
+// and with a CTA on most SMs its instruction fetches contend: the warps' stalls for instructions doubled from
+// 32 to 128 CTAs.  This, with the loops over 32-column halves kept rolled, took 12 % off a launch of 128 chains.
+__device__ __noinline__ bool wait_slow(uint64_t *bar, uint32_t parity, uint64_t limit_ns, volatile int *abort,
+                                       uint32_t bar_index) {
+    if (mbar_wait_ns(bar, parity, limit_ns, abort)) return true;
+    if (!*abort)
+        atomicCAS(&g_timeout_site, 0u,
+                  0x80000000u | ((threadIdx.x >> 5) << 24) | (bar_index << 16) | (parity << 15) |
+                      (blockIdx.x & 0x7fffu));
+    return false;
+}
+
 template <typename T, bool kGate, bool kOrdered>
 __global__ void __launch_bounds__(NT, 1)
 chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -417,12 +431,8 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 
     // a bounded wait: false when it ran out (the first such wait of the launch is recorded) or another group stopped
     auto bw = [&](uint64_t *bar, uint32_t parity) -> bool {
-        if (mbar_wait_ns(bar, parity, a.wait_ns, s_abort)) return true;
-        if (!*s_abort)
-            atomicCAS(&g_timeout_site, 0u,
-                      0x80000000u | ((uint32_t)warp << 24) | ((uint32_t)(bar - bars) << 16) | (parity << 15) |
-                          (blockIdx.x & 0x7fffu));
-        return false;
+        if (mbar_test(bar, parity)) return true;
+        return wait_slow(bar, parity, a.wait_ns, s_abort, (uint32_t)(bar - bars));
     };
     // loads issued per barrier by the thread that issues them (one phase each), for the drain at the exit
     int n_ld = 0, n_ldv = 0, n_cq = 0, n_ck = 0;
@@ -465,7 +475,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         // ---- initial state into TMEM (fp32) and the bf16 operand tile ----
         const T *s0 = reinterpret_cast<const T *>(a.initial_state);
         const size_t off = ((size_t)bh * D + row) * D + 64 * hf;
-#pragma unroll
+#pragma unroll 1
         for (int half = 0; half < 2; ++half) {
             float v[32];
 #pragma unroll
@@ -927,7 +937,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             PHASE(22);
             if (q4 >= 2) {  // W rows (TMEM lanes 64..127 of R) -> rows 0..63 of A1
                 const int t = row - 64;
-#pragma unroll
+#pragma unroll 1
                 for (int half = 0; half < 2; ++half) {
                     float w[32];
                     tmem_ld32(tmem + TM_R + lane_base + 64 * hf + 32 * half, w);
@@ -964,7 +974,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             // S <- e^{G_last} S in TMEM, onto which MMA2 accumulates (for c > 0 the previous chunk's
             // epilogue already wrote the scaled state back)
             if (kGate && c == 0) {
-#pragma unroll
+#pragma unroll 1
                 for (int half = 0; half < 2; ++half) {
                     float v[32];
                     const uint32_t ta = tmem + TM_S + lane_base + 64 * hf + 32 * half;
@@ -985,7 +995,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             PHASE(17);
             if (q4 < 2) {  // v_new = U - W S for token t, dv columns [64 hf, +64)
                 const int t = row;
-#pragma unroll
+#pragma unroll 1
                 for (int half = 0; half < 2; ++half) {
                     float u[32], r[32];
                     tmem_ld32(tmem + TM_U + lane_base + 64 * hf + 32 * half, u);
@@ -1004,7 +1014,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                                                                     ((size_t)bh * S + (size_t)c * C + row - 64) * D +
                                                                     64 * hf));
                 const float xs = vec[V_XS * 64 + row - 64];
-#pragma unroll
+#pragma unroll 1
                 for (int half = 0; half < 2; ++half) {
                     float r[32];
                     const uint32_t ta = tmem + TM_R + lane_base + 64 * hf + 32 * half;
@@ -1061,7 +1071,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             PHASE(19);
             // ---- S (fp32, TMEM) -> bf16 operand tile, and back to TMEM scaled by e^{G_last} of the next
             // chunk (its gate vectors were written before this chunk was handed over);  o rows -> out tile ----
-#pragma unroll
+#pragma unroll 1
             for (int half = 0; half < 2; ++half) {
                 float v[32];
                 const uint32_t ta = tmem + TM_S + lane_base + 64 * hf + 32 * half;
@@ -1087,7 +1097,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 const T *zr = nullptr;
                 if (epi) {
                     float ss = 0.f;
-#pragma unroll
+#pragma unroll 1
                     for (int half = 0; half < 2; ++half) {
                         float o[32];
                         tmem_ld32(tmem + TM_R + lane_base + 64 * hf + 32 * half, o);
@@ -1102,7 +1112,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     named_sync(BAR_EPI, 128);
                     inv = rsqrtf((eps2[t] + eps2[64 + t]) * (1.f / D) + a.epi_eps);
                 }
-#pragma unroll
+#pragma unroll 1
                 for (int half = 0; half < 2; ++half) {
                     float o[32];
                     tmem_ld32(tmem + TM_R + lane_base + 64 * hf + 32 * half, o);
@@ -1158,7 +1168,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             }
             if (a.final_state) {
                 T *fs = reinterpret_cast<T *>(a.final_state) + ((size_t)bh * D + row) * D + 64 * hf;
-#pragma unroll
+#pragma unroll 1
                 for (int half = 0; half < 2; ++half) {
                     float v[32];
                     tmem_ld32(tmem + TM_S + lane_base + 64 * hf + 32 * half, v);

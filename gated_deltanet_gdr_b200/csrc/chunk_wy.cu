@@ -634,6 +634,20 @@ __device__ __forceinline__ void stsm_x4_trans(uint32_t addr, const uint32_t (&r)
                  : "memory");
 }
 
+// The part of a bounded wait after its first test failed, out of line: one copy of the polling loop and the
+// timeout record instead of one per call site.  The kernel's code is large (every role's loop is hot at once),
+// and with a CTA on most SMs its instruction fetches contend: the warps' stalls for instructions doubled from
+// 32 to 128 CTAs.  This, with the loops over 32-column halves kept rolled, took 12 % off a launch of 128 chains.
+__device__ __noinline__ bool wait_slow(uint64_t *bar, uint32_t parity, uint64_t limit_ns, volatile int *abort,
+                                       uint32_t bar_index) {
+    if (mbar_wait_ns(bar, parity, limit_ns, abort)) return true;
+    if (!*abort)  // this wait ran out (rather than seeing another group stop): record where
+        atomicCAS(&g_timeout_site, 0u,
+                  0x80000000u | ((threadIdx.x >> 5) << 24) | (bar_index << 16) | (parity << 15) |
+                      (blockIdx.x & 0x7fffu));
+    return false;
+}
+
 template <typename T, bool kGate, bool kOrdered>
 __global__ void __launch_bounds__(CH_THREADS, 1)
 chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -697,14 +711,15 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         const bool ok = mbar_wait_ns(bars + idx, parity, wait_ns, s_abort);
         if (rep_thread) s_wcyc[role * 36 + idx] += (unsigned long long)(clock64() - t0);
         if (ok) return true;
-#else
-        if (mbar_wait_ns(bars + idx, parity, wait_ns, s_abort)) return true;
-#endif
         if (!*s_abort)  // this wait ran out (rather than seeing another group stop): record where
             atomicCAS(&g_timeout_site, 0u,
                       0x80000000u | ((uint32_t)warp << 24) | ((uint32_t)idx << 16) | (parity << 15) |
                           (blockIdx.x & 0x7fffu));
         return false;
+#else
+        if (mbar_test(bars + idx, parity)) return true;
+        return wait_slow(bars + idx, parity, wait_ns, s_abort, (uint32_t)idx);
+#endif
     };
 
     if (warp == W_VLD) {
@@ -1015,7 +1030,7 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             tc_fence_after();
             {
                 const int dk = q4 * 32 + lane;
-#pragma unroll
+#pragma unroll 1
                 for (int hv = 0; hv < 2; ++hv) {
                     float w[32];
                     tmem_ld32(tmem + TM_W + lane_base + 32 * hv, w);
@@ -1044,7 +1059,7 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                 const bool valid = t < n;
                 const float g2t = vc[V_G2 * 64 + t];
                 uint8_t *pm = sm + OFF_PM + par * 8192;
-#pragma unroll
+#pragma unroll 1
                 for (int hv = 0; hv < 2; ++hv) {
                     float v[32];
                     if (hv == 1 && q4 == 0) {  // rows 0..31, columns 32..63: above the diagonal
