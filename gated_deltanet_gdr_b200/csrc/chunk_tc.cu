@@ -139,7 +139,7 @@ constexpr int NVEC = 11;             // per-chunk vectors of 64 floats (enum bel
 constexpr uint32_t OFF_VEC = 215040;  // 2 sets x NVEC vectors x 64 floats
 static_assert(OFF_XM + 32 * SP * 4 <= OFF_VEC, "merge product");
 constexpr uint32_t OFF_BAR = OFF_VEC + 2 * NVEC * 64 * 4;
-constexpr uint32_t OFF_EPI = OFF_BAR + 128;  // epilogue: partial squared norms of the o rows (2 x 64 floats)
+constexpr uint32_t OFF_EPI = OFF_BAR + 256;  // epilogue: partial squared norms of the o rows (2 x 64 floats)
 // the order of the chains (see order_chain): the B lengths, then the selected sequence
 constexpr int kRankMaxB = 256;
 constexpr uint32_t OFF_LEN = OFF_EPI + 512;
@@ -408,10 +408,11 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     // bar_go: the carry group has taken chunk c over (its tail factors are in place); bar_kt: the helper warps
     // have scaled chunk c's K tile into K~ (one phase per chunk each)
     uint64_t *bar_go = bars + 12, *bar_kt = bars + 13;
-    // bar_dr: two commits, every MMA of the control warp and of the carry group completed (exit)
-    uint64_t *bar_dr = bars + 14;
-    constexpr int kNumBars = 15;
-    static_assert(kNumBars * 8 + 8 <= 128, "barriers, TMEM base and abort flag before the epilogue scratch");
+    // bar_dr: two commits, every MMA of the control warp and of the carry group completed (exit); bar_gf: the
+    // two helper warps of TMEM lanes 64..127 have written chunk c's epilogue gate factors (one phase per chunk)
+    uint64_t *bar_dr = bars + 14, *bar_gf = bars + 15;
+    constexpr int kNumBars = 16;
+    static_assert(kNumBars * 8 + 8 <= OFF_EPI - OFF_BAR, "barriers, TMEM base and abort flag before the epilogue scratch");
     uint32_t *s_tmem = reinterpret_cast<uint32_t *>(bars + kNumBars);
     volatile int *s_abort = reinterpret_cast<volatile int *>(s_tmem + 1);
 
@@ -453,7 +454,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 
     if (tid == 0) {
         if (bad_len) raise_device_error(a.err, GDR_DEVERR_LENGTH);
-        for (int i = 0; i < kNumBars; ++i) mbar_init(bars + i, i == 14 ? 2 : 1);
+        for (int i = 0; i < kNumBars; ++i) mbar_init(bars + i, i >= 14 ? 2 : 1);
         *s_abort = 0;
         fence_mbar_init();
         prefetch_tmap(&tm_q);
@@ -670,11 +671,25 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         // K~ = diag(e^{G_last - G} / |k|) K of each chunk, in place in the carry's raw K tile (rows past the
         // length, whatever they hold, become zero): the A operand of the state update, made off the carry's
         // serial chain.  The tile of chunk c lands after MMA2 of chunk c-1 and is needed at MMA2 of chunk c.
+        // With the epilogue, the two helper warps of TMEM lanes 64..127 (the lanes of the o rows) then write
+        // the chunk's gate factors w silu(z) for their row, all 128 columns, into columns TM_U.. of those
+        // lanes: the U product leaves them unused (its rows 64..127 are never read), they are free from the
+        // completion of the chunk's W/U products until the carry's epilogue has read them, and the next W/U
+        // products are issued only after that.
         const int hp = tid - (CTL_WARP + 1) * 32;
+        const bool gf_rows = a.epi_z != nullptr && q4 >= 2;  // warps 18 and 19
         bool to = false;
         for (int c = 0; c < nvalid; ++c) {
             const uint32_t par = c & 1;
             const float *vec = vecs + par * NVEC * 64;
+            const int t_gf = row - 64, n_gf = min(C, L - c * C);
+            const T *z_row = gf_rows && t_gf < n_gf
+                                 ? static_cast<const T *>(a.epi_z) + ((size_t)bh * S + (size_t)c * C + t_gf) * D
+                                 : nullptr;
+            if (z_row) {  // the row's 256 bytes of z into L1 while the K~ tile is scaled
+                asm volatile("prefetch.global.L1 [%0];" ::"l"(z_row));
+                asm volatile("prefetch.global.L1 [%0];" ::"l"(z_row + 64));
+            }
             // bar_go of chunk c+1 follows bar_kt of chunk c, and the K tile of chunk c+1 is loaded after MMA2 of
             // chunk c, which waits for bar_kt of chunk c: neither wait can be a phase behind
             if (!bw(bar_go, par)) to = true;
@@ -696,6 +711,34 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             fence_proxy_async_smem();
             if (named_sync_or(BAR_HELP, NHELP, to)) break;
             if (hp == 0) mbar_arrive(bar_kt);
+            if (gf_rows) {
+                // the chunk's W/U products (which also write these lanes of TM_U) have completed: bar_wu of
+                // chunk c+1 needs the carry's epilogue of chunk c, which waits for this warp's bar_gf
+                // (one verdict per warp: the TMEM stores below are warp-collective)
+                if (!__all_sync(0xffffffffu, bw(bar_wu, par))) to = true;
+                tc_fence_after();
+                if (!to) {
+#pragma unroll 1
+                    for (int blk = 0; blk < 4; ++blk) {
+                        float f[32];
+#pragma unroll
+                        for (int c8 = 0; c8 < 4; ++c8) {
+                            float zf[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+                            if (z_row) unpack8<T>(*reinterpret_cast<const uint4 *>(z_row + 32 * blk + 8 * c8), zf);
+                            const float4 *wp = reinterpret_cast<const float4 *>(a.epi_w + 32 * blk + 8 * c8);
+                            const float4 w0 = wp[0], w1 = wp[1];
+                            const float wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+#pragma unroll
+                            for (int i = 0; i < 8; ++i) f[8 * c8 + i] = wv[i] * silu_out<T>(zf[i]);
+                        }
+                        tmem_st32(tmem + TM_U + lane_base + 32 * blk, f);
+                    }
+                    tmem_st_wait();
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar_gf);
+            }
         }
         if (to && hp == 0) *s_abort = 1;
     } else if (!carry) {
@@ -1009,10 +1052,6 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                             pack8<T>(&u[8 * c8]);
                 }
             } else {  // rows of Q S: scale by e^{G_t} scale / |q_t| before Pm v_new accumulates onto them
-                if (a.epi_z && row - 64 < n)  // this thread's half row of z, for the epilogue
-                    asm volatile("prefetch.global.L1 [%0];" ::"l"(static_cast<const T *>(a.epi_z) +
-                                                                    ((size_t)bh * S + (size_t)c * C + row - 64) * D +
-                                                                    64 * hf));
                 const float xs = vec[V_XS * 64 + row - 64];
 #pragma unroll 1
                 for (int half = 0; half < 2; ++half) {
@@ -1094,7 +1133,6 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 // warp with the same lane), then o * inv * norm_w * silu(z) for this thread's 64 columns
                 const bool epi = a.epi_z != nullptr;
                 float inv = 1.f;
-                const T *zr = nullptr;
                 if (epi) {
                     float ss = 0.f;
 #pragma unroll 1
@@ -1107,26 +1145,24 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     }
                     float *eps2 = reinterpret_cast<float *>(sm + OFF_EPI);
                     eps2[hf * 64 + t] = ss;
-                    if (t < n)  // rows past the length are never read
-                        zr = static_cast<const T *>(a.epi_z) + ((size_t)bh * S + (size_t)c * C + t) * D + 64 * hf;
                     named_sync(BAR_EPI, 128);
                     inv = rsqrtf((eps2[t] + eps2[64 + t]) * (1.f / D) + a.epi_eps);
+                    wait_ok(bar_gf, par);  // the gate factors w silu(z) of this chunk's rows (helper warps)
+                    tc_fence_after();
                 }
 #pragma unroll 1
                 for (int half = 0; half < 2; ++half) {
                     float o[32];
                     tmem_ld32(tmem + TM_R + lane_base + 64 * hf + 32 * half, o);
                     tmem_ld_wait();
-                    if (epi && t < n) {
+                    if (epi) {
 #pragma unroll
-                        for (int c8 = 0; c8 < 4; ++c8) {
-                            float zf[8];
-                            unpack8<T>(*reinterpret_cast<const uint4 *>(zr + 32 * half + 8 * c8), zf);
-                            const float4 *wp = reinterpret_cast<const float4 *>(a.epi_w + 64 * hf + 32 * half + 8 * c8);
-                            const float4 w0 = wp[0], w1 = wp[1];
-                            const float wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+                        for (int q = 0; q < 2; ++q) {
+                            float gfv[16];
+                            tmem_ld16(tmem + TM_U + lane_base + 64 * hf + 32 * half + 16 * q, gfv);
+                            tmem_ld_wait();
 #pragma unroll
-                            for (int i = 0; i < 8; ++i) o[8 * c8 + i] *= inv * wv[i] * silu_out<T>(zf[i]);
+                            for (int j = 0; j < 16; ++j) o[16 * q + j] *= inv * gfv[j];
                         }
                     }
 #pragma unroll

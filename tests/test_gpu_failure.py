@@ -11,7 +11,7 @@ import torch
 import gated_deltanet_gdr_b200 as gdr
 import oracle
 import workloads
-from tests._helpers import assert_close, dev, dev_i32, host, unfused_inputs
+from tests._helpers import assert_close, dev, dev_i32, host, rnd, rnd32, unfused_inputs
 
 pytestmark = pytest.mark.gpu
 
@@ -21,9 +21,9 @@ def _tiny_tc_case():
     return w, unfused_inputs(w, "bf16")
 
 
-def _call(w, ins):
+def _call(w, ins, epi=None):
     return gdr.chunk_fwd(dev(ins["q"], "bf16"), dev(ins["k"], "bf16"), dev(ins["v"], "bf16"), dev(ins["beta"], "bf16"),
-                         dev(ins["g"], "f32"), dev(ins["initial_state"], "bf16"), None, w.scale)
+                         dev(ins["g"], "f32"), dev(ins["initial_state"], "bf16"), None, w.scale, epilogue=epi)
 
 
 def test_bounded_wait_runs_out_and_the_next_call_is_clean():
@@ -52,29 +52,38 @@ def test_bounded_wait_runs_out_and_the_next_call_is_clean():
 
 
 @pytest.mark.timeout(300)
-def test_bounded_wait_runs_out_one_kernel_schedule():
+@pytest.mark.parametrize("with_epilogue", [False, True])
+def test_bounded_wait_runs_out_one_kernel_schedule(with_epilogue):
     """The same with the one-kernel schedule (the prefill workload's): with the limit at 1 ns its waits run out,
     each warp group stops at its next collective hand-off (bar.red.or, so no group splits at a named barrier),
     the issuers wait for their copies and MMAs in flight, and the call returns with GDR_DEVERR_TIMEOUT and the
-    first site that ran out.  The next call with the default limit passes parity."""
+    first site that ran out.  The next call with the default limit passes parity.  With the gated RMSNorm
+    epilogue the helper warps that write its gate factors wait too."""
     w, ins = _tiny_tc_case()
+    epi = zr = wr = None
+    if with_epilogue:
+        z, nw = workloads.epilogue_inputs(w)
+        zr, wr = rnd(z, "bf16"), rnd32(nw)
+        epi = gdr.Epilogue(z=dev(zr, "bf16"), norm_w=dev(wr, "f32"), eps=1e-6)
     assert gdr.get_error() == 0 and gdr.take_timeout_site() == {}
     gdr.set_chunk_schedule(gdr.SCHEDULE_ONE_KERNEL)
     try:
         gdr.set_wait_limit_ns(1)
         try:
-            _call(w, ins)
+            _call(w, ins, epi)
             err = gdr.get_error()
             site = gdr.take_timeout_site()
         finally:
             gdr.set_wait_limit_ns(0)
         assert err & gdr.DEVERR_TIMEOUT, err
         assert site and 0 <= site["warp"] < 20 and site["cta"] < w.B * w.Nv, site
-        out, fin = _call(w, ins)
+        out, fin = _call(w, ins, epi)
         assert gdr.get_error() == 0 and gdr.take_timeout_site() == {}
     finally:
         gdr.set_chunk_schedule(gdr.SCHEDULE_AUTO)
     ro, rf = oracle.chunk_fwd(ins["q"], ins["k"], ins["v"], ins["beta"], ins["g"], ins["initial_state"], None, w.scale)
+    if with_epilogue:
+        ro = oracle.gated_rmsnorm(ro, zr, wr, 1e-6)
     assert_close(host(out), ro, "bf16", "out")
     assert_close(host(fin), rf, "bf16", "final_state")
 
