@@ -150,7 +150,8 @@ static_assert(OFF_TT % 1024 == 0, "swizzle atoms");
 static_assert(OFF_PM0 >= 8192 && OFF_PM1 == OFF_PM0 + 8192, "Pm buffers");
 
 // TMEM columns (all 128 lanes): the Gram [K; Q][K; Q]^T (then the solve's merge products); U (lanes
-// 0..63); R: first W of the chunk (lanes 64..127, written while R is otherwise free), then [W S; o]
+// 0..63; with the epilogue, lanes 64..127 take the chunk's gate factors norm_w * silu(z) once the U product
+// has completed); R: first W of the chunk (lanes 64..127, written while R is otherwise free), then [W S; o]
 // (lanes 0..63 / 64..127); the fp32 state S
 constexpr uint32_t TM_GPW = 0, TM_U = 128, TM_R = 256, TM_S = 384, TM_COLS = 512;
 
@@ -1130,7 +1131,8 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             if (q4 >= 2) {
                 const int t = row - 64;
                 // epilogue: the row's squared norm from its two halves (this thread and the one of the other hf
-                // warp with the same lane), then o * inv * norm_w * silu(z) for this thread's 64 columns
+                // warp with the same lane), then o * inv * (norm_w * silu(z)) for this thread's 64 columns, the
+                // gate factors read from TMEM where the helper warps put them
                 const bool epi = a.epi_z != nullptr;
                 float inv = 1.f;
                 if (epi) {
