@@ -8,7 +8,7 @@ import pytest
 
 import oracle
 import workloads
-from tests import _pins
+from tests import _decode_pins, _pins
 
 
 def chunk_impl(q, k, v, beta, g, S0, lengths, scale):
@@ -42,6 +42,12 @@ def test_decode_oracle_pin(check):
     check(decode_as_chunk)
 
 
+@pytest.mark.parametrize("check", _decode_pins.DECODE_CHECKS, ids=lambda c: c.__name__)
+def test_decode_feature_pin(check):
+    """The slot pool, the per-key gate, the accepted counts and the speculative reading (tests/_decode_pins)."""
+    check(oracle.recurrent_step)
+
+
 def test_prologue_values():
     with open(os.path.join(_pins.GOLDEN, "prologue_values.json")) as f:
         c = json.load(f)
@@ -71,85 +77,6 @@ def test_prologue_shapes_and_heads():
     q = rng.normal(size=(2, 2, 5, 7))
     qh = oracle.prologue(q=q)["q_hat"]
     assert np.allclose((qh * qh).sum(-1), (q * q).sum(-1) / ((q * q).sum(-1) + 1e-6), atol=1e-14)
-
-
-def test_decode_gk_closed_form():
-    """beta = 0 with a per-key gate: row i of the state decays by
-    exp(sum g + sum gk_i), so o_t = sum_i x_i exp(G_t + GK_t[i]) S0[i, :]
-    (lite_boost recurrent op: S = S * exp(g) * exp(gk))."""
-    rng = np.random.default_rng(30)
-    S, Dk, Dv = 5, 4, 3
-    q = rng.normal(size=(1, 1, S, Dk))
-    k = rng.normal(size=(1, 1, S, Dk))
-    v = rng.normal(size=(1, 1, S, Dv))
-    g = np.log(rng.uniform(0.7, 0.99, size=(1, 1, S)))
-    gk = np.log(rng.uniform(0.8, 0.999, size=(1, 1, S, Dk)))
-    pool = rng.normal(size=(2, 1, Dk, Dv))
-    idx = np.array([1] * S, np.int32)
-    out, newpool = oracle.recurrent_step(q, k, v, np.zeros((1, 1, S)), g, gk, pool, idx, np.array([S], np.int32),
-                                         None, 0.5)
-    G = np.cumsum(g[0, 0])
-    GK = np.cumsum(gk[0, 0], axis=0)
-    for t in range(S):
-        dec = np.exp(G[t] + GK[t])
-        assert np.allclose(out[0, 0, t], (0.5 * q[0, 0, t] * dec) @ pool[1, 0], atol=1e-13, rtol=0)
-    assert np.allclose(newpool[1, 0], np.exp(G[-1] + GK[-1])[:, None] * pool[1, 0], atol=1e-13, rtol=0)
-    assert np.array_equal(newpool[0], pool[0])
-    # a per-key gate equal on every row is the same as adding it to g
-    c = np.log(rng.uniform(0.8, 0.99, size=(1, 1, S)))
-    beta = rng.uniform(size=(1, 1, S))
-    o1, p1 = oracle.recurrent_step(q, k, v, beta, g, np.repeat(c[..., None], Dk, -1), pool, idx,
-                                   np.array([S], np.int32), None, 1.0)
-    o2, p2 = oracle.recurrent_step(q, k, v, beta, g + c, None, pool, idx, np.array([S], np.int32), None, 1.0)
-    assert np.allclose(o1, o2, atol=1e-13, rtol=0) and np.allclose(p1, p2, atol=1e-13, rtol=0)
-
-
-def test_decode_accepted_tokens():
-    """All L tokens are output; the slot receives the state after min(A, L)
-    tokens (reading of num_accepted_tokens); A = 0 leaves the slot untouched."""
-    w = workloads.random_case(B=4, Nk=1, Nv=2, S=4, Dk=5, Dv=3, seed=31, slots=6, initial_state=False)
-    w.lengths = np.array([4, 3, 2, 4], np.int32)
-    w.accepted = np.array([2, 3, 1, 0], np.int32)
-    pro = oracle.prologue(q=w.q, k=w.k, b=w.b)
-    args = (pro["q_hat"], pro["k_hat"], w.v, pro["beta"], w.g)
-    out, pool = oracle.recurrent_step(*args, None, w.pool, w.indices, w.lengths, w.accepted, w.scale)
-    for b in range(w.B):
-        slot = w.indices[b * w.S]
-        S0 = w.pool[slot][None]
-        L, A = int(w.lengths[b]), int(w.accepted[b])
-        sl = (slice(b, b + 1),)
-        o_full, _ = oracle.chunk_fwd(*(x[sl][:, :, :L] for x in args), S0, None, w.scale)
-        assert np.allclose(out[b, :, :L], o_full[0], atol=1e-13, rtol=0)
-        assert np.all(out[b, :, L:] == 0.0)
-        if A == 0:
-            assert np.array_equal(pool[slot], w.pool[slot])
-        else:
-            _, f_acc = oracle.chunk_fwd(*(x[sl][:, :, :A] for x in args), S0, None, w.scale)
-            assert np.allclose(pool[slot], f_acc[0], atol=1e-13, rtol=0)
-    used = set(w.indices.tolist())
-    for s in range(6):
-        if s not in used:
-            assert np.array_equal(pool[s], w.pool[s])
-
-
-def test_decode_distinct_token_slots():
-    """With one slot per token, the state after token t goes to slot
-    indices[b*S + t] for t < A; the chain starts from indices[b*S]."""
-    w = workloads.random_case(B=2, Nk=1, Nv=1, S=3, Dk=4, Dv=4, seed=32, slots=8, share_slot=False,
-                              initial_state=False)
-    w.accepted = np.array([3, 2], np.int32)
-    pro = oracle.prologue(q=w.q, k=w.k, b=w.b)
-    args = (pro["q_hat"], pro["k_hat"], w.v, pro["beta"], w.g)
-    out, pool = oracle.recurrent_step(*args, None, w.pool, w.indices, w.lengths, w.accepted, w.scale)
-    for b in range(2):
-        S0 = w.pool[w.indices[b * 3]][None]
-        for t in range(3):
-            slot = w.indices[b * 3 + t]
-            if t < w.accepted[b]:
-                _, f = oracle.chunk_fwd(*(x[b:b + 1, :, :t + 1] for x in args), S0, None, w.scale)
-                assert np.allclose(pool[slot], f[0], atol=1e-13, rtol=0)
-            else:
-                assert np.array_equal(pool[slot], w.pool[slot])
 
 
 def test_tiny_decode_chain_equals_prefill():
@@ -243,44 +170,6 @@ def _spec_case(seed, B=3, S=4, Nk=2, Nv=4, D=8):
     beta = rng.uniform(0.1, 0.9, (B, Nv, S))
     g = np.log(rng.uniform(0.8, 0.99, (B, Nv, S)))
     return q, k, v, beta, g
-
-
-def test_spec_reading_with_one_accepted_equals_committing_every_token():
-    """A = 1 starts from the slot of token 0, as the other reading does; with every token committed both
-    write the same states to the same per-token slots."""
-    q, k, v, beta, g = _spec_case(31)
-    B, S = q.shape[0], q.shape[2]
-    rng = np.random.default_rng(32)
-    pool = rng.standard_normal((B * S + 2, 4, 8, 8))
-    idx = rng.permutation(B * S + 2)[:B * S].astype(np.int32)
-    L = np.array([4, 2, 3], np.int32)
-    o1, p1 = oracle.recurrent_step(q, k, v, beta, g, None, pool, idx, L, np.ones(B, np.int32), 0.5, per_token=True)
-    o2, p2 = oracle.recurrent_step(q, k, v, beta, g, None, pool, idx, L, L, 0.5)
-    assert np.array_equal(o1, o2) and np.array_equal(p1, p2)
-
-
-def test_spec_two_steps_equal_the_chain_over_accepted_tokens():
-    """Step 1 verifies 4 draft tokens from slot s0 and writes each token's state to its own slot; 2 are
-    accepted.  Step 2 starts from the state after the second token (slot of token A - 1) and processes 4
-    new tokens: its outputs and states equal the prefill oracle's chain over x1, x2, y1..y4."""
-    q1, k1, v1, b1, g1 = _spec_case(33, B=1)
-    q2, k2, v2, b2, g2 = _spec_case(34, B=1)
-    S = 4
-    rng = np.random.default_rng(35)
-    pool = rng.standard_normal((6, 4, 8, 8))
-    slots = np.array([5, 1, 3, 0], np.int32)
-    _, p1 = oracle.recurrent_step(q1, k1, v1, b1, g1, None, pool, slots, np.array([S], np.int32),
-                                  np.array([1], np.int32), 0.5, per_token=True)
-    A = 2
-    o2, p2 = oracle.recurrent_step(q2, k2, v2, b2, g2, None, p1, slots, np.array([S], np.int32),
-                                   np.array([A], np.int32), 0.5, per_token=True)
-    cat = lambda a1, a2: np.concatenate([a1[:, :, :A], a2], axis=2)
-    s0 = pool[slots[0]][None]  # the chain's state before x1
-    oc, fc = oracle.chunk_fwd(cat(q1, q2), cat(k1, k2), cat(v1, v2), cat(b1, b2), cat(g1, g2), s0, None, 0.5)
-    assert np.allclose(o2, oc[:, :, A:], rtol=1e-12, atol=1e-12)
-    assert np.allclose(p2[slots[S - 1]], fc[0], rtol=1e-12, atol=1e-12)
-    untouched = [s for s in range(6) if s not in slots]
-    assert np.array_equal(p2[untouched], pool[untouched])
 
 
 def test_spec_reading_rejects_accepted_outside_range():

@@ -4,12 +4,14 @@ A plain numpy copy of the token-by-token rule is run through every pin in
 ``_pins``: unmodified it must pass them all (so the harness itself is sound),
 and with each planted mistake (a dropped term, a wrong sign, an operation in
 the wrong order, a wrong head index, padding left dirty) at least one pin
-must fail.  Everything here runs on the CPU; nothing touches the CUDA path.
+must fail.  The same is done for the output epilogue, the causal conv1d and the decode call's own
+features (slot pool, per-key gate, accepted counts, the speculative reading).  Everything here runs on the
+CPU; nothing touches the CUDA path.
 """
 import numpy as np
 import pytest
 
-from tests import _pins
+from tests import _decode_pins, _pins
 
 
 def make_impl(mutation=None):
@@ -166,5 +168,82 @@ def test_planted_conv_mistake_is_caught(mutation):
         try:
             check(impl)
         except (AssertionError, IndexError, ValueError):
+            caught += 1
+    assert caught > 0, mutation
+
+
+def make_decode(mutation=None):
+    """A plain copy of the decode call over a slot pool (the recurrent_gated_delta_rule page's reading, as the
+    oracle states it), with planted mistakes in the features only decode has."""
+    def dec(q, k, v, beta, g, gk, pool, indices, lengths, accepted=None, scale=1.0, per_token=False):
+        q, k, v, beta = (np.asarray(x, np.float64) for x in (q, k, v, beta))
+        B, Nk, S, Dk = q.shape
+        Nv, Dv = v.shape[1], v.shape[3]
+        grp = Nv // Nk
+        P = np.array(pool, np.float64, copy=True)
+        out = np.zeros((B, Nv, S, Dv))
+        for b in range(B):
+            L = int(lengths[b])
+            if L == 0:
+                continue
+            if per_token:
+                A = 1 if accepted is None else int(accepted[b])
+                if not 1 <= A <= S:
+                    raise ValueError("accepted count outside [1, S]")
+                start = int(indices[b * S + (0 if mutation == "spec_start_first" else A - 1)])
+                ncommit = L
+            else:
+                A = L if accepted is None else int(accepted[b])
+                start = int(indices[b * S])
+                ncommit = min(A, L)
+                if mutation == "commit_ignores_accepted":
+                    ncommit = L
+                elif mutation == "commit_one_short":
+                    ncommit = max(ncommit - 1, 0)
+            for h in range(Nv):
+                kh = (h % Nk) if mutation == "gqa_modulo" else h // grp
+                St = P[start, (Nv - 1 - h) if mutation == "pool_head_reversed" else h].copy()
+                for t in range(L):
+                    x = scale * q[b, kh, t]
+                    y = k[b, kh, t]
+                    St = St * (1.0 if g is None else np.exp(float(g[b, h, t])))
+                    e = None
+                    if gk is not None and mutation != "gk_ignored":
+                        gkt = np.asarray(gk[b, h, t], np.float64)
+                        e = np.exp(-gkt) if mutation == "gk_sign" else np.exp(gkt)
+                        if mutation != "gk_after_readout":
+                            St = St * e[:, None]
+                    m = y @ St
+                    if e is not None and mutation == "gk_after_readout":
+                        St = St * e[:, None]
+                    St = St + np.outer(y, beta[b, h, t] * (v[b, h, t] - m))
+                    out[b, h, t] = x @ St
+                    if t < ncommit and (mutation != "commit_only_last" or t == ncommit - 1):
+                        slot = int(indices[b * S + (min(t + 1, S - 1) if mutation == "commit_slot_shift" else t)])
+                        P[slot, h] = St
+                if mutation == "dirty_padding":
+                    out[b, h, L:] = 1.0
+        return out, P
+    return dec
+
+
+DECODE_MUTATIONS = ["gk_sign", "gk_ignored", "gk_after_readout", "commit_ignores_accepted", "commit_one_short",
+                    "commit_only_last", "commit_slot_shift", "spec_start_first", "pool_head_reversed", "gqa_modulo",
+                    "dirty_padding"]
+
+
+def test_unmodified_decode_copy_passes_every_pin():
+    for check in _decode_pins.DECODE_CHECKS:
+        check(make_decode())
+
+
+@pytest.mark.parametrize("mutation", DECODE_MUTATIONS)
+def test_planted_decode_mistake_is_caught(mutation):
+    impl = make_decode(mutation)
+    caught = 0
+    for check in _decode_pins.DECODE_CHECKS:
+        try:
+            check(impl)
+        except AssertionError:
             caught += 1
     assert caught > 0, mutation
